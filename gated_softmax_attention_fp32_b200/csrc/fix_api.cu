@@ -1,0 +1,331 @@
+// Host side of the FiX attention C ABI (include/fix_attn.h): argument
+// validation, workspace layout, the packed-sequence chunk schedule and the
+// kernel launches.  Nothing here allocates or synchronises.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "fix_attn.h"
+#include "fix_common.cuh"
+#include "fix_internal.h"
+
+namespace fix {
+
+static inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+static bool head_dim_ok(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Validates the problem descriptor and fills the kernel-side dims.
+static fix_status make_dims(const fix_attn_problem* p, Dims* d) {
+  if (!p) return FIX_ERR_NULL;
+  if (p->reserved != 0) return FIX_ERR_SHAPE;
+  if (p->y_dtype != FIX_DTYPE_BF16 && p->y_dtype != FIX_DTYPE_F32) return FIX_ERR_DTYPE;
+  if (p->algo < FIX_ALGO_AUTO || p->algo > FIX_ALGO_TC) return FIX_ERR_DTYPE;
+  if (p->batch < 1 || p->seqlen < 0 || p->num_q_heads < 1 || p->num_kv_heads < 1)
+    return FIX_ERR_SHAPE;
+  if (!head_dim_ok(p->head_dim_k) || !head_dim_ok(p->head_dim_v)) return FIX_ERR_HEAD_DIM;
+  if (p->num_q_heads % p->num_kv_heads) return FIX_ERR_GQA;
+  if (!(p->eps >= 0.f) || !std::isfinite(p->eps)) return FIX_ERR_SHAPE;
+  if (!std::isfinite(p->scale)) return FIX_ERR_SHAPE;
+  const long long N = (long long)p->batch * p->seqlen;
+  if (N > (1LL << 30)) return FIX_ERR_SHAPE;
+  if ((long long)N * p->num_q_heads * (p->head_dim_k > p->head_dim_v ? p->head_dim_k : p->head_dim_v) >
+      (1LL << 40))
+    return FIX_ERR_SHAPE;
+  d->N = (int)N;
+  d->B = p->batch;
+  d->T = p->seqlen;
+  d->Hq = p->num_q_heads;
+  d->Hkv = p->num_kv_heads;
+  d->Dk = p->head_dim_k;
+  d->Dv = p->head_dim_v;
+  d->grp = p->num_q_heads / p->num_kv_heads;
+  d->scale = p->scale > 0.f ? p->scale : 1.0f / std::sqrt((float)p->head_dim_k);
+  d->eps = p->eps;
+  long long nch = 0;
+  if (p->cu_seqlens) {
+    if (p->batch != 1) return FIX_ERR_SHAPE;
+    if (!p->cu_seqlens_host || p->num_seqs < 1) return FIX_ERR_CU_SEQLENS;
+    const int64_t* c = p->cu_seqlens_host;
+    if (c[0] != 0 || c[p->num_seqs] != p->seqlen) return FIX_ERR_CU_SEQLENS;
+    for (int i = 0; i < p->num_seqs; ++i) {
+      if (c[i + 1] < c[i]) return FIX_ERR_CU_SEQLENS;
+      nch += (c[i + 1] - c[i] + FIX_CHUNK - 1) / FIX_CHUNK;
+    }
+    d->nseq = p->num_seqs;
+  } else {
+    if (p->num_seqs != 0 || p->cu_seqlens_host) return FIX_ERR_CU_SEQLENS;
+    d->nseq = p->batch;
+    nch = (long long)p->batch * ((p->seqlen + FIX_CHUNK - 1) / FIX_CHUNK);
+  }
+  d->nchunks = (int)nch;
+  return FIX_OK;
+}
+
+static int dw_grid(const Dims& d) {
+  int g = (d.N + 3) / 4;
+  if (g > 128) g = 128;
+  if (g < 1) g = 1;
+  return g;
+}
+
+// Workspace layout (all offsets 256-byte aligned).
+struct Ws {
+  size_t status, chunks, L, vt, tot;          // forward and backward
+  size_t dow, A, dG, dtot, dwp;               // backward only
+  size_t total;
+};
+
+static Ws layout(const Dims& d, bool bwd) {
+  Ws w{};
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    size_t at = o;
+    o = align_up(o + bytes, 256);
+    return at;
+  };
+  const size_t nkv = (size_t)d.N * d.Hkv * d.Dv;
+  const size_t nch = (size_t)d.nchunks * d.Hkv * d.Dv;
+  w.status = take(256);
+  w.chunks = take((size_t)(d.nchunks > 0 ? d.nchunks : 1) * sizeof(Chunk));
+  w.L = take(nkv * 4);
+  w.vt = take(nkv * 2);
+  w.tot = take(nch * 4);
+  if (bwd) {
+    w.dow = take((size_t)d.N * d.Hq * d.Dv * 4);
+    w.A = take(nkv * 4);
+    w.dG = take(nkv * 4);
+    w.dtot = take(nch * 4);
+    w.dwp = take((size_t)dw_grid(d) * d.Hkv * d.Dv * 4);
+  }
+  w.total = o;
+  return w;
+}
+
+static fix_status check_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FIX_ERR_CUDA;
+  int major = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+    return FIX_ERR_CUDA;
+  return major == 10 ? FIX_OK : FIX_ERR_ARCH;
+}
+
+static fix_status launched() {
+  return cudaGetLastError() == cudaSuccess ? FIX_OK : FIX_ERR_CUDA;
+}
+
+// Records the profiling event of `stage` (begin = 0 / end = 1) if requested.
+static fix_status mark(const fix_attn_problem* p, int stage, int end, cudaStream_t st) {
+  if (!p->events) return FIX_OK;
+  cudaEvent_t e = static_cast<cudaEvent_t>(p->events[2 * stage + end]);
+  if (!e) return FIX_OK;
+  return cudaEventRecord(e, st) == cudaSuccess ? FIX_OK : FIX_ERR_CUDA;
+}
+
+#define FIX_TRY(expr)                 \
+  do {                                \
+    fix_status _s = (expr);           \
+    if (_s != FIX_OK) return _s;      \
+  } while (0)
+
+static size_t simt_fwd_smem(const Dims& d) {
+  return sizeof(float) * (size_t)(ST_ROWS * (2 * d.Dk + 1 + 3 * d.Dv));
+}
+static size_t simt_dq_smem(const Dims& d) {
+  return sizeof(float) * (size_t)(ST_ROWS * d.Dk + 2 * ST_ROWS * d.Dv + ST_ROWS + d.Dv +
+                                  ST_ROWS * (d.Dk + 1) + 2 * ST_ROWS * (d.Dv + 1));
+}
+static size_t simt_dkv_smem(const Dims& d) {
+  return sizeof(float) * (size_t)(ST_ROWS * d.Dk + 2 * ST_ROWS * d.Dv + ST_ROWS);
+}
+
+// Prefix pass + schedule (both directions).
+static fix_status run_prefix(const Dims& d, const fix_attn_problem* p, const Ws& ws, char* base,
+                             const float* g, const void* v, bool want_vt, cudaStream_t st) {
+  Chunk* chunks = reinterpret_cast<Chunk*>(base + ws.chunks);
+  schedule_kernel<<<1, 1024, 0, st>>>(p->cu_seqlens, d.nseq, d.T, d.N, d.nchunks, chunks);
+  FIX_TRY(launched());
+  if (d.nchunks == 0) return FIX_OK;
+  prefix_kernel<<<dim3(d.nchunks, d.Hkv), 128, 0, st>>>(
+      d, chunks, g, static_cast<const __nv_bfloat16*>(v), reinterpret_cast<float*>(base + ws.L),
+      want_vt ? reinterpret_cast<__nv_bfloat16*>(base + ws.vt) : nullptr,
+      reinterpret_cast<float*>(base + ws.tot));
+  return launched();
+}
+
+}  // namespace fix
+
+using namespace fix;
+
+extern "C" {
+
+size_t fix_attn_workspace_bytes(const fix_attn_problem* p, int backward) {
+  Dims d;
+  if (make_dims(p, &d) != FIX_OK) return 0;
+  return layout(d, backward != 0).total;
+}
+
+const char* fix_attn_status_string(int s) {
+  switch (s) {
+    case FIX_OK: return "FIX_OK";
+    case FIX_ERR_NULL: return "FIX_ERR_NULL: a required pointer is NULL";
+    case FIX_ERR_SHAPE: return "FIX_ERR_SHAPE: invalid or inconsistent sizes";
+    case FIX_ERR_HEAD_DIM: return "FIX_ERR_HEAD_DIM: head dims must be 16, 32, 64 or 128";
+    case FIX_ERR_GQA: return "FIX_ERR_GQA: num_q_heads must be a multiple of num_kv_heads";
+    case FIX_ERR_CU_SEQLENS: return "FIX_ERR_CU_SEQLENS: cu_seqlens must rise from 0 to the token count";
+    case FIX_ERR_ALIGN: return "FIX_ERR_ALIGN: pointers must be 16-byte aligned";
+    case FIX_ERR_WORKSPACE: return "FIX_ERR_WORKSPACE: workspace missing or too small";
+    case FIX_ERR_DTYPE: return "FIX_ERR_DTYPE: unknown y_dtype or algo";
+    case FIX_ERR_CUDA: return "FIX_ERR_CUDA: a CUDA call or kernel launch failed";
+    case FIX_ERR_DEVICE_TIMEOUT: return "FIX_ERR_DEVICE_TIMEOUT: a bounded device wait expired";
+    case FIX_ERR_ARCH: return "FIX_ERR_ARCH: the current device is not sm_100";
+    default: return "unknown fix_status";
+  }
+}
+
+fix_status fix_attn_fwd(const fix_attn_problem* p, const void* q, const void* k, const void* v,
+                        const float* g, const void* w, void* y, float* o_s, float* m_s,
+                        float* rstd_s, void* workspace, size_t ws_bytes, void* stream) {
+  Dims d;
+  FIX_TRY(make_dims(p, &d));
+  if (!q || !k || !v || !g || !w || !y || !workspace) return FIX_ERR_NULL;
+  const int nsaved = (o_s != nullptr) + (m_s != nullptr) + (rstd_s != nullptr);
+  if (nsaved != 0 && nsaved != 3) return FIX_ERR_NULL;
+  for (const void* ptr : {q, k, v, (const void*)g, w, (const void*)y, (const void*)workspace})
+    if (!aligned16(ptr)) return FIX_ERR_ALIGN;
+  if (nsaved && (!aligned16(o_s) || !aligned16(m_s) || !aligned16(rstd_s))) return FIX_ERR_ALIGN;
+  const Ws ws = layout(d, false);
+  if (ws_bytes < ws.total) return FIX_ERR_WORKSPACE;
+  FIX_TRY(check_device());
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* base = static_cast<char*>(workspace);
+  if (cudaMemsetAsync(base + ws.status, 0, 4, st) != cudaSuccess) return FIX_ERR_CUDA;
+  if (d.N == 0) return FIX_OK;
+  const bool tc = p->algo != FIX_ALGO_SIMT && tc_fwd_supported(d);
+  FIX_TRY(mark(p, FIX_STAGE_FWD_PREFIX, 0, st));
+  FIX_TRY(run_prefix(d, p, ws, base, g, v, tc, st));
+  FIX_TRY(mark(p, FIX_STAGE_FWD_PREFIX, 1, st));
+  const Chunk* chunks = reinterpret_cast<const Chunk*>(base + ws.chunks);
+  const float* L = reinterpret_cast<const float*>(base + ws.L);
+  const float* tot = reinterpret_cast<const float*>(base + ws.tot);
+  FIX_TRY(mark(p, FIX_STAGE_FWD_ATTN, 0, st));
+  if (tc) {
+    FIX_TRY(tc_fwd(d, chunks, q, k, reinterpret_cast<const __nv_bfloat16*>(base + ws.vt), v, L,
+                   tot, w, y, p->y_dtype == FIX_DTYPE_F32, o_s, m_s, rstd_s,
+                   reinterpret_cast<int*>(base + ws.status), st));
+  } else {
+    const size_t smem = simt_fwd_smem(d);
+    if (cudaFuncSetAttribute(fwd_simt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+      return FIX_ERR_CUDA;
+    fwd_simt_kernel<<<dim3(d.nchunks * 4, d.Hq), 256, smem, st>>>(
+        d, chunks, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+        static_cast<const __nv_bfloat16*>(v), L, tot, static_cast<const __nv_bfloat16*>(w), y,
+        p->y_dtype == FIX_DTYPE_F32, o_s, m_s, rstd_s);
+    FIX_TRY(launched());
+  }
+  return mark(p, FIX_STAGE_FWD_ATTN, 1, st);
+}
+
+fix_status fix_attn_bwd(const fix_attn_problem* p, const void* q, const void* k, const void* v,
+                        const float* g, const void* w, const void* dy, const float* o_s,
+                        const float* m_s, const float* rstd_s, void* dq, void* dk, void* dv,
+                        float* dg, void* dw, void* workspace, size_t ws_bytes, void* stream) {
+  Dims d;
+  FIX_TRY(make_dims(p, &d));
+  if (!q || !k || !v || !g || !w || !dy || !o_s || !m_s || !rstd_s || !dq || !dk || !dv || !dg ||
+      !dw || !workspace)
+    return FIX_ERR_NULL;
+  for (const void* ptr : {q, k, v, (const void*)g, w, dy, (const void*)o_s, (const void*)m_s,
+                          (const void*)rstd_s, (const void*)dq, (const void*)dk, (const void*)dv,
+                          (const void*)dg, (const void*)dw, (const void*)workspace})
+    if (!aligned16(ptr)) return FIX_ERR_ALIGN;
+  const Ws ws = layout(d, true);
+  if (ws_bytes < ws.total) return FIX_ERR_WORKSPACE;
+  FIX_TRY(check_device());
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* base = static_cast<char*>(workspace);
+  if (cudaMemsetAsync(base + ws.status, 0, 4, st) != cudaSuccess) return FIX_ERR_CUDA;
+  if (d.N == 0) {
+    if (cudaMemsetAsync(dw, 0, (size_t)d.Dv * 2, st) != cudaSuccess) return FIX_ERR_CUDA;
+    return FIX_OK;
+  }
+  const bool tc = p->algo != FIX_ALGO_SIMT && tc_bwd_supported(d);
+  FIX_TRY(mark(p, FIX_STAGE_BWD_PREFIX, 0, st));
+  FIX_TRY(run_prefix(d, p, ws, base, g, v, tc, st));
+  FIX_TRY(mark(p, FIX_STAGE_BWD_PREFIX, 1, st));
+  const Chunk* chunks = reinterpret_cast<const Chunk*>(base + ws.chunks);
+  const float* L = reinterpret_cast<const float*>(base + ws.L);
+  const float* tot = reinterpret_cast<const float*>(base + ws.tot);
+  float* dow = reinterpret_cast<float*>(base + ws.dow);
+  float* A = reinterpret_cast<float*>(base + ws.A);
+  float* dG = reinterpret_cast<float*>(base + ws.dG);
+  float* dtot = reinterpret_cast<float*>(base + ws.dtot);
+  float* dwp = reinterpret_cast<float*>(base + ws.dwp);
+  const int gx = dw_grid(d);
+  FIX_TRY(mark(p, FIX_STAGE_BWD_PRE, 0, st));
+  bwd_pre_kernel<<<dim3(gx, d.Hkv), 128, 0, st>>>(d, o_s, rstd_s,
+                                                   static_cast<const __nv_bfloat16*>(dy),
+                                                   static_cast<const __nv_bfloat16*>(w), dow, A, dwp);
+  FIX_TRY(launched());
+  dw_reduce_kernel<<<1, 128, 0, st>>>(dwp, gx * d.Hkv, d.Dv, static_cast<__nv_bfloat16*>(dw));
+  FIX_TRY(launched());
+  FIX_TRY(mark(p, FIX_STAGE_BWD_PRE, 1, st));
+  if (tc) {
+    FIX_TRY(tc_bwd(p, d, chunks, q, k, v, reinterpret_cast<const __nv_bfloat16*>(base + ws.vt), L,
+                   tot, m_s, dow, A, dq, dk, dv, dG, reinterpret_cast<int*>(base + ws.status), st));
+  } else {
+    const size_t smq = simt_dq_smem(d), smkv = simt_dkv_smem(d);
+    if (cudaFuncSetAttribute(dq_simt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smq) != cudaSuccess ||
+        cudaFuncSetAttribute(dkv_simt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smkv) != cudaSuccess)
+      return FIX_ERR_CUDA;
+    FIX_TRY(mark(p, FIX_STAGE_BWD_DQ, 0, st));
+    dq_simt_kernel<<<dim3(d.nchunks * 4, d.Hq), 256, smq, st>>>(
+        d, chunks, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+        static_cast<const __nv_bfloat16*>(v), L, tot, m_s, dow, static_cast<__nv_bfloat16*>(dq));
+    FIX_TRY(launched());
+    FIX_TRY(mark(p, FIX_STAGE_BWD_DQ, 1, st));
+    FIX_TRY(mark(p, FIX_STAGE_BWD_DKV, 0, st));
+    dkv_simt_kernel<<<dim3(d.nchunks * 4, d.Hkv), 256, smkv, st>>>(
+        d, chunks, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+        static_cast<const __nv_bfloat16*>(v), L, tot, m_s, dow, A,
+        static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv), dG);
+    FIX_TRY(launched());
+    FIX_TRY(mark(p, FIX_STAGE_BWD_DKV, 1, st));
+  }
+  FIX_TRY(mark(p, FIX_STAGE_BWD_DG, 0, st));
+  chunk_total_kernel<<<dim3(d.nchunks, d.Hkv), 128, 0, st>>>(d, chunks, dG, dtot);
+  FIX_TRY(launched());
+  reverse_cumsum_kernel<<<dim3(d.nchunks, d.Hkv), 128, 0, st>>>(d, chunks, dG, dtot, dg);
+  FIX_TRY(launched());
+  return mark(p, FIX_STAGE_BWD_DG, 1, st);
+}
+
+int fix_attn_kernel_count(const fix_attn_problem* p, int backward) {
+  Dims d;
+  if (make_dims(p, &d) != FIX_OK) return 0;
+  if (d.N == 0) return 0;
+  if (!backward) {
+    const bool tc = p->algo != FIX_ALGO_SIMT && tc_fwd_supported(d);
+    return 2 + (tc ? tc_fwd_kernel_count(d) : 1);
+  }
+  const bool tc = p->algo != FIX_ALGO_SIMT && tc_bwd_supported(d);
+  return 2 + 2 + (tc ? tc_bwd_kernel_count(d) : 2) + 2;
+}
+
+fix_status fix_attn_device_status(const void* workspace, void* stream) {
+  if (!workspace) return FIX_ERR_NULL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return FIX_ERR_CUDA;
+  int word = 0;
+  if (cudaMemcpy(&word, workspace, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return FIX_ERR_CUDA;
+  return word == 0 ? FIX_OK : FIX_ERR_DEVICE_TIMEOUT;
+}
+
+}  // extern "C"

@@ -1,0 +1,60 @@
+// Shared device-side definitions of the FiX attention library.
+//
+// Chunking.  Every sequence is cut into chunks of FIX_CHUNK = 128 tokens that
+// start at the sequence's first token (the last chunk may be short).  The
+// gate prefix sums are kept chunk-local: L_t[c] = sum of g over the chunk's
+// rows up to and including t, plus one total per chunk, tot_j[c].  For t in
+// chunk i and s in chunk j <= i the decay exponent is
+//     G_t - G_s = (L_t - L_s) + sum_{j <= j' < i} tot_j'
+// which never subtracts two large prefix sums (better fp32 accuracy than one
+// global cumsum) and lets the prefix pass run with no carry between chunks.
+#pragma once
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#define FIX_CHUNK 128
+
+namespace fix {
+
+// One chunk of the schedule: first token (index into the packed token
+// stream), number of valid rows, chunk index within its sequence and the
+// sequence's chunk count.  Chunks of a sequence are consecutive in the table,
+// so the sequence's first chunk has id (this id - j).
+struct Chunk {
+  int tok0;
+  int len;
+  int j;
+  int nch;
+};
+
+struct Dims {
+  int N;          // total tokens
+  int B, T;       // dense batch / length (T = N when packed)
+  int Hq, Hkv;    // heads
+  int Dk, Dv;     // head dims
+  int grp;        // Hq / Hkv
+  int nseq;       // sequences (B, or packed count)
+  int nchunks;    // chunks over all sequences
+  float scale;    // logit scale
+  float eps;      // RMSNorm epsilon
+};
+
+__device__ __forceinline__ float bf2f(__nv_bfloat16 x) { return __bfloat162float(x); }
+__device__ __forceinline__ __nv_bfloat16 f2bf(float x) { return __float2bfloat16_rn(x); }
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Status word at the head of the workspace.
+enum { FIX_DEV_OK = 0, FIX_DEV_TIMEOUT = 10 };
+
+}  // namespace fix

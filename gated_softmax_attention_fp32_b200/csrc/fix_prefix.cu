@@ -1,0 +1,141 @@
+// Gate prefix pass and packed-sequence schedule.
+//
+// FiX README, "Code Structure": intra_chunk_preprocess_fwd ("Intra-chunk
+// forward preprocessing") and inter_chunk_scale_v ("Inter-chunk scaling for
+// V").  Here one HBM-bound pass reads g and v once per chunk of 128 tokens and
+// writes
+//   L_t[c]  = sum_{r in chunk, r <= t} g_r[c]         chunk-local prefix (f32)
+//   tot[c]  = L_last[c]                                chunk total (f32)
+//   Vt_s[c] = v_s[c] * exp(L_last[c] - L_s[c])         values pre-decayed to the
+//                                                      chunk's last row (bf16)
+// For g <= 0 every factor exp(L_last - L_s) is <= 1, so Vt never overflows.
+// The backward reuses the same kernels for its reverse cumsum of dG.
+#include "fix_common.cuh"
+
+namespace fix {
+
+// Single CTA: turns sequence lengths (device cu_seqlens, or B sequences of T
+// tokens when cu is NULL) into the chunk table, sequences in order.  The table
+// has `cap` entries (the count the host derived from its cu_seqlens mirror);
+// every entry is first set empty, writes past `cap` are dropped and lengths
+// are clamped to the N tokens, so a device array that disagrees with the host
+// mirror cannot send any kernel outside its buffers.
+__global__ void __launch_bounds__(1024) schedule_kernel(const int64_t* __restrict__ cu, int nseq,
+                                                        int T, int N, int cap,
+                                                        Chunk* __restrict__ out) {
+  __shared__ int scan[1024];
+  for (int i = threadIdx.x; i < cap; i += blockDim.x) out[i] = Chunk{0, 0, 0, 0};
+  __syncthreads();
+  int carry = 0;
+  for (int first = 0; first < nseq; first += blockDim.x) {
+    const int i = first + threadIdx.x;
+    long long s0 = 0;
+    int L = 0;
+    if (i < nseq) {
+      if (cu) {
+        s0 = cu[i];
+        const long long e = cu[i + 1];
+        s0 = s0 < 0 ? 0 : (s0 > N ? N : s0);
+        L = (int)((e > N ? N : e) - s0);
+        if (L < 0) L = 0;
+      } else {
+        s0 = (long long)i * T;
+        L = T;
+      }
+    }
+    const int nc = (L + FIX_CHUNK - 1) / FIX_CHUNK;
+    scan[threadIdx.x] = nc;
+    __syncthreads();
+    for (int off = 1; off < (int)blockDim.x; off <<= 1) {
+      int add = threadIdx.x >= (unsigned)off ? scan[threadIdx.x - off] : 0;
+      __syncthreads();
+      scan[threadIdx.x] += add;
+      __syncthreads();
+    }
+    const int excl = carry + scan[threadIdx.x] - nc;
+    const int ncw = max(0, min(nc, cap - excl));   // chunks that fit the table
+    for (int j = 0; j < ncw; ++j) {
+      Chunk c;
+      c.tok0 = (int)(s0 + (long long)j * FIX_CHUNK);
+      c.len = min(FIX_CHUNK, L - j * FIX_CHUNK);
+      c.j = j;
+      c.nch = ncw;
+      out[excl + j] = c;
+    }
+    carry += scan[blockDim.x - 1];
+    __syncthreads();
+  }
+}
+
+// grid (nchunks, Hkv), block 128: thread = channel.
+__global__ void __launch_bounds__(128) prefix_kernel(Dims d, const Chunk* __restrict__ chunks,
+                                                     const float* __restrict__ g,
+                                                     const __nv_bfloat16* __restrict__ v,
+                                                     float* __restrict__ L,
+                                                     __nv_bfloat16* __restrict__ vt,
+                                                     float* __restrict__ tot) {
+  const int ci = blockIdx.x, kv = blockIdx.y, c = threadIdx.x;
+  if (c >= d.Dv) return;
+  const Chunk ch = chunks[ci];
+  const size_t rs = (size_t)d.Hkv * d.Dv;
+  const size_t base = (size_t)ch.tok0 * rs + (size_t)kv * d.Dv + c;
+  float acc = 0.f;
+  int r = 0;
+  for (; r + 8 <= ch.len; r += 8) {
+    float x[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) x[u] = g[base + (size_t)(r + u) * rs];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      acc += x[u];
+      L[base + (size_t)(r + u) * rs] = acc;
+    }
+  }
+  for (; r < ch.len; ++r) {
+    acc += g[base + (size_t)r * rs];
+    L[base + (size_t)r * rs] = acc;
+  }
+  tot[((size_t)ci * d.Hkv + kv) * d.Dv + c] = acc;
+  if (vt) {
+    for (r = 0; r < ch.len; ++r) {
+      const size_t a = base + (size_t)r * rs;
+      vt[a] = f2bf(bf2f(v[a]) * expf(acc - L[a]));
+    }
+  }
+}
+
+// Reverse cumsum of dG within each sequence (dg_r = sum_{t >= r} dG_t), in two
+// launches over the same chunk table: chunk totals, then local reverse scans
+// plus the totals of the later chunks of the same sequence.
+__global__ void __launch_bounds__(128) chunk_total_kernel(Dims d, const Chunk* __restrict__ chunks,
+                                                          const float* __restrict__ x,
+                                                          float* __restrict__ tot) {
+  const int ci = blockIdx.x, kv = blockIdx.y, c = threadIdx.x;
+  if (c >= d.Dv) return;
+  const Chunk ch = chunks[ci];
+  const size_t rs = (size_t)d.Hkv * d.Dv;
+  const size_t base = (size_t)ch.tok0 * rs + (size_t)kv * d.Dv + c;
+  float acc = 0.f;
+  for (int r = 0; r < ch.len; ++r) acc += x[base + (size_t)r * rs];
+  tot[((size_t)ci * d.Hkv + kv) * d.Dv + c] = acc;
+}
+
+__global__ void __launch_bounds__(128) reverse_cumsum_kernel(Dims d, const Chunk* __restrict__ chunks,
+                                                             const float* __restrict__ x,
+                                                             const float* __restrict__ tot,
+                                                             float* __restrict__ out) {
+  const int ci = blockIdx.x, kv = blockIdx.y, c = threadIdx.x;
+  if (c >= d.Dv) return;
+  const Chunk ch = chunks[ci];
+  const size_t rs = (size_t)d.Hkv * d.Dv;
+  const size_t base = (size_t)ch.tok0 * rs + (size_t)kv * d.Dv + c;
+  float acc = 0.f;
+  const int first = ci - ch.j;
+  for (int jj = ch.nch - 1; jj > ch.j; --jj) acc += tot[((size_t)(first + jj) * d.Hkv + kv) * d.Dv + c];
+  for (int r = ch.len - 1; r >= 0; --r) {
+    acc += x[base + (size_t)r * rs];
+    out[base + (size_t)r * rs] = acc;
+  }
+}
+
+}  // namespace fix

@@ -1,0 +1,477 @@
+// Exact fp32 CUDA-core kernels for FiX attention (FIX_ALGO_SIMT).
+//
+// Every decay factor exp(G_t[c] - G_s[c]) is formed element by element from
+// the chunk-local prefix sums (no factorisation through a reference row), so
+// these kernels are slow but follow the definition directly:
+//   o_t[c] = sum_{s<=t} exp(S_ts - m_t) exp(G_t[c] - G_s[c]) v_s[c]
+// (FiX poster abstract: element-wise forgetting on the values, softmax
+// denominator dropped under the RMSNorm).  They are a second GPU path that the
+// tensor-core kernels are cross-checked against.
+//
+// Tiling: a CTA owns 32 rows (query rows for fwd / dq, key rows for dk/dv) of
+// one 128-token chunk; keys (or queries) stream through shared memory in
+// tiles of 32.  Decay exponents across chunks add the chunk totals between
+// the two chunks (see fix_common.cuh).
+#include "fix_common.cuh"
+
+namespace fix {
+
+constexpr int ST = 32;          // rows per CTA and per streamed tile
+constexpr unsigned FULL = 0xffffffffu;
+
+// ---------------------------------------------------------------------------
+// Forward.  grid (nchunks * 4, Hq), block 256 (8 warps x 4 query rows).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) fwd_simt_kernel(
+    Dims d, const Chunk* __restrict__ chunks, const __nv_bfloat16* __restrict__ q,
+    const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
+    const float* __restrict__ L, const float* __restrict__ tot,
+    const __nv_bfloat16* __restrict__ w, void* __restrict__ y, int y_f32,
+    float* __restrict__ o_s, float* __restrict__ m_s, float* __restrict__ rstd_s) {
+  extern __shared__ float sm[];
+  const int Dk = d.Dk, Dv = d.Dv;
+  float* sQ = sm;                       // [ST][Dk]
+  float* sLq = sQ + ST * Dk;            // [ST][Dv]
+  float* sK = sLq + ST * Dv;            // [ST][Dk+1]
+  float* sV = sK + ST * (Dk + 1);       // [ST][Dv]
+  float* sLk = sV + ST * Dv;            // [ST][Dv]
+
+  const int ci = blockIdx.x >> 2, r0 = (blockIdx.x & 3) * ST;
+  const int h = blockIdx.y, kv = h / d.grp;
+  const Chunk ch = chunks[ci];
+  if (r0 >= ch.len) return;
+  const int nrows = min(ST, ch.len - r0);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const size_t qrs = (size_t)d.Hq * Dk, krs = (size_t)d.Hkv * Dk;
+  const size_t vrs = (size_t)d.Hkv * Dv, ors = (size_t)d.Hq * Dv;
+  const int seq0 = ch.tok0 - ch.j * FIX_CHUNK;
+  const int first = ci - ch.j;
+
+  for (int e = threadIdx.x; e < ST * Dk; e += blockDim.x) {
+    const int r = e / Dk, dd = e % Dk;
+    sQ[e] = r < nrows ? bf2f(q[(size_t)(ch.tok0 + r0 + r) * qrs + (size_t)h * Dk + dd]) : 0.f;
+  }
+  for (int e = threadIdx.x; e < ST * Dv; e += blockDim.x) {
+    const int r = e / Dv, c = e % Dv;
+    sLq[e] = r < nrows ? L[(size_t)(ch.tok0 + r0 + r) * vrs + (size_t)kv * Dv + c] : 0.f;
+  }
+
+  float o[4][4], mrow[4], delta[4];
+#pragma unroll
+  for (int a = 0; a < 4; ++a) {
+    mrow[a] = -INFINITY;
+    delta[a] = 0.f;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) o[a][u] = 0.f;
+  }
+
+  for (int jj = ch.j; jj >= 0; --jj) {
+    if (jj < ch.j) {  // delta = sum of chunk totals from jj up to (not incl.) this chunk
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int c = lane + 32 * u;
+        if (c < Dv) delta[u] += tot[((size_t)(first + jj) * d.Hkv + kv) * Dv + c];
+      }
+    }
+    const int klen = (jj == ch.j) ? (r0 + nrows) : FIX_CHUNK;
+    for (int kt = 0; kt < klen; kt += ST) {
+      const int nk = min(ST, klen - kt);
+      const int ktok = seq0 + jj * FIX_CHUNK + kt;
+      __syncthreads();
+      for (int e = threadIdx.x; e < ST * Dk; e += blockDim.x) {
+        const int s = e / Dk, dd = e % Dk;
+        sK[s * (Dk + 1) + dd] = s < nk ? bf2f(k[(size_t)(ktok + s) * krs + (size_t)kv * Dk + dd]) : 0.f;
+      }
+      for (int e = threadIdx.x; e < ST * Dv; e += blockDim.x) {
+        const int s = e / Dv, c = e % Dv;
+        const size_t a = (size_t)(ktok + s) * vrs + (size_t)kv * Dv + c;
+        sV[e] = s < nk ? bf2f(v[a]) : 0.f;
+        sLk[e] = s < nk ? L[a] : 0.f;
+      }
+      __syncthreads();
+#pragma unroll
+      for (int rr = 0; rr < 4; ++rr) {
+        const int r = warp * 4 + rr;
+        if (r >= nrows) break;
+        const int tpos = ch.j * FIX_CHUNK + r0 + r;
+        const int spos = jj * FIX_CHUNK + kt + lane;
+        const bool valid = lane < nk && spos <= tpos;
+        float acc = 0.f;
+        for (int dd = 0; dd < Dk; ++dd) acc += sQ[r * Dk + dd] * sK[lane * (Dk + 1) + dd];
+        const float sv = valid ? acc * d.scale : -INFINITY;
+        const float mnew = fmaxf(mrow[rr], warp_max(sv));
+        if (mnew == -INFINITY) continue;
+        const float alpha = (mrow[rr] == mnew) ? 1.f : expf(mrow[rr] - mnew);
+        mrow[rr] = mnew;
+        float lq[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          o[rr][u] *= alpha;
+          const int c = lane + 32 * u;
+          lq[u] = c < Dv ? sLq[r * Dv + c] + delta[u] : 0.f;
+        }
+        const float p = valid ? expf(sv - mnew) : 0.f;
+        for (int s = 0; s < nk; ++s) {
+          const float ps = __shfl_sync(FULL, p, s);
+          if (ps == 0.f) continue;  // masked key: its factor may be out of range
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int c = lane + 32 * u;
+            if (c < Dv) o[rr][u] += ps * expf(lq[u] - sLk[s * Dv + c]) * sV[s * Dv + c];
+          }
+        }
+      }
+    }
+  }
+
+#pragma unroll
+  for (int rr = 0; rr < 4; ++rr) {
+    const int r = warp * 4 + rr;
+    if (r >= nrows) break;
+    float ss = 0.f;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) ss += o[rr][u] * o[rr][u];
+    ss = warp_sum(ss);
+    const float rstd = 1.f / sqrtf(ss / (float)Dv + d.eps);
+    const size_t tok = (size_t)(ch.tok0 + r0 + r);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int c = lane + 32 * u;
+      if (c >= Dv) continue;
+      const size_t a = tok * ors + (size_t)h * Dv + c;
+      const float yv = o[rr][u] * rstd * bf2f(w[c]);
+      if (y_f32) reinterpret_cast<float*>(y)[a] = yv;
+      else reinterpret_cast<__nv_bfloat16*>(y)[a] = f2bf(yv);
+      if (o_s) o_s[a] = o[rr][u];
+    }
+    if (lane == 0 && m_s) {
+      m_s[tok * d.Hq + h] = mrow[rr];
+      rstd_s[tok * d.Hq + h] = rstd;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Backward preprocess (shared by all kernel families).  RMSNorm backward:
+//   n = o rstd, dn = dy w, do = rstd (dn - n mean(dn n)),
+// A_t[c] = sum_{h in group} do_t[c] o_t[c] (the per-row part of dG_t) and
+// per-CTA partial sums of dw = sum dy n.
+// grid (G, Hkv), block 128 (4 warps); a warp handles one token at a time.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(128) bwd_pre_kernel(
+    Dims d, const float* __restrict__ o_s, const float* __restrict__ rstd_s,
+    const __nv_bfloat16* __restrict__ dy, const __nv_bfloat16* __restrict__ w,
+    float* __restrict__ do_ws, float* __restrict__ A, float* __restrict__ dwpart) {
+  __shared__ float red[4][128];
+  const int Dv = d.Dv, kv = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float wv[4], dwl[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int c = lane + 32 * u;
+    wv[u] = c < Dv ? bf2f(w[c]) : 0.f;
+    dwl[u] = 0.f;
+  }
+  const size_t ors = (size_t)d.Hq * Dv, vrs = (size_t)d.Hkv * Dv;
+  for (int t = blockIdx.x * 4 + warp; t < d.N; t += gridDim.x * 4) {
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int hh = 0; hh < d.grp; ++hh) {
+      const int h = kv * d.grp + hh;
+      const float r = rstd_s[(size_t)t * d.Hq + h];
+      float ov[4], dn[4], n[4], dot = 0.f;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int c = lane + 32 * u;
+        const size_t a = (size_t)t * ors + (size_t)h * Dv + c;
+        ov[u] = c < Dv ? o_s[a] : 0.f;
+        const float dyv = c < Dv ? bf2f(dy[a]) : 0.f;
+        n[u] = ov[u] * r;
+        dn[u] = dyv * wv[u];
+        dot += dn[u] * n[u];
+        dwl[u] += dyv * n[u];
+      }
+      dot = warp_sum(dot) / (float)Dv;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int c = lane + 32 * u;
+        if (c >= Dv) continue;
+        const float dov = r * (dn[u] - n[u] * dot);
+        do_ws[(size_t)t * ors + (size_t)h * Dv + c] = dov;
+        acc[u] += dov * ov[u];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int c = lane + 32 * u;
+      if (c < Dv) A[(size_t)t * vrs + (size_t)kv * Dv + c] = acc[u];
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < 4; ++u) red[warp][lane + 32 * u] = dwl[u];
+  __syncthreads();
+  const int c = threadIdx.x;
+  if (c < Dv) {
+    const float s = red[0][c] + red[1][c] + red[2][c] + red[3][c];
+    dwpart[((size_t)blockIdx.y * gridDim.x + blockIdx.x) * Dv + c] = s;
+  }
+}
+
+// dw = sum of the partials in a fixed order (deterministic).  One CTA.
+__global__ void __launch_bounds__(128) dw_reduce_kernel(const float* __restrict__ parts, int nparts,
+                                                        int Dv, __nv_bfloat16* __restrict__ dw) {
+  const int c = threadIdx.x;
+  if (c >= Dv) return;
+  float s = 0.f;
+  for (int i = 0; i < nparts; ++i) s += parts[(size_t)i * Dv + c];
+  dw[c] = f2bf(s);
+}
+
+// ---------------------------------------------------------------------------
+// dq.  grid (nchunks * 4, Hq), block 256: 32 query rows per CTA.
+//   dP_ts = sum_c do_t[c] exp(G_t[c] - G_s[c]) v_s[c],  dS = P dP,
+//   dq_t  = scale sum_s dS_ts k_s
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) dq_simt_kernel(
+    Dims d, const Chunk* __restrict__ chunks, const __nv_bfloat16* __restrict__ q,
+    const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
+    const float* __restrict__ L, const float* __restrict__ tot,
+    const float* __restrict__ m_s, const float* __restrict__ do_ws,
+    __nv_bfloat16* __restrict__ dq) {
+  extern __shared__ float sm[];
+  const int Dk = d.Dk, Dv = d.Dv;
+  float* sQ = sm;                        // [ST][Dk]
+  float* sDo = sQ + ST * Dk;             // [ST][Dv]
+  float* sLq = sDo + ST * Dv;            // [ST][Dv]
+  float* sM = sLq + ST * Dv;             // [ST]
+  float* sDelta = sM + ST;               // [Dv]
+  float* sK = sDelta + Dv;               // [ST][Dk+1]
+  float* sV = sK + ST * (Dk + 1);        // [ST][Dv+1]
+  float* sLk = sV + ST * (Dv + 1);       // [ST][Dv+1]
+
+  const int ci = blockIdx.x >> 2, r0 = (blockIdx.x & 3) * ST;
+  const int h = blockIdx.y, kv = h / d.grp;
+  const Chunk ch = chunks[ci];
+  if (r0 >= ch.len) return;
+  const int nrows = min(ST, ch.len - r0);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const size_t qrs = (size_t)d.Hq * Dk, krs = (size_t)d.Hkv * Dk;
+  const size_t vrs = (size_t)d.Hkv * Dv, ors = (size_t)d.Hq * Dv;
+  const int seq0 = ch.tok0 - ch.j * FIX_CHUNK;
+  const int first = ci - ch.j;
+
+  for (int e = threadIdx.x; e < ST * Dk; e += blockDim.x) {
+    const int r = e / Dk, dd = e % Dk;
+    sQ[e] = r < nrows ? bf2f(q[(size_t)(ch.tok0 + r0 + r) * qrs + (size_t)h * Dk + dd]) : 0.f;
+  }
+  for (int e = threadIdx.x; e < ST * Dv; e += blockDim.x) {
+    const int r = e / Dv, c = e % Dv;
+    const size_t tok = (size_t)(ch.tok0 + r0 + r);
+    sDo[e] = r < nrows ? do_ws[tok * ors + (size_t)h * Dv + c] : 0.f;
+    sLq[e] = r < nrows ? L[tok * vrs + (size_t)kv * Dv + c] : 0.f;
+  }
+  for (int r = threadIdx.x; r < ST; r += blockDim.x)
+    sM[r] = r < nrows ? m_s[(size_t)(ch.tok0 + r0 + r) * d.Hq + h] : 0.f;
+  for (int c = threadIdx.x; c < Dv; c += blockDim.x) sDelta[c] = 0.f;
+
+  float acc[4][4];
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int u = 0; u < 4; ++u) acc[a][u] = 0.f;
+
+  for (int jj = ch.j; jj >= 0; --jj) {
+    const int klen = (jj == ch.j) ? (r0 + nrows) : FIX_CHUNK;
+    for (int kt = 0; kt < klen; kt += ST) {
+      const int nk = min(ST, klen - kt);
+      const int ktok = seq0 + jj * FIX_CHUNK + kt;
+      __syncthreads();
+      if (kt == 0 && jj < ch.j)
+        for (int c = threadIdx.x; c < Dv; c += blockDim.x)
+          sDelta[c] += tot[((size_t)(first + jj) * d.Hkv + kv) * Dv + c];
+      for (int e = threadIdx.x; e < ST * Dk; e += blockDim.x) {
+        const int s = e / Dk, dd = e % Dk;
+        sK[s * (Dk + 1) + dd] = s < nk ? bf2f(k[(size_t)(ktok + s) * krs + (size_t)kv * Dk + dd]) : 0.f;
+      }
+      for (int e = threadIdx.x; e < ST * Dv; e += blockDim.x) {
+        const int s = e / Dv, c = e % Dv;
+        const size_t a = (size_t)(ktok + s) * vrs + (size_t)kv * Dv + c;
+        sV[s * (Dv + 1) + c] = s < nk ? bf2f(v[a]) : 0.f;
+        sLk[s * (Dv + 1) + c] = s < nk ? L[a] : 0.f;
+      }
+      __syncthreads();
+#pragma unroll
+      for (int rr = 0; rr < 4; ++rr) {
+        const int r = warp * 4 + rr;
+        if (r >= nrows) break;
+        const int tpos = ch.j * FIX_CHUNK + r0 + r;
+        const int spos = jj * FIX_CHUNK + kt + lane;
+        const bool valid = lane < nk && spos <= tpos;
+        float ds = 0.f;
+        if (valid) {
+          float sacc = 0.f;
+          for (int dd = 0; dd < Dk; ++dd) sacc += sQ[r * Dk + dd] * sK[lane * (Dk + 1) + dd];
+          const float p = expf(sacc * d.scale - sM[r]);
+          if (p != 0.f) {
+            float dp = 0.f;
+            for (int c = 0; c < Dv; ++c)
+              dp += sDo[r * Dv + c] *
+                    expf(sLq[r * Dv + c] + sDelta[c] - sLk[lane * (Dv + 1) + c]) *
+                    sV[lane * (Dv + 1) + c];
+            ds = p * dp;
+          }
+        }
+        for (int s = 0; s < nk; ++s) {
+          const float dss = __shfl_sync(FULL, ds, s);
+          if (dss == 0.f) continue;
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int dd = lane + 32 * u;
+            if (dd < Dk) acc[rr][u] += dss * sK[s * (Dk + 1) + dd];
+          }
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int rr = 0; rr < 4; ++rr) {
+    const int r = warp * 4 + rr;
+    if (r >= nrows) break;
+    const size_t tok = (size_t)(ch.tok0 + r0 + r);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int dd = lane + 32 * u;
+      if (dd < Dk) dq[tok * qrs + (size_t)h * Dk + dd] = f2bf(acc[rr][u] * d.scale);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// dk, dv and dG.  grid (nchunks * 4, Hkv), block 256: 32 key rows per CTA,
+// 4 per warp, looping over the kv group's q heads and every later query row.
+//   dv_s += P_ts D_ts do_t ;  dk_s += scale dS_ts q_t ;
+//   dG_s  = A_s - v_s dv_s   (A from bwd_pre_kernel)
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) dkv_simt_kernel(
+    Dims d, const Chunk* __restrict__ chunks, const __nv_bfloat16* __restrict__ q,
+    const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
+    const float* __restrict__ L, const float* __restrict__ tot,
+    const float* __restrict__ m_s, const float* __restrict__ do_ws,
+    const float* __restrict__ A, __nv_bfloat16* __restrict__ dk,
+    __nv_bfloat16* __restrict__ dv, float* __restrict__ dG) {
+  extern __shared__ float sm[];
+  const int Dk = d.Dk, Dv = d.Dv;
+  float* sQ = sm;                        // [ST][Dk]
+  float* sDo = sQ + ST * Dk;             // [ST][Dv]
+  float* sLq = sDo + ST * Dv;            // [ST][Dv]
+  float* sM = sLq + ST * Dv;             // [ST]
+
+  const int ci = blockIdx.x >> 2, r0 = (blockIdx.x & 3) * ST;
+  const int kv = blockIdx.y;
+  const Chunk ch = chunks[ci];
+  if (r0 >= ch.len) return;
+  const int nkeys = min(ST, ch.len - r0);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const size_t qrs = (size_t)d.Hq * Dk, krs = (size_t)d.Hkv * Dk;
+  const size_t vrs = (size_t)d.Hkv * Dv, ors = (size_t)d.Hq * Dv;
+  const int first = ci - ch.j;
+
+  float kr[4][4], vr[4][4], lk[4][4], gk[4][4], gv[4][4];
+#pragma unroll
+  for (int a = 0; a < 4; ++a) {
+    const int key = warp * 4 + a;
+    const size_t tok = (size_t)(ch.tok0 + r0 + min(key, nkeys - 1));
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int dd = lane + 32 * u;
+      kr[a][u] = dd < Dk ? bf2f(k[tok * krs + (size_t)kv * Dk + dd]) : 0.f;
+      vr[a][u] = dd < Dv ? bf2f(v[tok * vrs + (size_t)kv * Dv + dd]) : 0.f;
+      lk[a][u] = dd < Dv ? L[tok * vrs + (size_t)kv * Dv + dd] : 0.f;
+      gk[a][u] = 0.f;
+      gv[a][u] = 0.f;
+    }
+  }
+
+  for (int hh = 0; hh < d.grp; ++hh) {
+    const int h = kv * d.grp + hh;
+    float delta[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int ii = ch.j; ii < ch.nch; ++ii) {
+      if (ii > ch.j) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int c = lane + 32 * u;
+          if (c < Dv) delta[u] += tot[((size_t)(first + ii - 1) * d.Hkv + kv) * Dv + c];
+        }
+      }
+      const Chunk qc = chunks[first + ii];
+      const int qstart = (ii == ch.j) ? r0 : 0;
+      for (int qt = qstart; qt < qc.len; qt += ST) {
+        const int nq = min(ST, qc.len - qt);
+        __syncthreads();
+        for (int e = threadIdx.x; e < ST * Dk; e += blockDim.x) {
+          const int r = e / Dk, dd = e % Dk;
+          sQ[e] = r < nq ? bf2f(q[(size_t)(qc.tok0 + qt + r) * qrs + (size_t)h * Dk + dd]) : 0.f;
+        }
+        for (int e = threadIdx.x; e < ST * Dv; e += blockDim.x) {
+          const int r = e / Dv, c = e % Dv;
+          const size_t tok = (size_t)(qc.tok0 + qt + r);
+          sDo[e] = r < nq ? do_ws[tok * ors + (size_t)h * Dv + c] : 0.f;
+          sLq[e] = r < nq ? L[tok * vrs + (size_t)kv * Dv + c] : 0.f;
+        }
+        for (int r = threadIdx.x; r < ST; r += blockDim.x)
+          sM[r] = r < nq ? m_s[(size_t)(qc.tok0 + qt + r) * d.Hq + h] : 0.f;
+        __syncthreads();
+        for (int r = 0; r < nq; ++r) {
+          const int tpos = ii * FIX_CHUNK + qt + r;
+#pragma unroll
+          for (int a = 0; a < 4; ++a) {
+            const int key = warp * 4 + a;
+            const int spos = ch.j * FIX_CHUNK + r0 + key;
+            if (key >= nkeys || spos > tpos) continue;  // warp-uniform
+            float sacc = 0.f;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int dd = lane + 32 * u;
+              if (dd < Dk) sacc += sQ[r * Dk + dd] * kr[a][u];
+            }
+            sacc = warp_sum(sacc);
+            const float p = expf(sacc * d.scale - sM[r]);
+            if (p == 0.f) continue;
+            float dc[4], dp = 0.f;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int c = lane + 32 * u;
+              dc[u] = c < Dv ? expf(sLq[r * Dv + c] + delta[u] - lk[a][u]) : 0.f;
+              if (c < Dv) dp += sDo[r * Dv + c] * dc[u] * vr[a][u];
+            }
+            dp = warp_sum(dp);
+            const float ds = p * dp;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int dd = lane + 32 * u;
+              if (dd < Dk) gk[a][u] += ds * sQ[r * Dk + dd];
+              if (dd < Dv) gv[a][u] += p * dc[u] * sDo[r * Dv + dd];
+            }
+          }
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int a = 0; a < 4; ++a) {
+    const int key = warp * 4 + a;
+    if (key >= nkeys) break;
+    const size_t tok = (size_t)(ch.tok0 + r0 + key);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int dd = lane + 32 * u;
+      if (dd < Dk) dk[tok * krs + (size_t)kv * Dk + dd] = f2bf(gk[a][u] * d.scale);
+      if (dd < Dv) {
+        const size_t av = tok * vrs + (size_t)kv * Dv + dd;
+        dv[av] = f2bf(gv[a][u]);
+        dG[av] = A[av] - vr[a][u] * gv[a][u];
+      }
+    }
+  }
+}
+
+}  // namespace fix

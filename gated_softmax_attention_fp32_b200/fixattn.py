@@ -1,0 +1,216 @@
+"""Python binding of libfixattn.so (include/fix_attn.h): argument marshalling only.
+
+Every step of FiX attention runs in the library's CUDA kernels; this module
+allocates the output tensors and the workspace with PyTorch, passes raw device
+pointers and the current CUDA stream through ctypes, and turns status codes
+into exceptions.  There is no fallback: if the library is missing or the
+device is not a B200 (sm_100), calls raise.
+
+Names mirror the C ABI: ``fix_attn_fwd``, ``fix_attn_bwd``,
+``fix_attn_workspace_bytes``, ``fix_attn_device_status``; ``fix_attn`` wraps
+the pair in a ``torch.autograd.Function`` with the FiX README's argument order
+("Quick Start": q, k, v, g, then cu_seqlens / o_norm_weight).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+__all__ = ["load", "Problem", "fix_attn_fwd", "fix_attn_bwd", "fix_attn_workspace_bytes",
+           "fix_attn_device_status", "fix_attn", "FixStatusError", "LIB_PATH", "EXPORTS"]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfixattn.so")
+EXPORTS = ("fix_attn_workspace_bytes", "fix_attn_fwd", "fix_attn_bwd", "fix_attn_device_status",
+           "fix_attn_kernel_count", "fix_attn_status_string")
+STAGES = ("fwd_prefix", "fwd_attn", "bwd_prefix", "bwd_pre", "bwd_dq", "bwd_dkv", "bwd_dg")
+
+ALGOS = {"auto": 0, "simt": 1, "tc": 2}
+_lib = None
+
+
+class Problem(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("seqlen", ctypes.c_int32),
+                ("num_q_heads", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32),
+                ("head_dim_k", ctypes.c_int32), ("head_dim_v", ctypes.c_int32),
+                ("num_seqs", ctypes.c_int32), ("y_dtype", ctypes.c_int32),
+                ("algo", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("cu_seqlens", ctypes.c_void_p), ("cu_seqlens_host", ctypes.c_void_p),
+                ("scale", ctypes.c_float), ("eps", ctypes.c_float),
+                ("events", ctypes.c_void_p)]
+
+
+class FixStatusError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {status_string(code)} (code {code})")
+
+
+def load():
+    """Load libfixattn.so (once).  Raises if it is missing: there is no fallback."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"FiX CUDA library not built: {LIB_PATH} is missing "
+                           "(run python -m gated_softmax_attention_fp32_b200.build)")
+    lib = ctypes.CDLL(LIB_PATH)
+    P = ctypes.POINTER(Problem)
+    vp, sz = ctypes.c_void_p, ctypes.c_size_t
+    lib.fix_attn_workspace_bytes.argtypes = [P, ctypes.c_int]
+    lib.fix_attn_workspace_bytes.restype = sz
+    lib.fix_attn_fwd.argtypes = [P] + [vp] * 10 + [sz, vp]
+    lib.fix_attn_fwd.restype = ctypes.c_int
+    lib.fix_attn_bwd.argtypes = [P] + [vp] * 15 + [sz, vp]
+    lib.fix_attn_bwd.restype = ctypes.c_int
+    lib.fix_attn_device_status.argtypes = [vp, vp]
+    lib.fix_attn_device_status.restype = ctypes.c_int
+    lib.fix_attn_kernel_count.argtypes = [P, ctypes.c_int]
+    lib.fix_attn_kernel_count.restype = ctypes.c_int
+    lib.fix_attn_status_string.argtypes = [ctypes.c_int]
+    lib.fix_attn_status_string.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def status_string(code: int) -> str:
+    return load().fix_attn_status_string(int(code)).decode()
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def make_problem(q, k, v, cu_seqlens=None, cu_seqlens_host=None, scale=None, eps=1e-6,
+                 y_dtype=torch.bfloat16, algo="auto", events=None):
+    """Build the C problem descriptor from [B,T,H,D] tensors.  Returns
+    (Problem, keepalive) where keepalive holds the host cu_seqlens tensor and
+    the event-handle array.  ``events``: optional list of 2*len(STAGES)
+    ``torch.cuda.Event(enable_timing=True)`` recorded around each stage."""
+    B, T, Hq, Dk = q.shape
+    Hkv, Dv = v.shape[2], v.shape[3]
+    p = Problem()
+    p.batch, p.seqlen, p.num_q_heads, p.num_kv_heads = B, T, Hq, Hkv
+    p.head_dim_k, p.head_dim_v = Dk, Dv
+    p.y_dtype = 1 if y_dtype == torch.float32 else 0
+    p.algo = ALGOS[algo]
+    p.reserved = 0
+    p.scale = float(scale) if scale is not None else 0.0
+    p.eps = float(eps)
+    keep = None
+    if cu_seqlens is not None:
+        if cu_seqlens_host is None:
+            cu_seqlens_host = cu_seqlens.detach().to("cpu")
+        keep = cu_seqlens_host.to(torch.int64).contiguous()
+        p.num_seqs = keep.numel() - 1
+        p.cu_seqlens = cu_seqlens.data_ptr()
+        p.cu_seqlens_host = keep.data_ptr()
+    else:
+        p.num_seqs = 0
+    if events is not None:
+        assert len(events) == 2 * len(STAGES)
+        arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
+        p.events = ctypes.cast(arr, ctypes.c_void_p)
+        keep = (keep, arr)
+    return p, keep
+
+
+def fix_attn_workspace_bytes(problem: Problem, backward: bool) -> int:
+    return int(load().fix_attn_workspace_bytes(ctypes.byref(problem), int(bool(backward))))
+
+
+def fix_attn_kernel_count(problem: Problem, backward: bool) -> int:
+    return int(load().fix_attn_kernel_count(ctypes.byref(problem), int(bool(backward))))
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def fix_attn_fwd(q, k, v, g, o_norm_weight, cu_seqlens=None, cu_seqlens_host=None, scale=None,
+                 eps=1e-6, y_dtype=torch.bfloat16, save=True, algo="auto", workspace=None,
+                 out=None, stream=None, events=None):
+    """Forward.  Returns (y, saved) with saved = (o, m, rstd) or None."""
+    lib = load()
+    p, keep = make_problem(q, k, v, cu_seqlens, cu_seqlens_host, scale, eps, y_dtype, algo,
+                           events)
+    B, T, Hq, _ = q.shape
+    Dv = v.shape[3]
+    dev = q.device
+    y = out if out is not None else torch.empty(B, T, Hq, Dv, device=dev, dtype=y_dtype)
+    saved = None
+    if save:
+        saved = (torch.empty(B, T, Hq, Dv, device=dev, dtype=torch.float32),
+                 torch.empty(B, T, Hq, device=dev, dtype=torch.float32),
+                 torch.empty(B, T, Hq, device=dev, dtype=torch.float32))
+    nbytes = fix_attn_workspace_bytes(p, False)
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 1), device=dev, dtype=torch.uint8)
+    s = lib.fix_attn_fwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(o_norm_weight),
+                         _ptr(y), *(map(_ptr, saved) if saved else (None, None, None)),
+                         _ptr(workspace), workspace.numel(), _stream(stream))
+    if s != 0:
+        raise FixStatusError(s, "fix_attn_fwd")
+    del keep
+    return y, saved
+
+
+def fix_attn_bwd(q, k, v, g, o_norm_weight, dy, saved, cu_seqlens=None, cu_seqlens_host=None,
+                 scale=None, eps=1e-6, algo="auto", workspace=None, stream=None, events=None,
+                 out=None):
+    """Backward of sum(dy * y).  Returns dq, dk, dv, dg, dw (``out`` may
+    supply those five tensors)."""
+    lib = load()
+    p, keep = make_problem(q, k, v, cu_seqlens, cu_seqlens_host, scale, eps, torch.bfloat16, algo,
+                           events)
+    if out is not None:
+        dq, dk, dv, dg, dw = out
+    else:
+        dq = torch.empty_like(q)
+        dk = torch.empty_like(k)
+        dv = torch.empty_like(v)
+        dg = torch.empty_like(g)
+        dw = torch.empty_like(o_norm_weight)
+    nbytes = fix_attn_workspace_bytes(p, True)
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 1), device=q.device, dtype=torch.uint8)
+    o_s, m_s, r_s = saved
+    s = lib.fix_attn_bwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(o_norm_weight),
+                         _ptr(dy), _ptr(o_s), _ptr(m_s), _ptr(r_s), _ptr(dq), _ptr(dk), _ptr(dv),
+                         _ptr(dg), _ptr(dw), _ptr(workspace), workspace.numel(), _stream(stream))
+    if s != 0:
+        raise FixStatusError(s, "fix_attn_bwd")
+    del keep
+    return dq, dk, dv, dg, dw
+
+
+def fix_attn_device_status(workspace, stream=None) -> int:
+    return int(load().fix_attn_device_status(_ptr(workspace), _stream(stream)))
+
+
+class _FixAttn(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, q, k, v, g, w, cu_seqlens, cu_host, scale, eps, algo):
+        y, saved = fix_attn_fwd(q, k, v, g, w, cu_seqlens, cu_host, scale, eps, save=True,
+                                algo=algo)
+        ctx.save_for_backward(q, k, v, g, w, *saved)
+        ctx.cfg = (cu_seqlens, cu_host, scale, eps, algo)
+        return y
+
+    @staticmethod
+    def backward(ctx, dy):
+        q, k, v, g, w, o_s, m_s, r_s = ctx.saved_tensors
+        cu, cu_host, scale, eps, algo = ctx.cfg
+        dq, dk, dv, dg, dw = fix_attn_bwd(q, k, v, g, w, dy.to(torch.bfloat16).contiguous(),
+                                          (o_s, m_s, r_s), cu, cu_host, scale, eps, algo)
+        return dq, dk, dv, dg, dw, None, None, None, None, None
+
+
+def fix_attn(q, k, v, g, o_norm_weight, cu_seqlens=None, cu_seqlens_host=None, scale=None,
+             eps=1e-6, algo="auto"):
+    """y = RMSNorm(FiX attention(q, k, v, g)) * o_norm_weight, differentiable."""
+    return _FixAttn.apply(q, k, v, g, o_norm_weight, cu_seqlens, cu_seqlens_host, scale, eps, algo)

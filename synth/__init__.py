@@ -43,6 +43,7 @@ class Case:
     seqlens: Optional[tuple] = None  # packed sequence lengths (B must be 1)
     varlen_draw: Optional[tuple] = None  # (total, lo, hi): lengths drawn U{lo..hi}
     channel_bias_std: float = 0.0   # per-channel shift of x (heterogeneous decay)
+    raw_gate: bool = False          # g = x itself (the README example draws g = randn)
     eps: float = 1e-6
     seed: int = 0
     name: str = ""
@@ -107,7 +108,7 @@ def draw(case: Case) -> dict:
     if case.channel_bias_std:
         bias = torch.randn(case.Hkv, case.Dv, generator=gen) * case.channel_bias_std
         x = x + bias
-    g = F.logsigmoid(x).to(torch.float32).contiguous()
+    g = (x if case.raw_gate else F.logsigmoid(x)).to(torch.float32).contiguous()
     if case.w_kind == "ones":
         w = torch.ones(case.Dv, dtype=torch.bfloat16)
     else:
@@ -126,10 +127,10 @@ def draw(case: Case) -> dict:
 
 
 def make_case(B, T, Hq, Hkv, Dk, Dv, *, g_mean=3.0, g_std=1.0, w_kind="normal",
-              backward=True, seqlens=None, channel_bias_std=0.0, eps=1e-6,
+              backward=True, seqlens=None, channel_bias_std=0.0, raw_gate=False, eps=1e-6,
               seed=0) -> dict:
     """Convenience wrapper: build a ``Case`` and draw it."""
     c = Case(B, T, Hq, Hkv, Dk, Dv, g_mean, g_std, w_kind, backward,
              tuple(seqlens) if seqlens is not None else None, None,
-             channel_bias_std, eps, seed)
+             channel_bias_std, raw_gate, eps, seed)
     return draw(c)

@@ -1,0 +1,91 @@
+"""Helpers for the GPU parity tests: run the CUDA path, sample the oracle."""
+from __future__ import annotations
+
+import os
+
+import numpy as np
+import torch
+
+from oracle import fix_ref
+
+# Parity bars (rel-L2 = ||x - ref|| / ||ref|| over a tensor).  Forward on the
+# float32 output y after the RMSNorm; gradients per tensor.
+FWD_REL_L2 = 5e-3
+FWD_MAX_ABS = 2e-2
+GRAD_REL_L2 = 1e-2
+
+
+def workers():
+    try:
+        return max(1, len(os.sched_getaffinity(0)))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def rel_l2(x, ref):
+    x = np.asarray(x, np.float64).ravel()
+    ref = np.asarray(ref, np.float64).ravel()
+    return float(np.linalg.norm(x - ref) / max(np.linalg.norm(ref), 1e-300))
+
+
+def max_abs(x, ref):
+    return float(np.max(np.abs(np.asarray(x, np.float64) - np.asarray(ref, np.float64))))
+
+
+def to_cuda(case):
+    out = {}
+    for key in ("q", "k", "v", "g", "w", "dy", "cu_seqlens"):
+        t = case.get(key)
+        out[key] = None if t is None else t.cuda().contiguous()
+    return out
+
+
+def run_gpu(case, algo="auto", backward=False, y_dtype=torch.float32):
+    """Forward (and backward) through the C ABI; returns numpy float64 dicts."""
+    from gated_softmax_attention_fp32_b200 import fixattn
+    t = to_cuda(case)
+    cu_host = case["cu_seqlens"]
+    y, saved = fixattn.fix_attn_fwd(t["q"], t["k"], t["v"], t["g"], t["w"], t["cu_seqlens"],
+                                    cu_host, None, case["eps"], y_dtype=y_dtype, save=True,
+                                    algo=algo)
+    res = dict(y=y, o=saved[0], m=saved[1], rstd=saved[2])
+    if backward:
+        dq, dk, dv, dg, dw = fixattn.fix_attn_bwd(t["q"], t["k"], t["v"], t["g"], t["w"], t["dy"],
+                                                  saved, t["cu_seqlens"], cu_host, None,
+                                                  case["eps"], algo=algo)
+        res.update(dq=dq, dk=dk, dv=dv, dg=dg, dw=dw)
+    torch.cuda.synchronize()
+    return {k: v.float().cpu().numpy().astype(np.float64) for k, v in res.items()}
+
+
+def oracle_full(case, backward=False):
+    args = (case["q"], case["k"], case["v"], case["g"], case["w"])
+    seqlens = case["seqlens"] if case["cu_seqlens"] is not None else None
+    f = fix_ref.forward(*args, seqlens, None, case["eps"], workers())
+    if backward:
+        f.update(fix_ref.backward(*args, case["dy"], seqlens, None, case["eps"], workers()))
+    return f
+
+
+def segments(case):
+    """(batch index, start token, length) of every sequence."""
+    if case["cu_seqlens"] is None:
+        return [(b, 0, case["T"]) for b in range(case["B"])]
+    out, s0 = [], 0
+    for L in case["seqlens"]:
+        out.append((0, s0, L))
+        s0 += L
+    return out
+
+
+def sample_rows(L, n, rng):
+    """Rows of a length-L sequence: first, last 8, tile edges and random."""
+    if L == 0:
+        return []
+    rows = {0, L - 1}
+    rows.update(range(max(0, L - 8), L))
+    for e in (127, 128, 129, 255, 256):
+        if e < L:
+            rows.add(e)
+    rows.update(int(x) for x in rng.integers(0, L, size=n))
+    return sorted(rows)

@@ -1,0 +1,153 @@
+"""Host-side checks of the C ABI (no GPU needed, no kernel is launched).
+
+The library must load, export every function that include/fix_attn.h
+declares, size its workspace, and reject bad arguments on the host with the
+documented status codes before touching the device.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from gated_softmax_attention_fp32_b200 import fixattn
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fix_attn.h")
+
+FIX_OK, FIX_ERR_NULL, FIX_ERR_SHAPE, FIX_ERR_HEAD_DIM, FIX_ERR_GQA = 0, 1, 2, 3, 4
+FIX_ERR_CU_SEQLENS, FIX_ERR_ALIGN, FIX_ERR_WORKSPACE, FIX_ERR_DTYPE = 5, 6, 7, 8
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fix_attn_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from gated_softmax_attention_fp32_b200 import build
+    if not os.path.exists(fixattn.LIB_PATH):
+        build.build()
+    return fixattn.load()
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert set(names) >= {"fix_attn_fwd", "fix_attn_bwd", "fix_attn_workspace_bytes",
+                          "fix_attn_device_status", "fix_attn_status_string"}
+    raw = ctypes.CDLL(fixattn.LIB_PATH)
+    for n in names:
+        assert hasattr(raw, n), n
+    assert set(names) == set(fixattn.EXPORTS) | (set(names) - set(fixattn.EXPORTS))
+
+
+def prob(B=2, T=100, Hq=4, Hkv=2, Dk=64, Dv=64, **kw):
+    p = fixattn.Problem()
+    p.batch, p.seqlen, p.num_q_heads, p.num_kv_heads = B, T, Hq, Hkv
+    p.head_dim_k, p.head_dim_v = Dk, Dv
+    p.num_seqs = 0
+    p.y_dtype = 0
+    p.algo = 0
+    p.reserved = 0
+    p.scale = 0.0
+    p.eps = 1e-6
+    for key, val in kw.items():
+        setattr(p, key, val)
+    return p
+
+
+def test_workspace_sizes(lib):
+    ws_f = lib.fix_attn_workspace_bytes(ctypes.byref(prob()), 0)
+    ws_b = lib.fix_attn_workspace_bytes(ctypes.byref(prob()), 1)
+    assert 0 < ws_f < ws_b
+    # L (f32) + pre-decayed v (bf16) dominate the forward workspace
+    assert ws_f >= 2 * 100 * 2 * 64 * 6
+    assert lib.fix_attn_workspace_bytes(ctypes.byref(prob(Dk=48)), 0) == 0
+    assert lib.fix_attn_workspace_bytes(None, 0) == 0
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(Dk=48), FIX_ERR_HEAD_DIM),
+    (dict(Dv=256), FIX_ERR_HEAD_DIM),
+    (dict(Hq=6, Hkv=4), FIX_ERR_GQA),
+    (dict(B=0), FIX_ERR_SHAPE),
+    (dict(T=-1), FIX_ERR_SHAPE),
+    (dict(y_dtype=7), FIX_ERR_DTYPE),
+    (dict(algo=9), FIX_ERR_DTYPE),
+    (dict(reserved=1), FIX_ERR_SHAPE),
+    (dict(eps=-1.0), FIX_ERR_SHAPE),
+    (dict(num_seqs=2), FIX_ERR_CU_SEQLENS),
+])
+def test_bad_problem_rejected_on_host(lib, kw, code):
+    p = prob(**kw)
+    buf = (ctypes.c_uint8 * 4096)()
+    a = ctypes.addressof(buf)
+    a = (a + 15) // 16 * 16
+    ptrs = [ctypes.c_void_p(a)] * 10
+    s = lib.fix_attn_fwd(ctypes.byref(p), *ptrs, 1 << 40, None)
+    assert s == code, fixattn.status_string(s)
+    ptrs = [ctypes.c_void_p(a)] * 15
+    s = lib.fix_attn_bwd(ctypes.byref(p), *ptrs, 1 << 40, None)
+    assert s == code, fixattn.status_string(s)
+
+
+def _cu_problem(cu):
+    host = torch.tensor(cu, dtype=torch.int64)
+    p = prob(B=1, T=int(cu[-1]) if cu else 0, num_seqs=len(cu) - 1)
+    p.cu_seqlens = host.data_ptr()          # any non-NULL pointer: never dereferenced here
+    p.cu_seqlens_host = host.data_ptr()
+    return p, host
+
+
+@pytest.mark.parametrize("cu,code", [
+    ([1, 5, 10], FIX_ERR_CU_SEQLENS),
+    ([0, 5, 3, 10], FIX_ERR_CU_SEQLENS),
+])
+def test_bad_cu_seqlens_rejected(lib, cu, code):
+    p, host = _cu_problem(cu)
+    p.seqlen = 10
+    assert lib.fix_attn_workspace_bytes(ctypes.byref(p), 0) == 0
+    buf = (ctypes.c_uint8 * 64)()
+    a = (ctypes.addressof(buf) + 15) // 16 * 16
+    s = lib.fix_attn_fwd(ctypes.byref(p), *[ctypes.c_void_p(a)] * 10, 1 << 40, None)
+    assert s == code
+
+
+def test_varlen_requires_batch_one_and_host_mirror(lib):
+    p, host = _cu_problem([0, 4, 10])
+    p.batch = 2
+    p.seqlen = 5
+    assert lib.fix_attn_workspace_bytes(ctypes.byref(p), 0) == 0
+    p, host = _cu_problem([0, 4, 10])
+    p.cu_seqlens_host = None
+    assert lib.fix_attn_workspace_bytes(ctypes.byref(p), 0) == 0
+    p, host = _cu_problem([0, 0, 4, 4, 10])       # empty sequences are legal
+    assert lib.fix_attn_workspace_bytes(ctypes.byref(p), 1) > 0
+
+
+def test_null_misaligned_and_small_workspace(lib):
+    p = prob()
+    need = lib.fix_attn_workspace_bytes(ctypes.byref(p), 0)
+    buf = (ctypes.c_uint8 * 4096)()
+    a = (ctypes.addressof(buf) + 15) // 16 * 16
+    good = [ctypes.c_void_p(a)] * 10
+    s = lib.fix_attn_fwd(ctypes.byref(p), *([None] + good[1:]), need, None)
+    assert s == FIX_ERR_NULL
+    bad = list(good)
+    bad[2] = ctypes.c_void_p(a + 2)
+    assert lib.fix_attn_fwd(ctypes.byref(p), *bad, need, None) == FIX_ERR_ALIGN
+    assert lib.fix_attn_fwd(ctypes.byref(p), *good, need - 1, None) == FIX_ERR_WORKSPACE
+    # saved tensors: all three or none
+    part = list(good)
+    part[7] = None
+    assert lib.fix_attn_fwd(ctypes.byref(p), *part, need, None) == FIX_ERR_NULL
+
+
+def test_status_strings(lib):
+    for c in range(12):
+        s = fixattn.status_string(c)
+        assert s.startswith("FIX_")
+    assert "unknown" in fixattn.status_string(99)
