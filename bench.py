@@ -267,6 +267,8 @@ def main():
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * nst)] for _ in range(args.steps)]
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    for e in [x for row in ev for x in row]:     # torch creates the CUDA event lazily
+        e.record(stream)
     if world > 1:
         import torch.distributed as dist
         dist.barrier()

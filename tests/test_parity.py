@@ -29,12 +29,16 @@ def check_fwd(y, ref, tag=""):
 
 
 def check_grad(name, x, ref, tag=""):
-    x = np.asarray(x); ref = np.asarray(ref)
-    nref = np.linalg.norm(ref.ravel())
-    if nref < 1e-9:                       # e.g. dg of length-1 sequences: exactly 0
-        assert np.linalg.norm(x.ravel()) < 1e-5, f"{tag} {name} should vanish"
-        return
-    e = rel_l2(x, ref)
+    """rel-L2 <= 1e-2, measured against max(||ref||, 1e-4 * sqrt(numel)).
+
+    The floor (1e-4 RMS per element, far below the O(0.01..1) size of these
+    gradients) only matters where a gradient vanishes analytically up to
+    eps-sized terms: e.g. dq of a sequence's first row, whose only key has
+    weight exactly 1, so dq there is proportional to the RMSNorm eps and both
+    sides hold rounding noise of the cancelling terms."""
+    x = np.asarray(x, np.float64); ref = np.asarray(ref, np.float64)
+    den = max(np.linalg.norm(ref.ravel()), 1e-4 * np.sqrt(ref.size))
+    e = np.linalg.norm((x - ref).ravel()) / den
     assert e <= GRAD_REL_L2, f"{tag} {name} rel-L2 {e:.2e}"
 
 
@@ -200,18 +204,13 @@ def test_workload4_long_context_sampled(cuda_lib):
     check_fwd(y, ref, "workload 4")
 
 
-def test_workload5_sampled(cuda_lib):
+def test_workload5_full(cuda_lib):
+    # 128 (sequence, head) units of T = 4096: the full oracle takes about a
+    # minute on 16 host cores, so every gradient is compared element-wise
     case = synth.draw(synth.workload(5))
     gpu = run_gpu(case, backward=True)
     _properties(case, gpu)
-    y, ref = _sampled_forward(case, gpu, 6, range(0, case["Hq"], 2))
-    check_fwd(y, ref, "workload 5")
-    x, ref = _sampled_dq(case, gpu, 3, range(0, case["Hq"], 5))
-    check_grad("dq", x, ref, "workload 5")
-    picks = [(b, 0, case["T"], kv) for b in (0, 7) for kv in (0, 9)]
-    for key, (x, ref) in _suffix(case, gpu, picks, 32).items():
-        check_grad(key, x, ref, "workload 5")
-    # dw needs every row: compare with the oracle's sum over all rows of its
-    # own forward is too slow here; check it against y and dy instead
-    dw_rows = (case["dy"].double().numpy() * gpu["o"] * gpu["rstd"][..., None]).sum((0, 1, 2))
-    check_grad("dw", gpu["dw"], dw_rows, "workload 5")
+    ref = oracle_full(case, backward=True)
+    check_fwd(gpu["y"], ref["y"], "workload 5")
+    for key in GRADS:
+        check_grad(key, gpu[key], ref[key], "workload 5")
