@@ -24,7 +24,8 @@ __all__ = ["load", "Problem", "fix_attn_fwd", "fix_attn_bwd", "fix_attn_workspac
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfixattn.so")
 EXPORTS = ("fix_attn_workspace_bytes", "fix_attn_fwd", "fix_attn_bwd", "fix_attn_device_status",
-           "fix_attn_kernel_count", "fix_attn_status_string")
+           "fix_attn_kernel_count", "fix_attn_status_string", "fix_attn_fwd_noalloc")
+NOALLOC_MAX_WORKSPACE_BYTES = 16 * 1024 * 1024
 STAGES = ("fwd_prefix", "fwd_attn", "bwd_prefix", "bwd_pre", "bwd_dq", "bwd_dkv", "bwd_dg")
 
 ALGOS = {"auto": 0, "simt": 1, "tc": 2}
@@ -65,6 +66,8 @@ def load():
     lib.fix_attn_fwd.restype = ctypes.c_int
     lib.fix_attn_bwd.argtypes = [P] + [vp] * 15 + [sz, vp]
     lib.fix_attn_bwd.restype = ctypes.c_int
+    lib.fix_attn_fwd_noalloc.argtypes = [P] + [vp] * 9 + [vp]
+    lib.fix_attn_fwd_noalloc.restype = ctypes.c_int
     lib.fix_attn_device_status.argtypes = [vp, vp]
     lib.fix_attn_device_status.restype = ctypes.c_int
     lib.fix_attn_kernel_count.argtypes = [P, ctypes.c_int]
@@ -155,6 +158,22 @@ def fix_attn_fwd(q, k, v, g, o_norm_weight, cu_seqlens=None, cu_seqlens_host=Non
                          _ptr(workspace), workspace.numel(), _stream(stream))
     if s != 0:
         raise FixStatusError(s, "fix_attn_fwd")
+    del keep
+    return y, saved
+
+
+def fix_attn_fwd_noalloc(q, k, v, g, o_norm_weight, y, saved, cu_seqlens=None,
+                         cu_seqlens_host=None, scale=None, eps=1e-6, algo="auto", stream=None):
+    """Forward into caller-provided ``y`` and ``saved`` = (o, m, rstd) or None,
+    with the library's own fixed device workspace (no allocation by anyone)."""
+    lib = load()
+    p, keep = make_problem(q, k, v, cu_seqlens, cu_seqlens_host, scale, eps, y.dtype, algo)
+    s = lib.fix_attn_fwd_noalloc(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
+                                 _ptr(o_norm_weight), _ptr(y),
+                                 *(map(_ptr, saved) if saved else (None, None, None)),
+                                 _stream(stream))
+    if s != 0:
+        raise FixStatusError(s, "fix_attn_fwd_noalloc")
     del keep
     return y, saved
 

@@ -141,6 +141,34 @@ fix_status fix_attn_bwd(const fix_attn_problem *p, const void *q, const void *k,
  * fix_attn_fwd / fix_attn_bwd call. */
 fix_status fix_attn_device_status(const void *workspace, void *stream);
 
+/* Largest workspace fix_attn_fwd_noalloc can provide (16 MiB; enough for the
+ * forward of e.g. 4096 tokens x 4 kv heads x Dv 128). */
+#define FIX_NOALLOC_MAX_WORKSPACE_BYTES (16u * 1024u * 1024u)
+
+/* Forward for callers that cannot allocate device memory.  (The FiX pages
+ * have no counterpart to this entry point; it only changes where the
+ * workspace lives.)
+ *
+ * Some callers cannot obtain a device workspace when they call: host code
+ * handed only tensors and a stream, or a runtime whose device memory is
+ * reserved up front, where an allocation would fail or synchronise.  This
+ * call runs exactly fix_attn_fwd, with the same arguments except the
+ * workspace, which it takes from one library-owned device array of
+ * FIX_NOALLOC_MAX_WORKSPACE_BYTES that every GPU loading the library holds
+ * until the process exits.  It calls no allocator.
+ *   - Returns FIX_ERR_WORKSPACE if fix_attn_workspace_bytes(p, 0) exceeds
+ *     FIX_NOALLOC_MAX_WORKSPACE_BYTES, and fix_attn_fwd's codes otherwise.
+ *   - The first call on a device, with that device current, looks up the
+ *     array's device address (cudaGetSymbolAddress) and caches it; make that
+ *     first call before any stream capture.
+ *   - All calls on a device share the array, which keeps the last call's
+ *     contents; calls that overlap on the GPU (other streams or unordered
+ *     host threads) race on it.  Order them on one stream. */
+fix_status fix_attn_fwd_noalloc(const fix_attn_problem *p, const void *q, const void *k,
+                                const void *v, const float *g, const void *o_norm_weight,
+                                void *y, float *o_saved, float *m_saved, float *rstd_saved,
+                                void *stream);
+
 /* Number of kernels that fix_attn_fwd (backward = 0) or fix_attn_bwd
  * (backward = 1) launches for this problem (0 if it is invalid). */
 int fix_attn_kernel_count(const fix_attn_problem *p, int backward);
