@@ -64,6 +64,17 @@ static fix_status make_dims(const fix_attn_problem* p, Dims* d) {
   return FIX_OK;
 }
 
+// Largest number of chunks of one sequence (bound for the order histogram).
+static int max_chunks_per_seq(const fix_attn_problem* p) {
+  if (!p->cu_seqlens) return (p->seqlen + FIX_CHUNK - 1) / FIX_CHUNK;
+  long long m = 0;
+  for (int i = 0; i < p->num_seqs; ++i) {
+    const long long n = (p->cu_seqlens_host[i + 1] - p->cu_seqlens_host[i] + FIX_CHUNK - 1) / FIX_CHUNK;
+    if (n > m) m = n;
+  }
+  return (int)m;
+}
+
 static int dw_grid(const Dims& d) {
   int g = (d.N + 3) / 4;
   if (g > 128) g = 128;
@@ -73,8 +84,8 @@ static int dw_grid(const Dims& d) {
 
 // Workspace layout (all offsets 256-byte aligned).
 struct Ws {
-  size_t status, chunks, L, vt, tot;          // forward and backward
-  size_t dow, A, dG, dtot, dwp;               // backward only
+  size_t status, chunks, order, safe, L, vt, vm, vml, tot, rho, hr;   // forward and backward
+  size_t dow, A, dG, dtot, dwp;                            // backward only
   size_t total;
 };
 
@@ -90,9 +101,15 @@ static Ws layout(const Dims& d, bool bwd) {
   const size_t nch = (size_t)d.nchunks * d.Hkv * d.Dv;
   w.status = take(256);
   w.chunks = take((size_t)(d.nchunks > 0 ? d.nchunks : 1) * sizeof(Chunk));
+  w.order = take((size_t)(d.nchunks > 0 ? d.nchunks : 1) * sizeof(int));
+  w.safe = take((size_t)(d.nchunks > 0 ? d.nchunks : 1) * d.Hkv * sizeof(int));
   w.L = take(nkv * 4);
   w.vt = take(nkv * 2);
+  w.vm = take(nkv * 2);
+  w.vml = take(nkv * 2);
   w.tot = take(nch * 4);
+  w.rho = take(nch * 4);
+  w.hr = take(nch * 4);
   if (bwd) {
     w.dow = take((size_t)d.N * d.Hq * d.Dv * 4);
     w.A = take(nkv * 4);
@@ -149,10 +166,18 @@ static fix_status run_prefix(const Dims& d, const fix_attn_problem* p, const Ws&
   schedule_kernel<<<1, 1024, 0, st>>>(p->cu_seqlens, d.nseq, d.T, d.N, d.nchunks, chunks);
   FIX_TRY(launched());
   if (d.nchunks == 0) return FIX_OK;
+  if (want_vt) {
+    order_kernel<<<1, 1024, 0, st>>>(chunks, d.nchunks, max_chunks_per_seq(p),
+                                     reinterpret_cast<int*>(base + ws.order));
+    FIX_TRY(launched());
+  }
   prefix_kernel<<<dim3(d.nchunks, d.Hkv), 128, 0, st>>>(
       d, chunks, g, static_cast<const __nv_bfloat16*>(v), reinterpret_cast<float*>(base + ws.L),
-      want_vt ? reinterpret_cast<__nv_bfloat16*>(base + ws.vt) : nullptr,
-      reinterpret_cast<float*>(base + ws.tot));
+      want_vt ? reinterpret_cast<uint16_t*>(base + ws.vt) : nullptr,
+      reinterpret_cast<__nv_bfloat16*>(base + ws.vm),
+      reinterpret_cast<__nv_bfloat16*>(base + ws.vml), reinterpret_cast<float*>(base + ws.tot),
+      reinterpret_cast<float*>(base + ws.rho), reinterpret_cast<float*>(base + ws.hr),
+      reinterpret_cast<int*>(base + ws.safe));
   return launched();
 }
 
@@ -213,9 +238,14 @@ fix_status fix_attn_fwd(const fix_attn_problem* p, const void* q, const void* k,
   const float* tot = reinterpret_cast<const float*>(base + ws.tot);
   FIX_TRY(mark(p, FIX_STAGE_FWD_ATTN, 0, st));
   if (tc) {
-    FIX_TRY(tc_fwd(d, chunks, q, k, reinterpret_cast<const __nv_bfloat16*>(base + ws.vt), v, L,
-                   tot, w, y, p->y_dtype == FIX_DTYPE_F32, o_s, m_s, rstd_s,
-                   reinterpret_cast<int*>(base + ws.status), st));
+    FIX_TRY(tc_fwd(d, chunks, reinterpret_cast<const int*>(base + ws.order), q, k,
+                   reinterpret_cast<const uint16_t*>(base + ws.vt),
+                   reinterpret_cast<const __nv_bfloat16*>(base + ws.vm),
+                   reinterpret_cast<const __nv_bfloat16*>(base + ws.vml), v, L, tot,
+                   reinterpret_cast<const float*>(base + ws.rho),
+                   reinterpret_cast<const float*>(base + ws.hr),
+                   reinterpret_cast<const int*>(base + ws.safe), w, y, p->y_dtype == FIX_DTYPE_F32,
+                   o_s, m_s, rstd_s, reinterpret_cast<int*>(base + ws.status), st));
   } else {
     const size_t smem = simt_fwd_smem(d);
     if (cudaFuncSetAttribute(fwd_simt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -275,7 +305,7 @@ fix_status fix_attn_bwd(const fix_attn_problem* p, const void* q, const void* k,
   FIX_TRY(launched());
   FIX_TRY(mark(p, FIX_STAGE_BWD_PRE, 1, st));
   if (tc) {
-    FIX_TRY(tc_bwd(p, d, chunks, q, k, v, reinterpret_cast<const __nv_bfloat16*>(base + ws.vt), L,
+    FIX_TRY(tc_bwd(p, d, chunks, q, k, v, reinterpret_cast<const uint16_t*>(base + ws.vt), L,
                    tot, m_s, dow, A, dq, dk, dv, dG, reinterpret_cast<int*>(base + ws.status), st));
   } else {
     const size_t smq = simt_dq_smem(d), smkv = simt_dkv_smem(d);
@@ -312,10 +342,10 @@ int fix_attn_kernel_count(const fix_attn_problem* p, int backward) {
   if (d.N == 0) return 0;
   if (!backward) {
     const bool tc = p->algo != FIX_ALGO_SIMT && tc_fwd_supported(d);
-    return 2 + (tc ? tc_fwd_kernel_count(d) : 1);
+    return 2 + (tc ? 1 + tc_fwd_kernel_count(d) : 1);
   }
   const bool tc = p->algo != FIX_ALGO_SIMT && tc_bwd_supported(d);
-  return 2 + 2 + (tc ? tc_bwd_kernel_count(d) : 2) + 2;
+  return 2 + (tc ? 1 : 0) + 2 + (tc ? tc_bwd_kernel_count(d) : 2) + 2;
 }
 
 fix_status fix_attn_device_status(const void* workspace, void* stream) {

@@ -11,9 +11,16 @@
 #pragma once
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 #define FIX_CHUNK 128
+// Largest half-range of a chunk's prefix sums that the in-chunk split
+// exp(L_t - rho) * exp(rho - L_s) keeps inside float range (e^80 ~ 5.5e34).
+#define FIX_HR_MAX 80.0f
+// Largest |v| for which the fp16 operand path is used (fp16 max is 65504;
+// every scaled value on that path is <= |v| when g <= 0).
+#define FIX_F16_VMAX 30000.0f
 
 namespace fix {
 

@@ -10,7 +10,9 @@ constexpr int ST_ROWS = 32;  // rows per CTA of the exact (SIMT) kernels
 // fix_prefix.cu
 __global__ void schedule_kernel(const int64_t* cu, int nseq, int T, int N, int cap, Chunk* out);
 __global__ void prefix_kernel(Dims d, const Chunk* chunks, const float* g, const __nv_bfloat16* v,
-                              float* L, __nv_bfloat16* vt, float* tot);
+                              float* L, uint16_t* vt, __nv_bfloat16* vm, __nv_bfloat16* vml,
+                              float* tot, float* rho, float* hr, int* safe);
+__global__ void order_kernel(const Chunk* chunks, int nchunks, int maxj, int* order);
 __global__ void chunk_total_kernel(Dims d, const Chunk* chunks, const float* x, float* tot);
 __global__ void reverse_cumsum_kernel(Dims d, const Chunk* chunks, const float* x,
                                       const float* tot, float* out);
@@ -35,15 +37,18 @@ __global__ void dkv_simt_kernel(Dims d, const Chunk* chunks, const __nv_bfloat16
 
 // Tensor-core (tcgen05) kernels.
 bool tc_fwd_supported(const Dims& d);
-fix_status tc_fwd(const Dims& d, const Chunk* chunks, const void* q, const void* k,
-                  const __nv_bfloat16* vt, const void* v, const float* L, const float* tot,
+fix_status tc_fwd(const Dims& d, const Chunk* chunks, const int* order, const void* q,
+                  const void* k, const uint16_t* vt, const __nv_bfloat16* vm,
+                  const __nv_bfloat16* vml, const void* v,
+                  const float* L, const float* tot, const float* rho, const float* hr,
+                  const int* safe,
                   const void* w, void* y, bool y_f32, float* o_s, float* m_s, float* rstd_s,
                   int* status, cudaStream_t st);
 int tc_fwd_kernel_count(const Dims& d);
 bool tc_bwd_supported(const Dims& d);
 int tc_bwd_kernel_count(const Dims& d);
 fix_status tc_bwd(const fix_attn_problem* p, const Dims& d, const Chunk* chunks, const void* q, const void* k, const void* v,
-                  const __nv_bfloat16* vt, const float* L, const float* tot, const float* m_s,
+                  const uint16_t* vt, const float* L, const float* tot, const float* m_s,
                   const float* do_ws, const float* A, void* dq, void* dk, void* dv, float* dG,
                   int* status, cudaStream_t st);
 

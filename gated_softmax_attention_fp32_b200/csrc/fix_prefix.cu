@@ -67,40 +67,116 @@ __global__ void __launch_bounds__(1024) schedule_kernel(const int64_t* __restric
   }
 }
 
+// Single CTA: order[] lists chunk ids by decreasing chunk index j (the
+// number of key blocks before the diagonal), so that grids walking order[]
+// start the longest causal rows first.  maxj is an upper bound on j + 1; if
+// it exceeds the histogram, order[] is the identity.
+__global__ void __launch_bounds__(1024) order_kernel(const Chunk* __restrict__ chunks, int nchunks,
+                                                     int maxj, int* __restrict__ order) {
+  constexpr int kBins = 4096;
+  __shared__ int hist[kBins];
+  if (maxj > kBins) {
+    for (int i = threadIdx.x; i < nchunks; i += blockDim.x) order[i] = i;
+    return;
+  }
+  for (int b = threadIdx.x; b < maxj; b += blockDim.x) hist[b] = 0;
+  __syncthreads();
+  for (int i = threadIdx.x; i < nchunks; i += blockDim.x)
+    atomicAdd(&hist[min(max(chunks[i].j, 0), maxj - 1)], 1);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int acc = 0;
+    for (int b = maxj - 1; b >= 0; --b) {
+      const int c = hist[b];
+      hist[b] = acc;
+      acc += c;
+    }
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < nchunks; i += blockDim.x)
+    order[atomicAdd(&hist[min(max(chunks[i].j, 0), maxj - 1)], 1)] = i;
+}
+
 // grid (nchunks, Hkv), block 128: thread = channel.
+//
+// Besides L and tot, the tensor-core path needs:
+//   Vt_s[c] = v_s[c] * exp(tot[c] - L_s[c])     values pre-decayed to the chunk's
+//             last row, for key blocks strictly before a query chunk.  Stored
+//             as fp16 when the chunk is "fp16-safe" (every g <= 0 and every
+//             |v| <= FIX_F16_VMAX, so that all later scalings stay <= |v|),
+//             else as bf16; safe[ci * Hkv + kv] records which.
+//   rho[c] = (min_t L_t[c] + max_t L_t[c]) / 2,  hr[c] = (max - min) / 2,
+//   Vm_s[c] = v_s[c] * exp(rho[c] - L_s[c])       (|exponent| <= hr), stored as
+//             a pair of bf16 (hi, lo = bf16(Vm - hi)) for a near-exact
+//             diagonal block,
+// so that exp(G_t - G_s) = exp(L_t - rho) * exp(rho - L_s) with both factors
+// inside [e^-hr, e^hr].  Channels with hr > FIX_HR_MAX cannot be split this
+// way in float range; for them Vm = 0 and rho = 0, and the kernels handle the
+// diagonal block of that channel exactly in fp32.
 __global__ void __launch_bounds__(128) prefix_kernel(Dims d, const Chunk* __restrict__ chunks,
                                                      const float* __restrict__ g,
                                                      const __nv_bfloat16* __restrict__ v,
                                                      float* __restrict__ L,
-                                                     __nv_bfloat16* __restrict__ vt,
-                                                     float* __restrict__ tot) {
+                                                     uint16_t* __restrict__ vt,
+                                                     __nv_bfloat16* __restrict__ vm,
+                                                     __nv_bfloat16* __restrict__ vml,
+                                                     float* __restrict__ tot,
+                                                     float* __restrict__ rho,
+                                                     float* __restrict__ hr,
+                                                     int* __restrict__ safe) {
   const int ci = blockIdx.x, kv = blockIdx.y, c = threadIdx.x;
-  if (c >= d.Dv) return;
+  const bool active = c < d.Dv;
   const Chunk ch = chunks[ci];
   const size_t rs = (size_t)d.Hkv * d.Dv;
-  const size_t base = (size_t)ch.tok0 * rs + (size_t)kv * d.Dv + c;
-  float acc = 0.f;
+  const size_t base = (size_t)ch.tok0 * rs + (size_t)kv * d.Dv + (active ? c : 0);
+  const int len = active ? ch.len : 0;
+  float acc = 0.f, lmin = INFINITY, lmax = -INFINITY;
+  bool nonpos = true;
   int r = 0;
-  for (; r + 8 <= ch.len; r += 8) {
+  for (; r + 8 <= len; r += 8) {
     float x[8];
 #pragma unroll
     for (int u = 0; u < 8; ++u) x[u] = g[base + (size_t)(r + u) * rs];
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
+      nonpos = nonpos && x[u] <= 0.f;
       acc += x[u];
+      lmin = fminf(lmin, acc);
+      lmax = fmaxf(lmax, acc);
       L[base + (size_t)(r + u) * rs] = acc;
     }
   }
-  for (; r < ch.len; ++r) {
-    acc += g[base + (size_t)r * rs];
+  for (; r < len; ++r) {
+    const float x = g[base + (size_t)r * rs];
+    nonpos = nonpos && x <= 0.f;
+    acc += x;
+    lmin = fminf(lmin, acc);
+    lmax = fmaxf(lmax, acc);
     L[base + (size_t)r * rs] = acc;
   }
-  tot[((size_t)ci * d.Hkv + kv) * d.Dv + c] = acc;
-  if (vt) {
-    for (r = 0; r < ch.len; ++r) {
-      const size_t a = base + (size_t)r * rs;
-      vt[a] = f2bf(bf2f(v[a]) * expf(acc - L[a]));
-    }
+  const size_t ti = ((size_t)ci * d.Hkv + kv) * d.Dv + c;
+  if (active) tot[ti] = acc;
+  if (!vt) return;  // uniform: the exact kernels need only L and tot
+  float vmax = 0.f;
+  for (r = 0; r < len; ++r) vmax = fmaxf(vmax, fabsf(bf2f(v[base + (size_t)r * rs])));
+  const int f16 = __syncthreads_and(nonpos && vmax <= FIX_F16_VMAX);
+  if (c == 0) safe[(size_t)ci * d.Hkv + kv] = f16;
+  if (!active) return;
+  const float half = 0.5f * (lmax - lmin);
+  const bool good = half <= FIX_HR_MAX;
+  const float ref = good ? 0.5f * (lmax + lmin) : 0.f;
+  rho[ti] = ref;
+  hr[ti] = len > 0 ? half : 0.f;
+  for (r = 0; r < len; ++r) {
+    const size_t a = base + (size_t)r * rs;
+    const float la = L[a];
+    const float va = bf2f(v[a]);
+    const float xt = va * expf(acc - la);
+    vt[a] = f16 ? __half_as_ushort(__float2half_rn(xt)) : __bfloat16_as_ushort(f2bf(xt));
+    const float xm = good ? va * expf(ref - la) : 0.f;
+    const __nv_bfloat16 xm_hi = f2bf(xm);
+    vm[a] = xm_hi;
+    vml[a] = f2bf(xm - bf2f(xm_hi));   // Vm = hi + lo to ~16 bits
   }
 }
 
