@@ -75,17 +75,10 @@ static int max_chunks_per_seq(const fix_attn_problem* p) {
   return (int)m;
 }
 
-static int dw_grid(const Dims& d) {
-  int g = (d.N + 3) / 4;
-  if (g > 128) g = 128;
-  if (g < 1) g = 1;
-  return g;
-}
-
 // Workspace layout (all offsets 256-byte aligned).
 struct Ws {
   size_t status, chunks, order, safe, L, vt, vm, vml, tot, rho, hr;   // forward and backward
-  size_t dow, A, dG, dtot, dwp;                            // backward only
+  size_t dow, dot, dom, dsafe, A, dG, dtot, dwp;           // backward only
   size_t total;
 };
 
@@ -112,10 +105,13 @@ static Ws layout(const Dims& d, bool bwd) {
   w.hr = take(nch * 4);
   if (bwd) {
     w.dow = take((size_t)d.N * d.Hq * d.Dv * 4);
+    w.dot = take((size_t)d.N * d.Hq * d.Dv * 4);
+    w.dom = take((size_t)d.N * d.Hq * d.Dv * 4);
+    w.dsafe = take((size_t)(d.nchunks > 0 ? d.nchunks : 1) * d.Hq * sizeof(int));
     w.A = take(nkv * 4);
     w.dG = take(nkv * 4);
     w.dtot = take(nch * 4);
-    w.dwp = take((size_t)dw_grid(d) * d.Hkv * d.Dv * 4);
+    w.dwp = take((size_t)(d.nchunks > 0 ? d.nchunks : 1) * d.Hkv * d.Dv * 4);
   }
   w.total = o;
   return w;
@@ -163,21 +159,18 @@ static size_t simt_dkv_smem(const Dims& d) {
 static fix_status run_prefix(const Dims& d, const fix_attn_problem* p, const Ws& ws, char* base,
                              const float* g, const void* v, bool want_vt, cudaStream_t st) {
   Chunk* chunks = reinterpret_cast<Chunk*>(base + ws.chunks);
-  schedule_kernel<<<1, 1024, 0, st>>>(p->cu_seqlens, d.nseq, d.T, d.N, d.nchunks, chunks);
+  schedule_kernel<<<1, 1024, 0, st>>>(p->cu_seqlens, d.nseq, d.T, d.N, d.nchunks, chunks,
+                                      max_chunks_per_seq(p),
+                                      want_vt ? reinterpret_cast<int*>(base + ws.order) : nullptr);
   FIX_TRY(launched());
   if (d.nchunks == 0) return FIX_OK;
-  if (want_vt) {
-    order_kernel<<<1, 1024, 0, st>>>(chunks, d.nchunks, max_chunks_per_seq(p),
-                                     reinterpret_cast<int*>(base + ws.order));
-    FIX_TRY(launched());
-  }
-  prefix_kernel<<<dim3(d.nchunks, d.Hkv), 128, 0, st>>>(
+  prefix_kernel<<<dim3(d.nchunks, d.Hkv), 512, 0, st>>>(
       d, chunks, g, static_cast<const __nv_bfloat16*>(v), reinterpret_cast<float*>(base + ws.L),
       want_vt ? reinterpret_cast<uint16_t*>(base + ws.vt) : nullptr,
       reinterpret_cast<__nv_bfloat16*>(base + ws.vm),
       reinterpret_cast<__nv_bfloat16*>(base + ws.vml), reinterpret_cast<float*>(base + ws.tot),
       reinterpret_cast<float*>(base + ws.rho), reinterpret_cast<float*>(base + ws.hr),
-      reinterpret_cast<int*>(base + ws.safe));
+      reinterpret_cast<int*>(base + ws.safe), reinterpret_cast<int*>(base + ws.status) + 1);
   return launched();
 }
 
@@ -227,7 +220,8 @@ fix_status fix_attn_fwd(const fix_attn_problem* p, const void* q, const void* k,
   FIX_TRY(check_device());
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* base = static_cast<char*>(workspace);
-  if (cudaMemsetAsync(base + ws.status, 0, 4, st) != cudaSuccess) return FIX_ERR_CUDA;
+  // status word and the out-of-range flag of the prefix pass start at zero
+  if (cudaMemsetAsync(base + ws.status, 0, 8, st) != cudaSuccess) return FIX_ERR_CUDA;
   if (d.N == 0) return FIX_OK;
   const bool tc = p->algo != FIX_ALGO_SIMT && tc_fwd_supported(d);
   FIX_TRY(mark(p, FIX_STAGE_FWD_PREFIX, 0, st));
@@ -278,7 +272,7 @@ fix_status fix_attn_bwd(const fix_attn_problem* p, const void* q, const void* k,
   FIX_TRY(check_device());
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* base = static_cast<char*>(workspace);
-  if (cudaMemsetAsync(base + ws.status, 0, 4, st) != cudaSuccess) return FIX_ERR_CUDA;
+  if (cudaMemsetAsync(base + ws.status, 0, 8, st) != cudaSuccess) return FIX_ERR_CUDA;
   if (d.N == 0) {
     if (cudaMemsetAsync(dw, 0, (size_t)d.Dv * 2, st) != cudaSuccess) return FIX_ERR_CUDA;
     return FIX_OK;
@@ -291,43 +285,76 @@ fix_status fix_attn_bwd(const fix_attn_problem* p, const void* q, const void* k,
   const float* L = reinterpret_cast<const float*>(base + ws.L);
   const float* tot = reinterpret_cast<const float*>(base + ws.tot);
   float* dow = reinterpret_cast<float*>(base + ws.dow);
+  float* dot = reinterpret_cast<float*>(base + ws.dot);
+  float* dom = reinterpret_cast<float*>(base + ws.dom);
+  int* dsafe = reinterpret_cast<int*>(base + ws.dsafe);
   float* A = reinterpret_cast<float*>(base + ws.A);
   float* dG = reinterpret_cast<float*>(base + ws.dG);
   float* dtot = reinterpret_cast<float*>(base + ws.dtot);
   float* dwp = reinterpret_cast<float*>(base + ws.dwp);
-  const int gx = dw_grid(d);
+  const int* badflag = reinterpret_cast<const int*>(base + ws.status) + 1;
+  const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(q);
+  const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(k);
+  const __nv_bfloat16* vb = static_cast<const __nv_bfloat16*>(v);
   FIX_TRY(mark(p, FIX_STAGE_BWD_PRE, 0, st));
-  bwd_pre_kernel<<<dim3(gx, d.Hkv), 128, 0, st>>>(d, o_s, rstd_s,
-                                                   static_cast<const __nv_bfloat16*>(dy),
-                                                   static_cast<const __nv_bfloat16*>(w), dow, A, dwp);
+  bwd_pre_kernel<<<dim3(d.nchunks, d.Hkv), 128, d.grp * sizeof(float), st>>>(
+      d, chunks, qb, kb, vb, o_s, m_s, rstd_s, static_cast<const __nv_bfloat16*>(dy),
+      static_cast<const __nv_bfloat16*>(w), L, reinterpret_cast<const float*>(base + ws.rho),
+      reinterpret_cast<const float*>(base + ws.hr), dow, tc ? dot : nullptr, tc ? dom : nullptr,
+      dsafe, A, dwp);
   FIX_TRY(launched());
-  dw_reduce_kernel<<<1, 128, 0, st>>>(dwp, gx * d.Hkv, d.Dv, static_cast<__nv_bfloat16*>(dw));
+  dw_reduce_kernel<<<1, 128, 0, st>>>(dwp, d.nchunks * d.Hkv, d.Dv, static_cast<__nv_bfloat16*>(dw));
   FIX_TRY(launched());
   FIX_TRY(mark(p, FIX_STAGE_BWD_PRE, 1, st));
+  TcBwdArgs ta{};
   if (tc) {
-    FIX_TRY(tc_bwd(p, d, chunks, q, k, v, reinterpret_cast<const uint16_t*>(base + ws.vt), L,
-                   tot, m_s, dow, A, dq, dk, dv, dG, reinterpret_cast<int*>(base + ws.status), st));
-  } else {
-    const size_t smq = simt_dq_smem(d), smkv = simt_dkv_smem(d);
-    if (cudaFuncSetAttribute(dq_simt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smq) != cudaSuccess ||
-        cudaFuncSetAttribute(dkv_simt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smkv) != cudaSuccess)
-      return FIX_ERR_CUDA;
-    FIX_TRY(mark(p, FIX_STAGE_BWD_DQ, 0, st));
-    dq_simt_kernel<<<dim3(d.nchunks * 4, d.Hq), 256, smq, st>>>(
-        d, chunks, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-        static_cast<const __nv_bfloat16*>(v), L, tot, m_s, dow, static_cast<__nv_bfloat16*>(dq));
-    FIX_TRY(launched());
-    FIX_TRY(mark(p, FIX_STAGE_BWD_DQ, 1, st));
-    FIX_TRY(mark(p, FIX_STAGE_BWD_DKV, 0, st));
-    dkv_simt_kernel<<<dim3(d.nchunks * 4, d.Hkv), 256, smkv, st>>>(
-        d, chunks, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-        static_cast<const __nv_bfloat16*>(v), L, tot, m_s, dow, A,
-        static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv), dG);
-    FIX_TRY(launched());
-    FIX_TRY(mark(p, FIX_STAGE_BWD_DKV, 1, st));
+    ta.chunks = chunks;
+    ta.order = reinterpret_cast<const int*>(base + ws.order);
+    ta.q = q;
+    ta.k = k;
+    ta.v = v;
+    ta.vt = reinterpret_cast<const uint16_t*>(base + ws.vt);
+    ta.vm = reinterpret_cast<const __nv_bfloat16*>(base + ws.vm);
+    ta.L = L;
+    ta.tot = tot;
+    ta.rho = reinterpret_cast<const float*>(base + ws.rho);
+    ta.hr = reinterpret_cast<const float*>(base + ws.hr);
+    ta.safe = reinterpret_cast<const int*>(base + ws.safe);
+    ta.dsafe = dsafe;
+    ta.m_s = m_s;
+    ta.do_ws = dow;
+    ta.dot_ws = dot;
+    ta.dom_ws = dom;
+    ta.A = A;
+    ta.badflag = badflag;
+    ta.dq = dq;
+    ta.dk = dk;
+    ta.dv = dv;
+    ta.dG = dG;
+    ta.status = reinterpret_cast<int*>(base + ws.status);
   }
+  // With the tensor-core kernels the exact kernels stay launched but return at
+  // once unless the prefix pass flagged a channel outside the split's range.
+  const int* gate = tc ? badflag : nullptr;
+  const size_t smq = simt_dq_smem(d), smkv = simt_dkv_smem(d);
+  if (cudaFuncSetAttribute(dq_simt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smq) != cudaSuccess ||
+      cudaFuncSetAttribute(dkv_simt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smkv) != cudaSuccess)
+    return FIX_ERR_CUDA;
+  FIX_TRY(mark(p, FIX_STAGE_BWD_DQ, 0, st));
+  if (tc) FIX_TRY(tc_bwd(p, d, ta, 0, st));
+  dq_simt_kernel<<<dim3(d.nchunks * 4, d.Hq), 256, smq, st>>>(
+      d, chunks, qb, kb, vb, L, tot, m_s, dow, static_cast<__nv_bfloat16*>(dq), gate);
+  FIX_TRY(launched());
+  FIX_TRY(mark(p, FIX_STAGE_BWD_DQ, 1, st));
+  FIX_TRY(mark(p, FIX_STAGE_BWD_DKV, 0, st));
+  if (tc) FIX_TRY(tc_bwd(p, d, ta, 1, st));
+  dkv_simt_kernel<<<dim3(d.nchunks * 4, d.Hkv), 256, smkv, st>>>(
+      d, chunks, qb, kb, vb, L, tot, m_s, dow, A, static_cast<__nv_bfloat16*>(dk),
+      static_cast<__nv_bfloat16*>(dv), dG, gate);
+  FIX_TRY(launched());
+  FIX_TRY(mark(p, FIX_STAGE_BWD_DKV, 1, st));
   FIX_TRY(mark(p, FIX_STAGE_BWD_DG, 0, st));
   chunk_total_kernel<<<dim3(d.nchunks, d.Hkv), 128, 0, st>>>(d, chunks, dG, dtot);
   FIX_TRY(launched());
@@ -342,10 +369,10 @@ int fix_attn_kernel_count(const fix_attn_problem* p, int backward) {
   if (d.N == 0) return 0;
   if (!backward) {
     const bool tc = p->algo != FIX_ALGO_SIMT && tc_fwd_supported(d);
-    return 2 + (tc ? 1 + tc_fwd_kernel_count(d) : 1);
+    return 2 + (tc ? tc_fwd_kernel_count(d) : 1);
   }
   const bool tc = p->algo != FIX_ALGO_SIMT && tc_bwd_supported(d);
-  return 2 + (tc ? 1 : 0) + 2 + (tc ? tc_bwd_kernel_count(d) : 2) + 2;
+  return 2 + 2 + (tc ? tc_bwd_kernel_count(d) : 0) + 2 + 2;
 }
 
 fix_status fix_attn_device_status(const void* workspace, void* stream) {

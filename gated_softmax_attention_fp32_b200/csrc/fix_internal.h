@@ -8,11 +8,11 @@ namespace fix {
 constexpr int ST_ROWS = 32;  // rows per CTA of the exact (SIMT) kernels
 
 // fix_prefix.cu
-__global__ void schedule_kernel(const int64_t* cu, int nseq, int T, int N, int cap, Chunk* out);
+__global__ void schedule_kernel(const int64_t* cu, int nseq, int T, int N, int cap, Chunk* out,
+                                int maxj, int* order);
 __global__ void prefix_kernel(Dims d, const Chunk* chunks, const float* g, const __nv_bfloat16* v,
                               float* L, uint16_t* vt, __nv_bfloat16* vm, __nv_bfloat16* vml,
-                              float* tot, float* rho, float* hr, int* safe);
-__global__ void order_kernel(const Chunk* chunks, int nchunks, int maxj, int* order);
+                              float* tot, float* rho, float* hr, int* safe, int* badflag);
 __global__ void chunk_total_kernel(Dims d, const Chunk* chunks, const float* x, float* tot);
 __global__ void reverse_cumsum_kernel(Dims d, const Chunk* chunks, const float* x,
                                       const float* tot, float* out);
@@ -22,18 +22,22 @@ __global__ void fwd_simt_kernel(Dims d, const Chunk* chunks, const __nv_bfloat16
                                 const __nv_bfloat16* k, const __nv_bfloat16* v, const float* L,
                                 const float* tot, const __nv_bfloat16* w, void* y, int y_f32,
                                 float* o_s, float* m_s, float* rstd_s);
-__global__ void bwd_pre_kernel(Dims d, const float* o_s, const float* rstd_s,
-                               const __nv_bfloat16* dy, const __nv_bfloat16* w, float* do_ws,
-                               float* A, float* dwpart);
+__global__ void bwd_pre_kernel(Dims d, const Chunk* chunks, const __nv_bfloat16* q,
+                               const __nv_bfloat16* k, const __nv_bfloat16* v, const float* o_s,
+                               const float* m_s, const float* rstd_s, const __nv_bfloat16* dy,
+                               const __nv_bfloat16* w, const float* L, const float* rho,
+                               const float* hr, float* do_ws, float* dot_ws, float* dom_ws,
+                               int* dsafe, float* A, float* dwpart);
 __global__ void dw_reduce_kernel(const float* parts, int nparts, int Dv, __nv_bfloat16* dw);
 __global__ void dq_simt_kernel(Dims d, const Chunk* chunks, const __nv_bfloat16* q,
                                const __nv_bfloat16* k, const __nv_bfloat16* v, const float* L,
                                const float* tot, const float* m_s, const float* do_ws,
-                               __nv_bfloat16* dq);
+                               __nv_bfloat16* dq, const int* gate);
 __global__ void dkv_simt_kernel(Dims d, const Chunk* chunks, const __nv_bfloat16* q,
                                 const __nv_bfloat16* k, const __nv_bfloat16* v, const float* L,
                                 const float* tot, const float* m_s, const float* do_ws,
-                                const float* A, __nv_bfloat16* dk, __nv_bfloat16* dv, float* dG);
+                                const float* A, __nv_bfloat16* dk, __nv_bfloat16* dv, float* dG,
+                                const int* gate);
 
 // Tensor-core (tcgen05) kernels.
 bool tc_fwd_supported(const Dims& d);
@@ -47,9 +51,36 @@ fix_status tc_fwd(const Dims& d, const Chunk* chunks, const int* order, const vo
 int tc_fwd_kernel_count(const Dims& d);
 bool tc_bwd_supported(const Dims& d);
 int tc_bwd_kernel_count(const Dims& d);
-fix_status tc_bwd(const fix_attn_problem* p, const Dims& d, const Chunk* chunks, const void* q, const void* k, const void* v,
-                  const uint16_t* vt, const float* L, const float* tot, const float* m_s,
-                  const float* do_ws, const float* A, void* dq, void* dk, void* dv, float* dG,
-                  int* status, cudaStream_t st);
+
+// Device buffers of one backward call for the tensor-core kernels.
+struct TcBwdArgs {
+  const Chunk* chunks;
+  const int* order;
+  const void* q;
+  const void* k;
+  const void* v;
+  const uint16_t* vt;
+  const __nv_bfloat16* vm;
+  const float* L;
+  const float* tot;
+  const float* rho;
+  const float* hr;
+  const int* safe;
+  const int* dsafe;
+  const float* m_s;
+  const float* do_ws;
+  const float* dot_ws;
+  const float* dom_ws;
+  const float* A;
+  const int* badflag;
+  void* dq;
+  void* dk;
+  void* dv;
+  float* dG;
+  int* status;
+};
+// which = 0: dq kernel, 1: dk/dv kernel
+fix_status tc_bwd(const fix_attn_problem* p, const Dims& d, const TcBwdArgs& a, int which,
+                  cudaStream_t st);
 
 }  // namespace fix

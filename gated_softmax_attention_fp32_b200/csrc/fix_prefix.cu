@@ -14,6 +14,36 @@
 
 namespace fix {
 
+// order[] lists chunk ids by decreasing chunk index j (the number of key
+// blocks before the diagonal), so that grids walking order[] start the
+// longest causal rows first.  maxj is an upper bound on j + 1; if it exceeds
+// the histogram, order[] is the identity.  Run by one whole CTA.
+__device__ void order_chunks(const Chunk* __restrict__ chunks, int nchunks, int maxj,
+                             int* __restrict__ order) {
+  constexpr int kBins = 4096;
+  __shared__ int hist[kBins];
+  if (maxj > kBins) {
+    for (int i = threadIdx.x; i < nchunks; i += blockDim.x) order[i] = i;
+    return;
+  }
+  for (int b = threadIdx.x; b < maxj; b += blockDim.x) hist[b] = 0;
+  __syncthreads();
+  for (int i = threadIdx.x; i < nchunks; i += blockDim.x)
+    atomicAdd(&hist[min(max(chunks[i].j, 0), maxj - 1)], 1);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int acc = 0;
+    for (int b = maxj - 1; b >= 0; --b) {
+      const int c = hist[b];
+      hist[b] = acc;
+      acc += c;
+    }
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < nchunks; i += blockDim.x)
+    order[atomicAdd(&hist[min(max(chunks[i].j, 0), maxj - 1)], 1)] = i;
+}
+
 // Single CTA: turns sequence lengths (device cu_seqlens, or B sequences of T
 // tokens when cu is NULL) into the chunk table, sequences in order.  The table
 // has `cap` entries (the count the host derived from its cu_seqlens mirror);
@@ -22,7 +52,8 @@ namespace fix {
 // mirror cannot send any kernel outside its buffers.
 __global__ void __launch_bounds__(1024) schedule_kernel(const int64_t* __restrict__ cu, int nseq,
                                                         int T, int N, int cap,
-                                                        Chunk* __restrict__ out) {
+                                                        Chunk* __restrict__ out, int maxj,
+                                                        int* __restrict__ order) {
   __shared__ int scan[1024];
   for (int i = threadIdx.x; i < cap; i += blockDim.x) out[i] = Chunk{0, 0, 0, 0};
   __syncthreads();
@@ -65,39 +96,16 @@ __global__ void __launch_bounds__(1024) schedule_kernel(const int64_t* __restric
     carry += scan[blockDim.x - 1];
     __syncthreads();
   }
+  if (order) {
+    __threadfence_block();
+    __syncthreads();
+    order_chunks(out, cap, maxj, order);
+  }
 }
 
-// Single CTA: order[] lists chunk ids by decreasing chunk index j (the
-// number of key blocks before the diagonal), so that grids walking order[]
-// start the longest causal rows first.  maxj is an upper bound on j + 1; if
-// it exceeds the histogram, order[] is the identity.
-__global__ void __launch_bounds__(1024) order_kernel(const Chunk* __restrict__ chunks, int nchunks,
-                                                     int maxj, int* __restrict__ order) {
-  constexpr int kBins = 4096;
-  __shared__ int hist[kBins];
-  if (maxj > kBins) {
-    for (int i = threadIdx.x; i < nchunks; i += blockDim.x) order[i] = i;
-    return;
-  }
-  for (int b = threadIdx.x; b < maxj; b += blockDim.x) hist[b] = 0;
-  __syncthreads();
-  for (int i = threadIdx.x; i < nchunks; i += blockDim.x)
-    atomicAdd(&hist[min(max(chunks[i].j, 0), maxj - 1)], 1);
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    int acc = 0;
-    for (int b = maxj - 1; b >= 0; --b) {
-      const int c = hist[b];
-      hist[b] = acc;
-      acc += c;
-    }
-  }
-  __syncthreads();
-  for (int i = threadIdx.x; i < nchunks; i += blockDim.x)
-    order[atomicAdd(&hist[min(max(chunks[i].j, 0), maxj - 1)], 1)] = i;
-}
-
-// grid (nchunks, Hkv), block 128: thread = channel.
+// grid (nchunks, Hkv), block 512: thread = (row group, channel); the chunk's
+// 128 rows are split into 512 / Dv groups scanned in parallel and joined
+// through shared memory.
 //
 // Besides L and tot, the tensor-core path needs:
 //   Vt_s[c] = v_s[c] * exp(tot[c] - L_s[c])     values pre-decayed to the chunk's
@@ -113,71 +121,92 @@ __global__ void __launch_bounds__(1024) order_kernel(const Chunk* __restrict__ c
 // inside [e^-hr, e^hr].  Channels with hr > FIX_HR_MAX cannot be split this
 // way in float range; for them Vm = 0 and rho = 0, and the kernels handle the
 // diagonal block of that channel exactly in fp32.
-__global__ void __launch_bounds__(128) prefix_kernel(Dims d, const Chunk* __restrict__ chunks,
-                                                     const float* __restrict__ g,
-                                                     const __nv_bfloat16* __restrict__ v,
-                                                     float* __restrict__ L,
-                                                     uint16_t* __restrict__ vt,
-                                                     __nv_bfloat16* __restrict__ vm,
-                                                     __nv_bfloat16* __restrict__ vml,
-                                                     float* __restrict__ tot,
-                                                     float* __restrict__ rho,
-                                                     float* __restrict__ hr,
-                                                     int* __restrict__ safe) {
-  const int ci = blockIdx.x, kv = blockIdx.y, c = threadIdx.x;
-  const bool active = c < d.Dv;
+constexpr int kPrefixThreads = 512;
+
+__global__ void __launch_bounds__(kPrefixThreads) prefix_kernel(
+    Dims d, const Chunk* __restrict__ chunks, const float* __restrict__ g,
+    const __nv_bfloat16* __restrict__ v, float* __restrict__ L, uint16_t* __restrict__ vt,
+    __nv_bfloat16* __restrict__ vm, __nv_bfloat16* __restrict__ vml, float* __restrict__ tot,
+    float* __restrict__ rho, float* __restrict__ hr, int* __restrict__ safe,
+    int* __restrict__ badflag) {
+  constexpr int kMaxRows = FIX_CHUNK * 128 / kPrefixThreads;  // rows per thread at Dv = 128
+  __shared__ float part[kPrefixThreads], pmin[kPrefixThreads], pmax[kPrefixThreads];
+  const int Dv = d.Dv;
+  const int groups = kPrefixThreads / Dv;
+  const int rows = FIX_CHUNK / groups;                       // rows per group
+  const int c = threadIdx.x % Dv, grp = threadIdx.x / Dv;
+  const int ci = blockIdx.x, kv = blockIdx.y;
   const Chunk ch = chunks[ci];
-  const size_t rs = (size_t)d.Hkv * d.Dv;
-  const size_t base = (size_t)ch.tok0 * rs + (size_t)kv * d.Dv + (active ? c : 0);
-  const int len = active ? ch.len : 0;
+  const size_t rs = (size_t)d.Hkv * Dv;
+  const size_t base = (size_t)ch.tok0 * rs + (size_t)kv * Dv + c;
+  const int r0 = grp * rows;
+  const int nr = max(0, min(rows, ch.len - r0));
+  float lv[kMaxRows];
   float acc = 0.f, lmin = INFINITY, lmax = -INFINITY;
   bool nonpos = true;
-  int r = 0;
-  for (; r + 8 <= len; r += 8) {
-    float x[8];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) x[u] = g[base + (size_t)(r + u) * rs];
+  for (int u = 0; u < kMaxRows; ++u)
+    if (u < nr) lv[u] = g[base + (size_t)(r0 + u) * rs];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      nonpos = nonpos && x[u] <= 0.f;
-      acc += x[u];
+  for (int u = 0; u < kMaxRows; ++u) {
+    if (u < nr) {
+      nonpos = nonpos && lv[u] <= 0.f;
+      acc += lv[u];
+      lv[u] = acc;
       lmin = fminf(lmin, acc);
       lmax = fmaxf(lmax, acc);
-      L[base + (size_t)(r + u) * rs] = acc;
     }
   }
-  for (; r < len; ++r) {
-    const float x = g[base + (size_t)r * rs];
-    nonpos = nonpos && x <= 0.f;
-    acc += x;
-    lmin = fminf(lmin, acc);
-    lmax = fmaxf(lmax, acc);
-    L[base + (size_t)r * rs] = acc;
+  part[threadIdx.x] = acc;
+  pmin[threadIdx.x] = lmin;
+  pmax[threadIdx.x] = lmax;
+  __syncthreads();
+  float off = 0.f, total = 0.f, cmin = INFINITY, cmax = -INFINITY;
+  for (int q = 0; q < groups; ++q) {
+    const float pq = part[q * Dv + c];
+    if (q < grp) off += pq;
+    cmin = fminf(cmin, total + pmin[q * Dv + c]);
+    cmax = fmaxf(cmax, total + pmax[q * Dv + c]);
+    total += pq;
   }
-  const size_t ti = ((size_t)ci * d.Hkv + kv) * d.Dv + c;
-  if (active) tot[ti] = acc;
+#pragma unroll
+  for (int u = 0; u < kMaxRows; ++u)
+    if (u < nr) {
+      lv[u] += off;
+      L[base + (size_t)(r0 + u) * rs] = lv[u];
+    }
+  const size_t ti = ((size_t)ci * d.Hkv + kv) * Dv + c;
+  if (grp == 0) tot[ti] = total;
   if (!vt) return;  // uniform: the exact kernels need only L and tot
   float vmax = 0.f;
-  for (r = 0; r < len; ++r) vmax = fmaxf(vmax, fabsf(bf2f(v[base + (size_t)r * rs])));
+  float vv[kMaxRows];
+#pragma unroll
+  for (int u = 0; u < kMaxRows; ++u)
+    if (u < nr) {
+      vv[u] = bf2f(v[base + (size_t)(r0 + u) * rs]);
+      vmax = fmaxf(vmax, fabsf(vv[u]));
+    }
   const int f16 = __syncthreads_and(nonpos && vmax <= FIX_F16_VMAX);
-  if (c == 0) safe[(size_t)ci * d.Hkv + kv] = f16;
-  if (!active) return;
-  const float half = 0.5f * (lmax - lmin);
+  if (threadIdx.x == 0) safe[(size_t)ci * d.Hkv + kv] = f16;
+  const float half = 0.5f * (cmax - cmin);
   const bool good = half <= FIX_HR_MAX;
-  const float ref = good ? 0.5f * (lmax + lmin) : 0.f;
-  rho[ti] = ref;
-  hr[ti] = len > 0 ? half : 0.f;
-  for (r = 0; r < len; ++r) {
-    const size_t a = base + (size_t)r * rs;
-    const float la = L[a];
-    const float va = bf2f(v[a]);
-    const float xt = va * expf(acc - la);
-    vt[a] = f16 ? __half_as_ushort(__float2half_rn(xt)) : __bfloat16_as_ushort(f2bf(xt));
-    const float xm = good ? va * expf(ref - la) : 0.f;
-    const __nv_bfloat16 xm_hi = f2bf(xm);
-    vm[a] = xm_hi;
-    vml[a] = f2bf(xm - bf2f(xm_hi));   // Vm = hi + lo to ~16 bits
+  const float ref = good ? 0.5f * (cmax + cmin) : 0.f;
+  if (__syncthreads_or(!good) && threadIdx.x == 0) atomicOr(badflag, 1);
+  if (grp == 0) {
+    rho[ti] = ref;
+    hr[ti] = ch.len > 0 ? half : 0.f;
   }
+#pragma unroll
+  for (int u = 0; u < kMaxRows; ++u)
+    if (u < nr) {
+      const size_t a = base + (size_t)(r0 + u) * rs;
+      const float xt = vv[u] * expf(total - lv[u]);
+      vt[a] = f16 ? __half_as_ushort(__float2half_rn(xt)) : __bfloat16_as_ushort(f2bf(xt));
+      const float xm = good ? vv[u] * expf(ref - lv[u]) : 0.f;
+      const __nv_bfloat16 xm_hi = f2bf(xm);
+      vm[a] = xm_hi;
+      vml[a] = f2bf(xm - bf2f(xm_hi));   // Vm = hi + lo to ~16 bits
+    }
 }
 
 // Reverse cumsum of dG within each sequence (dg_r = sum_{t >= r} dG_t), in two

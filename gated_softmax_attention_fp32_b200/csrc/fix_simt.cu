@@ -152,58 +152,108 @@ __global__ void __launch_bounds__(256) fwd_simt_kernel(
 }
 
 // ---------------------------------------------------------------------------
-// Backward preprocess (shared by all kernel families).  RMSNorm backward:
-//   n = o rstd, dn = dy w, do = rstd (dn - n mean(dn n)),
-// A_t[c] = sum_{h in group} do_t[c] o_t[c] (the per-row part of dG_t) and
-// per-CTA partial sums of dw = sum dy n.
-// grid (G, Hkv), block 128 (4 warps); a warp handles one token at a time.
+// Backward preprocess (shared by all kernel families), one CTA per (chunk, kv
+// head), 4 warps, a warp per row at a time over the kv group's q heads:
+//   RMSNorm backward   n = o rstd,  dn = dy w,  do = rstd (dn - n mean(dn n))
+//   A_t[c]  = sum_{h in group} do_t[c] (o_t[c] - P_tt v_t[c])
+//             the row part of dG_t without the s = t pair, whose counterpart
+//             the dk/dv kernels leave out of dv as well, so that
+//             dG = A - v dv_strict carries no cancelling diagonal terms
+//             (P_tt = exp(S_tt - m_t), S_tt recomputed from q_t, k_t)
+//   dw partials        sum_t dy_t n_t per CTA
+// and, for the tensor-core kernels (dot != NULL), the row-scaled upstream
+// gradients in the two references of the forward split:
+//   dOt_t = do_t exp(L_t)          (key blocks before the query chunk)
+//   dOm_t = do_t exp(L_t - rho)    (the diagonal block; 0 for channels outside
+//                                   the split's range)
+// plus dsafe[ci * Hq + h] = (max |do| over the chunk <= FIX_F16_VMAX).
+// Dynamic shared memory: grp floats.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(128) bwd_pre_kernel(
-    Dims d, const float* __restrict__ o_s, const float* __restrict__ rstd_s,
-    const __nv_bfloat16* __restrict__ dy, const __nv_bfloat16* __restrict__ w,
-    float* __restrict__ do_ws, float* __restrict__ A, float* __restrict__ dwpart) {
+    Dims d, const Chunk* __restrict__ chunks, const __nv_bfloat16* __restrict__ q,
+    const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
+    const float* __restrict__ o_s, const float* __restrict__ m_s,
+    const float* __restrict__ rstd_s, const __nv_bfloat16* __restrict__ dy,
+    const __nv_bfloat16* __restrict__ w, const float* __restrict__ L,
+    const float* __restrict__ rho, const float* __restrict__ hr, float* __restrict__ do_ws,
+    float* __restrict__ dot_ws, float* __restrict__ dom_ws, int* __restrict__ dsafe,
+    float* __restrict__ A, float* __restrict__ dwpart) {
   __shared__ float red[4][128];
-  const int Dv = d.Dv, kv = blockIdx.y;
+  extern __shared__ float hmax[];   // [grp] max |do| per head
+  const int Dv = d.Dv, Dk = d.Dk, kv = blockIdx.y, ci = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float wv[4], dwl[4];
+  const Chunk ch = chunks[ci];
+  for (int i = threadIdx.x; i < d.grp; i += blockDim.x) hmax[i] = 0.f;
+  __syncthreads();
+  float wv[4], dwl[4], rh[4], good[4];
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
     const int c = lane + 32 * u;
     wv[u] = c < Dv ? bf2f(w[c]) : 0.f;
     dwl[u] = 0.f;
+    const size_t ti = ((size_t)ci * d.Hkv + kv) * Dv + c;
+    rh[u] = (dot_ws && c < Dv) ? rho[ti] : 0.f;
+    good[u] = (dot_ws && c < Dv) ? (hr[ti] <= FIX_HR_MAX ? 1.f : 0.f) : 0.f;
   }
   const size_t ors = (size_t)d.Hq * Dv, vrs = (size_t)d.Hkv * Dv;
-  for (int t = blockIdx.x * 4 + warp; t < d.N; t += gridDim.x * 4) {
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  const size_t qrs = (size_t)d.Hq * Dk, krs = (size_t)d.Hkv * Dk;
+  for (int r = warp; r < ch.len; r += 4) {
+    const size_t t = (size_t)ch.tok0 + r;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f}, vr[4], lr[4], kr[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int c = lane + 32 * u;
+      vr[u] = c < Dv ? bf2f(v[t * vrs + (size_t)kv * Dv + c]) : 0.f;
+      lr[u] = (dot_ws && c < Dv) ? L[t * vrs + (size_t)kv * Dv + c] : 0.f;
+      kr[u] = c < Dk ? bf2f(k[t * krs + (size_t)kv * Dk + c]) : 0.f;
+    }
     for (int hh = 0; hh < d.grp; ++hh) {
       const int h = kv * d.grp + hh;
-      const float r = rstd_s[(size_t)t * d.Hq + h];
+      const float rs_ = rstd_s[t * d.Hq + h];
+      float sdot = 0.f;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int c = lane + 32 * u;
+        if (c < Dk) sdot += bf2f(q[t * qrs + (size_t)h * Dk + c]) * kr[u];
+      }
+      const float ptt = expf(warp_sum(sdot) * d.scale - m_s[t * d.Hq + h]);
       float ov[4], dn[4], n[4], dot = 0.f;
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int c = lane + 32 * u;
-        const size_t a = (size_t)t * ors + (size_t)h * Dv + c;
+        const size_t a = t * ors + (size_t)h * Dv + c;
         ov[u] = c < Dv ? o_s[a] : 0.f;
         const float dyv = c < Dv ? bf2f(dy[a]) : 0.f;
-        n[u] = ov[u] * r;
+        n[u] = ov[u] * rs_;
         dn[u] = dyv * wv[u];
         dot += dn[u] * n[u];
         dwl[u] += dyv * n[u];
       }
       dot = warp_sum(dot) / (float)Dv;
+      float mx = 0.f;
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int c = lane + 32 * u;
         if (c >= Dv) continue;
-        const float dov = r * (dn[u] - n[u] * dot);
-        do_ws[(size_t)t * ors + (size_t)h * Dv + c] = dov;
-        acc[u] += dov * ov[u];
+        const float dov = rs_ * (dn[u] - n[u] * dot);
+        const size_t a = t * ors + (size_t)h * Dv + c;
+        do_ws[a] = dov;
+        acc[u] += dov * (ov[u] - ptt * vr[u]);
+        if (dot_ws) {
+          dot_ws[a] = dov * expf(lr[u]);
+          dom_ws[a] = good[u] != 0.f ? dov * expf(lr[u] - rh[u]) : 0.f;
+          mx = fmaxf(mx, fabsf(dov));
+        }
+      }
+      if (dot_ws) {
+        mx = warp_max(mx);
+        if (lane == 0) atomicMax(reinterpret_cast<int*>(&hmax[hh]), __float_as_int(mx));
       }
     }
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int c = lane + 32 * u;
-      if (c < Dv) A[(size_t)t * vrs + (size_t)kv * Dv + c] = acc[u];
+      if (c < Dv) A[t * vrs + (size_t)kv * Dv + c] = acc[u];
     }
   }
 #pragma unroll
@@ -211,9 +261,12 @@ __global__ void __launch_bounds__(128) bwd_pre_kernel(
   __syncthreads();
   const int c = threadIdx.x;
   if (c < Dv) {
-    const float s = red[0][c] + red[1][c] + red[2][c] + red[3][c];
-    dwpart[((size_t)blockIdx.y * gridDim.x + blockIdx.x) * Dv + c] = s;
+    const float sm = red[0][c] + red[1][c] + red[2][c] + red[3][c];
+    dwpart[((size_t)ci * d.Hkv + kv) * Dv + c] = sm;
   }
+  if (dot_ws)
+    for (int i = threadIdx.x; i < d.grp; i += blockDim.x)
+      dsafe[(size_t)ci * d.Hq + kv * d.grp + i] = hmax[i] <= FIX_F16_VMAX ? 1 : 0;
 }
 
 // dw = sum of the partials in a fixed order (deterministic).  One CTA.
@@ -236,7 +289,8 @@ __global__ void __launch_bounds__(256) dq_simt_kernel(
     const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
     const float* __restrict__ L, const float* __restrict__ tot,
     const float* __restrict__ m_s, const float* __restrict__ do_ws,
-    __nv_bfloat16* __restrict__ dq) {
+    __nv_bfloat16* __restrict__ dq, const int* __restrict__ gate) {
+  if (gate && *gate == 0) return;  // the tensor-core kernel handles this problem
   extern __shared__ float sm[];
   const int Dk = d.Dk, Dv = d.Dv;
   float* sQ = sm;                        // [ST][Dk]
@@ -349,7 +403,8 @@ __global__ void __launch_bounds__(256) dq_simt_kernel(
 // dk, dv and dG.  grid (nchunks * 4, Hkv), block 256: 32 key rows per CTA,
 // 4 per warp, looping over the kv group's q heads and every later query row.
 //   dv_s += P_ts D_ts do_t ;  dk_s += scale dS_ts q_t ;
-//   dG_s  = A_s - v_s dv_s   (A from bwd_pre_kernel)
+//   dG_s  = A_s - v_s dv_strict_s   (A from bwd_pre_kernel, both without the
+//   s = t pair; dv_strict = dv minus that pair's P_ss do_s)
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) dkv_simt_kernel(
     Dims d, const Chunk* __restrict__ chunks, const __nv_bfloat16* __restrict__ q,
@@ -357,7 +412,8 @@ __global__ void __launch_bounds__(256) dkv_simt_kernel(
     const float* __restrict__ L, const float* __restrict__ tot,
     const float* __restrict__ m_s, const float* __restrict__ do_ws,
     const float* __restrict__ A, __nv_bfloat16* __restrict__ dk,
-    __nv_bfloat16* __restrict__ dv, float* __restrict__ dG) {
+    __nv_bfloat16* __restrict__ dv, float* __restrict__ dG, const int* __restrict__ gate) {
+  if (gate && *gate == 0) return;  // the tensor-core kernel handles this problem
   extern __shared__ float sm[];
   const int Dk = d.Dk, Dv = d.Dv;
   float* sQ = sm;                        // [ST][Dk]
@@ -375,7 +431,7 @@ __global__ void __launch_bounds__(256) dkv_simt_kernel(
   const size_t vrs = (size_t)d.Hkv * Dv, ors = (size_t)d.Hq * Dv;
   const int first = ci - ch.j;
 
-  float kr[4][4], vr[4][4], lk[4][4], gk[4][4], gv[4][4];
+  float kr[4][4], vr[4][4], lk[4][4], gk[4][4], gv[4][4], gd[4][4];
 #pragma unroll
   for (int a = 0; a < 4; ++a) {
     const int key = warp * 4 + a;
@@ -388,6 +444,7 @@ __global__ void __launch_bounds__(256) dkv_simt_kernel(
       lk[a][u] = dd < Dv ? L[tok * vrs + (size_t)kv * Dv + dd] : 0.f;
       gk[a][u] = 0.f;
       gv[a][u] = 0.f;
+      gd[a][u] = 0.f;
     }
   }
 
@@ -445,11 +502,16 @@ __global__ void __launch_bounds__(256) dkv_simt_kernel(
             }
             dp = warp_sum(dp);
             const float ds = p * dp;
+            const bool same = spos == tpos;
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
               const int dd = lane + 32 * u;
               if (dd < Dk) gk[a][u] += ds * sQ[r * Dk + dd];
-              if (dd < Dv) gv[a][u] += p * dc[u] * sDo[r * Dv + dd];
+              if (dd < Dv) {
+                const float x = p * dc[u] * sDo[r * Dv + dd];
+                if (same) gd[a][u] += x;
+                else gv[a][u] += x;
+              }
             }
           }
         }
@@ -467,7 +529,7 @@ __global__ void __launch_bounds__(256) dkv_simt_kernel(
       if (dd < Dk) dk[tok * krs + (size_t)kv * Dk + dd] = f2bf(gk[a][u] * d.scale);
       if (dd < Dv) {
         const size_t av = tok * vrs + (size_t)kv * Dv + dd;
-        dv[av] = f2bf(gv[a][u]);
+        dv[av] = f2bf(gv[a][u] + gd[a][u]);
         dG[av] = A[av] - vr[a][u] * gv[a][u];
       }
     }

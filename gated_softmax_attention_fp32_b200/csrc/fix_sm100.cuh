@@ -75,7 +75,7 @@ struct Ctl {
 // Waits for the phase with `parity` to complete; gives up after 1 s (sets the
 // status word to FIX_DEV_TIMEOUT and the CTA abort flag) or when another role
 // aborted.  Returns false when it gave up.
-__device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, Ctl ctl) {
+static __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, Ctl ctl) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer();
   while (true) {

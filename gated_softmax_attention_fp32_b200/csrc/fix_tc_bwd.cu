@@ -1,0 +1,906 @@
+// FiX attention backward on the tcgen05 tensor cores (sm_100a).
+//
+// With the row shift m_t held constant (it cancels under the RMSNorm), the
+// gradients of o_t[c] = sum_{s<=t} P_ts D_ts[c] v_s[c] are
+//   dP_ts = sum_c do_t[c] D_ts[c] v_s[c],   dS_ts = P_ts dP_ts,
+//   dq_t  = scale sum_s dS_ts k_s,          dk_s = scale sum_t dS_ts q_t,
+//   dv_s  = sum_t P_ts D_ts do_t,           dG_t = A_t - v_t dv_strict_t,
+// where A (row part, from the preprocess) and dv_strict both leave out the
+// s = t pair.  The FiX README lists the reference's backward as intra-chunk,
+// inter-chunk dKV and inter-chunk dQ passes with inter-chunk scaling of dO;
+// here two kernels cover every block pair, with the decay split exactly as in
+// the forward:
+//   * diagonal block (same chunk): reference rho, operands Vm (prefix pass)
+//     and dOm = do exp(L_t - rho) (preprocess);
+//   * earlier key blocks: reference = the query chunk's start, operands
+//     Vt (prefix pass, pre-decayed to the key chunk's end), dOt = do exp(L_t)
+//     and the per-pair channel factor f_ij = exp(sum_{j<j'<i} tot_j').
+//
+// dq kernel (one CTA per 128-row query chunk and q head, key blocks i..0):
+//   S = Q K^T and dP = dO V'^T into TMEM, dS = P dP (fp32, then bf16, written
+//   over S), dQ += dS K.  V' = Vt f_ij is formed in shared memory per block.
+// dk/dv kernel (one CTA per 128-row key chunk and kv head; the group's q heads
+// and 64-row query tiles of every later chunk stream through):
+//   S^T = K Q^T, dP^T = V X^T (X = dOt f_ij, or dOm on the diagonal),
+//   dV += P^T X, dK += dS^T Q.  On the diagonal, whose terms dominate dv and
+//   whose rounding would dominate dG, P and dOm are split into bf16 hi + lo
+//   parts (three MMAs into their own accumulator dV_d); elsewhere one MMA in
+//   fp16 when every gate <= 0 and |v|, |do| <= 3e4, else bf16, into dV_o.
+//   Epilogue: dv_strict = exp(rho - L_s) dV_d + exp(tot_j - L_s) dV_o,
+//   dv = dv_strict + sum_h P_ss do_s, dG = A - v dv_strict, dk = scale dK.
+// Problems with a channel outside the split's float range (flag set by the
+// prefix pass) are left to the exact CUDA-core kernels, which run instead.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "fix_internal.h"
+#include "fix_sm100.cuh"
+
+namespace fix {
+namespace tcb {
+
+using namespace sm100;
+
+constexpr int BN = FIX_CHUNK;   // keys per block / rows per chunk
+constexpr int kThreads = 384;
+constexpr uint32_t kTmemCols = 512;
+
+struct Params {
+  Dims d;
+  const Chunk* chunks;
+  const int* order;
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* k;
+  const __nv_bfloat16* v;
+  const float* L;
+  const float* tot;
+  const float* rho;
+  const float* hr;
+  const int* safe;
+  const int* dsafe;
+  const float* m_s;
+  const float* do_ws;
+  const float* dot_ws;
+  const float* dom_ws;
+  const float* A;
+  const int* badflag;
+  __nv_bfloat16* dq;
+  __nv_bfloat16* dk;
+  __nv_bfloat16* dv;
+  float* dG;
+  int* status;
+};
+
+// Byte offset of element (row, col) in a 128-byte-swizzled K-major tile of
+// `rows` rows whose columns come in 64-wide halves.
+__device__ __forceinline__ uint32_t sw_off(int rows, int row, int col) {
+  return (uint32_t)((col >> 6) * (rows * 128) + row * 128 + ((((col & 63) >> 3) ^ (row & 7)) << 4));
+}
+
+// Converts 8 floats to 8 16-bit values (fp16 or bf16) packed in a uint4.
+__device__ __forceinline__ uint4 pack8(const float* x, bool f16) {
+  uint4 r;
+  if (f16) {
+    r.x = pack_f16(x[0], x[1]); r.y = pack_f16(x[2], x[3]);
+    r.z = pack_f16(x[4], x[5]); r.w = pack_f16(x[6], x[7]);
+  } else {
+    r.x = pack_bf16(x[0], x[1]); r.y = pack_bf16(x[2], x[3]);
+    r.z = pack_bf16(x[4], x[5]); r.w = pack_bf16(x[6], x[7]);
+  }
+  return r;
+}
+__device__ __forceinline__ void unpack8(uint4 u, bool f16, float* x) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    if (f16) {
+      const float2 ab = __half22float2(*reinterpret_cast<const __half2*>(&w[i]));
+      x[2 * i] = ab.x;
+      x[2 * i + 1] = ab.y;
+    } else {
+      x[2 * i] = __uint_as_float(w[i] << 16);
+      x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+  }
+}
+
+// =========================================================================== dq
+
+struct DqBars {
+  uint64_t q_full, o_ready;
+  uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2], v_ready[2];
+  uint64_t s_full, ds_ready, dp0_done, done, drain;
+};
+
+template <int DK, int DV>
+struct DqLayout {
+  static constexpr int kQ = 0;                       // [128][DK] bf16
+  static constexpr int kO = kQ + BN * DK * 2;        // [128][DV] dO operand
+  static constexpr int kK = kO + BN * DV * 2;        // 2 x [128][DK]
+  static constexpr int kV = kK + 2 * BN * DK * 2;    // 2 x [128][DV]
+  static constexpr int kBars = kV + 2 * BN * DV * 2;
+  static constexpr int kTmem = kBars + (int)sizeof(DqBars);
+  static constexpr int kAbort = kTmem + 4;
+  static constexpr int kAlloc = kAbort + 4 + 1024;
+};
+
+template <int DK, int DV>
+__global__ void __launch_bounds__(kThreads, 1)
+    dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                 const __grid_constant__ CUtensorMap tm_vt, const __grid_constant__ CUtensorMap tm_vm,
+                 const Params P) {
+  using Lay = DqLayout<DK, DV>;
+  if (*P.badflag) return;  // exact kernels run instead
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const Dims& d = P.d;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int ci = P.order[blockIdx.x / d.Hq];
+  const int h = blockIdx.x % d.Hq, kv = h / d.grp;
+  const Chunk ch = P.chunks[ci];
+  if (ch.len <= 0) return;
+  const int nblk = ch.j + 1, first = ci - ch.j, seq0 = ch.tok0 - ch.j * FIX_CHUNK;
+
+  __nv_bfloat16* sQ = reinterpret_cast<__nv_bfloat16*>(smem + Lay::kQ);
+  uint8_t* sO = smem + Lay::kO;
+  __nv_bfloat16* sK = reinterpret_cast<__nv_bfloat16*>(smem + Lay::kK);
+  __nv_bfloat16* sV = reinterpret_cast<__nv_bfloat16*>(smem + Lay::kV);
+  DqBars* bar = reinterpret_cast<DqBars*>(smem + Lay::kBars);
+  uint32_t* sTmem = reinterpret_cast<uint32_t*>(smem + Lay::kTmem);
+  volatile int* sAbort = reinterpret_cast<volatile int*>(smem + Lay::kAbort);
+  const Ctl ctl{P.status, sAbort};
+
+  if (tid == 0) {
+    *sAbort = 0;
+    mbar_init(&bar->q_full, 1);
+    mbar_init(&bar->o_ready, 128);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bar->k_full[s], 1);
+      mbar_init(&bar->k_empty[s], 1);
+      mbar_init(&bar->v_full[s], 1);
+      mbar_init(&bar->v_empty[s], 1);
+      mbar_init(&bar->v_ready[s], 128);
+    }
+    mbar_init(&bar->s_full, 1);
+    mbar_init(&bar->ds_ready, 128);
+    mbar_init(&bar->dp0_done, 1);
+    mbar_init(&bar->done, 1);
+    mbar_init(&bar->drain, 1);
+    mbar_fence_init();
+  }
+  if (warp == 1) tmem_alloc(sTmem, kTmemCols);
+  bool my_safe = true;
+  for (int jj = tid; jj < nblk; jj += blockDim.x)
+    my_safe = my_safe && P.safe[(size_t)(first + jj) * d.Hkv + kv];
+  if (tid == 0) my_safe = my_safe && P.dsafe[(size_t)ci * d.Hq + h];
+  tc_fence_before();
+  const int cta_f16 = __syncthreads_and(my_safe);
+  tc_fence_after();
+  const uint32_t tmem = *sTmem;
+  constexpr uint32_t kColS = 0, kColP = 128, kColQ = 256;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      mbar_expect_tx(&bar->q_full, BN * DK * 2);
+      for (int hh = 0; hh < DK / 64; ++hh)
+        tma_load_3d(sQ + hh * BN * 64, &tm_q, &bar->q_full, hh * 64, h, ch.tok0);
+      int nk = 0, nv = 0;
+      for (int it = 0; it < nblk; ++it) {
+        const int st = it & 1;
+        const uint32_t ph = (it >> 1) & 1;
+        const int ktok = seq0 + (ch.j - it) * FIX_CHUNK;
+        if (it >= 2 && !mbar_wait(&bar->k_empty[st], ph ^ 1, ctl)) break;
+        mbar_expect_tx(&bar->k_full[st], BN * DK * 2);
+        for (int hh = 0; hh < DK / 64; ++hh)
+          tma_load_3d(sK + st * BN * DK + hh * BN * 64, &tm_k, &bar->k_full[st], hh * 64, kv, ktok);
+        ++nk;
+        if (it >= 2 && !mbar_wait(&bar->v_empty[st], ph ^ 1, ctl)) break;
+        mbar_expect_tx(&bar->v_full[st], BN * DV * 2);
+        const CUtensorMap* vmap = it == 0 ? &tm_vm : &tm_vt;
+        for (int hh = 0; hh < DV / 64; ++hh)
+          tma_load_3d(sV + st * BN * DV + hh * BN * 64, vmap, &bar->v_full[st], hh * 64, kv, ktok);
+        ++nv;
+      }
+      const Ctl drain{P.status, nullptr};
+      for (int it = nk - 1; it >= 0 && it >= nk - 2; --it)
+        mbar_wait(&bar->k_full[it & 1], (it >> 1) & 1, drain);
+      for (int it = nv - 1; it >= 0 && it >= nv - 2; --it)
+        mbar_wait(&bar->v_full[it & 1], (it >> 1) & 1, drain);
+      mbar_wait(&bar->q_full, 0, drain);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16(128, BN, false, false);
+      const uint32_t idesc_dp0 = idesc_bf16(128, BN, false, false);
+      const uint32_t idesc_dp = idesc_bf16(128, BN, false, false, cta_f16 != 0);
+      constexpr uint32_t idesc_dq = idesc_bf16(128, DK, false, true);
+      const uint32_t q_addr = smem_u32(sQ), o_addr = smem_u32(sO);
+      bool ok = mbar_wait(&bar->q_full, 0, ctl) && mbar_wait(&bar->o_ready, 0, ctl);
+      for (int it = 0; ok && it < nblk; ++it) {
+        const int st = it & 1;
+        const uint32_t ph = (it >> 1) & 1;
+        if (!mbar_wait(&bar->k_full[st], ph, ctl) || !mbar_wait(&bar->v_ready[st], ph, ctl)) break;
+        if (it == 1 && !mbar_wait(&bar->o_ready, 1, ctl)) break;
+        tc_fence_after();
+        const uint32_t k_addr = smem_u32(sK + st * BN * DK), v_addr = smem_u32(sV + st * BN * DV);
+#pragma unroll
+        for (int kk = 0; kk < DK / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (BN * 128) + (kk & 3) * 32;
+          mma_ss(tmem + kColS, desc_sw128(q_addr + off, 16, 1024), desc_sw128(k_addr + off, 16, 1024),
+                 idesc_s, kk > 0);
+        }
+#pragma unroll
+        for (int kk = 0; kk < DV / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (BN * 128) + (kk & 3) * 32;
+          mma_ss(tmem + kColP, desc_sw128(o_addr + off, 16, 1024), desc_sw128(v_addr + off, 16, 1024),
+                 it == 0 ? idesc_dp0 : idesc_dp, kk > 0);
+        }
+        tc_commit(&bar->s_full);
+        if (it == 0) tc_commit(&bar->dp0_done);
+        if (!mbar_wait(&bar->ds_ready, it & 1, ctl)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          const uint64_t b = desc_sw128(k_addr + kk * 2048, BN * 128, 1024);
+          mma_ts(tmem + kColQ, tmem + kColS + kk * 8, b, idesc_dq, (it > 0 || kk > 0));
+        }
+        tc_commit(&bar->k_empty[st]);
+        tc_commit(&bar->v_empty[st]);
+      }
+      tc_commit(&bar->done);
+      tc_commit(&bar->drain);
+      mbar_wait(&bar->drain, 0, Ctl{P.status, nullptr});
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // ------------------------------------------------------------ dS + epilogue
+    const int r = (warp - 4) * 32 + lane;
+    const uint32_t lane_base = tmem + ((uint32_t)((warp - 4) * 32) << 16);
+    const bool row_ok = r < ch.len;
+    const size_t tok = (size_t)ch.tok0 + (size_t)(row_ok ? r : 0);
+    const float moff = P.m_s[tok * d.Hq + h] * LOG2E;
+    const float c1 = d.scale * LOG2E;
+    bool ok = true;
+    for (int it = 0; it < nblk; ++it) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar->s_full, it & 1, ctl))) { ok = false; break; }
+      tc_fence_after();
+#pragma unroll
+      for (int c4 = 0; c4 < BN / 32; ++c4) {
+        uint32_t xs[32], xp[32], pk[16];
+        tmem_ld32(lane_base + kColS + c4 * 32, xs);
+        tmem_ld32(lane_base + kColP + c4 * 32, xp);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const int key = c4 * 32 + e;
+          const bool v0 = row_ok && (it > 0 || key <= r), v1 = row_ok && (it > 0 || key + 1 <= r);
+          const float p0 = v0 ? ex2(__uint_as_float(xs[e]) * c1 - moff) : 0.f;
+          const float p1 = v1 ? ex2(__uint_as_float(xs[e + 1]) * c1 - moff) : 0.f;
+          pk[e >> 1] = pack_bf16(p0 * __uint_as_float(xp[e]), p1 * __uint_as_float(xp[e + 1]));
+        }
+        tmem_st16(lane_base + kColS + c4 * 16, pk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bar->ds_ready);
+    }
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bar->done, 0, ctl));
+    tc_fence_after();
+    float acc[DK];
+#pragma unroll
+    for (int cc = 0; cc < DK / 32; ++cc) {
+      uint32_t x[32];
+      tmem_ld32(lane_base + kColQ + cc * 32, x);
+      tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 32; ++e) acc[cc * 32 + e] = __uint_as_float(x[e]) * d.scale;
+    }
+    if (ok && row_ok) {
+      __nv_bfloat16* dqp = P.dq + tok * (size_t)d.Hq * DK + (size_t)h * DK;
+#pragma unroll
+      for (int c = 0; c < DK; c += 8) {
+        uint4 pkd;
+        pkd.x = pack_bf16(acc[c], acc[c + 1]);
+        pkd.y = pack_bf16(acc[c + 2], acc[c + 3]);
+        pkd.z = pack_bf16(acc[c + 4], acc[c + 5]);
+        pkd.w = pack_bf16(acc[c + 6], acc[c + 7]);
+        *reinterpret_cast<uint4*>(dqp + c) = pkd;
+      }
+    }
+  } else if (warp >= 8) {
+    // ------------------------------------------------------------ operands in smem
+    const int dt = tid - 256;
+    constexpr int kChunks = DV / 8;
+    constexpr int kRowsPerPass = 128 / kChunks;
+    const int lc = dt % kChunks, r0 = dt / kChunks;
+    const size_t ors = (size_t)d.Hq * DV;
+    // dO operand: dOm (bf16) for the diagonal block, then dOt (CTA format)
+    for (int phase = 0; phase < (nblk > 1 ? 2 : 1); ++phase) {
+      if (phase == 1 && !mbar_wait(&bar->dp0_done, 0, ctl)) break;
+      const float* src = phase == 0 ? P.dom_ws : P.dot_ws;
+      const bool f16 = phase == 1 && cta_f16;
+      for (int rr = r0; rr < BN; rr += kRowsPerPass) {
+        float x[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        if (rr < ch.len) {
+          const float* p = src + ((size_t)ch.tok0 + rr) * ors + (size_t)h * DV + lc * 8;
+          const float4 a = *reinterpret_cast<const float4*>(p);
+          const float4 b = *reinterpret_cast<const float4*>(p + 4);
+          x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+          x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+        }
+        *reinterpret_cast<uint4*>(sO + sw_off(BN, rr, lc * 8)) = pack8(x, f16);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&bar->o_ready);
+      if (phase == 0) {
+        // the diagonal block's V (Vm) goes to the MMA as loaded
+        if (!mbar_wait(&bar->v_full[0], 0, ctl)) break;
+        mbar_arrive(&bar->v_ready[0]);
+      }
+    }
+    // V' = Vt f_ij for the earlier key blocks
+    float delta[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) delta[e] = 0.f;
+    for (int it = 1; it < nblk; ++it) {
+      const int st = it & 1, j = ch.j - it;
+      if (it >= 2) {
+        const float* tp = P.tot + ((size_t)(first + j + 1) * d.Hkv + kv) * DV + lc * 8;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) delta[e] += tp[e];
+      }
+      float f8[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) f8[e] = ex2(delta[e] * LOG2E);
+      if (!mbar_wait(&bar->v_full[st], (it >> 1) & 1, ctl)) break;
+      const bool in_f16 = P.safe[(size_t)(first + j) * d.Hkv + kv] != 0;
+      uint8_t* vb = reinterpret_cast<uint8_t*>(sV + st * BN * DV);
+      for (int rr = r0; rr < BN; rr += kRowsPerPass) {
+        uint4* p = reinterpret_cast<uint4*>(vb + sw_off(BN, rr, lc * 8));
+        float x[8];
+        unpack8(*p, in_f16, x);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[e] *= f8[e];
+        *p = pack8(x, cta_f16);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&bar->v_ready[st]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ========================================================================= dk/dv
+
+constexpr int BQ = 64;   // query rows per streamed tile
+
+struct KvBars {
+  uint64_t kv_full;
+  uint64_t q_full[2], q_empty[2], x_ready[2], x_empty[2];
+  uint64_t s_full, p_ready, done, drain;
+};
+
+template <int DK, int DV>
+struct KvLayout {
+  static constexpr int kK = 0;                         // [128][DK]
+  static constexpr int kVt = kK + BN * DK * 2;         // [128][DV] Vt
+  static constexpr int kVm = kVt + BN * DV * 2;        // [128][DV] Vm (hi)
+  static constexpr int kQ = kVm + BN * DV * 2;         // 2 x [64][DK]
+  static constexpr int kX = kQ + 2 * BQ * DK * 2;      // 2 x [64][DV]
+  static constexpr int kXl = kX + 2 * BQ * DV * 2;     // 2 x [64][DV] (diagonal lo part)
+  static constexpr int kM = kXl + 2 * BQ * DV * 2;     // 2 x [64] f32 row max
+  static constexpr int kBars = kM + 2 * BQ * 4;
+  static constexpr int kTmem = kBars + (int)sizeof(KvBars);
+  static constexpr int kAbort = kTmem + 4;
+  static constexpr int kAlloc = kAbort + 4 + 1024;
+};
+
+// The tiles a dk/dv CTA streams, in order: for each q head of the group, for
+// each query chunk i >= j, the 64-row halves that hold rows.
+struct TileIter {
+  int hh, i, half;
+};
+
+template <int DK, int DV>
+__global__ void __launch_bounds__(kThreads, 1)
+    dkv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_vt, const __grid_constant__ CUtensorMap tm_vm,
+                  const Params P) {
+  using Lay = KvLayout<DK, DV>;
+  if (*P.badflag) return;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const Dims& d = P.d;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int cj = P.order[P.d.nchunks - 1 - blockIdx.x / d.Hkv];   // short rows last -> long first
+  const int kv = blockIdx.x % d.Hkv;
+  const Chunk ch = P.chunks[cj];
+  if (ch.len <= 0) return;
+  const int first = cj - ch.j;
+  const int nq_chunks = ch.nch - ch.j;                 // chunks i = j .. nch-1
+  // tiles per head: every chunk after j has 128 rows except possibly the last
+  auto chunk_len = [&](int i) { return P.chunks[first + i].len; };
+  int tiles_per_head = 0;
+  for (int i = ch.j; i < ch.nch; ++i) tiles_per_head += (chunk_len(i) + BQ - 1) / BQ;
+  const int ntiles = tiles_per_head * d.grp;
+
+  uint8_t* sK = smem + Lay::kK;
+  uint8_t* sVt = smem + Lay::kVt;
+  uint8_t* sVm = smem + Lay::kVm;
+  uint8_t* sQ = smem + Lay::kQ;
+  uint8_t* sX = smem + Lay::kX;
+  uint8_t* sXl = smem + Lay::kXl;
+  float* sM = reinterpret_cast<float*>(smem + Lay::kM);
+  KvBars* bar = reinterpret_cast<KvBars*>(smem + Lay::kBars);
+  uint32_t* sTmem = reinterpret_cast<uint32_t*>(smem + Lay::kTmem);
+  volatile int* sAbort = reinterpret_cast<volatile int*>(smem + Lay::kAbort);
+  const Ctl ctl{P.status, sAbort};
+
+  if (tid == 0) {
+    *sAbort = 0;
+    mbar_init(&bar->kv_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bar->q_full[s], 1);
+      mbar_init(&bar->q_empty[s], 1);
+      mbar_init(&bar->x_ready[s], 128);
+      mbar_init(&bar->x_empty[s], 1);
+    }
+    mbar_init(&bar->s_full, 1);
+    mbar_init(&bar->p_ready, 128);
+    mbar_init(&bar->done, 1);
+    mbar_init(&bar->drain, 1);
+    mbar_fence_init();
+  }
+  if (warp == 1) tmem_alloc(sTmem, kTmemCols);
+  bool my_safe = true;
+  for (int i = tid; i < nq_chunks; i += blockDim.x) {
+    my_safe = my_safe && P.safe[(size_t)(first + ch.j + i) * d.Hkv + kv];
+    for (int hh = 0; hh < d.grp; ++hh)
+      my_safe = my_safe && P.dsafe[(size_t)(first + ch.j + i) * d.Hq + kv * d.grp + hh];
+  }
+  tc_fence_before();
+  const int cta_f16 = __syncthreads_and(my_safe);
+  tc_fence_after();
+  const uint32_t tmem = *sTmem;
+  constexpr uint32_t kColS = 0, kColP = 64, kColVd = 128, kColVo = 128 + DV, kColK = 128 + 2 * DV;
+
+  // walk the tile sequence (identical in every role)
+  auto next_tile = [&](TileIter& t) {
+    ++t.half;
+    if (t.half * BQ >= chunk_len(t.i)) {
+      t.half = 0;
+      ++t.i;
+      if (t.i >= ch.nch) {
+        t.i = ch.j;
+        ++t.hh;
+      }
+    }
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      mbar_expect_tx(&bar->kv_full, BN * DK * 2 + 2 * BN * DV * 2);
+      for (int hh = 0; hh < DK / 64; ++hh)
+        tma_load_3d(sK + hh * BN * 128, &tm_k, &bar->kv_full, hh * 64, kv, ch.tok0);
+      for (int hh = 0; hh < DV / 64; ++hh) {
+        tma_load_3d(sVt + hh * BN * 128, &tm_vt, &bar->kv_full, hh * 64, kv, ch.tok0);
+        tma_load_3d(sVm + hh * BN * 128, &tm_vm, &bar->kv_full, hh * 64, kv, ch.tok0);
+      }
+      TileIter t{0, ch.j, 0};
+      int nq = 0;
+      for (int n = 0; n < ntiles; ++n, next_tile(t)) {
+        const int st = n & 1;
+        if (n >= 2 && !mbar_wait(&bar->q_empty[st], ((n >> 1) & 1) ^ 1, ctl)) break;
+        mbar_expect_tx(&bar->q_full[st], BQ * DK * 2);
+        const int h = kv * d.grp + t.hh;
+        const int qtok = P.chunks[first + t.i].tok0 + t.half * BQ;
+        for (int hh = 0; hh < DK / 64; ++hh)
+          tma_load_3d(sQ + st * BQ * DK * 2 + hh * BQ * 128, &tm_q, &bar->q_full[st], hh * 64, h, qtok);
+        ++nq;
+      }
+      const Ctl drain{P.status, nullptr};
+      for (int n = nq - 1; n >= 0 && n >= nq - 2; --n)
+        mbar_wait(&bar->q_full[n & 1], (n >> 1) & 1, drain);
+      mbar_wait(&bar->kv_full, 0, drain);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16(128, BQ, false, false);
+      const uint32_t idesc_dp_off = idesc_bf16(128, BQ, false, false, cta_f16 != 0);
+      constexpr uint32_t idesc_dp_diag = idesc_bf16(128, BQ, false, false);
+      const uint32_t idesc_dv_off = idesc_bf16(128, DV, false, true, cta_f16 != 0);
+      constexpr uint32_t idesc_dv_diag = idesc_bf16(128, DV, false, true);
+      constexpr uint32_t idesc_dk = idesc_bf16(128, DK, false, true);
+      const uint32_t k_addr = smem_u32(sK), vt_addr = smem_u32(sVt), vm_addr = smem_u32(sVm);
+      bool ok = mbar_wait(&bar->kv_full, 0, ctl);
+      bool first_diag = true, first_off = true;
+      TileIter t{0, ch.j, 0};
+      for (int n = 0; ok && n < ntiles; ++n, next_tile(t)) {
+        const int st = n & 1;
+        const uint32_t ph = (n >> 1) & 1;
+        const bool diag = t.i == ch.j;
+        if (!mbar_wait(&bar->q_full[st], ph, ctl) || !mbar_wait(&bar->x_ready[st], ph, ctl)) break;
+        tc_fence_after();
+        const uint32_t q_addr = smem_u32(sQ + st * BQ * DK * 2);
+        const uint32_t x_addr = smem_u32(sX + st * BQ * DV * 2);
+        const uint32_t xl_addr = smem_u32(sXl + st * BQ * DV * 2);
+        // S^T = K Q^T   (M = 128 keys, N = 64 queries, K = DK)
+#pragma unroll
+        for (int kk = 0; kk < DK / 16; ++kk) {
+          const uint32_t ka = (kk >> 2) * (BN * 128) + (kk & 3) * 32;
+          const uint32_t qa = (kk >> 2) * (BQ * 128) + (kk & 3) * 32;
+          mma_ss(tmem + kColS, desc_sw128(k_addr + ka, 16, 1024), desc_sw128(q_addr + qa, 16, 1024),
+                 idesc_s, kk > 0);
+        }
+        // dP^T = V X^T  (V = Vm on the diagonal, Vt elsewhere)
+        const uint32_t va = diag ? vm_addr : vt_addr;
+#pragma unroll
+        for (int kk = 0; kk < DV / 16; ++kk) {
+          const uint32_t vo = (kk >> 2) * (BN * 128) + (kk & 3) * 32;
+          const uint32_t xo = (kk >> 2) * (BQ * 128) + (kk & 3) * 32;
+          mma_ss(tmem + kColP, desc_sw128(va + vo, 16, 1024), desc_sw128(x_addr + xo, 16, 1024),
+                 diag ? idesc_dp_diag : idesc_dp_off, kk > 0);
+        }
+        tc_commit(&bar->s_full);
+        if (!mbar_wait(&bar->p_ready, n & 1, ctl)) break;
+        tc_fence_after();
+        // dV += P^T X  (K = 64 queries; X read MN-major)
+#pragma unroll
+        for (int kk = 0; kk < BQ / 16; ++kk) {
+          const uint64_t bx = desc_sw128(x_addr + kk * 2048, BQ * 128, 1024);
+          if (diag) {
+            const uint64_t bxl = desc_sw128(xl_addr + kk * 2048, BQ * 128, 1024);
+            mma_ts(tmem + kColVd, tmem + kColS + kk * 8, bx, idesc_dv_diag, !(first_diag && kk == 0));
+            mma_ts(tmem + kColVd, tmem + kColS + 32 + kk * 8, bx, idesc_dv_diag, 1);
+            mma_ts(tmem + kColVd, tmem + kColS + kk * 8, bxl, idesc_dv_diag, 1);
+          } else {
+            mma_ts(tmem + kColVo, tmem + kColS + kk * 8, bx, idesc_dv_off, !(first_off && kk == 0));
+          }
+        }
+        // dK += dS^T Q
+#pragma unroll
+        for (int kk = 0; kk < BQ / 16; ++kk) {
+          const uint64_t bq = desc_sw128(q_addr + kk * 2048, BQ * 128, 1024);
+          mma_ts(tmem + kColK, tmem + kColP + kk * 8, bq, idesc_dk, !(n == 0 && kk == 0));
+        }
+        if (diag) first_diag = false;
+        else first_off = false;
+        tc_commit(&bar->q_empty[st]);
+        tc_commit(&bar->x_empty[st]);
+      }
+      tc_commit(&bar->done);
+      tc_commit(&bar->drain);
+      mbar_wait(&bar->drain, 0, Ctl{P.status, nullptr});
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // ------------------------------------------------------------ P, dS + epilogue
+    const int s = (warp - 4) * 32 + lane;            // key row in the chunk
+    const uint32_t lane_base = tmem + ((uint32_t)((warp - 4) * 32) << 16);
+    const float c1 = d.scale * LOG2E;
+    bool ok = true;
+    TileIter t{0, ch.j, 0};
+    for (int n = 0; n < ntiles; ++n, next_tile(t)) {
+      const int st = n & 1;
+      const bool diag = t.i == ch.j;
+      const int qlen = min(BQ, chunk_len(t.i) - t.half * BQ);
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar->s_full, n & 1, ctl))) { ok = false; break; }
+      tc_fence_after();
+      uint32_t xs[64], xp[64];
+      tmem_ld32(lane_base + kColS, *reinterpret_cast<uint32_t(*)[32]>(&xs[0]));
+      tmem_ld32(lane_base + kColS + 32, *reinterpret_cast<uint32_t(*)[32]>(&xs[32]));
+      tmem_ld32(lane_base + kColP, *reinterpret_cast<uint32_t(*)[32]>(&xp[0]));
+      tmem_ld32(lane_base + kColP + 32, *reinterpret_cast<uint32_t(*)[32]>(&xp[32]));
+      tmem_wait_ld();
+      const float* mrow = sM + st * BQ;
+      uint32_t ph[32], pl[32], pd[32];
+#pragma unroll
+      for (int e = 0; e < BQ; e += 2) {
+        float p[2], pv[2], ds[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int qi = e + u;
+          const int tpos = t.half * BQ + qi;          // query row in chunk i
+          const bool valid = qi < qlen && (!diag || tpos >= s);
+          p[u] = valid ? ex2(__uint_as_float(xs[qi]) * c1 - mrow[qi] * LOG2E) : 0.f;
+          pv[u] = (diag && tpos == s) ? 0.f : p[u];   // dv leaves out the s = t pair
+          ds[u] = p[u] * __uint_as_float(xp[qi]);
+        }
+        if (diag) {
+          ph[e >> 1] = pack_bf16(pv[0], pv[1]);
+          const float h0 = __uint_as_float(ph[e >> 1] << 16);
+          const float h1 = __uint_as_float(ph[e >> 1] & 0xFFFF0000u);
+          pl[e >> 1] = pack_bf16(pv[0] - h0, pv[1] - h1);
+        } else {
+          ph[e >> 1] = cta_f16 ? pack_f16(pv[0], pv[1]) : pack_bf16(pv[0], pv[1]);
+          pl[e >> 1] = 0u;
+        }
+        pd[e >> 1] = pack_bf16(ds[0], ds[1]);
+      }
+      tmem_st32(lane_base + kColS, ph);
+      if (diag) tmem_st32(lane_base + kColS + 32, pl);
+      tmem_st32(lane_base + kColP, pd);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bar->p_ready);
+    }
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bar->done, 0, ctl));
+    tc_fence_after();
+    // ---------------------------------------------------------- epilogue
+    const bool row_ok = ok && s < ch.len;
+    const size_t tok = (size_t)ch.tok0 + (size_t)(s < ch.len ? s : 0);
+    const size_t vrs = (size_t)d.Hkv * DV, krs = (size_t)d.Hkv * DK, qrs = (size_t)d.Hq * DK;
+    const size_t ors = (size_t)d.Hq * DV;
+    const bool has_off = ch.nch - ch.j > 1;
+    const float* Lrow = P.L + tok * vrs + (size_t)kv * DV;
+    const float* trow = P.tot + ((size_t)cj * d.Hkv + kv) * DV;
+    const float* rrow = P.rho + ((size_t)cj * d.Hkv + kv) * DV;
+    // P_ss of every q head of the group (the s = t pair left out of dv_strict)
+    float pss[16];
+    const int ng = min(d.grp, 16);
+    const __nv_bfloat16* krow = P.k + tok * krs + (size_t)kv * DK;
+    for (int hh = 0; hh < ng; ++hh) {
+      const int h = kv * d.grp + hh;
+      const __nv_bfloat16* qrow = P.q + tok * qrs + (size_t)h * DK;
+      float acc = 0.f;
+      for (int dd = 0; dd < DK; dd += 8) {
+        float a8[8], b8[8];
+        unpack8(*reinterpret_cast<const uint4*>(qrow + dd), false, a8);
+        unpack8(*reinterpret_cast<const uint4*>(krow + dd), false, b8);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc += a8[e] * b8[e];
+      }
+      pss[hh] = ex2((acc * d.scale - P.m_s[tok * d.Hq + h]) * LOG2E);
+    }
+#pragma unroll
+    for (int cc = 0; cc < DV / 32; ++cc) {
+      uint32_t xd[32], xo[32];
+      tmem_ld32(lane_base + kColVd + cc * 32, xd);
+      tmem_ld32(lane_base + kColVo + cc * 32, xo);
+      tmem_wait_ld();
+      if (row_ok) {
+        float dvo[32], dgo[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int c = cc * 32 + e;
+          const float ls = Lrow[c];
+          float strict = __uint_as_float(xd[e]) * ex2((rrow[c] - ls) * LOG2E);
+          if (has_off) strict += __uint_as_float(xo[e]) * ex2((trow[c] - ls) * LOG2E);
+          float diagsum = 0.f;
+          for (int hh = 0; hh < ng; ++hh)
+            diagsum += pss[hh] * P.do_ws[tok * ors + (size_t)(kv * d.grp + hh) * DV + c];
+          dvo[e] = strict + diagsum;
+          dgo[e] = P.A[tok * vrs + (size_t)kv * DV + c] - bf2f(P.v[tok * vrs + (size_t)kv * DV + c]) * strict;
+        }
+        __nv_bfloat16* dvp = P.dv + tok * vrs + (size_t)kv * DV + cc * 32;
+        float* dgp = P.dG + tok * vrs + (size_t)kv * DV + cc * 32;
+#pragma unroll
+        for (int e = 0; e < 32; e += 8) {
+          uint4 pkd;
+          pkd.x = pack_bf16(dvo[e], dvo[e + 1]);
+          pkd.y = pack_bf16(dvo[e + 2], dvo[e + 3]);
+          pkd.z = pack_bf16(dvo[e + 4], dvo[e + 5]);
+          pkd.w = pack_bf16(dvo[e + 6], dvo[e + 7]);
+          *reinterpret_cast<uint4*>(dvp + e) = pkd;
+          *reinterpret_cast<float4*>(dgp + e) = make_float4(dgo[e], dgo[e + 1], dgo[e + 2], dgo[e + 3]);
+          *reinterpret_cast<float4*>(dgp + e + 4) =
+              make_float4(dgo[e + 4], dgo[e + 5], dgo[e + 6], dgo[e + 7]);
+        }
+      }
+    }
+#pragma unroll
+    for (int cc = 0; cc < DK / 32; ++cc) {
+      uint32_t x[32];
+      tmem_ld32(lane_base + kColK + cc * 32, x);
+      tmem_wait_ld();
+      if (row_ok) {
+        __nv_bfloat16* dkp = P.dk + tok * krs + (size_t)kv * DK + cc * 32;
+#pragma unroll
+        for (int e = 0; e < 32; e += 8) {
+          uint4 pkd;
+          pkd.x = pack_bf16(__uint_as_float(x[e]) * d.scale, __uint_as_float(x[e + 1]) * d.scale);
+          pkd.y = pack_bf16(__uint_as_float(x[e + 2]) * d.scale, __uint_as_float(x[e + 3]) * d.scale);
+          pkd.z = pack_bf16(__uint_as_float(x[e + 4]) * d.scale, __uint_as_float(x[e + 5]) * d.scale);
+          pkd.w = pack_bf16(__uint_as_float(x[e + 6]) * d.scale, __uint_as_float(x[e + 7]) * d.scale);
+          *reinterpret_cast<uint4*>(dkp + e) = pkd;
+        }
+      }
+    }
+  } else if (warp >= 8) {
+    // ------------------------------------------------------------ X operand tiles
+    const int dt = tid - 256;
+    constexpr int kChunks = DV / 8;
+    constexpr int kRowsPerPass = 128 / kChunks;
+    const int lc = dt % kChunks, r0 = dt / kChunks;
+    const size_t ors = (size_t)d.Hq * DV;
+    // Vt arrives in its chunk's storage type; the off-diagonal MMAs read it in
+    // the CTA's type, so convert it once if they differ
+    if (!mbar_wait(&bar->kv_full, 0, ctl)) {
+      // aborted: fall through to the teardown
+    } else {
+      const bool vt_f16 = P.safe[(size_t)cj * d.Hkv + kv] != 0;
+      if (vt_f16 != (cta_f16 != 0)) {
+        for (int rr = r0; rr < BN; rr += kRowsPerPass) {
+          uint4* p = reinterpret_cast<uint4*>(sVt + sw_off(BN, rr, lc * 8));
+          float x[8];
+          unpack8(*p, vt_f16, x);
+          *p = pack8(x, cta_f16 != 0);
+        }
+        fence_proxy_async_smem();
+      }
+      // the MMA warp waited for kv_full before this conversion may have
+      // finished; the first x_ready below orders it (it covers this thread's
+      // writes and every X tile depends on it)
+      TileIter t{0, ch.j, 0};
+      float delta[8];
+      int cur_h = -1;
+      for (int n = 0; n < ntiles; ++n, next_tile(t)) {
+        const int st = n & 1;
+        const bool diag = t.i == ch.j;
+        const int h = kv * d.grp + t.hh;
+        if (t.hh != cur_h) {
+          cur_h = t.hh;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) delta[e] = 0.f;
+        }
+        if (t.half == 0 && t.i >= ch.j + 2) {
+          const float* tp = P.tot + ((size_t)(first + t.i - 1) * d.Hkv + kv) * DV + lc * 8;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) delta[e] += tp[e];
+        }
+        float f8[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) f8[e] = ex2(delta[e] * LOG2E);
+        if (n >= 2 && !mbar_wait(&bar->x_empty[st], ((n >> 1) & 1) ^ 1, ctl)) break;
+        const Chunk qc = P.chunks[first + t.i];
+        const int qlen = min(BQ, qc.len - t.half * BQ);
+        uint8_t* xb = sX + st * BQ * DV * 2;
+        uint8_t* xlb = sXl + st * BQ * DV * 2;
+        for (int rr = r0; rr < BQ; rr += kRowsPerPass) {
+          float x[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+          const size_t qtok = (size_t)qc.tok0 + t.half * BQ + rr;
+          if (rr < qlen) {
+            const float* p = (diag ? P.dom_ws : P.dot_ws) + qtok * ors + (size_t)h * DV + lc * 8;
+            const float4 a = *reinterpret_cast<const float4*>(p);
+            const float4 b = *reinterpret_cast<const float4*>(p + 4);
+            x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+            x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+          }
+          const uint32_t off = sw_off(BQ, rr, lc * 8);
+          if (diag) {
+            const uint4 hi = pack8(x, false);
+            float xh[8];
+            unpack8(hi, false, xh);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) xh[e] = x[e] - xh[e];
+            *reinterpret_cast<uint4*>(xb + off) = hi;
+            *reinterpret_cast<uint4*>(xlb + off) = pack8(xh, false);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) x[e] *= f8[e];
+            *reinterpret_cast<uint4*>(xb + off) = pack8(x, cta_f16 != 0);
+          }
+        }
+        if (dt < BQ) {
+          const size_t qtok = (size_t)qc.tok0 + t.half * BQ + dt;
+          sM[st * BQ + dt] = dt < qlen ? P.m_s[qtok * d.Hq + h] : 0.f;
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&bar->x_ready[st]);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;  // cached driver entry point
+  if (!fn) {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+static bool make_map(CUtensorMap* m, const void* base, int D, int H, int N, int rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)N};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
+  cuuint32_t box[3] = {64, 1, (cuuint32_t)rows};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int DK, int DV>
+static fix_status launch(const Params& prm, const void* vt, const void* vm, int which,
+                         cudaStream_t st) {
+  const Dims& d = prm.d;
+  CUtensorMap mq, mk, mvt, mvm;
+  if (!make_map(&mq, prm.q, DK, d.Hq, d.N, which == 0 ? 128 : BQ) ||
+      !make_map(&mk, prm.k, DK, d.Hkv, d.N, 128) || !make_map(&mvt, vt, DV, d.Hkv, d.N, 128) ||
+      !make_map(&mvm, vm, DV, d.Hkv, d.N, 128))
+    return FIX_ERR_CUDA;
+  if (which == 0) {
+    const int smem = DqLayout<DK, DV>::kAlloc;
+    auto kern = dq_tc_kernel<DK, DV>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return FIX_ERR_CUDA;
+    kern<<<(unsigned)((long long)d.nchunks * d.Hq), kThreads, smem, st>>>(mq, mk, mvt, mvm, prm);
+  } else {
+    const int smem = KvLayout<DK, DV>::kAlloc;
+    auto kern = dkv_tc_kernel<DK, DV>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return FIX_ERR_CUDA;
+    kern<<<(unsigned)((long long)d.nchunks * d.Hkv), kThreads, smem, st>>>(mq, mk, mvt, mvm, prm);
+  }
+  return cudaGetLastError() == cudaSuccess ? FIX_OK : FIX_ERR_CUDA;
+}
+
+}  // namespace tcb
+
+bool tc_bwd_supported(const Dims& d) {
+  const bool dims_ok = (d.Dk == 64 || d.Dk == 128) && (d.Dv == 64 || d.Dv == 128);
+  return dims_ok && d.N >= FIX_CHUNK && d.grp <= 16;
+}
+
+int tc_bwd_kernel_count(const Dims&) { return 2; }
+
+fix_status tc_bwd(const fix_attn_problem*, const Dims& d, const TcBwdArgs& a, int which,
+                  cudaStream_t st) {
+  tcb::Params prm{};
+  prm.d = d;
+  prm.chunks = a.chunks;
+  prm.order = a.order;
+  prm.q = static_cast<const __nv_bfloat16*>(a.q);
+  prm.k = static_cast<const __nv_bfloat16*>(a.k);
+  prm.v = static_cast<const __nv_bfloat16*>(a.v);
+  prm.L = a.L;
+  prm.tot = a.tot;
+  prm.rho = a.rho;
+  prm.hr = a.hr;
+  prm.safe = a.safe;
+  prm.dsafe = a.dsafe;
+  prm.m_s = a.m_s;
+  prm.do_ws = a.do_ws;
+  prm.dot_ws = a.dot_ws;
+  prm.dom_ws = a.dom_ws;
+  prm.A = a.A;
+  prm.badflag = a.badflag;
+  prm.dq = static_cast<__nv_bfloat16*>(a.dq);
+  prm.dk = static_cast<__nv_bfloat16*>(a.dk);
+  prm.dv = static_cast<__nv_bfloat16*>(a.dv);
+  prm.dG = a.dG;
+  prm.status = a.status;
+  if (d.Dk == 128 && d.Dv == 128) return tcb::launch<128, 128>(prm, a.vt, a.vm, which, st);
+  if (d.Dk == 64 && d.Dv == 64) return tcb::launch<64, 64>(prm, a.vt, a.vm, which, st);
+  if (d.Dk == 128 && d.Dv == 64) return tcb::launch<128, 64>(prm, a.vt, a.vm, which, st);
+  if (d.Dk == 64 && d.Dv == 128) return tcb::launch<64, 128>(prm, a.vt, a.vm, which, st);
+  return FIX_ERR_HEAD_DIM;
+}
+
+}  // namespace fix
