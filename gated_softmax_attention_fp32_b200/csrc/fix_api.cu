@@ -75,14 +75,61 @@ static int max_chunks_per_seq(const fix_attn_problem* p) {
   return (int)m;
 }
 
+// Work split of the dk/dv kernel: each key chunk's tiles (q heads x 64-row
+// query tiles of the chunks from it to the end of its sequence) are cut into
+// runs of at most P tiles, P chosen so that about two runs per SM cover the
+// problem.  Planned with the B200's 148 SMs whatever the device: the split
+// only affects load balance, and the plan must not depend on a device query
+// so that the workspace size agrees between sizing and calling.
+struct SplitPlan {
+  int P = 0;
+  long long nparts = 0, nslots = 0;
+};
+
+static int tiles64_host(long long L, int j) {
+  return (int)((L - (long long)j * FIX_CHUNK + 63) / 64);
+}
+
+static SplitPlan plan_split(const fix_attn_problem* p, const Dims& d) {
+  SplitPlan sp;
+  auto each_seq = [&](auto fn) {
+    if (p->cu_seqlens) {
+      for (int i = 0; i < p->num_seqs; ++i) fn(p->cu_seqlens_host[i + 1] - p->cu_seqlens_host[i], 1);
+    } else {
+      fn((long long)p->seqlen, (long long)p->batch);
+    }
+  };
+  long long total = 0;
+  each_seq([&](long long L, long long mult) {
+    const int nc = (int)((L + FIX_CHUNK - 1) / FIX_CHUNK);
+    for (int j = 0; j < nc; ++j) total += mult * d.grp * tiles64_host(L, j);
+  });
+  total *= d.Hkv;
+  constexpr int kSMs = 148;
+  long long P = (total + 2 * kSMs - 1) / (2 * kSMs);
+  if (P < 4) P = 4;
+  if (P > (1 << 30)) P = 1 << 30;
+  sp.P = (int)P;
+  each_seq([&](long long L, long long mult) {
+    const int nc = (int)((L + FIX_CHUNK - 1) / FIX_CHUNK);
+    for (int j = 0; j < nc; ++j) {
+      const long long npj = ((long long)d.grp * tiles64_host(L, j) + P - 1) / P;
+      sp.nparts += mult * npj;
+      if (npj > 1) sp.nslots += mult * npj;
+    }
+  });
+  return sp;
+}
+
 // Workspace layout (all offsets 256-byte aligned).
 struct Ws {
   size_t status, chunks, order, safe, L, vt, vm, vml, tot, rho, hr;   // forward and backward
-  size_t dow, dot, dom, dsafe, A, dG, dtot, dwp;           // backward only
+  size_t dow, dot, domh, doml, dsafe, A, dG, dtot, dwp;    // backward only
+  size_t parts, cpart, partial;                            // dk/dv work split
   size_t total;
 };
 
-static Ws layout(const Dims& d, bool bwd) {
+static Ws layout(const Dims& d, bool bwd, const SplitPlan& sp) {
   Ws w{};
   size_t o = 0;
   auto take = [&](size_t bytes) {
@@ -105,13 +152,17 @@ static Ws layout(const Dims& d, bool bwd) {
   w.hr = take(nch * 4);
   if (bwd) {
     w.dow = take((size_t)d.N * d.Hq * d.Dv * 4);
-    w.dot = take((size_t)d.N * d.Hq * d.Dv * 4);
-    w.dom = take((size_t)d.N * d.Hq * d.Dv * 4);
+    w.dot = take((size_t)d.N * d.Hq * d.Dv * 2);
+    w.domh = take((size_t)d.N * d.Hq * d.Dv * 2);
+    w.doml = take((size_t)d.N * d.Hq * d.Dv * 2);
     w.dsafe = take((size_t)(d.nchunks > 0 ? d.nchunks : 1) * d.Hq * sizeof(int));
     w.A = take(nkv * 4);
     w.dG = take(nkv * 4);
     w.dtot = take(nch * 4);
     w.dwp = take((size_t)(d.nchunks > 0 ? d.nchunks : 1) * d.Hkv * d.Dv * 4);
+    w.parts = take((size_t)(sp.nparts > 0 ? sp.nparts : 1) * sizeof(Part));
+    w.cpart = take((size_t)(d.nchunks > 0 ? d.nchunks : 1) * sizeof(int2));
+    w.partial = take((size_t)sp.nslots * d.Hkv * FIX_CHUNK * (d.Dk + 2 * d.Dv) * 4);
   }
   w.total = o;
   return w;
@@ -157,11 +208,20 @@ static size_t simt_dkv_smem(const Dims& d) {
 
 // Prefix pass + schedule (both directions).
 static fix_status run_prefix(const Dims& d, const fix_attn_problem* p, const Ws& ws, char* base,
-                             const float* g, const void* v, bool want_vt, cudaStream_t st) {
+                             const float* g, const void* v, bool want_vt, const SplitPlan* sp,
+                             cudaStream_t st) {
   Chunk* chunks = reinterpret_cast<Chunk*>(base + ws.chunks);
+  PartSpec ps{};
+  if (sp) {
+    ps.grp = d.grp;
+    ps.tiles_per_part = sp->P;
+    ps.cap_parts = (int)sp->nparts;
+    ps.parts = reinterpret_cast<Part*>(base + ws.parts);
+    ps.cpart = reinterpret_cast<int2*>(base + ws.cpart);
+  }
   schedule_kernel<<<1, 1024, 0, st>>>(p->cu_seqlens, d.nseq, d.T, d.N, d.nchunks, chunks,
                                       max_chunks_per_seq(p),
-                                      want_vt ? reinterpret_cast<int*>(base + ws.order) : nullptr);
+                                      want_vt ? reinterpret_cast<int*>(base + ws.order) : nullptr, ps);
   FIX_TRY(launched());
   if (d.nchunks == 0) return FIX_OK;
   prefix_kernel<<<dim3(d.nchunks, d.Hkv), 512, 0, st>>>(
@@ -183,7 +243,7 @@ extern "C" {
 size_t fix_attn_workspace_bytes(const fix_attn_problem* p, int backward) {
   Dims d;
   if (make_dims(p, &d) != FIX_OK) return 0;
-  return layout(d, backward != 0).total;
+  return layout(d, backward != 0, backward ? plan_split(p, d) : SplitPlan{}).total;
 }
 
 const char* fix_attn_status_string(int s) {
@@ -215,7 +275,7 @@ fix_status fix_attn_fwd(const fix_attn_problem* p, const void* q, const void* k,
   for (const void* ptr : {q, k, v, (const void*)g, w, (const void*)y, (const void*)workspace})
     if (!aligned16(ptr)) return FIX_ERR_ALIGN;
   if (nsaved && (!aligned16(o_s) || !aligned16(m_s) || !aligned16(rstd_s))) return FIX_ERR_ALIGN;
-  const Ws ws = layout(d, false);
+  const Ws ws = layout(d, false, SplitPlan{});
   if (ws_bytes < ws.total) return FIX_ERR_WORKSPACE;
   FIX_TRY(check_device());
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -225,7 +285,7 @@ fix_status fix_attn_fwd(const fix_attn_problem* p, const void* q, const void* k,
   if (d.N == 0) return FIX_OK;
   const bool tc = p->algo != FIX_ALGO_SIMT && tc_fwd_supported(d);
   FIX_TRY(mark(p, FIX_STAGE_FWD_PREFIX, 0, st));
-  FIX_TRY(run_prefix(d, p, ws, base, g, v, tc, st));
+  FIX_TRY(run_prefix(d, p, ws, base, g, v, tc, nullptr, st));
   FIX_TRY(mark(p, FIX_STAGE_FWD_PREFIX, 1, st));
   const Chunk* chunks = reinterpret_cast<const Chunk*>(base + ws.chunks);
   const float* L = reinterpret_cast<const float*>(base + ws.L);
@@ -267,7 +327,8 @@ fix_status fix_attn_bwd(const fix_attn_problem* p, const void* q, const void* k,
                           (const void*)rstd_s, (const void*)dq, (const void*)dk, (const void*)dv,
                           (const void*)dg, (const void*)dw, (const void*)workspace})
     if (!aligned16(ptr)) return FIX_ERR_ALIGN;
-  const Ws ws = layout(d, true);
+  const SplitPlan sp = plan_split(p, d);
+  const Ws ws = layout(d, true, sp);
   if (ws_bytes < ws.total) return FIX_ERR_WORKSPACE;
   FIX_TRY(check_device());
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -279,14 +340,15 @@ fix_status fix_attn_bwd(const fix_attn_problem* p, const void* q, const void* k,
   }
   const bool tc = p->algo != FIX_ALGO_SIMT && tc_bwd_supported(d);
   FIX_TRY(mark(p, FIX_STAGE_BWD_PREFIX, 0, st));
-  FIX_TRY(run_prefix(d, p, ws, base, g, v, tc, st));
+  FIX_TRY(run_prefix(d, p, ws, base, g, v, tc, tc ? &sp : nullptr, st));
   FIX_TRY(mark(p, FIX_STAGE_BWD_PREFIX, 1, st));
   const Chunk* chunks = reinterpret_cast<const Chunk*>(base + ws.chunks);
   const float* L = reinterpret_cast<const float*>(base + ws.L);
   const float* tot = reinterpret_cast<const float*>(base + ws.tot);
   float* dow = reinterpret_cast<float*>(base + ws.dow);
-  float* dot = reinterpret_cast<float*>(base + ws.dot);
-  float* dom = reinterpret_cast<float*>(base + ws.dom);
+  uint16_t* dot = reinterpret_cast<uint16_t*>(base + ws.dot);
+  __nv_bfloat16* domh = reinterpret_cast<__nv_bfloat16*>(base + ws.domh);
+  __nv_bfloat16* doml = reinterpret_cast<__nv_bfloat16*>(base + ws.doml);
   int* dsafe = reinterpret_cast<int*>(base + ws.dsafe);
   float* A = reinterpret_cast<float*>(base + ws.A);
   float* dG = reinterpret_cast<float*>(base + ws.dG);
@@ -297,11 +359,11 @@ fix_status fix_attn_bwd(const fix_attn_problem* p, const void* q, const void* k,
   const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(k);
   const __nv_bfloat16* vb = static_cast<const __nv_bfloat16*>(v);
   FIX_TRY(mark(p, FIX_STAGE_BWD_PRE, 0, st));
-  bwd_pre_kernel<<<dim3(d.nchunks, d.Hkv), 128, d.grp * sizeof(float), st>>>(
+  bwd_pre_kernel<<<dim3(d.nchunks, d.Hkv), 512, d.grp * sizeof(float), st>>>(
       d, chunks, qb, kb, vb, o_s, m_s, rstd_s, static_cast<const __nv_bfloat16*>(dy),
       static_cast<const __nv_bfloat16*>(w), L, reinterpret_cast<const float*>(base + ws.rho),
-      reinterpret_cast<const float*>(base + ws.hr), dow, tc ? dot : nullptr, tc ? dom : nullptr,
-      dsafe, A, dwp);
+      reinterpret_cast<const float*>(base + ws.hr), reinterpret_cast<const int*>(base + ws.safe),
+      dow, tc ? dot : nullptr, domh, doml, dsafe, A, dwp);
   FIX_TRY(launched());
   dw_reduce_kernel<<<1, 128, 0, st>>>(dwp, d.nchunks * d.Hkv, d.Dv, static_cast<__nv_bfloat16*>(dw));
   FIX_TRY(launched());
@@ -323,10 +385,17 @@ fix_status fix_attn_bwd(const fix_attn_problem* p, const void* q, const void* k,
     ta.dsafe = dsafe;
     ta.m_s = m_s;
     ta.do_ws = dow;
-    ta.dot_ws = dot;
-    ta.dom_ws = dom;
+    ta.dot = dot;
+    ta.domh = domh;
+    ta.doml = doml;
     ta.A = A;
     ta.badflag = badflag;
+    ta.parts = reinterpret_cast<const Part*>(base + ws.parts);
+    ta.cpart = reinterpret_cast<const int2*>(base + ws.cpart);
+    ta.tiles_per_part = sp.P;
+    ta.nparts = sp.nparts;
+    ta.nslots = sp.nslots;
+    ta.partial = reinterpret_cast<float*>(base + ws.partial);
     ta.dq = dq;
     ta.dk = dk;
     ta.dv = dv;
@@ -372,7 +441,7 @@ int fix_attn_kernel_count(const fix_attn_problem* p, int backward) {
     return 2 + (tc ? tc_fwd_kernel_count(d) : 1);
   }
   const bool tc = p->algo != FIX_ALGO_SIMT && tc_bwd_supported(d);
-  return 2 + 2 + (tc ? tc_bwd_kernel_count(d) : 0) + 2 + 2;
+  return 2 + 2 + (tc ? tc_bwd_kernel_count(d, plan_split(p, d).nslots) : 0) + 2 + 2;
 }
 
 fix_status fix_attn_device_status(const void* workspace, void* stream) {

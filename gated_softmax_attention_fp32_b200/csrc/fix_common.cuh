@@ -35,6 +35,25 @@ struct Chunk {
   int nch;
 };
 
+// One CTA's share of a key chunk's backward work: the key chunk, the index p
+// of its run of (at most `tiles_per_part`) 64-row query tiles, and the slot of
+// its partial sums (-1 when the chunk is done by a single CTA).
+struct Part {
+  int ci;
+  int p;
+  int slot;
+  int pad;
+};
+
+// Where the schedule kernel writes the dk/dv work split (parts == NULL: none).
+struct PartSpec {
+  int grp;            // q heads per kv head
+  int tiles_per_part; // P
+  int cap_parts;      // entries of parts[]
+  Part* parts;
+  int2* cpart;        // per chunk: {number of parts, first slot or -1}
+};
+
 struct Dims {
   int N;          // total tokens
   int B, T;       // dense batch / length (T = N when packed)

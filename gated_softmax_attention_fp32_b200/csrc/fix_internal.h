@@ -9,7 +9,7 @@ constexpr int ST_ROWS = 32;  // rows per CTA of the exact (SIMT) kernels
 
 // fix_prefix.cu
 __global__ void schedule_kernel(const int64_t* cu, int nseq, int T, int N, int cap, Chunk* out,
-                                int maxj, int* order);
+                                int maxj, int* order, PartSpec ps);
 __global__ void prefix_kernel(Dims d, const Chunk* chunks, const float* g, const __nv_bfloat16* v,
                               float* L, uint16_t* vt, __nv_bfloat16* vm, __nv_bfloat16* vml,
                               float* tot, float* rho, float* hr, int* safe, int* badflag);
@@ -26,8 +26,9 @@ __global__ void bwd_pre_kernel(Dims d, const Chunk* chunks, const __nv_bfloat16*
                                const __nv_bfloat16* k, const __nv_bfloat16* v, const float* o_s,
                                const float* m_s, const float* rstd_s, const __nv_bfloat16* dy,
                                const __nv_bfloat16* w, const float* L, const float* rho,
-                               const float* hr, float* do_ws, float* dot_ws, float* dom_ws,
-                               int* dsafe, float* A, float* dwpart);
+                               const float* hr, const int* safe, float* do_ws, uint16_t* dot,
+                               __nv_bfloat16* domh, __nv_bfloat16* doml, int* dsafe, float* A,
+                               float* dwpart);
 __global__ void dw_reduce_kernel(const float* parts, int nparts, int Dv, __nv_bfloat16* dw);
 __global__ void dq_simt_kernel(Dims d, const Chunk* chunks, const __nv_bfloat16* q,
                                const __nv_bfloat16* k, const __nv_bfloat16* v, const float* L,
@@ -50,7 +51,7 @@ fix_status tc_fwd(const Dims& d, const Chunk* chunks, const int* order, const vo
                   int* status, cudaStream_t st);
 int tc_fwd_kernel_count(const Dims& d);
 bool tc_bwd_supported(const Dims& d);
-int tc_bwd_kernel_count(const Dims& d);
+int tc_bwd_kernel_count(const Dims& d, long long nslots);
 
 // Device buffers of one backward call for the tensor-core kernels.
 struct TcBwdArgs {
@@ -69,10 +70,17 @@ struct TcBwdArgs {
   const int* dsafe;
   const float* m_s;
   const float* do_ws;
-  const float* dot_ws;
-  const float* dom_ws;
+  const uint16_t* dot;
+  const __nv_bfloat16* domh;
+  const __nv_bfloat16* doml;
   const float* A;
   const int* badflag;
+  const Part* parts;
+  const int2* cpart;
+  int tiles_per_part;
+  long long nparts;
+  long long nslots;
+  float* partial;
   void* dq;
   void* dk;
   void* dv;

@@ -50,10 +50,32 @@ __device__ void order_chunks(const Chunk* __restrict__ chunks, int nchunks, int 
 // every entry is first set empty, writes past `cap` are dropped and lengths
 // are clamped to the N tokens, so a device array that disagrees with the host
 // mirror cannot send any kernel outside its buffers.
+// Exclusive prefix sum over the 1024 threads of a CTA; *total gets the sum.
+__device__ int block_excl_scan(int v, int* scan, int* total) {
+  scan[threadIdx.x] = v;
+  __syncthreads();
+  for (int off = 1; off < (int)blockDim.x; off <<= 1) {
+    const int add = threadIdx.x >= (unsigned)off ? scan[threadIdx.x - off] : 0;
+    __syncthreads();
+    scan[threadIdx.x] += add;
+    __syncthreads();
+  }
+  const int incl = scan[threadIdx.x];
+  *total = scan[blockDim.x - 1];
+  __syncthreads();
+  return incl - v;
+}
+
+// Number of 64-row query tiles from chunk j to the end of a sequence of L
+// tokens (every chunk but the last is a whole number of tiles).
+__device__ __host__ inline int tiles64_from(int L, int j) {
+  return (L - j * FIX_CHUNK + 63) / 64;
+}
+
 __global__ void __launch_bounds__(1024) schedule_kernel(const int64_t* __restrict__ cu, int nseq,
                                                         int T, int N, int cap,
                                                         Chunk* __restrict__ out, int maxj,
-                                                        int* __restrict__ order) {
+                                                        int* __restrict__ order, PartSpec ps) {
   __shared__ int scan[1024];
   for (int i = threadIdx.x; i < cap; i += blockDim.x) out[i] = Chunk{0, 0, 0, 0};
   __syncthreads();
@@ -100,6 +122,47 @@ __global__ void __launch_bounds__(1024) schedule_kernel(const int64_t* __restric
     __threadfence_block();
     __syncthreads();
     order_chunks(out, cap, maxj, order);
+  }
+  if (!ps.parts) return;
+  // dk/dv work split: key chunk j of a sequence has grp * tiles64_from(L, j)
+  // tiles, cut into ceil(tiles / P) parts
+  int cbase = 0, pbase = 0, sbase = 0;
+  for (int first = 0; first < nseq; first += blockDim.x) {
+    const int i = first + threadIdx.x;
+    int L = 0;
+    if (i < nseq) {
+      if (cu) {
+        long long s0 = cu[i];
+        const long long e = cu[i + 1];
+        s0 = s0 < 0 ? 0 : (s0 > N ? N : s0);
+        L = (int)((e > N ? N : e) - s0);
+        if (L < 0) L = 0;
+      } else {
+        L = T;
+      }
+    }
+    const int nc = (L + FIX_CHUNK - 1) / FIX_CHUNK;
+    int np = 0, ns = 0;
+    for (int j = 0; j < nc; ++j) {
+      const int npj = (ps.grp * tiles64_from(L, j) + ps.tiles_per_part - 1) / ps.tiles_per_part;
+      np += npj;
+      if (npj > 1) ns += npj;
+    }
+    int ctot, ptot, stot;
+    const int c0 = cbase + block_excl_scan(nc, scan, &ctot);
+    const int p0 = pbase + block_excl_scan(np, scan, &ptot);
+    int s0 = sbase + block_excl_scan(ns, scan, &stot);
+    int e = p0;
+    for (int j = 0; j < nc && c0 + j < cap; ++j) {
+      const int npj = (ps.grp * tiles64_from(L, j) + ps.tiles_per_part - 1) / ps.tiles_per_part;
+      ps.cpart[c0 + j] = make_int2(npj, npj > 1 ? s0 : -1);
+      for (int p = 0; p < npj && e < ps.cap_parts; ++p, ++e)
+        ps.parts[e] = Part{c0 + j, p, npj > 1 ? s0 + p : -1, 0};
+      if (npj > 1) s0 += npj;
+    }
+    cbase += ctot;
+    pbase += ptot;
+    sbase += stot;
   }
 }
 

@@ -153,7 +153,7 @@ __global__ void __launch_bounds__(256) fwd_simt_kernel(
 
 // ---------------------------------------------------------------------------
 // Backward preprocess (shared by all kernel families), one CTA per (chunk, kv
-// head), 4 warps, a warp per row at a time over the kv group's q heads:
+// head), 16 warps, a warp per row at a time over the kv group's q heads:
 //   RMSNorm backward   n = o rstd,  dn = dy w,  do = rstd (dn - n mean(dn n))
 //   A_t[c]  = sum_{h in group} do_t[c] (o_t[c] - P_tt v_t[c])
 //             the row part of dG_t without the s = t pair, whose counterpart
@@ -161,50 +161,51 @@ __global__ void __launch_bounds__(256) fwd_simt_kernel(
 //             dG = A - v dv_strict carries no cancelling diagonal terms
 //             (P_tt = exp(S_tt - m_t), S_tt recomputed from q_t, k_t)
 //   dw partials        sum_t dy_t n_t per CTA
-// and, for the tensor-core kernels (dot != NULL), the row-scaled upstream
-// gradients in the two references of the forward split:
-//   dOt_t = do_t exp(L_t)          (key blocks before the query chunk)
+// and, for the tensor-core kernels (dot != NULL), a second pass writing the
+// row-scaled upstream gradients in the two references of the forward split,
+// as 16-bit MMA operands:
+//   dOt_t = do_t exp(L_t)          (key blocks before the query chunk): fp16
+//                                  when dsafe, else bf16
 //   dOm_t = do_t exp(L_t - rho)    (the diagonal block; 0 for channels outside
-//                                   the split's range)
-// plus dsafe[ci * Hq + h] = (max |do| over the chunk <= FIX_F16_VMAX).
+//                                  the split's range): bf16 hi + lo
+// with dsafe[ci * Hq + h] = (the chunk is fp16-safe and max |do| <= FIX_F16_VMAX).
 // Dynamic shared memory: grp floats.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(128) bwd_pre_kernel(
+constexpr int kPreWarps = 16;
+
+__global__ void __launch_bounds__(kPreWarps * 32) bwd_pre_kernel(
     Dims d, const Chunk* __restrict__ chunks, const __nv_bfloat16* __restrict__ q,
     const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
     const float* __restrict__ o_s, const float* __restrict__ m_s,
     const float* __restrict__ rstd_s, const __nv_bfloat16* __restrict__ dy,
     const __nv_bfloat16* __restrict__ w, const float* __restrict__ L,
-    const float* __restrict__ rho, const float* __restrict__ hr, float* __restrict__ do_ws,
-    float* __restrict__ dot_ws, float* __restrict__ dom_ws, int* __restrict__ dsafe,
-    float* __restrict__ A, float* __restrict__ dwpart) {
-  __shared__ float red[4][128];
+    const float* __restrict__ rho, const float* __restrict__ hr, const int* __restrict__ safe,
+    float* __restrict__ do_ws, uint16_t* __restrict__ dot, __nv_bfloat16* __restrict__ domh,
+    __nv_bfloat16* __restrict__ doml, int* __restrict__ dsafe, float* __restrict__ A,
+    float* __restrict__ dwpart) {
+  __shared__ float red[kPreWarps][128];
   extern __shared__ float hmax[];   // [grp] max |do| per head
   const int Dv = d.Dv, Dk = d.Dk, kv = blockIdx.y, ci = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const Chunk ch = chunks[ci];
   for (int i = threadIdx.x; i < d.grp; i += blockDim.x) hmax[i] = 0.f;
   __syncthreads();
-  float wv[4], dwl[4], rh[4], good[4];
+  float wv[4], dwl[4];
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
     const int c = lane + 32 * u;
     wv[u] = c < Dv ? bf2f(w[c]) : 0.f;
     dwl[u] = 0.f;
-    const size_t ti = ((size_t)ci * d.Hkv + kv) * Dv + c;
-    rh[u] = (dot_ws && c < Dv) ? rho[ti] : 0.f;
-    good[u] = (dot_ws && c < Dv) ? (hr[ti] <= FIX_HR_MAX ? 1.f : 0.f) : 0.f;
   }
   const size_t ors = (size_t)d.Hq * Dv, vrs = (size_t)d.Hkv * Dv;
   const size_t qrs = (size_t)d.Hq * Dk, krs = (size_t)d.Hkv * Dk;
-  for (int r = warp; r < ch.len; r += 4) {
+  for (int r = warp; r < ch.len; r += kPreWarps) {
     const size_t t = (size_t)ch.tok0 + r;
-    float acc[4] = {0.f, 0.f, 0.f, 0.f}, vr[4], lr[4], kr[4];
+    float acc[4] = {0.f, 0.f, 0.f, 0.f}, vr[4], kr[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int c = lane + 32 * u;
       vr[u] = c < Dv ? bf2f(v[t * vrs + (size_t)kv * Dv + c]) : 0.f;
-      lr[u] = (dot_ws && c < Dv) ? L[t * vrs + (size_t)kv * Dv + c] : 0.f;
       kr[u] = c < Dk ? bf2f(k[t * krs + (size_t)kv * Dk + c]) : 0.f;
     }
     for (int hh = 0; hh < d.grp; ++hh) {
@@ -217,7 +218,7 @@ __global__ void __launch_bounds__(128) bwd_pre_kernel(
         if (c < Dk) sdot += bf2f(q[t * qrs + (size_t)h * Dk + c]) * kr[u];
       }
       const float ptt = expf(warp_sum(sdot) * d.scale - m_s[t * d.Hq + h]);
-      float ov[4], dn[4], n[4], dot = 0.f;
+      float ov[4], dn[4], n[4], dot_ = 0.f;
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int c = lane + 32 * u;
@@ -226,26 +227,21 @@ __global__ void __launch_bounds__(128) bwd_pre_kernel(
         const float dyv = c < Dv ? bf2f(dy[a]) : 0.f;
         n[u] = ov[u] * rs_;
         dn[u] = dyv * wv[u];
-        dot += dn[u] * n[u];
+        dot_ += dn[u] * n[u];
         dwl[u] += dyv * n[u];
       }
-      dot = warp_sum(dot) / (float)Dv;
+      dot_ = warp_sum(dot_) / (float)Dv;
       float mx = 0.f;
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int c = lane + 32 * u;
         if (c >= Dv) continue;
-        const float dov = rs_ * (dn[u] - n[u] * dot);
-        const size_t a = t * ors + (size_t)h * Dv + c;
-        do_ws[a] = dov;
+        const float dov = rs_ * (dn[u] - n[u] * dot_);
+        do_ws[t * ors + (size_t)h * Dv + c] = dov;
         acc[u] += dov * (ov[u] - ptt * vr[u]);
-        if (dot_ws) {
-          dot_ws[a] = dov * expf(lr[u]);
-          dom_ws[a] = good[u] != 0.f ? dov * expf(lr[u] - rh[u]) : 0.f;
-          mx = fmaxf(mx, fabsf(dov));
-        }
+        mx = fmaxf(mx, fabsf(dov));
       }
-      if (dot_ws) {
+      if (dot) {
         mx = warp_max(mx);
         if (lane == 0) atomicMax(reinterpret_cast<int*>(&hmax[hh]), __float_as_int(mx));
       }
@@ -259,14 +255,52 @@ __global__ void __launch_bounds__(128) bwd_pre_kernel(
 #pragma unroll
   for (int u = 0; u < 4; ++u) red[warp][lane + 32 * u] = dwl[u];
   __syncthreads();
-  const int c = threadIdx.x;
-  if (c < Dv) {
-    const float sm = red[0][c] + red[1][c] + red[2][c] + red[3][c];
-    dwpart[((size_t)ci * d.Hkv + kv) * Dv + c] = sm;
+  const int c0 = threadIdx.x;
+  if (c0 < Dv) {
+    float sm = 0.f;
+#pragma unroll
+    for (int i = 0; i < kPreWarps; ++i) sm += red[i][c0];
+    dwpart[((size_t)ci * d.Hkv + kv) * Dv + c0] = sm;
   }
-  if (dot_ws)
-    for (int i = threadIdx.x; i < d.grp; i += blockDim.x)
-      dsafe[(size_t)ci * d.Hq + kv * d.grp + i] = hmax[i] <= FIX_F16_VMAX ? 1 : 0;
+  if (!dot) return;
+  // ---- second pass: 16-bit operands of the tensor-core kernels
+  const bool chunk_safe = safe[(size_t)ci * d.Hkv + kv] != 0;
+  for (int i = threadIdx.x; i < d.grp; i += blockDim.x)
+    dsafe[(size_t)ci * d.Hq + kv * d.grp + i] = (chunk_safe && hmax[i] <= FIX_F16_VMAX) ? 1 : 0;
+  float rh[4], good[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int c = lane + 32 * u;
+    const size_t ti = ((size_t)ci * d.Hkv + kv) * Dv + c;
+    rh[u] = c < Dv ? rho[ti] : 0.f;
+    good[u] = (c < Dv && hr[ti] <= FIX_HR_MAX) ? 1.f : 0.f;
+  }
+  for (int r = warp; r < ch.len; r += kPreWarps) {
+    const size_t t = (size_t)ch.tok0 + r;
+    float lr[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int c = lane + 32 * u;
+      lr[u] = c < Dv ? L[t * vrs + (size_t)kv * Dv + c] : 0.f;
+    }
+    for (int hh = 0; hh < d.grp; ++hh) {
+      const int h = kv * d.grp + hh;
+      const bool f16 = chunk_safe && hmax[hh] <= FIX_F16_VMAX;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int c = lane + 32 * u;
+        if (c >= Dv) continue;
+        const size_t a = t * ors + (size_t)h * Dv + c;
+        const float dov = do_ws[a];
+        const float xt = dov * expf(lr[u]);
+        dot[a] = f16 ? __half_as_ushort(__float2half_rn(xt)) : __bfloat16_as_ushort(f2bf(xt));
+        const float xm = good[u] != 0.f ? dov * expf(lr[u] - rh[u]) : 0.f;
+        const __nv_bfloat16 hi = f2bf(xm);
+        domh[a] = hi;
+        doml[a] = f2bf(xm - bf2f(hi));
+      }
+    }
+  }
 }
 
 // dw = sum of the partials in a fixed order (deterministic).  One CTA.

@@ -60,10 +60,16 @@ struct Params {
   const int* dsafe;
   const float* m_s;
   const float* do_ws;
-  const float* dot_ws;
-  const float* dom_ws;
+  const uint16_t* dot;      // do exp(L_t), fp16 where dsafe else bf16
+  const __nv_bfloat16* domh;  // do exp(L_t - rho), hi and lo bf16 parts
+  const __nv_bfloat16* doml;
   const float* A;
   const int* badflag;
+  const Part* parts;        // dk/dv work split (schedule kernel)
+  const int2* cpart;
+  int tiles_per_part;
+  long long nslots;         // rows of `partial` per kv head, in units of 128-row slots
+  float* partial;           // partial dK | dV_d | dV_o rows of split key chunks
   __nv_bfloat16* dq;
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
@@ -107,7 +113,7 @@ __device__ __forceinline__ void unpack8(uint4 u, bool f16, float* x) {
 // =========================================================================== dq
 
 struct DqBars {
-  uint64_t q_full, o_ready;
+  uint64_t q_full, o_full, o_ready;
   uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2], v_ready[2];
   uint64_t s_full, ds_ready, dp0_done, done, drain;
 };
@@ -128,6 +134,7 @@ template <int DK, int DV>
 __global__ void __launch_bounds__(kThreads, 1)
     dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_vt, const __grid_constant__ CUtensorMap tm_vm,
+                 const __grid_constant__ CUtensorMap tm_domh, const __grid_constant__ CUtensorMap tm_dot,
                  const Params P) {
   using Lay = DqLayout<DK, DV>;
   if (*P.badflag) return;  // exact kernels run instead
@@ -154,6 +161,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid == 0) {
     *sAbort = 0;
     mbar_init(&bar->q_full, 1);
+    mbar_init(&bar->o_full, 1);
     mbar_init(&bar->o_ready, 128);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bar->k_full[s], 1);
@@ -186,7 +194,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_expect_tx(&bar->q_full, BN * DK * 2);
       for (int hh = 0; hh < DK / 64; ++hh)
         tma_load_3d(sQ + hh * BN * 64, &tm_q, &bar->q_full, hh * 64, h, ch.tok0);
-      int nk = 0, nv = 0;
+      // dO operand: dOm (diagonal block) first, dOt once the first dP is done
+      mbar_expect_tx(&bar->o_full, BN * DV * 2);
+      for (int hh = 0; hh < DV / 64; ++hh)
+        tma_load_3d(sO + hh * BN * 128, &tm_domh, &bar->o_full, hh * 64, h, ch.tok0);
+      int nk = 0, nv = 0, no = 1;
       for (int it = 0; it < nblk; ++it) {
         const int st = it & 1;
         const uint32_t ph = (it >> 1) & 1;
@@ -202,6 +214,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int hh = 0; hh < DV / 64; ++hh)
           tma_load_3d(sV + st * BN * DV + hh * BN * 64, vmap, &bar->v_full[st], hh * 64, kv, ktok);
         ++nv;
+        if (it == 1) {
+          if (!mbar_wait(&bar->dp0_done, 0, ctl)) break;
+          mbar_expect_tx(&bar->o_full, BN * DV * 2);
+          for (int hh = 0; hh < DV / 64; ++hh)
+            tma_load_3d(sO + hh * BN * 128, &tm_dot, &bar->o_full, hh * 64, h, ch.tok0);
+          ++no;
+        }
       }
       const Ctl drain{P.status, nullptr};
       for (int it = nk - 1; it >= 0 && it >= nk - 2; --it)
@@ -209,6 +228,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int it = nv - 1; it >= 0 && it >= nv - 2; --it)
         mbar_wait(&bar->v_full[it & 1], (it >> 1) & 1, drain);
       mbar_wait(&bar->q_full, 0, drain);
+      mbar_wait(&bar->o_full, (no - 1) & 1, drain);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -272,13 +292,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(lane_base + kColS + c4 * 32, xs);
         tmem_ld32(lane_base + kColP + c4 * 32, xp);
         tmem_wait_ld();
+        // rows past the chunk's end only feed dQ rows that are never stored;
+        // only the diagonal block needs the causal mask (keys s <= t)
+        if (it > 0) {
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const int key = c4 * 32 + e;
-          const bool v0 = row_ok && (it > 0 || key <= r), v1 = row_ok && (it > 0 || key + 1 <= r);
-          const float p0 = v0 ? ex2(__uint_as_float(xs[e]) * c1 - moff) : 0.f;
-          const float p1 = v1 ? ex2(__uint_as_float(xs[e + 1]) * c1 - moff) : 0.f;
-          pk[e >> 1] = pack_bf16(p0 * __uint_as_float(xp[e]), p1 * __uint_as_float(xp[e + 1]));
+          for (int e = 0; e < 32; e += 2) {
+            const float p0 = ex2(__uint_as_float(xs[e]) * c1 - moff);
+            const float p1 = ex2(__uint_as_float(xs[e + 1]) * c1 - moff);
+            pk[e >> 1] = pack_bf16(p0 * __uint_as_float(xp[e]), p1 * __uint_as_float(xp[e + 1]));
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const int key = c4 * 32 + e;
+            const float p0 = key <= r ? ex2(__uint_as_float(xs[e]) * c1 - moff) : 0.f;
+            const float p1 = key + 1 <= r ? ex2(__uint_as_float(xs[e + 1]) * c1 - moff) : 0.f;
+            pk[e >> 1] = pack_bf16(p0 * __uint_as_float(xp[e]), p1 * __uint_as_float(xp[e + 1]));
+          }
         }
         tmem_st16(lane_base + kColS + c4 * 16, pk);
       }
@@ -316,23 +346,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int kRowsPerPass = 128 / kChunks;
     const int lc = dt % kChunks, r0 = dt / kChunks;
     const size_t ors = (size_t)d.Hq * DV;
-    // dO operand: dOm (bf16) for the diagonal block, then dOt (CTA format)
+    // dO operand (loaded by TMA): dOm (bf16) for the diagonal block, then dOt,
+    // converted in place when its storage type differs from the CTA's
     for (int phase = 0; phase < (nblk > 1 ? 2 : 1); ++phase) {
-      if (phase == 1 && !mbar_wait(&bar->dp0_done, 0, ctl)) break;
-      const float* src = phase == 0 ? P.dom_ws : P.dot_ws;
-      const bool f16 = phase == 1 && cta_f16;
-      for (int rr = r0; rr < BN; rr += kRowsPerPass) {
-        float x[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        if (rr < ch.len) {
-          const float* p = src + ((size_t)ch.tok0 + rr) * ors + (size_t)h * DV + lc * 8;
-          const float4 a = *reinterpret_cast<const float4*>(p);
-          const float4 b = *reinterpret_cast<const float4*>(p + 4);
-          x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
-          x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+      if (!mbar_wait(&bar->o_full, phase, ctl)) break;
+      if (phase == 1) {
+        const bool stored_f16 = P.dsafe[(size_t)ci * d.Hq + h] != 0;
+        if (stored_f16 != (cta_f16 != 0)) {
+          for (int rr = r0; rr < BN; rr += kRowsPerPass) {
+            uint4* p = reinterpret_cast<uint4*>(sO + sw_off(BN, rr, lc * 8));
+            float x[8];
+            unpack8(*p, stored_f16, x);
+            *p = pack8(x, cta_f16 != 0);
+          }
+          fence_proxy_async_smem();
         }
-        *reinterpret_cast<uint4*>(sO + sw_off(BN, rr, lc * 8)) = pack8(x, f16);
       }
-      fence_proxy_async_smem();
       mbar_arrive(&bar->o_ready);
       if (phase == 0) {
         // the diagonal block's V (Vm) goes to the MMA as loaded
@@ -382,9 +411,85 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 constexpr int BQ = 64;   // query rows per streamed tile
 
+// P_ss = exp(S_ss - m_s) of the group's q heads for key row `tok` (the s = t
+// pair, which dv_strict leaves out).
+template <int DK>
+__device__ void row_pss(const Params& P, int kv, size_t tok, float* pss, int ng) {
+  const Dims& d = P.d;
+  const __nv_bfloat16* krow = P.k + tok * (size_t)d.Hkv * DK + (size_t)kv * DK;
+  for (int hh = 0; hh < ng; ++hh) {
+    const int h = kv * d.grp + hh;
+    const __nv_bfloat16* qrow = P.q + tok * (size_t)d.Hq * DK + (size_t)h * DK;
+    float acc = 0.f;
+    for (int dd = 0; dd < DK; dd += 8) {
+      float a8[8], b8[8];
+      unpack8(*reinterpret_cast<const uint4*>(qrow + dd), false, a8);
+      unpack8(*reinterpret_cast<const uint4*>(krow + dd), false, b8);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc += a8[e] * b8[e];
+    }
+    pss[hh] = ex2((acc * d.scale - P.m_s[tok * d.Hq + h]) * LOG2E);
+  }
+}
+
+// dv and dG for 32 channels [32 cc, 32 cc + 32) of key row `tok` of key chunk
+// cj, from the two accumulators (diagonal reference rho, chunk-end reference):
+//   dv_strict = exp(rho - L_s) dV_d + exp(tot - L_s) dV_o
+//   dv = dv_strict + sum_h P_ss do_s,   dG = A - v dv_strict
+template <int DV>
+__device__ void finish_dv32(const Params& P, int cj, int kv, size_t tok, int cc, const float* dvd,
+                            const float* dvo, bool has_off, const float* pss, int ng) {
+  const Dims& d = P.d;
+  const size_t vrs = (size_t)d.Hkv * DV, ors = (size_t)d.Hq * DV;
+  const float* Lrow = P.L + tok * vrs + (size_t)kv * DV;
+  const float* trow = P.tot + ((size_t)cj * d.Hkv + kv) * DV;
+  const float* rrow = P.rho + ((size_t)cj * d.Hkv + kv) * DV;
+  float dvv[32], dgv[32];
+#pragma unroll
+  for (int e = 0; e < 32; ++e) {
+    const int c = cc * 32 + e;
+    const float ls = Lrow[c];
+    float strict = dvd[e] * ex2((rrow[c] - ls) * LOG2E);
+    if (has_off) strict += dvo[e] * ex2((trow[c] - ls) * LOG2E);
+    float diagsum = 0.f;
+    for (int hh = 0; hh < ng; ++hh)
+      diagsum += pss[hh] * P.do_ws[tok * ors + (size_t)(kv * d.grp + hh) * DV + c];
+    dvv[e] = strict + diagsum;
+    dgv[e] = P.A[tok * vrs + (size_t)kv * DV + c] - bf2f(P.v[tok * vrs + (size_t)kv * DV + c]) * strict;
+  }
+  __nv_bfloat16* dvp = P.dv + tok * vrs + (size_t)kv * DV + cc * 32;
+  float* dgp = P.dG + tok * vrs + (size_t)kv * DV + cc * 32;
+#pragma unroll
+  for (int e = 0; e < 32; e += 8) {
+    uint4 pkd;
+    pkd.x = pack_bf16(dvv[e], dvv[e + 1]);
+    pkd.y = pack_bf16(dvv[e + 2], dvv[e + 3]);
+    pkd.z = pack_bf16(dvv[e + 4], dvv[e + 5]);
+    pkd.w = pack_bf16(dvv[e + 6], dvv[e + 7]);
+    *reinterpret_cast<uint4*>(dvp + e) = pkd;
+    *reinterpret_cast<float4*>(dgp + e) = make_float4(dgv[e], dgv[e + 1], dgv[e + 2], dgv[e + 3]);
+    *reinterpret_cast<float4*>(dgp + e + 4) = make_float4(dgv[e + 4], dgv[e + 5], dgv[e + 6], dgv[e + 7]);
+  }
+}
+
+template <int DK>
+__device__ void finish_dk32(const Params& P, int kv, size_t tok, int cc, const float* acc) {
+  const Dims& d = P.d;
+  __nv_bfloat16* dkp = P.dk + tok * (size_t)d.Hkv * DK + (size_t)kv * DK + cc * 32;
+#pragma unroll
+  for (int e = 0; e < 32; e += 8) {
+    uint4 pkd;
+    pkd.x = pack_bf16(acc[e] * d.scale, acc[e + 1] * d.scale);
+    pkd.y = pack_bf16(acc[e + 2] * d.scale, acc[e + 3] * d.scale);
+    pkd.z = pack_bf16(acc[e + 4] * d.scale, acc[e + 5] * d.scale);
+    pkd.w = pack_bf16(acc[e + 6] * d.scale, acc[e + 7] * d.scale);
+    *reinterpret_cast<uint4*>(dkp + e) = pkd;
+  }
+}
+
 struct KvBars {
   uint64_t kv_full;
-  uint64_t q_full[2], q_empty[2], x_ready[2], x_empty[2];
+  uint64_t q_full[2], q_empty[2], x_ready[2];
   uint64_t s_full, p_ready, done, drain;
 };
 
@@ -413,7 +518,8 @@ template <int DK, int DV>
 __global__ void __launch_bounds__(kThreads, 1)
     dkv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_vt, const __grid_constant__ CUtensorMap tm_vm,
-                  const Params P) {
+                  const __grid_constant__ CUtensorMap tm_domh, const __grid_constant__ CUtensorMap tm_doml,
+                  const __grid_constant__ CUtensorMap tm_dot, const Params P) {
   using Lay = KvLayout<DK, DV>;
   if (*P.badflag) return;
   extern __shared__ uint8_t smem_raw[];
@@ -421,8 +527,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              ~static_cast<uintptr_t>(1023));
   const Dims& d = P.d;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int cj = P.order[P.d.nchunks - 1 - blockIdx.x / d.Hkv];   // short rows last -> long first
+  const Part pt = P.parts[blockIdx.x / d.Hkv];
   const int kv = blockIdx.x % d.Hkv;
+  const int cj = pt.ci;
   const Chunk ch = P.chunks[cj];
   if (ch.len <= 0) return;
   const int first = cj - ch.j;
@@ -431,7 +538,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto chunk_len = [&](int i) { return P.chunks[first + i].len; };
   int tiles_per_head = 0;
   for (int i = ch.j; i < ch.nch; ++i) tiles_per_head += (chunk_len(i) + BQ - 1) / BQ;
-  const int ntiles = tiles_per_head * d.grp;
+  // this CTA's run of tiles
+  const int t_begin = pt.p * P.tiles_per_part;
+  const int ntiles = min(P.tiles_per_part, tiles_per_head * d.grp - t_begin);
+  if (ntiles <= 0) return;
 
   uint8_t* sK = smem + Lay::kK;
   uint8_t* sVt = smem + Lay::kVt;
@@ -452,7 +562,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bar->q_full[s], 1);
       mbar_init(&bar->q_empty[s], 1);
       mbar_init(&bar->x_ready[s], 128);
-      mbar_init(&bar->x_empty[s], 1);
     }
     mbar_init(&bar->s_full, 1);
     mbar_init(&bar->p_ready, 128);
@@ -485,6 +594,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   };
+  auto tile_at = [&](int n) {
+    TileIter t{0, ch.j, 0};
+    for (int q = 0; q < n; ++q) next_tile(t);
+    return t;
+  };
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -496,16 +610,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_3d(sVt + hh * BN * 128, &tm_vt, &bar->kv_full, hh * 64, kv, ch.tok0);
         tma_load_3d(sVm + hh * BN * 128, &tm_vm, &bar->kv_full, hh * 64, kv, ch.tok0);
       }
-      TileIter t{0, ch.j, 0};
+      TileIter t = tile_at(t_begin);
       int nq = 0;
       for (int n = 0; n < ntiles; ++n, next_tile(t)) {
         const int st = n & 1;
+        const bool diag = t.i == ch.j;
         if (n >= 2 && !mbar_wait(&bar->q_empty[st], ((n >> 1) & 1) ^ 1, ctl)) break;
-        mbar_expect_tx(&bar->q_full[st], BQ * DK * 2);
+        // Q tile and the X operand (dOm hi + lo on the diagonal, dOt elsewhere)
+        mbar_expect_tx(&bar->q_full[st], BQ * DK * 2 + (diag ? 2 : 1) * BQ * DV * 2);
         const int h = kv * d.grp + t.hh;
         const int qtok = P.chunks[first + t.i].tok0 + t.half * BQ;
         for (int hh = 0; hh < DK / 64; ++hh)
           tma_load_3d(sQ + st * BQ * DK * 2 + hh * BQ * 128, &tm_q, &bar->q_full[st], hh * 64, h, qtok);
+        for (int hh = 0; hh < DV / 64; ++hh) {
+          tma_load_3d(sX + st * BQ * DV * 2 + hh * BQ * 128, diag ? &tm_domh : &tm_dot,
+                      &bar->q_full[st], hh * 64, h, qtok);
+          if (diag)
+            tma_load_3d(sXl + st * BQ * DV * 2 + hh * BQ * 128, &tm_doml, &bar->q_full[st], hh * 64,
+                        h, qtok);
+        }
         ++nq;
       }
       const Ctl drain{P.status, nullptr};
@@ -525,7 +648,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t k_addr = smem_u32(sK), vt_addr = smem_u32(sVt), vm_addr = smem_u32(sVm);
       bool ok = mbar_wait(&bar->kv_full, 0, ctl);
       bool first_diag = true, first_off = true;
-      TileIter t{0, ch.j, 0};
+      TileIter t = tile_at(t_begin);
       for (int n = 0; ok && n < ntiles; ++n, next_tile(t)) {
         const int st = n & 1;
         const uint32_t ph = (n >> 1) & 1;
@@ -577,7 +700,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (diag) first_diag = false;
         else first_off = false;
         tc_commit(&bar->q_empty[st]);
-        tc_commit(&bar->x_empty[st]);
       }
       tc_commit(&bar->done);
       tc_commit(&bar->drain);
@@ -589,47 +711,63 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_base = tmem + ((uint32_t)((warp - 4) * 32) << 16);
     const float c1 = d.scale * LOG2E;
     bool ok = true;
-    TileIter t{0, ch.j, 0};
+    TileIter t = tile_at(t_begin);
     for (int n = 0; n < ntiles; ++n, next_tile(t)) {
       const int st = n & 1;
       const bool diag = t.i == ch.j;
       const int qlen = min(BQ, chunk_len(t.i) - t.half * BQ);
       if (!__all_sync(0xffffffffu, mbar_wait(&bar->s_full, n & 1, ctl))) { ok = false; break; }
       tc_fence_after();
-      uint32_t xs[64], xp[64];
-      tmem_ld32(lane_base + kColS, *reinterpret_cast<uint32_t(*)[32]>(&xs[0]));
-      tmem_ld32(lane_base + kColS + 32, *reinterpret_cast<uint32_t(*)[32]>(&xs[32]));
-      tmem_ld32(lane_base + kColP, *reinterpret_cast<uint32_t(*)[32]>(&xp[0]));
-      tmem_ld32(lane_base + kColP + 32, *reinterpret_cast<uint32_t(*)[32]>(&xp[32]));
-      tmem_wait_ld();
       const float* mrow = sM + st * BQ;
-      uint32_t ph[32], pl[32], pd[32];
+      const bool full = !diag && qlen == BQ;
+      const int lo = diag ? s - t.half * BQ : 0;   // first valid query column
+      // two halves of 32 query columns; a half's packed P and dS go over
+      // columns of S and dP that the half has already read
+      uint32_t pl[32];
 #pragma unroll
-      for (int e = 0; e < BQ; e += 2) {
-        float p[2], pv[2], ds[2];
+      for (int h = 0; h < 2; ++h) {
+        uint32_t xs[32], xp[32], ph[16], pd[16];
+        tmem_ld32(lane_base + kColS + 32 * h, xs);
+        tmem_ld32(lane_base + kColP + 32 * h, xp);
+        tmem_wait_ld();
+        if (full) {
+          // full off-diagonal tile: no masking
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int qi = e + u;
-          const int tpos = t.half * BQ + qi;          // query row in chunk i
-          const bool valid = qi < qlen && (!diag || tpos >= s);
-          p[u] = valid ? ex2(__uint_as_float(xs[qi]) * c1 - mrow[qi] * LOG2E) : 0.f;
-          pv[u] = (diag && tpos == s) ? 0.f : p[u];   // dv leaves out the s = t pair
-          ds[u] = p[u] * __uint_as_float(xp[qi]);
-        }
-        if (diag) {
-          ph[e >> 1] = pack_bf16(pv[0], pv[1]);
-          const float h0 = __uint_as_float(ph[e >> 1] << 16);
-          const float h1 = __uint_as_float(ph[e >> 1] & 0xFFFF0000u);
-          pl[e >> 1] = pack_bf16(pv[0] - h0, pv[1] - h1);
+          for (int e = 0; e < 32; e += 2) {
+            const float p0 = ex2(__uint_as_float(xs[e]) * c1 - mrow[32 * h + e] * LOG2E);
+            const float p1 = ex2(__uint_as_float(xs[e + 1]) * c1 - mrow[32 * h + e + 1] * LOG2E);
+            ph[e >> 1] = cta_f16 ? pack_f16(p0, p1) : pack_bf16(p0, p1);
+            pd[e >> 1] = pack_bf16(p0 * __uint_as_float(xp[e]), p1 * __uint_as_float(xp[e + 1]));
+          }
         } else {
-          ph[e >> 1] = cta_f16 ? pack_f16(pv[0], pv[1]) : pack_bf16(pv[0], pv[1]);
-          pl[e >> 1] = 0u;
+          // diagonal tile (queries t >= s; the s = t pair stays out of dv) or
+          // a partial tile (columns past the chunk's end)
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            float p[2], pv[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const int qi = 32 * h + e + u;
+              const bool valid = qi >= lo && qi < qlen;
+              p[u] = valid ? ex2(__uint_as_float(xs[e + u]) * c1 - mrow[qi] * LOG2E) : 0.f;
+              pv[u] = (diag && qi == lo) ? 0.f : p[u];
+            }
+            if (diag) {
+              ph[e >> 1] = pack_bf16(pv[0], pv[1]);
+              const float h0 = __uint_as_float(ph[e >> 1] << 16);
+              const float h1 = __uint_as_float(ph[e >> 1] & 0xFFFF0000u);
+              pl[16 * h + (e >> 1)] = pack_bf16(pv[0] - h0, pv[1] - h1);
+            } else {
+              ph[e >> 1] = cta_f16 ? pack_f16(pv[0], pv[1]) : pack_bf16(pv[0], pv[1]);
+            }
+            pd[e >> 1] = pack_bf16(p[0] * __uint_as_float(xp[e]), p[1] * __uint_as_float(xp[e + 1]));
+          }
         }
-        pd[e >> 1] = pack_bf16(ds[0], ds[1]);
+        tmem_st16(lane_base + kColS + 16 * h, ph);
+        tmem_st16(lane_base + kColP + 16 * h, pd);
       }
-      tmem_st32(lane_base + kColS, ph);
+      // the low parts go over S columns [32, 64), read by the second half
       if (diag) tmem_st32(lane_base + kColS + 32, pl);
-      tmem_st32(lane_base + kColP, pd);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bar->p_ready);
@@ -639,80 +777,83 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------- epilogue
     const bool row_ok = ok && s < ch.len;
     const size_t tok = (size_t)ch.tok0 + (size_t)(s < ch.len ? s : 0);
-    const size_t vrs = (size_t)d.Hkv * DV, krs = (size_t)d.Hkv * DK, qrs = (size_t)d.Hq * DK;
-    const size_t ors = (size_t)d.Hq * DV;
-    const bool has_off = ch.nch - ch.j > 1;
-    const float* Lrow = P.L + tok * vrs + (size_t)kv * DV;
-    const float* trow = P.tot + ((size_t)cj * d.Hkv + kv) * DV;
-    const float* rrow = P.rho + ((size_t)cj * d.Hkv + kv) * DV;
-    // P_ss of every q head of the group (the s = t pair left out of dv_strict)
-    float pss[16];
-    const int ng = min(d.grp, 16);
-    const __nv_bfloat16* krow = P.k + tok * krs + (size_t)kv * DK;
-    for (int hh = 0; hh < ng; ++hh) {
-      const int h = kv * d.grp + hh;
-      const __nv_bfloat16* qrow = P.q + tok * qrs + (size_t)h * DK;
-      float acc = 0.f;
-      for (int dd = 0; dd < DK; dd += 8) {
-        float a8[8], b8[8];
-        unpack8(*reinterpret_cast<const uint4*>(qrow + dd), false, a8);
-        unpack8(*reinterpret_cast<const uint4*>(krow + dd), false, b8);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc += a8[e] * b8[e];
-      }
-      pss[hh] = ex2((acc * d.scale - P.m_s[tok * d.Hq + h]) * LOG2E);
-    }
-#pragma unroll
-    for (int cc = 0; cc < DV / 32; ++cc) {
-      uint32_t xd[32], xo[32];
-      tmem_ld32(lane_base + kColVd + cc * 32, xd);
-      tmem_ld32(lane_base + kColVo + cc * 32, xo);
-      tmem_wait_ld();
-      if (row_ok) {
-        float dvo[32], dgo[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int c = cc * 32 + e;
-          const float ls = Lrow[c];
-          float strict = __uint_as_float(xd[e]) * ex2((rrow[c] - ls) * LOG2E);
-          if (has_off) strict += __uint_as_float(xo[e]) * ex2((trow[c] - ls) * LOG2E);
-          float diagsum = 0.f;
-          for (int hh = 0; hh < ng; ++hh)
-            diagsum += pss[hh] * P.do_ws[tok * ors + (size_t)(kv * d.grp + hh) * DV + c];
-          dvo[e] = strict + diagsum;
-          dgo[e] = P.A[tok * vrs + (size_t)kv * DV + c] - bf2f(P.v[tok * vrs + (size_t)kv * DV + c]) * strict;
-        }
-        __nv_bfloat16* dvp = P.dv + tok * vrs + (size_t)kv * DV + cc * 32;
-        float* dgp = P.dG + tok * vrs + (size_t)kv * DV + cc * 32;
-#pragma unroll
-        for (int e = 0; e < 32; e += 8) {
-          uint4 pkd;
-          pkd.x = pack_bf16(dvo[e], dvo[e + 1]);
-          pkd.y = pack_bf16(dvo[e + 2], dvo[e + 3]);
-          pkd.z = pack_bf16(dvo[e + 4], dvo[e + 5]);
-          pkd.w = pack_bf16(dvo[e + 6], dvo[e + 7]);
-          *reinterpret_cast<uint4*>(dvp + e) = pkd;
-          *reinterpret_cast<float4*>(dgp + e) = make_float4(dgo[e], dgo[e + 1], dgo[e + 2], dgo[e + 3]);
-          *reinterpret_cast<float4*>(dgp + e + 4) =
-              make_float4(dgo[e + 4], dgo[e + 5], dgo[e + 6], dgo[e + 7]);
-        }
+    // which accumulators this CTA's tiles wrote
+    bool has_diag = false, has_off = false;
+    {
+      TileIter u = tile_at(t_begin);
+      for (int n = 0; n < ntiles; ++n, next_tile(u)) {
+        if (u.i == ch.j) has_diag = true;
+        else has_off = true;
       }
     }
+    if (pt.slot < 0) {
+      // the whole key chunk was this CTA's: finish dv, dG, dk here
+      float pss[16];
+      const int ng = min(d.grp, 16);
+      if (row_ok) row_pss<DK>(P, kv, tok, pss, ng);
 #pragma unroll
-    for (int cc = 0; cc < DK / 32; ++cc) {
-      uint32_t x[32];
-      tmem_ld32(lane_base + kColK + cc * 32, x);
-      tmem_wait_ld();
-      if (row_ok) {
-        __nv_bfloat16* dkp = P.dk + tok * krs + (size_t)kv * DK + cc * 32;
+      for (int cc = 0; cc < DV / 32; ++cc) {
+        uint32_t xd[32], xo[32];
+        tmem_ld32(lane_base + kColVd + cc * 32, xd);
+        tmem_ld32(lane_base + kColVo + cc * 32, xo);
+        tmem_wait_ld();
+        if (row_ok) {
+          float fd[32], fo[32];
 #pragma unroll
-        for (int e = 0; e < 32; e += 8) {
-          uint4 pkd;
-          pkd.x = pack_bf16(__uint_as_float(x[e]) * d.scale, __uint_as_float(x[e + 1]) * d.scale);
-          pkd.y = pack_bf16(__uint_as_float(x[e + 2]) * d.scale, __uint_as_float(x[e + 3]) * d.scale);
-          pkd.z = pack_bf16(__uint_as_float(x[e + 4]) * d.scale, __uint_as_float(x[e + 5]) * d.scale);
-          pkd.w = pack_bf16(__uint_as_float(x[e + 6]) * d.scale, __uint_as_float(x[e + 7]) * d.scale);
-          *reinterpret_cast<uint4*>(dkp + e) = pkd;
+          for (int e = 0; e < 32; ++e) {
+            fd[e] = __uint_as_float(xd[e]);
+            fo[e] = has_off ? __uint_as_float(xo[e]) : 0.f;
+          }
+          finish_dv32<DV>(P, cj, kv, tok, cc, fd, fo, has_off, pss, ng);
+        }
+      }
+#pragma unroll
+      for (int cc = 0; cc < DK / 32; ++cc) {
+        uint32_t x[32];
+        tmem_ld32(lane_base + kColK + cc * 32, x);
+        tmem_wait_ld();
+        if (row_ok) {
+          float fk[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) fk[e] = __uint_as_float(x[e]);
+          finish_dk32<DK>(P, kv, tok, cc, fk);
+        }
+      }
+    } else if (pt.slot < P.nslots) {
+      // one of several CTAs of this key chunk: raw partial sums, summed by
+      // the combine kernel in slot order
+      constexpr int kCols = DK + 2 * DV;
+      float* prow = P.partial + (((size_t)pt.slot * d.Hkv + kv) * BN + s) * kCols;
+#pragma unroll
+      for (int cc = 0; cc < DK / 32; ++cc) {
+        uint32_t x[32];
+        tmem_ld32(lane_base + kColK + cc * 32, x);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; e += 4)
+          *reinterpret_cast<float4*>(prow + cc * 32 + e) =
+              make_float4(__uint_as_float(x[e]), __uint_as_float(x[e + 1]),
+                          __uint_as_float(x[e + 2]), __uint_as_float(x[e + 3]));
+      }
+#pragma unroll
+      for (int cc = 0; cc < DV / 32; ++cc) {
+        uint32_t xd[32], xo[32];
+        tmem_ld32(lane_base + kColVd + cc * 32, xd);
+        tmem_ld32(lane_base + kColVo + cc * 32, xo);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; e += 4) {
+          float4 a, b;
+          a.x = has_diag ? __uint_as_float(xd[e]) : 0.f;
+          a.y = has_diag ? __uint_as_float(xd[e + 1]) : 0.f;
+          a.z = has_diag ? __uint_as_float(xd[e + 2]) : 0.f;
+          a.w = has_diag ? __uint_as_float(xd[e + 3]) : 0.f;
+          b.x = has_off ? __uint_as_float(xo[e]) : 0.f;
+          b.y = has_off ? __uint_as_float(xo[e + 1]) : 0.f;
+          b.z = has_off ? __uint_as_float(xo[e + 2]) : 0.f;
+          b.w = has_off ? __uint_as_float(xo[e + 3]) : 0.f;
+          *reinterpret_cast<float4*>(prow + DK + cc * 32 + e) = a;
+          *reinterpret_cast<float4*>(prow + DK + DV + cc * 32 + e) = b;
         }
       }
     }
@@ -741,55 +882,45 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the MMA warp waited for kv_full before this conversion may have
       // finished; the first x_ready below orders it (it covers this thread's
       // writes and every X tile depends on it)
-      TileIter t{0, ch.j, 0};
+      TileIter t = tile_at(t_begin);
       float delta[8];
-      int cur_h = -1;
+      int cur_h = -1, upto = 0;
       for (int n = 0; n < ntiles; ++n, next_tile(t)) {
         const int st = n & 1;
         const bool diag = t.i == ch.j;
         const int h = kv * d.grp + t.hh;
+        // f_ij = exp(sum_{j<j'<i} tot_j'): running sum over the query chunks of
+        // one head (they only increase within a head)
         if (t.hh != cur_h) {
-          cur_h = t.hh;
 #pragma unroll
           for (int e = 0; e < 8; ++e) delta[e] = 0.f;
+          upto = ch.j + 1;
+          cur_h = t.hh;
         }
-        if (t.half == 0 && t.i >= ch.j + 2) {
-          const float* tp = P.tot + ((size_t)(first + t.i - 1) * d.Hkv + kv) * DV + lc * 8;
+        for (; upto < t.i; ++upto) {
+          const float* tp = P.tot + ((size_t)(first + upto) * d.Hkv + kv) * DV + lc * 8;
 #pragma unroll
           for (int e = 0; e < 8; ++e) delta[e] += tp[e];
         }
         float f8[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) f8[e] = ex2(delta[e] * LOG2E);
-        if (n >= 2 && !mbar_wait(&bar->x_empty[st], ((n >> 1) & 1) ^ 1, ctl)) break;
+        if (!mbar_wait(&bar->q_full[st], (n >> 1) & 1, ctl)) break;
         const Chunk qc = P.chunks[first + t.i];
         const int qlen = min(BQ, qc.len - t.half * BQ);
-        uint8_t* xb = sX + st * BQ * DV * 2;
-        uint8_t* xlb = sXl + st * BQ * DV * 2;
-        for (int rr = r0; rr < BQ; rr += kRowsPerPass) {
-          float x[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-          const size_t qtok = (size_t)qc.tok0 + t.half * BQ + rr;
-          if (rr < qlen) {
-            const float* p = (diag ? P.dom_ws : P.dot_ws) + qtok * ors + (size_t)h * DV + lc * 8;
-            const float4 a = *reinterpret_cast<const float4*>(p);
-            const float4 b = *reinterpret_cast<const float4*>(p + 4);
-            x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
-            x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
-          }
-          const uint32_t off = sw_off(BQ, rr, lc * 8);
-          if (diag) {
-            const uint4 hi = pack8(x, false);
-            float xh[8];
-            unpack8(hi, false, xh);
+        if (!diag) {
+          // X = dOt f_ij, in the CTA's operand type
+          const bool in_f16 = P.dsafe[(size_t)(first + t.i) * d.Hq + h] != 0;
+          uint8_t* xb = sX + st * BQ * DV * 2;
+          for (int rr = r0; rr < BQ; rr += kRowsPerPass) {
+            uint4* p = reinterpret_cast<uint4*>(xb + sw_off(BQ, rr, lc * 8));
+            float x[8];
+            unpack8(*p, in_f16, x);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) xh[e] = x[e] - xh[e];
-            *reinterpret_cast<uint4*>(xb + off) = hi;
-            *reinterpret_cast<uint4*>(xlb + off) = pack8(xh, false);
-          } else {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) x[e] *= f8[e];
-            *reinterpret_cast<uint4*>(xb + off) = pack8(x, cta_f16 != 0);
+            for (int e = 0; e < 8; ++e) x[e] = rr < qlen ? x[e] * f8[e] : 0.f;
+            *p = pack8(x, cta_f16 != 0);
           }
+          fence_proxy_async_smem();
         }
         if (dt < BQ) {
           const size_t qtok = (size_t)qc.tok0 + t.half * BQ + dt;
@@ -806,6 +937,58 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// Sums the partial rows of key chunks split over several CTAs (in slot
+// order, so the result does not depend on scheduling) and finishes dv, dG,
+// dk.  grid (nchunks, Hkv), block 128: thread = key row.
+template <int DK, int DV>
+__global__ void __launch_bounds__(128) dkv_combine_kernel(const Params P) {
+  if (*P.badflag) return;
+  const Dims& d = P.d;
+  const int ci = blockIdx.x, kv = blockIdx.y, s = threadIdx.x;
+  const int2 cp = P.cpart[ci];
+  if (cp.x <= 1 || cp.y < 0 || cp.y + cp.x > P.nslots) return;
+  const Chunk ch = P.chunks[ci];
+  if (s >= ch.len) return;
+  const size_t tok = (size_t)ch.tok0 + s;
+  constexpr int kCols = DK + 2 * DV;
+  const bool has_off = ch.nch - ch.j > 1;
+  float pss[16];
+  const int ng = min(d.grp, 16);
+  row_pss<DK>(P, kv, tok, pss, ng);
+#pragma unroll 1
+  for (int cc = 0; cc < DV / 32; ++cc) {
+    float fd[32], fo[32];
+#pragma unroll
+    for (int e = 0; e < 32; ++e) fd[e] = fo[e] = 0.f;
+    for (int q = 0; q < cp.x; ++q) {
+      const float* prow = P.partial + (((size_t)(cp.y + q) * d.Hkv + kv) * BN + s) * kCols;
+#pragma unroll
+      for (int e = 0; e < 32; e += 4) {
+        const float4 a = *reinterpret_cast<const float4*>(prow + DK + cc * 32 + e);
+        const float4 b = *reinterpret_cast<const float4*>(prow + DK + DV + cc * 32 + e);
+        fd[e] += a.x; fd[e + 1] += a.y; fd[e + 2] += a.z; fd[e + 3] += a.w;
+        fo[e] += b.x; fo[e + 1] += b.y; fo[e + 2] += b.z; fo[e + 3] += b.w;
+      }
+    }
+    finish_dv32<DV>(P, ci, kv, tok, cc, fd, fo, has_off, pss, ng);
+  }
+#pragma unroll 1
+  for (int cc = 0; cc < DK / 32; ++cc) {
+    float fk[32];
+#pragma unroll
+    for (int e = 0; e < 32; ++e) fk[e] = 0.f;
+    for (int q = 0; q < cp.x; ++q) {
+      const float* prow = P.partial + (((size_t)(cp.y + q) * d.Hkv + kv) * BN + s) * kCols;
+#pragma unroll
+      for (int e = 0; e < 32; e += 4) {
+        const float4 a = *reinterpret_cast<const float4*>(prow + cc * 32 + e);
+        fk[e] += a.x; fk[e + 1] += a.y; fk[e + 2] += a.z; fk[e + 3] += a.w;
+      }
+    }
+    finish_dk32<DK>(P, kv, tok, cc, fk);
   }
 }
 
@@ -838,25 +1021,31 @@ static bool make_map(CUtensorMap* m, const void* base, int D, int H, int N, int 
 
 template <int DK, int DV>
 static fix_status launch(const Params& prm, const void* vt, const void* vm, int which,
-                         cudaStream_t st) {
+                         long long nparts, long long nslots, cudaStream_t st) {
   const Dims& d = prm.d;
-  CUtensorMap mq, mk, mvt, mvm;
-  if (!make_map(&mq, prm.q, DK, d.Hq, d.N, which == 0 ? 128 : BQ) ||
+  const int rows = which == 0 ? 128 : BQ;
+  CUtensorMap mq, mk, mvt, mvm, mdomh, mdoml, mdot;
+  if (!make_map(&mq, prm.q, DK, d.Hq, d.N, rows) ||
       !make_map(&mk, prm.k, DK, d.Hkv, d.N, 128) || !make_map(&mvt, vt, DV, d.Hkv, d.N, 128) ||
-      !make_map(&mvm, vm, DV, d.Hkv, d.N, 128))
+      !make_map(&mvm, vm, DV, d.Hkv, d.N, 128) || !make_map(&mdomh, prm.domh, DV, d.Hq, d.N, rows) ||
+      !make_map(&mdoml, prm.doml, DV, d.Hq, d.N, rows) || !make_map(&mdot, prm.dot, DV, d.Hq, d.N, rows))
     return FIX_ERR_CUDA;
   if (which == 0) {
     const int smem = DqLayout<DK, DV>::kAlloc;
     auto kern = dq_tc_kernel<DK, DV>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return FIX_ERR_CUDA;
-    kern<<<(unsigned)((long long)d.nchunks * d.Hq), kThreads, smem, st>>>(mq, mk, mvt, mvm, prm);
+    kern<<<(unsigned)((long long)d.nchunks * d.Hq), kThreads, smem, st>>>(mq, mk, mvt, mvm, mdomh,
+                                                                         mdot, prm);
   } else {
     const int smem = KvLayout<DK, DV>::kAlloc;
     auto kern = dkv_tc_kernel<DK, DV>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return FIX_ERR_CUDA;
-    kern<<<(unsigned)((long long)d.nchunks * d.Hkv), kThreads, smem, st>>>(mq, mk, mvt, mvm, prm);
+    kern<<<(unsigned)(nparts * d.Hkv), kThreads, smem, st>>>(mq, mk, mvt, mvm, mdomh, mdoml, mdot,
+                                                            prm);
+    if (cudaGetLastError() != cudaSuccess) return FIX_ERR_CUDA;
+    if (nslots > 0) dkv_combine_kernel<DK, DV><<<dim3(d.nchunks, d.Hkv), 128, 0, st>>>(prm);
   }
   return cudaGetLastError() == cudaSuccess ? FIX_OK : FIX_ERR_CUDA;
 }
@@ -868,7 +1057,7 @@ bool tc_bwd_supported(const Dims& d) {
   return dims_ok && d.N >= FIX_CHUNK && d.grp <= 16;
 }
 
-int tc_bwd_kernel_count(const Dims&) { return 2; }
+int tc_bwd_kernel_count(const Dims&, long long nslots) { return nslots > 0 ? 3 : 2; }
 
 fix_status tc_bwd(const fix_attn_problem*, const Dims& d, const TcBwdArgs& a, int which,
                   cudaStream_t st) {
@@ -887,19 +1076,25 @@ fix_status tc_bwd(const fix_attn_problem*, const Dims& d, const TcBwdArgs& a, in
   prm.dsafe = a.dsafe;
   prm.m_s = a.m_s;
   prm.do_ws = a.do_ws;
-  prm.dot_ws = a.dot_ws;
-  prm.dom_ws = a.dom_ws;
+  prm.dot = a.dot;
+  prm.domh = a.domh;
+  prm.doml = a.doml;
   prm.A = a.A;
   prm.badflag = a.badflag;
+  prm.parts = a.parts;
+  prm.cpart = a.cpart;
+  prm.tiles_per_part = a.tiles_per_part;
+  prm.nslots = a.nslots;
+  prm.partial = a.partial;
   prm.dq = static_cast<__nv_bfloat16*>(a.dq);
   prm.dk = static_cast<__nv_bfloat16*>(a.dk);
   prm.dv = static_cast<__nv_bfloat16*>(a.dv);
   prm.dG = a.dG;
   prm.status = a.status;
-  if (d.Dk == 128 && d.Dv == 128) return tcb::launch<128, 128>(prm, a.vt, a.vm, which, st);
-  if (d.Dk == 64 && d.Dv == 64) return tcb::launch<64, 64>(prm, a.vt, a.vm, which, st);
-  if (d.Dk == 128 && d.Dv == 64) return tcb::launch<128, 64>(prm, a.vt, a.vm, which, st);
-  if (d.Dk == 64 && d.Dv == 128) return tcb::launch<64, 128>(prm, a.vt, a.vm, which, st);
+  if (d.Dk == 128 && d.Dv == 128) return tcb::launch<128, 128>(prm, a.vt, a.vm, which, a.nparts, a.nslots, st);
+  if (d.Dk == 64 && d.Dv == 64) return tcb::launch<64, 64>(prm, a.vt, a.vm, which, a.nparts, a.nslots, st);
+  if (d.Dk == 128 && d.Dv == 64) return tcb::launch<128, 64>(prm, a.vt, a.vm, which, a.nparts, a.nslots, st);
+  if (d.Dk == 64 && d.Dv == 128) return tcb::launch<64, 128>(prm, a.vt, a.vm, which, a.nparts, a.nslots, st);
   return FIX_ERR_HEAD_DIM;
 }
 

@@ -79,14 +79,17 @@ struct Layout {
   static constexpr int kRho = kVl + BN * DV * 2;
   static constexpr int kHr = kRho + DV * 4;
   static constexpr int kW = kHr + DV * 4;
-  static constexpr int kBars = kW + DV * 4;
+  static constexpr int kRow = kW + DV * 4;              // per-row alpha, P_tt, m (3 x 128 f32)
+  static constexpr int kBars = kRow + 3 * BM * 4;
   static constexpr int kTmem = kBars + (int)sizeof(Bars);
   static constexpr int kAbort = kTmem + 4;
   static constexpr int kBytes = kAbort + 4;
   static constexpr int kAlloc = kBytes + 1024;   // slack for 1024-byte alignment
-  // scratch for the exact path, reusing the K/V ring after the last MMA
+  // after the last MMA: the exact path's P rows, then the accumulators of
+  // every row (fp32, 2 DV per row), reuse the K/V ring and Vm_lo
   static constexpr int kScratch = kK;
   static_assert(2 * BN * DK * 2 + 2 * BN * DV * 2 >= BM * BN * 4, "scratch does not fit");
+  static_assert(kRho - kK >= BM * 2 * DV * 4, "accumulator tile does not fit");
 };
 
 struct Params {
@@ -301,18 +304,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       const uint32_t sbase = lane_base + col_s(st);
+      // the whole S row in registers: four TMEM loads, one wait
+      uint32_t xs[BN];
+#pragma unroll
+      for (int c4 = 0; c4 < BN / 32; ++c4)
+        tmem_ld32(sbase + c4 * 32, *reinterpret_cast<uint32_t(*)[32]>(&xs[c4 * 32]));
+      tmem_wait_ld();
       float mx = -INFINITY;
+      if (it > 0) {
 #pragma unroll
-      for (int c4 = 0; c4 < BN / 32; ++c4) {
-        uint32_t x[32];
-        tmem_ld32(sbase + c4 * 32, x);
-        tmem_wait_ld();
+        for (int e = 0; e < BN; e += 2)
+          mx = fmaxf(mx, fmaxf(__uint_as_float(xs[e]), __uint_as_float(xs[e + 1])));
+      } else {
+        // diagonal block: keys s <= t; S_tt kept for the exact s = t term
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const float sv = __uint_as_float(x[e]);
-          const int key = c4 * 32 + e;
-          if (it > 0 || key <= r) mx = fmaxf(mx, sv);
-          if (it == 0 && key == r) s_diag = sv;
+        for (int e = 0; e < BN; ++e) {
+          const float sv = __uint_as_float(xs[e]);
+          mx = e <= r ? fmaxf(mx, sv) : mx;
+          s_diag = e == r ? sv : s_diag;
         }
       }
       const float mrow = mx * d.scale;
@@ -348,14 +357,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         // diagonal block: strictly causal P as bf16 hi + lo
 #pragma unroll
         for (int c4 = 0; c4 < BN / 32; ++c4) {
-          uint32_t x[32], pk[16], pl[16];
-          tmem_ld32(sbase + c4 * 32, x);
-          tmem_wait_ld();
+          uint32_t pk[16], pl[16];
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
             const int key = c4 * 32 + e;
-            const float p0 = key < r ? ex2(__uint_as_float(x[e]) * c1 - moff) : 0.f;
-            const float p1 = key + 1 < r ? ex2(__uint_as_float(x[e + 1]) * c1 - moff) : 0.f;
+            const float p0 = key < r ? ex2(__uint_as_float(xs[key]) * c1 - moff) : 0.f;
+            const float p1 = key + 1 < r ? ex2(__uint_as_float(xs[key + 1]) * c1 - moff) : 0.f;
             pk[e >> 1] = pack_bf16(p0, p1);
             const float h0 = __uint_as_float(pk[e >> 1] << 16);
             const float h1 = __uint_as_float(pk[e >> 1] & 0xFFFF0000u);
@@ -364,17 +371,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_st16(sbase + c4 * 16, pk);
           tmem_st16(lane_base + kColPlo + c4 * 16, pl);
         }
+      } else if (cta_f16) {
+#pragma unroll
+        for (int c4 = 0; c4 < BN / 32; ++c4) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const int key = c4 * 32 + e;
+            pk[e >> 1] = pack_f16(ex2(__uint_as_float(xs[key]) * c1 - moff),
+                                  ex2(__uint_as_float(xs[key + 1]) * c1 - moff));
+          }
+          tmem_st16(sbase + c4 * 16, pk);
+        }
       } else {
 #pragma unroll
         for (int c4 = 0; c4 < BN / 32; ++c4) {
-          uint32_t x[32], pk[16];
-          tmem_ld32(sbase + c4 * 32, x);
-          tmem_wait_ld();
+          uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
-            const float p0 = ex2(__uint_as_float(x[e]) * c1 - moff);
-            const float p1 = ex2(__uint_as_float(x[e + 1]) * c1 - moff);
-            pk[e >> 1] = cta_f16 ? pack_f16(p0, p1) : pack_bf16(p0, p1);
+            const int key = c4 * 32 + e;
+            pk[e >> 1] = pack_bf16(ex2(__uint_as_float(xs[key]) * c1 - moff),
+                                   ex2(__uint_as_float(xs[key + 1]) * c1 - moff));
           }
           tmem_st16(sbase + c4 * 16, pk);
         }
@@ -390,42 +407,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bar->pv_done, (nblk - 1) & 1, ctl));
     }
     tc_fence_after();
-    // every thread of the warpgroup reaches the named barrier below
     const bool row_ok = ok && r < ch.len;
     const size_t tok = (size_t)ch.tok0 + (size_t)(r < ch.len ? r : 0);
-    const float* Lrow = P.L + tok * vrs + (size_t)kv * DV;
-    const __nv_bfloat16* vrow = P.v + tok * vrs + (size_t)kv * DV;
-    const float alpha = ok ? ex2((m_used - m_true) * LOG2E) : 0.f;
-    const float ptt = ex2((s_diag * d.scale - m_true) * LOG2E);
-    const bool has_off = nblk > 1;
-    float o[DV];
-#pragma unroll
-    for (int cc = 0; cc < DV / 32; ++cc) {
-      uint32_t xd[32], xo[32];
-      tmem_ld32(lane_base + kColOd + cc * 32, xd);
-      tmem_ld32(lane_base + kColOd + DV + cc * 32, xo);
-      tmem_wait_ld();
-#pragma unroll
-      for (int e = 0; e < 32; e += 4) {
-        const int c = cc * 32 + e;
-        const float4 lt = *reinterpret_cast<const float4*>(Lrow + c);
-        const uint2 vv = *reinterpret_cast<const uint2*>(vrow + c);
-        const float vt[4] = {__uint_as_float(vv.x << 16), __uint_as_float(vv.x & 0xFFFF0000u),
-                             __uint_as_float(vv.y << 16), __uint_as_float(vv.y & 0xFFFF0000u)};
-        const float l4[4] = {lt.x, lt.y, lt.z, lt.w};
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          // bad channels have rho = 0 and O_d = 0 there; their exact part comes below
-          const float od = __uint_as_float(xd[e + u]) * ex2((l4[u] - sRho[c + u]) * LOG2E);
-          const float oo = has_off ? __uint_as_float(xo[e + u]) * ex2(l4[u] * LOG2E) : 0.f;
-          o[c + u] = (od + oo) * alpha + ptt * vt[u];
-        }
-      }
-    }
     if (any_bad) {
       // exact fp32 diagonal block for channels outside the split's range:
-      // P rows into the (now idle) K/V ring, then one pass per such channel
-      asm volatile("bar.sync 1, 128;" ::: "memory");
+      // P rows into the (now idle) K/V ring, then one pass per such channel;
+      // the result replaces that channel's (zero) diagonal accumulator column
       float* prow = reinterpret_cast<float*>(smem + Lay::kScratch) + (size_t)r * BN;
       const size_t krs = (size_t)d.Hkv * DK;
       const __nv_bfloat16* kbase = P.k + (size_t)ch.tok0 * krs + (size_t)kv * DK;
@@ -446,50 +433,38 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         prow[s] = ex2((acc * d.scale - m_true) * LOG2E);
       }
+      const float* Lrow = P.L + tok * vrs + (size_t)kv * DV;
       const float* Lcol0 = P.L + (size_t)ch.tok0 * vrs + (size_t)kv * DV;
       const __nv_bfloat16* vcol0 = P.v + (size_t)ch.tok0 * vrs + (size_t)kv * DV;
-#pragma unroll
       for (int c = 0; c < DV; ++c) {
-        if (sHr[c] > FIX_HR_MAX)
-          o[c] += exact_diag_channel(prow, nk, Lrow[c], Lcol0 + c, vcol0 + c, vrs);
+        if (sHr[c] <= FIX_HR_MAX) continue;   // CTA-uniform
+        const float e = exact_diag_channel(prow, nk, Lrow[c], Lcol0 + c, vcol0 + c, vrs);
+        tmem_st1(lane_base + kColOd + c, __float_as_uint(e));
       }
-      asm volatile("bar.sync 1, 128;" ::: "memory");
+      tmem_wait_st();
+      asm volatile("bar.sync 1, 128;" ::: "memory");   // P rows done before the tile overwrites them
     }
-    if (row_ok) {
-      float ss = 0.f;
+    // phase A: this row's two accumulators into a shared fp32 tile, its 16-byte
+    // groups XOR-swizzled by row so that neighbouring rows hit other banks
+    float* tile = reinterpret_cast<float*>(smem + Lay::kScratch);
+    float* trow = tile + (size_t)r * (2 * DV);
 #pragma unroll
-      for (int c = 0; c < DV; ++c) ss += o[c] * o[c];
-      const float rstd = 1.0f / sqrtf(ss / (float)DV + d.eps);
-      const size_t ors = (size_t)d.Hq * DV;
-      const size_t a0 = tok * ors + (size_t)h * DV;
-      if (P.y_f32) {
-        float* yp = reinterpret_cast<float*>(P.y) + a0;
+    for (int cc = 0; cc < 2 * DV / 32; ++cc) {
+      uint32_t x[32];
+      tmem_ld32(lane_base + kColOd + cc * 32, x);
+      tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < DV; c += 4)
-          *reinterpret_cast<float4*>(yp + c) =
-              make_float4(o[c] * rstd * sW[c], o[c + 1] * rstd * sW[c + 1],
-                          o[c + 2] * rstd * sW[c + 2], o[c + 3] * rstd * sW[c + 3]);
-      } else {
-        __nv_bfloat16* yp = reinterpret_cast<__nv_bfloat16*>(P.y) + a0;
-#pragma unroll
-        for (int c = 0; c < DV; c += 8) {
-          uint4 pkd;
-          pkd.x = pack_bf16(o[c] * rstd * sW[c], o[c + 1] * rstd * sW[c + 1]);
-          pkd.y = pack_bf16(o[c + 2] * rstd * sW[c + 2], o[c + 3] * rstd * sW[c + 3]);
-          pkd.z = pack_bf16(o[c + 4] * rstd * sW[c + 4], o[c + 5] * rstd * sW[c + 5]);
-          pkd.w = pack_bf16(o[c + 6] * rstd * sW[c + 6], o[c + 7] * rstd * sW[c + 7]);
-          *reinterpret_cast<uint4*>(yp + c) = pkd;
-        }
-      }
-      if (P.o_s) {
-        float* op = P.o_s + a0;
-#pragma unroll
-        for (int c = 0; c < DV; c += 4)
-          *reinterpret_cast<float4*>(op + c) = make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]);
-        P.m_s[tok * d.Hq + h] = m_true;
-        P.rstd_s[tok * d.Hq + h] = rstd;
+      for (int g4 = 0; g4 < 8; ++g4) {
+        const int grp = cc * 8 + g4;
+        *reinterpret_cast<float4*>(trow + ((grp ^ (r & 7)) << 2)) =
+            make_float4(__uint_as_float(x[4 * g4]), __uint_as_float(x[4 * g4 + 1]),
+                        __uint_as_float(x[4 * g4 + 2]), __uint_as_float(x[4 * g4 + 3]));
       }
     }
+    float* sRow = reinterpret_cast<float*>(smem + Lay::kRow);
+    sRow[r] = ok ? ex2((m_used - m_true) * LOG2E) : 0.f;                 // alpha
+    sRow[BM + r] = ex2((s_diag * d.scale - m_true) * LOG2E);              // P_tt
+    sRow[2 * BM + r] = m_true;
   } else if (warp >= 8) {
     // ------------------------------------------------------------ V decay (j < i)
     const int dt = tid - 256;                        // 0..127
@@ -547,6 +522,85 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
+  if (warp >= 4) {
+    // ---------------------------------------------------------- phase B
+    // warps 4..11, a row at a time, lanes over channels: coalesced L / v
+    // loads, the RMSNorm reduction and coalesced y / o stores
+    asm volatile("bar.sync 2, 256;" ::: "memory");
+    if (!*sAbort) {
+      const float* __restrict__ tile = reinterpret_cast<const float*>(smem + Lay::kScratch);
+      const float* __restrict__ sRow = reinterpret_cast<const float*>(smem + Lay::kRow);
+      const float* __restrict__ Lg = P.L + (size_t)kv * DV;
+      const __nv_bfloat16* __restrict__ vg = P.v + (size_t)kv * DV;
+      float* __restrict__ yf = P.y_f32 ? reinterpret_cast<float*>(P.y) : nullptr;
+      __nv_bfloat16* __restrict__ yb = P.y_f32 ? nullptr : reinterpret_cast<__nv_bfloat16*>(P.y);
+      float* __restrict__ osv = P.o_s;
+      const bool has_off = nblk > 1;
+      const size_t ors = (size_t)d.Hq * DV;
+      constexpr int kU = DV / 32;
+      constexpr int kRows = 4;                         // rows in flight per warp
+      float rho_l[kU], w_l[kU];
+      bool bad_l[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int c = lane + 32 * u;
+        rho_l[u] = sRho[c];
+        w_l[u] = sW[c];
+        bad_l[u] = sHr[c] > FIX_HR_MAX;           // od holds the exact diagonal sum
+      }
+      for (int r0 = (warp - 4) * kRows; r0 < ch.len; r0 += 8 * kRows) {
+        float lt[kRows][kU], vt[kRows][kU];
+#pragma unroll
+        for (int q = 0; q < kRows; ++q) {
+          const int rr = min(r0 + q, ch.len - 1);
+          const size_t tk = (size_t)ch.tok0 + rr;
+#pragma unroll
+          for (int u = 0; u < kU; ++u) {
+            const int c = lane + 32 * u;
+            lt[q][u] = Lg[tk * vrs + c];
+            vt[q][u] = bf2f(vg[tk * vrs + c]);
+          }
+        }
+#pragma unroll
+        for (int q = 0; q < kRows; ++q) {
+          const int rr = r0 + q;
+          if (rr >= ch.len) break;
+          const size_t tk = (size_t)ch.tok0 + rr;
+          const float* trow = tile + (size_t)rr * (2 * DV);
+          const float alpha = sRow[rr], ptt = sRow[BM + rr];
+          float o[kU];
+          float ss = 0.f;
+#pragma unroll
+          for (int u = 0; u < kU; ++u) {
+            const int c = lane + 32 * u;
+            const float od = trow[(((c >> 2) ^ (rr & 7)) << 2) + (c & 3)];
+            const int co = DV + c;
+            const float oo = trow[(((co >> 2) ^ (rr & 7)) << 2) + (co & 3)];
+            float x = bad_l[u] ? od : alpha * od * ex2((lt[q][u] - rho_l[u]) * LOG2E);
+            if (has_off) x += alpha * oo * ex2(lt[q][u] * LOG2E);
+            x += ptt * vt[q][u];
+            o[u] = x;
+            ss += x * x;
+          }
+          ss = warp_sum(ss);
+          const float rstd = 1.0f / sqrtf(ss / (float)DV + d.eps);
+          const size_t a0 = tk * ors + (size_t)h * DV;
+#pragma unroll
+          for (int u = 0; u < kU; ++u) {
+            const int c = lane + 32 * u;
+            const float yv = o[u] * rstd * w_l[u];
+            if (yf) yf[a0 + c] = yv;
+            else yb[a0 + c] = f2bf(yv);
+            if (osv) osv[a0 + c] = o[u];
+          }
+          if (osv && lane == 0) {
+            P.m_s[tk * d.Hq + h] = sRow[2 * BM + rr];
+            P.rstd_s[tk * d.Hq + h] = rstd;
+          }
+        }
+      }
+    }
+  }
   // ---------------------------------------------------------------- teardown
   tc_fence_before();
   __syncthreads();
