@@ -115,9 +115,9 @@ static SplitPlan plan_split(const fix_attn_problem* p, const Dims& d) {
     for (int j = 0; j < nc; ++j) {
       const long long npj = ((long long)d.grp * tiles64_host(L, j) + P - 1) / P;
       sp.nparts += mult * npj;
-      if (npj > 1) sp.nslots += mult * npj;
     }
   });
+  sp.nslots = sp.nparts;   // every part writes its own slot
   return sp;
 }
 
@@ -425,9 +425,9 @@ fix_status fix_attn_bwd(const fix_attn_problem* p, const void* q, const void* k,
   FIX_TRY(launched());
   FIX_TRY(mark(p, FIX_STAGE_BWD_DKV, 1, st));
   FIX_TRY(mark(p, FIX_STAGE_BWD_DG, 0, st));
-  chunk_total_kernel<<<dim3(d.nchunks, d.Hkv), 128, 0, st>>>(d, chunks, dG, dtot);
+  chunk_total_kernel<<<dim3(d.nchunks, d.Hkv), 512, 0, st>>>(d, chunks, dG, dtot);
   FIX_TRY(launched());
-  reverse_cumsum_kernel<<<dim3(d.nchunks, d.Hkv), 128, 0, st>>>(d, chunks, dG, dtot, dg);
+  reverse_cumsum_kernel<<<dim3(d.nchunks, d.Hkv), 512, 0, st>>>(d, chunks, dG, dtot, dg);
   FIX_TRY(launched());
   return mark(p, FIX_STAGE_BWD_DG, 1, st);
 }

@@ -37,7 +37,7 @@ struct Chunk {
 
 // One CTA's share of a key chunk's backward work: the key chunk, the index p
 // of its run of (at most `tiles_per_part`) 64-row query tiles, and the slot of
-// its partial sums (-1 when the chunk is done by a single CTA).
+// its fp32 partial sums in the partial buffer.
 struct Part {
   int ci;
   int p;
@@ -51,7 +51,7 @@ struct PartSpec {
   int tiles_per_part; // P
   int cap_parts;      // entries of parts[]
   Part* parts;
-  int2* cpart;        // per chunk: {number of parts, first slot or -1}
+  int2* cpart;        // per chunk: {number of parts, first slot}
 };
 
 struct Dims {

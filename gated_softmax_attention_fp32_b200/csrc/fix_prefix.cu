@@ -142,12 +142,10 @@ __global__ void __launch_bounds__(1024) schedule_kernel(const int64_t* __restric
       }
     }
     const int nc = (L + FIX_CHUNK - 1) / FIX_CHUNK;
-    int np = 0, ns = 0;
-    for (int j = 0; j < nc; ++j) {
-      const int npj = (ps.grp * tiles64_from(L, j) + ps.tiles_per_part - 1) / ps.tiles_per_part;
-      np += npj;
-      if (npj > 1) ns += npj;
-    }
+    int np = 0;
+    for (int j = 0; j < nc; ++j)
+      np += (ps.grp * tiles64_from(L, j) + ps.tiles_per_part - 1) / ps.tiles_per_part;
+    const int ns = np;   // every part owns a slot of the partial buffer
     int ctot, ptot, stot;
     const int c0 = cbase + block_excl_scan(nc, scan, &ctot);
     const int p0 = pbase + block_excl_scan(np, scan, &ptot);
@@ -155,10 +153,9 @@ __global__ void __launch_bounds__(1024) schedule_kernel(const int64_t* __restric
     int e = p0;
     for (int j = 0; j < nc && c0 + j < cap; ++j) {
       const int npj = (ps.grp * tiles64_from(L, j) + ps.tiles_per_part - 1) / ps.tiles_per_part;
-      ps.cpart[c0 + j] = make_int2(npj, npj > 1 ? s0 : -1);
-      for (int p = 0; p < npj && e < ps.cap_parts; ++p, ++e)
-        ps.parts[e] = Part{c0 + j, p, npj > 1 ? s0 + p : -1, 0};
-      if (npj > 1) s0 += npj;
+      ps.cpart[c0 + j] = make_int2(npj, s0);
+      for (int p = 0; p < npj && e < ps.cap_parts; ++p, ++e) ps.parts[e] = Part{c0 + j, p, s0 + p, 0};
+      s0 += npj;
     }
     cbase += ctot;
     pbase += ptot;
@@ -204,12 +201,18 @@ __global__ void __launch_bounds__(kPrefixThreads) prefix_kernel(
   const size_t base = (size_t)ch.tok0 * rs + (size_t)kv * Dv + c;
   const int r0 = grp * rows;
   const int nr = max(0, min(rows, ch.len - r0));
-  float lv[kMaxRows];
+  float lv[kMaxRows], vv[kMaxRows];
   float acc = 0.f, lmin = INFINITY, lmax = -INFINITY;
   bool nonpos = true;
+  // g and v in one round trip (v only on the tensor-core path)
 #pragma unroll
   for (int u = 0; u < kMaxRows; ++u)
     if (u < nr) lv[u] = g[base + (size_t)(r0 + u) * rs];
+  if (vt) {
+#pragma unroll
+    for (int u = 0; u < kMaxRows; ++u)
+      if (u < nr) vv[u] = bf2f(v[base + (size_t)(r0 + u) * rs]);
+  }
 #pragma unroll
   for (int u = 0; u < kMaxRows; ++u) {
     if (u < nr) {
@@ -242,13 +245,9 @@ __global__ void __launch_bounds__(kPrefixThreads) prefix_kernel(
   if (grp == 0) tot[ti] = total;
   if (!vt) return;  // uniform: the exact kernels need only L and tot
   float vmax = 0.f;
-  float vv[kMaxRows];
 #pragma unroll
   for (int u = 0; u < kMaxRows; ++u)
-    if (u < nr) {
-      vv[u] = bf2f(v[base + (size_t)(r0 + u) * rs]);
-      vmax = fmaxf(vmax, fabsf(vv[u]));
-    }
+    if (u < nr) vmax = fmaxf(vmax, fabsf(vv[u]));
   const int f16 = __syncthreads_and(nonpos && vmax <= FIX_F16_VMAX);
   if (threadIdx.x == 0) safe[(size_t)ci * d.Hkv + kv] = f16;
   const float half = 0.5f * (cmax - cmin);
@@ -274,36 +273,73 @@ __global__ void __launch_bounds__(kPrefixThreads) prefix_kernel(
 
 // Reverse cumsum of dG within each sequence (dg_r = sum_{t >= r} dG_t), in two
 // launches over the same chunk table: chunk totals, then local reverse scans
-// plus the totals of the later chunks of the same sequence.
-__global__ void __launch_bounds__(128) chunk_total_kernel(Dims d, const Chunk* __restrict__ chunks,
-                                                          const float* __restrict__ x,
-                                                          float* __restrict__ tot) {
-  const int ci = blockIdx.x, kv = blockIdx.y, c = threadIdx.x;
-  if (c >= d.Dv) return;
+// plus the totals of the later chunks of the same sequence.  Both use the
+// prefix pass's block shape: 512 threads = (row group, channel), every row of
+// a group loaded up front, groups joined through shared memory.
+__global__ void __launch_bounds__(kPrefixThreads) chunk_total_kernel(Dims d,
+                                                                     const Chunk* __restrict__ chunks,
+                                                                     const float* __restrict__ x,
+                                                                     float* __restrict__ tot) {
+  constexpr int kMaxRows = FIX_CHUNK * 128 / kPrefixThreads;
+  __shared__ float part[kPrefixThreads];
+  const int Dv = d.Dv;
+  const int groups = kPrefixThreads / Dv, rows = FIX_CHUNK / groups;
+  const int c = threadIdx.x % Dv, grp = threadIdx.x / Dv;
+  const int ci = blockIdx.x, kv = blockIdx.y;
   const Chunk ch = chunks[ci];
-  const size_t rs = (size_t)d.Hkv * d.Dv;
-  const size_t base = (size_t)ch.tok0 * rs + (size_t)kv * d.Dv + c;
+  const size_t rs = (size_t)d.Hkv * Dv;
+  const size_t base = (size_t)ch.tok0 * rs + (size_t)kv * Dv + c;
+  const int r0 = grp * rows;
+  const int nr = max(0, min(rows, ch.len - r0));
+  float xv[kMaxRows];
+#pragma unroll
+  for (int u = 0; u < kMaxRows; ++u) xv[u] = u < nr ? x[base + (size_t)(r0 + u) * rs] : 0.f;
   float acc = 0.f;
-  for (int r = 0; r < ch.len; ++r) acc += x[base + (size_t)r * rs];
-  tot[((size_t)ci * d.Hkv + kv) * d.Dv + c] = acc;
+#pragma unroll
+  for (int u = 0; u < kMaxRows; ++u) acc += xv[u];
+  part[threadIdx.x] = acc;
+  __syncthreads();
+  if (grp == 0) {
+    float t = 0.f;
+    for (int q = 0; q < groups; ++q) t += part[q * Dv + c];
+    tot[((size_t)ci * d.Hkv + kv) * Dv + c] = t;
+  }
 }
 
-__global__ void __launch_bounds__(128) reverse_cumsum_kernel(Dims d, const Chunk* __restrict__ chunks,
-                                                             const float* __restrict__ x,
-                                                             const float* __restrict__ tot,
-                                                             float* __restrict__ out) {
-  const int ci = blockIdx.x, kv = blockIdx.y, c = threadIdx.x;
-  if (c >= d.Dv) return;
+__global__ void __launch_bounds__(kPrefixThreads) reverse_cumsum_kernel(
+    Dims d, const Chunk* __restrict__ chunks, const float* __restrict__ x,
+    const float* __restrict__ tot, float* __restrict__ out) {
+  constexpr int kMaxRows = FIX_CHUNK * 128 / kPrefixThreads;
+  __shared__ float part[kPrefixThreads];
+  const int Dv = d.Dv;
+  const int groups = kPrefixThreads / Dv, rows = FIX_CHUNK / groups;
+  const int c = threadIdx.x % Dv, grp = threadIdx.x / Dv;
+  const int ci = blockIdx.x, kv = blockIdx.y;
   const Chunk ch = chunks[ci];
-  const size_t rs = (size_t)d.Hkv * d.Dv;
-  const size_t base = (size_t)ch.tok0 * rs + (size_t)kv * d.Dv + c;
+  const size_t rs = (size_t)d.Hkv * Dv;
+  const size_t base = (size_t)ch.tok0 * rs + (size_t)kv * Dv + c;
+  const int r0 = grp * rows;
+  const int nr = max(0, min(rows, ch.len - r0));
+  float xv[kMaxRows];
+#pragma unroll
+  for (int u = 0; u < kMaxRows; ++u) xv[u] = u < nr ? x[base + (size_t)(r0 + u) * rs] : 0.f;
+  // the later chunks of the sequence, in order
   float acc = 0.f;
   const int first = ci - ch.j;
-  for (int jj = ch.nch - 1; jj > ch.j; --jj) acc += tot[((size_t)(first + jj) * d.Hkv + kv) * d.Dv + c];
-  for (int r = ch.len - 1; r >= 0; --r) {
-    acc += x[base + (size_t)r * rs];
-    out[base + (size_t)r * rs] = acc;
-  }
+  for (int jj = ch.nch - 1; jj > ch.j; --jj) acc += tot[((size_t)(first + jj) * d.Hkv + kv) * Dv + c];
+  float own = 0.f;
+#pragma unroll
+  for (int u = 0; u < kMaxRows; ++u) own += xv[u];
+  part[threadIdx.x] = own;
+  __syncthreads();
+  // then the later row groups of this chunk, from the last one down
+  for (int q = groups - 1; q > grp; --q) acc += part[q * Dv + c];
+#pragma unroll
+  for (int u = kMaxRows - 1; u >= 0; --u)
+    if (u < nr) {
+      acc += xv[u];
+      out[base + (size_t)(r0 + u) * rs] = acc;
+    }
 }
 
 }  // namespace fix

@@ -411,82 +411,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 constexpr int BQ = 64;   // query rows per streamed tile
 
-// P_ss = exp(S_ss - m_s) of the group's q heads for key row `tok` (the s = t
-// pair, which dv_strict leaves out).
-template <int DK>
-__device__ void row_pss(const Params& P, int kv, size_t tok, float* pss, int ng) {
-  const Dims& d = P.d;
-  const __nv_bfloat16* krow = P.k + tok * (size_t)d.Hkv * DK + (size_t)kv * DK;
-  for (int hh = 0; hh < ng; ++hh) {
-    const int h = kv * d.grp + hh;
-    const __nv_bfloat16* qrow = P.q + tok * (size_t)d.Hq * DK + (size_t)h * DK;
-    float acc = 0.f;
-    for (int dd = 0; dd < DK; dd += 8) {
-      float a8[8], b8[8];
-      unpack8(*reinterpret_cast<const uint4*>(qrow + dd), false, a8);
-      unpack8(*reinterpret_cast<const uint4*>(krow + dd), false, b8);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) acc += a8[e] * b8[e];
-    }
-    pss[hh] = ex2((acc * d.scale - P.m_s[tok * d.Hq + h]) * LOG2E);
-  }
-}
-
-// dv and dG for 32 channels [32 cc, 32 cc + 32) of key row `tok` of key chunk
-// cj, from the two accumulators (diagonal reference rho, chunk-end reference):
-//   dv_strict = exp(rho - L_s) dV_d + exp(tot - L_s) dV_o
-//   dv = dv_strict + sum_h P_ss do_s,   dG = A - v dv_strict
-template <int DV>
-__device__ void finish_dv32(const Params& P, int cj, int kv, size_t tok, int cc, const float* dvd,
-                            const float* dvo, bool has_off, const float* pss, int ng) {
-  const Dims& d = P.d;
-  const size_t vrs = (size_t)d.Hkv * DV, ors = (size_t)d.Hq * DV;
-  const float* Lrow = P.L + tok * vrs + (size_t)kv * DV;
-  const float* trow = P.tot + ((size_t)cj * d.Hkv + kv) * DV;
-  const float* rrow = P.rho + ((size_t)cj * d.Hkv + kv) * DV;
-  float dvv[32], dgv[32];
-#pragma unroll
-  for (int e = 0; e < 32; ++e) {
-    const int c = cc * 32 + e;
-    const float ls = Lrow[c];
-    float strict = dvd[e] * ex2((rrow[c] - ls) * LOG2E);
-    if (has_off) strict += dvo[e] * ex2((trow[c] - ls) * LOG2E);
-    float diagsum = 0.f;
-    for (int hh = 0; hh < ng; ++hh)
-      diagsum += pss[hh] * P.do_ws[tok * ors + (size_t)(kv * d.grp + hh) * DV + c];
-    dvv[e] = strict + diagsum;
-    dgv[e] = P.A[tok * vrs + (size_t)kv * DV + c] - bf2f(P.v[tok * vrs + (size_t)kv * DV + c]) * strict;
-  }
-  __nv_bfloat16* dvp = P.dv + tok * vrs + (size_t)kv * DV + cc * 32;
-  float* dgp = P.dG + tok * vrs + (size_t)kv * DV + cc * 32;
-#pragma unroll
-  for (int e = 0; e < 32; e += 8) {
-    uint4 pkd;
-    pkd.x = pack_bf16(dvv[e], dvv[e + 1]);
-    pkd.y = pack_bf16(dvv[e + 2], dvv[e + 3]);
-    pkd.z = pack_bf16(dvv[e + 4], dvv[e + 5]);
-    pkd.w = pack_bf16(dvv[e + 6], dvv[e + 7]);
-    *reinterpret_cast<uint4*>(dvp + e) = pkd;
-    *reinterpret_cast<float4*>(dgp + e) = make_float4(dgv[e], dgv[e + 1], dgv[e + 2], dgv[e + 3]);
-    *reinterpret_cast<float4*>(dgp + e + 4) = make_float4(dgv[e + 4], dgv[e + 5], dgv[e + 6], dgv[e + 7]);
-  }
-}
-
-template <int DK>
-__device__ void finish_dk32(const Params& P, int kv, size_t tok, int cc, const float* acc) {
-  const Dims& d = P.d;
-  __nv_bfloat16* dkp = P.dk + tok * (size_t)d.Hkv * DK + (size_t)kv * DK + cc * 32;
-#pragma unroll
-  for (int e = 0; e < 32; e += 8) {
-    uint4 pkd;
-    pkd.x = pack_bf16(acc[e] * d.scale, acc[e + 1] * d.scale);
-    pkd.y = pack_bf16(acc[e + 2] * d.scale, acc[e + 3] * d.scale);
-    pkd.z = pack_bf16(acc[e + 4] * d.scale, acc[e + 5] * d.scale);
-    pkd.w = pack_bf16(acc[e + 6] * d.scale, acc[e + 7] * d.scale);
-    *reinterpret_cast<uint4*>(dkp + e) = pkd;
-  }
-}
-
 struct KvBars {
   uint64_t kv_full;
   uint64_t q_full[2], q_empty[2], x_ready[2];
@@ -775,8 +699,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bar->done, 0, ctl));
     tc_fence_after();
     // ---------------------------------------------------------- epilogue
-    const bool row_ok = ok && s < ch.len;
-    const size_t tok = (size_t)ch.tok0 + (size_t)(s < ch.len ? s : 0);
     // which accumulators this CTA's tiles wrote
     bool has_diag = false, has_off = false;
     {
@@ -786,76 +708,64 @@ __global__ void __launch_bounds__(kThreads, 1)
         else has_off = true;
       }
     }
-    if (pt.slot < 0) {
-      // the whole key chunk was this CTA's: finish dv, dG, dk here
-      float pss[16];
-      const int ng = min(d.grp, 16);
-      if (row_ok) row_pss<DK>(P, kv, tok, pss, ng);
-#pragma unroll
-      for (int cc = 0; cc < DV / 32; ++cc) {
-        uint32_t xd[32], xo[32];
-        tmem_ld32(lane_base + kColVd + cc * 32, xd);
-        tmem_ld32(lane_base + kColVo + cc * 32, xo);
-        tmem_wait_ld();
-        if (row_ok) {
-          float fd[32], fo[32];
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            fd[e] = __uint_as_float(xd[e]);
-            fo[e] = has_off ? __uint_as_float(xo[e]) : 0.f;
-          }
-          finish_dv32<DV>(P, cj, kv, tok, cc, fd, fo, has_off, pss, ng);
-        }
-      }
-#pragma unroll
-      for (int cc = 0; cc < DK / 32; ++cc) {
-        uint32_t x[32];
-        tmem_ld32(lane_base + kColK + cc * 32, x);
-        tmem_wait_ld();
-        if (row_ok) {
-          float fk[32];
-#pragma unroll
-          for (int e = 0; e < 32; ++e) fk[e] = __uint_as_float(x[e]);
-          finish_dk32<DK>(P, kv, tok, cc, fk);
-        }
-      }
-    } else if (pt.slot < P.nslots) {
-      // one of several CTAs of this key chunk: raw partial sums, summed by
-      // the combine kernel in slot order
-      constexpr int kCols = DK + 2 * DV;
-      float* prow = P.partial + (((size_t)pt.slot * d.Hkv + kv) * BN + s) * kCols;
-#pragma unroll
-      for (int cc = 0; cc < DK / 32; ++cc) {
-        uint32_t x[32];
-        tmem_ld32(lane_base + kColK + cc * 32, x);
-        tmem_wait_ld();
+    // The CTA's raw sums (dK | dV_d | dV_o, fp32, a row per key) go to its
+    // slot of the partial buffer; the combine kernel adds the slots of a key
+    // chunk in order and finishes dk, dv and dG.  Each thread stages its row,
+    // one segment at a time, in the operand buffers (free once every MMA has
+    // completed) and sends it with its own bulk copy.  Staged rows are padded
+    // by 16 bytes so that eight consecutive rows start on distinct banks; two
+    // buffers alternate.
+    constexpr int kCols = DK + 2 * DV;
+    constexpr int kPad0 = (DK > DV ? DK : DV) + 4;     // staged row strides, floats
+    constexpr int kPad1 = DV + 4;
+    static_assert(BN * (kPad0 + kPad1) * 4 <= Lay::kM, "two staging buffers must fit");
+    if (ok && pt.slot >= 0 && pt.slot < P.nslots) {
+      float* grow = P.partial + (((size_t)pt.slot * d.Hkv + kv) * BN + s) * kCols;
+      float* buf[2] = {reinterpret_cast<float*>(smem) + (size_t)s * kPad0,
+                       reinterpret_cast<float*>(smem) + (size_t)BN * kPad0 + (size_t)s * kPad1};
+      auto stage32 = [&](float* dst, const uint32_t (&x)[32], bool keep) {
 #pragma unroll
         for (int e = 0; e < 32; e += 4)
-          *reinterpret_cast<float4*>(prow + cc * 32 + e) =
-              make_float4(__uint_as_float(x[e]), __uint_as_float(x[e + 1]),
-                          __uint_as_float(x[e + 2]), __uint_as_float(x[e + 3]));
+          *reinterpret_cast<float4*>(dst + e) =
+              keep ? make_float4(__uint_as_float(x[e]), __uint_as_float(x[e + 1]),
+                                 __uint_as_float(x[e + 2]), __uint_as_float(x[e + 3]))
+                   : make_float4(0.f, 0.f, 0.f, 0.f);
+      };
+      // dK -> buffer 0
+#pragma unroll
+      for (int cc = 0; cc < DK / 32; ++cc) {
+        uint32_t x[32];
+        tmem_ld32(lane_base + kColK + cc * 32, x);
+        tmem_wait_ld();
+        stage32(buf[0] + cc * 32, x, true);
       }
+      fence_proxy_async_smem();
+      bulk_store(grow, buf[0], DK * 4);
+      bulk_commit();
+      // dV_d -> buffer 1
 #pragma unroll
       for (int cc = 0; cc < DV / 32; ++cc) {
-        uint32_t xd[32], xo[32];
-        tmem_ld32(lane_base + kColVd + cc * 32, xd);
-        tmem_ld32(lane_base + kColVo + cc * 32, xo);
+        uint32_t x[32];
+        tmem_ld32(lane_base + kColVd + cc * 32, x);
         tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; e += 4) {
-          float4 a, b;
-          a.x = has_diag ? __uint_as_float(xd[e]) : 0.f;
-          a.y = has_diag ? __uint_as_float(xd[e + 1]) : 0.f;
-          a.z = has_diag ? __uint_as_float(xd[e + 2]) : 0.f;
-          a.w = has_diag ? __uint_as_float(xd[e + 3]) : 0.f;
-          b.x = has_off ? __uint_as_float(xo[e]) : 0.f;
-          b.y = has_off ? __uint_as_float(xo[e + 1]) : 0.f;
-          b.z = has_off ? __uint_as_float(xo[e + 2]) : 0.f;
-          b.w = has_off ? __uint_as_float(xo[e + 3]) : 0.f;
-          *reinterpret_cast<float4*>(prow + DK + cc * 32 + e) = a;
-          *reinterpret_cast<float4*>(prow + DK + DV + cc * 32 + e) = b;
-        }
+        stage32(buf[1] + cc * 32, x, has_diag);
       }
+      fence_proxy_async_smem();
+      bulk_store(grow + DK, buf[1], DV * 4);
+      bulk_commit();
+      // dV_o -> buffer 0, once the dK copy has read it
+      bulk_wait_read<1>();
+#pragma unroll
+      for (int cc = 0; cc < DV / 32; ++cc) {
+        uint32_t x[32];
+        tmem_ld32(lane_base + kColVo + cc * 32, x);
+        tmem_wait_ld();
+        stage32(buf[0] + cc * 32, x, has_off);
+      }
+      fence_proxy_async_smem();
+      bulk_store(grow + DK + DV, buf[0], DV * 4);
+      bulk_commit();
+      bulk_wait_read<0>();
     }
   } else if (warp >= 8) {
     // ------------------------------------------------------------ X operand tiles
@@ -940,56 +850,118 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// V consecutive floats (V = 2 or 4) from a 4V-byte aligned address.
+template <int V>
+__device__ __forceinline__ void ldf(const float* p, float* x) {
+  if constexpr (V == 4) {
+    const float4 a = *reinterpret_cast<const float4*>(p);
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+  } else {
+    const float2 a = *reinterpret_cast<const float2*>(p);
+    x[0] = a.x; x[1] = a.y;
+  }
+}
+template <int V>
+__device__ __forceinline__ void stf(float* p, const float* x) {
+  if constexpr (V == 4) *reinterpret_cast<float4*>(p) = make_float4(x[0], x[1], x[2], x[3]);
+  else *reinterpret_cast<float2*>(p) = make_float2(x[0], x[1]);
+}
+template <int V>
+__device__ __forceinline__ void ldb(const __nv_bfloat16* p, float* x) {
+  if constexpr (V == 4) {
+    const uint2 a = *reinterpret_cast<const uint2*>(p);
+    x[0] = __uint_as_float(a.x << 16); x[1] = __uint_as_float(a.x & 0xFFFF0000u);
+    x[2] = __uint_as_float(a.y << 16); x[3] = __uint_as_float(a.y & 0xFFFF0000u);
+  } else {
+    const uint32_t a = *reinterpret_cast<const uint32_t*>(p);
+    x[0] = __uint_as_float(a << 16); x[1] = __uint_as_float(a & 0xFFFF0000u);
+  }
+}
+template <int V>
+__device__ __forceinline__ void stb(__nv_bfloat16* p, const float* x) {
+  if constexpr (V == 4) *reinterpret_cast<uint2*>(p) = make_uint2(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]));
+  else *reinterpret_cast<uint32_t*>(p) = pack_bf16(x[0], x[1]);
+}
+
 // Sums the partial rows of key chunks split over several CTAs (in slot
 // order, so the result does not depend on scheduling) and finishes dv, dG,
-// dk.  grid (nchunks, Hkv), block 128: thread = key row.
+// dk.  grid (nchunks * BN / 8, Hkv), block 256: a warp per key row, lanes
+// over channels, so that every row of every array is read and written in
+// one coalesced stretch.
 template <int DK, int DV>
-__global__ void __launch_bounds__(128) dkv_combine_kernel(const Params P) {
+__global__ void __launch_bounds__(256) dkv_combine_kernel(const Params P) {
   if (*P.badflag) return;
   const Dims& d = P.d;
-  const int ci = blockIdx.x, kv = blockIdx.y, s = threadIdx.x;
+  constexpr int kRowBlocks = BN / 8;
+  const int ci = blockIdx.x / kRowBlocks, kv = blockIdx.y, lane = threadIdx.x & 31;
+  const int s = (blockIdx.x % kRowBlocks) * 8 + (threadIdx.x >> 5);
   const int2 cp = P.cpart[ci];
-  if (cp.x <= 1 || cp.y < 0 || cp.y + cp.x > P.nslots) return;
+  if (cp.x < 1 || cp.y < 0 || cp.y + cp.x > P.nslots) return;
   const Chunk ch = P.chunks[ci];
   if (s >= ch.len) return;
   const size_t tok = (size_t)ch.tok0 + s;
   constexpr int kCols = DK + 2 * DV;
+  constexpr int VK = DK / 32, VV = DV / 32;            // channels per lane
+  const int ck = lane * VK, cv = lane * VV;
+  float fk[VK] = {}, fd[VV] = {}, fo[VV] = {};
+  for (int q = 0; q < cp.x; ++q) {
+    const float* prow = P.partial + (((size_t)(cp.y + q) * d.Hkv + kv) * BN + s) * kCols;
+    float a[VK], b[VV], c[VV];
+    ldf<VK>(prow + ck, a);
+    ldf<VV>(prow + DK + cv, b);
+    ldf<VV>(prow + DK + DV + cv, c);
+#pragma unroll
+    for (int e = 0; e < VK; ++e) fk[e] += a[e];
+#pragma unroll
+    for (int e = 0; e < VV; ++e) {
+      fd[e] += b[e];
+      fo[e] += c[e];
+    }
+  }
+  // dk = scale * sum dS^T Q
+  const size_t krs = (size_t)d.Hkv * DK;
+#pragma unroll
+  for (int e = 0; e < VK; ++e) fk[e] *= d.scale;
+  stb<VK>(P.dk + tok * krs + (size_t)kv * DK + ck, fk);
+  // the s = t terms: P_ss (one per q head of the group) times do_s
+  float kr[VK];
+  ldb<VK>(P.k + tok * krs + (size_t)kv * DK + ck, kr);
+  const size_t vrs = (size_t)d.Hkv * DV, ors = (size_t)d.Hq * DV;
+  float diag[VV] = {};
+  for (int hh = 0; hh < d.grp; ++hh) {
+    const int h = kv * d.grp + hh;
+    float qr[VK];
+    ldb<VK>(P.q + tok * (size_t)d.Hq * DK + (size_t)h * DK + ck, qr);
+    float acc = 0.f;
+#pragma unroll
+    for (int e = 0; e < VK; ++e) acc += qr[e] * kr[e];
+    acc = warp_sum(acc);
+    const float pss = ex2((acc * d.scale - P.m_s[tok * d.Hq + h]) * LOG2E);
+    float dw[VV];
+    ldf<VV>(P.do_ws + tok * ors + (size_t)h * DV + cv, dw);
+#pragma unroll
+    for (int e = 0; e < VV; ++e) diag[e] += pss * dw[e];
+  }
+  // dv_strict = exp(rho - L_s) dV_d + exp(tot - L_s) dV_o;
+  // dv = dv_strict + the s = t terms, dG = A - v dv_strict
+  const size_t cb = ((size_t)ci * d.Hkv + kv) * DV + cv, rb = tok * vrs + (size_t)kv * DV + cv;
   const bool has_off = ch.nch - ch.j > 1;
-  float pss[16];
-  const int ng = min(d.grp, 16);
-  row_pss<DK>(P, kv, tok, pss, ng);
-#pragma unroll 1
-  for (int cc = 0; cc < DV / 32; ++cc) {
-    float fd[32], fo[32];
+  float ls[VV], rh[VV], tt[VV], av[VV], vv[VV];
+  ldf<VV>(P.L + rb, ls);
+  ldf<VV>(P.rho + cb, rh);
+  ldf<VV>(P.tot + cb, tt);
+  ldf<VV>(P.A + rb, av);
+  ldb<VV>(P.v + rb, vv);
+  float dvv[VV], dgv[VV];
 #pragma unroll
-    for (int e = 0; e < 32; ++e) fd[e] = fo[e] = 0.f;
-    for (int q = 0; q < cp.x; ++q) {
-      const float* prow = P.partial + (((size_t)(cp.y + q) * d.Hkv + kv) * BN + s) * kCols;
-#pragma unroll
-      for (int e = 0; e < 32; e += 4) {
-        const float4 a = *reinterpret_cast<const float4*>(prow + DK + cc * 32 + e);
-        const float4 b = *reinterpret_cast<const float4*>(prow + DK + DV + cc * 32 + e);
-        fd[e] += a.x; fd[e + 1] += a.y; fd[e + 2] += a.z; fd[e + 3] += a.w;
-        fo[e] += b.x; fo[e + 1] += b.y; fo[e + 2] += b.z; fo[e + 3] += b.w;
-      }
-    }
-    finish_dv32<DV>(P, ci, kv, tok, cc, fd, fo, has_off, pss, ng);
+  for (int e = 0; e < VV; ++e) {
+    float strict = fd[e] * ex2((rh[e] - ls[e]) * LOG2E);
+    if (has_off) strict += fo[e] * ex2((tt[e] - ls[e]) * LOG2E);
+    dvv[e] = strict + diag[e];
+    dgv[e] = av[e] - vv[e] * strict;
   }
-#pragma unroll 1
-  for (int cc = 0; cc < DK / 32; ++cc) {
-    float fk[32];
-#pragma unroll
-    for (int e = 0; e < 32; ++e) fk[e] = 0.f;
-    for (int q = 0; q < cp.x; ++q) {
-      const float* prow = P.partial + (((size_t)(cp.y + q) * d.Hkv + kv) * BN + s) * kCols;
-#pragma unroll
-      for (int e = 0; e < 32; e += 4) {
-        const float4 a = *reinterpret_cast<const float4*>(prow + cc * 32 + e);
-        fk[e] += a.x; fk[e + 1] += a.y; fk[e + 2] += a.z; fk[e + 3] += a.w;
-      }
-    }
-    finish_dk32<DK>(P, kv, tok, cc, fk);
-  }
+  stb<VV>(P.dv + rb, dvv);
+  stf<VV>(P.dG + rb, dgv);
 }
 
 // ---------------------------------------------------------------- host side
@@ -1045,7 +1017,7 @@ static fix_status launch(const Params& prm, const void* vt, const void* vm, int 
     kern<<<(unsigned)(nparts * d.Hkv), kThreads, smem, st>>>(mq, mk, mvt, mvm, mdomh, mdoml, mdot,
                                                             prm);
     if (cudaGetLastError() != cudaSuccess) return FIX_ERR_CUDA;
-    if (nslots > 0) dkv_combine_kernel<DK, DV><<<dim3(d.nchunks, d.Hkv), 128, 0, st>>>(prm);
+    if (nslots > 0) dkv_combine_kernel<DK, DV><<<dim3(d.nchunks * (BN / 8), d.Hkv), 256, 0, st>>>(prm);
   }
   return cudaGetLastError() == cudaSuccess ? FIX_OK : FIX_ERR_CUDA;
 }
