@@ -124,7 +124,7 @@ static SplitPlan plan_split(const fix_attn_problem* p, const Dims& d) {
 // Workspace layout (all offsets 256-byte aligned).
 struct Ws {
   size_t status, chunks, order, safe, L, vt, vm, vml, tot, rho, hr;   // forward and backward
-  size_t dow, dot, domh, doml, dsafe, A, dG, dtot, dwp;    // backward only
+  size_t dow, dot, domh, doml, dsafe, hmax, A, dG, dtot, dwp;   // backward only
   size_t parts, cpart, partial;                            // dk/dv work split
   size_t total;
 };
@@ -156,10 +156,11 @@ static Ws layout(const Dims& d, bool bwd, const SplitPlan& sp) {
     w.domh = take((size_t)d.N * d.Hq * d.Dv * 2);
     w.doml = take((size_t)d.N * d.Hq * d.Dv * 2);
     w.dsafe = take((size_t)(d.nchunks > 0 ? d.nchunks : 1) * d.Hq * sizeof(int));
+    w.hmax = take((size_t)(d.nchunks > 0 ? d.nchunks : 1) * d.Hq * sizeof(int));
     w.A = take(nkv * 4);
     w.dG = take(nkv * 4);
     w.dtot = take(nch * 4);
-    w.dwp = take((size_t)(d.nchunks > 0 ? d.nchunks : 1) * d.Hkv * d.Dv * 4);
+    w.dwp = take((size_t)(d.nchunks > 0 ? d.nchunks : 1) * kPreSplit * d.Hkv * d.Dv * 4);
     w.parts = take((size_t)(sp.nparts > 0 ? sp.nparts : 1) * sizeof(Part));
     w.cpart = take((size_t)(d.nchunks > 0 ? d.nchunks : 1) * sizeof(int2));
     w.partial = take((size_t)sp.nslots * d.Hkv * FIX_CHUNK * (d.Dk + 2 * d.Dv) * 4);
@@ -209,7 +210,7 @@ static size_t simt_dkv_smem(const Dims& d) {
 // Prefix pass + schedule (both directions).
 static fix_status run_prefix(const Dims& d, const fix_attn_problem* p, const Ws& ws, char* base,
                              const float* g, const void* v, bool want_vt, const SplitPlan* sp,
-                             cudaStream_t st) {
+                             int* hmax, cudaStream_t st) {
   Chunk* chunks = reinterpret_cast<Chunk*>(base + ws.chunks);
   PartSpec ps{};
   if (sp) {
@@ -230,7 +231,7 @@ static fix_status run_prefix(const Dims& d, const fix_attn_problem* p, const Ws&
       reinterpret_cast<__nv_bfloat16*>(base + ws.vm),
       reinterpret_cast<__nv_bfloat16*>(base + ws.vml), reinterpret_cast<float*>(base + ws.tot),
       reinterpret_cast<float*>(base + ws.rho), reinterpret_cast<float*>(base + ws.hr),
-      reinterpret_cast<int*>(base + ws.safe), reinterpret_cast<int*>(base + ws.status) + 1);
+      reinterpret_cast<int*>(base + ws.safe), reinterpret_cast<int*>(base + ws.status) + 1, hmax);
   return launched();
 }
 
@@ -285,7 +286,7 @@ fix_status fix_attn_fwd(const fix_attn_problem* p, const void* q, const void* k,
   if (d.N == 0) return FIX_OK;
   const bool tc = p->algo != FIX_ALGO_SIMT && tc_fwd_supported(d);
   FIX_TRY(mark(p, FIX_STAGE_FWD_PREFIX, 0, st));
-  FIX_TRY(run_prefix(d, p, ws, base, g, v, tc, nullptr, st));
+  FIX_TRY(run_prefix(d, p, ws, base, g, v, tc, nullptr, nullptr, st));
   FIX_TRY(mark(p, FIX_STAGE_FWD_PREFIX, 1, st));
   const Chunk* chunks = reinterpret_cast<const Chunk*>(base + ws.chunks);
   const float* L = reinterpret_cast<const float*>(base + ws.L);
@@ -340,7 +341,8 @@ fix_status fix_attn_bwd(const fix_attn_problem* p, const void* q, const void* k,
   }
   const bool tc = p->algo != FIX_ALGO_SIMT && tc_bwd_supported(d);
   FIX_TRY(mark(p, FIX_STAGE_BWD_PREFIX, 0, st));
-  FIX_TRY(run_prefix(d, p, ws, base, g, v, tc, tc ? &sp : nullptr, st));
+  FIX_TRY(run_prefix(d, p, ws, base, g, v, tc, tc ? &sp : nullptr,
+                     tc ? reinterpret_cast<int*>(base + ws.hmax) : nullptr, st));
   FIX_TRY(mark(p, FIX_STAGE_BWD_PREFIX, 1, st));
   const Chunk* chunks = reinterpret_cast<const Chunk*>(base + ws.chunks);
   const float* L = reinterpret_cast<const float*>(base + ws.L);
@@ -359,13 +361,20 @@ fix_status fix_attn_bwd(const fix_attn_problem* p, const void* q, const void* k,
   const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(k);
   const __nv_bfloat16* vb = static_cast<const __nv_bfloat16*>(v);
   FIX_TRY(mark(p, FIX_STAGE_BWD_PRE, 0, st));
-  bwd_pre_kernel<<<dim3(d.nchunks, d.Hkv), 512, d.grp * sizeof(float), st>>>(
+  int* hmax = reinterpret_cast<int*>(base + ws.hmax);
+  bwd_pre_kernel<<<dim3(d.nchunks * kPreSplit, d.Hkv), 256, d.grp * sizeof(float), st>>>(
       d, chunks, qb, kb, vb, o_s, m_s, rstd_s, static_cast<const __nv_bfloat16*>(dy),
-      static_cast<const __nv_bfloat16*>(w), L, reinterpret_cast<const float*>(base + ws.rho),
-      reinterpret_cast<const float*>(base + ws.hr), reinterpret_cast<const int*>(base + ws.safe),
-      dow, tc ? dot : nullptr, domh, doml, dsafe, A, dwp);
+      static_cast<const __nv_bfloat16*>(w), dow, A, dwp, tc ? hmax : nullptr);
   FIX_TRY(launched());
-  dw_reduce_kernel<<<1, 128, 0, st>>>(dwp, d.nchunks * d.Hkv, d.Dv, static_cast<__nv_bfloat16*>(dw));
+  if (tc) {
+    bwd_pre_ops_kernel<<<dim3(d.nchunks * kPreSplit, d.Hkv), 256, 0, st>>>(
+        d, chunks, L, reinterpret_cast<const float*>(base + ws.rho),
+        reinterpret_cast<const float*>(base + ws.hr), reinterpret_cast<const int*>(base + ws.safe),
+        dow, hmax, dot, domh, doml, dsafe);
+    FIX_TRY(launched());
+  }
+  dw_reduce_kernel<<<1, 512, 0, st>>>(dwp, d.nchunks * kPreSplit * d.Hkv, d.Dv,
+                                      static_cast<__nv_bfloat16*>(dw));
   FIX_TRY(launched());
   FIX_TRY(mark(p, FIX_STAGE_BWD_PRE, 1, st));
   TcBwdArgs ta{};
@@ -441,7 +450,9 @@ int fix_attn_kernel_count(const fix_attn_problem* p, int backward) {
     return 2 + (tc ? tc_fwd_kernel_count(d) : 1);
   }
   const bool tc = p->algo != FIX_ALGO_SIMT && tc_bwd_supported(d);
-  return 2 + 2 + (tc ? tc_bwd_kernel_count(d, plan_split(p, d).nslots) : 0) + 2 + 2;
+  // prefix pass (2), preprocess (2, or 3 with the tensor-core operands),
+  // tensor-core dq / dk/dv, the exact kernels (2), the dG reverse cumsum (2)
+  return 2 + (tc ? 3 : 2) + (tc ? tc_bwd_kernel_count(d, plan_split(p, d).nslots) : 0) + 2 + 2;
 }
 
 fix_status fix_attn_device_status(const void* workspace, void* stream) {

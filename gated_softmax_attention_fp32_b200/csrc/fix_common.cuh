@@ -15,6 +15,8 @@
 #include <stdint.h>
 
 #define FIX_CHUNK 128
+// CTAs per chunk in the backward preprocess (FIX_CHUNK / kPreSplit rows each).
+constexpr int kPreSplit = 4;
 // Largest half-range of a chunk's prefix sums that the in-chunk split
 // exp(L_t - rho) * exp(rho - L_s) keeps inside float range (e^80 ~ 5.5e34).
 #define FIX_HR_MAX 80.0f

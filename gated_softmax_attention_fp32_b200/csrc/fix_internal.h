@@ -12,7 +12,8 @@ __global__ void schedule_kernel(const int64_t* cu, int nseq, int T, int N, int c
                                 int maxj, int* order, PartSpec ps);
 __global__ void prefix_kernel(Dims d, const Chunk* chunks, const float* g, const __nv_bfloat16* v,
                               float* L, uint16_t* vt, __nv_bfloat16* vm, __nv_bfloat16* vml,
-                              float* tot, float* rho, float* hr, int* safe, int* badflag);
+                              float* tot, float* rho, float* hr, int* safe, int* badflag,
+                              int* hmax);
 __global__ void chunk_total_kernel(Dims d, const Chunk* chunks, const float* x, float* tot);
 __global__ void reverse_cumsum_kernel(Dims d, const Chunk* chunks, const float* x,
                                       const float* tot, float* out);
@@ -25,10 +26,12 @@ __global__ void fwd_simt_kernel(Dims d, const Chunk* chunks, const __nv_bfloat16
 __global__ void bwd_pre_kernel(Dims d, const Chunk* chunks, const __nv_bfloat16* q,
                                const __nv_bfloat16* k, const __nv_bfloat16* v, const float* o_s,
                                const float* m_s, const float* rstd_s, const __nv_bfloat16* dy,
-                               const __nv_bfloat16* w, const float* L, const float* rho,
-                               const float* hr, const int* safe, float* do_ws, uint16_t* dot,
-                               __nv_bfloat16* domh, __nv_bfloat16* doml, int* dsafe, float* A,
-                               float* dwpart);
+                               const __nv_bfloat16* w, float* do_ws, float* A, float* dwpart,
+                               int* hmax_g);
+__global__ void bwd_pre_ops_kernel(Dims d, const Chunk* chunks, const float* L, const float* rho,
+                                   const float* hr, const int* safe, const float* do_ws,
+                                   const int* hmax_g, uint16_t* dot, __nv_bfloat16* domh,
+                                   __nv_bfloat16* doml, int* dsafe);
 __global__ void dw_reduce_kernel(const float* parts, int nparts, int Dv, __nv_bfloat16* dw);
 __global__ void dq_simt_kernel(Dims d, const Chunk* chunks, const __nv_bfloat16* q,
                                const __nv_bfloat16* k, const __nv_bfloat16* v, const float* L,

@@ -188,7 +188,7 @@ __global__ void __launch_bounds__(kPrefixThreads) prefix_kernel(
     const __nv_bfloat16* __restrict__ v, float* __restrict__ L, uint16_t* __restrict__ vt,
     __nv_bfloat16* __restrict__ vm, __nv_bfloat16* __restrict__ vml, float* __restrict__ tot,
     float* __restrict__ rho, float* __restrict__ hr, int* __restrict__ safe,
-    int* __restrict__ badflag) {
+    int* __restrict__ badflag, int* __restrict__ hmax) {
   constexpr int kMaxRows = FIX_CHUNK * 128 / kPrefixThreads;  // rows per thread at Dv = 128
   __shared__ float part[kPrefixThreads], pmin[kPrefixThreads], pmax[kPrefixThreads];
   const int Dv = d.Dv;
@@ -197,6 +197,8 @@ __global__ void __launch_bounds__(kPrefixThreads) prefix_kernel(
   const int c = threadIdx.x % Dv, grp = threadIdx.x / Dv;
   const int ci = blockIdx.x, kv = blockIdx.y;
   const Chunk ch = chunks[ci];
+  // the backward's per-(chunk, q head) max |do|, raised by its preprocess
+  if (hmax && threadIdx.x < d.grp) hmax[(size_t)ci * d.Hq + kv * d.grp + threadIdx.x] = 0;
   const size_t rs = (size_t)d.Hkv * Dv;
   const size_t base = (size_t)ch.tok0 * rs + (size_t)kv * Dv + c;
   const int r0 = grp * rows;

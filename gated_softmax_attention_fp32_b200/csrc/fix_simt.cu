@@ -152,8 +152,9 @@ __global__ void __launch_bounds__(256) fwd_simt_kernel(
 }
 
 // ---------------------------------------------------------------------------
-// Backward preprocess (shared by all kernel families), one CTA per (chunk, kv
-// head), 16 warps, a warp per row at a time over the kv group's q heads:
+// Backward preprocess (shared by all kernel families).  Pass 1, grid
+// (nchunks * kPreSplit, Hkv), 8 warps: a CTA takes a quarter of a chunk's rows
+// for one kv head, a warp a row at a time over the kv group's q heads:
 //   RMSNorm backward   n = o rstd,  dn = dy w,  do = rstd (dn - n mean(dn n))
 //   A_t[c]  = sum_{h in group} do_t[c] (o_t[c] - P_tt v_t[c])
 //             the row part of dG_t without the s = t pair, whose counterpart
@@ -161,31 +162,23 @@ __global__ void __launch_bounds__(256) fwd_simt_kernel(
 //             dG = A - v dv_strict carries no cancelling diagonal terms
 //             (P_tt = exp(S_tt - m_t), S_tt recomputed from q_t, k_t)
 //   dw partials        sum_t dy_t n_t per CTA
-// and, for the tensor-core kernels (dot != NULL), a second pass writing the
-// row-scaled upstream gradients in the two references of the forward split,
-// as 16-bit MMA operands:
-//   dOt_t = do_t exp(L_t)          (key blocks before the query chunk): fp16
-//                                  when dsafe, else bf16
-//   dOm_t = do_t exp(L_t - rho)    (the diagonal block; 0 for channels outside
-//                                  the split's range): bf16 hi + lo
-// with dsafe[ci * Hq + h] = (the chunk is fp16-safe and max |do| <= FIX_F16_VMAX).
+//   hmax[ci * Hq + h]  max |do| over the chunk (float bits, atomicMax; zeroed
+//                      by the prefix pass), only for the tensor-core kernels.
 // Dynamic shared memory: grp floats.
 // ---------------------------------------------------------------------------
-constexpr int kPreWarps = 16;
+constexpr int kPreWarps = 8;
 
 __global__ void __launch_bounds__(kPreWarps * 32) bwd_pre_kernel(
     Dims d, const Chunk* __restrict__ chunks, const __nv_bfloat16* __restrict__ q,
     const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
     const float* __restrict__ o_s, const float* __restrict__ m_s,
     const float* __restrict__ rstd_s, const __nv_bfloat16* __restrict__ dy,
-    const __nv_bfloat16* __restrict__ w, const float* __restrict__ L,
-    const float* __restrict__ rho, const float* __restrict__ hr, const int* __restrict__ safe,
-    float* __restrict__ do_ws, uint16_t* __restrict__ dot, __nv_bfloat16* __restrict__ domh,
-    __nv_bfloat16* __restrict__ doml, int* __restrict__ dsafe, float* __restrict__ A,
-    float* __restrict__ dwpart) {
+    const __nv_bfloat16* __restrict__ w, float* __restrict__ do_ws, float* __restrict__ A,
+    float* __restrict__ dwpart, int* __restrict__ hmax_g) {
   __shared__ float red[kPreWarps][128];
   extern __shared__ float hmax[];   // [grp] max |do| per head
-  const int Dv = d.Dv, Dk = d.Dk, kv = blockIdx.y, ci = blockIdx.x;
+  const int Dv = d.Dv, Dk = d.Dk, kv = blockIdx.y;
+  const int ci = blockIdx.x / kPreSplit, sub = blockIdx.x % kPreSplit;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const Chunk ch = chunks[ci];
   for (int i = threadIdx.x; i < d.grp; i += blockDim.x) hmax[i] = 0.f;
@@ -199,7 +192,9 @@ __global__ void __launch_bounds__(kPreWarps * 32) bwd_pre_kernel(
   }
   const size_t ors = (size_t)d.Hq * Dv, vrs = (size_t)d.Hkv * Dv;
   const size_t qrs = (size_t)d.Hq * Dk, krs = (size_t)d.Hkv * Dk;
-  for (int r = warp; r < ch.len; r += kPreWarps) {
+  constexpr int kRows = FIX_CHUNK / kPreSplit;
+  const int rend = min(ch.len, (sub + 1) * kRows);
+  for (int r = sub * kRows + warp; r < rend; r += kPreWarps) {
     const size_t t = (size_t)ch.tok0 + r;
     float acc[4] = {0.f, 0.f, 0.f, 0.f}, vr[4], kr[4];
 #pragma unroll
@@ -211,24 +206,24 @@ __global__ void __launch_bounds__(kPreWarps * 32) bwd_pre_kernel(
     for (int hh = 0; hh < d.grp; ++hh) {
       const int h = kv * d.grp + hh;
       const float rs_ = rstd_s[t * d.Hq + h];
-      float sdot = 0.f;
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int c = lane + 32 * u;
-        if (c < Dk) sdot += bf2f(q[t * qrs + (size_t)h * Dk + c]) * kr[u];
-      }
-      const float ptt = expf(warp_sum(sdot) * d.scale - m_s[t * d.Hq + h]);
-      float ov[4], dn[4], n[4], dot_ = 0.f;
+      const float mt = m_s[t * d.Hq + h];
+      float sdot = 0.f, ov[4], dyv[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int c = lane + 32 * u;
         const size_t a = t * ors + (size_t)h * Dv + c;
+        if (c < Dk) sdot += bf2f(q[t * qrs + (size_t)h * Dk + c]) * kr[u];
         ov[u] = c < Dv ? o_s[a] : 0.f;
-        const float dyv = c < Dv ? bf2f(dy[a]) : 0.f;
+        dyv[u] = c < Dv ? bf2f(dy[a]) : 0.f;
+      }
+      const float ptt = expf(warp_sum(sdot) * d.scale - mt);
+      float dn[4], n[4], dot_ = 0.f;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
         n[u] = ov[u] * rs_;
-        dn[u] = dyv * wv[u];
+        dn[u] = dyv[u] * wv[u];
         dot_ += dn[u] * n[u];
-        dwl[u] += dyv * n[u];
+        dwl[u] += dyv[u] * n[u];
       }
       dot_ = warp_sum(dot_) / (float)Dv;
       float mx = 0.f;
@@ -241,7 +236,7 @@ __global__ void __launch_bounds__(kPreWarps * 32) bwd_pre_kernel(
         acc[u] += dov * (ov[u] - ptt * vr[u]);
         mx = fmaxf(mx, fabsf(dov));
       }
-      if (dot) {
+      if (hmax_g) {
         mx = warp_max(mx);
         if (lane == 0) atomicMax(reinterpret_cast<int*>(&hmax[hh]), __float_as_int(mx));
       }
@@ -260,13 +255,38 @@ __global__ void __launch_bounds__(kPreWarps * 32) bwd_pre_kernel(
     float sm = 0.f;
 #pragma unroll
     for (int i = 0; i < kPreWarps; ++i) sm += red[i][c0];
-    dwpart[((size_t)ci * d.Hkv + kv) * Dv + c0] = sm;
+    dwpart[((size_t)blockIdx.x * d.Hkv + kv) * Dv + c0] = sm;
   }
-  if (!dot) return;
-  // ---- second pass: 16-bit operands of the tensor-core kernels
+  if (hmax_g)
+    for (int i = threadIdx.x; i < d.grp; i += blockDim.x)
+      atomicMax(hmax_g + (size_t)ci * d.Hq + kv * d.grp + i, __float_as_int(hmax[i]));
+}
+
+// ---------------------------------------------------------------------------
+// Backward preprocess, pass 2 (tensor-core kernels only), same grid: the
+// row-scaled upstream gradients in the two references of the forward split,
+// as 16-bit MMA operands:
+//   dOt_t = do_t exp(L_t)          (key blocks before the query chunk): fp16
+//                                  when dsafe, else bf16
+//   dOm_t = do_t exp(L_t - rho)    (the diagonal block; 0 for channels outside
+//                                  the split's range): bf16 hi + lo
+// with dsafe[ci * Hq + h] = (the chunk is fp16-safe and max |do| <= FIX_F16_VMAX).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kPreWarps * 32) bwd_pre_ops_kernel(
+    Dims d, const Chunk* __restrict__ chunks, const float* __restrict__ L,
+    const float* __restrict__ rho, const float* __restrict__ hr, const int* __restrict__ safe,
+    const float* __restrict__ do_ws, const int* __restrict__ hmax_g, uint16_t* __restrict__ dot,
+    __nv_bfloat16* __restrict__ domh, __nv_bfloat16* __restrict__ doml, int* __restrict__ dsafe) {
+  const int Dv = d.Dv, kv = blockIdx.y;
+  const int ci = blockIdx.x / kPreSplit, sub = blockIdx.x % kPreSplit;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const Chunk ch = chunks[ci];
   const bool chunk_safe = safe[(size_t)ci * d.Hkv + kv] != 0;
-  for (int i = threadIdx.x; i < d.grp; i += blockDim.x)
-    dsafe[(size_t)ci * d.Hq + kv * d.grp + i] = (chunk_safe && hmax[i] <= FIX_F16_VMAX) ? 1 : 0;
+  if (sub == 0)
+    for (int i = threadIdx.x; i < d.grp; i += blockDim.x)
+      dsafe[(size_t)ci * d.Hq + kv * d.grp + i] =
+          (chunk_safe && __int_as_float(hmax_g[(size_t)ci * d.Hq + kv * d.grp + i]) <= FIX_F16_VMAX) ? 1 : 0;
+  const size_t ors = (size_t)d.Hq * Dv, vrs = (size_t)d.Hkv * Dv;
   float rh[4], good[4];
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
@@ -275,7 +295,9 @@ __global__ void __launch_bounds__(kPreWarps * 32) bwd_pre_kernel(
     rh[u] = c < Dv ? rho[ti] : 0.f;
     good[u] = (c < Dv && hr[ti] <= FIX_HR_MAX) ? 1.f : 0.f;
   }
-  for (int r = warp; r < ch.len; r += kPreWarps) {
+  constexpr int kRows = FIX_CHUNK / kPreSplit;
+  const int rend = min(ch.len, (sub + 1) * kRows);
+  for (int r = sub * kRows + warp; r < rend; r += kPreWarps) {
     const size_t t = (size_t)ch.tok0 + r;
     float lr[4];
 #pragma unroll
@@ -285,16 +307,22 @@ __global__ void __launch_bounds__(kPreWarps * 32) bwd_pre_kernel(
     }
     for (int hh = 0; hh < d.grp; ++hh) {
       const int h = kv * d.grp + hh;
-      const bool f16 = chunk_safe && hmax[hh] <= FIX_F16_VMAX;
+      const bool f16 =
+          chunk_safe && __int_as_float(hmax_g[(size_t)ci * d.Hq + h]) <= FIX_F16_VMAX;
+      float dov[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int c = lane + 32 * u;
+        dov[u] = c < Dv ? do_ws[t * ors + (size_t)h * Dv + c] : 0.f;
+      }
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int c = lane + 32 * u;
         if (c >= Dv) continue;
         const size_t a = t * ors + (size_t)h * Dv + c;
-        const float dov = do_ws[a];
-        const float xt = dov * expf(lr[u]);
+        const float xt = dov[u] * expf(lr[u]);
         dot[a] = f16 ? __half_as_ushort(__float2half_rn(xt)) : __bfloat16_as_ushort(f2bf(xt));
-        const float xm = good[u] != 0.f ? dov * expf(lr[u] - rh[u]) : 0.f;
+        const float xm = good[u] != 0.f ? dov[u] * expf(lr[u] - rh[u]) : 0.f;
         const __nv_bfloat16 hi = f2bf(xm);
         domh[a] = hi;
         doml[a] = f2bf(xm - bf2f(hi));
@@ -303,14 +331,35 @@ __global__ void __launch_bounds__(kPreWarps * 32) bwd_pre_kernel(
   }
 }
 
-// dw = sum of the partials in a fixed order (deterministic).  One CTA.
-__global__ void __launch_bounds__(128) dw_reduce_kernel(const float* __restrict__ parts, int nparts,
-                                                        int Dv, __nv_bfloat16* __restrict__ dw) {
-  const int c = threadIdx.x;
-  if (c >= Dv) return;
+// dw = sum of the partials in a fixed order (deterministic).  One CTA of 512
+// threads: 512 / Dv interleaved groups of partial rows, then the groups in
+// order.
+__global__ void __launch_bounds__(512) dw_reduce_kernel(const float* __restrict__ parts,
+                                                        int nparts, int Dv,
+                                                        __nv_bfloat16* __restrict__ dw) {
+  __shared__ float red[512];
+  const int groups = 512 / Dv;
+  const int c = threadIdx.x % Dv, grp = threadIdx.x / Dv;
   float s = 0.f;
-  for (int i = 0; i < nparts; ++i) s += parts[(size_t)i * Dv + c];
-  dw[c] = f2bf(s);
+  if (grp < groups) {
+    int i = grp;
+    for (; i + 3 * groups < nparts; i += 4 * groups) {
+      const float a = parts[(size_t)i * Dv + c], b = parts[(size_t)(i + groups) * Dv + c];
+      const float e = parts[(size_t)(i + 2 * groups) * Dv + c], f = parts[(size_t)(i + 3 * groups) * Dv + c];
+      s += a;
+      s += b;
+      s += e;
+      s += f;
+    }
+    for (; i < nparts; i += groups) s += parts[(size_t)i * Dv + c];
+  }
+  red[threadIdx.x] = s;
+  __syncthreads();
+  if (threadIdx.x < Dv) {
+    float t = 0.f;
+    for (int g = 0; g < groups; ++g) t += red[g * Dv + threadIdx.x];
+    dw[threadIdx.x] = f2bf(t);
+  }
 }
 
 // ---------------------------------------------------------------------------
