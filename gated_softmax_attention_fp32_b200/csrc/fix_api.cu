@@ -110,11 +110,15 @@ static SplitPlan plan_split(const fix_attn_problem* p, const Dims& d) {
   if (P < 4) P = 4;
   if (P > (1 << 30)) P = 1 << 30;
   sp.P = (int)P;
+  // the schedule kernel's split: per key chunk, its diagonal tiles and its
+  // later tiles, each in runs of at most P
   each_seq([&](long long L, long long mult) {
     const int nc = (int)((L + FIX_CHUNK - 1) / FIX_CHUNK);
     for (int j = 0; j < nc; ++j) {
-      const long long npj = ((long long)d.grp * tiles64_host(L, j) + P - 1) / P;
-      sp.nparts += mult * npj;
+      const long long h = fix_halves((int)L, j);
+      const long long nd = ((long long)d.grp * h + P - 1) / P;
+      const long long no = ((long long)d.grp * (tiles64_host(L, j) - h) + P - 1) / P;
+      sp.nparts += mult * (nd + no);
     }
   });
   sp.nslots = sp.nparts;   // every part writes its own slot
@@ -163,7 +167,7 @@ static Ws layout(const Dims& d, bool bwd, const SplitPlan& sp) {
     w.dwp = take((size_t)(d.nchunks > 0 ? d.nchunks : 1) * kPreSplit * d.Hkv * d.Dv * 4);
     w.parts = take((size_t)(sp.nparts > 0 ? sp.nparts : 1) * sizeof(Part));
     w.cpart = take((size_t)(d.nchunks > 0 ? d.nchunks : 1) * sizeof(int2));
-    w.partial = take((size_t)sp.nslots * d.Hkv * FIX_CHUNK * (d.Dk + 2 * d.Dv) * 4);
+    w.partial = take((size_t)sp.nslots * d.Hkv * FIX_CHUNK * (d.Dk + d.Dv) * 4);
   }
   w.total = o;
   return w;

@@ -37,15 +37,22 @@ struct Chunk {
   int nch;
 };
 
-// One CTA's share of a key chunk's backward work: the key chunk, the index p
-// of its run of (at most `tiles_per_part`) 64-row query tiles, and the slot of
-// its fp32 partial sums in the partial buffer.
+// One CTA's share of a key chunk's backward work: the key chunk, the kind of
+// query tiles (diag = 1: those of the chunk itself, else those of later
+// chunks), the index p of its run of (at most `tiles_per_part`) 64-row tiles
+// of that kind, and the slot of its fp32 partial sums in the partial buffer.
 struct Part {
   int ci;
   int p;
   int slot;
-  int pad;
+  int diag;
 };
+
+// 64-row halves of chunk j of a sequence of L tokens.
+__device__ __host__ inline int fix_halves(int L, int j) {
+  const int len = L - j * FIX_CHUNK < FIX_CHUNK ? L - j * FIX_CHUNK : FIX_CHUNK;
+  return (len + 63) / 64;
+}
 
 // Where the schedule kernel writes the dk/dv work split (parts == NULL: none).
 struct PartSpec {
@@ -53,7 +60,8 @@ struct PartSpec {
   int tiles_per_part; // P
   int cap_parts;      // entries of parts[]
   Part* parts;
-  int2* cpart;        // per chunk: {number of parts, first slot}
+  int2* cpart;        // per chunk: {number of parts, first slot}; slots are
+                      // consecutive, the diagonal parts' first
 };
 
 struct Dims {

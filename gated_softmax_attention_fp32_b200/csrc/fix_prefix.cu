@@ -124,41 +124,61 @@ __global__ void __launch_bounds__(1024) schedule_kernel(const int64_t* __restric
     order_chunks(out, cap, maxj, order);
   }
   if (!ps.parts) return;
-  // dk/dv work split: key chunk j of a sequence has grp * tiles64_from(L, j)
-  // tiles, cut into ceil(tiles / P) parts
-  int cbase = 0, pbase = 0, sbase = 0;
+  // dk/dv work split: key chunk j of a sequence of L tokens has grp * h_j
+  // diagonal tiles (h_j = its 64-row halves) and grp * (tiles64_from(L, j) -
+  // h_j) later ones, each kind cut into runs of at most P tiles.  parts[]
+  // holds every later-block part first (the long ones start first), then the
+  // diagonal parts; a key chunk's slots are consecutive, diagonal parts first.
+  auto seq_len = [&](int i) -> int {
+    if (i >= nseq) return 0;
+    if (!cu) return T;
+    long long s0 = cu[i];
+    const long long e = cu[i + 1];
+    s0 = s0 < 0 ? 0 : (s0 > N ? N : s0);
+    const long long L = (e > N ? N : e) - s0;
+    return L < 0 ? 0 : (int)L;
+  };
+  const int P = ps.tiles_per_part;
+  auto n_diag = [&](int L, int j) { return (ps.grp * fix_halves(L, j) + P - 1) / P; };
+  auto n_off = [&](int L, int j) {
+    return (ps.grp * (tiles64_from(L, j) - fix_halves(L, j)) + P - 1) / P;
+  };
+  int total_off = 0;
   for (int first = 0; first < nseq; first += blockDim.x) {
-    const int i = first + threadIdx.x;
-    int L = 0;
-    if (i < nseq) {
-      if (cu) {
-        long long s0 = cu[i];
-        const long long e = cu[i + 1];
-        s0 = s0 < 0 ? 0 : (s0 > N ? N : s0);
-        L = (int)((e > N ? N : e) - s0);
-        if (L < 0) L = 0;
-      } else {
-        L = T;
-      }
-    }
+    const int L = seq_len(first + threadIdx.x);
     const int nc = (L + FIX_CHUNK - 1) / FIX_CHUNK;
-    int np = 0;
-    for (int j = 0; j < nc; ++j)
-      np += (ps.grp * tiles64_from(L, j) + ps.tiles_per_part - 1) / ps.tiles_per_part;
-    const int ns = np;   // every part owns a slot of the partial buffer
-    int ctot, ptot, stot;
+    int no = 0;
+    for (int j = 0; j < nc; ++j) no += n_off(L, j);
+    int t;
+    block_excl_scan(no, scan, &t);
+    total_off += t;
+  }
+  int cbase = 0, obase = 0, dbase = 0, sbase = 0;
+  for (int first = 0; first < nseq; first += blockDim.x) {
+    const int L = seq_len(first + threadIdx.x);
+    const int nc = (L + FIX_CHUNK - 1) / FIX_CHUNK;
+    int no = 0, nd = 0;
+    for (int j = 0; j < nc; ++j) {
+      no += n_off(L, j);
+      nd += n_diag(L, j);
+    }
+    int ctot, otot, dtot, stot;
     const int c0 = cbase + block_excl_scan(nc, scan, &ctot);
-    const int p0 = pbase + block_excl_scan(np, scan, &ptot);
-    int s0 = sbase + block_excl_scan(ns, scan, &stot);
-    int e = p0;
+    int o = obase + block_excl_scan(no, scan, &otot);
+    int e = total_off + dbase + block_excl_scan(nd, scan, &dtot);
+    int s0 = sbase + block_excl_scan(no + nd, scan, &stot);
     for (int j = 0; j < nc && c0 + j < cap; ++j) {
-      const int npj = (ps.grp * tiles64_from(L, j) + ps.tiles_per_part - 1) / ps.tiles_per_part;
-      ps.cpart[c0 + j] = make_int2(npj, s0);
-      for (int p = 0; p < npj && e < ps.cap_parts; ++p, ++e) ps.parts[e] = Part{c0 + j, p, s0 + p, 0};
-      s0 += npj;
+      const int ndj = n_diag(L, j), noj = n_off(L, j);
+      ps.cpart[c0 + j] = make_int2(ndj + noj, s0);
+      for (int p = 0; p < ndj; ++p, ++e)
+        if (e < ps.cap_parts) ps.parts[e] = Part{c0 + j, p, s0 + p, 1};
+      for (int p = 0; p < noj; ++p, ++o)
+        if (o < ps.cap_parts) ps.parts[o] = Part{c0 + j, p, s0 + ndj + p, 0};
+      s0 += ndj + noj;
     }
     cbase += ctot;
-    pbase += ptot;
+    obase += otot;
+    dbase += dtot;
     sbase += stot;
   }
 }

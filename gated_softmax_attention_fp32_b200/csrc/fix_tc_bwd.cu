@@ -19,14 +19,17 @@
 // dq kernel (one CTA per 128-row query chunk and q head, key blocks i..0):
 //   S = Q K^T and dP = dO V'^T into TMEM, dS = P dP (fp32, then bf16, written
 //   over S), dQ += dS K.  V' = Vt f_ij is formed in shared memory per block.
-// dk/dv kernel (one CTA per 128-row key chunk and kv head; the group's q heads
-// and 64-row query tiles of every later chunk stream through):
+// dk/dv kernel (one CTA per kv head and part of a 128-row key chunk's work:
+// either its diagonal query tiles or a run of the 64-row query tiles of later
+// chunks, over the group's q heads):
 //   S^T = K Q^T, dP^T = V X^T (X = dOt f_ij, or dOm on the diagonal),
 //   dV += P^T X, dK += dS^T Q.  On the diagonal, whose terms dominate dv and
 //   whose rounding would dominate dG, P and dOm are split into bf16 hi + lo
-//   parts (three MMAs into their own accumulator dV_d); elsewhere one MMA in
-//   fp16 when every gate <= 0 and |v|, |do| <= 3e4, else bf16, into dV_o.
-//   Epilogue: dv_strict = exp(rho - L_s) dV_d + exp(tot_j - L_s) dV_o,
+//   parts (three MMAs, accumulated as dV_d); elsewhere one MMA in fp16 when
+//   every gate <= 0 and |v|, |do| <= 3e4, else bf16 (accumulated as dV_o).
+//   Each part writes its fp32 dK and dV to a slot; the combine kernel adds a
+//   key chunk's slots in order and finishes
+//   dv_strict = exp(rho - L_s) dV_d + exp(tot_j - L_s) dV_o,
 //   dv = dv_strict + sum_h P_ss do_s, dG = A - v dv_strict, dk = scale dK.
 // Problems with a channel outside the split's float range (flag set by the
 // prefix pass) are left to the exact CUDA-core kernels, which run instead.
@@ -69,7 +72,7 @@ struct Params {
   const int2* cpart;
   int tiles_per_part;
   long long nslots;         // rows of `partial` per kv head, in units of 128-row slots
-  float* partial;           // partial dK | dV_d | dV_o rows of split key chunks
+  float* partial;           // [slot][kv][128 rows][dK | dV] fp32 sums of the dk/dv parts
   __nv_bfloat16* dq;
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
@@ -345,7 +348,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int kChunks = DV / 8;
     constexpr int kRowsPerPass = 128 / kChunks;
     const int lc = dt % kChunks, r0 = dt / kChunks;
-    const size_t ors = (size_t)d.Hq * DV;
     // dO operand (loaded by TMA): dOm (bf16) for the diagonal block, then dOt,
     // converted in place when its storage type differs from the CTA's
     for (int phase = 0; phase < (nblk > 1 ? 2 : 1); ++phase) {
@@ -409,35 +411,40 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ========================================================================= dk/dv
 
-constexpr int BQ = 64;   // query rows per streamed tile
+constexpr int BQ = 64;         // query rows per streamed tile
+constexpr int kQStages = 3;    // Q / X tiles in flight
 
 struct KvBars {
   uint64_t kv_full;
-  uint64_t q_full[2], q_empty[2], x_ready[2];
-  uint64_t s_full, p_ready, done, drain;
+  uint64_t q_full[kQStages], q_empty[kQStages], x_ready[kQStages];
+  uint64_t s_full[2], p_ready[2], done, drain;
 };
 
 template <int DK, int DV>
 struct KvLayout {
-  static constexpr int kK = 0;                         // [128][DK]
-  static constexpr int kVt = kK + BN * DK * 2;         // [128][DV] Vt
-  static constexpr int kVm = kVt + BN * DV * 2;        // [128][DV] Vm (hi)
-  static constexpr int kQ = kVm + BN * DV * 2;         // 2 x [64][DK]
-  static constexpr int kX = kQ + 2 * BQ * DK * 2;      // 2 x [64][DV]
-  static constexpr int kXl = kX + 2 * BQ * DV * 2;     // 2 x [64][DV] (diagonal lo part)
-  static constexpr int kM = kXl + 2 * BQ * DV * 2;     // 2 x [64] f32 row max
-  static constexpr int kBars = kM + 2 * BQ * 4;
+  static constexpr int kK = 0;                              // [128][DK]
+  static constexpr int kV = kK + BN * DK * 2;               // [128][DV] Vm (diagonal) or Vt
+  static constexpr int kQ = kV + BN * DV * 2;               // stages x [64][DK]
+  static constexpr int kX = kQ + kQStages * BQ * DK * 2;    // stages x [64][DV]
+  static constexpr int kXl = kX + kQStages * BQ * DV * 2;   // stages x [64][DV] (diagonal lo part)
+  static constexpr int kM = kXl + kQStages * BQ * DV * 2;   // stages x [64] f32 row max
+  static constexpr int kBars = kM + kQStages * BQ * 4;
   static constexpr int kTmem = kBars + (int)sizeof(KvBars);
   static constexpr int kAbort = kTmem + 4;
   static constexpr int kAlloc = kAbort + 4 + 1024;
 };
 
-// The tiles a dk/dv CTA streams, in order: for each q head of the group, for
-// each query chunk i >= j, the 64-row halves that hold rows.
+// A dk/dv CTA streams the tiles of one kind: the diagonal ones (query chunk
+// i = j) or the later ones (i > j); in order, for each q head of the group,
+// for each query chunk, the 64-row halves that hold rows.
 struct TileIter {
   int hh, i, half;
 };
 
+// One CTA per (part, kv head).  TMEM: S^T and dP^T double-buffered (128
+// columns per buffer: S [0, 64), dP [64, 128)), the dV accumulator at 256 and
+// dK at 256 + DV.  The MMA warp issues S / dP of tile n + 2 right after dV /
+// dK of tile n, so the softmax of one buffer overlaps the MMAs of the other.
 template <int DK, int DV>
 __global__ void __launch_bounds__(kThreads, 1)
     dkv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -455,21 +462,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int kv = blockIdx.x % d.Hkv;
   const int cj = pt.ci;
   const Chunk ch = P.chunks[cj];
-  if (ch.len <= 0) return;
+  const bool dmode = pt.diag != 0;
   const int first = cj - ch.j;
-  const int nq_chunks = ch.nch - ch.j;                 // chunks i = j .. nch-1
-  // tiles per head: every chunk after j has 128 rows except possibly the last
   auto chunk_len = [&](int i) { return P.chunks[first + i].len; };
+  const int i0 = dmode ? ch.j : ch.j + 1, i1 = dmode ? ch.j + 1 : ch.nch;   // query chunks
   int tiles_per_head = 0;
-  for (int i = ch.j; i < ch.nch; ++i) tiles_per_head += (chunk_len(i) + BQ - 1) / BQ;
-  // this CTA's run of tiles
+  for (int i = i0; i < i1; ++i) tiles_per_head += (chunk_len(i) + BQ - 1) / BQ;
   const int t_begin = pt.p * P.tiles_per_part;
-  const int ntiles = min(P.tiles_per_part, tiles_per_head * d.grp - t_begin);
-  if (ntiles <= 0) return;
+  const int ntiles = ch.len > 0 ? min(P.tiles_per_part, tiles_per_head * d.grp - t_begin) : 0;
+  constexpr int kCols = DK + DV;
+  if (ntiles <= 0) {
+    // nothing to stream (only for a chunk table that disagrees with the
+    // host's plan): the slot still has to read as zero
+    if (pt.slot >= 0 && pt.slot < P.nslots) {
+      float* dst = P.partial + ((size_t)pt.slot * d.Hkv + kv) * BN * kCols;
+      for (int i = tid; i < BN * kCols; i += blockDim.x) dst[i] = 0.f;
+    }
+    return;
+  }
 
   uint8_t* sK = smem + Lay::kK;
-  uint8_t* sVt = smem + Lay::kVt;
-  uint8_t* sVm = smem + Lay::kVm;
+  uint8_t* sV = smem + Lay::kV;
   uint8_t* sQ = smem + Lay::kQ;
   uint8_t* sX = smem + Lay::kX;
   uint8_t* sXl = smem + Lay::kXl;
@@ -482,44 +495,51 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid == 0) {
     *sAbort = 0;
     mbar_init(&bar->kv_full, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kQStages; ++s) {
       mbar_init(&bar->q_full[s], 1);
       mbar_init(&bar->q_empty[s], 1);
       mbar_init(&bar->x_ready[s], 128);
     }
-    mbar_init(&bar->s_full, 1);
-    mbar_init(&bar->p_ready, 128);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bar->s_full[b], 1);
+      mbar_init(&bar->p_ready[b], 128);
+    }
     mbar_init(&bar->done, 1);
     mbar_init(&bar->drain, 1);
     mbar_fence_init();
   }
   if (warp == 1) tmem_alloc(sTmem, kTmemCols);
-  bool my_safe = true;
-  for (int i = tid; i < nq_chunks; i += blockDim.x) {
-    my_safe = my_safe && P.safe[(size_t)(first + ch.j + i) * d.Hkv + kv];
-    for (int hh = 0; hh < d.grp; ++hh)
-      my_safe = my_safe && P.dsafe[(size_t)(first + ch.j + i) * d.Hq + kv * d.grp + hh];
-  }
+  // operand type of the later-block MMAs: fp16 when every chunk they span is
+  // fp16-safe for this kv head and its q heads (the diagonal ones are bf16)
+  bool my_safe = !dmode;
+  if (!dmode)
+    for (int i = tid; i < ch.nch - ch.j; i += blockDim.x) {
+      my_safe = my_safe && P.safe[(size_t)(first + ch.j + i) * d.Hkv + kv];
+      for (int hh = 0; hh < d.grp; ++hh)
+        my_safe = my_safe && P.dsafe[(size_t)(first + ch.j + i) * d.Hq + kv * d.grp + hh];
+    }
   tc_fence_before();
   const int cta_f16 = __syncthreads_and(my_safe);
   tc_fence_after();
   const uint32_t tmem = *sTmem;
-  constexpr uint32_t kColS = 0, kColP = 64, kColVd = 128, kColVo = 128 + DV, kColK = 128 + 2 * DV;
+  constexpr uint32_t kColV = 256, kColK = 256 + DV;
+  static_assert(256 + DV + DK <= (int)kTmemCols, "TMEM columns");
+  auto col_s = [](int b) { return (uint32_t)(b * 128); };
+  auto col_p = [](int b) { return (uint32_t)(b * 128 + 64); };
 
   // walk the tile sequence (identical in every role)
   auto next_tile = [&](TileIter& t) {
     ++t.half;
     if (t.half * BQ >= chunk_len(t.i)) {
       t.half = 0;
-      ++t.i;
-      if (t.i >= ch.nch) {
-        t.i = ch.j;
+      if (++t.i >= i1) {
+        t.i = i0;
         ++t.hh;
       }
     }
   };
   auto tile_at = [&](int n) {
-    TileIter t{0, ch.j, 0};
+    TileIter t{0, i0, 0};
     for (int q = 0; q < n; ++q) next_tile(t);
     return t;
   };
@@ -527,103 +547,104 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      mbar_expect_tx(&bar->kv_full, BN * DK * 2 + 2 * BN * DV * 2);
+      mbar_expect_tx(&bar->kv_full, BN * DK * 2 + BN * DV * 2);
       for (int hh = 0; hh < DK / 64; ++hh)
         tma_load_3d(sK + hh * BN * 128, &tm_k, &bar->kv_full, hh * 64, kv, ch.tok0);
-      for (int hh = 0; hh < DV / 64; ++hh) {
-        tma_load_3d(sVt + hh * BN * 128, &tm_vt, &bar->kv_full, hh * 64, kv, ch.tok0);
-        tma_load_3d(sVm + hh * BN * 128, &tm_vm, &bar->kv_full, hh * 64, kv, ch.tok0);
-      }
+      for (int hh = 0; hh < DV / 64; ++hh)
+        tma_load_3d(sV + hh * BN * 128, dmode ? &tm_vm : &tm_vt, &bar->kv_full, hh * 64, kv, ch.tok0);
       TileIter t = tile_at(t_begin);
       int nq = 0;
       for (int n = 0; n < ntiles; ++n, next_tile(t)) {
-        const int st = n & 1;
-        const bool diag = t.i == ch.j;
-        if (n >= 2 && !mbar_wait(&bar->q_empty[st], ((n >> 1) & 1) ^ 1, ctl)) break;
+        const int st = n % kQStages;
+        if (n >= kQStages && !mbar_wait(&bar->q_empty[st], ((n / kQStages) & 1) ^ 1, ctl)) break;
         // Q tile and the X operand (dOm hi + lo on the diagonal, dOt elsewhere)
-        mbar_expect_tx(&bar->q_full[st], BQ * DK * 2 + (diag ? 2 : 1) * BQ * DV * 2);
+        mbar_expect_tx(&bar->q_full[st], BQ * DK * 2 + (dmode ? 2 : 1) * BQ * DV * 2);
         const int h = kv * d.grp + t.hh;
         const int qtok = P.chunks[first + t.i].tok0 + t.half * BQ;
         for (int hh = 0; hh < DK / 64; ++hh)
           tma_load_3d(sQ + st * BQ * DK * 2 + hh * BQ * 128, &tm_q, &bar->q_full[st], hh * 64, h, qtok);
         for (int hh = 0; hh < DV / 64; ++hh) {
-          tma_load_3d(sX + st * BQ * DV * 2 + hh * BQ * 128, diag ? &tm_domh : &tm_dot,
+          tma_load_3d(sX + st * BQ * DV * 2 + hh * BQ * 128, dmode ? &tm_domh : &tm_dot,
                       &bar->q_full[st], hh * 64, h, qtok);
-          if (diag)
+          if (dmode)
             tma_load_3d(sXl + st * BQ * DV * 2 + hh * BQ * 128, &tm_doml, &bar->q_full[st], hh * 64,
                         h, qtok);
         }
         ++nq;
       }
       const Ctl drain{P.status, nullptr};
-      for (int n = nq - 1; n >= 0 && n >= nq - 2; --n)
-        mbar_wait(&bar->q_full[n & 1], (n >> 1) & 1, drain);
+      for (int n = nq - 1; n >= 0 && n >= nq - kQStages; --n)
+        mbar_wait(&bar->q_full[n % kQStages], (n / kQStages) & 1, drain);
       mbar_wait(&bar->kv_full, 0, drain);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16(128, BQ, false, false);
-      const uint32_t idesc_dp_off = idesc_bf16(128, BQ, false, false, cta_f16 != 0);
-      constexpr uint32_t idesc_dp_diag = idesc_bf16(128, BQ, false, false);
-      const uint32_t idesc_dv_off = idesc_bf16(128, DV, false, true, cta_f16 != 0);
-      constexpr uint32_t idesc_dv_diag = idesc_bf16(128, DV, false, true);
+      const uint32_t idesc_dp = idesc_bf16(128, BQ, false, false, cta_f16 != 0);
+      const uint32_t idesc_dv = idesc_bf16(128, DV, false, true, cta_f16 != 0);
       constexpr uint32_t idesc_dk = idesc_bf16(128, DK, false, true);
-      const uint32_t k_addr = smem_u32(sK), vt_addr = smem_u32(sVt), vm_addr = smem_u32(sVm);
+      const uint32_t k_addr = smem_u32(sK), v_addr = smem_u32(sV);
       bool ok = mbar_wait(&bar->kv_full, 0, ctl);
-      bool first_diag = true, first_off = true;
-      TileIter t = tile_at(t_begin);
-      for (int n = 0; ok && n < ntiles; ++n, next_tile(t)) {
-        const int st = n & 1;
-        const uint32_t ph = (n >> 1) & 1;
-        const bool diag = t.i == ch.j;
-        if (!mbar_wait(&bar->q_full[st], ph, ctl) || !mbar_wait(&bar->x_ready[st], ph, ctl)) break;
+      // the operand warps may convert V in place after kv_full; every
+      // x_ready covers their writes
+      auto issue_sdp = [&](int n) -> bool {
+        const int st = n % kQStages, b = n & 1;
+        const uint32_t ph = (n / kQStages) & 1;
+        if (!mbar_wait(&bar->q_full[st], ph, ctl) || !mbar_wait(&bar->x_ready[st], ph, ctl))
+          return false;
         tc_fence_after();
         const uint32_t q_addr = smem_u32(sQ + st * BQ * DK * 2);
         const uint32_t x_addr = smem_u32(sX + st * BQ * DV * 2);
-        const uint32_t xl_addr = smem_u32(sXl + st * BQ * DV * 2);
         // S^T = K Q^T   (M = 128 keys, N = 64 queries, K = DK)
 #pragma unroll
         for (int kk = 0; kk < DK / 16; ++kk) {
           const uint32_t ka = (kk >> 2) * (BN * 128) + (kk & 3) * 32;
           const uint32_t qa = (kk >> 2) * (BQ * 128) + (kk & 3) * 32;
-          mma_ss(tmem + kColS, desc_sw128(k_addr + ka, 16, 1024), desc_sw128(q_addr + qa, 16, 1024),
+          mma_ss(tmem + col_s(b), desc_sw128(k_addr + ka, 16, 1024), desc_sw128(q_addr + qa, 16, 1024),
                  idesc_s, kk > 0);
         }
-        // dP^T = V X^T  (V = Vm on the diagonal, Vt elsewhere)
-        const uint32_t va = diag ? vm_addr : vt_addr;
+        // dP^T = V X^T
 #pragma unroll
         for (int kk = 0; kk < DV / 16; ++kk) {
           const uint32_t vo = (kk >> 2) * (BN * 128) + (kk & 3) * 32;
           const uint32_t xo = (kk >> 2) * (BQ * 128) + (kk & 3) * 32;
-          mma_ss(tmem + kColP, desc_sw128(va + vo, 16, 1024), desc_sw128(x_addr + xo, 16, 1024),
-                 diag ? idesc_dp_diag : idesc_dp_off, kk > 0);
+          mma_ss(tmem + col_p(b), desc_sw128(v_addr + vo, 16, 1024), desc_sw128(x_addr + xo, 16, 1024),
+                 idesc_dp, kk > 0);
         }
-        tc_commit(&bar->s_full);
-        if (!mbar_wait(&bar->p_ready, n & 1, ctl)) break;
+        tc_commit(&bar->s_full[b]);
+        return true;
+      };
+      if (ok) ok = issue_sdp(0);
+      if (ok && ntiles > 1) ok = issue_sdp(1);
+      for (int n = 0; ok && n < ntiles; ++n) {
+        const int st = n % kQStages, b = n & 1;
+        if (!mbar_wait(&bar->p_ready[b], (n >> 1) & 1, ctl)) break;
         tc_fence_after();
-        // dV += P^T X  (K = 64 queries; X read MN-major)
+        const uint32_t q_addr = smem_u32(sQ + st * BQ * DK * 2);
+        const uint32_t x_addr = smem_u32(sX + st * BQ * DV * 2);
+        const uint32_t xl_addr = smem_u32(sXl + st * BQ * DV * 2);
+        // dV += P^T X  (K = 64 queries; X read MN-major); on the diagonal
+        // P_hi X_hi + P_lo X_hi + P_hi X_lo
 #pragma unroll
         for (int kk = 0; kk < BQ / 16; ++kk) {
           const uint64_t bx = desc_sw128(x_addr + kk * 2048, BQ * 128, 1024);
-          if (diag) {
+          mma_ts(tmem + kColV, tmem + col_s(b) + kk * 8, bx, idesc_dv, !(n == 0 && kk == 0));
+          if (dmode) {
             const uint64_t bxl = desc_sw128(xl_addr + kk * 2048, BQ * 128, 1024);
-            mma_ts(tmem + kColVd, tmem + kColS + kk * 8, bx, idesc_dv_diag, !(first_diag && kk == 0));
-            mma_ts(tmem + kColVd, tmem + kColS + 32 + kk * 8, bx, idesc_dv_diag, 1);
-            mma_ts(tmem + kColVd, tmem + kColS + kk * 8, bxl, idesc_dv_diag, 1);
-          } else {
-            mma_ts(tmem + kColVo, tmem + kColS + kk * 8, bx, idesc_dv_off, !(first_off && kk == 0));
+            mma_ts(tmem + kColV, tmem + col_s(b) + 32 + kk * 8, bx, idesc_dv, 1);
+            mma_ts(tmem + kColV, tmem + col_s(b) + kk * 8, bxl, idesc_dv, 1);
           }
         }
         // dK += dS^T Q
 #pragma unroll
         for (int kk = 0; kk < BQ / 16; ++kk) {
           const uint64_t bq = desc_sw128(q_addr + kk * 2048, BQ * 128, 1024);
-          mma_ts(tmem + kColK, tmem + kColP + kk * 8, bq, idesc_dk, !(n == 0 && kk == 0));
+          mma_ts(tmem + kColK, tmem + col_p(b) + kk * 8, bq, idesc_dk, !(n == 0 && kk == 0));
         }
-        if (diag) first_diag = false;
-        else first_off = false;
         tc_commit(&bar->q_empty[st]);
+        // tile n + 2 reuses buffer b: its MMAs run after the ones above
+        if (n + 2 < ntiles) ok = issue_sdp(n + 2);
       }
       tc_commit(&bar->done);
       tc_commit(&bar->drain);
@@ -637,25 +658,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     TileIter t = tile_at(t_begin);
     for (int n = 0; n < ntiles; ++n, next_tile(t)) {
-      const int st = n & 1;
-      const bool diag = t.i == ch.j;
+      const int st = n % kQStages, b = n & 1;
       const int qlen = min(BQ, chunk_len(t.i) - t.half * BQ);
-      if (!__all_sync(0xffffffffu, mbar_wait(&bar->s_full, n & 1, ctl))) { ok = false; break; }
+      // x_ready covers the row maxima of this tile in sM
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar->s_full[b], (n >> 1) & 1, ctl) &&
+                                       mbar_wait(&bar->x_ready[st], (n / kQStages) & 1, ctl))) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
       const float* mrow = sM + st * BQ;
-      const bool full = !diag && qlen == BQ;
-      const int lo = diag ? s - t.half * BQ : 0;   // first valid query column
+      const bool full = !dmode && qlen == BQ;
+      const int lo = dmode ? s - t.half * BQ : 0;   // first valid query column
       // two halves of 32 query columns; a half's packed P and dS go over
       // columns of S and dP that the half has already read
       uint32_t pl[32];
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         uint32_t xs[32], xp[32], ph[16], pd[16];
-        tmem_ld32(lane_base + kColS + 32 * h, xs);
-        tmem_ld32(lane_base + kColP + 32 * h, xp);
+        tmem_ld32(lane_base + col_s(b) + 32 * h, xs);
+        tmem_ld32(lane_base + col_p(b) + 32 * h, xp);
         tmem_wait_ld();
         if (full) {
-          // full off-diagonal tile: no masking
+          // full later tile: no masking
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
             const float p0 = ex2(__uint_as_float(xs[e]) * c1 - mrow[32 * h + e] * LOG2E);
@@ -674,9 +699,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               const int qi = 32 * h + e + u;
               const bool valid = qi >= lo && qi < qlen;
               p[u] = valid ? ex2(__uint_as_float(xs[e + u]) * c1 - mrow[qi] * LOG2E) : 0.f;
-              pv[u] = (diag && qi == lo) ? 0.f : p[u];
+              pv[u] = (dmode && qi == lo) ? 0.f : p[u];
             }
-            if (diag) {
+            if (dmode) {
               ph[e >> 1] = pack_bf16(pv[0], pv[1]);
               const float h0 = __uint_as_float(ph[e >> 1] << 16);
               const float h1 = __uint_as_float(ph[e >> 1] & 0xFFFF0000u);
@@ -687,83 +712,56 @@ __global__ void __launch_bounds__(kThreads, 1)
             pd[e >> 1] = pack_bf16(p[0] * __uint_as_float(xp[e]), p[1] * __uint_as_float(xp[e + 1]));
           }
         }
-        tmem_st16(lane_base + kColS + 16 * h, ph);
-        tmem_st16(lane_base + kColP + 16 * h, pd);
+        tmem_st16(lane_base + col_s(b) + 16 * h, ph);
+        tmem_st16(lane_base + col_p(b) + 16 * h, pd);
       }
       // the low parts go over S columns [32, 64), read by the second half
-      if (diag) tmem_st32(lane_base + kColS + 32, pl);
+      if (dmode) tmem_st32(lane_base + col_s(b) + 32, pl);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&bar->p_ready);
+      mbar_arrive(&bar->p_ready[b]);
     }
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bar->done, 0, ctl));
     tc_fence_after();
     // ---------------------------------------------------------- epilogue
-    // which accumulators this CTA's tiles wrote
-    bool has_diag = false, has_off = false;
-    {
-      TileIter u = tile_at(t_begin);
-      for (int n = 0; n < ntiles; ++n, next_tile(u)) {
-        if (u.i == ch.j) has_diag = true;
-        else has_off = true;
-      }
-    }
-    // The CTA's raw sums (dK | dV_d | dV_o, fp32, a row per key) go to its
-    // slot of the partial buffer; the combine kernel adds the slots of a key
-    // chunk in order and finishes dk, dv and dG.  Each thread stages its row,
-    // one segment at a time, in the operand buffers (free once every MMA has
+    // The CTA's raw sums (dK | dV, fp32, a row per key) go to its slot of the
+    // partial buffer; the combine kernel adds the slots of a key chunk in
+    // order and finishes dk, dv and dG.  Each thread stages its row, one
+    // segment at a time, in the operand buffers (free once every MMA has
     // completed) and sends it with its own bulk copy.  Staged rows are padded
-    // by 16 bytes so that eight consecutive rows start on distinct banks; two
-    // buffers alternate.
-    constexpr int kCols = DK + 2 * DV;
-    constexpr int kPad0 = (DK > DV ? DK : DV) + 4;     // staged row strides, floats
-    constexpr int kPad1 = DV + 4;
-    static_assert(BN * (kPad0 + kPad1) * 4 <= Lay::kM, "two staging buffers must fit");
+    // by 16 bytes so that eight consecutive rows start on distinct banks.
+    constexpr int kPad0 = DK + 4, kPad1 = DV + 4;     // staged row strides, floats
+    static_assert(BN * (kPad0 + kPad1) * 4 <= Lay::kM, "staging buffers must fit");
     if (ok && pt.slot >= 0 && pt.slot < P.nslots) {
       float* grow = P.partial + (((size_t)pt.slot * d.Hkv + kv) * BN + s) * kCols;
-      float* buf[2] = {reinterpret_cast<float*>(smem) + (size_t)s * kPad0,
-                       reinterpret_cast<float*>(smem) + (size_t)BN * kPad0 + (size_t)s * kPad1};
-      auto stage32 = [&](float* dst, const uint32_t (&x)[32], bool keep) {
+      float* b0 = reinterpret_cast<float*>(smem) + (size_t)s * kPad0;
+      float* b1 = reinterpret_cast<float*>(smem) + (size_t)BN * kPad0 + (size_t)s * kPad1;
+      auto stage32 = [&](float* dst, const uint32_t (&x)[32]) {
 #pragma unroll
         for (int e = 0; e < 32; e += 4)
           *reinterpret_cast<float4*>(dst + e) =
-              keep ? make_float4(__uint_as_float(x[e]), __uint_as_float(x[e + 1]),
-                                 __uint_as_float(x[e + 2]), __uint_as_float(x[e + 3]))
-                   : make_float4(0.f, 0.f, 0.f, 0.f);
+              make_float4(__uint_as_float(x[e]), __uint_as_float(x[e + 1]),
+                          __uint_as_float(x[e + 2]), __uint_as_float(x[e + 3]));
       };
-      // dK -> buffer 0
 #pragma unroll
       for (int cc = 0; cc < DK / 32; ++cc) {
         uint32_t x[32];
         tmem_ld32(lane_base + kColK + cc * 32, x);
         tmem_wait_ld();
-        stage32(buf[0] + cc * 32, x, true);
+        stage32(b0 + cc * 32, x);
       }
       fence_proxy_async_smem();
-      bulk_store(grow, buf[0], DK * 4);
+      bulk_store(grow, b0, DK * 4);
       bulk_commit();
-      // dV_d -> buffer 1
 #pragma unroll
       for (int cc = 0; cc < DV / 32; ++cc) {
         uint32_t x[32];
-        tmem_ld32(lane_base + kColVd + cc * 32, x);
+        tmem_ld32(lane_base + kColV + cc * 32, x);
         tmem_wait_ld();
-        stage32(buf[1] + cc * 32, x, has_diag);
+        stage32(b1 + cc * 32, x);
       }
       fence_proxy_async_smem();
-      bulk_store(grow + DK, buf[1], DV * 4);
-      bulk_commit();
-      // dV_o -> buffer 0, once the dK copy has read it
-      bulk_wait_read<1>();
-#pragma unroll
-      for (int cc = 0; cc < DV / 32; ++cc) {
-        uint32_t x[32];
-        tmem_ld32(lane_base + kColVo + cc * 32, x);
-        tmem_wait_ld();
-        stage32(buf[0] + cc * 32, x, has_off);
-      }
-      fence_proxy_async_smem();
-      bulk_store(grow + DK + DV, buf[0], DV * 4);
+      bulk_store(grow + DK, b1, DV * 4);
       bulk_commit();
       bulk_wait_read<0>();
     }
@@ -773,53 +771,53 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int kChunks = DV / 8;
     constexpr int kRowsPerPass = 128 / kChunks;
     const int lc = dt % kChunks, r0 = dt / kChunks;
-    const size_t ors = (size_t)d.Hq * DV;
-    // Vt arrives in its chunk's storage type; the off-diagonal MMAs read it in
-    // the CTA's type, so convert it once if they differ
     if (!mbar_wait(&bar->kv_full, 0, ctl)) {
       // aborted: fall through to the teardown
     } else {
-      const bool vt_f16 = P.safe[(size_t)cj * d.Hkv + kv] != 0;
-      if (vt_f16 != (cta_f16 != 0)) {
-        for (int rr = r0; rr < BN; rr += kRowsPerPass) {
-          uint4* p = reinterpret_cast<uint4*>(sVt + sw_off(BN, rr, lc * 8));
-          float x[8];
-          unpack8(*p, vt_f16, x);
-          *p = pack8(x, cta_f16 != 0);
+      if (!dmode) {
+        // Vt arrives in its chunk's storage type; the later-block MMAs read it
+        // in the CTA's type, so convert it once if they differ
+        const bool vt_f16 = P.safe[(size_t)cj * d.Hkv + kv] != 0;
+        if (vt_f16 != (cta_f16 != 0)) {
+          for (int rr = r0; rr < BN; rr += kRowsPerPass) {
+            uint4* p = reinterpret_cast<uint4*>(sV + sw_off(BN, rr, lc * 8));
+            float x[8];
+            unpack8(*p, vt_f16, x);
+            *p = pack8(x, cta_f16 != 0);
+          }
+          fence_proxy_async_smem();
         }
-        fence_proxy_async_smem();
       }
-      // the MMA warp waited for kv_full before this conversion may have
-      // finished; the first x_ready below orders it (it covers this thread's
-      // writes and every X tile depends on it)
       TileIter t = tile_at(t_begin);
       float delta[8];
       int cur_h = -1, upto = 0;
       for (int n = 0; n < ntiles; ++n, next_tile(t)) {
-        const int st = n & 1;
-        const bool diag = t.i == ch.j;
+        const int st = n % kQStages;
         const int h = kv * d.grp + t.hh;
-        // f_ij = exp(sum_{j<j'<i} tot_j'): running sum over the query chunks of
-        // one head (they only increase within a head)
-        if (t.hh != cur_h) {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) delta[e] = 0.f;
-          upto = ch.j + 1;
-          cur_h = t.hh;
-        }
-        for (; upto < t.i; ++upto) {
-          const float* tp = P.tot + ((size_t)(first + upto) * d.Hkv + kv) * DV + lc * 8;
-#pragma unroll
-          for (int e = 0; e < 8; ++e) delta[e] += tp[e];
-        }
         float f8[8];
+        if (!dmode) {
+          // f_ij = exp(sum_{j<j'<i} tot_j'): running sum over the query chunks
+          // of one head (they only increase within a head)
+          if (t.hh != cur_h) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) f8[e] = ex2(delta[e] * LOG2E);
-        if (!mbar_wait(&bar->q_full[st], (n >> 1) & 1, ctl)) break;
+            for (int e = 0; e < 8; ++e) delta[e] = 0.f;
+            upto = ch.j + 1;
+            cur_h = t.hh;
+          }
+          for (; upto < t.i; ++upto) {
+            const float* tp = P.tot + ((size_t)(first + upto) * d.Hkv + kv) * DV + lc * 8;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) delta[e] += tp[e];
+          }
+#pragma unroll
+          for (int e = 0; e < 8; ++e) f8[e] = ex2(delta[e] * LOG2E);
+        }
+        if (!mbar_wait(&bar->q_full[st], (n / kQStages) & 1, ctl)) break;
         const Chunk qc = P.chunks[first + t.i];
         const int qlen = min(BQ, qc.len - t.half * BQ);
-        if (!diag) {
-          // X = dOt f_ij, in the CTA's operand type
+        if (!dmode) {
+          // X = dOt f_ij, in the CTA's operand type; rows past the chunk's end
+          // are zeroed
           const bool in_f16 = P.dsafe[(size_t)(first + t.i) * d.Hq + h] != 0;
           uint8_t* xb = sX + st * BQ * DV * 2;
           for (int rr = r0; rr < BQ; rr += kRowsPerPass) {
@@ -836,7 +834,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           const size_t qtok = (size_t)qc.tok0 + t.half * BQ + dt;
           sM[st * BQ + dt] = dt < qlen ? P.m_s[qtok * d.Hq + h] : 0.f;
         }
-        fence_proxy_async_smem();
         mbar_arrive(&bar->x_ready[st]);
       }
     }
@@ -900,22 +897,27 @@ __global__ void __launch_bounds__(256) dkv_combine_kernel(const Params P) {
   const Chunk ch = P.chunks[ci];
   if (s >= ch.len) return;
   const size_t tok = (size_t)ch.tok0 + s;
-  constexpr int kCols = DK + 2 * DV;
+  constexpr int kCols = DK + DV;
   constexpr int VK = DK / 32, VV = DV / 32;            // channels per lane
   const int ck = lane * VK, cv = lane * VV;
+  // the chunk's first nd slots hold its diagonal parts (dV_d), the rest its
+  // later-block parts (dV_o)
+  const int halves = (ch.len + BQ - 1) / BQ;
+  const int nd = (d.grp * halves + P.tiles_per_part - 1) / P.tiles_per_part;
   float fk[VK] = {}, fd[VV] = {}, fo[VV] = {};
   for (int q = 0; q < cp.x; ++q) {
     const float* prow = P.partial + (((size_t)(cp.y + q) * d.Hkv + kv) * BN + s) * kCols;
-    float a[VK], b[VV], c[VV];
+    float a[VK], b[VV];
     ldf<VK>(prow + ck, a);
     ldf<VV>(prow + DK + cv, b);
-    ldf<VV>(prow + DK + DV + cv, c);
 #pragma unroll
     for (int e = 0; e < VK; ++e) fk[e] += a[e];
+    if (q < nd) {
 #pragma unroll
-    for (int e = 0; e < VV; ++e) {
-      fd[e] += b[e];
-      fo[e] += c[e];
+      for (int e = 0; e < VV; ++e) fd[e] += b[e];
+    } else {
+#pragma unroll
+      for (int e = 0; e < VV; ++e) fo[e] += b[e];
     }
   }
   // dk = scale * sum dS^T Q
