@@ -79,7 +79,7 @@ struct Ctl {
 // Waits for the phase with `parity` to complete; gives up after 1 s (sets the
 // status word to FIX_DEV_TIMEOUT and the CTA abort flag) or when another role
 // aborted.  Returns false when it gave up.
-static __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, Ctl ctl) {
+static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, Ctl ctl) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer();
   while (true) {
@@ -93,6 +93,26 @@ static __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, Ct
       return false;
     }
   }
+}
+
+// Non-blocking check of the phase with `parity` (acquire on success).
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// mbar_wait_slow with an inline check first: a wait whose phase has already
+// completed costs one shared-memory access instead of a call, which matters
+// to the MMA-issuing thread (the tensor core runs only a few MMAs ahead of it).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, Ctl ctl) {
+  return mbar_test(bar, parity) || mbar_wait_slow(bar, parity, ctl);
 }
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -231,6 +251,12 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr, uint32_t lbo_byte
          (static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16) |
          (static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
 }
+
+// The descriptor of a shared-memory address `bytes` past the one `d`
+// describes (same strides): the start-address field holds address / 16 in
+// its low 14 bits, which cannot carry while shared addresses stay below
+// 256 KB.  Lets the MMA issue loops build each base descriptor once.
+__device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
 
 // Instruction descriptor, kind::f16, bf16 x bf16 -> f32 (or f16 x f16 -> f32
 // with f16 = true; A and B always share one type).

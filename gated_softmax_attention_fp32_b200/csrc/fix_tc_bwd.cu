@@ -252,13 +252,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < DK / 16; ++kk) {
           const uint32_t off = (kk >> 2) * (BN * 128) + (kk & 3) * 32;
-          mma_ss(tmem + kColS, desc_sw128(q_addr + off, 16, 1024), desc_sw128(k_addr + off, 16, 1024),
+          mma_ss(tmem + kColS, desc_add(desc_sw128(q_addr, 16, 1024), off), desc_add(desc_sw128(k_addr, 16, 1024), off),
                  idesc_s, kk > 0);
         }
 #pragma unroll
         for (int kk = 0; kk < DV / 16; ++kk) {
           const uint32_t off = (kk >> 2) * (BN * 128) + (kk & 3) * 32;
-          mma_ss(tmem + kColP, desc_sw128(o_addr + off, 16, 1024), desc_sw128(v_addr + off, 16, 1024),
+          mma_ss(tmem + kColP, desc_add(desc_sw128(o_addr, 16, 1024), off), desc_add(desc_sw128(v_addr, 16, 1024), off),
                  it == 0 ? idesc_dp0 : idesc_dp, kk > 0);
         }
         tc_commit(&bar->s_full);
@@ -267,7 +267,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint64_t b = desc_sw128(k_addr + kk * 2048, BN * 128, 1024);
+          const uint64_t b = desc_add(desc_sw128(k_addr, BN * 128, 1024), kk * 2048);
           mma_ts(tmem + kColQ, tmem + kColS + kk * 8, b, idesc_dq, (it > 0 || kk > 0));
         }
         tc_commit(&bar->k_empty[st]);
@@ -412,7 +412,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ========================================================================= dk/dv
 
 constexpr int BQ = 64;         // query rows per streamed tile
-constexpr int kQStages = 3;    // Q / X tiles in flight
+constexpr int kQStages = 4;    // Q / X tiles in flight (later-block parts; diagonal parts: 2)
 
 struct KvBars {
   uint64_t kv_full;
@@ -420,14 +420,17 @@ struct KvBars {
   uint64_t s_full[2], p_ready[2], done, drain;
 };
 
+// The stage region holds kQStages stages of [Q | X] for later-block parts, or
+// two stages of [Q | X | X_lo] for diagonal parts (the smaller of the two).
 template <int DK, int DV>
 struct KvLayout {
   static constexpr int kK = 0;                              // [128][DK]
   static constexpr int kV = kK + BN * DK * 2;               // [128][DV] Vm (diagonal) or Vt
-  static constexpr int kQ = kV + BN * DV * 2;               // stages x [64][DK]
-  static constexpr int kX = kQ + kQStages * BQ * DK * 2;    // stages x [64][DV]
-  static constexpr int kXl = kX + kQStages * BQ * DV * 2;   // stages x [64][DV] (diagonal lo part)
-  static constexpr int kM = kXl + kQStages * BQ * DV * 2;   // stages x [64] f32 row max
+  static constexpr int kQ = kV + BN * DV * 2;               // stage region
+  static constexpr int kStageOff = BQ * (DK + DV) * 2;      // bytes per later-block stage
+  static constexpr int kStageDiag = BQ * (DK + 2 * DV) * 2; // bytes per diagonal stage
+  static constexpr int kM = kQ + kQStages * kStageOff;      // stages x [64] f32 row max
+  static_assert(2 * kStageDiag <= kQStages * kStageOff, "diagonal stages must fit the region");
   static constexpr int kBars = kM + kQStages * BQ * 4;
   static constexpr int kTmem = kBars + (int)sizeof(KvBars);
   static constexpr int kAbort = kTmem + 4;
@@ -483,9 +486,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   uint8_t* sK = smem + Lay::kK;
   uint8_t* sV = smem + Lay::kV;
-  uint8_t* sQ = smem + Lay::kQ;
-  uint8_t* sX = smem + Lay::kX;
-  uint8_t* sXl = smem + Lay::kXl;
+  // stage st: Q at sQ(st), X right after it, X_lo (diagonal) after X
+  const int nst = dmode ? 2 : kQStages, lgst = dmode ? 1 : 2;
+  const int stage_bytes = dmode ? Lay::kStageDiag : Lay::kStageOff;
+  auto sQ = [&](int st) { return smem + Lay::kQ + st * stage_bytes; };
+  auto sX = [&](int st) { return sQ(st) + BQ * DK * 2; };
+  auto sXl = [&](int st) { return sX(st) + BQ * DV * 2; };
   float* sM = reinterpret_cast<float*>(smem + Lay::kM);
   KvBars* bar = reinterpret_cast<KvBars*>(smem + Lay::kBars);
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(smem + Lay::kTmem);
@@ -555,26 +561,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       TileIter t = tile_at(t_begin);
       int nq = 0;
       for (int n = 0; n < ntiles; ++n, next_tile(t)) {
-        const int st = n % kQStages;
-        if (n >= kQStages && !mbar_wait(&bar->q_empty[st], ((n / kQStages) & 1) ^ 1, ctl)) break;
+        const int st = n & (nst - 1);
+        if (n >= nst && !mbar_wait(&bar->q_empty[st], ((n >> lgst) & 1) ^ 1, ctl)) break;
         // Q tile and the X operand (dOm hi + lo on the diagonal, dOt elsewhere)
         mbar_expect_tx(&bar->q_full[st], BQ * DK * 2 + (dmode ? 2 : 1) * BQ * DV * 2);
         const int h = kv * d.grp + t.hh;
         const int qtok = P.chunks[first + t.i].tok0 + t.half * BQ;
         for (int hh = 0; hh < DK / 64; ++hh)
-          tma_load_3d(sQ + st * BQ * DK * 2 + hh * BQ * 128, &tm_q, &bar->q_full[st], hh * 64, h, qtok);
+          tma_load_3d(sQ(st) + hh * BQ * 128, &tm_q, &bar->q_full[st], hh * 64, h, qtok);
         for (int hh = 0; hh < DV / 64; ++hh) {
-          tma_load_3d(sX + st * BQ * DV * 2 + hh * BQ * 128, dmode ? &tm_domh : &tm_dot,
-                      &bar->q_full[st], hh * 64, h, qtok);
+          tma_load_3d(sX(st) + hh * BQ * 128, dmode ? &tm_domh : &tm_dot, &bar->q_full[st], hh * 64,
+                      h, qtok);
           if (dmode)
-            tma_load_3d(sXl + st * BQ * DV * 2 + hh * BQ * 128, &tm_doml, &bar->q_full[st], hh * 64,
-                        h, qtok);
+            tma_load_3d(sXl(st) + hh * BQ * 128, &tm_doml, &bar->q_full[st], hh * 64, h, qtok);
         }
         ++nq;
       }
       const Ctl drain{P.status, nullptr};
-      for (int n = nq - 1; n >= 0 && n >= nq - kQStages; --n)
-        mbar_wait(&bar->q_full[n % kQStages], (n / kQStages) & 1, drain);
+      for (int n = nq - 1; n >= 0 && n >= nq - nst; --n)
+        mbar_wait(&bar->q_full[n & (nst - 1)], (n >> lgst) & 1, drain);
       mbar_wait(&bar->kv_full, 0, drain);
     }
   } else if (warp == 1) {
@@ -589,19 +594,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the operand warps may convert V in place after kv_full; every
       // x_ready covers their writes
       auto issue_sdp = [&](int n) -> bool {
-        const int st = n % kQStages, b = n & 1;
-        const uint32_t ph = (n / kQStages) & 1;
-        if (!mbar_wait(&bar->q_full[st], ph, ctl) || !mbar_wait(&bar->x_ready[st], ph, ctl))
-          return false;
+        const int st = n & (nst - 1), b = n & 1;
+        const uint32_t ph = (n >> lgst) & 1;
+        // the operand warps arrive on x_ready only after they saw q_full, so
+        // x_ready covers the TMA copies of the stage as well
+        if (!mbar_wait(&bar->x_ready[st], ph, ctl)) return false;
         tc_fence_after();
-        const uint32_t q_addr = smem_u32(sQ + st * BQ * DK * 2);
-        const uint32_t x_addr = smem_u32(sX + st * BQ * DV * 2);
+        const uint32_t q_addr = smem_u32(sQ(st));
+        const uint32_t x_addr = smem_u32(sX(st));
         // S^T = K Q^T   (M = 128 keys, N = 64 queries, K = DK)
 #pragma unroll
         for (int kk = 0; kk < DK / 16; ++kk) {
           const uint32_t ka = (kk >> 2) * (BN * 128) + (kk & 3) * 32;
           const uint32_t qa = (kk >> 2) * (BQ * 128) + (kk & 3) * 32;
-          mma_ss(tmem + col_s(b), desc_sw128(k_addr + ka, 16, 1024), desc_sw128(q_addr + qa, 16, 1024),
+          mma_ss(tmem + col_s(b), desc_add(desc_sw128(k_addr, 16, 1024), ka), desc_add(desc_sw128(q_addr, 16, 1024), qa),
                  idesc_s, kk > 0);
         }
         // dP^T = V X^T
@@ -609,7 +615,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kk = 0; kk < DV / 16; ++kk) {
           const uint32_t vo = (kk >> 2) * (BN * 128) + (kk & 3) * 32;
           const uint32_t xo = (kk >> 2) * (BQ * 128) + (kk & 3) * 32;
-          mma_ss(tmem + col_p(b), desc_sw128(v_addr + vo, 16, 1024), desc_sw128(x_addr + xo, 16, 1024),
+          mma_ss(tmem + col_p(b), desc_add(desc_sw128(v_addr, 16, 1024), vo), desc_add(desc_sw128(x_addr, 16, 1024), xo),
                  idesc_dp, kk > 0);
         }
         tc_commit(&bar->s_full[b]);
@@ -618,20 +624,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok) ok = issue_sdp(0);
       if (ok && ntiles > 1) ok = issue_sdp(1);
       for (int n = 0; ok && n < ntiles; ++n) {
-        const int st = n % kQStages, b = n & 1;
+        const int st = n & (nst - 1), b = n & 1;
         if (!mbar_wait(&bar->p_ready[b], (n >> 1) & 1, ctl)) break;
         tc_fence_after();
-        const uint32_t q_addr = smem_u32(sQ + st * BQ * DK * 2);
-        const uint32_t x_addr = smem_u32(sX + st * BQ * DV * 2);
-        const uint32_t xl_addr = smem_u32(sXl + st * BQ * DV * 2);
+        const uint32_t q_addr = smem_u32(sQ(st));
+        const uint32_t x_addr = smem_u32(sX(st));
+        const uint32_t xl_addr = smem_u32(sXl(st));
         // dV += P^T X  (K = 64 queries; X read MN-major); on the diagonal
         // P_hi X_hi + P_lo X_hi + P_hi X_lo
 #pragma unroll
         for (int kk = 0; kk < BQ / 16; ++kk) {
-          const uint64_t bx = desc_sw128(x_addr + kk * 2048, BQ * 128, 1024);
+          const uint64_t bx = desc_add(desc_sw128(x_addr, BQ * 128, 1024), kk * 2048);
           mma_ts(tmem + kColV, tmem + col_s(b) + kk * 8, bx, idesc_dv, !(n == 0 && kk == 0));
           if (dmode) {
-            const uint64_t bxl = desc_sw128(xl_addr + kk * 2048, BQ * 128, 1024);
+            const uint64_t bxl = desc_add(desc_sw128(xl_addr, BQ * 128, 1024), kk * 2048);
             mma_ts(tmem + kColV, tmem + col_s(b) + 32 + kk * 8, bx, idesc_dv, 1);
             mma_ts(tmem + kColV, tmem + col_s(b) + kk * 8, bxl, idesc_dv, 1);
           }
@@ -639,7 +645,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // dK += dS^T Q
 #pragma unroll
         for (int kk = 0; kk < BQ / 16; ++kk) {
-          const uint64_t bq = desc_sw128(q_addr + kk * 2048, BQ * 128, 1024);
+          const uint64_t bq = desc_add(desc_sw128(q_addr, BQ * 128, 1024), kk * 2048);
           mma_ts(tmem + kColK, tmem + col_p(b) + kk * 8, bq, idesc_dk, !(n == 0 && kk == 0));
         }
         tc_commit(&bar->q_empty[st]);
@@ -658,11 +664,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     TileIter t = tile_at(t_begin);
     for (int n = 0; n < ntiles; ++n, next_tile(t)) {
-      const int st = n % kQStages, b = n & 1;
+      const int st = n & (nst - 1), b = n & 1;
       const int qlen = min(BQ, chunk_len(t.i) - t.half * BQ);
       // x_ready covers the row maxima of this tile in sM
       if (!__all_sync(0xffffffffu, mbar_wait(&bar->s_full[b], (n >> 1) & 1, ctl) &&
-                                       mbar_wait(&bar->x_ready[st], (n / kQStages) & 1, ctl))) {
+                                       mbar_wait(&bar->x_ready[st], (n >> lgst) & 1, ctl))) {
         ok = false;
         break;
       }
@@ -788,38 +794,60 @@ __global__ void __launch_bounds__(kThreads, 1)
           fence_proxy_async_smem();
         }
       }
+      // Per tile: the row maxima into sM and, for later blocks, X = dOt f_ij
+      // with f_ij = exp(sum_{j<j'<i} tot_j').  The global values a tile needs
+      // (its row maxima and the totals that extend the running sum) are
+      // loaded one tile ahead, so that x_ready follows q_full closely.
       TileIter t = tile_at(t_begin);
+      // what a tile needs from global memory besides its totals
+      struct Pre {
+        float m;     // row maximum of query row dt (dt < 64)
+        int qlen;    // rows of the tile
+        int in_f16;  // storage type of its dOt
+      };
+      auto fetch = [&](const TileIter& u) {
+        const Chunk qc = P.chunks[first + u.i];
+        Pre r;
+        r.qlen = min(BQ, qc.len - u.half * BQ);
+        r.m = dt < r.qlen ? P.m_s[((size_t)qc.tok0 + u.half * BQ + dt) * d.Hq + kv * d.grp + u.hh] : 0.f;
+        r.in_f16 = dmode ? 0 : P.dsafe[(size_t)(first + u.i) * d.Hq + kv * d.grp + u.hh];
+        return r;
+      };
+      // sum of tot over query chunks [a, b) for this thread's 8 channels
+      auto tot_sum = [&](int a, int b, float* acc) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+        for (int i = a; i < b; ++i) {
+          const float* tp = P.tot + ((size_t)(first + i) * d.Hkv + kv) * DV + lc * 8;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[e] += tp[e];
+        }
+      };
       float delta[8];
-      int cur_h = -1, upto = 0;
-      for (int n = 0; n < ntiles; ++n, next_tile(t)) {
-        const int st = n % kQStages;
-        const int h = kv * d.grp + t.hh;
+      if (!dmode) tot_sum(ch.j + 1, t.i, delta);
+      Pre cur = fetch(t);
+      for (int n = 0; n < ntiles; ++n) {
+        const int st = n & (nst - 1);
         float f8[8];
         if (!dmode) {
-          // f_ij = exp(sum_{j<j'<i} tot_j'): running sum over the query chunks
-          // of one head (they only increase within a head)
-          if (t.hh != cur_h) {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) delta[e] = 0.f;
-            upto = ch.j + 1;
-            cur_h = t.hh;
-          }
-          for (; upto < t.i; ++upto) {
-            const float* tp = P.tot + ((size_t)(first + upto) * d.Hkv + kv) * DV + lc * 8;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) delta[e] += tp[e];
-          }
 #pragma unroll
           for (int e = 0; e < 8; ++e) f8[e] = ex2(delta[e] * LOG2E);
         }
-        if (!mbar_wait(&bar->q_full[st], (n / kQStages) & 1, ctl)) break;
-        const Chunk qc = P.chunks[first + t.i];
-        const int qlen = min(BQ, qc.len - t.half * BQ);
+        // prefetch for tile n + 1
+        TileIter u = t;
+        next_tile(u);
+        const bool more = n + 1 < ntiles;
+        const Pre nxt = more ? fetch(u) : cur;
+        float add[8];
+        const bool new_head = u.hh != t.hh;
+        if (!dmode) tot_sum(t.i, (more && !new_head) ? u.i : t.i, add);
+        if (!mbar_wait(&bar->q_full[st], (n >> lgst) & 1, ctl)) break;
+        const int qlen = cur.qlen;
         if (!dmode) {
           // X = dOt f_ij, in the CTA's operand type; rows past the chunk's end
           // are zeroed
-          const bool in_f16 = P.dsafe[(size_t)(first + t.i) * d.Hq + h] != 0;
-          uint8_t* xb = sX + st * BQ * DV * 2;
+          const bool in_f16 = cur.in_f16 != 0;
+          uint8_t* xb = sX(st);
           for (int rr = r0; rr < BQ; rr += kRowsPerPass) {
             uint4* p = reinterpret_cast<uint4*>(xb + sw_off(BQ, rr, lc * 8));
             float x[8];
@@ -830,11 +858,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           fence_proxy_async_smem();
         }
-        if (dt < BQ) {
-          const size_t qtok = (size_t)qc.tok0 + t.half * BQ + dt;
-          sM[st * BQ + dt] = dt < qlen ? P.m_s[qtok * d.Hq + h] : 0.f;
-        }
+        if (dt < BQ) sM[st * BQ + dt] = cur.m;
         mbar_arrive(&bar->x_ready[st]);
+        // advance to tile n + 1
+        if (!dmode) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) delta[e] = new_head ? 0.f : delta[e] + add[e];
+        }
+        cur = nxt;
+        t = u;
       }
     }
   }

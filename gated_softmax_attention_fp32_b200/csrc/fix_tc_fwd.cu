@@ -246,8 +246,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < DK / 16; ++kk) {
           const uint32_t off = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
-          const uint64_t a = desc_sw128(q_addr + off, 16, 1024);
-          const uint64_t b = desc_sw128(k_addr + (kk >> 2) * (BN * 128) + (kk & 3) * 32, 16, 1024);
+          const uint64_t a = desc_add(desc_sw128(q_addr, 16, 1024), off);
+          const uint64_t b = desc_add(desc_sw128(k_addr, 16, 1024), (kk >> 2) * (BN * 128) + (kk & 3) * 32);
           mma_ss(tmem + col_s(st), a, b, idesc_qk, kk > 0);
         }
         tc_commit(&bar->s_full[st]);
@@ -266,8 +266,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t vl_addr = smem_u32(sVl);
 #pragma unroll
           for (int kk = 0; kk < BN / 16; ++kk) {
-            const uint64_t bh = desc_sw128(v_addr + kk * 2048, BN * 128, 1024);
-            const uint64_t bl = desc_sw128(vl_addr + kk * 2048, BN * 128, 1024);
+            const uint64_t bh = desc_add(desc_sw128(v_addr, BN * 128, 1024), kk * 2048);
+            const uint64_t bl = desc_add(desc_sw128(vl_addr, BN * 128, 1024), kk * 2048);
             mma_ts(tmem + kColOd, tmem + col_s(0) + kk * 8, bh, idesc_pv, kk > 0);
             mma_ts(tmem + kColOd, tmem + kColPlo + kk * 8, bh, idesc_pv, 1);
             mma_ts(tmem + kColOd, tmem + col_s(0) + kk * 8, bl, idesc_pv, 1);
@@ -275,7 +275,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
 #pragma unroll
           for (int kk = 0; kk < BN / 16; ++kk) {
-            const uint64_t b = desc_sw128(v_addr + kk * 2048, BN * 128, 1024);
+            const uint64_t b = desc_add(desc_sw128(v_addr, BN * 128, 1024), kk * 2048);
             mma_ts(tmem + kColOd + DV, tmem + col_s(st) + kk * 8, b, idesc_pv_off,
                    (it > 1 || kk > 0));
           }
