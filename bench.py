@@ -344,14 +344,16 @@ def main():
     achieved = share * f_fwd / (stage_ms[dom] * 1e-3) / 1e12
     peak = pk.get("bf16_tflops_sustained" if args.steps * ms_per_step > 2000 else "bf16_tflops")
     ncu_traffic = None
-    prof = os.path.join(ROOT, "profiles", "roofline_traffic.json")
+    prof = os.path.join(ROOT, "profiles", "roofline_traffic.txt")
     if os.path.exists(prof):
         try:
-            tr = json.load(open(prof))
-            if tr.get("kernel_stage") == dom and tr.get("workload") == args.workload and \
+            tr = dict(line.split(None, 1) for line in open(prof)
+                      if line.strip() and not line.startswith("#"))
+            tr = {key: val.strip() for key, val in tr.items()}
+            if tr.get("kernel_stage") == dom and tr.get("workload") == str(args.workload) and \
                     tr.get("algo") == args.algo:
-                ncu_traffic = tr.get("bytes_per_launch")
-        except (OSError, ValueError):
+                ncu_traffic = int(tr["bytes_per_launch"])
+        except (OSError, ValueError, KeyError):
             pass
     gpu_launches = args.steps * (fixattn.fix_attn_kernel_count(p, False) +
                                  fixattn.fix_attn_kernel_count(p, True))

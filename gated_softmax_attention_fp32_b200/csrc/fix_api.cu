@@ -426,17 +426,31 @@ fix_status fix_attn_bwd(const fix_attn_problem* p, const void* q, const void* k,
     return FIX_ERR_CUDA;
   FIX_TRY(mark(p, FIX_STAGE_BWD_DQ, 0, st));
   if (tc) FIX_TRY(tc_bwd(p, d, ta, 0, st));
-  dq_simt_kernel<<<dim3(d.nchunks * 4, d.Hq), 256, smq, st>>>(
-      d, chunks, qb, kb, vb, L, tot, m_s, dow, static_cast<__nv_bfloat16*>(dq), gate);
+  else
+    dq_simt_kernel<<<dim3(d.nchunks * 4, d.Hq), 256, smq, st>>>(
+        d, chunks, qb, kb, vb, L, tot, m_s, dow, static_cast<__nv_bfloat16*>(dq), nullptr);
   FIX_TRY(launched());
   FIX_TRY(mark(p, FIX_STAGE_BWD_DQ, 1, st));
   FIX_TRY(mark(p, FIX_STAGE_BWD_DKV, 0, st));
   if (tc) FIX_TRY(tc_bwd(p, d, ta, 1, st));
-  dkv_simt_kernel<<<dim3(d.nchunks * 4, d.Hkv), 256, smkv, st>>>(
-      d, chunks, qb, kb, vb, L, tot, m_s, dow, A, static_cast<__nv_bfloat16*>(dk),
-      static_cast<__nv_bfloat16*>(dv), dG, gate);
+  else
+    dkv_simt_kernel<<<dim3(d.nchunks * 4, d.Hkv), 256, smkv, st>>>(
+        d, chunks, qb, kb, vb, L, tot, m_s, dow, A, static_cast<__nv_bfloat16*>(dk),
+        static_cast<__nv_bfloat16*>(dv), dG, nullptr);
   FIX_TRY(launched());
   FIX_TRY(mark(p, FIX_STAGE_BWD_DKV, 1, st));
+  FIX_TRY(mark(p, FIX_STAGE_BWD_FINISH, 0, st));
+  if (tc) {
+    FIX_TRY(tc_bwd(p, d, ta, 2, st));
+    dq_simt_kernel<<<dim3(d.nchunks * 4, d.Hq), 256, smq, st>>>(
+        d, chunks, qb, kb, vb, L, tot, m_s, dow, static_cast<__nv_bfloat16*>(dq), gate);
+    FIX_TRY(launched());
+    dkv_simt_kernel<<<dim3(d.nchunks * 4, d.Hkv), 256, smkv, st>>>(
+        d, chunks, qb, kb, vb, L, tot, m_s, dow, A, static_cast<__nv_bfloat16*>(dk),
+        static_cast<__nv_bfloat16*>(dv), dG, gate);
+    FIX_TRY(launched());
+  }
+  FIX_TRY(mark(p, FIX_STAGE_BWD_FINISH, 1, st));
   FIX_TRY(mark(p, FIX_STAGE_BWD_DG, 0, st));
   chunk_total_kernel<<<dim3(d.nchunks, d.Hkv), 512, 0, st>>>(d, chunks, dG, dtot);
   FIX_TRY(launched());

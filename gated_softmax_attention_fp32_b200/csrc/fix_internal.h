@@ -90,7 +90,7 @@ struct TcBwdArgs {
   float* dG;
   int* status;
 };
-// which = 0: dq kernel, 1: dk/dv kernel
+// which = 0: dq kernel, 1: dk/dv kernel, 2: combine of the dk/dv partials
 fix_status tc_bwd(const fix_attn_problem* p, const Dims& d, const TcBwdArgs& a, int which,
                   cudaStream_t st);
 

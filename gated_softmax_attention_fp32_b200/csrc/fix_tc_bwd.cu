@@ -1050,9 +1050,15 @@ static fix_status launch(const Params& prm, const void* vt, const void* vm, int 
       return FIX_ERR_CUDA;
     kern<<<(unsigned)(nparts * d.Hkv), kThreads, smem, st>>>(mq, mk, mvt, mvm, mdomh, mdoml, mdot,
                                                             prm);
-    if (cudaGetLastError() != cudaSuccess) return FIX_ERR_CUDA;
-    if (nslots > 0) dkv_combine_kernel<DK, DV><<<dim3(d.nchunks * (BN / 8), d.Hkv), 256, 0, st>>>(prm);
   }
+  return cudaGetLastError() == cudaSuccess ? FIX_OK : FIX_ERR_CUDA;
+}
+
+// The combine of the dk/dv partial slots (which = 2).
+template <int DK, int DV>
+static fix_status launch_combine(const Params& prm, long long nslots, cudaStream_t st) {
+  const Dims& d = prm.d;
+  if (nslots > 0) dkv_combine_kernel<DK, DV><<<dim3(d.nchunks * (BN / 8), d.Hkv), 256, 0, st>>>(prm);
   return cudaGetLastError() == cudaSuccess ? FIX_OK : FIX_ERR_CUDA;
 }
 
@@ -1097,6 +1103,13 @@ fix_status tc_bwd(const fix_attn_problem*, const Dims& d, const TcBwdArgs& a, in
   prm.dv = static_cast<__nv_bfloat16*>(a.dv);
   prm.dG = a.dG;
   prm.status = a.status;
+  if (which == 2) {
+    if (d.Dk == 128 && d.Dv == 128) return tcb::launch_combine<128, 128>(prm, a.nslots, st);
+    if (d.Dk == 64 && d.Dv == 64) return tcb::launch_combine<64, 64>(prm, a.nslots, st);
+    if (d.Dk == 128 && d.Dv == 64) return tcb::launch_combine<128, 64>(prm, a.nslots, st);
+    if (d.Dk == 64 && d.Dv == 128) return tcb::launch_combine<64, 128>(prm, a.nslots, st);
+    return FIX_ERR_HEAD_DIM;
+  }
   if (d.Dk == 128 && d.Dv == 128) return tcb::launch<128, 128>(prm, a.vt, a.vm, which, a.nparts, a.nslots, st);
   if (d.Dk == 64 && d.Dv == 64) return tcb::launch<64, 64>(prm, a.vt, a.vm, which, a.nparts, a.nslots, st);
   if (d.Dk == 128 && d.Dv == 64) return tcb::launch<128, 64>(prm, a.vt, a.vm, which, a.nparts, a.nslots, st);

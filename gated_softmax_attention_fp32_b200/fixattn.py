@@ -26,7 +26,8 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfixattn.
 EXPORTS = ("fix_attn_workspace_bytes", "fix_attn_fwd", "fix_attn_bwd", "fix_attn_device_status",
            "fix_attn_kernel_count", "fix_attn_status_string", "fix_attn_fwd_noalloc")
 NOALLOC_MAX_WORKSPACE_BYTES = 16 * 1024 * 1024
-STAGES = ("fwd_prefix", "fwd_attn", "bwd_prefix", "bwd_pre", "bwd_dq", "bwd_dkv", "bwd_dg")
+STAGES = ("fwd_prefix", "fwd_attn", "bwd_prefix", "bwd_pre", "bwd_dq", "bwd_dkv", "bwd_dg",
+          "bwd_finish")
 
 ALGOS = {"auto": 0, "simt": 1, "tc": 2}
 _lib = None

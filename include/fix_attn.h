@@ -95,10 +95,15 @@ enum {
   FIX_STAGE_FWD_ATTN = 1,   /* attention forward with the fused RMSNorm      */
   FIX_STAGE_BWD_PREFIX = 2, /* schedule + gate prefix sums + pre-decayed v   */
   FIX_STAGE_BWD_PRE = 3,    /* RMSNorm backward, dw                          */
-  FIX_STAGE_BWD_DQ = 4,     /* dq                                            */
-  FIX_STAGE_BWD_DKV = 5,    /* dk, dv, dG                                    */
+  FIX_STAGE_BWD_DQ = 4,     /* dq (tensor-core kernel, else exact kernel)    */
+  FIX_STAGE_BWD_DKV = 5,    /* dk/dv partial sums (tensor-core kernel, else  */
+                            /* the exact dk, dv, dG kernel)                  */
   FIX_STAGE_BWD_DG = 6,     /* reverse cumsum dG -> dg                        */
-  FIX_NUM_STAGES = 7
+  FIX_STAGE_BWD_FINISH = 7, /* tensor-core path: combine of the dk/dv        */
+                            /* partials into dk, dv, dG, and the exact       */
+                            /* kernels (they return at once unless a channel */
+                            /* is outside the split's range)                 */
+  FIX_NUM_STAGES = 8
 };
 
 /* Bytes of device workspace that fix_attn_fwd (backward = 0) or fix_attn_bwd
