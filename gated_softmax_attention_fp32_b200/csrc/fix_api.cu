@@ -128,7 +128,7 @@ static SplitPlan plan_split(const fix_attn_problem* p, const Dims& d) {
 // Workspace layout (all offsets 256-byte aligned).
 struct Ws {
   size_t status, chunks, order, safe, L, vt, vm, vml, tot, rho, hr;   // forward and backward
-  size_t dow, dot, domh, doml, dsafe, hmax, A, dG, dtot, dwp;   // backward only
+  size_t dow, dot, domh, doml, dsafe, hmax, ptt, A, dG, dtot, dwp;   // backward only
   size_t parts, cpart, partial;                            // dk/dv work split
   size_t total;
 };
@@ -161,6 +161,7 @@ static Ws layout(const Dims& d, bool bwd, const SplitPlan& sp) {
     w.doml = take((size_t)d.N * d.Hq * d.Dv * 2);
     w.dsafe = take((size_t)(d.nchunks > 0 ? d.nchunks : 1) * d.Hq * sizeof(int));
     w.hmax = take((size_t)(d.nchunks > 0 ? d.nchunks : 1) * d.Hq * sizeof(int));
+    w.ptt = take((size_t)d.N * d.Hq * sizeof(float));
     w.A = take(nkv * 4);
     w.dG = take(nkv * 4);
     w.dtot = take(nch * 4);
@@ -224,7 +225,7 @@ static fix_status run_prefix(const Dims& d, const fix_attn_problem* p, const Ws&
     ps.parts = reinterpret_cast<Part*>(base + ws.parts);
     ps.cpart = reinterpret_cast<int2*>(base + ws.cpart);
   }
-  schedule_kernel<<<1, 1024, 0, st>>>(p->cu_seqlens, d.nseq, d.T, d.N, d.nchunks, chunks,
+  schedule_kernel<<<1, kScheduleThreads, 0, st>>>(p->cu_seqlens, d.nseq, d.T, d.N, d.nchunks, chunks,
                                       max_chunks_per_seq(p),
                                       want_vt ? reinterpret_cast<int*>(base + ws.order) : nullptr, ps);
   FIX_TRY(launched());
@@ -368,7 +369,8 @@ fix_status fix_attn_bwd(const fix_attn_problem* p, const void* q, const void* k,
   int* hmax = reinterpret_cast<int*>(base + ws.hmax);
   bwd_pre_kernel<<<dim3(d.nchunks * kPreSplit, d.Hkv), 256, d.grp * sizeof(float), st>>>(
       d, chunks, qb, kb, vb, o_s, m_s, rstd_s, static_cast<const __nv_bfloat16*>(dy),
-      static_cast<const __nv_bfloat16*>(w), dow, A, dwp, tc ? hmax : nullptr);
+      static_cast<const __nv_bfloat16*>(w), dow, A, dwp, tc ? hmax : nullptr,
+      tc ? reinterpret_cast<float*>(base + ws.ptt) : nullptr);
   FIX_TRY(launched());
   if (tc) {
     bwd_pre_ops_kernel<<<dim3(d.nchunks * kPreSplit, d.Hkv), 256, 0, st>>>(
@@ -377,8 +379,8 @@ fix_status fix_attn_bwd(const fix_attn_problem* p, const void* q, const void* k,
         dow, hmax, dot, domh, doml, dsafe);
     FIX_TRY(launched());
   }
-  dw_reduce_kernel<<<1, 512, 0, st>>>(dwp, d.nchunks * kPreSplit * d.Hkv, d.Dv,
-                                      static_cast<__nv_bfloat16*>(dw));
+  dw_reduce_kernel<<<(d.Dv + 31) / 32, 1024, 0, st>>>(dwp, d.nchunks * kPreSplit * d.Hkv, d.Dv,
+                                                     static_cast<__nv_bfloat16*>(dw));
   FIX_TRY(launched());
   FIX_TRY(mark(p, FIX_STAGE_BWD_PRE, 1, st));
   TcBwdArgs ta{};
@@ -402,6 +404,7 @@ fix_status fix_attn_bwd(const fix_attn_problem* p, const void* q, const void* k,
     ta.domh = domh;
     ta.doml = doml;
     ta.A = A;
+    ta.ptt = reinterpret_cast<const float*>(base + ws.ptt);
     ta.badflag = badflag;
     ta.parts = reinterpret_cast<const Part*>(base + ws.parts);
     ta.cpart = reinterpret_cast<const int2*>(base + ws.cpart);

@@ -17,6 +17,13 @@
 #define FIX_CHUNK 128
 // CTAs per chunk in the backward preprocess (FIX_CHUNK / kPreSplit rows each).
 constexpr int kPreSplit = 4;
+// Threads of the single schedule CTA (a multiple of 32).
+constexpr int kScheduleThreads = 128;
+
+// exp for the 16-bit tensor-core operands (pre-decayed values and gradients,
+// rounded to fp16 / bf16 right after): exp2f of x log2(e), whose error is far
+// below their rounding.  The exact CUDA-core kernels keep expf.
+__device__ __forceinline__ float exp_op(float x) { return exp2f(x * 1.4426950408889634f); }
 // Largest half-range of a chunk's prefix sums that the in-chunk split
 // exp(L_t - rho) * exp(rho - L_s) keeps inside float range (e^80 ~ 5.5e34).
 #define FIX_HR_MAX 80.0f

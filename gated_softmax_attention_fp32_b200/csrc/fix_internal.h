@@ -27,7 +27,7 @@ __global__ void bwd_pre_kernel(Dims d, const Chunk* chunks, const __nv_bfloat16*
                                const __nv_bfloat16* k, const __nv_bfloat16* v, const float* o_s,
                                const float* m_s, const float* rstd_s, const __nv_bfloat16* dy,
                                const __nv_bfloat16* w, float* do_ws, float* A, float* dwpart,
-                               int* hmax_g);
+                               int* hmax_g, float* ptt);
 __global__ void bwd_pre_ops_kernel(Dims d, const Chunk* chunks, const float* L, const float* rho,
                                    const float* hr, const int* safe, const float* do_ws,
                                    const int* hmax_g, uint16_t* dot, __nv_bfloat16* domh,
@@ -77,6 +77,7 @@ struct TcBwdArgs {
   const __nv_bfloat16* domh;
   const __nv_bfloat16* doml;
   const float* A;
+  const float* ptt;      // P_tt per (token, q head), from the preprocess
   const int* badflag;
   const Part* parts;
   const int2* cpart;

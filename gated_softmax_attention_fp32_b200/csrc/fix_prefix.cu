@@ -50,20 +50,27 @@ __device__ void order_chunks(const Chunk* __restrict__ chunks, int nchunks, int 
 // every entry is first set empty, writes past `cap` are dropped and lengths
 // are clamped to the N tokens, so a device array that disagrees with the host
 // mirror cannot send any kernel outside its buffers.
-// Exclusive prefix sum over the 1024 threads of a CTA; *total gets the sum.
+// Exclusive prefix sum over the threads of a CTA (blockDim a multiple of 32):
+// warp shuffles, then the warp totals through `scan`; *total gets the sum.
 __device__ int block_excl_scan(int v, int* scan, int* total) {
-  scan[threadIdx.x] = v;
-  __syncthreads();
-  for (int off = 1; off < (int)blockDim.x; off <<= 1) {
-    const int add = threadIdx.x >= (unsigned)off ? scan[threadIdx.x - off] : 0;
-    __syncthreads();
-    scan[threadIdx.x] += add;
-    __syncthreads();
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
   }
-  const int incl = scan[threadIdx.x];
-  *total = scan[blockDim.x - 1];
+  if (lane == 31) scan[w] = x;
   __syncthreads();
-  return incl - v;
+  int off = 0, tot = 0;
+  for (int i = 0; i < nw; ++i) {
+    const int t = scan[i];
+    if (i < w) off += t;
+    tot += t;
+  }
+  __syncthreads();   // scan[] is reused by the next call
+  *total = tot;
+  return off + x - v;
 }
 
 // Number of 64-row query tiles from chunk j to the end of a sequence of L
@@ -72,11 +79,11 @@ __device__ __host__ inline int tiles64_from(int L, int j) {
   return (L - j * FIX_CHUNK + 63) / 64;
 }
 
-__global__ void __launch_bounds__(1024) schedule_kernel(const int64_t* __restrict__ cu, int nseq,
+__global__ void __launch_bounds__(kScheduleThreads) schedule_kernel(const int64_t* __restrict__ cu, int nseq,
                                                         int T, int N, int cap,
                                                         Chunk* __restrict__ out, int maxj,
                                                         int* __restrict__ order, PartSpec ps) {
-  __shared__ int scan[1024];
+  __shared__ int scan[kScheduleThreads / 32];
   for (int i = threadIdx.x; i < cap; i += blockDim.x) out[i] = Chunk{0, 0, 0, 0};
   __syncthreads();
   int carry = 0;
@@ -97,15 +104,8 @@ __global__ void __launch_bounds__(1024) schedule_kernel(const int64_t* __restric
       }
     }
     const int nc = (L + FIX_CHUNK - 1) / FIX_CHUNK;
-    scan[threadIdx.x] = nc;
-    __syncthreads();
-    for (int off = 1; off < (int)blockDim.x; off <<= 1) {
-      int add = threadIdx.x >= (unsigned)off ? scan[threadIdx.x - off] : 0;
-      __syncthreads();
-      scan[threadIdx.x] += add;
-      __syncthreads();
-    }
-    const int excl = carry + scan[threadIdx.x] - nc;
+    int tot;
+    const int excl = carry + block_excl_scan(nc, scan, &tot);
     const int ncw = max(0, min(nc, cap - excl));   // chunks that fit the table
     for (int j = 0; j < ncw; ++j) {
       Chunk c;
@@ -115,8 +115,7 @@ __global__ void __launch_bounds__(1024) schedule_kernel(const int64_t* __restric
       c.nch = ncw;
       out[excl + j] = c;
     }
-    carry += scan[blockDim.x - 1];
-    __syncthreads();
+    carry += tot;
   }
   if (order) {
     __threadfence_block();
@@ -284,9 +283,9 @@ __global__ void __launch_bounds__(kPrefixThreads) prefix_kernel(
   for (int u = 0; u < kMaxRows; ++u)
     if (u < nr) {
       const size_t a = base + (size_t)(r0 + u) * rs;
-      const float xt = vv[u] * expf(total - lv[u]);
+      const float xt = vv[u] * exp_op(total - lv[u]);
       vt[a] = f16 ? __half_as_ushort(__float2half_rn(xt)) : __bfloat16_as_ushort(f2bf(xt));
-      const float xm = good ? vv[u] * expf(ref - lv[u]) : 0.f;
+      const float xm = good ? vv[u] * exp_op(ref - lv[u]) : 0.f;
       const __nv_bfloat16 xm_hi = f2bf(xm);
       vm[a] = xm_hi;
       vml[a] = f2bf(xm - bf2f(xm_hi));   // Vm = hi + lo to ~16 bits

@@ -163,7 +163,8 @@ __global__ void __launch_bounds__(256) fwd_simt_kernel(
 //             (P_tt = exp(S_tt - m_t), S_tt recomputed from q_t, k_t)
 //   dw partials        sum_t dy_t n_t per CTA
 //   hmax[ci * Hq + h]  max |do| over the chunk (float bits, atomicMax; zeroed
-//                      by the prefix pass), only for the tensor-core kernels.
+//                      by the prefix pass), only for the tensor-core kernels;
+//   ptt[t * Hq + h]    P_tt, for the tensor-core dk/dv combine (optional).
 // Dynamic shared memory: grp floats.
 // ---------------------------------------------------------------------------
 constexpr int kPreWarps = 8;
@@ -174,7 +175,7 @@ __global__ void __launch_bounds__(kPreWarps * 32) bwd_pre_kernel(
     const float* __restrict__ o_s, const float* __restrict__ m_s,
     const float* __restrict__ rstd_s, const __nv_bfloat16* __restrict__ dy,
     const __nv_bfloat16* __restrict__ w, float* __restrict__ do_ws, float* __restrict__ A,
-    float* __restrict__ dwpart, int* __restrict__ hmax_g) {
+    float* __restrict__ dwpart, int* __restrict__ hmax_g, float* __restrict__ ptt_out) {
   __shared__ float red[kPreWarps][128];
   extern __shared__ float hmax[];   // [grp] max |do| per head
   const int Dv = d.Dv, Dk = d.Dk, kv = blockIdx.y;
@@ -217,6 +218,7 @@ __global__ void __launch_bounds__(kPreWarps * 32) bwd_pre_kernel(
         dyv[u] = c < Dv ? bf2f(dy[a]) : 0.f;
       }
       const float ptt = expf(warp_sum(sdot) * d.scale - mt);
+      if (ptt_out && lane == 0) ptt_out[t * d.Hq + h] = ptt;
       float dn[4], n[4], dot_ = 0.f;
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
@@ -320,9 +322,9 @@ __global__ void __launch_bounds__(kPreWarps * 32) bwd_pre_ops_kernel(
         const int c = lane + 32 * u;
         if (c >= Dv) continue;
         const size_t a = t * ors + (size_t)h * Dv + c;
-        const float xt = dov[u] * expf(lr[u]);
+        const float xt = dov[u] * exp_op(lr[u]);
         dot[a] = f16 ? __half_as_ushort(__float2half_rn(xt)) : __bfloat16_as_ushort(f2bf(xt));
-        const float xm = good[u] != 0.f ? dov[u] * expf(lr[u] - rh[u]) : 0.f;
+        const float xm = good[u] != 0.f ? dov[u] * exp_op(lr[u] - rh[u]) : 0.f;
         const __nv_bfloat16 hi = f2bf(xm);
         domh[a] = hi;
         doml[a] = f2bf(xm - bf2f(hi));
@@ -331,21 +333,24 @@ __global__ void __launch_bounds__(kPreWarps * 32) bwd_pre_ops_kernel(
   }
 }
 
-// dw = sum of the partials in a fixed order (deterministic).  One CTA of 512
-// threads: 512 / Dv interleaved groups of partial rows, then the groups in
+// dw = sum of the partials in a fixed order (deterministic).  grid
+// ceil(Dv / 32), block 1024: a CTA takes 32 channels (all of them for Dv <
+// 32), its threads interleaved groups of partial rows, then the groups in
 // order.
-__global__ void __launch_bounds__(512) dw_reduce_kernel(const float* __restrict__ parts,
-                                                        int nparts, int Dv,
-                                                        __nv_bfloat16* __restrict__ dw) {
-  __shared__ float red[512];
-  const int groups = 512 / Dv;
-  const int c = threadIdx.x % Dv, grp = threadIdx.x / Dv;
+__global__ void __launch_bounds__(1024) dw_reduce_kernel(const float* __restrict__ parts,
+                                                         int nparts, int Dv,
+                                                         __nv_bfloat16* __restrict__ dw) {
+  __shared__ float red[1024];
+  const int cw = Dv < 32 ? Dv : 32;
+  const int groups = 1024 / cw;
+  const int c = blockIdx.x * cw + (int)threadIdx.x % cw, grp = (int)threadIdx.x / cw;
   float s = 0.f;
-  if (grp < groups) {
+  if (grp < groups && c < Dv) {
     int i = grp;
     for (; i + 3 * groups < nparts; i += 4 * groups) {
       const float a = parts[(size_t)i * Dv + c], b = parts[(size_t)(i + groups) * Dv + c];
-      const float e = parts[(size_t)(i + 2 * groups) * Dv + c], f = parts[(size_t)(i + 3 * groups) * Dv + c];
+      const float e = parts[(size_t)(i + 2 * groups) * Dv + c];
+      const float f = parts[(size_t)(i + 3 * groups) * Dv + c];
       s += a;
       s += b;
       s += e;
@@ -355,10 +360,10 @@ __global__ void __launch_bounds__(512) dw_reduce_kernel(const float* __restrict_
   }
   red[threadIdx.x] = s;
   __syncthreads();
-  if (threadIdx.x < Dv) {
+  if ((int)threadIdx.x < cw && c < Dv) {
     float t = 0.f;
-    for (int g = 0; g < groups; ++g) t += red[g * Dv + threadIdx.x];
-    dw[threadIdx.x] = f2bf(t);
+    for (int g = 0; g < groups; ++g) t += red[g * cw + threadIdx.x];
+    dw[c] = f2bf(t);
   }
 }
 

@@ -67,6 +67,7 @@ struct Params {
   const __nv_bfloat16* domh;  // do exp(L_t - rho), hi and lo bf16 parts
   const __nv_bfloat16* doml;
   const float* A;
+  const float* ptt;         // P_tt per (token, q head), from the preprocess
   const int* badflag;
   const Part* parts;        // dk/dv work split (schedule kernel)
   const int2* cpart;
@@ -957,20 +958,13 @@ __global__ void __launch_bounds__(256) dkv_combine_kernel(const Params P) {
 #pragma unroll
   for (int e = 0; e < VK; ++e) fk[e] *= d.scale;
   stb<VK>(P.dk + tok * krs + (size_t)kv * DK + ck, fk);
-  // the s = t terms: P_ss (one per q head of the group) times do_s
-  float kr[VK];
-  ldb<VK>(P.k + tok * krs + (size_t)kv * DK + ck, kr);
+  // the s = t terms: P_ss (one per q head of the group, as the preprocess
+  // used it in A) times do_s
   const size_t vrs = (size_t)d.Hkv * DV, ors = (size_t)d.Hq * DV;
   float diag[VV] = {};
   for (int hh = 0; hh < d.grp; ++hh) {
     const int h = kv * d.grp + hh;
-    float qr[VK];
-    ldb<VK>(P.q + tok * (size_t)d.Hq * DK + (size_t)h * DK + ck, qr);
-    float acc = 0.f;
-#pragma unroll
-    for (int e = 0; e < VK; ++e) acc += qr[e] * kr[e];
-    acc = warp_sum(acc);
-    const float pss = ex2((acc * d.scale - P.m_s[tok * d.Hq + h]) * LOG2E);
+    const float pss = P.ptt[tok * d.Hq + h];
     float dw[VV];
     ldf<VV>(P.do_ws + tok * ors + (size_t)h * DV + cv, dw);
 #pragma unroll
@@ -1092,6 +1086,7 @@ fix_status tc_bwd(const fix_attn_problem*, const Dims& d, const TcBwdArgs& a, in
   prm.domh = a.domh;
   prm.doml = a.doml;
   prm.A = a.A;
+  prm.ptt = a.ptt;
   prm.badflag = a.badflag;
   prm.parts = a.parts;
   prm.cpart = a.cpart;

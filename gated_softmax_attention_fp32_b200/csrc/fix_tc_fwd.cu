@@ -402,10 +402,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     // ---------------------------------------------------------- epilogue
-    if (ok) {
-      if (nblk >= 2) ok = __all_sync(0xffffffffu, mbar_wait(&bar->pv_done, (nblk - 2) & 1, ctl));
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bar->pv_done, (nblk - 1) & 1, ctl));
-    }
+    // Every MMA of the CTA has completed once `drain` has: the MMA warp
+    // commits it once, after its last PV.  (pv_done completes once per PV, so
+    // a warp that reaches this point late could find it two phases on and
+    // wait for a phase that never comes.)
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bar->drain, 0, ctl));
     tc_fence_after();
     const bool row_ok = ok && r < ch.len;
     const size_t tok = (size_t)ch.tok0 + (size_t)(r < ch.len ? r : 0);
@@ -522,11 +523,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
-  if (warp >= 4) {
-    // ---------------------------------------------------------- phase B
-    // warps 4..11, a row at a time, lanes over channels: coalesced L / v
-    // loads, the RMSNorm reduction and coalesced y / o stores
-    asm volatile("bar.sync 2, 256;" ::: "memory");
+  // ------------------------------------------------------------ phase B
+  // every warp once the roles are done, rows in batches, lanes over
+  // channels: coalesced L / v loads, the RMSNorm reduction and coalesced
+  // y / o stores
+  __syncthreads();
+  {
     if (!*sAbort) {
       const float* __restrict__ tile = reinterpret_cast<const float*>(smem + Lay::kScratch);
       const float* __restrict__ sRow = reinterpret_cast<const float*>(smem + Lay::kRow);
@@ -548,7 +550,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         w_l[u] = sW[c];
         bad_l[u] = sHr[c] > FIX_HR_MAX;           // od holds the exact diagonal sum
       }
-      for (int r0 = (warp - 4) * kRows; r0 < ch.len; r0 += 8 * kRows) {
+      for (int r0 = warp * kRows; r0 < ch.len; r0 += (kThreads / 32) * kRows) {
         float lt[kRows][kU], vt[kRows][kU];
 #pragma unroll
         for (int q = 0; q < kRows; ++q) {
