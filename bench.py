@@ -355,6 +355,8 @@ def main():
                 ncu_traffic = int(tr["bytes_per_launch"])
         except (OSError, ValueError, KeyError):
             pass
+    # a bounded device wait that expired would leave its status in the workspace
+    dev_status = fixattn.fix_attn_device_status(ws)
     gpu_launches = args.steps * (fixattn.fix_attn_kernel_count(p, False) +
                                  fixattn.fix_attn_kernel_count(p, True))
 
@@ -378,6 +380,7 @@ def main():
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": gpu_launches,
         "clocks": clk,
+        "device_status": fixattn.status_string(dev_status),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         sampler = OracleSampler(case)
@@ -396,7 +399,7 @@ def main():
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
-    return 0
+    return 0 if dev_status == 0 else 3
 
 
 if __name__ == "__main__":

@@ -45,14 +45,22 @@ def run_gpu(case, algo="auto", backward=False, y_dtype=torch.float32):
     from gated_softmax_attention_fp32_b200 import fixattn
     t = to_cuda(case)
     cu_host = case["cu_seqlens"]
+    # one workspace for both calls, so that the device status word (where a
+    # bounded device wait that expired reports) can be checked after each
+    p, _keep = fixattn.make_problem(t["q"], t["k"], t["v"], t["cu_seqlens"], cu_host, None,
+                                    case["eps"], y_dtype, algo)
+    ws = torch.empty(max(fixattn.fix_attn_workspace_bytes(p, backward), 1), device="cuda",
+                     dtype=torch.uint8)
     y, saved = fixattn.fix_attn_fwd(t["q"], t["k"], t["v"], t["g"], t["w"], t["cu_seqlens"],
                                     cu_host, None, case["eps"], y_dtype=y_dtype, save=True,
-                                    algo=algo)
+                                    algo=algo, workspace=ws)
+    assert fixattn.fix_attn_device_status(ws) == 0, "forward: device status not OK"
     res = dict(y=y, o=saved[0], m=saved[1], rstd=saved[2])
     if backward:
         dq, dk, dv, dg, dw = fixattn.fix_attn_bwd(t["q"], t["k"], t["v"], t["g"], t["w"], t["dy"],
                                                   saved, t["cu_seqlens"], cu_host, None,
-                                                  case["eps"], algo=algo)
+                                                  case["eps"], algo=algo, workspace=ws)
+        assert fixattn.fix_attn_device_status(ws) == 0, "backward: device status not OK"
         res.update(dq=dq, dk=dk, dv=dv, dg=dg, dw=dw)
     torch.cuda.synchronize()
     return {k: v.float().cpu().numpy().astype(np.float64) for k, v in res.items()}
