@@ -257,7 +257,7 @@ def main():
         yy, saved = fixattn.fix_attn_fwd(q, k, v, g, w, cu, cu_host, None, eps, save=True,
                                          algo=args.algo, workspace=ws, out=y, events=events)
         fixattn.fix_attn_bwd(q, k, v, g, w, dy, saved, cu, cu_host, None, eps, algo=args.algo,
-                             workspace=ws, events=events, out=grads)
+                             workspace=ws, events=events, out=grads, reuse_forward_workspace=True)
         return saved
 
     for _ in range(max(3, args.warmup)):
@@ -275,18 +275,49 @@ def main():
     torch.cuda.synchronize()
     vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
     smi_id = vis.split(",")[local].strip() if vis else str(local)
+    # eager steps with the per-stage events (stage times, forward time)
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)                     # evict L2 outside the timed step
+        starts[i].record(stream)
+        step(ev[i])
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    eager_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends)) / args.steps
+    stage_ms = {name: statistics.mean(ev[i][2 * j].elapsed_time(ev[i][2 * j + 1])
+                                      for i in range(args.steps))
+                for j, name in enumerate(fixattn.STAGES)}
+    # the step as one CUDA graph (the library's calls are stream-ordered and
+    # capturable): its replays are the timed region, free of host launch gaps
+    side = torch.cuda.Stream()
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        step()
+    stream.wait_stream(side)
+    torch.cuda.synchronize()
+    graph, launch = torch.cuda.CUDAGraph(), "one CUDA graph per step (fix_attn_fwd + fix_attn_bwd)"
+    try:
+        with torch.cuda.graph(graph):
+            step()
+        torch.cuda.synchronize()
+    except Exception as exc:                      # capture refused: time the eager calls
+        graph, launch = None, f"eager calls (graph capture failed: {type(exc).__name__})"
+        torch.cuda.synchronize()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
     with ClockSampler(smi_id) as clocks:
         for i in range(args.steps):
             flush.fill_(i & 0xFF)                 # evict L2 outside the timed step
             starts[i].record(stream)
-            step(ev[i])
+            if graph is not None:
+                graph.replay()
+            else:
+                step()
             ends[i].record(stream)
         torch.cuda.synchronize()
     clk = clocks.summary()
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    stage_ms = {name: statistics.mean(ev[i][2 * j].elapsed_time(ev[i][2 * j + 1])
-                                      for i in range(args.steps))
-                for j, name in enumerate(fixattn.STAGES)}
     tot_ms = sum(step_ms)
     fwd_ms = statistics.mean(ev[i][0].elapsed_time(ev[i][3]) for i in range(args.steps))
     if world > 1:
@@ -368,7 +399,9 @@ def main():
         "config": {"workload": workload_name, "B": B, "T": T, "Hq": Hq, "Hkv": Hkv,
                    "Dk": Dk, "Dv": Dv, "algo": args.algo,
                    "l2": "flushed (256 MB write) before every timed step",
-                   "flops_per_step": f_step, "parallelism": f"{world} independent replicas"},
+                   "flops_per_step": f_step, "parallelism": f"{world} independent replicas",
+                   "launch": launch},
+        "eager_ms_per_step": eager_ms,
         "fwd_tflops": fwd_tflops,
         "fwd_frac_of_peak": fwd_tflops / pk["bf16_tflops"],
         "frac_of_peak": value / pk["bf16_tflops"] / world,

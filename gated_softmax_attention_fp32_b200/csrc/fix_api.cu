@@ -4,6 +4,8 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
+#include <vector>
 
 #include "fix_attn.h"
 #include "fix_common.cuh"
@@ -20,7 +22,7 @@ static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 // Validates the problem descriptor and fills the kernel-side dims.
 static fix_status make_dims(const fix_attn_problem* p, Dims* d) {
   if (!p) return FIX_ERR_NULL;
-  if (p->reserved != 0) return FIX_ERR_SHAPE;
+  if (p->flags & ~FIX_FLAG_REUSE_FWD_WORKSPACE) return FIX_ERR_SHAPE;
   if (p->y_dtype != FIX_DTYPE_BF16 && p->y_dtype != FIX_DTYPE_F32) return FIX_ERR_DTYPE;
   if (p->algo < FIX_ALGO_AUTO || p->algo > FIX_ALGO_TC) return FIX_ERR_DTYPE;
   if (p->batch < 1 || p->seqlen < 0 || p->num_q_heads < 1 || p->num_kv_heads < 1)
@@ -213,9 +215,34 @@ static size_t simt_dkv_smem(const Dims& d) {
 }
 
 // Prefix pass + schedule (both directions).
+bool set_smem_limit(const void* func, int bytes) {
+  struct Entry {
+    const void* func;
+    int dev, bytes;
+  };
+  static std::mutex mu;
+  static std::vector<Entry> done;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  std::lock_guard<std::mutex> lock(mu);
+  for (Entry& e : done)
+    if (e.func == func && e.dev == dev) {
+      if (bytes <= e.bytes) return true;
+      if (cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+          cudaSuccess)
+        return false;
+      e.bytes = bytes;
+      return true;
+    }
+  if (cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+    return false;
+  done.push_back(Entry{func, dev, bytes});
+  return true;
+}
+
 static fix_status run_prefix(const Dims& d, const fix_attn_problem* p, const Ws& ws, char* base,
                              const float* g, const void* v, bool want_vt, const SplitPlan* sp,
-                             int* hmax, cudaStream_t st) {
+                             int* hmax, bool reuse, cudaStream_t st) {
   Chunk* chunks = reinterpret_cast<Chunk*>(base + ws.chunks);
   PartSpec ps{};
   if (sp) {
@@ -230,6 +257,13 @@ static fix_status run_prefix(const Dims& d, const fix_attn_problem* p, const Ws&
                                       want_vt ? reinterpret_cast<int*>(base + ws.order) : nullptr, ps);
   FIX_TRY(launched());
   if (d.nchunks == 0) return FIX_OK;
+  if (reuse) {
+    // the forward's prefix results stay; only the per-(chunk, q head) max
+    // |do| of this backward starts from zero
+    if (hmax && cudaMemsetAsync(hmax, 0, (size_t)d.nchunks * d.Hq * sizeof(int), st) != cudaSuccess)
+      return FIX_ERR_CUDA;
+    return FIX_OK;
+  }
   prefix_kernel<<<dim3(d.nchunks, d.Hkv), 512, 0, st>>>(
       d, chunks, g, static_cast<const __nv_bfloat16*>(v), reinterpret_cast<float*>(base + ws.L),
       want_vt ? reinterpret_cast<uint16_t*>(base + ws.vt) : nullptr,
@@ -291,7 +325,7 @@ fix_status fix_attn_fwd(const fix_attn_problem* p, const void* q, const void* k,
   if (d.N == 0) return FIX_OK;
   const bool tc = p->algo != FIX_ALGO_SIMT && tc_fwd_supported(d);
   FIX_TRY(mark(p, FIX_STAGE_FWD_PREFIX, 0, st));
-  FIX_TRY(run_prefix(d, p, ws, base, g, v, tc, nullptr, nullptr, st));
+  FIX_TRY(run_prefix(d, p, ws, base, g, v, tc, nullptr, nullptr, false, st));
   FIX_TRY(mark(p, FIX_STAGE_FWD_PREFIX, 1, st));
   const Chunk* chunks = reinterpret_cast<const Chunk*>(base + ws.chunks);
   const float* L = reinterpret_cast<const float*>(base + ws.L);
@@ -308,8 +342,7 @@ fix_status fix_attn_fwd(const fix_attn_problem* p, const void* q, const void* k,
                    o_s, m_s, rstd_s, reinterpret_cast<int*>(base + ws.status), st));
   } else {
     const size_t smem = simt_fwd_smem(d);
-    if (cudaFuncSetAttribute(fwd_simt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem) != cudaSuccess)
+    if (!set_smem_limit(reinterpret_cast<const void*>(fwd_simt_kernel), (int)smem))
       return FIX_ERR_CUDA;
     fwd_simt_kernel<<<dim3(d.nchunks * 4, d.Hq), 256, smem, st>>>(
         d, chunks, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
@@ -339,15 +372,21 @@ fix_status fix_attn_bwd(const fix_attn_problem* p, const void* q, const void* k,
   FIX_TRY(check_device());
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* base = static_cast<char*>(workspace);
-  if (cudaMemsetAsync(base + ws.status, 0, 8, st) != cudaSuccess) return FIX_ERR_CUDA;
+  const bool tc = p->algo != FIX_ALGO_SIMT && tc_bwd_supported(d);
+  // The forward's prefix results can stand in for the backward's when the
+  // caller says the workspace is the forward's and the forward produced what
+  // this backward reads (the 16-bit operands only on its tensor-core path).
+  const bool fwd_tc = p->algo != FIX_ALGO_SIMT && tc_fwd_supported(d);
+  const bool reuse = (p->flags & FIX_FLAG_REUSE_FWD_WORKSPACE) && (!tc || fwd_tc);
+  // status word, and (unless reused) the prefix pass's out-of-range flag
+  if (cudaMemsetAsync(base + ws.status, 0, reuse ? 4 : 8, st) != cudaSuccess) return FIX_ERR_CUDA;
   if (d.N == 0) {
     if (cudaMemsetAsync(dw, 0, (size_t)d.Dv * 2, st) != cudaSuccess) return FIX_ERR_CUDA;
     return FIX_OK;
   }
-  const bool tc = p->algo != FIX_ALGO_SIMT && tc_bwd_supported(d);
   FIX_TRY(mark(p, FIX_STAGE_BWD_PREFIX, 0, st));
   FIX_TRY(run_prefix(d, p, ws, base, g, v, tc, tc ? &sp : nullptr,
-                     tc ? reinterpret_cast<int*>(base + ws.hmax) : nullptr, st));
+                     tc ? reinterpret_cast<int*>(base + ws.hmax) : nullptr, reuse, st));
   FIX_TRY(mark(p, FIX_STAGE_BWD_PREFIX, 1, st));
   const Chunk* chunks = reinterpret_cast<const Chunk*>(base + ws.chunks);
   const float* L = reinterpret_cast<const float*>(base + ws.L);
@@ -422,10 +461,8 @@ fix_status fix_attn_bwd(const fix_attn_problem* p, const void* q, const void* k,
   // once unless the prefix pass flagged a channel outside the split's range.
   const int* gate = tc ? badflag : nullptr;
   const size_t smq = simt_dq_smem(d), smkv = simt_dkv_smem(d);
-  if (cudaFuncSetAttribute(dq_simt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smq) != cudaSuccess ||
-      cudaFuncSetAttribute(dkv_simt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smkv) != cudaSuccess)
+  if (!set_smem_limit(reinterpret_cast<const void*>(dq_simt_kernel), (int)smq) ||
+      !set_smem_limit(reinterpret_cast<const void*>(dkv_simt_kernel), (int)smkv))
     return FIX_ERR_CUDA;
   FIX_TRY(mark(p, FIX_STAGE_BWD_DQ, 0, st));
   if (tc) FIX_TRY(tc_bwd(p, d, ta, 0, st));

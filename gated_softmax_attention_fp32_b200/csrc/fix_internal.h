@@ -44,6 +44,11 @@ __global__ void dkv_simt_kernel(Dims d, const Chunk* chunks, const __nv_bfloat16
                                 const int* gate);
 
 // Tensor-core (tcgen05) kernels.
+// Raises a kernel's dynamic shared-memory limit to at least `bytes` on the
+// current device.  The attribute is set once per (kernel, device) and size
+// increase, so the launch path makes no further runtime calls for it (which
+// keeps the calls cheap and lets a stream capture record the launches).
+bool set_smem_limit(const void* func, int bytes);
 bool tc_fwd_supported(const Dims& d);
 fix_status tc_fwd(const Dims& d, const Chunk* chunks, const int* order, const void* q,
                   const void* k, const uint16_t* vt, const __nv_bfloat16* vm,

@@ -1033,14 +1033,14 @@ static fix_status launch(const Params& prm, const void* vt, const void* vm, int 
   if (which == 0) {
     const int smem = DqLayout<DK, DV>::kAlloc;
     auto kern = dq_tc_kernel<DK, DV>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    if (!set_smem_limit(reinterpret_cast<const void*>(kern), smem))
       return FIX_ERR_CUDA;
     kern<<<(unsigned)((long long)d.nchunks * d.Hq), kThreads, smem, st>>>(mq, mk, mvt, mvm, mdomh,
                                                                          mdot, prm);
   } else {
     const int smem = KvLayout<DK, DV>::kAlloc;
     auto kern = dkv_tc_kernel<DK, DV>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    if (!set_smem_limit(reinterpret_cast<const void*>(kern), smem))
       return FIX_ERR_CUDA;
     kern<<<(unsigned)(nparts * d.Hkv), kThreads, smem, st>>>(mq, mk, mvt, mvm, mdomh, mdoml, mdot,
                                                             prm);

@@ -652,7 +652,7 @@ static fix_status launch(const Params& prm, const void* q, const void* k, const 
     return FIX_ERR_CUDA;
   const int smem = Layout<DK, DV>::kAlloc;
   auto kern = fwd_tc_kernel<DK, DV>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+  if (!set_smem_limit(reinterpret_cast<const void*>(kern), smem))
     return FIX_ERR_CUDA;
   const long long grid = (long long)d.nchunks * d.Hq;
   if (grid <= 0) return FIX_OK;

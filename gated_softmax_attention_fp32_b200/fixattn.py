@@ -20,12 +20,14 @@ from typing import Optional
 import torch
 
 __all__ = ["load", "Problem", "fix_attn_fwd", "fix_attn_bwd", "fix_attn_workspace_bytes",
-           "fix_attn_device_status", "fix_attn", "FixStatusError", "LIB_PATH", "EXPORTS"]
+           "fix_attn_device_status", "fix_attn", "training_workspace", "FixStatusError", "LIB_PATH",
+           "EXPORTS"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfixattn.so")
 EXPORTS = ("fix_attn_workspace_bytes", "fix_attn_fwd", "fix_attn_bwd", "fix_attn_device_status",
            "fix_attn_kernel_count", "fix_attn_status_string", "fix_attn_fwd_noalloc")
 NOALLOC_MAX_WORKSPACE_BYTES = 16 * 1024 * 1024
+FIX_FLAG_REUSE_FWD_WORKSPACE = 1
 STAGES = ("fwd_prefix", "fwd_attn", "bwd_prefix", "bwd_pre", "bwd_dq", "bwd_dkv", "bwd_dg",
           "bwd_finish")
 
@@ -38,7 +40,7 @@ class Problem(ctypes.Structure):
                 ("num_q_heads", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32),
                 ("head_dim_k", ctypes.c_int32), ("head_dim_v", ctypes.c_int32),
                 ("num_seqs", ctypes.c_int32), ("y_dtype", ctypes.c_int32),
-                ("algo", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("algo", ctypes.c_int32), ("flags", ctypes.c_int32),
                 ("cu_seqlens", ctypes.c_void_p), ("cu_seqlens_host", ctypes.c_void_p),
                 ("scale", ctypes.c_float), ("eps", ctypes.c_float),
                 ("events", ctypes.c_void_p)]
@@ -100,7 +102,7 @@ def make_problem(q, k, v, cu_seqlens=None, cu_seqlens_host=None, scale=None, eps
     p.head_dim_k, p.head_dim_v = Dk, Dv
     p.y_dtype = 1 if y_dtype == torch.float32 else 0
     p.algo = ALGOS[algo]
-    p.reserved = 0
+    p.flags = 0
     p.scale = float(scale) if scale is not None else 0.0
     p.eps = float(eps)
     keep = None
@@ -181,12 +183,19 @@ def fix_attn_fwd_noalloc(q, k, v, g, o_norm_weight, y, saved, cu_seqlens=None,
 
 def fix_attn_bwd(q, k, v, g, o_norm_weight, dy, saved, cu_seqlens=None, cu_seqlens_host=None,
                  scale=None, eps=1e-6, algo="auto", workspace=None, stream=None, events=None,
-                 out=None):
+                 out=None, reuse_forward_workspace=False):
     """Backward of sum(dy * y).  Returns dq, dk, dv, dg, dw (``out`` may
-    supply those five tensors)."""
+    supply those five tensors).  ``reuse_forward_workspace``: ``workspace`` is
+    the one the matching training forward used (sized for the backward, see
+    ``training_workspace``) and has not been written since; the backward then
+    reuses the forward's gate prefix results (FIX_FLAG_REUSE_FWD_WORKSPACE)."""
     lib = load()
     p, keep = make_problem(q, k, v, cu_seqlens, cu_seqlens_host, scale, eps, torch.bfloat16, algo,
                            events)
+    if reuse_forward_workspace:
+        if workspace is None:
+            raise ValueError("reuse_forward_workspace needs the forward's workspace")
+        p.flags = FIX_FLAG_REUSE_FWD_WORKSPACE
     if out is not None:
         dq, dk, dv, dg, dw = out
     else:
@@ -208,6 +217,15 @@ def fix_attn_bwd(q, k, v, g, o_norm_weight, dy, saved, cu_seqlens=None, cu_seqle
     return dq, dk, dv, dg, dw
 
 
+def training_workspace(q, k, v, cu_seqlens=None, cu_seqlens_host=None, algo="auto"):
+    """A workspace sized for the backward, to pass to a training forward and
+    then to its backward with ``reuse_forward_workspace=True``."""
+    p, keep = make_problem(q, k, v, cu_seqlens, cu_seqlens_host, None, 1e-6, torch.bfloat16, algo)
+    n = fix_attn_workspace_bytes(p, True)
+    del keep
+    return torch.empty(max(n, 1), device=q.device, dtype=torch.uint8)
+
+
 def fix_attn_device_status(workspace, stream=None) -> int:
     return int(load().fix_attn_device_status(_ptr(workspace), _stream(stream)))
 
@@ -215,10 +233,12 @@ def fix_attn_device_status(workspace, stream=None) -> int:
 class _FixAttn(torch.autograd.Function):
     @staticmethod
     def forward(ctx, q, k, v, g, w, cu_seqlens, cu_host, scale, eps, algo):
+        ws = training_workspace(q, k, v, cu_seqlens, cu_host, algo)
         y, saved = fix_attn_fwd(q, k, v, g, w, cu_seqlens, cu_host, scale, eps, save=True,
-                                algo=algo)
+                                algo=algo, workspace=ws)
         ctx.save_for_backward(q, k, v, g, w, *saved)
         ctx.cfg = (cu_seqlens, cu_host, scale, eps, algo)
+        ctx.ws = ws
         return y
 
     @staticmethod
@@ -226,7 +246,9 @@ class _FixAttn(torch.autograd.Function):
         q, k, v, g, w, o_s, m_s, r_s = ctx.saved_tensors
         cu, cu_host, scale, eps, algo = ctx.cfg
         dq, dk, dv, dg, dw = fix_attn_bwd(q, k, v, g, w, dy.to(torch.bfloat16).contiguous(),
-                                          (o_s, m_s, r_s), cu, cu_host, scale, eps, algo)
+                                          (o_s, m_s, r_s), cu, cu_host, scale, eps, algo,
+                                          workspace=ctx.ws, reuse_forward_workspace=True)
+        ctx.ws = None
         return dq, dk, dv, dg, dw, None, None, None, None, None
 
 

@@ -68,6 +68,16 @@ enum { FIX_DTYPE_BF16 = 0, FIX_DTYPE_F32 = 1 };
  * a second, independent GPU path for cross-checks. */
 enum { FIX_ALGO_AUTO = 0, FIX_ALGO_SIMT = 1, FIX_ALGO_TC = 2 };
 
+/* fix_attn_problem.flags.
+ * FIX_FLAG_REUSE_FWD_WORKSPACE (fix_attn_bwd only): the caller promises that
+ *   `workspace` is the one the matching training-mode fix_attn_fwd call used
+ *   (same problem, q, k, v, g) and that nothing has written it since.  The
+ *   backward then reuses the forward's gate prefix results (the prefix pass
+ *   of the README's "Code Structure": chunk-local cumsums and pre-decayed
+ *   values) instead of recomputing them.  Undefined results if the promise
+ *   does not hold.  Any other bit: FIX_ERR_SHAPE. */
+enum { FIX_FLAG_REUSE_FWD_WORKSPACE = 1 };
+
 typedef struct {
   int32_t batch;          /* B; must be 1 when cu_seqlens is given           */
   int32_t seqlen;         /* T; the total token count N when packed          */
@@ -78,7 +88,7 @@ typedef struct {
   int32_t num_seqs;       /* packed sequence count S (0 when not packed)      */
   int32_t y_dtype;        /* FIX_DTYPE_BF16 or FIX_DTYPE_F32                  */
   int32_t algo;           /* FIX_ALGO_*                                       */
-  int32_t reserved;       /* must be 0                                        */
+  int32_t flags;          /* FIX_FLAG_* bits; 0 by default                    */
   const int64_t *cu_seqlens;      /* device [S+1] or NULL                     */
   const int64_t *cu_seqlens_host; /* host mirror [S+1]; required with cu_seqlens */
   float scale;            /* logit scale; <= 0 selects Dk^-1/2                */

@@ -40,8 +40,9 @@ def to_cuda(case):
     return out
 
 
-def run_gpu(case, algo="auto", backward=False, y_dtype=torch.float32):
-    """Forward (and backward) through the C ABI; returns numpy float64 dicts."""
+def run_gpu(case, algo="auto", backward=False, y_dtype=torch.float32, reuse=True):
+    """Forward (and backward) through the C ABI; returns numpy float64 dicts.
+    ``reuse``: the backward reuses the forward's workspace (its gate prefix)."""
     from gated_softmax_attention_fp32_b200 import fixattn
     t = to_cuda(case)
     cu_host = case["cu_seqlens"]
@@ -59,7 +60,8 @@ def run_gpu(case, algo="auto", backward=False, y_dtype=torch.float32):
     if backward:
         dq, dk, dv, dg, dw = fixattn.fix_attn_bwd(t["q"], t["k"], t["v"], t["g"], t["w"], t["dy"],
                                                   saved, t["cu_seqlens"], cu_host, None,
-                                                  case["eps"], algo=algo, workspace=ws)
+                                                  case["eps"], algo=algo, workspace=ws,
+                                                  reuse_forward_workspace=reuse)
         assert fixattn.fix_attn_device_status(ws) == 0, "backward: device status not OK"
         res.update(dq=dq, dk=dk, dv=dv, dg=dg, dw=dw)
     torch.cuda.synchronize()

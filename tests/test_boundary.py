@@ -51,7 +51,7 @@ def prob(B=2, T=100, Hq=4, Hkv=2, Dk=64, Dv=64, **kw):
     p.num_seqs = 0
     p.y_dtype = 0
     p.algo = 0
-    p.reserved = 0
+    p.flags = 0
     p.scale = 0.0
     p.eps = 1e-6
     for key, val in kw.items():
@@ -77,7 +77,7 @@ def test_workspace_sizes(lib):
     (dict(T=-1), FIX_ERR_SHAPE),
     (dict(y_dtype=7), FIX_ERR_DTYPE),
     (dict(algo=9), FIX_ERR_DTYPE),
-    (dict(reserved=1), FIX_ERR_SHAPE),
+    (dict(flags=2), FIX_ERR_SHAPE),
     (dict(eps=-1.0), FIX_ERR_SHAPE),
     (dict(num_seqs=2), FIX_ERR_CU_SEQLENS),
 ])

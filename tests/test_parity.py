@@ -64,6 +64,19 @@ SMALL = {
 POSITIVE_GATE_MAX_ABS = 1e-1
 
 
+@pytest.mark.parametrize("name", ["T520-D128", "fast-channels", "varlen"])
+def test_backward_reusing_forward_workspace_is_identical(cuda_lib, name):
+    """FIX_FLAG_REUSE_FWD_WORKSPACE: the backward reads the forward's gate
+    prefix results instead of recomputing them (for "fast-channels" that
+    includes the flag that sends out-of-range channels to the exact kernels);
+    the gradients are bit-identical to a backward that recomputes."""
+    case = synth.make_case(**SMALL[name], seed=7)
+    a = run_gpu(case, "auto", backward=True, reuse=True)
+    b = run_gpu(case, "auto", backward=True, reuse=False)
+    for key in ("y",) + tuple(GRADS):
+        assert np.array_equal(a[key], b[key]), (name, key)
+
+
 @pytest.mark.parametrize("algo", ["auto", "simt"])
 @pytest.mark.parametrize("name", list(SMALL))
 def test_small_shapes(cuda_lib, name, algo):
