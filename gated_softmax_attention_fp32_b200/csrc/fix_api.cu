@@ -508,9 +508,13 @@ int fix_attn_kernel_count(const fix_attn_problem* p, int backward) {
     return 2 + (tc ? tc_fwd_kernel_count(d) : 1);
   }
   const bool tc = p->algo != FIX_ALGO_SIMT && tc_bwd_supported(d);
-  // prefix pass (2), preprocess (2, or 3 with the tensor-core operands),
-  // tensor-core dq / dk/dv, the exact kernels (2), the dG reverse cumsum (2)
-  return 2 + (tc ? 3 : 2) + (tc ? tc_bwd_kernel_count(d, plan_split(p, d).nslots) : 0) + 2 + 2;
+  const bool fwd_tc = p->algo != FIX_ALGO_SIMT && tc_fwd_supported(d);
+  const bool reuse = (p->flags & FIX_FLAG_REUSE_FWD_WORKSPACE) && (!tc || fwd_tc);
+  // schedule + prefix pass (the schedule alone when the forward's prefix is
+  // reused), preprocess (2, or 3 with the tensor-core operands), tensor-core
+  // dq / dk/dv / combine, the exact kernels (2), the dG reverse cumsum (2)
+  return (reuse ? 1 : 2) + (tc ? 3 : 2) + (tc ? tc_bwd_kernel_count(d, plan_split(p, d).nslots) : 0) +
+         2 + 2;
 }
 
 fix_status fix_attn_device_status(const void* workspace, void* stream) {
