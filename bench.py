@@ -169,6 +169,27 @@ class OracleSampler:
         self.pool.shutdown()
 
 
+# ------------------------------------------------------------------ ranks
+
+def max_over_ranks(values, device=None):
+    """Element-wise maximum of this rank's timings (ms) over the process group
+    (the job is as slow as its slowest rank); the values themselves when no
+    group is initialised or it has one rank."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(x) for x in values]
+    t = torch.tensor([float(x) for x in values], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t]
+
+
+def job_tflops(world, flops_per_step, steps, max_ms):
+    """Whole-job throughput under weak scaling: every rank runs `steps` steps of
+    `flops_per_step`, and the job takes the slowest rank's `max_ms`."""
+    return world * flops_per_step * steps / (max_ms * 1e-3) / 1e12
+
+
 # ------------------------------------------------------------------ main
 
 def main():
@@ -320,17 +341,13 @@ def main():
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     tot_ms = sum(step_ms)
     fwd_ms = statistics.mean(ev[i][0].elapsed_time(ev[i][3]) for i in range(args.steps))
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([tot_ms, fwd_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        tot_ms, fwd_ms = float(t[0]), float(t[1])
+    tot_ms, fwd_ms = max_over_ranks([tot_ms, fwd_ms], dev)
     ms_per_step = tot_ms / args.steps
 
     f_fwd = fwd_flops(case["seqlens"], Hq, Dk, Dv)
     f_step = 3.5 * f_fwd
-    value = world * f_step * args.steps / (tot_ms * 1e-3) / 1e12
-    fwd_tflops = world * f_fwd / (fwd_ms * 1e-3) / 1e12
+    value = job_tflops(world, f_step, args.steps, tot_ms)
+    fwd_tflops = job_tflops(world, f_fwd, 1, fwd_ms)
 
     # ---- end to end through host buffers (pinned), same metric
     e2e_ms = []
@@ -356,13 +373,8 @@ def main():
         torch.cuda.synchronize()
         if i > 0:
             e2e_ms.append(s_ev.elapsed_time(e_ev))
-    e2e_tot = sum(e2e_ms)
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([e2e_tot], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_tot = float(t[0])
-    e2e_val = world * f_step * len(e2e_ms) / (e2e_tot * 1e-3) / 1e12
+    e2e_tot, = max_over_ranks([sum(e2e_ms)], dev)
+    e2e_val = job_tflops(world, f_step, len(e2e_ms), e2e_tot)
 
     # ---- roofline of the dominant kernel stage
     pk, pk_kind = peaks()
