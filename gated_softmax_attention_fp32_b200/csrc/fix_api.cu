@@ -78,11 +78,13 @@ static int max_chunks_per_seq(const fix_attn_problem* p) {
 }
 
 // Work split of the dk/dv kernel: each key chunk's tiles (q heads x 64-row
-// query tiles of the chunks from it to the end of its sequence) are cut into
-// runs of at most P tiles, P chosen so that about two runs per SM cover the
-// problem.  Planned with the B200's 148 SMs whatever the device: the split
-// only affects load balance, and the plan must not depend on a device query
-// so that the workspace size agrees between sizing and calling.
+// query tiles) are taken in two kinds, those of the chunk itself (the
+// diagonal) and those of the later chunks of its sequence, and each kind is
+// cut into runs of at most P tiles, P chosen so that about two runs per SM
+// cover the problem.  Every run (part) owns one slot of fp32 partial sums.
+// Planned with the B200's 148 SMs whatever the device: the split only affects
+// load balance, and the plan must not depend on a device query so that the
+// workspace size agrees between sizing and calling.
 struct SplitPlan {
   int P = 0;
   long long nparts = 0, nslots = 0;
