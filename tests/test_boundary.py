@@ -69,6 +69,73 @@ def test_workspace_sizes(lib):
     assert lib.fix_attn_workspace_bytes(None, 0) == 0
 
 
+def _ceil(a, b):
+    return -(-a // b)
+
+
+def _expected_workspace(seqlens, Hq, Hkv, Dk, Dv, backward):
+    """The workspace layout written out from its documented parts: 256-byte
+    aligned buffers, and for the backward the dk/dv split (per key chunk, its
+    diagonal tiles and its later tiles, each cut into runs of at most P tiles,
+    P sized for about two runs per SM of a 148-SM B200), one partial slot of
+    128 rows x (Dk + Dv) floats per run and kv head."""
+    grp = Hq // Hkv
+    N = sum(seqlens)
+    nchunks = sum(_ceil(L, 128) for L in seqlens)
+    nc1 = max(nchunks, 1)
+    o = 0
+
+    def take(nbytes):
+        nonlocal o
+        o = _ceil(o + nbytes, 256) * 256
+
+    nkv, nch = N * Hkv * Dv, nchunks * Hkv * Dv
+    for nbytes in (256, nc1 * 16, nc1 * 4, nc1 * Hkv * 4, nkv * 4, nkv * 2, nkv * 2, nkv * 2,
+                   nch * 4, nch * 4, nch * 4):
+        take(nbytes)
+    if not backward:
+        return o
+    t64 = lambda L, j: (L - 128 * j + 63) // 64          # query tiles from chunk j on
+    half = lambda L, j: (min(128, L - 128 * j) + 63) // 64
+    total = Hkv * sum(grp * t64(L, j) for L in seqlens for j in range(_ceil(L, 128)))
+    P = max(4, _ceil(total, 2 * 148))
+    nparts = sum(_ceil(grp * half(L, j), P) + _ceil(grp * (t64(L, j) - half(L, j)), P)
+                 for L in seqlens for j in range(_ceil(L, 128)))
+    for nbytes in (N * Hq * Dv * 4, N * Hq * Dv * 2, N * Hq * Dv * 2, N * Hq * Dv * 2,
+                   nc1 * Hq * 4, nc1 * Hq * 4, N * Hq * 4, nkv * 4, nkv * 4, nch * 4,
+                   nc1 * 4 * Hkv * Dv * 4, max(nparts, 1) * 16, nc1 * 8,
+                   nparts * Hkv * 128 * (Dk + Dv) * 4):
+        take(nbytes)
+    return o
+
+
+@pytest.mark.parametrize("seqlens,Hq,Hkv,Dk,Dv", [
+    ([2048, 2048], 8, 4, 128, 128),
+    ([100, 100], 4, 2, 64, 64),
+    ([2817, 6892, 6576, 99], 16, 4, 128, 128),
+    ([0, 1, 130, 7, 255, 0, 64, 300], 4, 2, 64, 128),
+    ([4096] * 8, 16, 16, 64, 64),
+    ([129, 640], 32, 2, 128, 64),
+])
+def test_workspace_layout_and_dkv_split(lib, seqlens, Hq, Hkv, Dk, Dv):
+    """Sizes the workspace (and so the dk/dv work split it holds slots for)
+    the way the host plans it, for fixed-length and packed problems."""
+    if len(set(seqlens)) == 1:
+        p = prob(B=len(seqlens), T=seqlens[0], Hq=Hq, Hkv=Hkv, Dk=Dk, Dv=Dv)
+        keep = None
+    else:
+        cu = [0]
+        for L in seqlens:
+            cu.append(cu[-1] + L)
+        keep = (ctypes.c_int64 * len(cu))(*cu)
+        p = prob(B=1, T=cu[-1], Hq=Hq, Hkv=Hkv, Dk=Dk, Dv=Dv, num_seqs=len(seqlens),
+                 cu_seqlens_host=ctypes.addressof(keep), cu_seqlens=ctypes.addressof(keep))
+    for backward in (0, 1):
+        got = lib.fix_attn_workspace_bytes(ctypes.byref(p), backward)
+        assert got == _expected_workspace(seqlens, Hq, Hkv, Dk, Dv, backward), (backward, got)
+    del keep
+
+
 @pytest.mark.parametrize("kw,code", [
     (dict(Dk=48), FIX_ERR_HEAD_DIM),
     (dict(Dv=256), FIX_ERR_HEAD_DIM),
