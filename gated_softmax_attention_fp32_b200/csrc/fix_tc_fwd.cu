@@ -33,10 +33,13 @@
 //
 // Warp roles (384 threads): warp 0 issues TMA loads (Q once; K and V tiles
 // through a 2-stage ring), warp 1 issues the MMAs (one thread) and owns TMEM,
-// warps 4-7 turn S into P (one TMEM lane = one query row per thread) and run
-// the epilogue (row factor, RMSNorm, stores), warps 8-11 scale the V tiles in
-// shared memory by f_ij.  TMEM: two S buffers (P is written over the S it came
-// from, as bf16 pairs) and the O accumulator.
+// warps 4-7 turn S into P (one TMEM lane = one query row per thread) and move
+// the accumulators to a shared fp32 tile (epilogue phase A), warps 8-11 scale
+// the V tiles in shared memory by f_ij.  Once every MMA has completed (the
+// MMA warp's single-use `drain` barrier), all twelve warps run epilogue phase
+// B: row factor, the s = t term, RMSNorm and coalesced stores, a row per warp
+// at a time.  TMEM: two S buffers (P is written over the S it came from, as
+// 16-bit pairs) and the two O accumulators.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
