@@ -218,3 +218,22 @@ def test_status_strings(lib):
         s = fixattn.status_string(c)
         assert s.startswith("FIX_")
     assert "unknown" in fixattn.status_string(99)
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    """No fallback on the product path: without the CUDA library every call
+    raises instead of computing anything another way."""
+    import subprocess
+    import sys
+    code = (
+        "import sys; sys.path.insert(0, %r)\n"
+        "from gated_softmax_attention_fp32_b200 import fixattn\n"
+        "fixattn.LIB_PATH = %r\n"
+        "try:\n"
+        "    fixattn.load()\n"
+        "except RuntimeError as e:\n"
+        "    print('raised:', e)\n"
+        "    sys.exit(0)\n"
+        "sys.exit(1)\n" % (ROOT, str(tmp_path / "absent.so")))
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0 and "not built" in r.stdout, r.stdout + r.stderr
