@@ -19,6 +19,10 @@
 // device status word) and writes every other workspace byte before reading
 // it.  Calls whose executions overlap on the GPU (different streams, or
 // different host threads without ordering) race on the array.
+//
+// Status: the array's first word is the forward's device status word (where a
+// bounded device wait that expired reports); fix_attn_noalloc_device_status
+// reads it, since a caller of this entry point never sees the array's address.
 #include <mutex>
 
 #include "fix_attn.h"
@@ -64,4 +68,11 @@ extern "C" fix_status fix_attn_fwd_noalloc(const fix_attn_problem* p, const void
   if (s != FIX_OK) return s;
   return fix_attn_fwd(p, q, k, v, g, o_norm_weight, y, o_saved, m_saved, rstd_saved, ws,
                       FIX_NOALLOC_MAX_WORKSPACE_BYTES, stream);
+}
+
+extern "C" fix_status fix_attn_noalloc_device_status(void* stream) {
+  void* ws = nullptr;
+  const fix_status s = scratch_on_current_device(&ws);
+  if (s != FIX_OK) return s;
+  return fix_attn_device_status(ws, stream);
 }

@@ -25,7 +25,8 @@ __all__ = ["load", "Problem", "fix_attn_fwd", "fix_attn_bwd", "fix_attn_workspac
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfixattn.so")
 EXPORTS = ("fix_attn_workspace_bytes", "fix_attn_fwd", "fix_attn_bwd", "fix_attn_device_status",
-           "fix_attn_kernel_count", "fix_attn_status_string", "fix_attn_fwd_noalloc")
+           "fix_attn_kernel_count", "fix_attn_status_string", "fix_attn_fwd_noalloc",
+           "fix_attn_noalloc_device_status")
 NOALLOC_MAX_WORKSPACE_BYTES = 16 * 1024 * 1024
 FIX_FLAG_REUSE_FWD_WORKSPACE = 1
 STAGES = ("fwd_prefix", "fwd_attn", "bwd_prefix", "bwd_pre", "bwd_dq", "bwd_dkv", "bwd_dg",
@@ -73,6 +74,8 @@ def load():
     lib.fix_attn_fwd_noalloc.restype = ctypes.c_int
     lib.fix_attn_device_status.argtypes = [vp, vp]
     lib.fix_attn_device_status.restype = ctypes.c_int
+    lib.fix_attn_noalloc_device_status.argtypes = [vp]
+    lib.fix_attn_noalloc_device_status.restype = ctypes.c_int
     lib.fix_attn_kernel_count.argtypes = [P, ctypes.c_int]
     lib.fix_attn_kernel_count.restype = ctypes.c_int
     lib.fix_attn_status_string.argtypes = [ctypes.c_int]
@@ -228,6 +231,12 @@ def training_workspace(q, k, v, cu_seqlens=None, cu_seqlens_host=None, algo="aut
 
 def fix_attn_device_status(workspace, stream=None) -> int:
     return int(load().fix_attn_device_status(_ptr(workspace), _stream(stream)))
+
+
+def fix_attn_noalloc_device_status(stream=None) -> int:
+    """Device status word of the last fix_attn_fwd_noalloc call on the current
+    device (synchronises the stream)."""
+    return int(load().fix_attn_noalloc_device_status(_stream(stream)))
 
 
 class _FixAttn(torch.autograd.Function):

@@ -20,8 +20,10 @@
  *
  * Conventions for every entry point:
  *   - Ownership: the caller allocates and owns every buffer.  The library never
- *     allocates, frees or synchronises (except fix_attn_device_status) and keeps
- *     no mutable global state besides cached kernel attributes.
+ *     allocates, frees or synchronises (except the two device-status readers)
+ *     and keeps no mutable global state besides cached kernel attributes, with
+ *     one exception: the fixed device array behind fix_attn_fwd_noalloc (and
+ *     its per-device address cache), described beside that entry point.
  *   - Execution: calls are asynchronous and ordered on `stream` (a cudaStream_t
  *     passed as void*; NULL = legacy default stream).  Every element of every
  *     output is written.
@@ -156,8 +158,11 @@ fix_status fix_attn_bwd(const fix_attn_problem *p, const void *q, const void *k,
  * fix_attn_fwd / fix_attn_bwd call. */
 fix_status fix_attn_device_status(const void *workspace, void *stream);
 
-/* Largest workspace fix_attn_fwd_noalloc can provide (16 MiB; enough for the
- * forward of e.g. 4096 tokens x 4 kv heads x Dv 128). */
+/* Largest workspace fix_attn_fwd_noalloc can provide: 16 MiB.  The forward's
+ * workspace is about 10 bytes per (token, kv head, value channel) plus a few
+ * KB, so the array covers N * Hkv * Dv up to about 1.6 million: e.g. 3,200
+ * tokens x 4 kv heads x Dv 128, or 6,400 tokens x 4 kv heads x Dv 64.
+ * fix_attn_workspace_bytes(p, 0) gives the exact figure for a problem. */
 #define FIX_NOALLOC_MAX_WORKSPACE_BYTES (16u * 1024u * 1024u)
 
 /* Forward for callers that cannot allocate device memory.  (The FiX pages
@@ -178,11 +183,20 @@ fix_status fix_attn_device_status(const void *workspace, void *stream);
  *     first call before any stream capture.
  *   - All calls on a device share the array, which keeps the last call's
  *     contents; calls that overlap on the GPU (other streams or unordered
- *     host threads) race on it.  Order them on one stream. */
+ *     host threads) race on it.  Order them on one stream.
+ *   - A bounded device wait that expires records FIX_ERR_DEVICE_TIMEOUT in
+ *     the array's status word; fix_attn_noalloc_device_status reads it. */
 fix_status fix_attn_fwd_noalloc(const fix_attn_problem *p, const void *q, const void *k,
                                 const void *v, const float *g, const void *o_norm_weight,
                                 void *y, float *o_saved, float *m_saved, float *rstd_saved,
                                 void *stream);
+
+/* fix_attn_device_status for fix_attn_fwd_noalloc: synchronises `stream`,
+ * then returns the status word that the last fix_attn_fwd_noalloc call on
+ * the current device left in the library's array (FIX_OK or
+ * FIX_ERR_DEVICE_TIMEOUT; FIX_OK before any such call), or FIX_ERR_CUDA if
+ * the stream reports an error.  Allocates nothing. */
+fix_status fix_attn_noalloc_device_status(void *stream);
 
 /* Number of kernels that fix_attn_fwd (backward = 0) or fix_attn_bwd
  * (backward = 1) launches for this problem (0 if it is invalid). */

@@ -99,3 +99,41 @@ def sample_rows(L, n, rng):
             rows.add(e)
     rows.update(int(x) for x in rng.integers(0, L, size=n))
     return sorted(rows)
+
+
+def sequence_case(case, b, s0, L):
+    """The inputs of one sequence of ``case`` as a dense B = 1 problem (the
+    operator never mixes sequences, so its outputs on these rows are the same
+    as in the packed problem)."""
+    out = dict(case)
+    for key in ("q", "k", "v", "g", "dy"):
+        if case.get(key) is not None:
+            out[key] = case[key][b:b + 1, s0:s0 + L].contiguous()
+    out.update(B=1, T=L, cu_seqlens=None, seqlens=[L])
+    return out
+
+
+def _suffix_job(args):
+    q, k, v, g, w, dy, L, R, eps = args
+    return fix_ref.suffix_backward(q, k, v, g, w, dy, 0, L, 0, R, None, eps)
+
+
+def oracle_suffix(case, picks, R):
+    """dk, dv, dg of the last R key rows of (b, start, L, kv) picks, from the
+    oracle's suffix backward, one pick per process of a spawn pool.  Each job
+    gets only its sequence and its kv group (so kv = 0 inside the job)."""
+    import multiprocessing as mp
+    from concurrent.futures import ProcessPoolExecutor
+    grp = case["Hq"] // case["Hkv"]
+    jobs = []
+    for b, s0, L, kv in picks:
+        sl = slice(s0, s0 + L)
+        hs = slice(kv * grp, (kv + 1) * grp)
+        jobs.append((case["q"][b:b + 1, sl, hs], case["k"][b:b + 1, sl, kv:kv + 1],
+                     case["v"][b:b + 1, sl, kv:kv + 1], case["g"][b:b + 1, sl, kv:kv + 1],
+                     case["w"], case["dy"][b:b + 1, sl, hs], L, min(R, L), case["eps"]))
+    n = max(1, min(workers(), len(jobs)))
+    if n == 1:
+        return [_suffix_job(j) for j in jobs]
+    with ProcessPoolExecutor(max_workers=n, mp_context=mp.get_context("spawn")) as ex:
+        return list(ex.map(_suffix_job, jobs))

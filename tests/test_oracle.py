@@ -334,3 +334,29 @@ def test_row_helpers_match_full_oracle():
     sl = slice(start + L - R, start + L)
     for key in ("dk", "dv", "dg"):
         assert relerr(sb[key], grads[key][0, sl, 1]) < 1e-12, key
+
+
+def test_process_pool_equals_serial():
+    """The GPU parity tests run the oracle over a spawn process pool
+    (workers > 1); its results must be bit-identical to the serial branch,
+    which the pins above check.  Each (sequence, head) unit is computed by the
+    same function either way, so any difference would come from the pool's
+    job bookkeeping (a unit written to the wrong place, a group sum taken
+    twice or missed)."""
+    rng = np.random.default_rng(17)
+    q, k, v, g, w, dy = make(rng, 1, 23, 4, 2, 4, 4)
+    seqlens = [5, 0, 11, 7]
+    serial_f = fix_ref.forward(q, k, v, g, w, seqlens, None, 1e-6, workers=1)
+    pool_f = fix_ref.forward(q, k, v, g, w, seqlens, None, 1e-6, workers=2)
+    serial_b = fix_ref.backward(q, k, v, g, w, dy, seqlens, None, 1e-6, workers=1)
+    pool_b = fix_ref.backward(q, k, v, g, w, dy, seqlens, None, 1e-6, workers=2)
+    for key in serial_f:
+        assert np.array_equal(serial_f[key], pool_f[key]), key
+    for key in serial_b:
+        assert np.array_equal(serial_b[key], pool_b[key]), key
+    # batched (B > 1) problems take the same path
+    q, k, v, g, w, dy = make(rng, 3, 9, 2, 1, 4, 2)
+    a = fix_ref.backward(q, k, v, g, w, dy, None, None, 1e-6, workers=1)
+    b = fix_ref.backward(q, k, v, g, w, dy, None, None, 1e-6, workers=3)
+    for key in a:
+        assert np.array_equal(a[key], b[key]), key

@@ -14,8 +14,9 @@ import pytest
 import torch
 
 import synth
-from fixtools import (FWD_MAX_ABS, FWD_REL_L2, GRAD_REL_L2, max_abs, oracle_full, rel_l2,
-                      run_gpu, sample_rows, segments, workers)
+from fixtools import (FWD_MAX_ABS, FWD_REL_L2, GRAD_REL_L2, max_abs, oracle_full,
+                      oracle_suffix, rel_l2, run_gpu, sample_rows, segments, sequence_case,
+                      workers)
 from oracle import fix_ref
 
 pytestmark = pytest.mark.gpu
@@ -44,8 +45,11 @@ def check_grad(name, x, ref, tag=""):
 
 SMALL = {
     "T1": dict(B=1, T=1, Hq=1, Hkv=1, Dk=64, Dv=64),
-    "B2-T63-gqa": dict(B=2, T=63, Hq=4, Hkv=2, Dk=64, Dv=64),
-    "T100-D128": dict(B=1, T=100, Hq=2, Hkv=1, Dk=128, Dv=128),
+    # fewer than 128 tokens in all: the exact CUDA-core kernels
+    "B2-T63-gqa-exact": dict(B=2, T=63, Hq=4, Hkv=2, Dk=64, Dv=64),
+    # one ragged chunk per sequence on the tensor-core kernels
+    "B3-T63-gqa": dict(B=3, T=63, Hq=4, Hkv=2, Dk=64, Dv=64),
+    "B2-T100-D128": dict(B=2, T=100, Hq=2, Hkv=1, Dk=128, Dv=128),
     "T129-D32": dict(B=1, T=129, Hq=2, Hkv=2, Dk=32, Dv=32),
     "B2-T300-D16": dict(B=2, T=300, Hq=4, Hkv=1, Dk=16, Dv=16),
     "T257-Dk64-Dv128": dict(B=1, T=257, Hq=2, Hkv=1, Dk=64, Dv=128),
@@ -185,10 +189,9 @@ def _sampled_dq(case, gpu, rows_per_seq, heads, seed=1):
 
 
 def _suffix(case, gpu, picks, R):
+    res = oracle_suffix(case, picks, R)
     out = {k: ([], []) for k in ("dk", "dv", "dg")}
-    for b, s0, L, kv in picks:
-        r = fix_ref.suffix_backward(case["q"], case["k"], case["v"], case["g"], case["w"],
-                                    case["dy"], s0, L, kv, min(R, L), None, case["eps"], b=b)
+    for (b, s0, L, kv), r in zip(picks, res):
         sl = slice(s0 + L - min(R, L), s0 + L)
         for key in out:
             out[key][0].append(gpu[key][b, sl, kv])
@@ -207,17 +210,39 @@ def _properties(case, gpu):
 
 
 def test_workload3_varlen_sampled(cuda_lib):
+    """Packed sequences of 2817, 6892, 6576 and 99 tokens.  The two short ones
+    get the full oracle (every output and gradient of their rows); the two
+    long ones sampled forward / dq rows and the last 384 key rows of dk, dv,
+    dg for the first and last kv head: those keys span three 128-token
+    chunks, so their later-block dk/dv parts and the combine of several
+    partial slots are compared, not only the diagonal.  dw is a sum over all
+    rows: it is checked against sum(dy * y / w), which holds exactly for the
+    float32 y whose rows are compared with the oracle above."""
     case = synth.draw(synth.workload(3))
     gpu = run_gpu(case, backward=True)
     _properties(case, gpu)
+    segs = segments(case)
+    short = [s for s in segs if s[2] <= 3000]
+    long_ = [s for s in segs if s[2] > 3000]
+    assert short and long_
+    for b, s0, L in short:
+        sub = sequence_case(case, b, s0, L)
+        ref = oracle_full(sub, backward=True)
+        sl = slice(s0, s0 + L)
+        check_fwd(gpu["y"][b, sl], ref["y"][0], f"workload 3 seq len {L}")
+        for key in ("dq", "dk", "dv", "dg"):
+            check_grad(key, gpu[key][b, sl], ref[key][0], f"workload 3 seq len {L}")
     y, ref = _sampled_forward(case, gpu, 24, range(case["Hq"]))
     check_fwd(y, ref, "workload 3")
     x, ref = _sampled_dq(case, gpu, 6, range(0, case["Hq"], 3))
     check_grad("dq", x, ref, "workload 3")
-    segs = segments(case)
-    picks = [(b, s0, L, kv) for (b, s0, L) in segs for kv in (0, case["Hkv"] - 1)]
-    for key, (x, ref) in _suffix(case, gpu, picks, 48).items():
-        check_grad(key, x, ref, "workload 3")
+    picks = [(b, s0, L, kv) for (b, s0, L) in long_ for kv in (0, case["Hkv"] - 1)]
+    for key, (x, ref) in _suffix(case, gpu, picks, 384).items():
+        check_grad(key, x, ref, "workload 3 (last 384 keys)")
+    w = case["w"].double().numpy()
+    dy = case["dy"].double().numpy()
+    dw_from_y = (dy * gpu["y"] / w).sum(axis=(0, 1, 2))
+    check_grad("dw", gpu["dw"], dw_from_y, "workload 3 (sum dy*y/w)")
 
 
 def test_workload4_long_context_sampled(cuda_lib):
