@@ -41,6 +41,21 @@ factorisation, no cancellation-prone identity):
       dg_r   = sum_{t>=r} dG_t                    (within the sequence)
     dk, dv, dg are summed over the q heads of each kv group.
 
+Options of the same call (FiX README, "Quick Start": ``o_norm``,
+``o_norm_weight``, ``o_gate``; Forgetting Transformer abstract: scalar
+forget gates), each a reading of points the pages leave open:
+
+  o_norm = False   no RMSNorm; the output is the attention average with the
+                   ordinary softmax denominator, o_t / l_t with
+                   l_t = sum_{s<=t} P_ts (so g = 0 gives causal softmax
+                   attention), and m_t drops out exactly
+  o_gate z         y <- y * swish(z) = y * z * sigmoid(z), after the norm and
+                   its weight (the output-gate form of the library FiX is
+                   forked from); z has y's shape [B,T,Hq,Dv]
+  scalar gate      g of shape [B,T,Hkv]: one forget gate per (token, kv head),
+                   the same for every value channel; FiX with g broadcast over
+                   the channels, and dg is the channel sum of that gradient
+
 Pins (see tests/test_oracle.py): brute-force loops, finite differences,
 library identities (g = 0 is RMSNorm of ordinary causal softmax attention;
 channel-constant g is Forgetting-Transformer attention), closed forms and
@@ -55,7 +70,7 @@ import numpy as np
 
 __all__ = [
     "unit_forward", "unit_backward", "forward", "backward",
-    "forward_rows", "dq_rows", "suffix_backward", "to64",
+    "forward_rows", "dq_rows", "suffix_backward", "to64", "swish", "swish_grad",
 ]
 
 
@@ -74,12 +89,24 @@ def to64(x) -> np.ndarray:
 # One (sequence, q-head) unit
 # --------------------------------------------------------------------------
 
-def unit_forward(Q, K, V, g, w, scale, eps, m_fixed=None):
+def swish(z):
+    """z * sigmoid(z)."""
+    return z / (1.0 + np.exp(-z))
+
+
+def swish_grad(z):
+    """d/dz of z * sigmoid(z) = sigmoid(z) * (1 + z * (1 - sigmoid(z)))."""
+    sg = 1.0 / (1.0 + np.exp(-z))
+    return sg * (1.0 + z * (1.0 - sg))
+
+
+def unit_forward(Q, K, V, g, w, scale, eps, m_fixed=None, norm=True, z=None):
     """Forward of one (sequence, q head) unit in fp64.
 
     Q [L,Dk], K [L,Dk], V [L,Dv], g [L,Dv] (the kv head's tensors), w [Dv].
     ``m_fixed`` (optional [L]) replaces the row max; used by finite-difference
-    tests that hold the per-row shift constant.
+    tests that hold the per-row shift constant.  ``norm = False``: y is
+    o_t / l_t (no RMSNorm, no weight); ``z`` [L,Dv]: y <- y * swish(z).
     Returns y, o, m, rstd, P, G.
     """
     L = Q.shape[0]
@@ -99,25 +126,45 @@ def unit_forward(Q, K, V, g, w, scale, eps, m_fixed=None):
         o[t] = np.einsum("s,sc,sc->c", P[t, : t + 1], D, V[: t + 1])
     rstd = 1.0 / np.sqrt((o * o).mean(axis=1) + eps)
     y = o * rstd[:, None] * w[None, :]
+    if not norm:
+        y = o / P.sum(axis=1)[:, None]             # softmax denominator l_t
+    if z is not None:
+        y = y * swish(z)
     return y, o, m, rstd, P, G
 
 
-def unit_backward(Q, K, V, g, w, dy, scale, eps):
+def unit_backward(Q, K, V, g, w, dy, scale, eps, norm=True, z=None):
     """Analytic backward of one (sequence, q head) unit in fp64.
 
-    Returns dQ [L,Dk], dK [L,Dk], dV [L,Dv], dg [L,Dv], dw [Dv] for this q
-    head (dK, dV, dg are this head's share of the kv head's gradients).
+    Returns dQ [L,Dk], dK [L,Dk], dV [L,Dv], dg [L,Dv], dw [Dv], dz [L,Dv]
+    (None without an output gate) for this q head (dK, dV, dg are this
+    head's share of the kv head's gradients).  With ``norm = False`` the
+    softmax denominator is part of the function: P is normalised and
+    dS_ts = P_ts (dP_ts - sum_c do_t[c] o_t[c]), the exact derivative.
     """
     L, Dk = Q.shape
     Dv = V.shape[1]
     if L == 0:
         return (np.zeros((0, Dk)), np.zeros((0, Dk)), np.zeros((0, Dv)),
-                np.zeros((0, Dv)), np.zeros(Dv))
+                np.zeros((0, Dv)), np.zeros(Dv), None if z is None else np.zeros((0, Dv)))
     y, o, m, rstd, P, G = unit_forward(Q, K, V, g, w, scale, eps)
-    n = o * rstd[:, None]
-    dw = (dy * n).sum(axis=0)
-    dn = dy * w[None, :]
-    do = rstd[:, None] * (dn - n * (dn * n).mean(axis=1, keepdims=True))
+    if z is not None:
+        dy_gated = dy
+        dy = dy_gated * swish(z)                   # gradient of the ungated output
+    if norm:
+        n = o * rstd[:, None]
+        u = n * w[None, :]                         # ungated output
+        dw = (dy * n).sum(axis=0)
+        dn = dy * w[None, :]
+        do = rstd[:, None] * (dn - n * (dn * n).mean(axis=1, keepdims=True))
+    else:
+        ell = P.sum(axis=1)
+        P = P / ell[:, None]                       # normalised weights
+        o = o / ell[:, None]
+        u = o
+        dw = np.zeros(Dv)
+        do = dy
+    dz = None if z is None else dy_gated * u * swish_grad(z)
     dV = np.zeros((L, Dv))
     dG = np.zeros((L, Dv))
     dP = np.zeros((L, L))
@@ -129,10 +176,12 @@ def unit_backward(Q, K, V, g, w, dy, scale, eps):
         dG[t] += do[t] * o[t]
         dG[: t + 1] -= W * do[t][None, :] * V[: t + 1]
     dS = P * dP
+    if not norm:
+        dS = P * (dP - (do * o).sum(axis=1)[:, None])
     dQ = scale * (dS @ K)
     dK = scale * (dS.T @ Q)
     dg = np.cumsum(dG[::-1], axis=0)[::-1]         # dg_r = sum_{t>=r} dG_t
-    return dQ, dK, dV, dg, dw
+    return dQ, dK, dV, dg, dw, dz
 
 
 # --------------------------------------------------------------------------
@@ -152,8 +201,9 @@ def _segments(B, T, seqlens):
 
 
 def _fwd_job(args):
-    Q, K, V, g, w, scale, eps = args
-    y, o, m, rstd, _, _ = unit_forward(Q, K, V, g, w, scale, eps)
+    Q, K, V, g, w, scale, eps = args[:7]
+    norm, z = (args[7], args[8]) if len(args) > 7 else (True, None)
+    y, o, m, rstd, _, _ = unit_forward(Q, K, V, g, w, scale, eps, None, norm, z)
     return y, o, m, rstd
 
 
@@ -174,15 +224,24 @@ def _pool_map(fn, jobs, workers):
         return list(ex.map(fn, jobs))
 
 
-def forward(q, k, v, g, w, seqlens=None, scale=None, eps=1e-6, workers=None):
-    """Full forward.  q [B,T,Hq,Dk], k [B,T,Hkv,Dk], v/g [B,T,Hkv,Dv], w [Dv].
+def _channel_gate(g, Dv):
+    """A scalar gate [B,T,Hkv] as the element-wise gate it stands for."""
+    return np.repeat(g[..., None], Dv, axis=-1) if g.ndim == 3 else g
+
+
+def forward(q, k, v, g, w, seqlens=None, scale=None, eps=1e-6, workers=None, norm=True,
+            o_gate=None):
+    """Full forward.  q [B,T,Hq,Dk], k [B,T,Hkv,Dk], v [B,T,Hkv,Dv], g
+    [B,T,Hkv,Dv] (or [B,T,Hkv]: scalar gate), w [Dv], o_gate None or
+    [B,T,Hq,Dv].
 
     ``seqlens`` (B == 1) lists packed sequence lengths.  Returns a dict of
     float64 arrays: y, o [B,T,Hq,Dv]; m, rstd [B,T,Hq].
     """
-    q, k, v, g, w = (to64(x) for x in (q, k, v, g, w))
+    q, k, v, g, w, o_gate = (to64(x) for x in (q, k, v, g, w, o_gate))
     B, T, Hq, Dk = q.shape
     Hkv, Dv = v.shape[2], v.shape[3]
+    g = _channel_gate(g, Dv)
     assert Hq % Hkv == 0
     grp = Hq // Hkv
     if scale is None:
@@ -193,6 +252,8 @@ def forward(q, k, v, g, w, seqlens=None, scale=None, eps=1e-6, workers=None):
             kv = h // grp
             sl = slice(s0, s0 + L)
             jobs.append((q[b, sl, h], k[b, sl, kv], v[b, sl, kv], g[b, sl, kv], w, scale, eps))
+            if not norm or o_gate is not None:
+                jobs[-1] += (norm, None if o_gate is None else o_gate[b, sl, h])
             where.append((b, sl, h))
     res = _pool_map(_fwd_job, jobs, workers)
     y = np.zeros((B, T, Hq, Dv)); o = np.zeros((B, T, Hq, Dv))
@@ -202,11 +263,16 @@ def forward(q, k, v, g, w, seqlens=None, scale=None, eps=1e-6, workers=None):
     return dict(y=y, o=o, m=m, rstd=rstd)
 
 
-def backward(q, k, v, g, w, dy, seqlens=None, scale=None, eps=1e-6, workers=None):
-    """Full analytic backward of L = sum(dy * y).  Returns dq, dk, dv, dg, dw."""
-    q, k, v, g, w, dy = (to64(x) for x in (q, k, v, g, w, dy))
+def backward(q, k, v, g, w, dy, seqlens=None, scale=None, eps=1e-6, workers=None, norm=True,
+             o_gate=None):
+    """Full analytic backward of L = sum(dy * y).  Returns dq, dk, dv, dg, dw
+    (and d_o_gate with an output gate); for a scalar gate [B,T,Hkv], dg has
+    that shape."""
+    q, k, v, g, w, dy, o_gate = (to64(x) for x in (q, k, v, g, w, dy, o_gate))
     B, T, Hq, Dk = q.shape
     Hkv, Dv = v.shape[2], v.shape[3]
+    scalar_gate = g.ndim == 3
+    g = _channel_gate(g, Dv)
     grp = Hq // Hkv
     if scale is None:
         scale = Dk ** -0.5
@@ -217,17 +283,25 @@ def backward(q, k, v, g, w, dy, seqlens=None, scale=None, eps=1e-6, workers=None
             sl = slice(s0, s0 + L)
             jobs.append((q[b, sl, h], k[b, sl, kv], v[b, sl, kv], g[b, sl, kv], w,
                          dy[b, sl, h], scale, eps))
+            if not norm or o_gate is not None:
+                jobs[-1] += (norm, None if o_gate is None else o_gate[b, sl, h])
             where.append((b, sl, h, kv))
     res = _pool_map(_bwd_job, jobs, workers)
     dq = np.zeros_like(q); dk = np.zeros_like(k); dv = np.zeros_like(v)
     dg = np.zeros_like(g); dw = np.zeros(Dv)
-    for (b, sl, h, kv), (a, bk, bv, bg, bw) in zip(where, res):
+    dz = None if o_gate is None else np.zeros_like(o_gate)
+    for (b, sl, h, kv), (a, bk, bv, bg, bw, bz) in zip(where, res):
         dq[b, sl, h] = a
         dk[b, sl, kv] += bk
         dv[b, sl, kv] += bv
         dg[b, sl, kv] += bg
         dw += bw
-    return dict(dq=dq, dk=dk, dv=dv, dg=dg, dw=dw)
+        if dz is not None:
+            dz[b, sl, h] = bz
+    out = dict(dq=dq, dk=dk, dv=dv, dg=dg.sum(axis=-1) if scalar_gate else dg, dw=dw)
+    if dz is not None:
+        out["d_o_gate"] = dz
+    return out
 
 
 # --------------------------------------------------------------------------

@@ -360,3 +360,114 @@ def test_process_pool_equals_serial():
     b = fix_ref.backward(q, k, v, g, w, dy, None, None, 1e-6, workers=3)
     for key in a:
         assert np.array_equal(a[key], b[key]), key
+
+
+# ----------------------------------------- o_gate, o_norm = False, scalar gate
+# FiX README "Quick Start": o_norm, o_norm_weight and o_gate are arguments of
+# the same call; the Forgetting Transformer abstract: scalar forget gates.
+
+def test_output_gate_is_swish_after_norm_and_weight():
+    """y with o_gate z equals y without it times torch's silu(z) = z sigmoid(z),
+    element by element, with and without the RMSNorm."""
+    rng = np.random.default_rng(31)
+    q, k, v, g, w, _ = make(rng, 2, 9, 4, 2, 4, 6)
+    z = 2.0 * rnd(rng, 2, 9, 4, 6)
+    silu = torch.nn.functional.silu(torch.from_numpy(z)).numpy()
+    for norm in (True, False):
+        a = fix_ref.forward(q, k, v, g, w, None, 0.6, 1e-6, norm=norm)["y"]
+        b = fix_ref.forward(q, k, v, g, w, None, 0.6, 1e-6, norm=norm, o_gate=z)["y"]
+        assert relerr(b, a * silu) < 1e-14
+
+
+def test_no_norm_zero_gate_is_causal_softmax_attention():
+    """o_norm = False with g = 0 is ordinary causal softmax attention (torch
+    SDPA), whatever eps, and does not depend on the row shift."""
+    rng = np.random.default_rng(32)
+    T, Hq, Hkv, D = 31, 4, 2, 8
+    q, k, v, _, w, _ = make(rng, 1, T, Hq, Hkv, D, D)
+    g = np.zeros((1, T, Hkv, D))
+    kr, vr = np.repeat(k[0], 2, axis=1), np.repeat(v[0], 2, axis=1)
+    sd = _sdpa(q[0], kr, vr, scale=0.3)
+    y = fix_ref.forward(q, k, v, g, w, None, 0.3, 1e-3, norm=False)["y"][0]
+    assert relerr(y, sd) < 1e-13
+
+
+def test_no_norm_closed_forms():
+    rng = np.random.default_rng(33)
+    # T = 1: the output is v_0
+    q, k, v, g, w, _ = make(rng, 2, 1, 2, 1, 4, 4)
+    y = fix_ref.forward(q, k, v, g, w, None, None, 1e-6, norm=False)["y"]
+    assert relerr(y, np.repeat(v, 2, axis=2)) < 1e-15
+    # total forgetting: o_t = softmax_t(S)[t] v_t
+    T = 7
+    q, k, v, _, w, _ = make(rng, 1, T, 1, 1, 3, 3)
+    g = np.full(v.shape, -1e4)
+    y = fix_ref.forward(q, k, v, g, w, None, 0.5, 0.0, norm=False)["y"][0, :, 0]
+    S = 0.5 * q[0, :, 0] @ k[0, :, 0].T
+    Sm = np.where(np.tri(T, dtype=bool), S, -np.inf)
+    p = np.exp(Sm - Sm.max(1, keepdims=True))
+    p /= p.sum(1, keepdims=True)
+    assert relerr(y, np.diag(p)[:, None] * v[0, :, 0]) < 1e-13
+
+
+def _fd_variant(norm, gated, scalar, seed):
+    rng = np.random.default_rng(seed)
+    B, T, Hq, Hkv, Dk, Dv = 1, 5, 2, 1, 3, 3
+    q, k, v, g, w, dy = make(rng, B, T, Hq, Hkv, Dk, Dv)
+    if scalar:
+        g = g[..., 0].copy()
+    z = rnd(rng, B, T, Hq, Dv) if gated else None
+    scale, eps = 0.8, 1e-2
+    grads = fix_ref.backward(q, k, v, g, w, dy, None, scale, eps, norm=norm, o_gate=z)
+    m0 = fix_ref.forward(q, k, v, g, w, None, scale, eps)["m"]
+    args = dict(q=q, k=k, v=v, g=g, w=w)
+    names = [("q", "dq"), ("k", "dk"), ("v", "dv"), ("g", "dg"), ("w", "dw")]
+    if gated:
+        args["z"] = z
+        names.append(("z", "d_o_gate"))
+    h = 1e-5
+    for name, gname in names:
+        x = args[name]
+        fd = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            old = x[idx]
+            x[idx] = old + h
+            # norm = False: the output does not depend on m at all, so m free
+            lp = brute_loss(q, k, v, g, w, dy, None, scale, eps, m0 if norm else None, norm, z)
+            x[idx] = old - h
+            lm = brute_loss(q, k, v, g, w, dy, None, scale, eps, m0 if norm else None, norm, z)
+            x[idx] = old
+            fd[idx] = (lp - lm) / (2 * h)
+        assert grads[gname].shape == x.shape, gname
+        err = relerr(grads[gname], fd)
+        assert err < 1e-7 or np.abs(fd).max() < 1e-12, (name, err)
+
+
+@pytest.mark.parametrize("norm,gated,scalar", [
+    (True, True, False), (False, False, False), (False, True, False),
+    (True, False, True), (False, True, True),
+])
+def test_variant_gradients_match_finite_differences(norm, gated, scalar):
+    _fd_variant(norm, gated, scalar, seed=34)
+
+
+def test_scalar_gate_is_the_channel_broadcast_and_forgetting_attention():
+    """A gate [B,T,Hkv] is the element-wise gate broadcast over channels; at
+    eps = 0 that is RMSNorm of Forgetting-Transformer attention (SDPA with the
+    additive bias G_t - G_s); its dg is the channel sum."""
+    rng = np.random.default_rng(35)
+    T, H, D = 21, 2, 5
+    q, k, v, _, w, dy = make(rng, 1, T, H, H, D, D)
+    a = -np.log1p(np.exp(-(rnd(rng, 1, T, H) + 1.0)))
+    gb = np.repeat(a[..., None], D, axis=3)
+    ys = fix_ref.forward(q, k, v, a, w, None, 0.4, 0.0)["y"]
+    yb = fix_ref.forward(q, k, v, gb, w, None, 0.4, 0.0)["y"]
+    assert np.array_equal(ys, yb)
+    for h in range(H):
+        M = _fox_mask(a[0, :, h])
+        sd = _sdpa(q[0, :, h:h + 1], k[0, :, h:h + 1], v[0, :, h:h + 1], M[None], 0.4)[:, 0]
+        assert relerr(ys[0, :, h], _rms(sd, w, 0.0)) < 1e-12
+    gs = fix_ref.backward(q, k, v, a, w, dy, None, 0.4, 1e-6)
+    gbr = fix_ref.backward(q, k, v, gb, w, dy, None, 0.4, 1e-6)
+    assert gs["dg"].shape == a.shape
+    assert relerr(gs["dg"], gbr["dg"].sum(axis=-1)) < 1e-14

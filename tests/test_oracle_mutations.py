@@ -35,6 +35,16 @@ MUTATIONS = {
     # GQA: q head h mapped to kv head h % Hkv instead of h // group
     "gqa_modulo": ("kv = h // grp\n            sl = slice(s0, s0 + L)\n            jobs.append((q[b, sl, h], k[b, sl, kv], v[b, sl, kv], g[b, sl, kv], w, scale, eps))",
                    "kv = h % Hkv\n            sl = slice(s0, s0 + L)\n            jobs.append((q[b, sl, h], k[b, sl, kv], v[b, sl, kv], g[b, sl, kv], w, scale, eps))"),
+    # output gate applied as sigmoid(z) instead of z * sigmoid(z)
+    "gate_sigmoid_only": ("    return z / (1.0 + np.exp(-z))", "    return 1.0 / (1.0 + np.exp(-z))"),
+    # swish derivative without its second term
+    "gate_grad_drops_term": ("    return sg * (1.0 + z * (1.0 - sg))", "    return sg"),
+    # no-norm backward without the softmax-denominator term
+    "nonorm_drops_delta": ("        dS = P * (dP - (do * o).sum(axis=1)[:, None])",
+                           "        dS = P * dP"),
+    # no-norm output divided by the row maximum's weight instead of the sum
+    "nonorm_wrong_denominator": ("        y = o / P.sum(axis=1)[:, None]             # softmax denominator l_t",
+                                 "        y = o / P.max(axis=1)[:, None]"),
 }
 
 
@@ -55,32 +65,50 @@ def _inputs(seed=1, T=5, Hq=2, Hkv=1, D=3):
     return q, k, v, g, w, dy
 
 
+VARIANTS = [dict(norm=True, gated=False), dict(norm=True, gated=True),
+            dict(norm=False, gated=False), dict(norm=False, gated=True)]
+
+
+def _gate(seed, q):
+    return np.random.default_rng(seed + 100).standard_normal(q.shape[:3] + (3,))
+
+
 def _forward_pin_fails(mod):
     q, k, v, g, w, _ = _inputs(Hq=4, Hkv=2)
-    y = mod.forward(q, k, v, g, w, None, 0.7, 1e-2)["y"]
-    yb, _ = brute_forward(q, k, v, g, w, None, 0.7, 1e-2)
-    return not np.allclose(y, np.array(yb), rtol=1e-10, atol=1e-12)
+    for var in VARIANTS:
+        z = _gate(1, q) if var["gated"] else None
+        y = mod.forward(q, k, v, g, w, None, 0.7, 1e-2, norm=var["norm"], o_gate=z)["y"]
+        yb, _ = brute_forward(q, k, v, g, w, None, 0.7, 1e-2, None, var["norm"], z)
+        if not np.allclose(y, np.array(yb), rtol=1e-10, atol=1e-12):
+            return True
+    return False
 
 
 def _fd_pin_fails(mod):
     q, k, v, g, w, dy = _inputs()
     scale, eps = 0.8, 1e-2
-    gr = mod.backward(q, k, v, g, w, dy, None, scale, eps)
-    m0 = fix_ref.forward(q, k, v, g, w, None, scale, eps)["m"]
-    args = dict(q=q, k=k, v=v, g=g, w=w)
-    for name, gname in [("q", "dq"), ("k", "dk"), ("v", "dv"), ("g", "dg"), ("w", "dw")]:
-        x = args[name]
-        fd = np.zeros_like(x)
-        for idx in np.ndindex(x.shape):
-            old = x[idx]
-            x[idx] = old + 1e-5
-            lp = brute_loss(q, k, v, g, w, dy, None, scale, eps, m0)
-            x[idx] = old - 1e-5
-            lm = brute_loss(q, k, v, g, w, dy, None, scale, eps, m0)
-            x[idx] = old
-            fd[idx] = (lp - lm) / 2e-5
-        if not np.allclose(gr[gname], fd, rtol=1e-6, atol=1e-8):
-            return True
+    for var in VARIANTS:
+        z = _gate(2, q) if var["gated"] else None
+        gr = mod.backward(q, k, v, g, w, dy, None, scale, eps, norm=var["norm"], o_gate=z)
+        m0 = fix_ref.forward(q, k, v, g, w, None, scale, eps)["m"]
+        args = dict(q=q, k=k, v=v, g=g, w=w)
+        names = [("q", "dq"), ("k", "dk"), ("v", "dv"), ("g", "dg"), ("w", "dw")]
+        if z is not None:
+            args["z"] = z
+            names.append(("z", "d_o_gate"))
+        for name, gname in names:
+            x = args[name]
+            fd = np.zeros_like(x)
+            for idx in np.ndindex(x.shape):
+                old = x[idx]
+                x[idx] = old + 1e-5
+                lp = brute_loss(q, k, v, g, w, dy, None, scale, eps, m0, var["norm"], z)
+                x[idx] = old - 1e-5
+                lm = brute_loss(q, k, v, g, w, dy, None, scale, eps, m0, var["norm"], z)
+                x[idx] = old
+                fd[idx] = (lp - lm) / 2e-5
+            if not np.allclose(gr[gname], fd, rtol=1e-6, atol=1e-8):
+                return True
     return False
 
 
