@@ -4,8 +4,11 @@
 
 Each ``csrc/*.cu`` file is compiled to an object under ``_build/`` and the
 objects are linked into ``gated_softmax_attention_fp32_b200/libfixattn.so``.
-A file is recompiled only when it or any header under ``csrc/``/``include/``
-changed (content hash).
+A second link, ``libfixattn_test.so``, is built from the same sources with
+``-DFIX_TEST_HOOKS``: it adds the hooks the failure-detection tests use (a
+forward whose waits expire on purpose) and is never loaded by the product
+path.  A file is recompiled only when it or any header under
+``csrc/``/``include/`` changed (content hash).
 """
 from __future__ import annotations
 
@@ -23,6 +26,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libfixattn.so")
+TEST_LIB = os.path.join(PKG, "libfixattn_test.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-O3",
@@ -46,15 +50,17 @@ def _headers_digest() -> str:
     return h.hexdigest()
 
 
-def _compile(src: str, hdr: str, force: bool) -> tuple:
+def _compile(src: str, hdr: str, force: bool, variant: str = "") -> tuple:
     base = os.path.splitext(os.path.basename(src))[0]
-    obj = os.path.join(BUILD, base + ".o")
+    outdir = os.path.join(BUILD, variant) if variant else BUILD
+    obj = os.path.join(outdir, base + ".o")
     stamp = obj + ".hash"
+    extra = ["-DFIX_TEST_HOOKS"] if variant == "test" else []
     with open(src, "rb") as f:
-        digest = hashlib.sha256(f.read() + hdr.encode() + " ".join(FLAGS).encode()).hexdigest()
+        digest = hashlib.sha256(f.read() + hdr.encode() + " ".join(FLAGS + extra).encode()).hexdigest()
     if not force and os.path.exists(obj) and os.path.exists(stamp) and open(stamp).read() == digest:
         return obj, "", False
-    cmd = [nvcc(), *FLAGS, "-I", INCLUDE, "-I", CSRC, "-c", src, "-o", obj]
+    cmd = [nvcc(), *FLAGS, *extra, "-I", INCLUDE, "-I", CSRC, "-c", src, "-o", obj]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"nvcc failed on {src}:\n{r.stdout}\n{r.stderr}")
@@ -63,26 +69,31 @@ def _compile(src: str, hdr: str, force: bool) -> tuple:
     return obj, r.stderr, True
 
 
-def build(force: bool = False, jobs: int = 0, verbose: bool = False) -> str:
-    os.makedirs(BUILD, exist_ok=True)
-    srcs = sorted(os.path.join(CSRC, n) for n in os.listdir(CSRC) if n.endswith(".cu"))
-    hdr = _headers_digest()
-    jobs = jobs or min(len(srcs), os.cpu_count() or 1)
-    with cf.ThreadPoolExecutor(max_workers=jobs) as ex:
-        results = list(ex.map(lambda s: _compile(s, hdr, force), srcs))
-    objs = [r[0] for r in results]
-    if verbose:
-        for r in results:
-            if r[1]:
-                sys.stderr.write(r[1])
-    rebuilt = any(r[2] for r in results)
-    if rebuilt or force or not os.path.exists(LIB):
-        tmp = LIB + ".tmp"
+def _link(objs, out, rebuilt, force):
+    if rebuilt or force or not os.path.exists(out):
+        tmp = out + ".tmp"
         cmd = [nvcc(), *ARCH, "-shared", "-Xcompiler", "-fPIC", "-o", tmp, *objs]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-        os.replace(tmp, LIB)
+        os.replace(tmp, out)
+
+
+def build(force: bool = False, jobs: int = 0, verbose: bool = False) -> str:
+    os.makedirs(os.path.join(BUILD, "test"), exist_ok=True)
+    srcs = sorted(os.path.join(CSRC, n) for n in os.listdir(CSRC) if n.endswith(".cu"))
+    hdr = _headers_digest()
+    jobs = jobs or min(2 * len(srcs), os.cpu_count() or 1)
+    work = [(s_, "") for s_ in srcs] + [(s_, "test") for s_ in srcs]
+    with cf.ThreadPoolExecutor(max_workers=jobs) as ex:
+        results = list(ex.map(lambda a: _compile(a[0], hdr, force, a[1]), work))
+    if verbose:
+        for r in results:
+            if r[1]:
+                sys.stderr.write(r[1])
+    prod, test = results[:len(srcs)], results[len(srcs):]
+    _link([r[0] for r in prod], LIB, any(r[2] for r in prod), force)
+    _link([r[0] for r in test], TEST_LIB, any(r[2] for r in test), force)
     return LIB
 
 

@@ -1,6 +1,9 @@
 // Host side of the FiX attention C ABI (include/fix_attn.h): argument
-// validation, workspace layout, the packed-sequence chunk schedule and the
-// kernel launches.  Nothing here allocates or synchronises.
+// validation, workspace layout, the packed-sequence chunk schedule (built
+// here from the host mirror of cu_seqlens and uploaded through kernel
+// parameters) and the kernel launches.  Nothing here allocates device memory
+// or synchronises.
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -66,17 +69,6 @@ static fix_status make_dims(const fix_attn_problem* p, Dims* d) {
   return FIX_OK;
 }
 
-// Largest number of chunks of one sequence (bound for the order histogram).
-static int max_chunks_per_seq(const fix_attn_problem* p) {
-  if (!p->cu_seqlens) return (p->seqlen + FIX_CHUNK - 1) / FIX_CHUNK;
-  long long m = 0;
-  for (int i = 0; i < p->num_seqs; ++i) {
-    const long long n = (p->cu_seqlens_host[i + 1] - p->cu_seqlens_host[i] + FIX_CHUNK - 1) / FIX_CHUNK;
-    if (n > m) m = n;
-  }
-  return (int)m;
-}
-
 // Work split of the dk/dv kernel: each key chunk's tiles (q heads x 64-row
 // query tiles) are taken in two kinds, those of the chunk itself (the
 // diagonal) and those of the later chunks of its sequence, and each kind is
@@ -114,8 +106,8 @@ static SplitPlan plan_split(const fix_attn_problem* p, const Dims& d) {
   if (P < 4) P = 4;
   if (P > (1 << 30)) P = 1 << 30;
   sp.P = (int)P;
-  // the schedule kernel's split: per key chunk, its diagonal tiles and its
-  // later tiles, each in runs of at most P
+  // the split: per key chunk, its diagonal tiles and its later tiles, each
+  // in runs of at most P
   each_seq([&](long long L, long long mult) {
     const int nc = (int)((L + FIX_CHUNK - 1) / FIX_CHUNK);
     for (int j = 0; j < nc; ++j) {
@@ -131,7 +123,7 @@ static SplitPlan plan_split(const fix_attn_problem* p, const Dims& d) {
 
 // Workspace layout (all offsets 256-byte aligned).
 struct Ws {
-  size_t status, chunks, order, safe, L, vt, vm, vml, tot, rho, hr;   // forward and backward
+  size_t status, chunks, order, safe, L, vt, vm, vml, tot, rho, hr, lvt;   // forward and backward
   size_t dow, dot, domh, doml, dsafe, hmax, ptt, A, dG, dtot, dwp;   // backward only
   size_t parts, cpart, partial;                            // dk/dv work split
   size_t total;
@@ -158,6 +150,7 @@ static Ws layout(const Dims& d, bool bwd, const SplitPlan& sp) {
   w.tot = take(nch * 4);
   w.rho = take(nch * 4);
   w.hr = take(nch * 4);
+  w.lvt = take(nch * 4);
   if (bwd) {
     w.dow = take((size_t)d.N * d.Hq * d.Dv * 4);
     w.dot = take((size_t)d.N * d.Hq * d.Dv * 2);
@@ -216,7 +209,6 @@ static size_t simt_dkv_smem(const Dims& d) {
   return sizeof(float) * (size_t)(ST_ROWS * d.Dk + 2 * ST_ROWS * d.Dv + ST_ROWS);
 }
 
-// Prefix pass + schedule (both directions).
 bool set_smem_limit(const void* func, int bytes) {
   struct Entry {
     const void* func;
@@ -242,22 +234,118 @@ bool set_smem_limit(const void* func, int bytes) {
   return true;
 }
 
+// Copies `bytes` (a multiple of 4) from host memory to the device through
+// the parameter blocks of upload launches, in pieces of at most 31 KB.
+static fix_status upload(void* dst, const uint32_t* src, size_t bytes, cudaStream_t st) {
+  size_t words = bytes / 4, off = 0;
+  while (off < words) {
+    const size_t n = std::min(words - off, (size_t)kBlobMaxWords);
+    uint32_t* to = static_cast<uint32_t*>(dst) + off;
+    auto send = [&](auto blob) {
+      std::memcpy(blob.w, src + off, n * 4);
+      upload_kernel<sizeof(blob.w) / 4><<<1, 256, 0, st>>>(blob, to, (int)n);
+    };
+    if (n <= 256) send(Blob<256>{});
+    else if (n <= 1024) send(Blob<1024>{});
+    else if (n <= 4096) send(Blob<4096>{});
+    else send(Blob<kBlobMaxWords>{});
+    FIX_TRY(launched());
+    off += n;
+  }
+  return FIX_OK;
+}
+
+// Launches that upload() makes for `bytes`.
+static int upload_launches(size_t bytes) {
+  return (int)((bytes / 4 + kBlobMaxWords - 1) / kBlobMaxWords);
+}
+
+// Sequence lengths of the problem, in order (B sequences of T tokens, or the
+// packed lengths of the host mirror of cu_seqlens).
+template <class Fn>
+static void each_sequence(const fix_attn_problem* p, Fn fn) {
+  if (p->cu_seqlens) {
+    for (int i = 0; i < p->num_seqs; ++i)
+      fn(p->cu_seqlens_host[i], p->cu_seqlens_host[i + 1] - p->cu_seqlens_host[i]);
+  } else {
+    for (int b = 0; b < p->batch; ++b) fn((long long)b * p->seqlen, (long long)p->seqlen);
+  }
+}
+
+// Builds the schedule on the host and uploads it into the workspace:
+//   chunks[]  the chunk table, sequences in order, 128-token chunks from each
+//             sequence's first token;
+//   order[]   chunk ids by decreasing chunk index j (the number of key blocks
+//             before the diagonal; ties in table order), so that grids
+//             walking order[] start the longest causal rows first;
+//   with the dk/dv split plan `sp`: parts[] holds every later-block part
+//   first (sequences, then chunks, in order), then every diagonal part; a key
+//   chunk's slots are consecutive, its diagonal parts' first, and
+//   cpart[ci] = {number of parts, first slot}.
+// With `tables_kept` (the backward reusing its forward's workspace) only the
+// split is uploaded: the chunk table and order are the forward's.
+static fix_status upload_schedule(const fix_attn_problem* p, const Dims& d, const Ws& ws,
+                                  char* base, const SplitPlan* sp, bool tables_kept,
+                                  cudaStream_t st) {
+  if (d.nchunks == 0) return FIX_OK;
+  thread_local std::vector<uint32_t> bufA, bufB;
+  const size_t spanA = ws.order - ws.chunks + (size_t)d.nchunks * sizeof(int);
+  bufA.assign(spanA / 4, 0u);
+  Chunk* chunks = reinterpret_cast<Chunk*>(bufA.data());
+  int* order = reinterpret_cast<int*>(reinterpret_cast<char*>(bufA.data()) + (ws.order - ws.chunks));
+  int ci = 0, maxj = 0;
+  each_sequence(p, [&](long long s0, long long L) {
+    const int nc = (int)((L + FIX_CHUNK - 1) / FIX_CHUNK);
+    for (int j = 0; j < nc; ++j, ++ci) {
+      chunks[ci] = Chunk{(int)(s0 + (long long)j * FIX_CHUNK),
+                         (int)std::min<long long>(FIX_CHUNK, L - (long long)j * FIX_CHUNK), j, nc};
+      maxj = std::max(maxj, j);
+    }
+  });
+  if (ci != d.nchunks) return FIX_ERR_CU_SEQLENS;
+  {
+    std::vector<int> count(maxj + 2, 0);
+    for (int i = 0; i < ci; ++i) ++count[maxj - chunks[i].j + 1];
+    for (int k = 1; k <= maxj + 1; ++k) count[k] += count[k - 1];
+    for (int i = 0; i < ci; ++i) order[count[maxj - chunks[i].j]++] = i;
+  }
+  if (!tables_kept) FIX_TRY(upload(base + ws.chunks, bufA.data(), spanA, st));
+  if (!sp) return FIX_OK;
+  const size_t spanB = ws.cpart - ws.parts + (size_t)d.nchunks * sizeof(int2);
+  bufB.assign(spanB / 4, 0u);
+  Part* parts = reinterpret_cast<Part*>(bufB.data());
+  int2* cpart = reinterpret_cast<int2*>(reinterpret_cast<char*>(bufB.data()) + (ws.cpart - ws.parts));
+  const long long P = sp->P;
+  auto n_diag = [&](long long L, int j) { return ((long long)d.grp * fix_halves((int)L, j) + P - 1) / P; };
+  auto n_off = [&](long long L, int j) {
+    return ((long long)d.grp * (tiles64_host(L, j) - fix_halves((int)L, j)) + P - 1) / P;
+  };
+  long long total_off = 0;
+  each_sequence(p, [&](long long, long long L) {
+    const int nc = (int)((L + FIX_CHUNK - 1) / FIX_CHUNK);
+    for (int j = 0; j < nc; ++j) total_off += n_off(L, j);
+  });
+  long long o = 0, e = total_off, slot = 0;
+  int c = 0;
+  each_sequence(p, [&](long long, long long L) {
+    const int nc = (int)((L + FIX_CHUNK - 1) / FIX_CHUNK);
+    for (int j = 0; j < nc; ++j, ++c) {
+      const long long nd = n_diag(L, j), no = n_off(L, j);
+      cpart[c] = make_int2((int)(nd + no), (int)slot);
+      for (long long q = 0; q < nd; ++q) parts[e++] = Part{c, (int)q, (int)(slot + q), 1};
+      for (long long q = 0; q < no; ++q) parts[o++] = Part{c, (int)q, (int)(slot + nd + q), 0};
+      slot += nd + no;
+    }
+  });
+  if (e != sp->nparts || slot != sp->nslots) return FIX_ERR_CU_SEQLENS;
+  return upload(base + ws.parts, bufB.data(), spanB, st);
+}
+
 static fix_status run_prefix(const Dims& d, const fix_attn_problem* p, const Ws& ws, char* base,
                              const float* g, const void* v, bool want_vt, const SplitPlan* sp,
                              int* hmax, bool reuse, cudaStream_t st) {
-  Chunk* chunks = reinterpret_cast<Chunk*>(base + ws.chunks);
-  PartSpec ps{};
-  if (sp) {
-    ps.grp = d.grp;
-    ps.tiles_per_part = sp->P;
-    ps.cap_parts = (int)sp->nparts;
-    ps.parts = reinterpret_cast<Part*>(base + ws.parts);
-    ps.cpart = reinterpret_cast<int2*>(base + ws.cpart);
-  }
-  schedule_kernel<<<1, kScheduleThreads, 0, st>>>(p->cu_seqlens, d.nseq, d.T, d.N, d.nchunks, chunks,
-                                      max_chunks_per_seq(p),
-                                      want_vt ? reinterpret_cast<int*>(base + ws.order) : nullptr, ps);
-  FIX_TRY(launched());
+  const Chunk* chunks = reinterpret_cast<const Chunk*>(base + ws.chunks);
+  FIX_TRY(upload_schedule(p, d, ws, base, sp, reuse, st));
   if (d.nchunks == 0) return FIX_OK;
   if (reuse) {
     // the forward's prefix results stay; only the per-(chunk, q head) max
@@ -272,7 +360,8 @@ static fix_status run_prefix(const Dims& d, const fix_attn_problem* p, const Ws&
       reinterpret_cast<__nv_bfloat16*>(base + ws.vm),
       reinterpret_cast<__nv_bfloat16*>(base + ws.vml), reinterpret_cast<float*>(base + ws.tot),
       reinterpret_cast<float*>(base + ws.rho), reinterpret_cast<float*>(base + ws.hr),
-      reinterpret_cast<int*>(base + ws.safe), reinterpret_cast<int*>(base + ws.status) + 1, hmax);
+      reinterpret_cast<float*>(base + ws.lvt), reinterpret_cast<int*>(base + ws.safe),
+      reinterpret_cast<int*>(base + ws.status) + 1, hmax);
   return launched();
 }
 
@@ -340,6 +429,7 @@ fix_status fix_attn_fwd(const fix_attn_problem* p, const void* q, const void* k,
                    reinterpret_cast<const __nv_bfloat16*>(base + ws.vml), v, L, tot,
                    reinterpret_cast<const float*>(base + ws.rho),
                    reinterpret_cast<const float*>(base + ws.hr),
+                   reinterpret_cast<const float*>(base + ws.lvt),
                    reinterpret_cast<const int*>(base + ws.safe), w, y, p->y_dtype == FIX_DTYPE_F32,
                    o_s, m_s, rstd_s, reinterpret_cast<int*>(base + ws.status), st));
   } else {
@@ -437,6 +527,7 @@ fix_status fix_attn_bwd(const fix_attn_problem* p, const void* q, const void* k,
     ta.tot = tot;
     ta.rho = reinterpret_cast<const float*>(base + ws.rho);
     ta.hr = reinterpret_cast<const float*>(base + ws.hr);
+    ta.lvt = reinterpret_cast<const float*>(base + ws.lvt);
     ta.safe = reinterpret_cast<const int*>(base + ws.safe);
     ta.dsafe = dsafe;
     ta.m_s = m_s;
@@ -505,18 +596,24 @@ int fix_attn_kernel_count(const fix_attn_problem* p, int backward) {
   Dims d;
   if (make_dims(p, &d) != FIX_OK) return 0;
   if (d.N == 0) return 0;
+  const SplitPlan sp = backward ? plan_split(p, d) : SplitPlan{};
+  const Ws ws = layout(d, backward != 0, sp);
+  const int upA = d.nchunks ? upload_launches(ws.order - ws.chunks + (size_t)d.nchunks * 4) : 0;
   if (!backward) {
     const bool tc = p->algo != FIX_ALGO_SIMT && tc_fwd_supported(d);
-    return 2 + (tc ? tc_fwd_kernel_count(d) : 1);
+    // schedule upload, prefix pass, attention
+    return upA + 1 + (tc ? tc_fwd_kernel_count(d) : 1);
   }
   const bool tc = p->algo != FIX_ALGO_SIMT && tc_bwd_supported(d);
   const bool fwd_tc = p->algo != FIX_ALGO_SIMT && tc_fwd_supported(d);
   const bool reuse = (p->flags & FIX_FLAG_REUSE_FWD_WORKSPACE) && (!tc || fwd_tc);
-  // schedule + prefix pass (the schedule alone when the forward's prefix is
-  // reused), preprocess (2, or 3 with the tensor-core operands), tensor-core
-  // dq / dk/dv / combine, the exact kernels (2), the dG reverse cumsum (2)
-  return (reuse ? 1 : 2) + (tc ? 3 : 2) + (tc ? tc_bwd_kernel_count(d, plan_split(p, d).nslots) : 0) +
-         2 + 2;
+  const int upB = (tc && d.nchunks) ? upload_launches(ws.cpart - ws.parts + (size_t)d.nchunks * 8) : 0;
+  // schedule uploads (the split only when the forward's tables are reused),
+  // the prefix pass unless reused, the preprocess (2, or 3 with the
+  // tensor-core operands), tensor-core dq / dk/dv / combine, the exact
+  // kernels (2), the dG reverse cumsum (2)
+  return (reuse ? 0 : upA + 1) + upB + (tc ? 3 : 2) +
+         (tc ? tc_bwd_kernel_count(d, sp.nslots) : 0) + 2 + 2;
 }
 
 fix_status fix_attn_device_status(const void* workspace, void* stream) {

@@ -17,26 +17,41 @@
 #define FIX_CHUNK 128
 // CTAs per chunk in the backward preprocess (FIX_CHUNK / kPreSplit rows each).
 constexpr int kPreSplit = 4;
-// Threads of the single schedule CTA (a multiple of 32).
-constexpr int kScheduleThreads = 128;
+// Largest schedule piece one upload launch carries in its parameter block
+// (31 KB of the 32 KB that kernel parameters may take).
+constexpr int kBlobMaxWords = 7936;
 
 // exp for the 16-bit tensor-core operands (pre-decayed values and gradients,
 // rounded to fp16 / bf16 right after): exp2f of x log2(e), whose error is far
 // below their rounding.  The exact CUDA-core kernels keep expf.
 __device__ __forceinline__ float exp_op(float x) { return exp2f(x * 1.4426950408889634f); }
 // Largest half-range of a chunk's prefix sums that the in-chunk split
-// exp(L_t - rho) * exp(rho - L_s) keeps inside float range (e^80 ~ 5.5e34).
+// exp(L_t - rho) * exp(rho - L_s) keeps inside float range (e^80 ~ 5.5e34),
+// and the largest |rho| for which the forward's column factor exp(rho) stays
+// a normal float.  A channel outside either bound is "out of range": its
+// rho is 0, its hr is stored as FIX_HR_BAD, its Vm is 0, and its diagonal
+// block is summed exactly in fp32.
 #define FIX_HR_MAX 80.0f
+#define FIX_RHO_MAX 80.0f
+#define FIX_HR_BAD 1e30f
+// Pre-decayed values Vt (key blocks before the query chunk) are stored as
+// fp16 scaled by 2^-e per (chunk, kv head, channel), e = vt_exponent(lvt)
+// from lvt = log2 of the column's largest |Vt|, so that every stored value
+// is at most 2^15 in magnitude (e = 0 whenever that already holds).
+__host__ __device__ __forceinline__ float vt_exponent(float lvt) {
+  return lvt > 15.0f ? ceilf(lvt - 15.0f) : 0.0f;
+}
 // Largest |v| for which the fp16 operand path is used (fp16 max is 65504;
 // every scaled value on that path is <= |v| when g <= 0).
 #define FIX_F16_VMAX 30000.0f
 
 namespace fix {
 
-// One chunk of the schedule: first token (index into the packed token
-// stream), number of valid rows, chunk index within its sequence and the
-// sequence's chunk count.  Chunks of a sequence are consecutive in the table,
-// so the sequence's first chunk has id (this id - j).
+// One chunk of the schedule (built on the host from the sequence lengths):
+// first token (index into the packed token stream), number of valid rows,
+// chunk index within its sequence and the sequence's chunk count.  Chunks of
+// a sequence are consecutive in the table, so the sequence's first chunk has
+// id (this id - j).
 struct Chunk {
   int tok0;
   int len;
@@ -61,14 +76,10 @@ __device__ __host__ inline int fix_halves(int L, int j) {
   return (len + 63) / 64;
 }
 
-// Where the schedule kernel writes the dk/dv work split (parts == NULL: none).
-struct PartSpec {
-  int grp;            // q heads per kv head
-  int tiles_per_part; // P
-  int cap_parts;      // entries of parts[]
-  Part* parts;
-  int2* cpart;        // per chunk: {number of parts, first slot}; slots are
-                      // consecutive, the diagonal parts' first
+// A schedule table carried in a kernel's parameter block.
+template <int NW>
+struct Blob {
+  uint32_t w[NW];
 };
 
 struct Dims {

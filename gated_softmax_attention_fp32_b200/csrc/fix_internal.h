@@ -8,12 +8,12 @@ namespace fix {
 constexpr int ST_ROWS = 32;  // rows per CTA of the exact (SIMT) kernels
 
 // fix_prefix.cu
-__global__ void schedule_kernel(const int64_t* cu, int nseq, int T, int N, int cap, Chunk* out,
-                                int maxj, int* order, PartSpec ps);
+template <int NW>
+__global__ void upload_kernel(const __grid_constant__ Blob<NW> b, uint32_t* dst, int nwords);
 __global__ void prefix_kernel(Dims d, const Chunk* chunks, const float* g, const __nv_bfloat16* v,
                               float* L, uint16_t* vt, __nv_bfloat16* vm, __nv_bfloat16* vml,
-                              float* tot, float* rho, float* hr, int* safe, int* badflag,
-                              int* hmax);
+                              float* tot, float* rho, float* hr, float* lvt, int* safe,
+                              int* badflag, int* hmax);
 __global__ void chunk_total_kernel(Dims d, const Chunk* chunks, const float* x, float* tot);
 __global__ void reverse_cumsum_kernel(Dims d, const Chunk* chunks, const float* x,
                                       const float* tot, float* out);
@@ -54,10 +54,15 @@ fix_status tc_fwd(const Dims& d, const Chunk* chunks, const int* order, const vo
                   const void* k, const uint16_t* vt, const __nv_bfloat16* vm,
                   const __nv_bfloat16* vml, const void* v,
                   const float* L, const float* tot, const float* rho, const float* hr,
-                  const int* safe,
+                  const float* lvt, const int* safe,
                   const void* w, void* y, bool y_f32, float* o_s, float* m_s, float* rstd_s,
                   int* status, cudaStream_t st);
 int tc_fwd_kernel_count(const Dims& d);
+#ifdef FIX_TEST_HOOKS
+// Test builds (libfixattn_test.so) only: whether the tensor-core forward runs
+// stalled (no loads issued, every wait gives up after 1 ms).
+int test_stall_forward();
+#endif
 bool tc_bwd_supported(const Dims& d);
 int tc_bwd_kernel_count(const Dims& d, long long nslots);
 
@@ -74,6 +79,7 @@ struct TcBwdArgs {
   const float* tot;
   const float* rho;
   const float* hr;
+  const float* lvt;      // log2 of the largest |Vt| per (chunk, kv head, channel)
   const int* safe;
   const int* dsafe;
   const float* m_s;

@@ -74,6 +74,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 struct Ctl {
   int* status;           // device status word (global)
   volatile int* abort;   // CTA-wide abort flag (shared)
+  uint64_t limit_ns = kWaitTimeoutNs;   // how long one wait may take
 };
 
 // Waits for the phase with `parity` to complete; gives up after 1 s (sets the
@@ -87,7 +88,7 @@ static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parit
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait(bar, parity)) return true;
     if (ctl.abort && *ctl.abort) return false;
-    if (global_timer() - t0 > kWaitTimeoutNs) {
+    if (global_timer() - t0 > ctl.limit_ns) {
       atomicExch(ctl.status, FIX_DEV_TIMEOUT);
       if (ctl.abort) *ctl.abort = 1;
       return false;

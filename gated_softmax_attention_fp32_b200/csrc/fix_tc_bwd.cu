@@ -59,6 +59,7 @@ struct Params {
   const float* tot;
   const float* rho;
   const float* hr;
+  const float* lvt;
   const int* safe;
   const int* dsafe;
   const float* m_s;
@@ -383,16 +384,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int e = 0; e < 8; ++e) delta[e] += tp[e];
       }
+      // Vt is stored as fp16 times 2^-e per channel (prefix pass)
+      const float* lv = P.lvt + ((size_t)(first + j) * d.Hkv + kv) * DV + lc * 8;
       float f8[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) f8[e] = ex2(delta[e] * LOG2E);
+      for (int e = 0; e < 8; ++e) f8[e] = ex2(delta[e] * LOG2E + vt_exponent(lv[e]));
       if (!mbar_wait(&bar->v_full[st], (it >> 1) & 1, ctl)) break;
-      const bool in_f16 = P.safe[(size_t)(first + j) * d.Hkv + kv] != 0;
       uint8_t* vb = reinterpret_cast<uint8_t*>(sV + st * BN * DV);
       for (int rr = r0; rr < BN; rr += kRowsPerPass) {
         uint4* p = reinterpret_cast<uint4*>(vb + sw_off(BN, rr, lc * 8));
         float x[8];
-        unpack8(*p, in_f16, x);
+        unpack8(*p, true, x);
 #pragma unroll
         for (int e = 0; e < 8; ++e) x[e] *= f8[e];
         *p = pack8(x, cta_f16);
@@ -782,18 +784,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       // aborted: fall through to the teardown
     } else {
       if (!dmode) {
-        // Vt arrives in its chunk's storage type; the later-block MMAs read it
-        // in the CTA's type, so convert it once if they differ
-        const bool vt_f16 = P.safe[(size_t)cj * d.Hkv + kv] != 0;
-        if (vt_f16 != (cta_f16 != 0)) {
+        // Vt arrives as fp16 times 2^-e per channel; the later-block MMAs read
+        // it unscaled in the CTA's operand type, so this thread rewrites its
+        // channels once if either differs
+        const float* lv = P.lvt + ((size_t)cj * d.Hkv + kv) * DV + lc * 8;
+        float sc[8];
+        bool unit = true;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float ve = vt_exponent(lv[e]);
+          sc[e] = exp2f(ve);
+          unit = unit && ve == 0.f;
+        }
+        if (!unit || !cta_f16) {
           for (int rr = r0; rr < BN; rr += kRowsPerPass) {
             uint4* p = reinterpret_cast<uint4*>(sV + sw_off(BN, rr, lc * 8));
             float x[8];
-            unpack8(*p, vt_f16, x);
+            unpack8(*p, true, x);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) x[e] *= sc[e];
             *p = pack8(x, cta_f16 != 0);
           }
-          fence_proxy_async_smem();
         }
+        fence_proxy_async_smem();
       }
       // Per tile: the row maxima into sM and, for later blocks, X = dOt f_ij
       // with f_ij = exp(sum_{j<j'<i} tot_j').  The global values a tile needs
@@ -1078,6 +1091,7 @@ fix_status tc_bwd(const fix_attn_problem*, const Dims& d, const TcBwdArgs& a, in
   prm.tot = a.tot;
   prm.rho = a.rho;
   prm.hr = a.hr;
+  prm.lvt = a.lvt;
   prm.safe = a.safe;
   prm.dsafe = a.dsafe;
   prm.m_s = a.m_s;

@@ -5,41 +5,56 @@
 // RMSNorm follows.  The README's "Code Structure" splits the reference into
 // intra-chunk preprocessing, inter-chunk scaling of V and a parallel forward;
 // here the preprocessing is the prefix pass (fix_prefix.cu) and the rest is
-// this one kernel.
+// this one persistent kernel.
 //
-// One CTA computes one query chunk (128 rows) of one q head against the key
-// blocks j = i, i-1, ..., 0 of its sequence (diagonal block first).  Every
-// decay factor is split at a per-channel reference so that the row part is
-// applied once in the epilogue and the key part scales the value tiles:
-//   * diagonal block (j = i), reference rho (the middle of the chunk's range
-//     of prefix sums):  exp(G_t - G_s) = exp(L_t - rho) * exp(rho - L_s),
-//     both factors in [e^-80, e^80]; Vm_s = v_s exp(rho - L_s) comes from the
-//     prefix pass.  Accumulator O_d.
-//   * earlier blocks (j < i), reference = the chunk start:
-//     exp(G_t - G_s) = exp(L_t) * Vt_s f_ij / v_s, with Vt_s = v_s exp(tot_j -
-//     L_s) (prefix pass) and f_ij[c] = exp(sum_{j<j'<i} tot_j'[c]); for g <= 0
-//     every factor is <= 1.  Accumulator O_o.
-// Epilogue: o_t = exp(L_t - rho) O_d + exp(L_t) O_o + P_tt v_t (the s = t term,
-// in fp32), then the RMSNorm.
-// The diagonal block carries most of the attention weight whenever the gate
-// decays within a chunk, so its bf16 rounding would dominate the error: there
-// both P and Vm are split into bf16 hi + lo parts and the block costs three
-// MMAs (P_hi Vm_hi + P_lo Vm_hi + P_hi Vm_lo, near-exact).  The other blocks
-// use one MMA in fp16 (11-bit significand) when every gate of the sequence up
-// to this chunk is <= 0 and |v| <= 3e4, since then P <= e^8 and |V'| <= |v|
-// fit fp16; otherwise (rising gates, huge values) in bf16.  Channels whose
-// chunk range exceeds the split's float range (Vm = 0, rho = 0 there) get
-// their diagonal block exactly in fp32 in the epilogue.
+// Work unit ("tile"): one query chunk i (128 rows) of one q head against the
+// key blocks of its sequence: first the earlier blocks j = i-1, ..., 0, then
+// the diagonal block j = i.  Tiles are sorted longest first (the host-side
+// order of chunks) and dealt to the persistent CTAs in snake order, so that
+// every CTA gets a mix of long and short tiles.
 //
-// Warp roles (384 threads): warp 0 issues TMA loads (Q once; K and V tiles
-// through a 2-stage ring), warp 1 issues the MMAs (one thread) and owns TMEM,
-// warps 4-7 turn S into P (one TMEM lane = one query row per thread) and move
-// the accumulators to a shared fp32 tile (epilogue phase A), warps 8-11 scale
-// the V tiles in shared memory by f_ij.  Once every MMA has completed (the
-// MMA warp's single-use `drain` barrier), all twelve warps run epilogue phase
-// B: row factor, the s = t term, RMSNorm and coalesced stores, a row per warp
-// at a time.  TMEM: two S buffers (P is written over the S it came from, as
-// 16-bit pairs) and the two O accumulators.
+// Decay split, per channel c (L = chunk-local prefix sums of g, rho = the
+// middle of the chunk's range of L, tot = chunk totals):
+//   * earlier blocks: exp(G_t - G_s) = exp(L_t) * f_ij * exp(tot_j - L_s),
+//     f_ij = exp(sum_{j<j'<i} tot_j').  The prefix pass stores Vt_s = v_s
+//     exp(tot_j - L_s) (fp16, times 2^-e per channel); the V-scaling warps
+//     form V'' = Vt f_ij 2^-k_c in shared memory, with one power of two k_c per
+//     (tile, channel) chosen so that every V'' fits fp16 (k_c = 0 whenever
+//     every gate is <= 0).  P V'' accumulates in fp16 MMAs into A.
+//   * fold: once those MMAs are done, A is scaled per column by
+//     F_c = exp(rho_c) 2^k_c, which moves the accumulator to the diagonal
+//     block's reference: A = sum_{j<i} exp(rho - L_t) ... (see below).
+//   * diagonal block: exp(G_t - G_s) = exp(L_t - rho) exp(rho - L_s), both
+//     factors in [e^-80, e^80]; Vm_s = v_s exp(rho - L_s) comes from the
+//     prefix pass as bf16 hi + lo, and P as bf16 hi + lo, so the block costs
+//     three MMAs (P_hi Vm_hi + P_lo Vm_hi + P_hi Vm_lo) and is near-exact.
+//     The s = t pair is left out of the MMAs.
+//   * epilogue: o_t = alpha_t exp(L_t - rho) A_t + P_tt v_t (alpha_t =
+//     exp(m_used - m_t) undoes the lazily updated row shift; the s = t term
+//     is exact in fp32), then the RMSNorm.
+// Channels outside the split's range (prefix pass: rho = 0, Vm = 0) get no
+// fold beyond 2^k_c, and the softmax warps add their exact diagonal sum
+// exp(L_t) A_t + sum_{s<t} P_ts exp(L_t - L_s) v_s (fp32) in place; the
+// epilogue then applies no row factor to them.
+//
+// Warp roles (512 threads):
+//   warp 0       TMA producer: Q per tile, K and V (Vt / Vm hi) through
+//                2-stage rings, Vm lo of the diagonal block
+//   warp 1       MMA issuer (one thread) and TMEM owner
+//   warps 4-7    softmax: S -> P in TMEM, lazy row-max rescale, the fold,
+//                the exact sums of out-of-range channels
+//   warps 8-11   V scaling: V'' in shared memory, the tile's fold factors
+//   warps 12-15  epilogue of the previous tile, overlapping this one's MMAs:
+//                TMEM -> registers -> a per-warp transpose in shared memory,
+//                lanes over channels for coalesced loads of L, v and stores
+//                of y, o, m, rstd
+// TMEM (512 columns): S/P double buffer at 0 and 128 (P written over S as
+// 16-bit pairs; the diagonal's P_lo in the buffer's upper half), and the
+// accumulator A double-buffered by tile parity at 256 and 256 + DV.
+//
+// Every mbarrier wait is bounded (1 s); a wait that expires sets the status
+// word to FIX_DEV_TIMEOUT and the CTA's abort flag, the roles stop, copies in
+// flight are drained and TMEM is released.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -51,26 +66,24 @@ namespace tcf {
 
 using namespace sm100;
 
-constexpr int BM = 128;          // query rows per CTA
+constexpr int BM = 128;          // query rows per tile
 constexpr int BN = FIX_CHUNK;    // keys per block
-constexpr int kThreads = 384;
+constexpr int kThreads = 512;
 constexpr uint32_t kTmemCols = 512;
-__host__ __device__ constexpr uint32_t col_s(int st) { return st ? 128u : 0u; }
-constexpr uint32_t kColOd = 256;           // diagonal-block accumulator [256, 256 + DV)
-// off-diagonal accumulator O_o at [256 + DV, 256 + 2 DV).  P_lo of the
-// diagonal block (64 columns at 384) may share O_o's columns: it is consumed
-// by the diagonal PV MMAs, which complete before the first off-diagonal PV
-// MMA overwrites O_o (MMAs run in issue order).
-constexpr uint32_t kColPlo = 384;
-constexpr float kRescaleThreshold = 8.0f;  // lazy row-max update (natural log units)
+constexpr float kRescaleThreshold = 8.0f;  // lazy row-max update, natural-log units
+__host__ __device__ constexpr uint32_t col_s(int b) { return b ? 128u : 0u; }
 
 struct Bars {
-  uint64_t q_full;
+  uint64_t q_full, q_empty;
   uint64_t k_full[2], k_empty[2];
   uint64_t v_full[2], v_empty[2], v_ready[2];
+  uint64_t vlo_empty;
   uint64_t s_full[2], p_full[2];
   uint64_t pv_done;
-  uint64_t drain;        // final commit: every MMA issued has completed
+  uint64_t acc_full[2], acc_empty[2];
+  uint64_t fold_ready[2];
+  uint64_t rows_ready[2], rows_free[2];
+  uint64_t drain;
 };
 
 template <int DK, int DV>
@@ -78,27 +91,28 @@ struct Layout {
   static constexpr int kQ = 0;
   static constexpr int kK = kQ + BM * DK * 2;
   static constexpr int kV = kK + 2 * BN * DK * 2;
-  static constexpr int kVl = kV + 2 * BN * DV * 2;       // Vm_lo of the diagonal block
-  static constexpr int kRho = kVl + BN * DV * 2;
-  static constexpr int kHr = kRho + DV * 4;
-  static constexpr int kW = kHr + DV * 4;
-  static constexpr int kRow = kW + DV * 4;              // per-row alpha, P_tt, m (3 x 128 f32)
-  static constexpr int kBars = kRow + 3 * BM * 4;
+  static constexpr int kVl = kV + 2 * BN * DV * 2;       // Vm lo of the diagonal block
+  static constexpr int kF = kVl + BN * DV * 2;           // [2][DV] f32 fold factors
+  static constexpr int kBad = kF + 2 * DV * 4;           // [2][DV] int out-of-range flags
+  static constexpr int kAnyBad = kBad + 2 * DV * 4;      // [2] int
+  static constexpr int kRows = kAnyBad + 16;             // [2][3][BM] f32: alpha, P_tt, m
+  static constexpr int kEpiT = kRows + 2 * 3 * BM * 4;   // [4][32][33] f32 transposes
+  static constexpr int kEpiW = kEpiT + 4 * 32 * 33 * 4;  // [DV] f32 w
+  static constexpr int kEpiRho = kEpiW + DV * 4;         // [DV] f32 rho of the epilogue's tile
+  static constexpr int kEpiBad = kEpiRho + DV * 4;       // [DV] int
+  static constexpr int kBars = (kEpiBad + DV * 4 + 7) / 8 * 8;
   static constexpr int kTmem = kBars + (int)sizeof(Bars);
   static constexpr int kAbort = kTmem + 4;
   static constexpr int kBytes = kAbort + 4;
   static constexpr int kAlloc = kBytes + 1024;   // slack for 1024-byte alignment
-  // after the last MMA: the exact path's P rows, then the accumulators of
-  // every row (fp32, 2 DV per row), reuse the K/V ring and Vm_lo
-  static constexpr int kScratch = kK;
-  static_assert(2 * BN * DK * 2 + 2 * BN * DV * 2 >= BM * BN * 4, "scratch does not fit");
-  static_assert(kRho - kK >= BM * 2 * DV * 4, "accumulator tile does not fit");
+  static_assert(kAlloc <= 232448, "shared memory");
 };
 
 struct Params {
   Dims d;
   const Chunk* chunks;
   const int* order;
+  int ntiles;
   const __nv_bfloat16* q;
   const __nv_bfloat16* k;
   const __nv_bfloat16* v;
@@ -106,6 +120,7 @@ struct Params {
   const float* tot;
   const float* rho;
   const float* hr;
+  const float* lvt;
   const int* safe;
   const __nv_bfloat16* w;
   void* y;
@@ -114,21 +129,64 @@ struct Params {
   float* m_s;
   float* rstd_s;
   int* status;
+  int stall;       // test builds only: issue no loads, waits give up after 1 ms
 };
 
-// Exact diagonal-block sum of one channel whose chunk range is too wide for
-// the split: sum_{s<t} P_ts exp(L_t - L_s) v_s in fp32 (P rows in scratch).
-__device__ __noinline__ float exact_diag_channel(const float* __restrict__ prow, int nkeys,
-                                                 float lt, const float* __restrict__ Lcol,
-                                                 const __nv_bfloat16* __restrict__ vcol,
-                                                 size_t rs) {
-  float acc = 0.f;
-  for (int s = 0; s < nkeys; ++s) {
-    const float p = prow[s];
-    if (p == 0.f) continue;
-    acc += p * ex2((lt - Lcol[(size_t)s * rs]) * LOG2E) * bf2f(vcol[(size_t)s * rs]);
-  }
-  return acc;
+// The tile a CTA takes in a given round: snake order over the longest-first
+// tile list, so that the long tiles of round 0 pair with the short ones of
+// round 1.
+__device__ __forceinline__ int tile_of(int round, int G, int c) {
+  return round * G + ((round & 1) ? (G - 1 - c) : c);
+}
+
+struct Tile {
+  int ci, h, kv;
+  int j, nblk, first, seq0, tok0, len;
+};
+
+__device__ __forceinline__ Tile tile_info(const Params& P, int t) {
+  Tile x;
+  const int ci = P.order[t / P.d.Hq];
+  x.ci = ci;
+  x.h = t % P.d.Hq;
+  x.kv = x.h / P.d.grp;
+  const Chunk ch = P.chunks[ci];
+  x.j = ch.j;
+  x.nblk = ch.j + 1;
+  x.first = ci - ch.j;
+  x.seq0 = ch.tok0 - ch.j * FIX_CHUNK;
+  x.tok0 = ch.tok0;
+  x.len = ch.len;
+  return x;
+}
+
+// Named barriers for one warpgroup (ids 1..3; 0 is __syncthreads).
+__device__ __forceinline__ void wg_sync(int id) {
+  asm volatile("bar.sync %0, 128;" ::"r"(id) : "memory");
+}
+__device__ __forceinline__ int wg_and(int id, int pred) {
+  int out;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.b32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, 128, p;\n\t"
+      "selp.s32 %0, 1, 0, q;\n\t}"
+      : "=r"(out)
+      : "r"(pred), "r"(id)
+      : "memory");
+  return out;
+}
+__device__ __forceinline__ int wg_or(int id, int pred) {
+  int out;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.b32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, 128, p;\n\t"
+      "selp.s32 %0, 1, 0, q;\n\t}"
+      : "=r"(out)
+      : "r"(pred), "r"(id)
+      : "memory");
+  return out;
 }
 
 template <int DK, int DV>
@@ -142,40 +200,28 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              ~static_cast<uintptr_t>(1023));
   const Dims& d = P.d;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int ci = P.order[blockIdx.x / d.Hq];
-  const int h = blockIdx.x % d.Hq, kv = h / d.grp;
-  const Chunk ch = P.chunks[ci];
-  if (ch.len <= 0) return;
-  const int nblk = ch.j + 1;
-  const int first = ci - ch.j;
-  const int seq0 = ch.tok0 - ch.j * FIX_CHUNK;
+  const int G = gridDim.x, cta = blockIdx.x;
+  const int rounds = (P.ntiles + G - 1) / G;
   const size_t vrs = (size_t)d.Hkv * DV;
 
   __nv_bfloat16* sQ = reinterpret_cast<__nv_bfloat16*>(smem + Lay::kQ);
   __nv_bfloat16* sK = reinterpret_cast<__nv_bfloat16*>(smem + Lay::kK);
   __nv_bfloat16* sV = reinterpret_cast<__nv_bfloat16*>(smem + Lay::kV);
   __nv_bfloat16* sVl = reinterpret_cast<__nv_bfloat16*>(smem + Lay::kVl);
-  float* sRho = reinterpret_cast<float*>(smem + Lay::kRho);
-  float* sHr = reinterpret_cast<float*>(smem + Lay::kHr);
-  float* sW = reinterpret_cast<float*>(smem + Lay::kW);
+  float* sF = reinterpret_cast<float*>(smem + Lay::kF);
+  int* sBad = reinterpret_cast<int*>(smem + Lay::kBad);
+  int* sAnyBad = reinterpret_cast<int*>(smem + Lay::kAnyBad);
+  float* sRows = reinterpret_cast<float*>(smem + Lay::kRows);
   Bars* bar = reinterpret_cast<Bars*>(smem + Lay::kBars);
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(smem + Lay::kTmem);
   volatile int* sAbort = reinterpret_cast<volatile int*>(smem + Lay::kAbort);
-  const Ctl ctl{P.status, sAbort};
+  const Ctl ctl{P.status, sAbort, P.stall ? 1000000ull : kWaitTimeoutNs};
 
   // ---------------------------------------------------------------- setup
-  bool my_bad = false;
-  if (tid < DV) {
-    const size_t ti = ((size_t)ci * d.Hkv + kv) * DV + tid;
-    const float hrv = P.hr[ti];
-    my_bad = hrv > FIX_HR_MAX;
-    sHr[tid] = hrv;
-    sRho[tid] = P.rho[ti];
-    sW[tid] = bf2f(P.w[tid]);
-  }
   if (tid == 0) {
     *sAbort = 0;
     mbar_init(&bar->q_full, 1);
+    mbar_init(&bar->q_empty, 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bar->k_full[s], 1);
       mbar_init(&bar->k_empty[s], 1);
@@ -184,428 +230,581 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bar->v_ready[s], 128);
       mbar_init(&bar->s_full[s], 1);
       mbar_init(&bar->p_full[s], 128);
+      mbar_init(&bar->acc_full[s], 1);
+      mbar_init(&bar->acc_empty[s], 128);
+      mbar_init(&bar->fold_ready[s], 128);
+      mbar_init(&bar->rows_ready[s], 128);
+      mbar_init(&bar->rows_free[s], 128);
     }
+    mbar_init(&bar->vlo_empty, 1);
     mbar_init(&bar->pv_done, 1);
     mbar_init(&bar->drain, 1);
     mbar_fence_init();
   }
   if (warp == 1) tmem_alloc(sTmem, kTmemCols);
-  bool my_safe = true;
-  for (int jj = tid; jj < nblk; jj += blockDim.x) my_safe = my_safe && P.safe[(size_t)(first + jj) * d.Hkv + kv];
-  const int cta_f16 = __syncthreads_and(my_safe);
+  if (tid >= 384 && tid - 384 < DV)
+    reinterpret_cast<float*>(smem + Lay::kEpiW)[tid - 384] = bf2f(P.w[tid - 384]);
   tc_fence_before();
-  const int any_bad = __syncthreads_or(my_bad);
+  __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *sTmem;
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      mbar_expect_tx(&bar->q_full, BM * DK * 2);
-      for (int hh = 0; hh < DK / 64; ++hh)
-        tma_load_3d(sQ + hh * BM * 64, &tm_q, &bar->q_full, hh * 64, h, ch.tok0);
-      int nk = 0, nv = 0;  // K / V tiles issued
-      for (int it = 0; it < nblk; ++it) {
-        const int st = it & 1;
-        const uint32_t ph = (it >> 1) & 1;
-        const int ktok = seq0 + (ch.j - it) * FIX_CHUNK;
-        if (it >= 2 && !mbar_wait(&bar->k_empty[st], ph ^ 1, ctl)) break;
-        mbar_expect_tx(&bar->k_full[st], BN * DK * 2);
+      int kc = 0, vc = 0, nq = 0, ndiag = 0;
+      bool ok = !P.stall;   // a stalled producer (test builds) issues nothing
+      for (int round = 0; ok && round < rounds; ++round) {
+        const int t = tile_of(round, G, cta);
+        if (t >= P.ntiles) continue;
+        const Tile x = tile_info(P, t);
+        if (x.len <= 0) continue;
+        // Q of this tile once the previous tile's last QK^T has completed
+        if (nq > 0 && !mbar_wait(&bar->q_empty, (nq - 1) & 1, ctl)) { ok = false; break; }
+        mbar_expect_tx(&bar->q_full, BM * DK * 2);
         for (int hh = 0; hh < DK / 64; ++hh)
-          tma_load_3d(sK + st * BN * DK + hh * BN * 64, &tm_k, &bar->k_full[st], hh * 64, kv, ktok);
-        ++nk;
-        if (it >= 2 && !mbar_wait(&bar->v_empty[st], ph ^ 1, ctl)) break;
-        mbar_expect_tx(&bar->v_full[st], (it == 0 ? 2 : 1) * BN * DV * 2);
-        const CUtensorMap* vmap = it == 0 ? &tm_vm : &tm_vt;
-        for (int hh = 0; hh < DV / 64; ++hh)
-          tma_load_3d(sV + st * BN * DV + hh * BN * 64, vmap, &bar->v_full[st], hh * 64, kv, ktok);
-        if (it == 0)
+          tma_load_3d(sQ + hh * BM * 64, &tm_q, &bar->q_full, hh * 64, x.h, x.tok0);
+        ++nq;
+        for (int it = 0; it < x.nblk; ++it) {
+          const bool diag = it == x.nblk - 1;
+          const int j = diag ? x.j : x.j - 1 - it;
+          const int ktok = x.seq0 + j * BN;
+          const int st = kc & 1;
+          if (kc >= 2 && !mbar_wait(&bar->k_empty[st], ((kc >> 1) & 1) ^ 1, ctl)) { ok = false; break; }
+          mbar_expect_tx(&bar->k_full[st], BN * DK * 2);
+          for (int hh = 0; hh < DK / 64; ++hh)
+            tma_load_3d(sK + st * BN * DK + hh * BN * 64, &tm_k, &bar->k_full[st], hh * 64, x.kv, ktok);
+          ++kc;
+          const int sv = vc & 1;
+          if (vc >= 2 && !mbar_wait(&bar->v_empty[sv], ((vc >> 1) & 1) ^ 1, ctl)) { ok = false; break; }
+          if (diag && ndiag > 0 && !mbar_wait(&bar->vlo_empty, (ndiag - 1) & 1, ctl)) { ok = false; break; }
+          mbar_expect_tx(&bar->v_full[sv], (diag ? 2 : 1) * BN * DV * 2);
+          const CUtensorMap* vmap = diag ? &tm_vm : &tm_vt;
           for (int hh = 0; hh < DV / 64; ++hh)
-            tma_load_3d(sVl + hh * BN * 64, &tm_vml, &bar->v_full[0], hh * 64, kv, ktok);
-        ++nv;
+            tma_load_3d(sV + sv * BN * DV + hh * BN * 64, vmap, &bar->v_full[sv], hh * 64, x.kv, ktok);
+          if (diag) {
+            for (int hh = 0; hh < DV / 64; ++hh)
+              tma_load_3d(sVl + hh * BN * 64, &tm_vml, &bar->v_full[sv], hh * 64, x.kv, ktok);
+            ++ndiag;
+          }
+          ++vc;
+        }
       }
       // every issued copy must land before the CTA may exit (also after an
       // abort): wait for the last one or two issued per ring, timeout only
-      const Ctl drain{P.status, nullptr};
-      for (int it = nk - 1; it >= 0 && it >= nk - 2; --it)
-        mbar_wait(&bar->k_full[it & 1], (it >> 1) & 1, drain);
-      for (int it = nv - 1; it >= 0 && it >= nv - 2; --it)
-        mbar_wait(&bar->v_full[it & 1], (it >> 1) & 1, drain);
-      mbar_wait(&bar->q_full, 0, drain);
+      const Ctl drain{P.status, nullptr, ctl.limit_ns};
+      for (int n = kc - 1; n >= 0 && n >= kc - 2; --n) mbar_wait(&bar->k_full[n & 1], (n >> 1) & 1, drain);
+      for (int n = vc - 1; n >= 0 && n >= vc - 2; --n) mbar_wait(&bar->v_full[n & 1], (n >> 1) & 1, drain);
+      if (nq > 0) mbar_wait(&bar->q_full, (nq - 1) & 1, drain);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16(BM, BN, false, false);
-      constexpr uint32_t idesc_pv = idesc_bf16(BM, DV, false, true);
-      const uint32_t idesc_pv_off = idesc_bf16(BM, DV, false, true, cta_f16 != 0);
+      constexpr uint32_t idesc_off = idesc_bf16(BM, DV, false, true, true);   // fp16 P V''
+      constexpr uint32_t idesc_diag = idesc_bf16(BM, DV, false, true);        // bf16 hi/lo
       const uint32_t q_addr = smem_u32(sQ);
-      bool ok = mbar_wait(&bar->q_full, 0, ctl);
-      auto issue_qk = [&](int it) -> bool {
-        const int st = it & 1;
-        if (!mbar_wait(&bar->k_full[st], (it >> 1) & 1, ctl)) return false;
+      // the PV of block g - 1 is issued right after the QK^T of block g
+      struct Pend {
+        int g, it, vc, ab, use;
+        bool diag, valid;
+      } pend{0, 0, 0, 0, 0, false, false};
+      int g = 0, kc = 0, vc = 0, nt = 0;
+      bool ok = true;
+      auto issue_pv = [&](const Pend& pb) -> bool {
+        const int b = pb.g & 1, sv = pb.vc & 1;
+        if (!mbar_wait(&bar->p_full[b], (pb.g >> 1) & 1, ctl)) return false;
+        if (!mbar_wait(&bar->v_ready[sv], (pb.vc >> 1) & 1, ctl)) return false;
+        // the tile's first PV overwrites A: the epilogue of the tile that
+        // used this buffer before must have released it
+        if (pb.it == 0 && pb.use >= 1 && !mbar_wait(&bar->acc_empty[pb.ab], (pb.use - 1) & 1, ctl))
+          return false;
         tc_fence_after();
-        const uint32_t k_addr = smem_u32(sK + st * BN * DK);
+        const uint32_t acol = tmem + 256u + (uint32_t)(pb.ab * DV);
+        const uint32_t scol = tmem + col_s(b);
+        const uint32_t v_addr = smem_u32(sV + sv * BN * DV);
+        if (!pb.diag) {
 #pragma unroll
-        for (int kk = 0; kk < DK / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
-          const uint64_t a = desc_add(desc_sw128(q_addr, 16, 1024), off);
-          const uint64_t b = desc_add(desc_sw128(k_addr, 16, 1024), (kk >> 2) * (BN * 128) + (kk & 3) * 32);
-          mma_ss(tmem + col_s(st), a, b, idesc_qk, kk > 0);
-        }
-        tc_commit(&bar->s_full[st]);
-        tc_commit(&bar->k_empty[st]);
-        return true;
-      };
-      if (ok) ok = issue_qk(0);
-      if (ok && nblk > 1) ok = issue_qk(1);
-      for (int it = 0; ok && it < nblk; ++it) {
-        const int st = it & 1;
-        const uint32_t ph = (it >> 1) & 1;
-        if (!mbar_wait(&bar->p_full[st], ph, ctl) || !mbar_wait(&bar->v_ready[st], ph, ctl)) break;
-        tc_fence_after();
-        const uint32_t v_addr = smem_u32(sV + st * BN * DV);
-        if (it == 0) {
+          for (int kk = 0; kk < BN / 16; ++kk) {
+            const uint64_t bd = desc_add(desc_sw128(v_addr, BN * 128, 1024), kk * 2048);
+            mma_ts(acol, scol + kk * 8, bd, idesc_off, (pb.it > 0 || kk > 0));
+          }
+        } else {
+          // A holds the folded earlier blocks, or (first block of a chunk-0
+          // tile) what the softmax warps wrote: always accumulate
           const uint32_t vl_addr = smem_u32(sVl);
 #pragma unroll
           for (int kk = 0; kk < BN / 16; ++kk) {
             const uint64_t bh = desc_add(desc_sw128(v_addr, BN * 128, 1024), kk * 2048);
             const uint64_t bl = desc_add(desc_sw128(vl_addr, BN * 128, 1024), kk * 2048);
-            mma_ts(tmem + kColOd, tmem + col_s(0) + kk * 8, bh, idesc_pv, kk > 0);
-            mma_ts(tmem + kColOd, tmem + kColPlo + kk * 8, bh, idesc_pv, 1);
-            mma_ts(tmem + kColOd, tmem + col_s(0) + kk * 8, bl, idesc_pv, 1);
-          }
-        } else {
-#pragma unroll
-          for (int kk = 0; kk < BN / 16; ++kk) {
-            const uint64_t b = desc_add(desc_sw128(v_addr, BN * 128, 1024), kk * 2048);
-            mma_ts(tmem + kColOd + DV, tmem + col_s(st) + kk * 8, b, idesc_pv_off,
-                   (it > 1 || kk > 0));
+            mma_ts(acol, scol + kk * 8, bh, idesc_diag, 1);
+            mma_ts(acol, scol + 64 + kk * 8, bh, idesc_diag, 1);
+            mma_ts(acol, scol + kk * 8, bl, idesc_diag, 1);
           }
         }
-        tc_commit(&bar->v_empty[st]);
+        tc_commit(&bar->v_empty[sv]);
         tc_commit(&bar->pv_done);
-        if (it + 2 < nblk) ok = issue_qk(it + 2);
+        if (pb.diag) {
+          tc_commit(&bar->acc_full[pb.ab]);
+          tc_commit(&bar->vlo_empty);
+        }
+        return true;
+      };
+      for (int round = 0; ok && round < rounds; ++round) {
+        const int t = tile_of(round, G, cta);
+        if (t >= P.ntiles) continue;
+        const Tile x = tile_info(P, t);
+        if (x.len <= 0) continue;
+        const int ab = nt & 1, use = nt >> 1;
+        if (!mbar_wait(&bar->q_full, nt & 1, ctl)) { ok = false; break; }
+        for (int it = 0; it < x.nblk; ++it) {
+          const bool diag = it == x.nblk - 1;
+          const int b = g & 1, st = kc & 1;
+          if (!mbar_wait(&bar->k_full[st], (kc >> 1) & 1, ctl)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t k_addr = smem_u32(sK + st * BN * DK);
+#pragma unroll
+          for (int kk = 0; kk < DK / 16; ++kk) {
+            const uint64_t a = desc_add(desc_sw128(q_addr, 16, 1024), (kk >> 2) * (BM * 128) + (kk & 3) * 32);
+            const uint64_t bd = desc_add(desc_sw128(k_addr, 16, 1024), (kk >> 2) * (BN * 128) + (kk & 3) * 32);
+            mma_ss(tmem + col_s(b), a, bd, idesc_qk, kk > 0);
+          }
+          tc_commit(&bar->s_full[b]);
+          tc_commit(&bar->k_empty[st]);
+          if (diag) tc_commit(&bar->q_empty);
+          ++kc;
+          if (pend.valid && !issue_pv(pend)) { ok = false; break; }
+          pend = Pend{g, it, vc, ab, use, diag, true};
+          ++g;
+          ++vc;
+        }
+        ++nt;
       }
+      if (ok && pend.valid) issue_pv(pend);
       // TMEM must not be released while an issued MMA may still write it
       tc_commit(&bar->drain);
-      mbar_wait(&bar->drain, 0, Ctl{P.status, nullptr});
+      mbar_wait(&bar->drain, 0, Ctl{P.status, nullptr, ctl.limit_ns});
     }
   } else if (warp >= 4 && warp < 8) {
-    // ------------------------------------------------------------ softmax + epilogue
-    const int r = (warp - 4) * 32 + lane;              // query row in the chunk
+    // ------------------------------------------------------------ softmax
+    const int r = (warp - 4) * 32 + lane;              // query row in the tile
     const uint32_t lane_base = tmem + ((uint32_t)((warp - 4) * 32) << 16);
     const float c1 = d.scale * LOG2E;
-    float m_used = -INFINITY, m_true = -INFINITY, s_diag = 0.f;
+    int g = 0, nt = 0;
     bool ok = true;
-    for (int it = 0; it < nblk; ++it) {
-      const int st = it & 1;
-      // waits vote warp-wide: the TMEM accesses below are warp-collective
-      if (!__all_sync(0xffffffffu, mbar_wait(&bar->s_full[st], (it >> 1) & 1, ctl))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const uint32_t sbase = lane_base + col_s(st);
-      // the whole S row in registers: four TMEM loads, one wait
-      uint32_t xs[BN];
-#pragma unroll
-      for (int c4 = 0; c4 < BN / 32; ++c4)
-        tmem_ld32(sbase + c4 * 32, *reinterpret_cast<uint32_t(*)[32]>(&xs[c4 * 32]));
-      tmem_wait_ld();
-      float mx = -INFINITY;
-      if (it > 0) {
-#pragma unroll
-        for (int e = 0; e < BN; e += 2)
-          mx = fmaxf(mx, fmaxf(__uint_as_float(xs[e]), __uint_as_float(xs[e + 1])));
-      } else {
-        // diagonal block: keys s <= t; S_tt kept for the exact s = t term
-#pragma unroll
-        for (int e = 0; e < BN; ++e) {
-          const float sv = __uint_as_float(xs[e]);
-          mx = e <= r ? fmaxf(mx, sv) : mx;
-          s_diag = e == r ? sv : s_diag;
-        }
-      }
-      const float mrow = mx * d.scale;
-      m_true = fmaxf(m_true, mrow);
-      if (it == 0) {
-        m_used = m_true;
-      } else if (__any_sync(0xffffffffu, m_true > m_used + kRescaleThreshold)) {
-        // rare: some row's max grew past the threshold; the whole warp (the
-        // TMEM accesses are warp-collective) rescales its rows of O to their
-        // new max before P_it is formed against it
-        if (!__all_sync(0xffffffffu, mbar_wait(&bar->pv_done, (it - 1) & 1, ctl))) {
-          ok = false;
-          break;
-        }
+    for (int round = 0; ok && round < rounds; ++round) {
+      const int t = tile_of(round, G, cta);
+      if (t >= P.ntiles) continue;
+      const Tile x = tile_info(P, t);
+      if (x.len <= 0) continue;
+      const int tb = nt & 1, use = nt >> 1;
+      const uint32_t acol = lane_base + 256u + (uint32_t)(tb * DV);
+      float m_used = -INFINITY, m_true = -INFINITY, s_diag = 0.f;
+      for (int it = 0; it < x.nblk; ++it) {
+        const bool diag = it == x.nblk - 1;
+        const int b = g & 1;
+        const uint32_t sbase = lane_base + col_s(b);
+        // waits vote warp-wide: the TMEM accesses below are warp-collective
+        if (!__all_sync(0xffffffffu, mbar_wait(&bar->s_full[b], (g >> 1) & 1, ctl))) { ok = false; break; }
         tc_fence_after();
-        const float alpha = ex2((m_used - m_true) * LOG2E);
-        // both accumulators (before the first off-diagonal PV the O_o columns
-        // hold stale data that PV_1 overwrites, so scaling them is harmless)
+        // pass 1: the row maximum (diagonal block: keys s <= t; S_tt kept
+        // for the exact s = t term)
+        float mx = -INFINITY;
 #pragma unroll
-        for (int cc = 0; cc < 2 * DV / 32; ++cc) {
-          uint32_t x[32];
-          tmem_ld32(lane_base + kColOd + cc * 32, x);
+        for (int c4 = 0; c4 < BN / 32; ++c4) {
+          uint32_t xs[32];
+          tmem_ld32(sbase + c4 * 32, xs);
           tmem_wait_ld();
+          if (!diag) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) x[e] = __float_as_uint(__uint_as_float(x[e]) * alpha);
-          tmem_st32(lane_base + kColOd + cc * 32, x);
+            for (int e = 0; e < 32; e += 2)
+              mx = fmaxf(mx, fmaxf(__uint_as_float(xs[e]), __uint_as_float(xs[e + 1])));
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const float sv = __uint_as_float(xs[e]);
+              const int key = c4 * 32 + e;
+              mx = key <= r ? fmaxf(mx, sv) : mx;
+              s_diag = key == r ? sv : s_diag;
+            }
+          }
+        }
+        m_true = fmaxf(m_true, mx * d.scale);
+        bool rescale = false;
+        if (it == 0) m_used = m_true;
+        else rescale = __any_sync(0xffffffffu, m_true > m_used + kRescaleThreshold);
+        const bool fold = diag && x.nblk > 1;
+        // the fold factors and out-of-range flags of this tile
+        if (diag && !__all_sync(0xffffffffu, mbar_wait(&bar->fold_ready[tb], use & 1, ctl))) { ok = false; break; }
+        if (rescale || fold) {
+          // A must be quiescent: the previous block's PV has completed
+          if (!__all_sync(0xffffffffu, mbar_wait(&bar->pv_done, (g - 1) & 1, ctl))) { ok = false; break; }
+          tc_fence_after();
+          const float a_r = rescale ? ex2((m_used - m_true) * LOG2E) : 1.f;
+          const float* F = sF + tb * DV;
+#pragma unroll 1
+          for (int cc = 0; cc < DV / 32; ++cc) {
+            uint32_t xa[32];
+            tmem_ld32(acol + cc * 32, xa);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const float f = fold ? F[cc * 32 + e] * a_r : a_r;
+              xa[e] = __float_as_uint(__uint_as_float(xa[e]) * f);
+            }
+            tmem_st32(acol + cc * 32, xa);
+          }
+          tmem_wait_st();
+          if (rescale) m_used = m_true;
+        }
+        if (diag && x.nblk == 1) {
+          // chunk 0: the diagonal MMAs accumulate into A, which starts at
+          // zero here; the epilogue of the tile that used it before must be
+          // done with it
+          if (use >= 1 && !__all_sync(0xffffffffu, mbar_wait(&bar->acc_empty[tb], (use - 1) & 1, ctl))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          uint32_t z[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) z[e] = 0u;
+#pragma unroll
+          for (int cc = 0; cc < DV / 32; ++cc) tmem_st32(acol + cc * 32, z);
+          tmem_wait_st();
+        }
+        const float moff = m_used * LOG2E;
+        if (diag && sAnyBad[tb]) {
+          // exact diagonal sums of out-of-range channels, in fp32 from the
+          // fp32 logits: A_tc <- exp(L_t) A_tc + sum_{s<t} P_ts exp(L_t - L_s) v_s
+          const int* bad = sBad + tb * DV;
+          const int nk = r < x.len ? r : 0;
+          const size_t rowL = ((size_t)x.tok0 + (r < x.len ? r : 0)) * vrs + (size_t)x.kv * DV;
+          const float* Lk = P.L + (size_t)x.tok0 * vrs + (size_t)x.kv * DV;
+          const __nv_bfloat16* vk = P.v + (size_t)x.tok0 * vrs + (size_t)x.kv * DV;
+#pragma unroll 1
+          for (int c = 0; c < DV; ++c) {
+            if (!bad[c]) continue;   // tile-uniform
+            const float lt = P.L[rowL + c];
+            float acc = 0.f;
+#pragma unroll 1
+            for (int c4 = 0; c4 < BN / 32; ++c4) {
+              uint32_t xs[32];
+              tmem_ld32(sbase + c4 * 32, xs);
+              tmem_wait_ld();
+#pragma unroll 4
+              for (int e = 0; e < 32; ++e) {
+                const int s = c4 * 32 + e;
+                if (s < nk) {
+                  const float p = ex2(__uint_as_float(xs[e]) * c1 - moff);
+                  acc += p * ex2((lt - Lk[(size_t)s * vrs + c]) * LOG2E) * bf2f(vk[(size_t)s * vrs + c]);
+                }
+              }
+            }
+            uint32_t xa;
+            asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(xa) : "r"(acol + c));
+            tmem_wait_ld();
+            tmem_st1(acol + c, __float_as_uint(ex2(lt * LOG2E) * __uint_as_float(xa) + acc));
+          }
+          tmem_wait_st();
+        }
+        // pass 2: P, written over the S columns already read
+        if (!diag) {
+#pragma unroll
+          for (int c4 = 0; c4 < BN / 32; ++c4) {
+            uint32_t xs[32], pk[16];
+            tmem_ld32(sbase + c4 * 32, xs);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; e += 2)
+              pk[e >> 1] = pack_f16(ex2(__uint_as_float(xs[e]) * c1 - moff),
+                                    ex2(__uint_as_float(xs[e + 1]) * c1 - moff));
+            tmem_st16(sbase + c4 * 16, pk);
+          }
+        } else {
+          // strictly causal P as bf16 hi (columns [0, 64)) + lo ([64, 128));
+          // lo parts are stored only over S columns already read: those of
+          // key chunks 0 and 1 after chunk 2 is read, those of 2 and 3 after
+          // chunk 3 (separate register arrays: a tcgen05.st may still read
+          // its source registers until the wait)
+          uint32_t plo0[16], plo1[16], plo2[16];
+#pragma unroll
+          for (int c4 = 0; c4 < BN / 32; ++c4) {
+            uint32_t xs[32], ph[16], pl[16];
+            tmem_ld32(sbase + c4 * 32, xs);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              const int key = c4 * 32 + e;
+              const float p0 = key < r ? ex2(__uint_as_float(xs[e]) * c1 - moff) : 0.f;
+              const float p1 = key + 1 < r ? ex2(__uint_as_float(xs[e + 1]) * c1 - moff) : 0.f;
+              ph[e >> 1] = pack_bf16(p0, p1);
+              const float h0 = __uint_as_float(ph[e >> 1] << 16);
+              const float h1 = __uint_as_float(ph[e >> 1] & 0xFFFF0000u);
+              pl[e >> 1] = pack_bf16(p0 - h0, p1 - h1);
+            }
+            tmem_st16(sbase + c4 * 16, ph);
+            if (c4 == 0) {
+#pragma unroll
+              for (int e = 0; e < 16; ++e) plo0[e] = pl[e];
+            } else if (c4 == 1) {
+#pragma unroll
+              for (int e = 0; e < 16; ++e) plo1[e] = pl[e];
+            } else if (c4 == 2) {
+              tmem_st16(sbase + 64, plo0);
+              tmem_st16(sbase + 80, plo1);
+#pragma unroll
+              for (int e = 0; e < 16; ++e) plo2[e] = pl[e];
+            } else {
+              tmem_st16(sbase + 96, plo2);
+              tmem_st16(sbase + 112, pl);
+            }
+          }
         }
         tmem_wait_st();
-        m_used = m_true;
+        tc_fence_before();
+        mbar_arrive(&bar->p_full[b]);
+        ++g;
       }
-      const float moff = m_used * LOG2E;
-      if (it == 0) {
-        // diagonal block: strictly causal P as bf16 hi + lo
-#pragma unroll
-        for (int c4 = 0; c4 < BN / 32; ++c4) {
-          uint32_t pk[16], pl[16];
-#pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const int key = c4 * 32 + e;
-            const float p0 = key < r ? ex2(__uint_as_float(xs[key]) * c1 - moff) : 0.f;
-            const float p1 = key + 1 < r ? ex2(__uint_as_float(xs[key + 1]) * c1 - moff) : 0.f;
-            pk[e >> 1] = pack_bf16(p0, p1);
-            const float h0 = __uint_as_float(pk[e >> 1] << 16);
-            const float h1 = __uint_as_float(pk[e >> 1] & 0xFFFF0000u);
-            pl[e >> 1] = pack_bf16(p0 - h0, p1 - h1);
-          }
-          tmem_st16(sbase + c4 * 16, pk);
-          tmem_st16(lane_base + kColPlo + c4 * 16, pl);
-        }
-      } else if (cta_f16) {
-#pragma unroll
-        for (int c4 = 0; c4 < BN / 32; ++c4) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const int key = c4 * 32 + e;
-            pk[e >> 1] = pack_f16(ex2(__uint_as_float(xs[key]) * c1 - moff),
-                                  ex2(__uint_as_float(xs[key + 1]) * c1 - moff));
-          }
-          tmem_st16(sbase + c4 * 16, pk);
-        }
-      } else {
-#pragma unroll
-        for (int c4 = 0; c4 < BN / 32; ++c4) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const int key = c4 * 32 + e;
-            pk[e >> 1] = pack_bf16(ex2(__uint_as_float(xs[key]) * c1 - moff),
-                                   ex2(__uint_as_float(xs[key + 1]) * c1 - moff));
-          }
-          tmem_st16(sbase + c4 * 16, pk);
-        }
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&bar->p_full[st]);
+      if (!ok) break;
+      // per-row results of the tile for its epilogue
+      if (use >= 1 && !__all_sync(0xffffffffu, mbar_wait(&bar->rows_free[tb], (use - 1) & 1, ctl))) { ok = false; break; }
+      float* rows = sRows + tb * 3 * BM;
+      rows[r] = ex2((m_used - m_true) * LOG2E);                    // alpha
+      rows[BM + r] = ex2((s_diag * d.scale - m_true) * LOG2E);    // P_tt
+      rows[2 * BM + r] = m_true;
+      mbar_arrive(&bar->rows_ready[tb]);
+      ++nt;
     }
-
-    // ---------------------------------------------------------- epilogue
-    // Every MMA of the CTA has completed once `drain` has: the MMA warp
-    // commits it once, after its last PV.  (pv_done completes once per PV, so
-    // a warp that reaches this point late could find it two phases on and
-    // wait for a phase that never comes.)
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bar->drain, 0, ctl));
-    tc_fence_after();
-    const bool row_ok = ok && r < ch.len;
-    const size_t tok = (size_t)ch.tok0 + (size_t)(r < ch.len ? r : 0);
-    if (any_bad) {
-      // exact fp32 diagonal block for channels outside the split's range:
-      // P rows into the (now idle) K/V ring, then one pass per such channel;
-      // the result replaces that channel's (zero) diagonal accumulator column
-      float* prow = reinterpret_cast<float*>(smem + Lay::kScratch) + (size_t)r * BN;
-      const size_t krs = (size_t)d.Hkv * DK;
-      const __nv_bfloat16* kbase = P.k + (size_t)ch.tok0 * krs + (size_t)kv * DK;
-      const __nv_bfloat16* qrow = P.q + tok * (size_t)d.Hq * DK + (size_t)h * DK;
-      const int nk = row_ok ? r : 0;
-      for (int s = 0; s < nk; ++s) {
-        const __nv_bfloat16* krow = kbase + (size_t)s * krs;
-        float acc = 0.f;
-        for (int dd = 0; dd < DK; dd += 8) {
-          const uint4 qa = *reinterpret_cast<const uint4*>(qrow + dd);
-          const uint4 ka = *reinterpret_cast<const uint4*>(krow + dd);
-          const uint32_t qw[4] = {qa.x, qa.y, qa.z, qa.w}, kw[4] = {ka.x, ka.y, ka.z, ka.w};
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            acc += __uint_as_float(qw[u] << 16) * __uint_as_float(kw[u] << 16);
-            acc += __uint_as_float(qw[u] & 0xFFFF0000u) * __uint_as_float(kw[u] & 0xFFFF0000u);
-          }
-        }
-        prow[s] = ex2((acc * d.scale - m_true) * LOG2E);
-      }
-      const float* Lrow = P.L + tok * vrs + (size_t)kv * DV;
-      const float* Lcol0 = P.L + (size_t)ch.tok0 * vrs + (size_t)kv * DV;
-      const __nv_bfloat16* vcol0 = P.v + (size_t)ch.tok0 * vrs + (size_t)kv * DV;
-      for (int c = 0; c < DV; ++c) {
-        if (sHr[c] <= FIX_HR_MAX) continue;   // CTA-uniform
-        const float e = exact_diag_channel(prow, nk, Lrow[c], Lcol0 + c, vcol0 + c, vrs);
-        tmem_st1(lane_base + kColOd + c, __float_as_uint(e));
-      }
-      tmem_wait_st();
-      asm volatile("bar.sync 1, 128;" ::: "memory");   // P rows done before the tile overwrites them
-    }
-    // phase A: this row's two accumulators into a shared fp32 tile, its 16-byte
-    // groups XOR-swizzled by row so that neighbouring rows hit other banks
-    float* tile = reinterpret_cast<float*>(smem + Lay::kScratch);
-    float* trow = tile + (size_t)r * (2 * DV);
-#pragma unroll
-    for (int cc = 0; cc < 2 * DV / 32; ++cc) {
-      uint32_t x[32];
-      tmem_ld32(lane_base + kColOd + cc * 32, x);
-      tmem_wait_ld();
-#pragma unroll
-      for (int g4 = 0; g4 < 8; ++g4) {
-        const int grp = cc * 8 + g4;
-        *reinterpret_cast<float4*>(trow + ((grp ^ (r & 7)) << 2)) =
-            make_float4(__uint_as_float(x[4 * g4]), __uint_as_float(x[4 * g4 + 1]),
-                        __uint_as_float(x[4 * g4 + 2]), __uint_as_float(x[4 * g4 + 3]));
-      }
-    }
-    float* sRow = reinterpret_cast<float*>(smem + Lay::kRow);
-    sRow[r] = ok ? ex2((m_used - m_true) * LOG2E) : 0.f;                 // alpha
-    sRow[BM + r] = ex2((s_diag * d.scale - m_true) * LOG2E);              // P_tt
-    sRow[2 * BM + r] = m_true;
-  } else if (warp >= 8) {
-    // ------------------------------------------------------------ V decay (j < i)
+  } else if (warp >= 8 && warp < 12) {
+    // ------------------------------------------------------------ V scaling
     const int dt = tid - 256;                        // 0..127
     constexpr int kChunks = DV / 8;                  // 16-byte chunks per row
     constexpr int kRowsPerPass = 128 / kChunks;
     const int lc = dt % kChunks;                     // logical chunk: channels lc*8 .. +7
     const int r0 = dt / kChunks;
     const int half = lc >> 3, lcc = lc & 7;
-    float delta[8], f8[8];
+    int vc = 0, nt = 0;
+    bool ok = true;
+    for (int round = 0; ok && round < rounds; ++round) {
+      const int t = tile_of(round, G, cta);
+      if (t >= P.ntiles) continue;
+      const Tile x = tile_info(P, t);
+      if (x.len <= 0) continue;
+      const int tb = nt & 1, use = nt >> 1;
+      // the fold factors of two tiles ago are consumed once its diagonal PV
+      // has completed (it follows the fold)
+      // (every wait of this warpgroup ends in a vote on a named barrier, so
+      // that all 128 threads leave together after an abort)
+      if (!wg_and(2, use < 1 || mbar_wait(&bar->acc_full[tb], (use - 1) & 1, ctl))) { ok = false; break; }
+      // tile-wide power-of-two scale k_c of the earlier blocks' operands:
+      // not needed (0) when every earlier chunk is fp16-safe (g <= 0)
+      int my_safe = 1;
+      for (int jj = dt; jj < x.nblk - 1; jj += 128) my_safe &= P.safe[(size_t)(x.first + jj) * d.Hkv + x.kv];
+      const int tile_safe = wg_and(2, my_safe);
+      float kexp[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) delta[e] = 0.f;
-    for (int it = 0; it < nblk; ++it) {
-      const int st = it & 1;
-      const int j = ch.j - it;
-      if (it >= 2) {
-        const float* tp = P.tot + ((size_t)(first + j + 1) * d.Hkv + kv) * DV + lc * 8;
-        const float4 t0 = *reinterpret_cast<const float4*>(tp);
-        const float4 t1 = *reinterpret_cast<const float4*>(tp + 4);
-        delta[0] += t0.x; delta[1] += t0.y; delta[2] += t0.z; delta[3] += t0.w;
-        delta[4] += t1.x; delta[5] += t1.y; delta[6] += t1.z; delta[7] += t1.w;
-      }
+      for (int e = 0; e < 8; ++e) kexp[e] = 0.f;
+      if (!tile_safe) {
+        float delta[8], kmax[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) f8[e] = ex2(delta[e] * LOG2E);
-      if (!mbar_wait(&bar->v_full[st], (it >> 1) & 1, ctl)) break;
-      if (it > 0) {
-        // Vt arrives as fp16 or bf16 (per chunk, see the prefix pass); V' is
-        // written in the operand type of this CTA's off-diagonal MMAs
-        const bool in_f16 = P.safe[(size_t)(first + j) * d.Hkv + kv] != 0;
-        uint8_t* vb = reinterpret_cast<uint8_t*>(sV + st * BN * DV) + half * (BN * 128);
-#pragma unroll 4
-        for (int s = r0; s < BN; s += kRowsPerPass) {
-          uint4* p = reinterpret_cast<uint4*>(vb + s * 128 + ((lcc ^ (s & 7)) << 4));
-          uint4 x = *p;
-          uint32_t w4[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            float a, b;
-            if (in_f16) {
-              const float2 ab = __half22float2(*reinterpret_cast<const __half2*>(&w4[u]));
-              a = ab.x;
-              b = ab.y;
-            } else {
-              a = __uint_as_float(w4[u] << 16);
-              b = __uint_as_float(w4[u] & 0xFFFF0000u);
-            }
-            a *= f8[2 * u];
-            b *= f8[2 * u + 1];
-            w4[u] = cta_f16 ? pack_f16(a, b) : pack_bf16(a, b);
-          }
-          *p = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+        for (int e = 0; e < 8; ++e) {
+          delta[e] = 0.f;
+          kmax[e] = -1e30f;
         }
-        fence_proxy_async_smem();
+        for (int it = 0; it < x.nblk - 1; ++it) {
+          const int j = x.j - 1 - it;
+          if (it >= 1) {
+            const float* tp = P.tot + ((size_t)(x.first + j + 1) * d.Hkv + x.kv) * DV + lc * 8;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) delta[e] += tp[e];
+          }
+          const float* lv = P.lvt + ((size_t)(x.first + j) * d.Hkv + x.kv) * DV + lc * 8;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) kmax[e] = fmaxf(kmax[e], lv[e] + delta[e] * LOG2E);
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) kexp[e] = kmax[e] > 15.f ? ceilf(kmax[e] - 15.f) : 0.f;
       }
-      mbar_arrive(&bar->v_ready[st]);
+      if (r0 == 0) {
+        const size_t ti = ((size_t)x.ci * d.Hkv + x.kv) * DV + lc * 8;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const bool bad = P.hr[ti + e] > FIX_HR_MAX;
+          sF[tb * DV + lc * 8 + e] = ex2(P.rho[ti + e] * LOG2E + kexp[e]);
+          sBad[tb * DV + lc * 8 + e] = bad ? 1 : 0;
+        }
+      }
+      {
+        int my_bad = 0;
+        if (r0 == 0) {
+          const size_t ti = ((size_t)x.ci * d.Hkv + x.kv) * DV + lc * 8;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) my_bad |= P.hr[ti + e] > FIX_HR_MAX ? 1 : 0;
+        }
+        const int any = wg_or(2, my_bad);
+        if (dt == 0) sAnyBad[tb] = any;
+      }
+      mbar_arrive(&bar->fold_ready[tb]);
+      float delta[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) delta[e] = 0.f;
+      for (int it = 0; it < x.nblk; ++it) {
+        const bool diag = it == x.nblk - 1;
+        const int sv = vc & 1;
+        float f8[8];
+        if (!diag) {
+          const int j = x.j - 1 - it;
+          if (it >= 1) {
+            const float* tp = P.tot + ((size_t)(x.first + j + 1) * d.Hkv + x.kv) * DV + lc * 8;
+            const float4 t0 = *reinterpret_cast<const float4*>(tp);
+            const float4 t1 = *reinterpret_cast<const float4*>(tp + 4);
+            delta[0] += t0.x; delta[1] += t0.y; delta[2] += t0.z; delta[3] += t0.w;
+            delta[4] += t1.x; delta[5] += t1.y; delta[6] += t1.z; delta[7] += t1.w;
+          }
+          // Vt is stored as fp16 times 2^-e; V'' = Vt_true f_ij 2^-k
+          const float* lv = P.lvt + ((size_t)(x.first + j) * d.Hkv + x.kv) * DV + lc * 8;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) f8[e] = ex2(delta[e] * LOG2E + vt_exponent(lv[e]) - kexp[e]);
+        }
+        if (!wg_and(2, mbar_wait(&bar->v_full[sv], (vc >> 1) & 1, ctl))) { ok = false; break; }
+        if (!diag) {
+          uint8_t* vb = reinterpret_cast<uint8_t*>(sV + sv * BN * DV) + half * (BN * 128);
+#pragma unroll 4
+          for (int s = r0; s < BN; s += kRowsPerPass) {
+            uint4* p = reinterpret_cast<uint4*>(vb + s * 128 + ((lcc ^ (s & 7)) << 4));
+            uint4 xv = *p;
+            uint32_t w4[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const float2 ab = __half22float2(*reinterpret_cast<const __half2*>(&w4[u]));
+              w4[u] = pack_f16(ab.x * f8[2 * u], ab.y * f8[2 * u + 1]);
+            }
+            *p = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+          }
+          fence_proxy_async_smem();
+        }
+        mbar_arrive(&bar->v_ready[sv]);
+        ++vc;
+      }
+      ++nt;
+    }
+  } else if (warp >= 12) {
+    // ------------------------------------------------------------ epilogue
+    const int ew = warp - 12;                        // TMEM lanes [32 ew, 32 ew + 32)
+    const uint32_t lane_base = tmem + ((uint32_t)(ew * 32) << 16);
+    float* tr = reinterpret_cast<float*>(smem + Lay::kEpiT) + ew * 32 * 33;
+    const float* sW = reinterpret_cast<const float*>(smem + Lay::kEpiW);
+    float* eRho = reinterpret_cast<float*>(smem + Lay::kEpiRho);
+    int* eBad = reinterpret_cast<int*>(smem + Lay::kEpiBad);
+    const int et = tid - 384;                        // 0..127
+    float* __restrict__ yf = P.y_f32 ? reinterpret_cast<float*>(P.y) : nullptr;
+    __nv_bfloat16* __restrict__ yb = P.y_f32 ? nullptr : reinterpret_cast<__nv_bfloat16*>(P.y);
+    const size_t ors = (size_t)d.Hq * DV;
+    constexpr int kU = DV / 32;                      // 32-channel chunks
+    constexpr int kR = 8;                            // rows per pass
+    int nt = 0;
+    bool ok = true;
+    for (int round = 0; ok && round < rounds; ++round) {
+      const int t = tile_of(round, G, cta);
+      if (t >= P.ntiles) continue;
+      const Tile x = tile_info(P, t);
+      if (x.len <= 0) continue;
+      const int tb = nt & 1, use = nt >> 1;
+      // channel data of this tile (the previous tile's readers are done:
+      // every epilogue thread passed the sync at the end of that tile)
+      if (et < DV) {
+        const size_t ti = ((size_t)x.ci * d.Hkv + x.kv) * DV + et;
+        eRho[et] = P.rho[ti];
+        eBad[et] = P.hr[ti] > FIX_HR_MAX ? 1 : 0;
+      }
+      wg_sync(3);
+      if (!wg_and(3, mbar_wait(&bar->acc_full[tb], use & 1, ctl) &&
+                         mbar_wait(&bar->rows_ready[tb], use & 1, ctl))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const float* rows = sRows + tb * 3 * BM;
+      const uint32_t acol = lane_base + 256u + (uint32_t)(tb * DV);
+      const float* Lg = P.L + (size_t)x.kv * DV;
+      const __nv_bfloat16* vg = P.v + (size_t)x.kv * DV;
+#pragma unroll 1
+      for (int grp = 0; grp < 32 / kR; ++grp) {
+        const int rbase = ew * 32 + grp * kR;          // first tile row of this pass
+        float o[kR][kU];
+        float ss[kR];
+#pragma unroll
+        for (int q = 0; q < kR; ++q) ss[q] = 0.f;
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+          const int c = u * 32 + lane;
+          // L and v of the pass's rows (lanes over channels: coalesced)
+          float lt[kR], vt[kR];
+#pragma unroll
+          for (int q = 0; q < kR; ++q) {
+            const int rr = min(rbase + q, x.len - 1);
+            const size_t tk = (size_t)x.tok0 + rr;
+            lt[q] = Lg[tk * vrs + c];
+            vt[q] = bf2f(vg[tk * vrs + c]);
+          }
+          // A columns [32u, 32u + 32) of the warp's 32 rows, transposed
+          uint32_t xa[32];
+          tmem_ld32(acol + u * 32, xa);
+          tmem_wait_ld();
+          __syncwarp();
+          if (lane >= grp * kR && lane < grp * kR + kR) {
+            float* trow = tr + (lane - grp * kR) * 33;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) trow[e] = __uint_as_float(xa[e]);
+          }
+          __syncwarp();
+          const float rc = eRho[c];
+          const bool bc = eBad[c] != 0;
+#pragma unroll
+          for (int q = 0; q < kR; ++q) {
+            const float a = tr[q * 33 + lane];
+            const float alpha = rows[rbase + q], ptt = rows[BM + rbase + q];
+            const float fac = bc ? 1.f : ex2((lt[q] - rc) * LOG2E);
+            const float val = alpha * fac * a + ptt * vt[q];
+            o[q][u] = val;
+            ss[q] += val * val;
+          }
+        }
+        float rstd[kR];
+#pragma unroll
+        for (int q = 0; q < kR; ++q) rstd[q] = 1.0f / sqrtf(warp_sum(ss[q]) / (float)DV + d.eps);
+#pragma unroll
+        for (int q = 0; q < kR; ++q) {
+          const int rr = rbase + q;
+          if (rr >= x.len) break;
+          const size_t a0 = ((size_t)x.tok0 + rr) * ors + (size_t)x.h * DV;
+#pragma unroll
+          for (int u = 0; u < kU; ++u) {
+            const int c = u * 32 + lane;
+            const float yv = o[q][u] * rstd[q] * sW[c];
+            if (yf) yf[a0 + c] = yv;
+            else yb[a0 + c] = f2bf(yv);
+            if (P.o_s) P.o_s[a0 + c] = o[q][u];
+          }
+        }
+        if (P.o_s && lane < kR && rbase + lane < x.len) {
+          float rs = rstd[0];
+#pragma unroll
+          for (int q = 1; q < kR; ++q) rs = lane == q ? rstd[q] : rs;
+          const size_t tk = (size_t)x.tok0 + rbase + lane;
+          P.m_s[tk * d.Hq + x.h] = rows[2 * BM + rbase + lane];
+          P.rstd_s[tk * d.Hq + x.h] = rs;
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&bar->acc_empty[tb]);
+      mbar_arrive(&bar->rows_free[tb]);
+      wg_sync(3);
+      ++nt;
     }
   }
 
-  // ------------------------------------------------------------ phase B
-  // every warp once the roles are done, rows in batches, lanes over
-  // channels: coalesced L / v loads, the RMSNorm reduction and coalesced
-  // y / o stores
-  __syncthreads();
-  {
-    if (!*sAbort) {
-      const float* __restrict__ tile = reinterpret_cast<const float*>(smem + Lay::kScratch);
-      const float* __restrict__ sRow = reinterpret_cast<const float*>(smem + Lay::kRow);
-      const float* __restrict__ Lg = P.L + (size_t)kv * DV;
-      const __nv_bfloat16* __restrict__ vg = P.v + (size_t)kv * DV;
-      float* __restrict__ yf = P.y_f32 ? reinterpret_cast<float*>(P.y) : nullptr;
-      __nv_bfloat16* __restrict__ yb = P.y_f32 ? nullptr : reinterpret_cast<__nv_bfloat16*>(P.y);
-      float* __restrict__ osv = P.o_s;
-      const bool has_off = nblk > 1;
-      const size_t ors = (size_t)d.Hq * DV;
-      constexpr int kU = DV / 32;
-      constexpr int kRows = 4;                         // rows in flight per warp
-      float rho_l[kU], w_l[kU];
-      bool bad_l[kU];
-#pragma unroll
-      for (int u = 0; u < kU; ++u) {
-        const int c = lane + 32 * u;
-        rho_l[u] = sRho[c];
-        w_l[u] = sW[c];
-        bad_l[u] = sHr[c] > FIX_HR_MAX;           // od holds the exact diagonal sum
-      }
-      for (int r0 = warp * kRows; r0 < ch.len; r0 += (kThreads / 32) * kRows) {
-        float lt[kRows][kU], vt[kRows][kU];
-#pragma unroll
-        for (int q = 0; q < kRows; ++q) {
-          const int rr = min(r0 + q, ch.len - 1);
-          const size_t tk = (size_t)ch.tok0 + rr;
-#pragma unroll
-          for (int u = 0; u < kU; ++u) {
-            const int c = lane + 32 * u;
-            lt[q][u] = Lg[tk * vrs + c];
-            vt[q][u] = bf2f(vg[tk * vrs + c]);
-          }
-        }
-#pragma unroll
-        for (int q = 0; q < kRows; ++q) {
-          const int rr = r0 + q;
-          if (rr >= ch.len) break;
-          const size_t tk = (size_t)ch.tok0 + rr;
-          const float* trow = tile + (size_t)rr * (2 * DV);
-          const float alpha = sRow[rr], ptt = sRow[BM + rr];
-          float o[kU];
-          float ss = 0.f;
-#pragma unroll
-          for (int u = 0; u < kU; ++u) {
-            const int c = lane + 32 * u;
-            const float od = trow[(((c >> 2) ^ (rr & 7)) << 2) + (c & 3)];
-            const int co = DV + c;
-            const float oo = trow[(((co >> 2) ^ (rr & 7)) << 2) + (co & 3)];
-            float x = bad_l[u] ? od : alpha * od * ex2((lt[q][u] - rho_l[u]) * LOG2E);
-            if (has_off) x += alpha * oo * ex2(lt[q][u] * LOG2E);
-            x += ptt * vt[q][u];
-            o[u] = x;
-            ss += x * x;
-          }
-          ss = warp_sum(ss);
-          const float rstd = 1.0f / sqrtf(ss / (float)DV + d.eps);
-          const size_t a0 = tk * ors + (size_t)h * DV;
-#pragma unroll
-          for (int u = 0; u < kU; ++u) {
-            const int c = lane + 32 * u;
-            const float yv = o[u] * rstd * w_l[u];
-            if (yf) yf[a0 + c] = yv;
-            else yb[a0 + c] = f2bf(yv);
-            if (osv) osv[a0 + c] = o[u];
-          }
-          if (osv && lane == 0) {
-            P.m_s[tk * d.Hq + h] = sRow[2 * BM + rr];
-            P.rstd_s[tk * d.Hq + h] = rstd;
-          }
-        }
-      }
-    }
-  }
   // ---------------------------------------------------------------- teardown
   tc_fence_before();
   __syncthreads();
@@ -630,7 +829,7 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// [N, H, D] bf16 viewed as a 3-D tensor (D, H, N); box = 64 x 1 x 128 rows,
+// [N, H, D] 16-bit viewed as a 3-D tensor (D, H, N); box = 64 x 1 x 128 rows,
 // 128-byte swizzle (the canonical K-major / MN-major operand layout).
 static bool make_map(CUtensorMap* m, const void* base, int D, int H, int N) {
   auto fn = encode_fn();
@@ -642,6 +841,14 @@ static bool make_map(CUtensorMap* m, const void* base, int D, int H, int N) {
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+static int num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    return 148;
+  return n;
 }
 
 template <int DK, int DV>
@@ -657,8 +864,10 @@ static fix_status launch(const Params& prm, const void* q, const void* k, const 
   auto kern = fwd_tc_kernel<DK, DV>;
   if (!set_smem_limit(reinterpret_cast<const void*>(kern), smem))
     return FIX_ERR_CUDA;
-  const long long grid = (long long)d.nchunks * d.Hq;
-  if (grid <= 0) return FIX_OK;
+  if (prm.ntiles <= 0) return FIX_OK;
+  static int sms = 0;   // one CTA per SM, persistent
+  if (!sms) sms = num_sms();
+  const int grid = prm.ntiles < sms ? prm.ntiles : sms;
   kern<<<(unsigned)grid, kThreads, smem, st>>>(mq, mk, mvt, mvm, mvml, prm);
   return cudaGetLastError() == cudaSuccess ? FIX_OK : FIX_ERR_CUDA;
 }
@@ -676,13 +885,16 @@ fix_status tc_fwd(const Dims& d, const Chunk* chunks, const int* order, const vo
                   const void* k, const uint16_t* vt, const __nv_bfloat16* vm,
                   const __nv_bfloat16* vml, const void* v,
                   const float* L, const float* tot, const float* rho, const float* hr,
-                  const int* safe,
+                  const float* lvt, const int* safe,
                   const void* w, void* y, bool y_f32, float* o_s, float* m_s, float* rstd_s,
                   int* status, cudaStream_t st) {
   tcf::Params prm{};
   prm.d = d;
   prm.chunks = chunks;
   prm.order = order;
+  const long long nt = (long long)d.nchunks * d.Hq;
+  if (nt > (1LL << 30)) return FIX_ERR_SHAPE;
+  prm.ntiles = (int)nt;
   prm.q = static_cast<const __nv_bfloat16*>(q);
   prm.k = static_cast<const __nv_bfloat16*>(k);
   prm.v = static_cast<const __nv_bfloat16*>(v);
@@ -690,6 +902,7 @@ fix_status tc_fwd(const Dims& d, const Chunk* chunks, const int* order, const vo
   prm.tot = tot;
   prm.rho = rho;
   prm.hr = hr;
+  prm.lvt = lvt;
   prm.safe = safe;
   prm.w = static_cast<const __nv_bfloat16*>(w);
   prm.y = y;
@@ -698,6 +911,9 @@ fix_status tc_fwd(const Dims& d, const Chunk* chunks, const int* order, const vo
   prm.m_s = m_s;
   prm.rstd_s = rstd_s;
   prm.status = status;
+#ifdef FIX_TEST_HOOKS
+  prm.stall = test_stall_forward();
+#endif
   if (d.Dk == 128 && d.Dv == 128) return tcf::launch<128, 128>(prm, q, k, vt, vm, vml, st);
   if (d.Dk == 64 && d.Dv == 64) return tcf::launch<64, 64>(prm, q, k, vt, vm, vml, st);
   if (d.Dk == 128 && d.Dv == 64) return tcf::launch<128, 64>(prm, q, k, vt, vm, vml, st);
