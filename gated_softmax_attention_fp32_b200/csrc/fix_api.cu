@@ -25,7 +25,8 @@ static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 // Validates the problem descriptor and fills the kernel-side dims.
 static fix_status make_dims(const fix_attn_problem* p, Dims* d) {
   if (!p) return FIX_ERR_NULL;
-  if (p->flags & ~FIX_FLAG_REUSE_FWD_WORKSPACE) return FIX_ERR_SHAPE;
+  if (p->flags & ~(FIX_FLAG_REUSE_FWD_WORKSPACE | FIX_FLAG_NO_NORM | FIX_FLAG_SCALAR_GATE))
+    return FIX_ERR_SHAPE;
   if (p->y_dtype != FIX_DTYPE_BF16 && p->y_dtype != FIX_DTYPE_F32) return FIX_ERR_DTYPE;
   if (p->algo < FIX_ALGO_AUTO || p->algo > FIX_ALGO_TC) return FIX_ERR_DTYPE;
   if (p->batch < 1 || p->seqlen < 0 || p->num_q_heads < 1 || p->num_kv_heads < 1)
@@ -49,6 +50,8 @@ static fix_status make_dims(const fix_attn_problem* p, Dims* d) {
   d->grp = p->num_q_heads / p->num_kv_heads;
   d->scale = p->scale > 0.f ? p->scale : 1.0f / std::sqrt((float)p->head_dim_k);
   d->eps = p->eps;
+  d->no_norm = (p->flags & FIX_FLAG_NO_NORM) ? 1 : 0;
+  d->scalar_gate = (p->flags & FIX_FLAG_SCALAR_GATE) ? 1 : 0;
   long long nch = 0;
   if (p->cu_seqlens) {
     if (p->batch != 1) return FIX_ERR_SHAPE;
@@ -124,7 +127,7 @@ static SplitPlan plan_split(const fix_attn_problem* p, const Dims& d) {
 // Workspace layout (all offsets 256-byte aligned).
 struct Ws {
   size_t status, chunks, order, safe, L, vt, vm, vml, tot, rho, hr, lvt;   // forward and backward
-  size_t dow, dot, domh, doml, dsafe, hmax, ptt, A, dG, dtot, dwp;   // backward only
+  size_t dow, dot, domh, doml, dsafe, hmax, ptt, delta, A, dG, dtot, dwp, dgf;   // backward only
   size_t parts, cpart, partial;                            // dk/dv work split
   size_t total;
 };
@@ -159,6 +162,7 @@ static Ws layout(const Dims& d, bool bwd, const SplitPlan& sp) {
     w.dsafe = take((size_t)(d.nchunks > 0 ? d.nchunks : 1) * d.Hq * sizeof(int));
     w.hmax = take((size_t)(d.nchunks > 0 ? d.nchunks : 1) * d.Hq * sizeof(int));
     w.ptt = take((size_t)d.N * d.Hq * sizeof(float));
+    w.delta = take((size_t)d.N * d.Hq * sizeof(float));
     w.A = take(nkv * 4);
     w.dG = take(nkv * 4);
     w.dtot = take(nch * 4);
@@ -166,6 +170,8 @@ static Ws layout(const Dims& d, bool bwd, const SplitPlan& sp) {
     w.parts = take((size_t)(sp.nparts > 0 ? sp.nparts : 1) * sizeof(Part));
     w.cpart = take((size_t)(d.nchunks > 0 ? d.nchunks : 1) * sizeof(int2));
     w.partial = take((size_t)sp.nslots * d.Hkv * FIX_CHUNK * (d.Dk + d.Dv) * 4);
+    // a scalar gate's per-channel dg, summed over the channels at the end
+    w.dgf = d.scalar_gate ? take(nkv * 4) : 0;
   }
   w.total = o;
   return w;
@@ -396,15 +402,16 @@ const char* fix_attn_status_string(int s) {
 }
 
 fix_status fix_attn_fwd(const fix_attn_problem* p, const void* q, const void* k, const void* v,
-                        const float* g, const void* w, void* y, float* o_s, float* m_s,
-                        float* rstd_s, void* workspace, size_t ws_bytes, void* stream) {
+                        const float* g, const void* w, const void* z, void* y, float* o_s,
+                        float* m_s, float* rstd_s, void* workspace, size_t ws_bytes,
+                        void* stream) {
   Dims d;
   FIX_TRY(make_dims(p, &d));
-  if (!q || !k || !v || !g || !w || !y || !workspace) return FIX_ERR_NULL;
+  if (!q || !k || !v || !g || (!w && !d.no_norm) || !y || !workspace) return FIX_ERR_NULL;
   const int nsaved = (o_s != nullptr) + (m_s != nullptr) + (rstd_s != nullptr);
   if (nsaved != 0 && nsaved != 3) return FIX_ERR_NULL;
-  for (const void* ptr : {q, k, v, (const void*)g, w, (const void*)y, (const void*)workspace})
-    if (!aligned16(ptr)) return FIX_ERR_ALIGN;
+  for (const void* ptr : {q, k, v, (const void*)g, w, z, (const void*)y, (const void*)workspace})
+    if (ptr && !aligned16(ptr)) return FIX_ERR_ALIGN;
   if (nsaved && (!aligned16(o_s) || !aligned16(m_s) || !aligned16(rstd_s))) return FIX_ERR_ALIGN;
   const Ws ws = layout(d, false, SplitPlan{});
   if (ws_bytes < ws.total) return FIX_ERR_WORKSPACE;
@@ -430,34 +437,37 @@ fix_status fix_attn_fwd(const fix_attn_problem* p, const void* q, const void* k,
                    reinterpret_cast<const float*>(base + ws.rho),
                    reinterpret_cast<const float*>(base + ws.hr),
                    reinterpret_cast<const float*>(base + ws.lvt),
-                   reinterpret_cast<const int*>(base + ws.safe), w, y, p->y_dtype == FIX_DTYPE_F32,
-                   o_s, m_s, rstd_s, reinterpret_cast<int*>(base + ws.status), st));
+                   reinterpret_cast<const int*>(base + ws.safe), w, z, y,
+                   p->y_dtype == FIX_DTYPE_F32, o_s, m_s, rstd_s,
+                   reinterpret_cast<int*>(base + ws.status), st));
   } else {
     const size_t smem = simt_fwd_smem(d);
     if (!set_smem_limit(reinterpret_cast<const void*>(fwd_simt_kernel), (int)smem))
       return FIX_ERR_CUDA;
     fwd_simt_kernel<<<dim3(d.nchunks * 4, d.Hq), 256, smem, st>>>(
         d, chunks, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-        static_cast<const __nv_bfloat16*>(v), L, tot, static_cast<const __nv_bfloat16*>(w), y,
-        p->y_dtype == FIX_DTYPE_F32, o_s, m_s, rstd_s);
+        static_cast<const __nv_bfloat16*>(v), L, tot, static_cast<const __nv_bfloat16*>(w),
+        static_cast<const __nv_bfloat16*>(z), y, p->y_dtype == FIX_DTYPE_F32, o_s, m_s, rstd_s);
     FIX_TRY(launched());
   }
   return mark(p, FIX_STAGE_FWD_ATTN, 1, st);
 }
 
 fix_status fix_attn_bwd(const fix_attn_problem* p, const void* q, const void* k, const void* v,
-                        const float* g, const void* w, const void* dy, const float* o_s,
-                        const float* m_s, const float* rstd_s, void* dq, void* dk, void* dv,
-                        float* dg, void* dw, void* workspace, size_t ws_bytes, void* stream) {
+                        const float* g, const void* w, const void* z, const void* dy,
+                        const float* o_s, const float* m_s, const float* rstd_s, void* dq,
+                        void* dk, void* dv, float* dg, void* dw, void* dz, void* workspace,
+                        size_t ws_bytes, void* stream) {
   Dims d;
   FIX_TRY(make_dims(p, &d));
-  if (!q || !k || !v || !g || !w || !dy || !o_s || !m_s || !rstd_s || !dq || !dk || !dv || !dg ||
-      !dw || !workspace)
+  if (!q || !k || !v || !g || (!w && !d.no_norm) || !dy || !o_s || !m_s || !rstd_s || !dq || !dk ||
+      !dv || !dg || (!dw && !d.no_norm) || !workspace || (!z != !dz))
     return FIX_ERR_NULL;
-  for (const void* ptr : {q, k, v, (const void*)g, w, dy, (const void*)o_s, (const void*)m_s,
+  for (const void* ptr : {q, k, v, (const void*)g, w, z, dy, (const void*)o_s, (const void*)m_s,
                           (const void*)rstd_s, (const void*)dq, (const void*)dk, (const void*)dv,
-                          (const void*)dg, (const void*)dw, (const void*)workspace})
-    if (!aligned16(ptr)) return FIX_ERR_ALIGN;
+                          (const void*)dg, (const void*)dw, (const void*)dz,
+                          (const void*)workspace})
+    if (ptr && !aligned16(ptr)) return FIX_ERR_ALIGN;
   const SplitPlan sp = plan_split(p, d);
   const Ws ws = layout(d, true, sp);
   if (ws_bytes < ws.total) return FIX_ERR_WORKSPACE;
@@ -473,7 +483,7 @@ fix_status fix_attn_bwd(const fix_attn_problem* p, const void* q, const void* k,
   // status word, and (unless reused) the prefix pass's out-of-range flag
   if (cudaMemsetAsync(base + ws.status, 0, reuse ? 4 : 8, st) != cudaSuccess) return FIX_ERR_CUDA;
   if (d.N == 0) {
-    if (cudaMemsetAsync(dw, 0, (size_t)d.Dv * 2, st) != cudaSuccess) return FIX_ERR_CUDA;
+    if (dw && cudaMemsetAsync(dw, 0, (size_t)d.Dv * 2, st) != cudaSuccess) return FIX_ERR_CUDA;
     return FIX_OK;
   }
   FIX_TRY(mark(p, FIX_STAGE_BWD_PREFIX, 0, st));
@@ -498,9 +508,11 @@ fix_status fix_attn_bwd(const fix_attn_problem* p, const void* q, const void* k,
   const __nv_bfloat16* vb = static_cast<const __nv_bfloat16*>(v);
   FIX_TRY(mark(p, FIX_STAGE_BWD_PRE, 0, st));
   int* hmax = reinterpret_cast<int*>(base + ws.hmax);
+  float* delta = reinterpret_cast<float*>(base + ws.delta);
   bwd_pre_kernel<<<dim3(d.nchunks * kPreSplit, d.Hkv), 256, d.grp * sizeof(float), st>>>(
       d, chunks, qb, kb, vb, o_s, m_s, rstd_s, static_cast<const __nv_bfloat16*>(dy),
-      static_cast<const __nv_bfloat16*>(w), dow, A, dwp, tc ? hmax : nullptr,
+      static_cast<const __nv_bfloat16*>(w), static_cast<const __nv_bfloat16*>(z),
+      static_cast<__nv_bfloat16*>(dz), dow, A, delta, dwp, tc ? hmax : nullptr,
       tc ? reinterpret_cast<float*>(base + ws.ptt) : nullptr);
   FIX_TRY(launched());
   if (tc) {
@@ -510,9 +522,13 @@ fix_status fix_attn_bwd(const fix_attn_problem* p, const void* q, const void* k,
         dow, hmax, dot, domh, doml, dsafe);
     FIX_TRY(launched());
   }
-  dw_reduce_kernel<<<(d.Dv + 31) / 32, 1024, 0, st>>>(dwp, d.nchunks * kPreSplit * d.Hkv, d.Dv,
-                                                     static_cast<__nv_bfloat16*>(dw));
-  FIX_TRY(launched());
+  if (!d.no_norm) {
+    dw_reduce_kernel<<<(d.Dv + 31) / 32, 1024, 0, st>>>(dwp, d.nchunks * kPreSplit * d.Hkv, d.Dv,
+                                                       static_cast<__nv_bfloat16*>(dw));
+    FIX_TRY(launched());
+  } else if (dw && cudaMemsetAsync(dw, 0, (size_t)d.Dv * 2, st) != cudaSuccess) {
+    return FIX_ERR_CUDA;   // no weight without the norm: its gradient is zero
+  }
   FIX_TRY(mark(p, FIX_STAGE_BWD_PRE, 1, st));
   TcBwdArgs ta{};
   if (tc) {
@@ -537,6 +553,7 @@ fix_status fix_attn_bwd(const fix_attn_problem* p, const void* q, const void* k,
     ta.doml = doml;
     ta.A = A;
     ta.ptt = reinterpret_cast<const float*>(base + ws.ptt);
+    ta.delta = d.no_norm ? delta : nullptr;
     ta.badflag = badflag;
     ta.parts = reinterpret_cast<const Part*>(base + ws.parts);
     ta.cpart = reinterpret_cast<const int2*>(base + ws.cpart);
@@ -561,34 +578,43 @@ fix_status fix_attn_bwd(const fix_attn_problem* p, const void* q, const void* k,
   if (tc) FIX_TRY(tc_bwd(p, d, ta, 0, st));
   else
     dq_simt_kernel<<<dim3(d.nchunks * 4, d.Hq), 256, smq, st>>>(
-        d, chunks, qb, kb, vb, L, tot, m_s, dow, static_cast<__nv_bfloat16*>(dq), nullptr);
+        d, chunks, qb, kb, vb, L, tot, m_s, dow, d.no_norm ? delta : nullptr,
+        static_cast<__nv_bfloat16*>(dq), nullptr);
   FIX_TRY(launched());
   FIX_TRY(mark(p, FIX_STAGE_BWD_DQ, 1, st));
   FIX_TRY(mark(p, FIX_STAGE_BWD_DKV, 0, st));
   if (tc) FIX_TRY(tc_bwd(p, d, ta, 1, st));
   else
     dkv_simt_kernel<<<dim3(d.nchunks * 4, d.Hkv), 256, smkv, st>>>(
-        d, chunks, qb, kb, vb, L, tot, m_s, dow, A, static_cast<__nv_bfloat16*>(dk),
-        static_cast<__nv_bfloat16*>(dv), dG, nullptr);
+        d, chunks, qb, kb, vb, L, tot, m_s, dow, d.no_norm ? delta : nullptr, A,
+        static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv), dG, nullptr);
   FIX_TRY(launched());
   FIX_TRY(mark(p, FIX_STAGE_BWD_DKV, 1, st));
   FIX_TRY(mark(p, FIX_STAGE_BWD_FINISH, 0, st));
   if (tc) {
     FIX_TRY(tc_bwd(p, d, ta, 2, st));
     dq_simt_kernel<<<dim3(d.nchunks * 4, d.Hq), 256, smq, st>>>(
-        d, chunks, qb, kb, vb, L, tot, m_s, dow, static_cast<__nv_bfloat16*>(dq), gate);
+        d, chunks, qb, kb, vb, L, tot, m_s, dow, d.no_norm ? delta : nullptr,
+        static_cast<__nv_bfloat16*>(dq), gate);
     FIX_TRY(launched());
     dkv_simt_kernel<<<dim3(d.nchunks * 4, d.Hkv), 256, smkv, st>>>(
-        d, chunks, qb, kb, vb, L, tot, m_s, dow, A, static_cast<__nv_bfloat16*>(dk),
-        static_cast<__nv_bfloat16*>(dv), dG, gate);
+        d, chunks, qb, kb, vb, L, tot, m_s, dow, d.no_norm ? delta : nullptr, A,
+        static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv), dG, gate);
     FIX_TRY(launched());
   }
   FIX_TRY(mark(p, FIX_STAGE_BWD_FINISH, 1, st));
   FIX_TRY(mark(p, FIX_STAGE_BWD_DG, 0, st));
   chunk_total_kernel<<<dim3(d.nchunks, d.Hkv), 512, 0, st>>>(d, chunks, dG, dtot);
   FIX_TRY(launched());
-  reverse_cumsum_kernel<<<dim3(d.nchunks, d.Hkv), 512, 0, st>>>(d, chunks, dG, dtot, dg);
+  float* dgf = d.scalar_gate ? reinterpret_cast<float*>(base + ws.dgf) : dg;
+  reverse_cumsum_kernel<<<dim3(d.nchunks, d.Hkv), 512, 0, st>>>(d, chunks, dG, dtot, dgf);
   FIX_TRY(launched());
+  if (d.scalar_gate) {
+    // a scalar gate acts on every channel: its gradient is the channel sum
+    const long long rows = (long long)d.N * d.Hkv;
+    channel_sum_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(dgf, rows, d.Dv, dg);
+    FIX_TRY(launched());
+  }
   return mark(p, FIX_STAGE_BWD_DG, 1, st);
 }
 
@@ -612,8 +638,9 @@ int fix_attn_kernel_count(const fix_attn_problem* p, int backward) {
   // the prefix pass unless reused, the preprocess (2, or 3 with the
   // tensor-core operands), tensor-core dq / dk/dv / combine, the exact
   // kernels (2), the dG reverse cumsum (2)
-  return (reuse ? 0 : upA + 1) + upB + (tc ? 3 : 2) +
-         (tc ? tc_bwd_kernel_count(d, sp.nslots) : 0) + 2 + 2;
+  const bool has_dw = !d.no_norm;   // dw is optional only without the norm
+  return (reuse ? 0 : upA + 1) + upB + (tc ? 2 : 1) + (has_dw ? 1 : 0) +
+         (tc ? tc_bwd_kernel_count(d, sp.nslots) : 0) + 2 + 2 + (d.scalar_gate ? 1 : 0);
 }
 
 fix_status fix_attn_device_status(const void* workspace, void* stream) {

@@ -92,9 +92,19 @@ struct Dims {
   int nchunks;    // chunks over all sequences
   float scale;    // logit scale
   float eps;      // RMSNorm epsilon
+  int no_norm;    // FIX_FLAG_NO_NORM: y = o / l, no RMSNorm
+  int scalar_gate;  // FIX_FLAG_SCALAR_GATE: g is [N, Hkv]
 };
 
 __device__ __forceinline__ float bf2f(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+// The output gate's activation, swish(z) = z sigmoid(z), and its derivative
+// sigmoid(z) (1 + z (1 - sigmoid(z))).
+__device__ __forceinline__ float swish(float z) { return z / (1.0f + __expf(-z)); }
+__device__ __forceinline__ float swish_grad(float z) {
+  const float sg = 1.0f / (1.0f + __expf(-z));
+  return sg * (1.0f + z * (1.0f - sg));
+}
 __device__ __forceinline__ __nv_bfloat16 f2bf(float x) { return __float2bfloat16_rn(x); }
 
 __device__ __forceinline__ float warp_sum(float v) {

@@ -15,19 +15,22 @@ __global__ void prefix_kernel(Dims d, const Chunk* chunks, const float* g, const
                               float* tot, float* rho, float* hr, float* lvt, int* safe,
                               int* badflag, int* hmax);
 __global__ void chunk_total_kernel(Dims d, const Chunk* chunks, const float* x, float* tot);
+__global__ void channel_sum_kernel(const float* x, long long rows, int D, float* out);
 __global__ void reverse_cumsum_kernel(Dims d, const Chunk* chunks, const float* x,
                                       const float* tot, float* out);
 
 // fix_simt.cu
 __global__ void fwd_simt_kernel(Dims d, const Chunk* chunks, const __nv_bfloat16* q,
                                 const __nv_bfloat16* k, const __nv_bfloat16* v, const float* L,
-                                const float* tot, const __nv_bfloat16* w, void* y, int y_f32,
-                                float* o_s, float* m_s, float* rstd_s);
+                                const float* tot, const __nv_bfloat16* w,
+                                const __nv_bfloat16* z, void* y, int y_f32, float* o_s,
+                                float* m_s, float* rstd_s);
 __global__ void bwd_pre_kernel(Dims d, const Chunk* chunks, const __nv_bfloat16* q,
                                const __nv_bfloat16* k, const __nv_bfloat16* v, const float* o_s,
                                const float* m_s, const float* rstd_s, const __nv_bfloat16* dy,
-                               const __nv_bfloat16* w, float* do_ws, float* A, float* dwpart,
-                               int* hmax_g, float* ptt);
+                               const __nv_bfloat16* w, const __nv_bfloat16* z,
+                               __nv_bfloat16* dz, float* do_ws, float* A, float* delta,
+                               float* dwpart, int* hmax_g, float* ptt);
 __global__ void bwd_pre_ops_kernel(Dims d, const Chunk* chunks, const float* L, const float* rho,
                                    const float* hr, const int* safe, const float* do_ws,
                                    const int* hmax_g, uint16_t* dot, __nv_bfloat16* domh,
@@ -36,12 +39,12 @@ __global__ void dw_reduce_kernel(const float* parts, int nparts, int Dv, __nv_bf
 __global__ void dq_simt_kernel(Dims d, const Chunk* chunks, const __nv_bfloat16* q,
                                const __nv_bfloat16* k, const __nv_bfloat16* v, const float* L,
                                const float* tot, const float* m_s, const float* do_ws,
-                               __nv_bfloat16* dq, const int* gate);
+                               const float* delta, __nv_bfloat16* dq, const int* gate);
 __global__ void dkv_simt_kernel(Dims d, const Chunk* chunks, const __nv_bfloat16* q,
                                 const __nv_bfloat16* k, const __nv_bfloat16* v, const float* L,
                                 const float* tot, const float* m_s, const float* do_ws,
-                                const float* A, __nv_bfloat16* dk, __nv_bfloat16* dv, float* dG,
-                                const int* gate);
+                                const float* delta, const float* A, __nv_bfloat16* dk,
+                                __nv_bfloat16* dv, float* dG, const int* gate);
 
 // Tensor-core (tcgen05) kernels.
 // Raises a kernel's dynamic shared-memory limit to at least `bytes` on the
@@ -55,8 +58,8 @@ fix_status tc_fwd(const Dims& d, const Chunk* chunks, const int* order, const vo
                   const __nv_bfloat16* vml, const void* v,
                   const float* L, const float* tot, const float* rho, const float* hr,
                   const float* lvt, const int* safe,
-                  const void* w, void* y, bool y_f32, float* o_s, float* m_s, float* rstd_s,
-                  int* status, cudaStream_t st);
+                  const void* w, const void* z, void* y, bool y_f32, float* o_s, float* m_s,
+                  float* rstd_s, int* status, cudaStream_t st);
 int tc_fwd_kernel_count(const Dims& d);
 #ifdef FIX_TEST_HOOKS
 // Test builds (libfixattn_test.so) only: whether the tensor-core forward runs
@@ -89,6 +92,7 @@ struct TcBwdArgs {
   const __nv_bfloat16* doml;
   const float* A;
   const float* ptt;      // P_tt per (token, q head), from the preprocess
+  const float* delta;    // without the norm: sum_c do_t o_t per (token, q head); else NULL
   const int* badflag;
   const Part* parts;
   const int2* cpart;

@@ -56,17 +56,18 @@ fix_status scratch_on_current_device(void** out) {
 
 extern "C" fix_status fix_attn_fwd_noalloc(const fix_attn_problem* p, const void* q,
                                            const void* k, const void* v, const float* g,
-                                           const void* o_norm_weight, void* y, float* o_saved,
-                                           float* m_saved, float* rstd_saved, void* stream) {
+                                           const void* o_norm_weight, const void* o_gate,
+                                           void* y, float* o_saved, float* m_saved,
+                                           float* rstd_saved, void* stream) {
   const size_t need = fix_attn_workspace_bytes(p, 0);
   if (need == 0)  // invalid problem: let the forward report the exact reason
-    return fix_attn_fwd(p, q, k, v, g, o_norm_weight, y, o_saved, m_saved, rstd_saved, nullptr,
-                        0, stream);
+    return fix_attn_fwd(p, q, k, v, g, o_norm_weight, o_gate, y, o_saved, m_saved, rstd_saved,
+                        nullptr, 0, stream);
   if (need > FIX_NOALLOC_MAX_WORKSPACE_BYTES) return FIX_ERR_WORKSPACE;
   void* ws = nullptr;
   const fix_status s = scratch_on_current_device(&ws);
   if (s != FIX_OK) return s;
-  return fix_attn_fwd(p, q, k, v, g, o_norm_weight, y, o_saved, m_saved, rstd_saved, ws,
+  return fix_attn_fwd(p, q, k, v, g, o_norm_weight, o_gate, y, o_saved, m_saved, rstd_saved, ws,
                       FIX_NOALLOC_MAX_WORKSPACE_BYTES, stream);
 }
 

@@ -73,9 +73,12 @@ __global__ void __launch_bounds__(kPrefixThreads) prefix_kernel(
   float acc = 0.f, lmin = INFINITY, lmax = -INFINITY;
   bool nonpos = true;
   // g and v in one round trip (v only on the tensor-core path)
+  // a scalar gate ([N, Hkv]) is the same for every channel of the token
+  const size_t gbase = d.scalar_gate ? (size_t)ch.tok0 * d.Hkv + kv : base;
+  const size_t grs = d.scalar_gate ? (size_t)d.Hkv : rs;
 #pragma unroll
   for (int u = 0; u < kMaxRows; ++u)
-    if (u < nr) lv[u] = g[base + (size_t)(r0 + u) * rs];
+    if (u < nr) lv[u] = g[gbase + (size_t)(r0 + u) * grs];
   if (vt) {
 #pragma unroll
     for (int u = 0; u < kMaxRows; ++u)
@@ -182,6 +185,19 @@ __global__ void __launch_bounds__(kPrefixThreads) chunk_total_kernel(Dims d,
     for (int q = 0; q < groups; ++q) t += part[q * Dv + c];
     tot[((size_t)ci * d.Hkv + kv) * Dv + c] = t;
   }
+}
+
+// out[r] = sum of the D values of row r (a warp per row, fixed order).
+__global__ void __launch_bounds__(256) channel_sum_kernel(const float* __restrict__ x,
+                                                          long long rows, int D,
+                                                          float* __restrict__ out) {
+  const long long r = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (r >= rows) return;
+  float s = 0.f;
+  for (int c = lane; c < D; c += 32) s += x[r * D + c];
+  s = warp_sum(s);
+  if (lane == 0) out[r] = s;
 }
 
 __global__ void __launch_bounds__(kPrefixThreads) reverse_cumsum_kernel(

@@ -26,8 +26,9 @@ __global__ void __launch_bounds__(256) fwd_simt_kernel(
     Dims d, const Chunk* __restrict__ chunks, const __nv_bfloat16* __restrict__ q,
     const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
     const float* __restrict__ L, const float* __restrict__ tot,
-    const __nv_bfloat16* __restrict__ w, void* __restrict__ y, int y_f32,
-    float* __restrict__ o_s, float* __restrict__ m_s, float* __restrict__ rstd_s) {
+    const __nv_bfloat16* __restrict__ w, const __nv_bfloat16* __restrict__ z,
+    void* __restrict__ y, int y_f32, float* __restrict__ o_s, float* __restrict__ m_s,
+    float* __restrict__ rstd_s) {
   extern __shared__ float sm[];
   const int Dk = d.Dk, Dv = d.Dv;
   float* sQ = sm;                       // [ST][Dk]
@@ -56,10 +57,11 @@ __global__ void __launch_bounds__(256) fwd_simt_kernel(
     sLq[e] = r < nrows ? L[(size_t)(ch.tok0 + r0 + r) * vrs + (size_t)kv * Dv + c] : 0.f;
   }
 
-  float o[4][4], mrow[4], delta[4];
+  float o[4][4], mrow[4], lrow[4], delta[4];
 #pragma unroll
   for (int a = 0; a < 4; ++a) {
     mrow[a] = -INFINITY;
+    lrow[a] = 0.f;
     delta[a] = 0.f;
 #pragma unroll
     for (int u = 0; u < 4; ++u) o[a][u] = 0.f;
@@ -111,6 +113,7 @@ __global__ void __launch_bounds__(256) fwd_simt_kernel(
           lq[u] = c < Dv ? sLq[r * Dv + c] + delta[u] : 0.f;
         }
         const float p = valid ? expf(sv - mnew) : 0.f;
+        lrow[rr] = lrow[rr] * alpha + warp_sum(p);   // softmax denominator (no norm)
         for (int s = 0; s < nk; ++s) {
           const float ps = __shfl_sync(FULL, p, s);
           if (ps == 0.f) continue;  // masked key: its factor may be out of range
@@ -132,21 +135,24 @@ __global__ void __launch_bounds__(256) fwd_simt_kernel(
 #pragma unroll
     for (int u = 0; u < 4; ++u) ss += o[rr][u] * o[rr][u];
     ss = warp_sum(ss);
-    const float rstd = 1.f / sqrtf(ss / (float)Dv + d.eps);
+    // RMSNorm, or (no norm) the softmax denominator; the saved tensors are
+    // then o / l, the log-sum-exp and ones
+    const float rstd = d.no_norm ? 1.f / lrow[rr] : 1.f / sqrtf(ss / (float)Dv + d.eps);
     const size_t tok = (size_t)(ch.tok0 + r0 + r);
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int c = lane + 32 * u;
       if (c >= Dv) continue;
       const size_t a = tok * ors + (size_t)h * Dv + c;
-      const float yv = o[rr][u] * rstd * bf2f(w[c]);
+      float yv = o[rr][u] * rstd * (d.no_norm ? 1.f : bf2f(w[c]));
+      if (z) yv *= swish(bf2f(z[a]));
       if (y_f32) reinterpret_cast<float*>(y)[a] = yv;
       else reinterpret_cast<__nv_bfloat16*>(y)[a] = f2bf(yv);
-      if (o_s) o_s[a] = o[rr][u];
+      if (o_s) o_s[a] = d.no_norm ? o[rr][u] * rstd : o[rr][u];
     }
     if (lane == 0 && m_s) {
-      m_s[tok * d.Hq + h] = mrow[rr];
-      rstd_s[tok * d.Hq + h] = rstd;
+      m_s[tok * d.Hq + h] = d.no_norm ? mrow[rr] + logf(lrow[rr]) : mrow[rr];
+      rstd_s[tok * d.Hq + h] = d.no_norm ? 1.f : rstd;
     }
   }
 }
@@ -174,8 +180,10 @@ __global__ void __launch_bounds__(kPreWarps * 32) bwd_pre_kernel(
     const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
     const float* __restrict__ o_s, const float* __restrict__ m_s,
     const float* __restrict__ rstd_s, const __nv_bfloat16* __restrict__ dy,
-    const __nv_bfloat16* __restrict__ w, float* __restrict__ do_ws, float* __restrict__ A,
-    float* __restrict__ dwpart, int* __restrict__ hmax_g, float* __restrict__ ptt_out) {
+    const __nv_bfloat16* __restrict__ w, const __nv_bfloat16* __restrict__ z,
+    __nv_bfloat16* __restrict__ dz, float* __restrict__ do_ws, float* __restrict__ A,
+    float* __restrict__ delta_out, float* __restrict__ dwpart, int* __restrict__ hmax_g,
+    float* __restrict__ ptt_out) {
   __shared__ float red[kPreWarps][128];
   extern __shared__ float hmax[];   // [grp] max |do| per head
   const int Dv = d.Dv, Dk = d.Dk, kv = blockIdx.y;
@@ -188,7 +196,7 @@ __global__ void __launch_bounds__(kPreWarps * 32) bwd_pre_kernel(
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
     const int c = lane + 32 * u;
-    wv[u] = c < Dv ? bf2f(w[c]) : 0.f;
+    wv[u] = (c < Dv && w) ? bf2f(w[c]) : 0.f;
     dwl[u] = 0.f;
   }
   const size_t ors = (size_t)d.Hq * Dv, vrs = (size_t)d.Hkv * Dv;
@@ -219,24 +227,40 @@ __global__ void __launch_bounds__(kPreWarps * 32) bwd_pre_kernel(
       }
       const float ptt = expf(warp_sum(sdot) * d.scale - mt);
       if (ptt_out && lane == 0) ptt_out[t * d.Hq + h] = ptt;
+      // output gate: y = u swish(z) with u the normed (or, without the norm,
+      // the averaged) output; du = dy swish(z), dz = dy u swish'(z)
+      float du[4], zv[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int c = lane + 32 * u;
+        zv[u] = (z && c < Dv) ? bf2f(z[t * ors + (size_t)h * Dv + c]) : 0.f;
+        du[u] = z ? dyv[u] * swish(zv[u]) : dyv[u];
+      }
       float dn[4], n[4], dot_ = 0.f;
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        n[u] = ov[u] * rs_;
-        dn[u] = dyv[u] * wv[u];
+        n[u] = d.no_norm ? ov[u] : ov[u] * rs_;
+        dn[u] = d.no_norm ? du[u] : du[u] * wv[u];
         dot_ += dn[u] * n[u];
-        dwl[u] += dyv[u] * n[u];
+        if (!d.no_norm) dwl[u] += du[u] * n[u];
       }
       dot_ = warp_sum(dot_) / (float)Dv;
+      // without the norm: do = du, and sum_c do o (the softmax-denominator
+      // term of dS) goes to the dq and dk/dv kernels
+      if (d.no_norm && lane == 0) delta_out[t * d.Hq + h] = dot_ * (float)Dv;
       float mx = 0.f;
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int c = lane + 32 * u;
         if (c >= Dv) continue;
-        const float dov = rs_ * (dn[u] - n[u] * dot_);
+        const float dov = d.no_norm ? du[u] : rs_ * (dn[u] - n[u] * dot_);
         do_ws[t * ors + (size_t)h * Dv + c] = dov;
         acc[u] += dov * (ov[u] - ptt * vr[u]);
         mx = fmaxf(mx, fabsf(dov));
+        if (z) {
+          const float uo = d.no_norm ? ov[u] : n[u] * wv[u];
+          dz[t * ors + (size_t)h * Dv + c] = f2bf(dyv[u] * uo * swish_grad(zv[u]));
+        }
       }
       if (hmax_g) {
         mx = warp_max(mx);
@@ -377,7 +401,8 @@ __global__ void __launch_bounds__(256) dq_simt_kernel(
     const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
     const float* __restrict__ L, const float* __restrict__ tot,
     const float* __restrict__ m_s, const float* __restrict__ do_ws,
-    __nv_bfloat16* __restrict__ dq, const int* __restrict__ gate) {
+    const float* __restrict__ delta_in, __nv_bfloat16* __restrict__ dq,
+    const int* __restrict__ gate) {
   if (gate && *gate == 0) return;  // the tensor-core kernel handles this problem
   extern __shared__ float sm[];
   const int Dk = d.Dk, Dv = d.Dv;
@@ -459,6 +484,8 @@ __global__ void __launch_bounds__(256) dq_simt_kernel(
               dp += sDo[r * Dv + c] *
                     expf(sLq[r * Dv + c] + sDelta[c] - sLk[lane * (Dv + 1) + c]) *
                     sV[lane * (Dv + 1) + c];
+            // without the norm, dS carries the softmax-denominator term
+            if (delta_in) dp -= delta_in[(size_t)(ch.tok0 + r0 + r) * d.Hq + h];
             ds = p * dp;
           }
         }
@@ -499,8 +526,9 @@ __global__ void __launch_bounds__(256) dkv_simt_kernel(
     const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
     const float* __restrict__ L, const float* __restrict__ tot,
     const float* __restrict__ m_s, const float* __restrict__ do_ws,
-    const float* __restrict__ A, __nv_bfloat16* __restrict__ dk,
-    __nv_bfloat16* __restrict__ dv, float* __restrict__ dG, const int* __restrict__ gate) {
+    const float* __restrict__ delta_in, const float* __restrict__ A,
+    __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv, float* __restrict__ dG,
+    const int* __restrict__ gate) {
   if (gate && *gate == 0) return;  // the tensor-core kernel handles this problem
   extern __shared__ float sm[];
   const int Dk = d.Dk, Dv = d.Dv;
@@ -589,6 +617,8 @@ __global__ void __launch_bounds__(256) dkv_simt_kernel(
               if (c < Dv) dp += sDo[r * Dv + c] * dc[u] * vr[a][u];
             }
             dp = warp_sum(dp);
+            // without the norm, dS carries the softmax-denominator term
+            if (delta_in) dp -= delta_in[(size_t)(qc.tok0 + qt + r) * d.Hq + h];
             const float ds = p * dp;
             const bool same = spos == tpos;
 #pragma unroll

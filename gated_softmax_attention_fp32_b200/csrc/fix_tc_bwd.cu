@@ -69,6 +69,7 @@ struct Params {
   const __nv_bfloat16* doml;
   const float* A;
   const float* ptt;         // P_tt per (token, q head), from the preprocess
+  const float* delta;       // without the norm: sum_c do o per (token, q head); else NULL
   const int* badflag;
   const Part* parts;        // dk/dv work split (schedule kernel)
   const int2* cpart;
@@ -287,6 +288,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const size_t tok = (size_t)ch.tok0 + (size_t)(row_ok ? r : 0);
     const float moff = P.m_s[tok * d.Hq + h] * LOG2E;
     const float c1 = d.scale * LOG2E;
+    // without the norm: dS = P (dP - sum_c do o) (the softmax denominator)
+    const float dl = P.delta ? P.delta[tok * d.Hq + h] : 0.f;
     bool ok = true;
     for (int it = 0; it < nblk; ++it) {
       if (!__all_sync(0xffffffffu, mbar_wait(&bar->s_full, it & 1, ctl))) { ok = false; break; }
@@ -304,7 +307,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int e = 0; e < 32; e += 2) {
             const float p0 = ex2(__uint_as_float(xs[e]) * c1 - moff);
             const float p1 = ex2(__uint_as_float(xs[e + 1]) * c1 - moff);
-            pk[e >> 1] = pack_bf16(p0 * __uint_as_float(xp[e]), p1 * __uint_as_float(xp[e + 1]));
+            pk[e >> 1] = pack_bf16(p0 * (__uint_as_float(xp[e]) - dl), p1 * (__uint_as_float(xp[e + 1]) - dl));
           }
         } else {
 #pragma unroll
@@ -312,7 +315,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int key = c4 * 32 + e;
             const float p0 = key <= r ? ex2(__uint_as_float(xs[e]) * c1 - moff) : 0.f;
             const float p1 = key + 1 <= r ? ex2(__uint_as_float(xs[e + 1]) * c1 - moff) : 0.f;
-            pk[e >> 1] = pack_bf16(p0 * __uint_as_float(xp[e]), p1 * __uint_as_float(xp[e + 1]));
+            pk[e >> 1] = pack_bf16(p0 * (__uint_as_float(xp[e]) - dl), p1 * (__uint_as_float(xp[e + 1]) - dl));
           }
         }
         tmem_st16(lane_base + kColS + c4 * 16, pk);
@@ -434,7 +437,8 @@ struct KvLayout {
   static constexpr int kStageDiag = BQ * (DK + 2 * DV) * 2; // bytes per diagonal stage
   static constexpr int kM = kQ + kQStages * kStageOff;      // stages x [64] f32 row max
   static_assert(2 * kStageDiag <= kQStages * kStageOff, "diagonal stages must fit the region");
-  static constexpr int kBars = kM + kQStages * BQ * 4;
+  static constexpr int kDl = kM + kQStages * BQ * 4;        // stages x [64] f32 sum do o
+  static constexpr int kBars = kDl + kQStages * BQ * 4;
   static constexpr int kTmem = kBars + (int)sizeof(KvBars);
   static constexpr int kAbort = kTmem + 4;
   static constexpr int kAlloc = kAbort + 4 + 1024;
@@ -496,6 +500,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto sX = [&](int st) { return sQ(st) + BQ * DK * 2; };
   auto sXl = [&](int st) { return sX(st) + BQ * DV * 2; };
   float* sM = reinterpret_cast<float*>(smem + Lay::kM);
+  float* sDl = reinterpret_cast<float*>(smem + Lay::kDl);
   KvBars* bar = reinterpret_cast<KvBars*>(smem + Lay::kBars);
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(smem + Lay::kTmem);
   volatile int* sAbort = reinterpret_cast<volatile int*>(smem + Lay::kAbort);
@@ -677,6 +682,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       const float* mrow = sM + st * BQ;
+      const float* dlrow = sDl + st * BQ;     // zeros with the norm
       const bool full = !dmode && qlen == BQ;
       const int lo = dmode ? s - t.half * BQ : 0;   // first valid query column
       // two halves of 32 query columns; a half's packed P and dS go over
@@ -695,7 +701,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float p0 = ex2(__uint_as_float(xs[e]) * c1 - mrow[32 * h + e] * LOG2E);
             const float p1 = ex2(__uint_as_float(xs[e + 1]) * c1 - mrow[32 * h + e + 1] * LOG2E);
             ph[e >> 1] = cta_f16 ? pack_f16(p0, p1) : pack_bf16(p0, p1);
-            pd[e >> 1] = pack_bf16(p0 * __uint_as_float(xp[e]), p1 * __uint_as_float(xp[e + 1]));
+            pd[e >> 1] = pack_bf16(p0 * (__uint_as_float(xp[e]) - dlrow[32 * h + e]),
+                                   p1 * (__uint_as_float(xp[e + 1]) - dlrow[32 * h + e + 1]));
           }
         } else {
           // diagonal tile (queries t >= s; the s = t pair stays out of dv) or
@@ -718,7 +725,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             } else {
               ph[e >> 1] = cta_f16 ? pack_f16(pv[0], pv[1]) : pack_bf16(pv[0], pv[1]);
             }
-            pd[e >> 1] = pack_bf16(p[0] * __uint_as_float(xp[e]), p[1] * __uint_as_float(xp[e + 1]));
+            pd[e >> 1] = pack_bf16(p[0] * (__uint_as_float(xp[e]) - dlrow[32 * h + e]),
+                                   p[1] * (__uint_as_float(xp[e + 1]) - dlrow[32 * h + e + 1]));
           }
         }
         tmem_st16(lane_base + col_s(b) + 16 * h, ph);
@@ -816,6 +824,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // what a tile needs from global memory besides its totals
       struct Pre {
         float m;     // row maximum of query row dt (dt < 64)
+        float dl;    // its sum_c do o (without the norm; else 0)
         int qlen;    // rows of the tile
         int in_f16;  // storage type of its dOt
       };
@@ -823,7 +832,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Chunk qc = P.chunks[first + u.i];
         Pre r;
         r.qlen = min(BQ, qc.len - u.half * BQ);
-        r.m = dt < r.qlen ? P.m_s[((size_t)qc.tok0 + u.half * BQ + dt) * d.Hq + kv * d.grp + u.hh] : 0.f;
+        const size_t ri = ((size_t)qc.tok0 + u.half * BQ + dt) * d.Hq + kv * d.grp + u.hh;
+        r.m = dt < r.qlen ? P.m_s[ri] : 0.f;
+        r.dl = (dt < r.qlen && P.delta) ? P.delta[ri] : 0.f;
         r.in_f16 = dmode ? 0 : P.dsafe[(size_t)(first + u.i) * d.Hq + kv * d.grp + u.hh];
         return r;
       };
@@ -872,7 +883,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           fence_proxy_async_smem();
         }
-        if (dt < BQ) sM[st * BQ + dt] = cur.m;
+        if (dt < BQ) {
+          sM[st * BQ + dt] = cur.m;
+          sDl[st * BQ + dt] = cur.dl;
+        }
         mbar_arrive(&bar->x_ready[st]);
         // advance to tile n + 1
         if (!dmode) {
@@ -1101,6 +1115,7 @@ fix_status tc_bwd(const fix_attn_problem*, const Dims& d, const TcBwdArgs& a, in
   prm.doml = a.doml;
   prm.A = a.A;
   prm.ptt = a.ptt;
+  prm.delta = a.delta;
   prm.badflag = a.badflag;
   prm.parts = a.parts;
   prm.cpart = a.cpart;

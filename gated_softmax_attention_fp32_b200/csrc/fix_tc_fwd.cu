@@ -95,8 +95,8 @@ struct Layout {
   static constexpr int kF = kVl + BN * DV * 2;           // [2][DV] f32 fold factors
   static constexpr int kBad = kF + 2 * DV * 4;           // [2][DV] int out-of-range flags
   static constexpr int kAnyBad = kBad + 2 * DV * 4;      // [2] int
-  static constexpr int kRows = kAnyBad + 16;             // [2][3][BM] f32: alpha, P_tt, m
-  static constexpr int kEpiT = kRows + 2 * 3 * BM * 4;   // [4][32][33] f32 transposes
+  static constexpr int kRows = kAnyBad + 16;             // [2][4][BM] f32: alpha, P_tt, m, l
+  static constexpr int kEpiT = kRows + 2 * 4 * BM * 4;   // [4][32][33] f32 transposes
   static constexpr int kEpiW = kEpiT + 4 * 32 * 33 * 4;  // [DV] f32 w
   static constexpr int kEpiRho = kEpiW + DV * 4;         // [DV] f32 rho of the epilogue's tile
   static constexpr int kEpiBad = kEpiRho + DV * 4;       // [DV] int
@@ -122,7 +122,8 @@ struct Params {
   const float* hr;
   const float* lvt;
   const int* safe;
-  const __nv_bfloat16* w;
+  const __nv_bfloat16* w;     // NULL allowed without the norm
+  const __nv_bfloat16* z;     // output gate or NULL
   void* y;
   int y_f32;
   float* o_s;
@@ -243,7 +244,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (warp == 1) tmem_alloc(sTmem, kTmemCols);
   if (tid >= 384 && tid - 384 < DV)
-    reinterpret_cast<float*>(smem + Lay::kEpiW)[tid - 384] = bf2f(P.w[tid - 384]);
+    reinterpret_cast<float*>(smem + Lay::kEpiW)[tid - 384] =
+        (P.w && !d.no_norm) ? bf2f(P.w[tid - 384]) : 1.f;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -400,6 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int tb = nt & 1, use = nt >> 1;
       const uint32_t acol = lane_base + 256u + (uint32_t)(tb * DV);
       float m_used = -INFINITY, m_true = -INFINITY, s_diag = 0.f;
+      float l_used = 0.f;   // without the norm: sum of P relative to m_used
       for (int it = 0; it < x.nblk; ++it) {
         const bool diag = it == x.nblk - 1;
         const int b = g & 1;
@@ -455,7 +458,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_st32(acol + cc * 32, xa);
           }
           tmem_wait_st();
-          if (rescale) m_used = m_true;
+          if (rescale) {
+            m_used = m_true;
+            l_used *= a_r;
+          }
         }
         if (diag && x.nblk == 1) {
           // chunk 0: the diagonal MMAs accumulate into A, which starts at
@@ -515,10 +521,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t xs[32], pk[16];
             tmem_ld32(sbase + c4 * 32, xs);
             tmem_wait_ld();
+            float ls = 0.f;
 #pragma unroll
-            for (int e = 0; e < 32; e += 2)
-              pk[e >> 1] = pack_f16(ex2(__uint_as_float(xs[e]) * c1 - moff),
-                                    ex2(__uint_as_float(xs[e + 1]) * c1 - moff));
+            for (int e = 0; e < 32; e += 2) {
+              const float p0 = ex2(__uint_as_float(xs[e]) * c1 - moff);
+              const float p1 = ex2(__uint_as_float(xs[e + 1]) * c1 - moff);
+              ls += p0 + p1;
+              pk[e >> 1] = pack_f16(p0, p1);
+            }
+            if (d.no_norm) l_used += ls;
             tmem_st16(sbase + c4 * 16, pk);
           }
         } else {
@@ -538,6 +549,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               const int key = c4 * 32 + e;
               const float p0 = key < r ? ex2(__uint_as_float(xs[e]) * c1 - moff) : 0.f;
               const float p1 = key + 1 < r ? ex2(__uint_as_float(xs[e + 1]) * c1 - moff) : 0.f;
+              if (d.no_norm) l_used += p0 + p1;
               ph[e >> 1] = pack_bf16(p0, p1);
               const float h0 = __uint_as_float(ph[e >> 1] << 16);
               const float h1 = __uint_as_float(ph[e >> 1] & 0xFFFF0000u);
@@ -569,10 +581,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       // per-row results of the tile for its epilogue
       if (use >= 1 && !__all_sync(0xffffffffu, mbar_wait(&bar->rows_free[tb], (use - 1) & 1, ctl))) { ok = false; break; }
-      float* rows = sRows + tb * 3 * BM;
-      rows[r] = ex2((m_used - m_true) * LOG2E);                    // alpha
-      rows[BM + r] = ex2((s_diag * d.scale - m_true) * LOG2E);    // P_tt
+      float* rows = sRows + tb * 4 * BM;
+      const float alpha = ex2((m_used - m_true) * LOG2E);
+      const float ptt = ex2((s_diag * d.scale - m_true) * LOG2E);
+      rows[r] = alpha;
+      rows[BM + r] = ptt;                                          // P_tt
       rows[2 * BM + r] = m_true;
+      rows[3 * BM + r] = alpha * l_used + ptt;                     // l (no norm)
       mbar_arrive(&bar->rows_ready[tb]);
       ++nt;
     }
@@ -725,7 +740,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      const float* rows = sRows + tb * 3 * BM;
+      const float* rows = sRows + tb * 4 * BM;
       const uint32_t acol = lane_base + 256u + (uint32_t)(tb * DV);
       const float* Lg = P.L + (size_t)x.kv * DV;
       const __nv_bfloat16* vg = P.v + (size_t)x.kv * DV;
@@ -771,9 +786,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             ss[q] += val * val;
           }
         }
+        // the RMSNorm, or without it the softmax denominator: y = o / l; the
+        // saved tensors are then o / l, the log-sum-exp and ones
         float rstd[kR];
 #pragma unroll
-        for (int q = 0; q < kR; ++q) rstd[q] = 1.0f / sqrtf(warp_sum(ss[q]) / (float)DV + d.eps);
+        for (int q = 0; q < kR; ++q)
+          rstd[q] = d.no_norm ? 1.0f / rows[3 * BM + rbase + q]
+                              : 1.0f / sqrtf(warp_sum(ss[q]) / (float)DV + d.eps);
 #pragma unroll
         for (int q = 0; q < kR; ++q) {
           const int rr = rbase + q;
@@ -782,10 +801,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int u = 0; u < kU; ++u) {
             const int c = u * 32 + lane;
-            const float yv = o[q][u] * rstd[q] * sW[c];
+            float yv = o[q][u] * rstd[q] * sW[c];
+            if (P.z) yv *= swish(bf2f(P.z[a0 + c]));
             if (yf) yf[a0 + c] = yv;
             else yb[a0 + c] = f2bf(yv);
-            if (P.o_s) P.o_s[a0 + c] = o[q][u];
+            if (P.o_s) P.o_s[a0 + c] = d.no_norm ? o[q][u] * rstd[q] : o[q][u];
           }
         }
         if (P.o_s && lane < kR && rbase + lane < x.len) {
@@ -793,8 +813,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int q = 1; q < kR; ++q) rs = lane == q ? rstd[q] : rs;
           const size_t tk = (size_t)x.tok0 + rbase + lane;
-          P.m_s[tk * d.Hq + x.h] = rows[2 * BM + rbase + lane];
-          P.rstd_s[tk * d.Hq + x.h] = rs;
+          const float mt = rows[2 * BM + rbase + lane];
+          P.m_s[tk * d.Hq + x.h] = d.no_norm ? mt + logf(rows[3 * BM + rbase + lane]) : mt;
+          P.rstd_s[tk * d.Hq + x.h] = d.no_norm ? 1.f : rs;
         }
       }
       tc_fence_before();
@@ -886,8 +907,8 @@ fix_status tc_fwd(const Dims& d, const Chunk* chunks, const int* order, const vo
                   const __nv_bfloat16* vml, const void* v,
                   const float* L, const float* tot, const float* rho, const float* hr,
                   const float* lvt, const int* safe,
-                  const void* w, void* y, bool y_f32, float* o_s, float* m_s, float* rstd_s,
-                  int* status, cudaStream_t st) {
+                  const void* w, const void* z, void* y, bool y_f32, float* o_s, float* m_s,
+                  float* rstd_s, int* status, cudaStream_t st) {
   tcf::Params prm{};
   prm.d = d;
   prm.chunks = chunks;
@@ -905,6 +926,7 @@ fix_status tc_fwd(const Dims& d, const Chunk* chunks, const int* order, const vo
   prm.lvt = lvt;
   prm.safe = safe;
   prm.w = static_cast<const __nv_bfloat16*>(w);
+  prm.z = static_cast<const __nv_bfloat16*>(z);
   prm.y = y;
   prm.y_f32 = y_f32 ? 1 : 0;
   prm.o_s = o_s;

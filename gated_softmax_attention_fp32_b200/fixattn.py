@@ -29,6 +29,8 @@ EXPORTS = ("fix_attn_workspace_bytes", "fix_attn_fwd", "fix_attn_bwd", "fix_attn
            "fix_attn_noalloc_device_status")
 NOALLOC_MAX_WORKSPACE_BYTES = 16 * 1024 * 1024
 FIX_FLAG_REUSE_FWD_WORKSPACE = 1
+FIX_FLAG_NO_NORM = 2
+FIX_FLAG_SCALAR_GATE = 4
 STAGES = ("fwd_prefix", "fwd_attn", "bwd_prefix", "bwd_pre", "bwd_dq", "bwd_dkv", "bwd_dg",
           "bwd_finish")
 
@@ -66,11 +68,11 @@ def load():
     vp, sz = ctypes.c_void_p, ctypes.c_size_t
     lib.fix_attn_workspace_bytes.argtypes = [P, ctypes.c_int]
     lib.fix_attn_workspace_bytes.restype = sz
-    lib.fix_attn_fwd.argtypes = [P] + [vp] * 10 + [sz, vp]
+    lib.fix_attn_fwd.argtypes = [P] + [vp] * 11 + [sz, vp]
     lib.fix_attn_fwd.restype = ctypes.c_int
-    lib.fix_attn_bwd.argtypes = [P] + [vp] * 15 + [sz, vp]
+    lib.fix_attn_bwd.argtypes = [P] + [vp] * 17 + [sz, vp]
     lib.fix_attn_bwd.restype = ctypes.c_int
-    lib.fix_attn_fwd_noalloc.argtypes = [P] + [vp] * 9 + [vp]
+    lib.fix_attn_fwd_noalloc.argtypes = [P] + [vp] * 10 + [vp]
     lib.fix_attn_fwd_noalloc.restype = ctypes.c_int
     lib.fix_attn_device_status.argtypes = [vp, vp]
     lib.fix_attn_device_status.restype = ctypes.c_int
@@ -93,11 +95,14 @@ def _ptr(t: Optional[torch.Tensor]):
 
 
 def make_problem(q, k, v, cu_seqlens=None, cu_seqlens_host=None, scale=None, eps=1e-6,
-                 y_dtype=torch.bfloat16, algo="auto", events=None):
+                 y_dtype=torch.bfloat16, algo="auto", events=None, o_norm=True,
+                 scalar_gate=False):
     """Build the C problem descriptor from [B,T,H,D] tensors.  Returns
     (Problem, keepalive) where keepalive holds the host cu_seqlens tensor and
     the event-handle array.  ``events``: optional list of 2*len(STAGES)
-    ``torch.cuda.Event(enable_timing=True)`` recorded around each stage."""
+    ``torch.cuda.Event(enable_timing=True)`` recorded around each stage.
+    ``o_norm=False`` sets FIX_FLAG_NO_NORM, ``scalar_gate`` (g of shape
+    [B,T,Hkv]) FIX_FLAG_SCALAR_GATE."""
     B, T, Hq, Dk = q.shape
     Hkv, Dv = v.shape[2], v.shape[3]
     p = Problem()
@@ -105,7 +110,7 @@ def make_problem(q, k, v, cu_seqlens=None, cu_seqlens_host=None, scale=None, eps
     p.head_dim_k, p.head_dim_v = Dk, Dv
     p.y_dtype = 1 if y_dtype == torch.float32 else 0
     p.algo = ALGOS[algo]
-    p.flags = 0
+    p.flags = (0 if o_norm else FIX_FLAG_NO_NORM) | (FIX_FLAG_SCALAR_GATE if scalar_gate else 0)
     p.scale = float(scale) if scale is not None else 0.0
     p.eps = float(eps)
     keep = None
@@ -142,11 +147,14 @@ def _stream(stream):
 
 def fix_attn_fwd(q, k, v, g, o_norm_weight, cu_seqlens=None, cu_seqlens_host=None, scale=None,
                  eps=1e-6, y_dtype=torch.bfloat16, save=True, algo="auto", workspace=None,
-                 out=None, stream=None, events=None):
-    """Forward.  Returns (y, saved) with saved = (o, m, rstd) or None."""
+                 out=None, stream=None, events=None, o_gate=None, o_norm=True):
+    """Forward.  Returns (y, saved) with saved = (o, m, rstd) or None.  g of
+    shape [B,T,Hkv] is a scalar gate; ``o_gate`` [B,T,Hq,Dv] bf16 gates the
+    output with swish; ``o_norm=False`` drops the RMSNorm (o_norm_weight may
+    then be None)."""
     lib = load()
     p, keep = make_problem(q, k, v, cu_seqlens, cu_seqlens_host, scale, eps, y_dtype, algo,
-                           events)
+                           events, o_norm, g.dim() == 3)
     B, T, Hq, _ = q.shape
     Dv = v.shape[3]
     dev = q.device
@@ -160,7 +168,8 @@ def fix_attn_fwd(q, k, v, g, o_norm_weight, cu_seqlens=None, cu_seqlens_host=Non
     if workspace is None:
         workspace = torch.empty(max(nbytes, 1), device=dev, dtype=torch.uint8)
     s = lib.fix_attn_fwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(o_norm_weight),
-                         _ptr(y), *(map(_ptr, saved) if saved else (None, None, None)),
+                         _ptr(o_gate), _ptr(y),
+                         *(map(_ptr, saved) if saved else (None, None, None)),
                          _ptr(workspace), workspace.numel(), _stream(stream))
     if s != 0:
         raise FixStatusError(s, "fix_attn_fwd")
@@ -169,13 +178,15 @@ def fix_attn_fwd(q, k, v, g, o_norm_weight, cu_seqlens=None, cu_seqlens_host=Non
 
 
 def fix_attn_fwd_noalloc(q, k, v, g, o_norm_weight, y, saved, cu_seqlens=None,
-                         cu_seqlens_host=None, scale=None, eps=1e-6, algo="auto", stream=None):
+                         cu_seqlens_host=None, scale=None, eps=1e-6, algo="auto", stream=None,
+                         o_gate=None, o_norm=True):
     """Forward into caller-provided ``y`` and ``saved`` = (o, m, rstd) or None,
     with the library's own fixed device workspace (no allocation by anyone)."""
     lib = load()
-    p, keep = make_problem(q, k, v, cu_seqlens, cu_seqlens_host, scale, eps, y.dtype, algo)
+    p, keep = make_problem(q, k, v, cu_seqlens, cu_seqlens_host, scale, eps, y.dtype, algo,
+                           None, o_norm, g.dim() == 3)
     s = lib.fix_attn_fwd_noalloc(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
-                                 _ptr(o_norm_weight), _ptr(y),
+                                 _ptr(o_norm_weight), _ptr(o_gate), _ptr(y),
                                  *(map(_ptr, saved) if saved else (None, None, None)),
                                  _stream(stream))
     if s != 0:
@@ -186,44 +197,53 @@ def fix_attn_fwd_noalloc(q, k, v, g, o_norm_weight, y, saved, cu_seqlens=None,
 
 def fix_attn_bwd(q, k, v, g, o_norm_weight, dy, saved, cu_seqlens=None, cu_seqlens_host=None,
                  scale=None, eps=1e-6, algo="auto", workspace=None, stream=None, events=None,
-                 out=None, reuse_forward_workspace=False):
-    """Backward of sum(dy * y).  Returns dq, dk, dv, dg, dw (``out`` may
-    supply those five tensors).  ``reuse_forward_workspace``: ``workspace`` is
-    the one the matching training forward used (sized for the backward, see
-    ``training_workspace``) and has not been written since; the backward then
-    reuses the forward's gate prefix results (FIX_FLAG_REUSE_FWD_WORKSPACE)."""
+                 out=None, reuse_forward_workspace=False, o_gate=None, o_norm=True):
+    """Backward of sum(dy * y).  Returns dq, dk, dv, dg, dw, d_o_gate (the last
+    None without an output gate; dw None without the norm and no ``out``)
+    (``out`` may supply those six tensors).  ``reuse_forward_workspace``:
+    ``workspace`` is the one the matching training forward used (sized for the
+    backward, see ``training_workspace``) and has not been written since; the
+    backward then reuses the forward's gate prefix results
+    (FIX_FLAG_REUSE_FWD_WORKSPACE)."""
     lib = load()
     p, keep = make_problem(q, k, v, cu_seqlens, cu_seqlens_host, scale, eps, torch.bfloat16, algo,
-                           events)
+                           events, o_norm, g.dim() == 3)
     if reuse_forward_workspace:
         if workspace is None:
             raise ValueError("reuse_forward_workspace needs the forward's workspace")
-        p.flags = FIX_FLAG_REUSE_FWD_WORKSPACE
+        p.flags |= FIX_FLAG_REUSE_FWD_WORKSPACE
     if out is not None:
-        dq, dk, dv, dg, dw = out
+        dq, dk, dv, dg, dw = out[:5]
+        dz = out[5] if len(out) > 5 else None
     else:
         dq = torch.empty_like(q)
         dk = torch.empty_like(k)
         dv = torch.empty_like(v)
         dg = torch.empty_like(g)
-        dw = torch.empty_like(o_norm_weight)
+        dw = torch.empty_like(o_norm_weight) if o_norm_weight is not None else None
+        dz = None
+    if o_gate is not None and dz is None:
+        dz = torch.empty_like(o_gate)
     nbytes = fix_attn_workspace_bytes(p, True)
     if workspace is None:
         workspace = torch.empty(max(nbytes, 1), device=q.device, dtype=torch.uint8)
     o_s, m_s, r_s = saved
     s = lib.fix_attn_bwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(o_norm_weight),
-                         _ptr(dy), _ptr(o_s), _ptr(m_s), _ptr(r_s), _ptr(dq), _ptr(dk), _ptr(dv),
-                         _ptr(dg), _ptr(dw), _ptr(workspace), workspace.numel(), _stream(stream))
+                         _ptr(o_gate), _ptr(dy), _ptr(o_s), _ptr(m_s), _ptr(r_s), _ptr(dq),
+                         _ptr(dk), _ptr(dv), _ptr(dg), _ptr(dw), _ptr(dz), _ptr(workspace),
+                         workspace.numel(), _stream(stream))
     if s != 0:
         raise FixStatusError(s, "fix_attn_bwd")
     del keep
-    return dq, dk, dv, dg, dw
+    return dq, dk, dv, dg, dw, dz
 
 
-def training_workspace(q, k, v, cu_seqlens=None, cu_seqlens_host=None, algo="auto"):
+def training_workspace(q, k, v, cu_seqlens=None, cu_seqlens_host=None, algo="auto", g=None,
+                       o_norm=True):
     """A workspace sized for the backward, to pass to a training forward and
     then to its backward with ``reuse_forward_workspace=True``."""
-    p, keep = make_problem(q, k, v, cu_seqlens, cu_seqlens_host, None, 1e-6, torch.bfloat16, algo)
+    p, keep = make_problem(q, k, v, cu_seqlens, cu_seqlens_host, None, 1e-6, torch.bfloat16, algo,
+                           None, o_norm, g is not None and g.dim() == 3)
     n = fix_attn_workspace_bytes(p, True)
     del keep
     return torch.empty(max(n, 1), device=q.device, dtype=torch.uint8)
@@ -241,27 +261,35 @@ def fix_attn_noalloc_device_status(stream=None) -> int:
 
 class _FixAttn(torch.autograd.Function):
     @staticmethod
-    def forward(ctx, q, k, v, g, w, cu_seqlens, cu_host, scale, eps, algo):
-        ws = training_workspace(q, k, v, cu_seqlens, cu_host, algo)
+    def forward(ctx, q, k, v, g, w, z, cu_seqlens, cu_host, scale, eps, algo, o_norm):
+        ws = training_workspace(q, k, v, cu_seqlens, cu_host, algo, g, o_norm)
         y, saved = fix_attn_fwd(q, k, v, g, w, cu_seqlens, cu_host, scale, eps, save=True,
-                                algo=algo, workspace=ws)
-        ctx.save_for_backward(q, k, v, g, w, *saved)
-        ctx.cfg = (cu_seqlens, cu_host, scale, eps, algo)
+                                algo=algo, workspace=ws, o_gate=z, o_norm=o_norm)
+        ctx.save_for_backward(q, k, v, g, w, z, *saved)
+        ctx.cfg = (cu_seqlens, cu_host, scale, eps, algo, o_norm)
         ctx.ws = ws
         return y
 
     @staticmethod
     def backward(ctx, dy):
-        q, k, v, g, w, o_s, m_s, r_s = ctx.saved_tensors
-        cu, cu_host, scale, eps, algo = ctx.cfg
-        dq, dk, dv, dg, dw = fix_attn_bwd(q, k, v, g, w, dy.to(torch.bfloat16).contiguous(),
-                                          (o_s, m_s, r_s), cu, cu_host, scale, eps, algo,
-                                          workspace=ctx.ws, reuse_forward_workspace=True)
+        q, k, v, g, w, z, o_s, m_s, r_s = ctx.saved_tensors
+        cu, cu_host, scale, eps, algo, o_norm = ctx.cfg
+        dq, dk, dv, dg, dw, dz = fix_attn_bwd(q, k, v, g, w, dy.to(torch.bfloat16).contiguous(),
+                                              (o_s, m_s, r_s), cu, cu_host, scale, eps, algo,
+                                              workspace=ctx.ws, reuse_forward_workspace=True,
+                                              o_gate=z, o_norm=o_norm)
         ctx.ws = None
-        return dq, dk, dv, dg, dw, None, None, None, None, None
+        return dq, dk, dv, dg, dw, dz, None, None, None, None, None, None
 
 
-def fix_attn(q, k, v, g, o_norm_weight, cu_seqlens=None, cu_seqlens_host=None, scale=None,
-             eps=1e-6, algo="auto"):
-    """y = RMSNorm(FiX attention(q, k, v, g)) * o_norm_weight, differentiable."""
-    return _FixAttn.apply(q, k, v, g, o_norm_weight, cu_seqlens, cu_seqlens_host, scale, eps, algo)
+def fix_attn(q, k, v, g, o_norm_weight=None, cu_seqlens=None, cu_seqlens_host=None, scale=None,
+             eps=1e-6, algo="auto", o_gate=None, o_norm=True):
+    """FiX attention, differentiable, with the FiX README's arguments ("Quick
+    Start"): y = RMSNorm(FiX attention(q, k, v, g)) * o_norm_weight
+    [* swish(o_gate)]; with ``o_norm=False`` the output is the attention
+    average o_t / l_t [* swish(o_gate)].  g [B,T,Hkv,Dv] (element-wise gate)
+    or [B,T,Hkv] (scalar gate)."""
+    if o_norm and o_norm_weight is None:
+        raise ValueError("o_norm=True needs o_norm_weight")
+    return _FixAttn.apply(q, k, v, g, o_norm_weight, o_gate, cu_seqlens, cu_seqlens_host, scale,
+                          eps, algo, o_norm)

@@ -77,8 +77,19 @@ enum { FIX_ALGO_AUTO = 0, FIX_ALGO_SIMT = 1, FIX_ALGO_TC = 2 };
  *   backward then reuses the forward's gate prefix results (the prefix pass
  *   of the README's "Code Structure": chunk-local cumsums and pre-decayed
  *   values) instead of recomputing them.  Undefined results if the promise
- *   does not hold.  Any other bit: FIX_ERR_SHAPE. */
-enum { FIX_FLAG_REUSE_FWD_WORKSPACE = 1 };
+ *   does not hold.
+ * FIX_FLAG_NO_NORM: the README's o_norm = False.  No RMSNorm and no weight:
+ *   y_t = o_t / l_t with the softmax denominator l_t = sum_{s<=t} exp(S_ts
+ *   - m_t), i.e. the attention average with the element-wise decay on v (for
+ *   g = 0 ordinary causal softmax attention).  o_norm_weight may be NULL;
+ *   the saved tensors are then o_t / l_t, the log-sum-exp m_t + log l_t and
+ *   ones; the backward is the exact one and fills dw (if given) with zeros.
+ * FIX_FLAG_SCALAR_GATE: g (and dg) have shape [N, Hkv]: one log forget gate
+ *   per token and kv head, applied to every value channel (the Forgetting
+ *   Transformer's scalar gate, FoX abstract); dg is its gradient.
+ * Both must be set identically for a forward and its backward.  Any other
+ * bit: FIX_ERR_SHAPE. */
+enum { FIX_FLAG_REUSE_FWD_WORKSPACE = 1, FIX_FLAG_NO_NORM = 2, FIX_FLAG_SCALAR_GATE = 4 };
 
 typedef struct {
   int32_t batch;          /* B; must be 1 when cu_seqlens is given           */
@@ -126,31 +137,41 @@ enum {
 size_t fix_attn_workspace_bytes(const fix_attn_problem *p, int backward);
 
 /* Forward (training or inference).
- *   q [N,Hq,Dk] bf16, k [N,Hkv,Dk] bf16, v [N,Hkv,Dv] bf16, g [N,Hkv,Dv] f32,
- *   o_norm_weight [Dv] bf16  ->  y [N,Hq,Dv] (bf16 or f32, problem.y_dtype).
+ *   q [N,Hq,Dk] bf16, k [N,Hkv,Dk] bf16, v [N,Hkv,Dv] bf16, g [N,Hkv,Dv] f32
+ *   ([N,Hkv] with FIX_FLAG_SCALAR_GATE), o_norm_weight [Dv] bf16 (NULL allowed
+ *   with FIX_FLAG_NO_NORM), o_gate [N,Hq,Dv] bf16 or NULL
+ *   ->  y [N,Hq,Dv] (bf16 or f32, problem.y_dtype).
+ * With o_gate z, y is multiplied element-wise by swish(z) = z sigmoid(z)
+ * after the norm and its weight (the README's o_gate argument; the
+ * activation is not on the pages: swish is the output-gate form of the
+ * library FiX is forked from).
  * Saved tensors for fix_attn_bwd (pass all three, or all NULL for inference):
- *   o_saved [N,Hq,Dv] f32 (o before the norm), m_saved [N,Hq] f32 (row shift
- *   m_t), rstd_saved [N,Hq] f32.
+ *   o_saved [N,Hq,Dv] f32 (o before the norm and gate), m_saved [N,Hq] f32
+ *   (row shift m_t), rstd_saved [N,Hq] f32.
  * g should be <= 0 (a log forget gate); positive values are computed the same
  * way but the factors exp(G_t - G_s) are then only safe while they stay inside
- * the float32 range.  Definition: FiX poster abstract; shapes: FiX README,
- * "Quick Start". */
+ * the float32 range.  Definition: FiX poster abstract; shapes and arguments:
+ * FiX README, "Quick Start". */
 fix_status fix_attn_fwd(const fix_attn_problem *p, const void *q, const void *k,
                         const void *v, const float *g, const void *o_norm_weight,
-                        void *y, float *o_saved, float *m_saved, float *rstd_saved,
-                        void *workspace, size_t workspace_bytes, void *stream);
+                        const void *o_gate, void *y, float *o_saved, float *m_saved,
+                        float *rstd_saved, void *workspace, size_t workspace_bytes,
+                        void *stream);
 
-/* Backward of L = sum(dy * y) with the row shift m_t held constant.
- *   dy [N,Hq,Dv] bf16 and the saved o, m, rstd of the matching forward call
- *   -> dq [N,Hq,Dk], dk [N,Hkv,Dk], dv [N,Hkv,Dv] bf16, dg [N,Hkv,Dv] f32,
- *      dw [Dv] bf16 (gradient of o_norm_weight).
+/* Backward of L = sum(dy * y) with the row shift m_t held constant (the exact
+ * derivative with FIX_FLAG_NO_NORM, where y does not depend on m_t).
+ *   dy [N,Hq,Dv] bf16, o_gate as given to the forward, and the saved o, m,
+ *   rstd of the matching forward call
+ *   -> dq [N,Hq,Dk], dk [N,Hkv,Dk], dv [N,Hkv,Dv] bf16, dg f32 (g's shape),
+ *      dw [Dv] bf16 (gradient of o_norm_weight; may be NULL with
+ *      FIX_FLAG_NO_NORM), d_o_gate [N,Hq,Dv] bf16 (NULL iff o_gate is NULL).
  * dk, dv and dg sum over the q heads of each kv group. */
 fix_status fix_attn_bwd(const fix_attn_problem *p, const void *q, const void *k,
                         const void *v, const float *g, const void *o_norm_weight,
-                        const void *dy, const float *o_saved, const float *m_saved,
-                        const float *rstd_saved, void *dq, void *dk, void *dv,
-                        float *dg, void *dw, void *workspace, size_t workspace_bytes,
-                        void *stream);
+                        const void *o_gate, const void *dy, const float *o_saved,
+                        const float *m_saved, const float *rstd_saved, void *dq, void *dk,
+                        void *dv, float *dg, void *dw, void *d_o_gate, void *workspace,
+                        size_t workspace_bytes, void *stream);
 
 /* Synchronises `stream`, then returns the device status word that the last
  * call on this workspace left (FIX_OK or FIX_ERR_DEVICE_TIMEOUT), or
@@ -188,8 +209,8 @@ fix_status fix_attn_device_status(const void *workspace, void *stream);
  *     the array's status word; fix_attn_noalloc_device_status reads it. */
 fix_status fix_attn_fwd_noalloc(const fix_attn_problem *p, const void *q, const void *k,
                                 const void *v, const float *g, const void *o_norm_weight,
-                                void *y, float *o_saved, float *m_saved, float *rstd_saved,
-                                void *stream);
+                                const void *o_gate, void *y, float *o_saved, float *m_saved,
+                                float *rstd_saved, void *stream);
 
 /* fix_attn_device_status for fix_attn_fwd_noalloc: synchronises `stream`,
  * then returns the status word that the last fix_attn_fwd_noalloc call on

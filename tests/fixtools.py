@@ -40,40 +40,51 @@ def to_cuda(case):
     return out
 
 
-def run_gpu(case, algo="auto", backward=False, y_dtype=torch.float32, reuse=True):
+def run_gpu(case, algo="auto", backward=False, y_dtype=torch.float32, reuse=True, o_gate=None,
+            o_norm=True):
     """Forward (and backward) through the C ABI; returns numpy float64 dicts.
-    ``reuse``: the backward reuses the forward's workspace (its gate prefix)."""
+    ``reuse``: the backward reuses the forward's workspace (its gate prefix).
+    ``o_gate``: a CPU bf16 tensor [B,T,Hq,Dv]; a gate g of shape [B,T,Hkv]
+    runs the scalar-gate mode."""
     from gated_softmax_attention_fp32_b200 import fixattn
     t = to_cuda(case)
+    z = o_gate.cuda().contiguous() if o_gate is not None else None
     cu_host = case["cu_seqlens"]
+    scalar = t["g"].dim() == 3
     # one workspace for both calls, so that the device status word (where a
     # bounded device wait that expired reports) can be checked after each
     p, _keep = fixattn.make_problem(t["q"], t["k"], t["v"], t["cu_seqlens"], cu_host, None,
-                                    case["eps"], y_dtype, algo)
+                                    case["eps"], y_dtype, algo, None, o_norm, scalar)
     ws = torch.empty(max(fixattn.fix_attn_workspace_bytes(p, backward), 1), device="cuda",
                      dtype=torch.uint8)
-    y, saved = fixattn.fix_attn_fwd(t["q"], t["k"], t["v"], t["g"], t["w"], t["cu_seqlens"],
+    w = t["w"] if o_norm else None
+    y, saved = fixattn.fix_attn_fwd(t["q"], t["k"], t["v"], t["g"], w, t["cu_seqlens"],
                                     cu_host, None, case["eps"], y_dtype=y_dtype, save=True,
-                                    algo=algo, workspace=ws)
+                                    algo=algo, workspace=ws, o_gate=z, o_norm=o_norm)
     assert fixattn.fix_attn_device_status(ws) == 0, "forward: device status not OK"
     res = dict(y=y, o=saved[0], m=saved[1], rstd=saved[2])
     if backward:
-        dq, dk, dv, dg, dw = fixattn.fix_attn_bwd(t["q"], t["k"], t["v"], t["g"], t["w"], t["dy"],
-                                                  saved, t["cu_seqlens"], cu_host, None,
-                                                  case["eps"], algo=algo, workspace=ws,
-                                                  reuse_forward_workspace=reuse)
+        dq, dk, dv, dg, dw, dz = fixattn.fix_attn_bwd(
+            t["q"], t["k"], t["v"], t["g"], w, t["dy"], saved, t["cu_seqlens"], cu_host, None,
+            case["eps"], algo=algo, workspace=ws, reuse_forward_workspace=reuse, o_gate=z,
+            o_norm=o_norm)
         assert fixattn.fix_attn_device_status(ws) == 0, "backward: device status not OK"
-        res.update(dq=dq, dk=dk, dv=dv, dg=dg, dw=dw)
+        res.update(dq=dq, dk=dk, dv=dv, dg=dg)
+        if dw is not None:
+            res["dw"] = dw
+        if dz is not None:
+            res["d_o_gate"] = dz
     torch.cuda.synchronize()
     return {k: v.float().cpu().numpy().astype(np.float64) for k, v in res.items()}
 
 
-def oracle_full(case, backward=False):
+def oracle_full(case, backward=False, o_gate=None, o_norm=True):
     args = (case["q"], case["k"], case["v"], case["g"], case["w"])
     seqlens = case["seqlens"] if case["cu_seqlens"] is not None else None
-    f = fix_ref.forward(*args, seqlens, None, case["eps"], workers())
+    f = fix_ref.forward(*args, seqlens, None, case["eps"], workers(), norm=o_norm, o_gate=o_gate)
     if backward:
-        f.update(fix_ref.backward(*args, case["dy"], seqlens, None, case["eps"], workers()))
+        f.update(fix_ref.backward(*args, case["dy"], seqlens, None, case["eps"], workers(),
+                                  norm=o_norm, o_gate=o_gate))
     return f
 
 

@@ -105,7 +105,7 @@ def _expected_workspace(seqlens, Hq, Hkv, Dk, Dv, backward):
     nparts = sum(_ceil(grp * half(L, j), P) + _ceil(grp * (t64(L, j) - half(L, j)), P)
                  for L in seqlens for j in range(_ceil(L, 128)))
     for nbytes in (N * Hq * Dv * 4, N * Hq * Dv * 2, N * Hq * Dv * 2, N * Hq * Dv * 2,
-                   nc1 * Hq * 4, nc1 * Hq * 4, N * Hq * 4, nkv * 4, nkv * 4, nch * 4,
+                   nc1 * Hq * 4, nc1 * Hq * 4, N * Hq * 4, N * Hq * 4, nkv * 4, nkv * 4, nch * 4,
                    nc1 * 4 * Hkv * Dv * 4, max(nparts, 1) * 16, nc1 * 8,
                    nparts * Hkv * 128 * (Dk + Dv) * 4):
         take(nbytes)
@@ -147,7 +147,7 @@ def test_workspace_layout_and_dkv_split(lib, seqlens, Hq, Hkv, Dk, Dv):
     (dict(T=-1), FIX_ERR_SHAPE),
     (dict(y_dtype=7), FIX_ERR_DTYPE),
     (dict(algo=9), FIX_ERR_DTYPE),
-    (dict(flags=2), FIX_ERR_SHAPE),
+    (dict(flags=8), FIX_ERR_SHAPE),
     (dict(eps=-1.0), FIX_ERR_SHAPE),
     (dict(num_seqs=2), FIX_ERR_CU_SEQLENS),
 ])
@@ -156,10 +156,10 @@ def test_bad_problem_rejected_on_host(lib, kw, code):
     buf = (ctypes.c_uint8 * 4096)()
     a = ctypes.addressof(buf)
     a = (a + 15) // 16 * 16
-    ptrs = [ctypes.c_void_p(a)] * 10
+    ptrs = [ctypes.c_void_p(a)] * 11
     s = lib.fix_attn_fwd(ctypes.byref(p), *ptrs, 1 << 40, None)
     assert s == code, fixattn.status_string(s)
-    ptrs = [ctypes.c_void_p(a)] * 15
+    ptrs = [ctypes.c_void_p(a)] * 17
     s = lib.fix_attn_bwd(ctypes.byref(p), *ptrs, 1 << 40, None)
     assert s == code, fixattn.status_string(s)
 
@@ -182,7 +182,7 @@ def test_bad_cu_seqlens_rejected(lib, cu, code):
     assert lib.fix_attn_workspace_bytes(ctypes.byref(p), 0) == 0
     buf = (ctypes.c_uint8 * 64)()
     a = (ctypes.addressof(buf) + 15) // 16 * 16
-    s = lib.fix_attn_fwd(ctypes.byref(p), *[ctypes.c_void_p(a)] * 10, 1 << 40, None)
+    s = lib.fix_attn_fwd(ctypes.byref(p), *[ctypes.c_void_p(a)] * 11, 1 << 40, None)
     assert s == code
 
 
@@ -203,17 +203,44 @@ def test_null_misaligned_and_small_workspace(lib):
     need = lib.fix_attn_workspace_bytes(ctypes.byref(p), 0)
     buf = (ctypes.c_uint8 * 4096)()
     a = (ctypes.addressof(buf) + 15) // 16 * 16
-    good = [ctypes.c_void_p(a)] * 10
+    # q, k, v, g, w, o_gate, y, o_saved, m_saved, rstd_saved, workspace
+    good = [ctypes.c_void_p(a)] * 11
     s = lib.fix_attn_fwd(ctypes.byref(p), *([None] + good[1:]), need, None)
     assert s == FIX_ERR_NULL
     bad = list(good)
     bad[2] = ctypes.c_void_p(a + 2)
     assert lib.fix_attn_fwd(ctypes.byref(p), *bad, need, None) == FIX_ERR_ALIGN
+    bad = list(good)
+    bad[5] = ctypes.c_void_p(a + 4)                 # a misaligned output gate
+    assert lib.fix_attn_fwd(ctypes.byref(p), *bad, need, None) == FIX_ERR_ALIGN
     assert lib.fix_attn_fwd(ctypes.byref(p), *good, need - 1, None) == FIX_ERR_WORKSPACE
     # saved tensors: all three or none
     part = list(good)
-    part[7] = None
+    part[8] = None
     assert lib.fix_attn_fwd(ctypes.byref(p), *part, need, None) == FIX_ERR_NULL
+    # o_norm_weight is required with the norm, optional without it
+    now = list(good)
+    now[4] = None
+    assert lib.fix_attn_fwd(ctypes.byref(p), *now, need, None) == FIX_ERR_NULL
+    # backward: o_gate and d_o_gate both given or both NULL
+    pb = prob()
+    needb = lib.fix_attn_workspace_bytes(ctypes.byref(pb), 1)
+    gb = [ctypes.c_void_p(a)] * 17
+    half = list(gb)
+    half[16] = None                                  # d_o_gate missing, o_gate given
+    assert lib.fix_attn_bwd(ctypes.byref(pb), *half, needb, None) == FIX_ERR_NULL
+
+
+def test_flag_dependent_workspace(lib):
+    """Without the norm the forward workspace is the same; a scalar gate adds
+    the per-channel dg buffer to the backward's."""
+    base0 = lib.fix_attn_workspace_bytes(ctypes.byref(prob()), 0)
+    base1 = lib.fix_attn_workspace_bytes(ctypes.byref(prob()), 1)
+    assert lib.fix_attn_workspace_bytes(ctypes.byref(prob(flags=2)), 0) == base0
+    assert lib.fix_attn_workspace_bytes(ctypes.byref(prob(flags=2)), 1) == base1
+    assert lib.fix_attn_workspace_bytes(ctypes.byref(prob(flags=4)), 0) == base0
+    extra = lib.fix_attn_workspace_bytes(ctypes.byref(prob(flags=4)), 1) - base1
+    assert extra == -(-(2 * 100 * 2 * 64 * 4) // 256) * 256
 
 
 def test_status_strings(lib):

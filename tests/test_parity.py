@@ -263,3 +263,71 @@ def test_workload5_full(cuda_lib):
     check_fwd(gpu["y"], ref["y"], "workload 5")
     for key in GRADS:
         check_grad(key, gpu[key], ref[key], "workload 5")
+
+
+# ------------------------------------------ o_gate, o_norm = False, scalar gate
+# FiX README "Quick Start" (o_norm, o_norm_weight, o_gate arguments) and the
+# Forgetting Transformer abstract (scalar forget gates); readings in the
+# oracle's header.
+
+OPTION_SHAPES = {
+    "T300-D64-gqa": dict(B=1, T=300, Hq=4, Hkv=2, Dk=64, Dv=64),
+    "B2-T257-D128": dict(B=2, T=257, Hq=2, Hkv=1, Dk=128, Dv=128),
+    "varlen-D64": dict(B=1, T=0, Hq=2, Hkv=1, Dk=64, Dv=64, seqlens=[0, 1, 130, 7, 255]),
+    "T129-D32": dict(B=1, T=129, Hq=2, Hkv=2, Dk=32, Dv=32),
+}
+
+
+def _gate(case, seed):
+    gen = torch.Generator().manual_seed(seed)
+    return torch.randn(case["B"], case["T"], case["Hq"], case["Dv"], generator=gen).to(
+        torch.bfloat16)
+
+
+def _check_all(gpu, ref, tag, o_norm=True):
+    check_fwd(gpu["y"], ref["y"], tag)
+    keys = ["dq", "dk", "dv", "dg"] + (["dw"] if o_norm else []) + \
+        (["d_o_gate"] if "d_o_gate" in ref else [])
+    for key in keys:
+        check_grad(key, gpu[key], ref[key], tag)
+
+
+@pytest.mark.parametrize("algo", ["auto", "simt"])
+@pytest.mark.parametrize("name", list(OPTION_SHAPES))
+def test_output_gate(cuda_lib, name, algo):
+    case = synth.make_case(**OPTION_SHAPES[name], seed=51)
+    z = _gate(case, 52)
+    gpu = run_gpu(case, algo, backward=True, o_gate=z)
+    ref = oracle_full(case, backward=True, o_gate=z)
+    _check_all(gpu, ref, f"{name} o_gate")
+
+
+@pytest.mark.parametrize("algo", ["auto", "simt"])
+@pytest.mark.parametrize("name", list(OPTION_SHAPES))
+def test_no_norm(cuda_lib, name, algo):
+    case = synth.make_case(**OPTION_SHAPES[name], seed=53)
+    gpu = run_gpu(case, algo, backward=True, o_norm=False)
+    ref = oracle_full(case, backward=True, o_norm=False)
+    _check_all(gpu, ref, f"{name} no norm", o_norm=False)
+
+
+@pytest.mark.parametrize("algo", ["auto", "simt"])
+@pytest.mark.parametrize("name", list(OPTION_SHAPES))
+def test_scalar_gate(cuda_lib, name, algo):
+    case = synth.make_case(**OPTION_SHAPES[name], seed=54)
+    case = dict(case, g=case["g"][..., 0].contiguous())     # one gate per (token, kv head)
+    gpu = run_gpu(case, algo, backward=True)
+    ref = oracle_full(case, backward=True)
+    assert gpu["dg"].shape == ref["dg"].shape == tuple(case["g"].shape)
+    _check_all(gpu, ref, f"{name} scalar gate")
+
+
+def test_all_options_together_workload2_shape(cuda_lib):
+    """Scalar gate, no norm and an output gate on the README's example shape
+    (B2 T2048 H8/4 D128), every output and gradient against the full oracle."""
+    case = synth.draw(synth.workload(2))
+    case = dict(case, g=case["g"][..., 0].contiguous())
+    z = _gate(case, 55)
+    gpu = run_gpu(case, backward=True, o_gate=z, o_norm=False)
+    ref = oracle_full(case, backward=True, o_gate=z, o_norm=False)
+    _check_all(gpu, ref, "workload 2 shape, all options", o_norm=False)

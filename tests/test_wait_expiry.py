@@ -31,7 +31,7 @@ def _test_lib():
         pytest.fail(f"test build of the library missing: {path}")
     lib = ctypes.CDLL(path)
     vp, sz = ctypes.c_void_p, ctypes.c_size_t
-    lib.fix_attn_fwd.argtypes = [ctypes.POINTER(fixattn.Problem)] + [vp] * 10 + [sz, vp]
+    lib.fix_attn_fwd.argtypes = [ctypes.POINTER(fixattn.Problem)] + [vp] * 11 + [sz, vp]
     lib.fix_attn_fwd.restype = ctypes.c_int
     lib.fix_attn_device_status.argtypes = [vp, vp]
     lib.fix_attn_device_status.restype = ctypes.c_int
@@ -57,7 +57,7 @@ def test_forward_wait_expiry_reports_timeout_and_recovers(cuda_lib):
     def call():
         ptr = lambda x: ctypes.c_void_p(x.data_ptr())
         return lib.fix_attn_fwd(ctypes.byref(p), ptr(t["q"]), ptr(t["k"]), ptr(t["v"]),
-                                ptr(t["g"]), ptr(t["w"]), ptr(y), None, None, None, ptr(ws),
+                                ptr(t["g"]), ptr(t["w"]), None, ptr(y), None, None, None, ptr(ws),
                                 ws.numel(), stream)
 
     try:

@@ -40,8 +40,8 @@ def _noalloc_call(lib, fixattn, t, cu=None, cu_host=None):
     r = torch.full((B, T, Hq), float("nan"), device="cuda")
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     s = lib.fix_attn_fwd_noalloc(ctypes.byref(p), _ptr(t["q"]), _ptr(t["k"]), _ptr(t["v"]),
-                                 _ptr(t["g"]), _ptr(t["w"]), _ptr(y), _ptr(o), _ptr(m), _ptr(r),
-                                 stream)
+                                 _ptr(t["g"]), _ptr(t["w"]), None, _ptr(y), _ptr(o), _ptr(m),
+                                 _ptr(r), stream)
     torch.cuda.synchronize()
     del keep
     return s, y, (o, m, r)
@@ -121,6 +121,6 @@ def test_noalloc_rejects_problem_far_beyond_its_workspace(cuda_lib):
     p = _problem(fixattn, 1 << 16, Hq=8, Hkv=8)
     assert fixattn.fix_attn_workspace_bytes(p, False) > fixattn.NOALLOC_MAX_WORKSPACE_BYTES
     buf = torch.empty(64, dtype=torch.uint8, device="cuda")     # never touched
-    ptrs = [_ptr(buf)] * 9
+    ptrs = [_ptr(buf)] * 10
     s = lib.fix_attn_fwd_noalloc(ctypes.byref(p), *ptrs, None)
     assert s == FIX_ERR_WORKSPACE
