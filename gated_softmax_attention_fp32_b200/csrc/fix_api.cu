@@ -23,6 +23,8 @@ static bool head_dim_ok(int d) { return d == 16 || d == 32 || d == 64 || d == 12
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Validates the problem descriptor and fills the kernel-side dims.
+static fix_status make_dims(const fix_attn_problem* p, Dims* d);
+fix_status validate_problem(const fix_attn_problem* p, Dims* d) { return make_dims(p, d); }
 static fix_status make_dims(const fix_attn_problem* p, Dims* d) {
   if (!p) return FIX_ERR_NULL;
   if (p->flags & ~(FIX_FLAG_REUSE_FWD_WORKSPACE | FIX_FLAG_NO_NORM | FIX_FLAG_SCALAR_GATE))

@@ -7,6 +7,18 @@ namespace fix {
 
 constexpr int ST_ROWS = 32;  // rows per CTA of the exact (SIMT) kernels
 
+// Validates a problem descriptor and fills the kernel-side dims (fix_api.cu).
+fix_status validate_problem(const fix_attn_problem* p, Dims* d);
+
+// Sizes of one decode call (fix_decode.cu).
+struct DecodeDims {
+  int B, Tmax, Hq, Hkv, Dk, Dv, grp;
+  int R;        // keys per range of the split
+  int nsplit;   // ranges over Tmax
+  float scale, eps;
+  int no_norm, scalar_gate;
+};
+
 // fix_prefix.cu
 template <int NW>
 __global__ void upload_kernel(const __grid_constant__ Blob<NW> b, uint32_t* dst, int nwords);

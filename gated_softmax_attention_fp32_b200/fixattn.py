@@ -20,13 +20,15 @@ from typing import Optional
 import torch
 
 __all__ = ["load", "Problem", "fix_attn_fwd", "fix_attn_bwd", "fix_attn_workspace_bytes",
+           "fix_attn_decode",
            "fix_attn_device_status", "fix_attn", "training_workspace", "FixStatusError", "LIB_PATH",
            "EXPORTS"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfixattn.so")
 EXPORTS = ("fix_attn_workspace_bytes", "fix_attn_fwd", "fix_attn_bwd", "fix_attn_device_status",
            "fix_attn_kernel_count", "fix_attn_status_string", "fix_attn_fwd_noalloc",
-           "fix_attn_noalloc_device_status")
+           "fix_attn_noalloc_device_status", "fix_attn_decode_workspace_bytes",
+           "fix_attn_decode")
 NOALLOC_MAX_WORKSPACE_BYTES = 16 * 1024 * 1024
 FIX_FLAG_REUSE_FWD_WORKSPACE = 1
 FIX_FLAG_NO_NORM = 2
@@ -78,6 +80,10 @@ def load():
     lib.fix_attn_device_status.restype = ctypes.c_int
     lib.fix_attn_noalloc_device_status.argtypes = [vp]
     lib.fix_attn_noalloc_device_status.restype = ctypes.c_int
+    lib.fix_attn_decode_workspace_bytes.argtypes = [P]
+    lib.fix_attn_decode_workspace_bytes.restype = sz
+    lib.fix_attn_decode.argtypes = [P] + [vp] * 10 + [sz, vp]
+    lib.fix_attn_decode.restype = ctypes.c_int
     lib.fix_attn_kernel_count.argtypes = [P, ctypes.c_int]
     lib.fix_attn_kernel_count.restype = ctypes.c_int
     lib.fix_attn_status_string.argtypes = [ctypes.c_int]
@@ -247,6 +253,35 @@ def training_workspace(q, k, v, cu_seqlens=None, cu_seqlens_host=None, algo="aut
     n = fix_attn_workspace_bytes(p, True)
     del keep
     return torch.empty(max(n, 1), device=q.device, dtype=torch.uint8)
+
+
+def fix_attn_decode(q, k_cache, v_cache, g_cache, seqlens, o_norm_weight=None, scale=None,
+                    eps=1e-6, y_dtype=torch.bfloat16, o_gate=None, o_norm=True, workspace=None,
+                    out=None, stream=None):
+    """One new query per sequence against its cache.  q [B,Hq,Dk];
+    k_cache [B,Tmax,Hkv,Dk], v_cache [B,Tmax,Hkv,Dv] bf16; g_cache
+    [B,Tmax,Hkv,Dv] (or [B,Tmax,Hkv]) f32; seqlens int32 [B] on the device
+    (tokens per cache, the new one included).  Returns y [B,Hq,Dv]."""
+    lib = load()
+    B, Hq, Dk = q.shape
+    Tmax, Hkv, Dv = v_cache.shape[1], v_cache.shape[2], v_cache.shape[3]
+    p = Problem()
+    p.batch, p.seqlen, p.num_q_heads, p.num_kv_heads = B, Tmax, Hq, Hkv
+    p.head_dim_k, p.head_dim_v = Dk, Dv
+    p.y_dtype = 1 if y_dtype == torch.float32 else 0
+    p.flags = (0 if o_norm else FIX_FLAG_NO_NORM) | (FIX_FLAG_SCALAR_GATE if g_cache.dim() == 3 else 0)
+    p.scale = float(scale) if scale is not None else 0.0
+    p.eps = float(eps)
+    y = out if out is not None else torch.empty(B, Hq, Dv, device=q.device, dtype=y_dtype)
+    nbytes = int(lib.fix_attn_decode_workspace_bytes(ctypes.byref(p)))
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 1), device=q.device, dtype=torch.uint8)
+    s = lib.fix_attn_decode(ctypes.byref(p), _ptr(seqlens), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                            _ptr(g_cache), _ptr(o_norm_weight), _ptr(o_gate), _ptr(y),
+                            _ptr(workspace), workspace.numel(), _stream(stream))
+    if s != 0:
+        raise FixStatusError(s, "fix_attn_decode")
+    return y
 
 
 def fix_attn_device_status(workspace, stream=None) -> int:

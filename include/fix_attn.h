@@ -173,6 +173,29 @@ fix_status fix_attn_bwd(const fix_attn_problem *p, const void *q, const void *k,
                         void *dv, float *dg, void *dw, void *d_o_gate, void *workspace,
                         size_t workspace_bytes, void *stream);
 
+/* Decode: one new query per sequence against the cache of its tokens.
+ * The problem gives batch = B sequences, seqlen = Tmax (cache capacity),
+ * heads, head dims, scale, eps, y_dtype and the flags FIX_FLAG_NO_NORM /
+ * FIX_FLAG_SCALAR_GATE; cu_seqlens must be NULL and num_seqs 0.
+ *   seqlens   device int32 [B]: L_b, the tokens in sequence b's cache, the
+ *             new token included (0 < L_b <= Tmax; L_b = 0 gives y = 0)
+ *   q         [B,Hq,Dk] bf16: the new token's queries
+ *   k_cache   [B,Tmax,Hkv,Dk] bf16, v_cache [B,Tmax,Hkv,Dv] bf16,
+ *   g_cache   [B,Tmax,Hkv,Dv] f32 ([B,Tmax,Hkv] with the scalar gate): the
+ *             keys, values and log forget gates of tokens 0..L_b-1
+ *   o_norm_weight [Dv] bf16 (NULL allowed without the norm), o_gate [B,Hq,Dv]
+ *             bf16 or NULL  ->  y [B,Hq,Dv] (bf16 or f32)
+ * y is row t = L_b - 1 of fix_attn_fwd on the same sequence (the FiX poster
+ * abstract names inference memory as a challenge FiX addresses; the pages
+ * give no decode algorithm, so this evaluates the definition for the last
+ * row).  Requires Hq/Hkv * Dv <= 2048 (FIX_ERR_GQA otherwise).  The cache is
+ * read once, split over CTAs by key ranges. */
+size_t fix_attn_decode_workspace_bytes(const fix_attn_problem *p);
+fix_status fix_attn_decode(const fix_attn_problem *p, const int32_t *seqlens, const void *q,
+                           const void *k_cache, const void *v_cache, const float *g_cache,
+                           const void *o_norm_weight, const void *o_gate, void *y,
+                           void *workspace, size_t workspace_bytes, void *stream);
+
 /* Synchronises `stream`, then returns the device status word that the last
  * call on this workspace left (FIX_OK or FIX_ERR_DEVICE_TIMEOUT), or
  * FIX_ERR_CUDA if the stream reports an error.  The word is reset by every

@@ -331,3 +331,73 @@ def test_all_options_together_workload2_shape(cuda_lib):
     gpu = run_gpu(case, backward=True, o_gate=z, o_norm=False)
     ref = oracle_full(case, backward=True, o_gate=z, o_norm=False)
     _check_all(gpu, ref, "workload 2 shape, all options", o_norm=False)
+
+
+# ------------------------------------------------------------------ decode
+# One new query per sequence against its (k, v, g) cache: y must equal row
+# L - 1 of the forward of the same sequence.  Cache slots past each length
+# hold NaN, so any read beyond L would show.
+
+def _decode_case(lengths, Tmax, Hq, Hkv, D, seed, scalar=False):
+    B = len(lengths)
+    case = synth.make_case(B, Tmax, Hq, Hkv, D, D, seed=seed)
+    if scalar:
+        case = dict(case, g=case["g"][..., 0].contiguous())
+    return case
+
+
+def _decode_ref(case, lengths, o_gate=None, o_norm=True):
+    ys = []
+    for b, L in enumerate(lengths):
+        sub = sequence_case(case, b, 0, L)
+        z = None if o_gate is None else o_gate[b:b + 1, :, None].expand(1, L, -1, -1).contiguous()
+        ref = oracle_full(sub, o_gate=z, o_norm=o_norm)
+        ys.append(ref["y"][0, L - 1])
+    return np.stack(ys)
+
+
+@pytest.mark.parametrize("opts", [dict(), dict(gate=True), dict(o_norm=False),
+                                  dict(scalar=True, gate=True)])
+def test_decode_matches_last_forward_row(cuda_lib, opts):
+    from gated_softmax_attention_fp32_b200 import fixattn
+    lengths, Tmax = [1, 70, 300, 129], 320
+    case = _decode_case(lengths, Tmax, 4, 2, 64, 61, opts.get("scalar", False))
+    B = len(lengths)
+    qd = torch.stack([case["q"][b, L - 1] for b, L in enumerate(lengths)])
+    kc, vc, gc = (case[x].clone() for x in ("k", "v", "g"))
+    for b, L in enumerate(lengths):
+        kc[b, L:] = float("nan"); vc[b, L:] = float("nan"); gc[b, L:] = float("nan")
+    z = None
+    if opts.get("gate"):
+        z = torch.randn(B, 4, 64, generator=torch.Generator().manual_seed(62)).to(torch.bfloat16)
+    o_norm = opts.get("o_norm", True)
+    y = fixattn.fix_attn_decode(qd.cuda(), kc.cuda(), vc.cuda(), gc.cuda(),
+                                torch.tensor(lengths, dtype=torch.int32).cuda(),
+                                case["w"].cuda() if o_norm else None, eps=case["eps"],
+                                y_dtype=torch.float32, o_norm=o_norm,
+                                o_gate=None if z is None else z.cuda())
+    torch.cuda.synchronize()
+    ref = _decode_ref(case, lengths, z, o_norm)
+    check_fwd(y.double().cpu().numpy(), ref, f"decode {opts}")
+
+
+def test_decode_long_context_rows(cuda_lib):
+    """Workload 4's shape (T = 32768, H 32/8, D 128) as a decode of its last
+    token, and of a shorter cache, against the oracle's rows."""
+    from gated_softmax_attention_fp32_b200 import fixattn
+    case = synth.draw(synth.workload(4))
+    T = case["T"]
+    lengths = [T, 20000]
+    kc = case["k"].expand(2, -1, -1, -1).contiguous()
+    vc = case["v"].expand(2, -1, -1, -1).contiguous()
+    gc = case["g"].expand(2, -1, -1, -1).contiguous()
+    qd = torch.stack([case["q"][0, L - 1] for L in lengths])
+    y = fixattn.fix_attn_decode(qd.cuda(), kc.cuda(), vc.cuda(), gc.cuda(),
+                                torch.tensor(lengths, dtype=torch.int32).cuda(),
+                                case["w"].cuda(), eps=case["eps"], y_dtype=torch.float32)
+    torch.cuda.synchronize()
+    for b, L in enumerate(lengths):
+        for h in (0, 13, 31):
+            r = fix_ref.forward_rows(case["q"], case["k"], case["v"], case["g"], case["w"],
+                                     (0, 0), L, h, [L - 1], None, case["eps"])
+            check_fwd(y[b, h].double().cpu().numpy()[None], r["y"], f"decode L={L} h={h}")
