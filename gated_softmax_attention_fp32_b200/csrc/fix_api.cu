@@ -282,7 +282,8 @@ static void each_sequence(const fix_attn_problem* p, Fn fn) {
 
 // Builds the schedule on the host and uploads it into the workspace:
 //   chunks[]  the chunk table, sequences in order, 128-token chunks from each
-//             sequence's first token;
+//             sequence's first token (followed by safe[] = 1, see the prefix
+//             pass);
 //   order[]   chunk ids by decreasing chunk index j (the number of key blocks
 //             before the diagonal; ties in table order), so that grids
 //             walking order[] start the longest causal rows first;
@@ -297,8 +298,11 @@ static fix_status upload_schedule(const fix_attn_problem* p, const Dims& d, cons
                                   cudaStream_t st) {
   if (d.nchunks == 0) return FIX_OK;
   thread_local std::vector<uint32_t> bufA, bufB;
-  const size_t spanA = ws.order - ws.chunks + (size_t)d.nchunks * sizeof(int);
+  // chunk table, order, and the fp16-safe flags of the prefix pass set to 1
+  // (its CTAs AND their part in)
+  const size_t spanA = ws.safe - ws.chunks + (size_t)d.nchunks * d.Hkv * sizeof(int);
   bufA.assign(spanA / 4, 0u);
+  std::fill(bufA.begin() + (ws.safe - ws.chunks) / 4, bufA.end(), 1u);
   Chunk* chunks = reinterpret_cast<Chunk*>(bufA.data());
   int* order = reinterpret_cast<int*>(reinterpret_cast<char*>(bufA.data()) + (ws.order - ws.chunks));
   int ci = 0, maxj = 0;
@@ -362,7 +366,7 @@ static fix_status run_prefix(const Dims& d, const fix_attn_problem* p, const Ws&
       return FIX_ERR_CUDA;
     return FIX_OK;
   }
-  prefix_kernel<<<dim3(d.nchunks, d.Hkv), 512, 0, st>>>(
+  prefix_kernel<<<dim3(d.nchunks, d.Hkv, (d.Dv + 31) / 32), 128, 0, st>>>(
       d, chunks, g, static_cast<const __nv_bfloat16*>(v), reinterpret_cast<float*>(base + ws.L),
       want_vt ? reinterpret_cast<uint16_t*>(base + ws.vt) : nullptr,
       reinterpret_cast<__nv_bfloat16*>(base + ws.vm),
@@ -606,10 +610,11 @@ fix_status fix_attn_bwd(const fix_attn_problem* p, const void* q, const void* k,
   }
   FIX_TRY(mark(p, FIX_STAGE_BWD_FINISH, 1, st));
   FIX_TRY(mark(p, FIX_STAGE_BWD_DG, 0, st));
-  chunk_total_kernel<<<dim3(d.nchunks, d.Hkv), 512, 0, st>>>(d, chunks, dG, dtot);
+  chunk_total_kernel<<<dim3(d.nchunks, d.Hkv, (d.Dv + 31) / 32), 128, 0, st>>>(d, chunks, dG, dtot);
   FIX_TRY(launched());
   float* dgf = d.scalar_gate ? reinterpret_cast<float*>(base + ws.dgf) : dg;
-  reverse_cumsum_kernel<<<dim3(d.nchunks, d.Hkv), 512, 0, st>>>(d, chunks, dG, dtot, dgf);
+  reverse_cumsum_kernel<<<dim3(d.nchunks, d.Hkv, (d.Dv + 31) / 32), 128, 0, st>>>(d, chunks, dG,
+                                                                                 dtot, dgf);
   FIX_TRY(launched());
   if (d.scalar_gate) {
     // a scalar gate acts on every channel: its gradient is the channel sum
@@ -626,7 +631,8 @@ int fix_attn_kernel_count(const fix_attn_problem* p, int backward) {
   if (d.N == 0) return 0;
   const SplitPlan sp = backward ? plan_split(p, d) : SplitPlan{};
   const Ws ws = layout(d, backward != 0, sp);
-  const int upA = d.nchunks ? upload_launches(ws.order - ws.chunks + (size_t)d.nchunks * 4) : 0;
+  const int upA =
+      d.nchunks ? upload_launches(ws.safe - ws.chunks + (size_t)d.nchunks * d.Hkv * 4) : 0;
   if (!backward) {
     const bool tc = p->algo != FIX_ALGO_SIMT && tc_fwd_supported(d);
     // schedule upload, prefix pass, attention
