@@ -366,7 +366,7 @@ static fix_status run_prefix(const Dims& d, const fix_attn_problem* p, const Ws&
       return FIX_ERR_CUDA;
     return FIX_OK;
   }
-  prefix_kernel<<<dim3(d.nchunks, d.Hkv, (d.Dv + 31) / 32), 128, 0, st>>>(
+  prefix_kernel<<<dim3(d.nchunks, d.Hkv, (d.Dv + 31) / 32), 256, 0, st>>>(
       d, chunks, g, static_cast<const __nv_bfloat16*>(v), reinterpret_cast<float*>(base + ws.L),
       want_vt ? reinterpret_cast<uint16_t*>(base + ws.vt) : nullptr,
       reinterpret_cast<__nv_bfloat16*>(base + ws.vm),
@@ -610,10 +610,10 @@ fix_status fix_attn_bwd(const fix_attn_problem* p, const void* q, const void* k,
   }
   FIX_TRY(mark(p, FIX_STAGE_BWD_FINISH, 1, st));
   FIX_TRY(mark(p, FIX_STAGE_BWD_DG, 0, st));
-  chunk_total_kernel<<<dim3(d.nchunks, d.Hkv, (d.Dv + 31) / 32), 128, 0, st>>>(d, chunks, dG, dtot);
+  chunk_total_kernel<<<dim3(d.nchunks, d.Hkv, (d.Dv + 31) / 32), 256, 0, st>>>(d, chunks, dG, dtot);
   FIX_TRY(launched());
   float* dgf = d.scalar_gate ? reinterpret_cast<float*>(base + ws.dgf) : dg;
-  reverse_cumsum_kernel<<<dim3(d.nchunks, d.Hkv, (d.Dv + 31) / 32), 128, 0, st>>>(d, chunks, dG,
+  reverse_cumsum_kernel<<<dim3(d.nchunks, d.Hkv, (d.Dv + 31) / 32), 256, 0, st>>>(d, chunks, dG,
                                                                                  dtot, dgf);
   FIX_TRY(launched());
   if (d.scalar_gate) {

@@ -29,11 +29,11 @@ template __global__ void upload_kernel<4096>(const __grid_constant__ Blob<4096>,
 template __global__ void upload_kernel<kBlobMaxWords>(const __grid_constant__ Blob<kBlobMaxWords>,
                                                       uint32_t*, int);
 
-// grid (nchunks, Hkv, ceil(Dv / 32)), block 128: a CTA takes 32 channels of
-// one chunk and kv head, thread = (row group of 32 rows, channel); the four
-// groups are scanned in parallel and joined through shared memory.  Small
-// CTAs keep several per SM, so that one CTA's loads overlap another's scan
-// and stores.
+// grid (nchunks, Hkv, ceil(Dv / 32)), block 256: a CTA takes 32 channels of
+// one chunk and kv head, thread = (row group of 16 rows, channel); the eight
+// groups are scanned in parallel and joined through shared memory.  Few
+// registers per thread keep many warps per SM, so that many loads are in
+// flight and one CTA's loads overlap another's scan and stores.
 //
 // Besides L and tot, the tensor-core path needs:
 //   Vt_s[c] = v_s[c] * exp(tot[c] - L_s[c])     values pre-decayed to the chunk's
@@ -51,8 +51,9 @@ template __global__ void upload_kernel<kBlobMaxWords>(const __grid_constant__ Bl
 // so that exp(G_t - G_s) = exp(L_t - rho) * exp(rho - L_s) with both factors
 // inside [e^-hr, e^hr].  Channels with hr > FIX_HR_MAX or |rho| > FIX_RHO_MAX
 // are out of range (see fix_common.cuh): Vm = 0, rho = 0, hr = FIX_HR_BAD.
-constexpr int kPrefixThreads = 128;
-constexpr int kPrefixRows = FIX_CHUNK / 4;     // rows per thread
+constexpr int kPrefixThreads = 256;
+constexpr int kPrefixGroups = kPrefixThreads / 32;        // row groups of 32 channels
+constexpr int kPrefixRows = FIX_CHUNK / kPrefixGroups;    // rows per thread
 
 __global__ void __launch_bounds__(kPrefixThreads) prefix_kernel(
     Dims d, const Chunk* __restrict__ chunks, const float* __restrict__ g,
@@ -105,7 +106,7 @@ __global__ void __launch_bounds__(kPrefixThreads) prefix_kernel(
   __syncthreads();
   float off = 0.f, total = 0.f, cmin = INFINITY, cmax = -INFINITY;
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
+  for (int q = 0; q < kPrefixGroups; ++q) {
     const float pq = part[q * 32 + cl];
     if (q < grp) off += pq;
     cmin = fminf(cmin, total + pmin[q * 32 + cl]);
@@ -138,7 +139,7 @@ __global__ void __launch_bounds__(kPrefixThreads) prefix_kernel(
   if (__syncthreads_or(!good) && threadIdx.x == 0) atomicOr(badflag, 1);
   float cx = 0.f;
 #pragma unroll
-  for (int q = 0; q < 4; ++q) cx = fmaxf(cx, part[q * 32 + cl]);
+  for (int q = 0; q < kPrefixGroups; ++q) cx = fmaxf(cx, part[q * 32 + cl]);
   const float lg = cx > 0.f ? log2f(cx) : -1e30f;
   const float sc = exp2f(-vt_exponent(lg));
   if (grp == 0 && act) {
@@ -162,7 +163,7 @@ __global__ void __launch_bounds__(kPrefixThreads) prefix_kernel(
 // Reverse cumsum of dG within each sequence (dg_r = sum_{t >= r} dG_t), in two
 // launches over the same chunk table: chunk totals, then local reverse scans
 // plus the totals of the later chunks of the same sequence.  Both use the
-// prefix pass's block shape: grid (nchunks, Hkv, ceil(Dv / 32)), 128 threads =
+// prefix pass's block shape: grid (nchunks, Hkv, ceil(Dv / 32)), 256 threads =
 // (row group, channel), every row of a group loaded up front, groups joined
 // through shared memory.
 __global__ void __launch_bounds__(kPrefixThreads) chunk_total_kernel(Dims d,
@@ -191,7 +192,7 @@ __global__ void __launch_bounds__(kPrefixThreads) chunk_total_kernel(Dims d,
   if (grp == 0 && act) {
     float t = 0.f;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) t += part[q * 32 + cl];
+    for (int q = 0; q < kPrefixGroups; ++q) t += part[q * 32 + cl];
     tot[((size_t)ci * d.Hkv + kv) * Dv + c] = t;
   }
 }
@@ -237,7 +238,7 @@ __global__ void __launch_bounds__(kPrefixThreads) reverse_cumsum_kernel(
   part[threadIdx.x] = own;
   __syncthreads();
   // then the later row groups of this chunk, from the last one down
-  for (int q = 3; q > grp; --q) acc += part[q * 32 + cl];
+  for (int q = kPrefixGroups - 1; q > grp; --q) acc += part[q * 32 + cl];
 #pragma unroll
   for (int u = kPrefixRows - 1; u >= 0; --u)
     if (u < nr) {

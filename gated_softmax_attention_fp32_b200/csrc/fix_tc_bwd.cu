@@ -101,6 +101,15 @@ __device__ __forceinline__ uint4 pack8(const float* x, bool f16) {
   }
   return r;
 }
+// Whether 8 scale factors are normal fp16 numbers no larger than 2, so that a
+// packed fp16 multiply by them loses nothing to range.
+__device__ __forceinline__ bool f16_factors(const float* f) {
+  bool ok = true;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) ok = ok && f[e] >= 6.2e-5f && f[e] <= 2.f;
+  return ok;
+}
+
 __device__ __forceinline__ void unpack8(uint4 u, bool f16, float* x) {
   const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
@@ -394,13 +403,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int e = 0; e < 8; ++e) f8[e] = ex2(delta[e] * LOG2E + vt_exponent(lv[e]));
       if (!mbar_wait(&bar->v_full[st], (it >> 1) & 1, ctl)) break;
       uint8_t* vb = reinterpret_cast<uint8_t*>(sV + st * BN * DV);
-      for (int rr = r0; rr < BN; rr += kRowsPerPass) {
-        uint4* p = reinterpret_cast<uint4*>(vb + sw_off(BN, rr, lc * 8));
-        float x[8];
-        unpack8(*p, true, x);
+      if (cta_f16 && f16_factors(f8)) {
+        // fp16 in and out: packed multiplies, no conversions
+        __half2 fh[4];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) x[e] *= f8[e];
-        *p = pack8(x, cta_f16);
+        for (int u = 0; u < 4; ++u) fh[u] = __floats2half2_rn(f8[2 * u], f8[2 * u + 1]);
+        for (int rr = r0; rr < BN; rr += kRowsPerPass) {
+          uint4* p = reinterpret_cast<uint4*>(vb + sw_off(BN, rr, lc * 8));
+          uint4 xv = *p;
+          __half2* hx = reinterpret_cast<__half2*>(&xv);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) hx[u] = __hmul2(hx[u], fh[u]);
+          *p = xv;
+        }
+      } else {
+        for (int rr = r0; rr < BN; rr += kRowsPerPass) {
+          uint4* p = reinterpret_cast<uint4*>(vb + sw_off(BN, rr, lc * 8));
+          float x[8];
+          unpack8(*p, true, x);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) x[e] *= f8[e];
+          *p = pack8(x, cta_f16);
+        }
       }
       fence_proxy_async_smem();
       mbar_arrive(&bar->v_ready[st]);
@@ -873,13 +897,28 @@ __global__ void __launch_bounds__(kThreads, 1)
           // are zeroed
           const bool in_f16 = cur.in_f16 != 0;
           uint8_t* xb = sX(st);
-          for (int rr = r0; rr < BQ; rr += kRowsPerPass) {
-            uint4* p = reinterpret_cast<uint4*>(xb + sw_off(BQ, rr, lc * 8));
-            float x[8];
-            unpack8(*p, in_f16, x);
+          if (in_f16 && cta_f16 && f16_factors(f8)) {
+            // fp16 in and out: packed multiplies, no conversions
+            __half2 fh[4];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) x[e] = rr < qlen ? x[e] * f8[e] : 0.f;
-            *p = pack8(x, cta_f16 != 0);
+            for (int u = 0; u < 4; ++u) fh[u] = __floats2half2_rn(f8[2 * u], f8[2 * u + 1]);
+            for (int rr = r0; rr < BQ; rr += kRowsPerPass) {
+              uint4* p = reinterpret_cast<uint4*>(xb + sw_off(BQ, rr, lc * 8));
+              uint4 xv = *p;
+              __half2* hx = reinterpret_cast<__half2*>(&xv);
+#pragma unroll
+              for (int u = 0; u < 4; ++u) hx[u] = __hmul2(hx[u], fh[u]);
+              *p = rr < qlen ? xv : make_uint4(0u, 0u, 0u, 0u);
+            }
+          } else {
+            for (int rr = r0; rr < BQ; rr += kRowsPerPass) {
+              uint4* p = reinterpret_cast<uint4*>(xb + sw_off(BQ, rr, lc * 8));
+              float x[8];
+              unpack8(*p, in_f16, x);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) x[e] = rr < qlen ? x[e] * f8[e] : 0.f;
+              *p = pack8(x, cta_f16 != 0);
+            }
           }
           fence_proxy_async_smem();
         }

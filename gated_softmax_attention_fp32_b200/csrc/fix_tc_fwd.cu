@@ -682,20 +682,45 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 8; ++e) f8[e] = ex2(delta[e] * LOG2E + vt_exponent(lv[e]) - kexp[e]);
         }
+        // factors in fp16 when they are normal fp16 numbers (always with g <=
+        // 0): then V'' = Vt f is one packed fp16 multiply per channel pair on
+        // the FMA pipe, with no conversion; otherwise in fp32
+        bool h16 = true;
+        __half2 fh[4];
+        if (!diag) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            h16 = h16 && f8[2 * u] >= 6.2e-5f && f8[2 * u + 1] >= 6.2e-5f && f8[2 * u] <= 2.f &&
+                  f8[2 * u + 1] <= 2.f;
+            fh[u] = __floats2half2_rn(f8[2 * u], f8[2 * u + 1]);
+          }
+        }
         if (!wg_and(2, mbar_wait(&bar->v_full[sv], (vc >> 1) & 1, ctl))) { ok = false; break; }
         if (!diag) {
           uint8_t* vb = reinterpret_cast<uint8_t*>(sV + sv * BN * DV) + half * (BN * 128);
+          if (h16) {
 #pragma unroll 4
-          for (int s = r0; s < BN; s += kRowsPerPass) {
-            uint4* p = reinterpret_cast<uint4*>(vb + s * 128 + ((lcc ^ (s & 7)) << 4));
-            uint4 xv = *p;
-            uint32_t w4[4] = {xv.x, xv.y, xv.z, xv.w};
+            for (int s = r0; s < BN; s += kRowsPerPass) {
+              uint4* p = reinterpret_cast<uint4*>(vb + s * 128 + ((lcc ^ (s & 7)) << 4));
+              uint4 xv = *p;
+              __half2* hx = reinterpret_cast<__half2*>(&xv);
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const float2 ab = __half22float2(*reinterpret_cast<const __half2*>(&w4[u]));
-              w4[u] = pack_f16(ab.x * f8[2 * u], ab.y * f8[2 * u + 1]);
+              for (int u = 0; u < 4; ++u) hx[u] = __hmul2(hx[u], fh[u]);
+              *p = xv;
             }
-            *p = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+          } else {
+#pragma unroll 4
+            for (int s = r0; s < BN; s += kRowsPerPass) {
+              uint4* p = reinterpret_cast<uint4*>(vb + s * 128 + ((lcc ^ (s & 7)) << 4));
+              uint4 xv = *p;
+              uint32_t w4[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                const float2 ab = __half22float2(*reinterpret_cast<const __half2*>(&w4[u]));
+                w4[u] = pack_f16(ab.x * f8[2 * u], ab.y * f8[2 * u + 1]);
+              }
+              *p = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+            }
           }
           fence_proxy_async_smem();
         }
@@ -717,7 +742,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __nv_bfloat16* __restrict__ yb = P.y_f32 ? nullptr : reinterpret_cast<__nv_bfloat16*>(P.y);
     const size_t ors = (size_t)d.Hq * DV;
     constexpr int kU = DV / 32;                      // 32-channel chunks
-    constexpr int kR = 8;                            // rows per pass
+    constexpr int kR = 4;                            // rows per pass
     int nt = 0;
     bool ok = true;
     for (int round = 0; ok && round < rounds; ++round) {
@@ -726,6 +751,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Tile x = tile_info(P, t);
       if (x.len <= 0) continue;
       const int tb = nt & 1, use = nt >> 1;
+      const float* Lg = P.L + (size_t)x.kv * DV;
+      const __nv_bfloat16* vg = P.v + (size_t)x.kv * DV;
+      // While the tile's MMAs run, pull its rows of L, v (and the output
+      // gate) into L2, so that the loads below hit L2: one row per thread.
+      if (et < x.len) {
+        const size_t tk = (size_t)x.tok0 + et;
+        const char* lr = reinterpret_cast<const char*>(Lg + tk * vrs);
+        const char* vr = reinterpret_cast<const char*>(vg + tk * vrs);
+#pragma unroll
+        for (int b = 0; b < DV * 4; b += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(lr + b));
+#pragma unroll
+        for (int b = 0; b < DV * 2; b += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(vr + b));
+        if (P.z) {
+          const char* zr = reinterpret_cast<const char*>(P.z + (tk * d.Hq + x.h) * DV);
+#pragma unroll
+          for (int b = 0; b < DV * 2; b += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(zr + b));
+        }
+      }
       // channel data of this tile (the previous tile's readers are done:
       // every epilogue thread passed the sync at the end of that tile)
       if (et < DV) {
@@ -742,11 +785,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const float* rows = sRows + tb * 4 * BM;
       const uint32_t acol = lane_base + 256u + (uint32_t)(tb * DV);
-      const float* Lg = P.L + (size_t)x.kv * DV;
-      const __nv_bfloat16* vg = P.v + (size_t)x.kv * DV;
 #pragma unroll 1
       for (int grp = 0; grp < 32 / kR; ++grp) {
         const int rbase = ew * 32 + grp * kR;          // first tile row of this pass
+        // L and v of the pass's rows for every chunk, all loads in flight at
+        // once (lanes over channels: coalesced)
+        float lt[kU][kR], vt[kU][kR];
+#pragma unroll
+        for (int u = 0; u < kU; ++u)
+#pragma unroll
+          for (int q = 0; q < kR; ++q) {
+            const int rr = min(rbase + q, x.len - 1);
+            const size_t tk = (size_t)x.tok0 + rr;
+            lt[u][q] = Lg[tk * vrs + u * 32 + lane];
+            vt[u][q] = bf2f(vg[tk * vrs + u * 32 + lane]);
+          }
         float o[kR][kU];
         float ss[kR];
 #pragma unroll
@@ -754,15 +807,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int u = 0; u < kU; ++u) {
           const int c = u * 32 + lane;
-          // L and v of the pass's rows (lanes over channels: coalesced)
-          float lt[kR], vt[kR];
-#pragma unroll
-          for (int q = 0; q < kR; ++q) {
-            const int rr = min(rbase + q, x.len - 1);
-            const size_t tk = (size_t)x.tok0 + rr;
-            lt[q] = Lg[tk * vrs + c];
-            vt[q] = bf2f(vg[tk * vrs + c]);
-          }
           // A columns [32u, 32u + 32) of the warp's 32 rows, transposed
           uint32_t xa[32];
           tmem_ld32(acol + u * 32, xa);
@@ -780,8 +824,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int q = 0; q < kR; ++q) {
             const float a = tr[q * 33 + lane];
             const float alpha = rows[rbase + q], ptt = rows[BM + rbase + q];
-            const float fac = bc ? 1.f : ex2((lt[q] - rc) * LOG2E);
-            const float val = alpha * fac * a + ptt * vt[q];
+            const float fac = bc ? 1.f : ex2((lt[u][q] - rc) * LOG2E);
+            const float val = alpha * fac * a + ptt * vt[u][q];
             o[q][u] = val;
             ss[q] += val * val;
           }

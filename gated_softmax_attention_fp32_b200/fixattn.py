@@ -82,7 +82,7 @@ def load():
     lib.fix_attn_noalloc_device_status.restype = ctypes.c_int
     lib.fix_attn_decode_workspace_bytes.argtypes = [P]
     lib.fix_attn_decode_workspace_bytes.restype = sz
-    lib.fix_attn_decode.argtypes = [P] + [vp] * 10 + [sz, vp]
+    lib.fix_attn_decode.argtypes = [P] + [vp] * 9 + [sz, vp]
     lib.fix_attn_decode.restype = ctypes.c_int
     lib.fix_attn_kernel_count.argtypes = [P, ctypes.c_int]
     lib.fix_attn_kernel_count.restype = ctypes.c_int
