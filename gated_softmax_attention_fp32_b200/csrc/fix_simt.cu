@@ -175,7 +175,7 @@ __global__ void __launch_bounds__(256) fwd_simt_kernel(
 // ---------------------------------------------------------------------------
 constexpr int kPreWarps = 8;
 
-__global__ void __launch_bounds__(kPreWarps * 32) bwd_pre_kernel(
+__global__ void __launch_bounds__(kPreWarps * 32, 3) bwd_pre_kernel(
     Dims d, const Chunk* __restrict__ chunks, const __nv_bfloat16* __restrict__ q,
     const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
     const float* __restrict__ o_s, const float* __restrict__ m_s,

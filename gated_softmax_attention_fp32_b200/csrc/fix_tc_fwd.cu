@@ -522,10 +522,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_ld32(sbase + c4 * 32, xs);
             tmem_wait_ld();
             float ls = 0.f;
+            // half of the exponentials on the MUFU unit, half as a polynomial
+            // on the FMA pipe (both well inside fp16's rounding)
 #pragma unroll
             for (int e = 0; e < 32; e += 2) {
               const float p0 = ex2(__uint_as_float(xs[e]) * c1 - moff);
-              const float p1 = ex2(__uint_as_float(xs[e + 1]) * c1 - moff);
+              const float p1 = exp2_poly3(__uint_as_float(xs[e + 1]) * c1 - moff);
               ls += p0 + p1;
               pk[e >> 1] = pack_f16(p0, p1);
             }

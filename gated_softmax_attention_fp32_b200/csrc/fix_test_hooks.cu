@@ -8,10 +8,17 @@
 // status word, leave every role, release TMEM -- and the next ordinary call
 // must succeed.  This exercises the device-side failure detection without a
 // GPU fault or a hang.
+//
+// fix_attn_test_exp2_poly(x, out, n, stream) evaluates the forward's
+// polynomial 2^x on n device floats, so that a test can hold it to its error
+// bound against exact powers of two.
 #ifdef FIX_TEST_HOOKS
+#include <cuda_runtime.h>
+
 #include <atomic>
 
 #include "fix_internal.h"
+#include "fix_sm100.cuh"
 
 namespace fix {
 static std::atomic<int> g_stall{0};
@@ -19,4 +26,17 @@ int test_stall_forward() { return g_stall.load(); }
 }  // namespace fix
 
 extern "C" void fix_attn_test_stall_forward(int on) { fix::g_stall.store(on ? 1 : 0); }
+
+namespace {
+__global__ void exp2_poly_kernel(const float* __restrict__ x, float* __restrict__ out, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) out[i] = fix::sm100::exp2_poly3(x[i]);
+}
+}  // namespace
+
+extern "C" int fix_attn_test_exp2_poly(const float* x, float* out, int n, void* stream) {
+  if (n <= 0) return 0;
+  exp2_poly_kernel<<<(n + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, out, n);
+  return cudaGetLastError() == cudaSuccess ? 0 : 1;
+}
 #endif
