@@ -350,7 +350,7 @@ def _decode_ref(case, lengths, o_gate=None, o_norm=True):
     ys = []
     for b, L in enumerate(lengths):
         sub = sequence_case(case, b, 0, L)
-        z = None if o_gate is None else o_gate[b:b + 1, :, None].expand(1, L, -1, -1).contiguous()
+        z = None if o_gate is None else o_gate[b:b + 1, None].expand(1, L, -1, -1).contiguous()
         ref = oracle_full(sub, o_gate=z, o_norm=o_norm)
         ys.append(ref["y"][0, L - 1])
     return np.stack(ys)
