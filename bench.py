@@ -4,7 +4,7 @@
                     [--impl fix|reference] [--algo auto|simt|tc]
 
 A step is one pass of the whole hot path over one batch of synthetic input.
-For the training workloads (2, 3, 5) that is fix_attn_fwd (training mode:
+For the training workloads (2, 3, 5, 6) that is fix_attn_fwd (training mode:
 saves o, m, rstd) then fix_attn_bwd, i.e. gate prefix sums, attention forward
 with the fused RMSNorm, RMSNorm backward, dq, dk/dv/dG and the reverse cumsum
 of dG; for the forward-only workloads (1, 4) it is one inference fix_attn_fwd

@@ -573,12 +573,9 @@ fix_status fix_attn_bwd(const fix_attn_problem* p, const void* q, const void* k,
     ta.dG = dG;
     ta.status = reinterpret_cast<int*>(base + ws.status);
   }
-  // With the tensor-core kernels the exact kernels stay launched but return at
-  // once unless the prefix pass flagged a channel outside the split's range.
-  const int* gate = tc ? badflag : nullptr;
   const size_t smq = simt_dq_smem(d), smkv = simt_dkv_smem(d);
-  if (!set_smem_limit(reinterpret_cast<const void*>(dq_simt_kernel), (int)smq) ||
-      !set_smem_limit(reinterpret_cast<const void*>(dkv_simt_kernel), (int)smkv))
+  if (!tc && (!set_smem_limit(reinterpret_cast<const void*>(dq_simt_kernel), (int)smq) ||
+              !set_smem_limit(reinterpret_cast<const void*>(dkv_simt_kernel), (int)smkv)))
     return FIX_ERR_CUDA;
   FIX_TRY(mark(p, FIX_STAGE_BWD_DQ, 0, st));
   if (tc) FIX_TRY(tc_bwd(p, d, ta, 0, st));
@@ -597,17 +594,7 @@ fix_status fix_attn_bwd(const fix_attn_problem* p, const void* q, const void* k,
   FIX_TRY(launched());
   FIX_TRY(mark(p, FIX_STAGE_BWD_DKV, 1, st));
   FIX_TRY(mark(p, FIX_STAGE_BWD_FINISH, 0, st));
-  if (tc) {
-    FIX_TRY(tc_bwd(p, d, ta, 2, st));
-    dq_simt_kernel<<<dim3(d.nchunks * 4, d.Hq), 256, smq, st>>>(
-        d, chunks, qb, kb, vb, L, tot, m_s, dow, d.no_norm ? delta : nullptr,
-        static_cast<__nv_bfloat16*>(dq), gate);
-    FIX_TRY(launched());
-    dkv_simt_kernel<<<dim3(d.nchunks * 4, d.Hkv), 256, smkv, st>>>(
-        d, chunks, qb, kb, vb, L, tot, m_s, dow, d.no_norm ? delta : nullptr, A,
-        static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv), dG, gate);
-    FIX_TRY(launched());
-  }
+  if (tc) FIX_TRY(tc_bwd(p, d, ta, 2, st));
   FIX_TRY(mark(p, FIX_STAGE_BWD_FINISH, 1, st));
   FIX_TRY(mark(p, FIX_STAGE_BWD_DG, 0, st));
   chunk_total_kernel<<<dim3(d.nchunks, d.Hkv, (d.Dv + 31) / 32), 256, 0, st>>>(d, chunks, dG, dtot);
@@ -644,11 +631,12 @@ int fix_attn_kernel_count(const fix_attn_problem* p, int backward) {
   const int upB = (tc && d.nchunks) ? upload_launches(ws.cpart - ws.parts + (size_t)d.nchunks * 8) : 0;
   // schedule uploads (the split only when the forward's tables are reused),
   // the prefix pass unless reused, the preprocess (2, or 3 with the
-  // tensor-core operands), tensor-core dq / dk/dv / combine, the exact
-  // kernels (2), the dG reverse cumsum (2)
+  // tensor-core operands), then either tensor-core dq / dk/dv / exact
+  // out-of-range terms / combine or the exact kernels (2), the dG reverse
+  // cumsum (2)
   const bool has_dw = !d.no_norm;   // dw is optional only without the norm
   return (reuse ? 0 : upA + 1) + upB + (tc ? 2 : 1) + (has_dw ? 1 : 0) +
-         (tc ? tc_bwd_kernel_count(d, sp.nslots) : 0) + 2 + 2 + (d.scalar_gate ? 1 : 0);
+         (tc ? tc_bwd_kernel_count(d, sp.nslots) : 2) + 2 + (d.scalar_gate ? 1 : 0);
 }
 
 fix_status fix_attn_device_status(const void* workspace, void* stream) {

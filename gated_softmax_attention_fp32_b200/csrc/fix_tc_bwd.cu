@@ -31,8 +31,10 @@
 //   key chunk's slots in order and finishes
 //   dv_strict = exp(rho - L_s) dV_d + exp(tot_j - L_s) dV_o,
 //   dv = dv_strict + sum_h P_ss do_s, dG = A - v dv_strict, dk = scale dK.
-// Problems with a channel outside the split's float range (flag set by the
-// prefix pass) are left to the exact CUDA-core kernels, which run instead.
+// Channels outside the split's float range (flagged by the prefix pass) have
+// no diagonal operands; their diagonal terms are added exactly in fp32: by
+// the dq kernel's dS warps into dP, and by dkv_diag_exact_kernel into the
+// dk/dv slots.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -152,7 +154,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                  const __grid_constant__ CUtensorMap tm_domh, const __grid_constant__ CUtensorMap tm_dot,
                  const Params P) {
   using Lay = DqLayout<DK, DV>;
-  if (*P.badflag) return;  // exact kernels run instead
+  // channels of this chunk outside the split's range (bit c of word c / 32):
+  // their diagonal terms are missing from the MMA's dP and are added exactly
+  __shared__ uint32_t sBadMask[4];
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -193,6 +197,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_fence_init();
   }
   if (warp == 1) tmem_alloc(sTmem, kTmemCols);
+  if (warp < 4) {
+    const int c = tid;
+    const bool bad = c < DV && *P.badflag != 0 &&
+                     P.hr[((size_t)ci * d.Hkv + kv) * DV + c] > FIX_HR_MAX;
+    const uint32_t m = __ballot_sync(0xffffffffu, bad);
+    if (lane == 0) sBadMask[warp] = m;
+  }
   bool my_safe = true;
   for (int jj = tid; jj < nblk; jj += blockDim.x)
     my_safe = my_safe && P.safe[(size_t)(first + jj) * d.Hkv + kv];
@@ -299,6 +310,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float c1 = d.scale * LOG2E;
     // without the norm: dS = P (dP - sum_c do o) (the softmax denominator)
     const float dl = P.delta ? P.delta[tok * d.Hq + h] : 0.f;
+    const bool any_bad = (sBadMask[0] | sBadMask[1] | sBadMask[2] | sBadMask[3]) != 0;
+    const size_t vrs = (size_t)d.Hkv * DV;
     bool ok = true;
     for (int it = 0; it < nblk; ++it) {
       if (!__all_sync(0xffffffffu, mbar_wait(&bar->s_full, it & 1, ctl))) { ok = false; break; }
@@ -319,6 +332,32 @@ __global__ void __launch_bounds__(kThreads, 1)
             pk[e >> 1] = pack_bf16(p0 * (__uint_as_float(xp[e]) - dl), p1 * (__uint_as_float(xp[e + 1]) - dl));
           }
         } else {
+          if (any_bad) {
+            // out-of-range channels c: dP_ts += do_t[c] exp(L_t[c] - L_s[c])
+            // v_s[c] for keys s <= t, in fp32 (L_s, v_s are the same address
+            // across the warp)
+            const float* Lc = P.L + (size_t)ch.tok0 * vrs + (size_t)kv * DV;
+            const __nv_bfloat16* vc = P.v + (size_t)ch.tok0 * vrs + (size_t)kv * DV;
+            const int kmax = min(r, ch.len - 1);
+#pragma unroll 1
+            for (int w = 0; w < DV / 32; ++w) {
+              uint32_t msk = sBadMask[w];
+              while (msk) {
+                const int c = w * 32 + __ffs(msk) - 1;
+                msk &= msk - 1;
+                const float dtc = row_ok ? P.do_ws[tok * (size_t)d.Hq * DV + (size_t)h * DV + c] : 0.f;
+                const float ltc = P.L[tok * vrs + (size_t)kv * DV + c];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                  const int key = c4 * 32 + e;
+                  if (key <= kmax) {
+                    const float f = ex2((ltc - Lc[(size_t)key * vrs + c]) * LOG2E);
+                    xp[e] = __float_as_uint(__uint_as_float(xp[e]) + dtc * f * bf2f(vc[(size_t)key * vrs + c]));
+                  }
+                }
+              }
+            }
+          }
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
             const int key = c4 * 32 + e;
@@ -486,7 +525,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                   const __grid_constant__ CUtensorMap tm_domh, const __grid_constant__ CUtensorMap tm_doml,
                   const __grid_constant__ CUtensorMap tm_dot, const Params P) {
   using Lay = KvLayout<DK, DV>;
-  if (*P.badflag) return;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -986,7 +1024,6 @@ __device__ __forceinline__ void stb(__nv_bfloat16* p, const float* x) {
 // one coalesced stretch.
 template <int DK, int DV>
 __global__ void __launch_bounds__(256) dkv_combine_kernel(const Params P) {
-  if (*P.badflag) return;
   const Dims& d = P.d;
   constexpr int kRowBlocks = BN / 8;
   const int ci = blockIdx.x / kRowBlocks, kv = blockIdx.y, lane = threadIdx.x & 31;
@@ -1036,26 +1073,254 @@ __global__ void __launch_bounds__(256) dkv_combine_kernel(const Params P) {
 #pragma unroll
     for (int e = 0; e < VV; ++e) diag[e] += pss * dw[e];
   }
-  // dv_strict = exp(rho - L_s) dV_d + exp(tot - L_s) dV_o;
+  // dv_strict = exp(rho - L_s) dV_d + exp(tot - L_s) dV_o (dV_d of a channel
+  // outside the split's range is already exact: factor 1);
   // dv = dv_strict + the s = t terms, dG = A - v dv_strict
   const size_t cb = ((size_t)ci * d.Hkv + kv) * DV + cv, rb = tok * vrs + (size_t)kv * DV + cv;
   const bool has_off = ch.nch - ch.j > 1;
-  float ls[VV], rh[VV], tt[VV], av[VV], vv[VV];
+  float ls[VV], rh[VV], hr[VV], tt[VV], av[VV], vv[VV];
   ldf<VV>(P.L + rb, ls);
   ldf<VV>(P.rho + cb, rh);
+  ldf<VV>(P.hr + cb, hr);
   ldf<VV>(P.tot + cb, tt);
   ldf<VV>(P.A + rb, av);
   ldb<VV>(P.v + rb, vv);
   float dvv[VV], dgv[VV];
 #pragma unroll
   for (int e = 0; e < VV; ++e) {
-    float strict = fd[e] * ex2((rh[e] - ls[e]) * LOG2E);
+    float strict = hr[e] > FIX_HR_MAX ? fd[e] : fd[e] * ex2((rh[e] - ls[e]) * LOG2E);
     if (has_off) strict += fo[e] * ex2((tt[e] - ls[e]) * LOG2E);
     dvv[e] = strict + diag[e];
     dgv[e] = av[e] - vv[e] * strict;
   }
   stb<VV>(P.dv + rb, dvv);
   stf<VV>(P.dG + rb, dgv);
+}
+
+// ======================================================= out-of-range channels
+// A channel whose in-chunk range exceeds the split's float range (hr > 80 or
+// |rho| > 80) has Vm = 0 and dOm = 0 on the diagonal block, so the dk/dv
+// kernel's diagonal parts leave out its terms:
+//   dP_ts  gains  sum_{c bad} do_t[c] exp(L_t[c] - L_s[c]) v_s[c]   (s <= t),
+//   so dK_s gains sum_t P_ts dP^bad_ts q_t,  and
+//   dv_s[c] (c bad) gets its diagonal part sum_{t > s} P_ts exp(L_t[c] - L_s[c]) do_t[c].
+// This kernel adds them, in fp32 on the CUDA cores, to the first diagonal
+// slot of the key chunk (its dV columns of bad channels hold exact zeros,
+// and the combine takes them unscaled).  One CTA per (chunk, kv head); CTAs
+// of chunks without such a channel return at once.  P is recomputed from q,
+// k and the saved row maxima as in the tensor-core kernels.
+constexpr int kFixThreads = 256;
+constexpr int kFixBatch = 8;      // bad channels staged per pass
+
+template <int DK, int DV>
+struct FixLayout {
+  static constexpr int kPs = BN + 4;                          // sP row stride (floats)
+  static constexpr int kQt = 0;                               // [DK][BN] f32, q transposed
+  static constexpr int kKt = kQt + DK * BN * 4;               // [DK][BN] f32, k transposed
+  static constexpr int kP = kKt + DK * BN * 4;                // [BN][kPs] f32: P, then dS^bad
+  static constexpr int kL = kP + BN * kPs * 4;                // [kFixBatch][BN] L of the batch
+  static constexpr int kV = kL + kFixBatch * BN * 4;          // [kFixBatch][BN] v
+  static constexpr int kDo = kV + kFixBatch * BN * 4;         // [kFixBatch][BN] do (one head)
+  static constexpr int kM = kDo + kFixBatch * BN * 4;         // [BN] row maxima (one head)
+  static constexpr int kIdx = kM + BN * 4;                    // [DV] bad channel list
+  static constexpr int kBytes = kIdx + DV * 4 + 16;
+  static_assert(kBytes <= 232448, "shared memory");
+};
+
+template <int DK, int DV>
+__global__ void __launch_bounds__(kFixThreads, 1) dkv_diag_exact_kernel(const Params P) {
+  using Lay = FixLayout<DK, DV>;
+  if (*P.badflag == 0) return;
+  extern __shared__ __align__(16) uint8_t fsm[];
+  const Dims& d = P.d;
+  const int ci = blockIdx.x, kv = blockIdx.y;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const Chunk ch = P.chunks[ci];
+  const int n = ch.len;
+  const int2 cp = P.cpart[ci];
+  if (n <= 0 || cp.x < 1 || cp.y < 0 || cp.y >= P.nslots) return;
+  float* sQt = reinterpret_cast<float*>(fsm + Lay::kQt);
+  float* sKt = reinterpret_cast<float*>(fsm + Lay::kKt);
+  float* sP = reinterpret_cast<float*>(fsm + Lay::kP);
+  float* sL = reinterpret_cast<float*>(fsm + Lay::kL);
+  float* sV = reinterpret_cast<float*>(fsm + Lay::kV);
+  float* sDo = reinterpret_cast<float*>(fsm + Lay::kDo);
+  float* sM = reinterpret_cast<float*>(fsm + Lay::kM);
+  int* sIdx = reinterpret_cast<int*>(fsm + Lay::kIdx);
+  int* sNb = sIdx + DV;
+  uint32_t* sMask = reinterpret_cast<uint32_t*>(sNb + 1);
+  // the chunk's bad channels, in channel order
+  if (warp < 4) {
+    const int c = tid;
+    const bool bad = c < DV && P.hr[((size_t)ci * d.Hkv + kv) * DV + c] > FIX_HR_MAX;
+    const uint32_t m = __ballot_sync(0xffffffffu, bad);
+    if (lane == 0) sMask[warp] = m;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int nb = 0;
+    for (int w = 0; w < DV / 32; ++w)
+      for (uint32_t m = sMask[w]; m; m &= m - 1) sIdx[nb++] = w * 32 + __ffs(m) - 1;
+    *sNb = nb;
+  }
+  __syncthreads();
+  const int nbad = *sNb;
+  if (nbad == 0) return;
+
+  const size_t qrs = (size_t)d.Hq * DK, krs = (size_t)d.Hkv * DK;
+  const size_t vrs = (size_t)d.Hkv * DV, ors = (size_t)d.Hq * DV;
+  const size_t tok0 = (size_t)ch.tok0;
+  // k of the chunk, transposed (rows past its end are zero)
+  for (int i = tid; i < BN * DK; i += kFixThreads) {
+    const int r = i / DK, c = i % DK;
+    sKt[c * BN + r] = r < n ? bf2f(P.k[(tok0 + r) * krs + (size_t)kv * DK + c]) : 0.f;
+  }
+  // dK accumulator: keys 4 sq .. 4 sq + 3, columns cb * CK .. + CK
+  constexpr int CK = DK / 8;
+  const int sq = tid % 32, cb = tid / 32;
+  float dk[4][CK];
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int e = 0; e < CK; ++e) dk[a][e] = 0.f;
+  // P / dS block of this thread: rows 8 tb .. + 7, keys 8 sb .. + 7
+  const int tb = tid / 16, sb = tid % 16;
+  // dv of a batch: key s_dv, batch channels 4 cg .. 4 cg + 3
+  const int s_dv = tid % BN, cg = tid / BN;
+  const int t_dv = s_dv & ~31;               // first query row of the warp's keys
+  const float c1 = d.scale * LOG2E;
+  float* slot = P.partial + ((size_t)cp.y * d.Hkv + kv) * BN * (DK + DV);
+
+  for (int hh = 0; hh < d.grp; ++hh) {
+    const int h = kv * d.grp + hh;
+    __syncthreads();
+    for (int i = tid; i < BN * DK; i += kFixThreads) {
+      const int r = i / DK, c = i % DK;
+      sQt[c * BN + r] = r < n ? bf2f(P.q[(tok0 + r) * qrs + (size_t)h * DK + c]) : 0.f;
+    }
+    for (int r = tid; r < BN; r += kFixThreads) sM[r] = r < n ? P.m_s[(tok0 + r) * d.Hq + h] : 0.f;
+    __syncthreads();
+    // P_ts for s <= t < n, else 0
+    {
+      float acc[8][8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+      if (sb <= tb) {
+#pragma unroll 2
+        for (int c = 0; c < DK; ++c) {
+          const float4 q0 = *reinterpret_cast<const float4*>(sQt + c * BN + 8 * tb);
+          const float4 q1 = *reinterpret_cast<const float4*>(sQt + c * BN + 8 * tb + 4);
+          const float4 k0 = *reinterpret_cast<const float4*>(sKt + c * BN + 8 * sb);
+          const float4 k1 = *reinterpret_cast<const float4*>(sKt + c * BN + 8 * sb + 4);
+          const float qa[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+          const float ka[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(qa[i], ka[j], acc[i][j]);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int t = 8 * tb + i;
+        const float mo = sM[t] * LOG2E;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int sk = 8 * sb + j;
+          sP[t * Lay::kPs + sk] = (sk <= t && t < n) ? ex2(acc[i][j] * c1 - mo) : 0.f;
+        }
+      }
+    }
+    // dP^bad over all bad channels, batch by batch
+    float dp[8][8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) dp[i][j] = 0.f;
+    for (int b0 = 0; b0 < nbad; b0 += kFixBatch) {
+      const int nb = min(kFixBatch, nbad - b0);
+      __syncthreads();   // P written; the previous batch's readers are done
+      for (int i = tid; i < kFixBatch * BN; i += kFixThreads) {
+        const int b = i / BN, r = i % BN;
+        const bool ok = b < nb && r < n;
+        const int c = ok ? sIdx[b0 + b] : 0;
+        const size_t a = (tok0 + (ok ? r : 0)) * vrs + (size_t)kv * DV + c;
+        sL[i] = ok ? P.L[a] : 0.f;
+        sV[i] = ok ? bf2f(P.v[a]) : 0.f;
+        sDo[i] = ok ? P.do_ws[(tok0 + r) * ors + (size_t)h * DV + c] : 0.f;
+      }
+      __syncthreads();
+      // dv_s[c] += sum_{t > s} P_ts exp(L_t[c] - L_s[c]) do_t[c], into the slot
+      if (4 * cg < nb && s_dv < n) {
+        float ls[4], dvb[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) ls[u] = sL[(4 * cg + u) * BN + s_dv];
+        for (int t = t_dv; t < n; ++t) {   // warp-uniform t: broadcast reads
+          const float pts = t > s_dv ? sP[t * Lay::kPs + s_dv] : 0.f;
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int b = 4 * cg + u;
+            dvb[u] += pts * ex2((sL[b * BN + t] - ls[u]) * LOG2E) * sDo[b * BN + t];
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (4 * cg + u < nb) slot[(size_t)s_dv * (DK + DV) + DK + sIdx[b0 + 4 * cg + u]] += dvb[u];
+      }
+      // dP^bad_ts += sum_{c in batch} do_t[c] exp(L_t[c] - L_s[c]) v_s[c]
+      if (sb <= tb) {
+        for (int b = 0; b < nb; ++b) {
+          float lt[8], dt[8], ls[8], vs[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            lt[i] = sL[b * BN + 8 * tb + i];
+            dt[i] = sDo[b * BN + 8 * tb + i];
+            ls[i] = sL[b * BN + 8 * sb + i];
+            vs[i] = sV[b * BN + 8 * sb + i];
+          }
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              if (8 * sb + j <= 8 * tb + i)
+                dp[i][j] += dt[i] * ex2((lt[i] - ls[j]) * LOG2E) * vs[j];
+        }
+      }
+    }
+    __syncthreads();   // every dv reader of P is done
+    // dS^bad = P dP^bad, over P
+    if (sb <= tb) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          float* e = sP + (8 * tb + i) * Lay::kPs + 8 * sb + j;
+          *e = *e * dp[i][j];
+        }
+    }
+    __syncthreads();
+    // dK_s += sum_t dS^bad_ts q_t (unscaled, like the slots)
+    for (int t = 0; t < n; ++t) {   // dS^bad is zero for t < s
+      const float4 ds = *reinterpret_cast<const float4*>(sP + t * Lay::kPs + 4 * sq);
+      const float dsa[4] = {ds.x, ds.y, ds.z, ds.w};
+#pragma unroll
+      for (int e = 0; e < CK; ++e) {
+        const float qv = sQt[(cb * CK + e) * BN + t];
+#pragma unroll
+        for (int a = 0; a < 4; ++a) dk[a][e] = fmaf(dsa[a], qv, dk[a][e]);
+      }
+    }
+  }
+#pragma unroll
+  for (int a = 0; a < 4; ++a) {
+    const int sk = 4 * sq + a;
+    if (sk < n) {
+#pragma unroll
+      for (int e = 0; e < CK; ++e) slot[(size_t)sk * (DK + DV) + cb * CK + e] += dk[a][e];
+    }
+  }
 }
 
 // ---------------------------------------------------------------- host side
@@ -1114,11 +1379,17 @@ static fix_status launch(const Params& prm, const void* vt, const void* vm, int 
   return cudaGetLastError() == cudaSuccess ? FIX_OK : FIX_ERR_CUDA;
 }
 
-// The combine of the dk/dv partial slots (which = 2).
+// The exact terms of out-of-range channels, then the combine of the dk/dv
+// partial slots (which = 2).
 template <int DK, int DV>
 static fix_status launch_combine(const Params& prm, long long nslots, cudaStream_t st) {
   const Dims& d = prm.d;
-  if (nslots > 0) dkv_combine_kernel<DK, DV><<<dim3(d.nchunks * (BN / 8), d.Hkv), 256, 0, st>>>(prm);
+  if (nslots <= 0) return FIX_OK;
+  const int smem = FixLayout<DK, DV>::kBytes;
+  auto fix = dkv_diag_exact_kernel<DK, DV>;
+  if (!set_smem_limit(reinterpret_cast<const void*>(fix), smem)) return FIX_ERR_CUDA;
+  fix<<<dim3(d.nchunks, d.Hkv), kFixThreads, smem, st>>>(prm);
+  dkv_combine_kernel<DK, DV><<<dim3(d.nchunks * (BN / 8), d.Hkv), 256, 0, st>>>(prm);
   return cudaGetLastError() == cudaSuccess ? FIX_OK : FIX_ERR_CUDA;
 }
 
@@ -1129,7 +1400,7 @@ bool tc_bwd_supported(const Dims& d) {
   return dims_ok && d.N >= FIX_CHUNK && d.grp <= 16;
 }
 
-int tc_bwd_kernel_count(const Dims&, long long nslots) { return nslots > 0 ? 3 : 2; }
+int tc_bwd_kernel_count(const Dims&, long long nslots) { return nslots > 0 ? 4 : 2; }
 
 fix_status tc_bwd(const fix_attn_problem*, const Dims& d, const TcBwdArgs& a, int which,
                   cudaStream_t st) {

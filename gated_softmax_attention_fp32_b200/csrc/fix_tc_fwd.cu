@@ -68,9 +68,11 @@ using namespace sm100;
 
 constexpr int BM = 128;          // query rows per tile
 constexpr int BN = FIX_CHUNK;    // keys per block
-constexpr int kThreads = 512;
+constexpr int kThreads = 384;
+constexpr int kVsThreads = 64;   // V-scaling threads (warps 2-3)
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // lazy row-max update, natural-log units
+constexpr int kPolyOf4 = 1;      // of every 4 softmax exponentials, how many (0 or 1) by polynomial
 __host__ __device__ constexpr uint32_t col_s(int b) { return b ? 128u : 0u; }
 
 struct Bars {
@@ -96,8 +98,8 @@ struct Layout {
   static constexpr int kBad = kF + 2 * DV * 4;           // [2][DV] int out-of-range flags
   static constexpr int kAnyBad = kBad + 2 * DV * 4;      // [2] int
   static constexpr int kRows = kAnyBad + 16;             // [2][4][BM] f32: alpha, P_tt, m, l
-  static constexpr int kEpiT = kRows + 2 * 4 * BM * 4;   // [4][32][33] f32 transposes
-  static constexpr int kEpiW = kEpiT + 4 * 32 * 33 * 4;  // [DV] f32 w
+  static constexpr int kPlo = kRows + 2 * 4 * BM * 4;    // [BM][33] u32: diagonal P_lo, key chunks 0-1
+  static constexpr int kEpiW = kPlo + BM * 33 * 4;       // [DV] f32 w
   static constexpr int kEpiRho = kEpiW + DV * 4;         // [DV] f32 rho of the epilogue's tile
   static constexpr int kEpiBad = kEpiRho + DV * 4;       // [DV] int
   static constexpr int kBars = (kEpiBad + DV * 4 + 7) / 8 * 8;
@@ -161,31 +163,32 @@ __device__ __forceinline__ Tile tile_info(const Params& P, int t) {
   return x;
 }
 
-// Named barriers for one warpgroup (ids 1..3; 0 is __syncthreads).
-__device__ __forceinline__ void wg_sync(int id) {
-  asm volatile("bar.sync %0, 128;" ::"r"(id) : "memory");
+// Named barriers for the threads of one role (ids 1..3; 0 is __syncthreads):
+// id 2 the V-scaling warps, id 3 the epilogue warps.
+__device__ __forceinline__ void wg_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
-__device__ __forceinline__ int wg_and(int id, int pred) {
+__device__ __forceinline__ int wg_and(int id, int n, int pred) {
   int out;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
       "setp.ne.b32 p, %1, 0;\n\t"
-      "bar.red.and.pred q, %2, 128, p;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
       "selp.s32 %0, 1, 0, q;\n\t}"
       : "=r"(out)
-      : "r"(pred), "r"(id)
+      : "r"(pred), "r"(id), "r"(n)
       : "memory");
   return out;
 }
-__device__ __forceinline__ int wg_or(int id, int pred) {
+__device__ __forceinline__ int wg_or(int id, int n, int pred) {
   int out;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
       "setp.ne.b32 p, %1, 0;\n\t"
-      "bar.red.or.pred q, %2, 128, p;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\t"
       "selp.s32 %0, 1, 0, q;\n\t}"
       : "=r"(out)
-      : "r"(pred), "r"(id)
+      : "r"(pred), "r"(id), "r"(n)
       : "memory");
   return out;
 }
@@ -228,12 +231,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bar->k_empty[s], 1);
       mbar_init(&bar->v_full[s], 1);
       mbar_init(&bar->v_empty[s], 1);
-      mbar_init(&bar->v_ready[s], 128);
+      mbar_init(&bar->v_ready[s], kVsThreads);
       mbar_init(&bar->s_full[s], 1);
       mbar_init(&bar->p_full[s], 128);
       mbar_init(&bar->acc_full[s], 1);
       mbar_init(&bar->acc_empty[s], 128);
-      mbar_init(&bar->fold_ready[s], 128);
+      mbar_init(&bar->fold_ready[s], kVsThreads);
       mbar_init(&bar->rows_ready[s], 128);
       mbar_init(&bar->rows_free[s], 128);
     }
@@ -243,9 +246,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_fence_init();
   }
   if (warp == 1) tmem_alloc(sTmem, kTmemCols);
-  if (tid >= 384 && tid - 384 < DV)
-    reinterpret_cast<float*>(smem + Lay::kEpiW)[tid - 384] =
-        (P.w && !d.no_norm) ? bf2f(P.w[tid - 384]) : 1.f;
+  if (tid >= 256 && tid - 256 < DV)
+    reinterpret_cast<float*>(smem + Lay::kEpiW)[tid - 256] =
+        (P.w && !d.no_norm) ? bf2f(P.w[tid - 256]) : 1.f;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -410,19 +413,108 @@ __global__ void __launch_bounds__(kThreads, 1)
         // waits vote warp-wide: the TMEM accesses below are warp-collective
         if (!__all_sync(0xffffffffu, mbar_wait(&bar->s_full[b], (g >> 1) & 1, ctl))) { ok = false; break; }
         tc_fence_after();
-        // pass 1: the row maximum (diagonal block: keys s <= t; S_tt kept
-        // for the exact s = t term)
-        float mx = -INFINITY;
+        if (!diag) {
+          // One pass: P = exp(S scale - m_used) chunk by chunk (fp16, over the
+          // S columns already read), with the next chunk's TMEM load in
+          // flight.  A chunk whose maximum exceeds m_used by more than the
+          // lazy threshold moves the reference (warp-wide): the P already
+          // written in this block, the running sum and A (the earlier blocks,
+          // once their last PV has completed) are scaled by exp(m_used - m_new).
+          float ls = 0.f;
+          auto chunk = [&](const uint32_t (&xs)[32], int c4) -> bool {
+            float ma = __uint_as_float(xs[0]), mb = __uint_as_float(xs[1]);
 #pragma unroll
-        for (int c4 = 0; c4 < BN / 32; ++c4) {
-          uint32_t xs[32];
-          tmem_ld32(sbase + c4 * 32, xs);
-          tmem_wait_ld();
-          if (!diag) {
+            for (int e = 2; e < 32; e += 2) {
+              ma = fmaxf(ma, __uint_as_float(xs[e]));
+              mb = fmaxf(mb, __uint_as_float(xs[e + 1]));
+            }
+            const float cm = fmaxf(ma, mb) * d.scale;
+            m_true = fmaxf(m_true, cm);
+            if (__any_sync(0xffffffffu, cm > m_used + kRescaleThreshold)) {
+              const float m_new = fmaxf(m_used, m_true);
+              const float rr = m_used == -INFINITY ? 0.f : ex2((m_used - m_new) * LOG2E);
+              if (c4 > 0) {
+                tmem_wait_st();
+                const __half2 r2 = __float2half2_rn(rr);
+                for (int cp = 0; cp < c4; ++cp) {
+                  uint32_t pk[16];
+                  tmem_ld16(sbase + cp * 16, pk);
+                  tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; e += 2)
-              mx = fmaxf(mx, fmaxf(__uint_as_float(xs[e]), __uint_as_float(xs[e + 1])));
-          } else {
+                  for (int e = 0; e < 16; ++e) {
+                    __half2 h = *reinterpret_cast<__half2*>(&pk[e]);
+                    h = __hmul2(h, r2);
+                    pk[e] = *reinterpret_cast<uint32_t*>(&h);
+                  }
+                  tmem_st16(sbase + cp * 16, pk);
+                }
+              }
+              if (it > 0) {
+                // A is quiescent once the previous block's PV has completed
+                if (!__all_sync(0xffffffffu, mbar_wait(&bar->pv_done, (g - 1) & 1, ctl))) return false;
+                tc_fence_after();
+#pragma unroll 1
+                for (int cc = 0; cc < DV / 32; ++cc) {
+                  uint32_t xa[32];
+                  tmem_ld32(acol + cc * 32, xa);
+                  tmem_wait_ld(xa);
+#pragma unroll
+                  for (int e = 0; e < 32; ++e) xa[e] = __float_as_uint(__uint_as_float(xa[e]) * rr);
+                  tmem_st32(acol + cc * 32, xa);
+                }
+              }
+              ls *= rr;
+              l_used *= rr;
+              m_used = m_new;
+            }
+            const float moff = m_used * LOG2E;
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              const float a0 = __uint_as_float(xs[e]) * c1 - moff;
+              const float a1 = __uint_as_float(xs[e + 1]) * c1 - moff;
+              // one exponential in four on the FMA pipe (kPolyOf4), the rest
+              // on the MUFU unit; both well inside fp16's rounding
+              const float p0 = ex2(a0);
+              const float p1 = ((e >> 1) & 1) && kPolyOf4 ? exp2_poly3(a1) : ex2(a1);
+              ls += p0 + p1;
+              pk[e >> 1] = pack_f16(p0, p1);
+            }
+            tmem_st16(sbase + c4 * 16, pk);
+            return true;
+          };
+          uint32_t xa[32], xb[32];
+          tmem_ld32(sbase, xa);
+          tmem_wait_ld(xa);
+          tmem_ld32(sbase + 32, xb);
+          bool good = chunk(xa, 0);
+          tmem_wait_ld(xb);
+          if (good) {
+            tmem_ld32(sbase + 64, xa);
+            good = chunk(xb, 1);
+            tmem_wait_ld(xa);
+          }
+          if (good) {
+            tmem_ld32(sbase + 96, xb);
+            good = chunk(xa, 2);
+            tmem_wait_ld(xb);
+          }
+          if (good) good = chunk(xb, 3);
+          if (!good) {
+            tmem_wait_ld();   // no TMEM load may stay in flight
+            ok = false;
+            break;
+          }
+          if (d.no_norm) l_used += ls;
+        } else {
+          // pass 1: the row maximum (diagonal block: keys s <= t; S_tt kept
+          // for the exact s = t term)
+          float mx = -INFINITY;
+#pragma unroll
+          for (int c4 = 0; c4 < BN / 32; ++c4) {
+            uint32_t xs[32];
+            tmem_ld32(sbase + c4 * 32, xs);
+            tmem_wait_ld(xs);
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
               const float sv = __uint_as_float(xs[e]);
@@ -431,147 +523,130 @@ __global__ void __launch_bounds__(kThreads, 1)
               s_diag = key == r ? sv : s_diag;
             }
           }
-        }
-        m_true = fmaxf(m_true, mx * d.scale);
-        bool rescale = false;
-        if (it == 0) m_used = m_true;
-        else rescale = __any_sync(0xffffffffu, m_true > m_used + kRescaleThreshold);
-        const bool fold = diag && x.nblk > 1;
-        // the fold factors and out-of-range flags of this tile
-        if (diag && !__all_sync(0xffffffffu, mbar_wait(&bar->fold_ready[tb], use & 1, ctl))) { ok = false; break; }
-        if (rescale || fold) {
-          // A must be quiescent: the previous block's PV has completed
-          if (!__all_sync(0xffffffffu, mbar_wait(&bar->pv_done, (g - 1) & 1, ctl))) { ok = false; break; }
-          tc_fence_after();
-          const float a_r = rescale ? ex2((m_used - m_true) * LOG2E) : 1.f;
-          const float* F = sF + tb * DV;
+          m_true = fmaxf(m_true, mx * d.scale);
+          bool rescale = false;
+          if (it == 0) m_used = m_true;
+          else rescale = __any_sync(0xffffffffu, m_true > m_used + kRescaleThreshold);
+          const bool fold = diag && x.nblk > 1;
+          // the fold factors and out-of-range flags of this tile
+          if (diag && !__all_sync(0xffffffffu, mbar_wait(&bar->fold_ready[tb], use & 1, ctl))) { ok = false; break; }
+          if (rescale || fold) {
+            // A must be quiescent: the previous block's PV has completed
+            if (!__all_sync(0xffffffffu, mbar_wait(&bar->pv_done, (g - 1) & 1, ctl))) { ok = false; break; }
+            tc_fence_after();
+            const float a_r = rescale ? ex2((m_used - m_true) * LOG2E) : 1.f;
+            const float* F = sF + tb * DV;
 #pragma unroll 1
-          for (int cc = 0; cc < DV / 32; ++cc) {
-            uint32_t xa[32];
-            tmem_ld32(acol + cc * 32, xa);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const float f = fold ? F[cc * 32 + e] * a_r : a_r;
-              xa[e] = __float_as_uint(__uint_as_float(xa[e]) * f);
-            }
-            tmem_st32(acol + cc * 32, xa);
-          }
-          tmem_wait_st();
-          if (rescale) {
-            m_used = m_true;
-            l_used *= a_r;
-          }
-        }
-        if (diag && x.nblk == 1) {
-          // chunk 0: the diagonal MMAs accumulate into A, which starts at
-          // zero here; the epilogue of the tile that used it before must be
-          // done with it
-          if (use >= 1 && !__all_sync(0xffffffffu, mbar_wait(&bar->acc_empty[tb], (use - 1) & 1, ctl))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          uint32_t z[32];
-#pragma unroll
-          for (int e = 0; e < 32; ++e) z[e] = 0u;
-#pragma unroll
-          for (int cc = 0; cc < DV / 32; ++cc) tmem_st32(acol + cc * 32, z);
-          tmem_wait_st();
-        }
-        const float moff = m_used * LOG2E;
-        if (diag && sAnyBad[tb]) {
-          // exact diagonal sums of out-of-range channels, in fp32 from the
-          // fp32 logits: A_tc <- exp(L_t) A_tc + sum_{s<t} P_ts exp(L_t - L_s) v_s
-          const int* bad = sBad + tb * DV;
-          const int nk = r < x.len ? r : 0;
-          const size_t rowL = ((size_t)x.tok0 + (r < x.len ? r : 0)) * vrs + (size_t)x.kv * DV;
-          const float* Lk = P.L + (size_t)x.tok0 * vrs + (size_t)x.kv * DV;
-          const __nv_bfloat16* vk = P.v + (size_t)x.tok0 * vrs + (size_t)x.kv * DV;
-#pragma unroll 1
-          for (int c = 0; c < DV; ++c) {
-            if (!bad[c]) continue;   // tile-uniform
-            const float lt = P.L[rowL + c];
-            float acc = 0.f;
-#pragma unroll 1
-            for (int c4 = 0; c4 < BN / 32; ++c4) {
-              uint32_t xs[32];
-              tmem_ld32(sbase + c4 * 32, xs);
+            for (int cc = 0; cc < DV / 32; ++cc) {
+              uint32_t xa[32];
+              tmem_ld32(acol + cc * 32, xa);
               tmem_wait_ld();
-#pragma unroll 4
+#pragma unroll
               for (int e = 0; e < 32; ++e) {
-                const int s = c4 * 32 + e;
-                if (s < nk) {
-                  const float p = ex2(__uint_as_float(xs[e]) * c1 - moff);
-                  acc += p * ex2((lt - Lk[(size_t)s * vrs + c]) * LOG2E) * bf2f(vk[(size_t)s * vrs + c]);
+                const float f = fold ? F[cc * 32 + e] * a_r : a_r;
+                xa[e] = __float_as_uint(__uint_as_float(xa[e]) * f);
+              }
+              tmem_st32(acol + cc * 32, xa);
+            }
+            tmem_wait_st();
+            if (rescale) {
+              m_used = m_true;
+              l_used *= a_r;
+            }
+          }
+          if (diag && x.nblk == 1) {
+            // chunk 0: the diagonal MMAs accumulate into A, which starts at
+            // zero here; the epilogue of the tile that used it before must be
+            // done with it
+            if (use >= 1 && !__all_sync(0xffffffffu, mbar_wait(&bar->acc_empty[tb], (use - 1) & 1, ctl))) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            uint32_t z[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) z[e] = 0u;
+#pragma unroll
+            for (int cc = 0; cc < DV / 32; ++cc) tmem_st32(acol + cc * 32, z);
+            tmem_wait_st();
+          }
+          const float moff = m_used * LOG2E;
+          if (diag && sAnyBad[tb]) {
+            // exact diagonal sums of out-of-range channels, in fp32 from the
+            // fp32 logits: A_tc <- exp(L_t) A_tc + sum_{s<t} P_ts exp(L_t - L_s) v_s
+            const int* bad = sBad + tb * DV;
+            const int nk = r < x.len ? r : 0;
+            const size_t rowL = ((size_t)x.tok0 + (r < x.len ? r : 0)) * vrs + (size_t)x.kv * DV;
+            const float* Lk = P.L + (size_t)x.tok0 * vrs + (size_t)x.kv * DV;
+            const __nv_bfloat16* vk = P.v + (size_t)x.tok0 * vrs + (size_t)x.kv * DV;
+#pragma unroll 1
+            for (int c = 0; c < DV; ++c) {
+              if (!bad[c]) continue;   // tile-uniform
+              const float lt = P.L[rowL + c];
+              float acc = 0.f;
+#pragma unroll 1
+              for (int c4 = 0; c4 < BN / 32; ++c4) {
+                uint32_t xs[32];
+                tmem_ld32(sbase + c4 * 32, xs);
+                tmem_wait_ld();
+#pragma unroll 4
+                for (int e = 0; e < 32; ++e) {
+                  const int s = c4 * 32 + e;
+                  if (s < nk) {
+                    const float p = ex2(__uint_as_float(xs[e]) * c1 - moff);
+                    acc += p * ex2((lt - Lk[(size_t)s * vrs + c]) * LOG2E) * bf2f(vk[(size_t)s * vrs + c]);
+                  }
                 }
               }
+              uint32_t xa;
+              asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(xa) : "r"(acol + c));
+              tmem_wait_ld();
+              tmem_st1(acol + c, __float_as_uint(ex2(lt * LOG2E) * __uint_as_float(xa) + acc));
             }
-            uint32_t xa;
-            asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(xa) : "r"(acol + c));
-            tmem_wait_ld();
-            tmem_st1(acol + c, __float_as_uint(ex2(lt * LOG2E) * __uint_as_float(xa) + acc));
+            tmem_wait_st();
           }
-          tmem_wait_st();
-        }
-        // pass 2: P, written over the S columns already read
-        if (!diag) {
+          // pass 2: P, written over the S columns already read
+          {
+            // strictly causal P as bf16 hi (columns [0, 64)) + lo ([64, 128));
+            // lo parts are stored only over S columns already read: those of
+            // key chunks 0 and 1 (staged in shared memory meanwhile) after
+            // chunk 2 is read, those of 2 and 3 after chunk 3
+            uint32_t* plo = reinterpret_cast<uint32_t*>(smem + Lay::kPlo) + r * 33;
+            uint32_t plo2[16];
+#pragma unroll 1
+            for (int c4 = 0; c4 < BN / 32; ++c4) {
+              uint32_t xs[32], ph[16], pl[16];
+              tmem_ld32(sbase + c4 * 32, xs);
+              tmem_wait_ld(xs);
 #pragma unroll
-          for (int c4 = 0; c4 < BN / 32; ++c4) {
-            uint32_t xs[32], pk[16];
-            tmem_ld32(sbase + c4 * 32, xs);
-            tmem_wait_ld();
-            float ls = 0.f;
-            // half of the exponentials on the MUFU unit, half as a polynomial
-            // on the FMA pipe (both well inside fp16's rounding)
+              for (int e = 0; e < 32; e += 2) {
+                const int key = c4 * 32 + e;
+                const float p0 = key < r ? ex2(__uint_as_float(xs[e]) * c1 - moff) : 0.f;
+                const float p1 = key + 1 < r ? ex2(__uint_as_float(xs[e + 1]) * c1 - moff) : 0.f;
+                if (d.no_norm) l_used += p0 + p1;
+                ph[e >> 1] = pack_bf16(p0, p1);
+                const float h0 = __uint_as_float(ph[e >> 1] << 16);
+                const float h1 = __uint_as_float(ph[e >> 1] & 0xFFFF0000u);
+                pl[e >> 1] = pack_bf16(p0 - h0, p1 - h1);
+              }
+              tmem_st16(sbase + c4 * 16, ph);
+              if (c4 < 2) {
 #pragma unroll
-            for (int e = 0; e < 32; e += 2) {
-              const float p0 = ex2(__uint_as_float(xs[e]) * c1 - moff);
-              const float p1 = exp2_poly3(__uint_as_float(xs[e + 1]) * c1 - moff);
-              ls += p0 + p1;
-              pk[e >> 1] = pack_f16(p0, p1);
-            }
-            if (d.no_norm) l_used += ls;
-            tmem_st16(sbase + c4 * 16, pk);
-          }
-        } else {
-          // strictly causal P as bf16 hi (columns [0, 64)) + lo ([64, 128));
-          // lo parts are stored only over S columns already read: those of
-          // key chunks 0 and 1 after chunk 2 is read, those of 2 and 3 after
-          // chunk 3 (separate register arrays: a tcgen05.st may still read
-          // its source registers until the wait)
-          uint32_t plo0[16], plo1[16], plo2[16];
+                for (int e = 0; e < 16; ++e) plo[c4 * 16 + e] = pl[e];
+              } else if (c4 == 2) {
 #pragma unroll
-          for (int c4 = 0; c4 < BN / 32; ++c4) {
-            uint32_t xs[32], ph[16], pl[16];
-            tmem_ld32(sbase + c4 * 32, xs);
-            tmem_wait_ld();
+                for (int h = 0; h < 2; ++h) {
+                  uint32_t t16[16];
 #pragma unroll
-            for (int e = 0; e < 32; e += 2) {
-              const int key = c4 * 32 + e;
-              const float p0 = key < r ? ex2(__uint_as_float(xs[e]) * c1 - moff) : 0.f;
-              const float p1 = key + 1 < r ? ex2(__uint_as_float(xs[e + 1]) * c1 - moff) : 0.f;
-              if (d.no_norm) l_used += p0 + p1;
-              ph[e >> 1] = pack_bf16(p0, p1);
-              const float h0 = __uint_as_float(ph[e >> 1] << 16);
-              const float h1 = __uint_as_float(ph[e >> 1] & 0xFFFF0000u);
-              pl[e >> 1] = pack_bf16(p0 - h0, p1 - h1);
-            }
-            tmem_st16(sbase + c4 * 16, ph);
-            if (c4 == 0) {
+                  for (int e = 0; e < 16; ++e) t16[e] = plo[h * 16 + e];
+                  tmem_st16(sbase + 64 + h * 16, t16);
+                }
 #pragma unroll
-              for (int e = 0; e < 16; ++e) plo0[e] = pl[e];
-            } else if (c4 == 1) {
-#pragma unroll
-              for (int e = 0; e < 16; ++e) plo1[e] = pl[e];
-            } else if (c4 == 2) {
-              tmem_st16(sbase + 64, plo0);
-              tmem_st16(sbase + 80, plo1);
-#pragma unroll
-              for (int e = 0; e < 16; ++e) plo2[e] = pl[e];
-            } else {
-              tmem_st16(sbase + 96, plo2);
-              tmem_st16(sbase + 112, pl);
+                for (int e = 0; e < 16; ++e) plo2[e] = pl[e];
+              } else {
+                tmem_st16(sbase + 96, plo2);
+                tmem_st16(sbase + 112, pl);
+              }
             }
           }
         }
@@ -593,11 +668,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(&bar->rows_ready[tb]);
       ++nt;
     }
-  } else if (warp >= 8 && warp < 12) {
+  } else if (warp == 2 || warp == 3) {
     // ------------------------------------------------------------ V scaling
-    const int dt = tid - 256;                        // 0..127
+    const int dt = tid - 64;                         // 0..63
     constexpr int kChunks = DV / 8;                  // 16-byte chunks per row
-    constexpr int kRowsPerPass = 128 / kChunks;
+    constexpr int kRowsPerPass = kVsThreads / kChunks;
     const int lc = dt % kChunks;                     // logical chunk: channels lc*8 .. +7
     const int r0 = dt / kChunks;
     const int half = lc >> 3, lcc = lc & 7;
@@ -613,12 +688,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       // has completed (it follows the fold)
       // (every wait of this warpgroup ends in a vote on a named barrier, so
       // that all 128 threads leave together after an abort)
-      if (!wg_and(2, use < 1 || mbar_wait(&bar->acc_full[tb], (use - 1) & 1, ctl))) { ok = false; break; }
+      if (!wg_and(2, kVsThreads, use < 1 || mbar_wait(&bar->acc_full[tb], (use - 1) & 1, ctl))) { ok = false; break; }
       // tile-wide power-of-two scale k_c of the earlier blocks' operands:
       // not needed (0) when every earlier chunk is fp16-safe (g <= 0)
       int my_safe = 1;
-      for (int jj = dt; jj < x.nblk - 1; jj += 128) my_safe &= P.safe[(size_t)(x.first + jj) * d.Hkv + x.kv];
-      const int tile_safe = wg_and(2, my_safe);
+      for (int jj = dt; jj < x.nblk - 1; jj += kVsThreads) my_safe &= P.safe[(size_t)(x.first + jj) * d.Hkv + x.kv];
+      const int tile_safe = wg_and(2, kVsThreads, my_safe);
       float kexp[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) kexp[e] = 0.f;
@@ -659,7 +734,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 8; ++e) my_bad |= P.hr[ti + e] > FIX_HR_MAX ? 1 : 0;
         }
-        const int any = wg_or(2, my_bad);
+        const int any = wg_or(2, kVsThreads, my_bad);
         if (dt == 0) sAnyBad[tb] = any;
       }
       mbar_arrive(&bar->fold_ready[tb]);
@@ -697,7 +772,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             fh[u] = __floats2half2_rn(f8[2 * u], f8[2 * u + 1]);
           }
         }
-        if (!wg_and(2, mbar_wait(&bar->v_full[sv], (vc >> 1) & 1, ctl))) { ok = false; break; }
+        if (!wg_and(2, kVsThreads, mbar_wait(&bar->v_full[sv], (vc >> 1) & 1, ctl))) { ok = false; break; }
         if (!diag) {
           uint8_t* vb = reinterpret_cast<uint8_t*>(sV + sv * BN * DV) + half * (BN * 128);
           if (h16) {
@@ -731,20 +806,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       ++nt;
     }
-  } else if (warp >= 12) {
+  } else if (warp >= 8) {
     // ------------------------------------------------------------ epilogue
-    const int ew = warp - 12;                        // TMEM lanes [32 ew, 32 ew + 32)
+    // A thread per tile row (its TMEM lane): two passes over the row's
+    // channels in chunks of 32, the first for the RMSNorm's sum of squares
+    // (and the saved o), the second for y.  The row's L, v (and output gate)
+    // are contiguous: each thread loads them with 16-byte accesses.
+    const int ew = warp - 8;                         // TMEM lanes [32 ew, 32 ew + 32)
     const uint32_t lane_base = tmem + ((uint32_t)(ew * 32) << 16);
-    float* tr = reinterpret_cast<float*>(smem + Lay::kEpiT) + ew * 32 * 33;
+    const int r = ew * 32 + lane;                    // tile row
     const float* sW = reinterpret_cast<const float*>(smem + Lay::kEpiW);
     float* eRho = reinterpret_cast<float*>(smem + Lay::kEpiRho);
     int* eBad = reinterpret_cast<int*>(smem + Lay::kEpiBad);
-    const int et = tid - 384;                        // 0..127
-    float* __restrict__ yf = P.y_f32 ? reinterpret_cast<float*>(P.y) : nullptr;
-    __nv_bfloat16* __restrict__ yb = P.y_f32 ? nullptr : reinterpret_cast<__nv_bfloat16*>(P.y);
+    const int et = tid - 256;                        // 0..127
     const size_t ors = (size_t)d.Hq * DV;
     constexpr int kU = DV / 32;                      // 32-channel chunks
-    constexpr int kR = 4;                            // rows per pass
     int nt = 0;
     bool ok = true;
     for (int round = 0; ok && round < rounds; ++round) {
@@ -753,22 +829,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Tile x = tile_info(P, t);
       if (x.len <= 0) continue;
       const int tb = nt & 1, use = nt >> 1;
-      const float* Lg = P.L + (size_t)x.kv * DV;
-      const __nv_bfloat16* vg = P.v + (size_t)x.kv * DV;
-      // While the tile's MMAs run, pull its rows of L, v (and the output
-      // gate) into L2, so that the loads below hit L2: one row per thread.
-      if (et < x.len) {
-        const size_t tk = (size_t)x.tok0 + et;
-        const char* lr = reinterpret_cast<const char*>(Lg + tk * vrs);
-        const char* vr = reinterpret_cast<const char*>(vg + tk * vrs);
+      const bool valid = r < x.len;
+      const size_t tk = (size_t)x.tok0 + (valid ? r : 0);
+      const float* Lr = P.L + tk * vrs + (size_t)x.kv * DV;
+      const __nv_bfloat16* vr = P.v + tk * vrs + (size_t)x.kv * DV;
+      const size_t orow = tk * ors + (size_t)x.h * DV;
+      // While the tile's MMAs run, pull this row's L, v (and output gate)
+      // into L2.
+      if (valid) {
 #pragma unroll
-        for (int b = 0; b < DV * 4; b += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(lr + b));
+        for (int b = 0; b < DV * 4; b += 128)
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<const char*>(Lr) + b));
 #pragma unroll
-        for (int b = 0; b < DV * 2; b += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(vr + b));
+        for (int b = 0; b < DV * 2; b += 128)
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<const char*>(vr) + b));
         if (P.z) {
-          const char* zr = reinterpret_cast<const char*>(P.z + (tk * d.Hq + x.h) * DV);
 #pragma unroll
-          for (int b = 0; b < DV * 2; b += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(zr + b));
+          for (int b = 0; b < DV * 2; b += 128)
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<const char*>(P.z + orow) + b));
         }
       }
       // channel data of this tile (the previous tile's readers are done:
@@ -778,96 +856,107 @@ __global__ void __launch_bounds__(kThreads, 1)
         eRho[et] = P.rho[ti];
         eBad[et] = P.hr[ti] > FIX_HR_MAX ? 1 : 0;
       }
-      wg_sync(3);
-      if (!wg_and(3, mbar_wait(&bar->acc_full[tb], use & 1, ctl) &&
-                         mbar_wait(&bar->rows_ready[tb], use & 1, ctl))) {
+      wg_sync(3, 128);
+      if (!wg_and(3, 128, mbar_wait(&bar->acc_full[tb], use & 1, ctl) &&
+                              mbar_wait(&bar->rows_ready[tb], use & 1, ctl))) {
         ok = false;
         break;
       }
       tc_fence_after();
       const float* rows = sRows + tb * 4 * BM;
+      const float alpha = rows[r], ptt = rows[BM + r], mt = rows[2 * BM + r], lsum = rows[3 * BM + r];
       const uint32_t acol = lane_base + 256u + (uint32_t)(tb * DV);
+      // o for channels [32 u, 32 u + 32): alpha exp(L - rho) A + P_tt v
+      // (no row factor for out-of-range channels)
+      auto chunk_o = [&](int u, float (&o)[32]) {
+        uint32_t xa[32];
+        tmem_ld32(acol + u * 32, xa);
+        float4 l4[8];
+        uint4 v4[4];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) l4[q] = reinterpret_cast<const float4*>(Lr + u * 32)[q];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) v4[q] = reinterpret_cast<const uint4*>(vr + u * 32)[q];
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int c = u * 32 + e;
+          const float4 lq = l4[e >> 2];
+          const float le = (e & 3) == 0 ? lq.x : (e & 3) == 1 ? lq.y : (e & 3) == 2 ? lq.z : lq.w;
+          const uint4 vq = v4[e >> 3];
+          const uint32_t vw = ((e >> 1) & 3) == 0 ? vq.x : ((e >> 1) & 3) == 1 ? vq.y
+                            : ((e >> 1) & 3) == 2 ? vq.z : vq.w;
+          const float ve = __uint_as_float((e & 1) ? (vw & 0xFFFF0000u) : (vw << 16));
+          const float fac = eBad[c] ? 1.f : ex2((le - eRho[c]) * LOG2E);
+          o[e] = alpha * fac * __uint_as_float(xa[e]) + ptt * ve;
+        }
+      };
+      // pass 1: the sum of squares (and the saved o)
+      float ss = 0.f;
 #pragma unroll 1
-      for (int grp = 0; grp < 32 / kR; ++grp) {
-        const int rbase = ew * 32 + grp * kR;          // first tile row of this pass
-        // L and v of the pass's rows for every chunk, all loads in flight at
-        // once (lanes over channels: coalesced)
-        float lt[kU][kR], vt[kU][kR];
+      for (int u = 0; u < kU; ++u) {
+        float o[32];
+        chunk_o(u, o);
 #pragma unroll
-        for (int u = 0; u < kU; ++u)
+        for (int e = 0; e < 32; ++e) ss += o[e] * o[e];
+        if (P.o_s && valid && !d.no_norm) {
+          float4* dst = reinterpret_cast<float4*>(P.o_s + orow + u * 32);
 #pragma unroll
-          for (int q = 0; q < kR; ++q) {
-            const int rr = min(rbase + q, x.len - 1);
-            const size_t tk = (size_t)x.tok0 + rr;
-            lt[u][q] = Lg[tk * vrs + u * 32 + lane];
-            vt[u][q] = bf2f(vg[tk * vrs + u * 32 + lane]);
-          }
-        float o[kR][kU];
-        float ss[kR];
+          for (int q = 0; q < 8; ++q) dst[q] = make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+        }
+      }
+      // the RMSNorm, or without it the softmax denominator: y = o / l; the
+      // saved tensors are then o / l, the log-sum-exp and ones
+      const float rstd = d.no_norm ? 1.0f / lsum : 1.0f / sqrtf(ss / (float)DV + d.eps);
+      // pass 2: y (and without the norm the saved o / l)
+#pragma unroll 1
+      for (int u = 0; u < kU; ++u) {
+        float o[32];
+        chunk_o(u, o);
+        // without the norm the saved o / l
+        if (P.o_s && d.no_norm && valid) {
+          float4* dst = reinterpret_cast<float4*>(P.o_s + orow + u * 32);
 #pragma unroll
-        for (int q = 0; q < kR; ++q) ss[q] = 0.f;
+          for (int q = 0; q < 8; ++q)
+            dst[q] = make_float4(o[4 * q] * rstd, o[4 * q + 1] * rstd, o[4 * q + 2] * rstd, o[4 * q + 3] * rstd);
+        }
+        float* yv = o;   // y = o rstd w (swish(z)), in place
 #pragma unroll
-        for (int u = 0; u < kU; ++u) {
-          const int c = u * 32 + lane;
-          // A columns [32u, 32u + 32) of the warp's 32 rows, transposed
-          uint32_t xa[32];
-          tmem_ld32(acol + u * 32, xa);
-          tmem_wait_ld();
-          __syncwarp();
-          if (lane >= grp * kR && lane < grp * kR + kR) {
-            float* trow = tr + (lane - grp * kR) * 33;
+        for (int e = 0; e < 32; ++e) yv[e] *= rstd * sW[u * 32 + e];
+        if (P.z) {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) trow[e] = __uint_as_float(xa[e]);
-          }
-          __syncwarp();
-          const float rc = eRho[c];
-          const bool bc = eBad[c] != 0;
+          for (int q = 0; q < 4; ++q) {
+            const uint4 z4 = reinterpret_cast<const uint4*>(P.z + orow + u * 32)[q];
+            const uint32_t w4[4] = {z4.x, z4.y, z4.z, z4.w};
 #pragma unroll
-          for (int q = 0; q < kR; ++q) {
-            const float a = tr[q * 33 + lane];
-            const float alpha = rows[rbase + q], ptt = rows[BM + rbase + q];
-            const float fac = bc ? 1.f : ex2((lt[u][q] - rc) * LOG2E);
-            const float val = alpha * fac * a + ptt * vt[u][q];
-            o[q][u] = val;
-            ss[q] += val * val;
+            for (int i = 0; i < 4; ++i) {
+              yv[8 * q + 2 * i] *= swish(__uint_as_float(w4[i] << 16));
+              yv[8 * q + 2 * i + 1] *= swish(__uint_as_float(w4[i] & 0xFFFF0000u));
+            }
           }
         }
-        // the RMSNorm, or without it the softmax denominator: y = o / l; the
-        // saved tensors are then o / l, the log-sum-exp and ones
-        float rstd[kR];
+        if (valid) {
+          if (P.y_f32) {
+            float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(P.y) + orow + u * 32);
 #pragma unroll
-        for (int q = 0; q < kR; ++q)
-          rstd[q] = d.no_norm ? 1.0f / rows[3 * BM + rbase + q]
-                              : 1.0f / sqrtf(warp_sum(ss[q]) / (float)DV + d.eps);
+            for (int q = 0; q < 8; ++q) dst[q] = make_float4(yv[4 * q], yv[4 * q + 1], yv[4 * q + 2], yv[4 * q + 3]);
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(P.y) + orow + u * 32);
 #pragma unroll
-        for (int q = 0; q < kR; ++q) {
-          const int rr = rbase + q;
-          if (rr >= x.len) break;
-          const size_t a0 = ((size_t)x.tok0 + rr) * ors + (size_t)x.h * DV;
-#pragma unroll
-          for (int u = 0; u < kU; ++u) {
-            const int c = u * 32 + lane;
-            float yv = o[q][u] * rstd[q] * sW[c];
-            if (P.z) yv *= swish(bf2f(P.z[a0 + c]));
-            if (yf) yf[a0 + c] = yv;
-            else yb[a0 + c] = f2bf(yv);
-            if (P.o_s) P.o_s[a0 + c] = d.no_norm ? o[q][u] * rstd[q] : o[q][u];
+            for (int q = 0; q < 4; ++q)
+              dst[q] = make_uint4(pack_bf16(yv[8 * q], yv[8 * q + 1]), pack_bf16(yv[8 * q + 2], yv[8 * q + 3]),
+                                  pack_bf16(yv[8 * q + 4], yv[8 * q + 5]), pack_bf16(yv[8 * q + 6], yv[8 * q + 7]));
           }
         }
-        if (P.o_s && lane < kR && rbase + lane < x.len) {
-          float rs = rstd[0];
-#pragma unroll
-          for (int q = 1; q < kR; ++q) rs = lane == q ? rstd[q] : rs;
-          const size_t tk = (size_t)x.tok0 + rbase + lane;
-          const float mt = rows[2 * BM + rbase + lane];
-          P.m_s[tk * d.Hq + x.h] = d.no_norm ? mt + logf(rows[3 * BM + rbase + lane]) : mt;
-          P.rstd_s[tk * d.Hq + x.h] = d.no_norm ? 1.f : rs;
-        }
+      }
+      if (P.o_s && valid) {
+        P.m_s[tk * d.Hq + x.h] = d.no_norm ? mt + logf(lsum) : mt;
+        P.rstd_s[tk * d.Hq + x.h] = d.no_norm ? 1.f : rstd;
       }
       tc_fence_before();
       mbar_arrive(&bar->acc_empty[tb]);
       mbar_arrive(&bar->rows_free[tb]);
-      wg_sync(3);
+      wg_sync(3, 128);
       ++nt;
     }
   }

@@ -49,7 +49,7 @@ class Case:
     name: str = ""
 
 
-# The five workloads of the FiX operator studied here.  Sizes are those of the
+# The workloads of the FiX operator studied here.  Sizes are those of the
 # FiX README's Quick Start example (B2, T2048, 8 q heads over 4 kv heads, D128)
 # and of typical long-context / training shapes.
 WORKLOADS = {
@@ -64,6 +64,12 @@ WORKLOADS = {
             name="fwd B1 T32768 Hq32 Hkv8 D128"),
     5: Case(8, 4096, 16, 16, 64, 64, 2.0, 2.0, "normal", backward=True,
             name="fwd+bwd B8 T4096 Hq16 Hkv16 D64"),
+    # workload 2's shape with heterogeneous decay: a per-channel shift of the
+    # gate logit (std 2.5) makes about a fifth of the channels forget fast
+    # enough that their in-chunk range exceeds the decay split's float range
+    6: Case(2, 2048, 8, 4, 128, 128, 1.0, 1.0, "normal", backward=True,
+            channel_bias_std=2.5,
+            name="fwd+bwd B2 T2048 Hq8 Hkv4 D128, fast-decay channels (bias std 2.5)"),
 }
 
 

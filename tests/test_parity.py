@@ -57,23 +57,35 @@ SMALL = {
     "T520-D128": dict(B=1, T=520, Hq=2, Hkv=1, Dk=128, Dv=128),
     "varlen": dict(B=1, T=0, Hq=4, Hkv=2, Dk=64, Dv=64, seqlens=[0, 1, 130, 7, 255, 0, 64, 300]),
     "fast-channels": dict(B=1, T=300, Hq=2, Hkv=1, Dk=64, Dv=64, g_mean=1.0, channel_bias_std=2.5),
+    "T520-D128-gqa-fast-channels": dict(B=1, T=520, Hq=4, Hkv=2, Dk=128, Dv=128, g_mean=1.0,
+                                        channel_bias_std=2.5),
     "readme-randn-gate": dict(B=1, T=200, Hq=2, Hkv=1, Dk=64, Dv=64, raw_gate=True, g_mean=0.0),
 }
 
 
-# Gates above 0 (the README draws g = randn) make exp(G_t - G_s) grow with
-# distance; the tensor-core path then runs the off-diagonal blocks in bf16
-# (8-bit significand) instead of fp16, so its largest element error is looser
-# than the workloads' bar (measured 7e-2 at max |y| ~ 8).  rel-L2 keeps the bar.
-POSITIVE_GATE_MAX_ABS = 1e-1
+def out_of_range_channels(case):
+    """(chunk, kv head, channel) triples whose in-chunk gate range exceeds
+    the decay split's float range (half-range above 80): the kernels handle
+    their diagonal terms exactly in fp32."""
+    g = case["g"].double().numpy()
+    n = 0
+    for b, T in enumerate(case["seqlens"] if case["cu_seqlens"] is None else [None]):
+        seqs = ([(b, 0, T)] if T is not None else
+                [(0, int(a), int(e)) for a, e in zip(case["cu_seqlens"][:-1], case["cu_seqlens"][1:])])
+        for bb, a, e in seqs:
+            for c0 in range(a, e, 128):
+                L = np.cumsum(g[bb, c0:min(c0 + 128, e)], axis=0)
+                rng = L.max(axis=0) - L.min(axis=0)
+                n += int((rng / 2 > 80).sum())
+    return n
 
 
 @pytest.mark.parametrize("name", ["T520-D128", "fast-channels", "varlen"])
 def test_backward_reusing_forward_workspace_is_identical(cuda_lib, name):
     """FIX_FLAG_REUSE_FWD_WORKSPACE: the backward reads the forward's gate
     prefix results instead of recomputing them (for "fast-channels" that
-    includes the flag that sends out-of-range channels to the exact kernels);
-    the gradients are bit-identical to a backward that recomputes."""
+    includes the out-of-range channel flags); the gradients are bit-identical
+    to a backward that recomputes."""
     case = synth.make_case(**SMALL[name], seed=7)
     a = run_gpu(case, "auto", backward=True, reuse=True)
     b = run_gpu(case, "auto", backward=True, reuse=False)
@@ -85,13 +97,11 @@ def test_backward_reusing_forward_workspace_is_identical(cuda_lib, name):
 @pytest.mark.parametrize("name", list(SMALL))
 def test_small_shapes(cuda_lib, name, algo):
     case = synth.make_case(**SMALL[name], seed=42)
+    if "fast-channels" in name:
+        assert out_of_range_channels(case) > 0, "the case must exercise the exact diagonal terms"
     gpu = run_gpu(case, algo, backward=True)
     ref = oracle_full(case, backward=True)
-    if SMALL[name].get("raw_gate") and algo != "simt":
-        e, m = rel_l2(gpu["y"], ref["y"]), max_abs(gpu["y"], ref["y"])
-        assert e <= FWD_REL_L2 and m <= POSITIVE_GATE_MAX_ABS, (name, e, m)
-    else:
-        check_fwd(gpu["y"], ref["y"], name)
+    check_fwd(gpu["y"], ref["y"], name)
     for key in GRADS:
         check_grad(key, gpu[key], ref[key], name)
     # the saved tensors are consistent with y
