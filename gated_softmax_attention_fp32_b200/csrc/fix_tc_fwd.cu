@@ -37,17 +37,18 @@
 // exp(L_t) A_t + sum_{s<t} P_ts exp(L_t - L_s) v_s (fp32) in place; the
 // epilogue then applies no row factor to them.
 //
-// Warp roles (512 threads):
+// Warp roles (384 threads):
 //   warp 0       TMA producer: Q per tile, K and V (Vt / Vm hi) through
 //                2-stage rings, Vm lo of the diagonal block
 //   warp 1       MMA issuer (one thread) and TMEM owner
-//   warps 4-7    softmax: S -> P in TMEM, lazy row-max rescale, the fold,
-//                the exact sums of out-of-range channels
-//   warps 8-11   V scaling: V'' in shared memory, the tile's fold factors
-//   warps 12-15  epilogue of the previous tile, overlapping this one's MMAs:
-//                TMEM -> registers -> a per-warp transpose in shared memory,
-//                lanes over channels for coalesced loads of L, v and stores
-//                of y, o, m, rstd
+//   warps 2-3    V scaling: V'' in shared memory, the tile's fold factors
+//   warps 4-7    softmax, a thread per query row: S -> P in TMEM.  Earlier
+//                blocks in one pass (lazy row-max reference, moved in place
+//                when a 32-key chunk exceeds it), the diagonal in two (row
+//                max first); the fold; the exact sums of out-of-range channels
+//   warps 8-11   epilogue of the previous tile, overlapping this one's MMAs:
+//                a thread per row, its L, v and output rows loaded and
+//                stored with 16-byte accesses
 // TMEM (512 columns): S/P double buffer at 0 and 128 (P written over S as
 // 16-bit pairs; the diagonal's P_lo in the buffer's upper half), and the
 // accumulator A double-buffered by tile parity at 256 and 256 + DV.
