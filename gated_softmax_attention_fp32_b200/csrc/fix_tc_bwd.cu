@@ -358,12 +358,14 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             }
           }
+          // masked by selection: above the diagonal dOm Vm pairs
+          // exp(L_t - rho) with exp(rho - L_s) for s > t and may overflow
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
             const int key = c4 * 32 + e;
-            const float p0 = key <= r ? ex2(__uint_as_float(xs[e]) * c1 - moff) : 0.f;
-            const float p1 = key + 1 <= r ? ex2(__uint_as_float(xs[e + 1]) * c1 - moff) : 0.f;
-            pk[e >> 1] = pack_bf16(p0 * (__uint_as_float(xp[e]) - dl), p1 * (__uint_as_float(xp[e + 1]) - dl));
+            const float d0 = key <= r ? ex2(__uint_as_float(xs[e]) * c1 - moff) * (__uint_as_float(xp[e]) - dl) : 0.f;
+            const float d1 = key + 1 <= r ? ex2(__uint_as_float(xs[e + 1]) * c1 - moff) * (__uint_as_float(xp[e + 1]) - dl) : 0.f;
+            pk[e >> 1] = pack_bf16(d0, d1);
           }
         }
         tmem_st16(lane_base + kColS + c4 * 16, pk);
@@ -787,8 +789,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             } else {
               ph[e >> 1] = cta_f16 ? pack_f16(pv[0], pv[1]) : pack_bf16(pv[0], pv[1]);
             }
-            pd[e >> 1] = pack_bf16(p[0] * (__uint_as_float(xp[e]) - dlrow[32 * h + e]),
-                                   p[1] * (__uint_as_float(xp[e + 1]) - dlrow[32 * h + e + 1]));
+            // masked by selection (dP^T above the diagonal may overflow)
+            const float d0 = 32 * h + e >= lo && 32 * h + e < qlen
+                                 ? p[0] * (__uint_as_float(xp[e]) - dlrow[32 * h + e]) : 0.f;
+            const float d1 = 32 * h + e + 1 >= lo && 32 * h + e + 1 < qlen
+                                 ? p[1] * (__uint_as_float(xp[e + 1]) - dlrow[32 * h + e + 1]) : 0.f;
+            pd[e >> 1] = pack_bf16(d0, d1);
           }
         }
         tmem_st16(lane_base + col_s(b) + 16 * h, ph);

@@ -742,23 +742,44 @@ __global__ void __launch_bounds__(kThreads, 1)
       float delta[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) delta[e] = 0.f;
+      // the per-block values (the total of chunk j + 1 that extends the
+      // running sum, the exponents of chunk j) are loaded one block ahead
+      auto fetch = [&](int it, float4 (&t)[2], float4 (&l)[2]) {
+        const int j = x.j - 1 - it;
+        const bool off = it < x.nblk - 1;
+        const size_t cb = (size_t)x.kv * DV + lc * 8;
+        if (off && it >= 1) {
+          const float4* tp = reinterpret_cast<const float4*>(P.tot + (size_t)(x.first + j + 1) * d.Hkv * DV + cb);
+          t[0] = tp[0];
+          t[1] = tp[1];
+        } else {
+          t[0] = t[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        if (off) {
+          const float4* lp = reinterpret_cast<const float4*>(P.lvt + (size_t)(x.first + j) * d.Hkv * DV + cb);
+          l[0] = lp[0];
+          l[1] = lp[1];
+        } else {
+          l[0] = l[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      };
+      float4 tcur[2], lcur[2];
+      fetch(0, tcur, lcur);
       for (int it = 0; it < x.nblk; ++it) {
         const bool diag = it == x.nblk - 1;
         const int sv = vc & 1;
+        float4 tnxt[2], lnxt[2];
+        if (!diag) fetch(it + 1, tnxt, lnxt);
         float f8[8];
         if (!diag) {
-          const int j = x.j - 1 - it;
-          if (it >= 1) {
-            const float* tp = P.tot + ((size_t)(x.first + j + 1) * d.Hkv + x.kv) * DV + lc * 8;
-            const float4 t0 = *reinterpret_cast<const float4*>(tp);
-            const float4 t1 = *reinterpret_cast<const float4*>(tp + 4);
-            delta[0] += t0.x; delta[1] += t0.y; delta[2] += t0.z; delta[3] += t0.w;
-            delta[4] += t1.x; delta[5] += t1.y; delta[6] += t1.z; delta[7] += t1.w;
-          }
+          const float t8[8] = {tcur[0].x, tcur[0].y, tcur[0].z, tcur[0].w, tcur[1].x, tcur[1].y, tcur[1].z, tcur[1].w};
+          const float l8[8] = {lcur[0].x, lcur[0].y, lcur[0].z, lcur[0].w, lcur[1].x, lcur[1].y, lcur[1].z, lcur[1].w};
           // Vt is stored as fp16 times 2^-e; V'' = Vt_true f_ij 2^-k
-          const float* lv = P.lvt + ((size_t)(x.first + j) * d.Hkv + x.kv) * DV + lc * 8;
 #pragma unroll
-          for (int e = 0; e < 8; ++e) f8[e] = ex2(delta[e] * LOG2E + vt_exponent(lv[e]) - kexp[e]);
+          for (int e = 0; e < 8; ++e) {
+            delta[e] += t8[e];
+            f8[e] = ex2(delta[e] * LOG2E + vt_exponent(l8[e]) - kexp[e]);
+          }
         }
         // factors in fp16 when they are normal fp16 numbers (always with g <=
         // 0): then V'' = Vt f is one packed fp16 multiply per channel pair on
@@ -804,6 +825,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mbar_arrive(&bar->v_ready[sv]);
         ++vc;
+        if (!diag) {
+          tcur[0] = tnxt[0]; tcur[1] = tnxt[1];
+          lcur[0] = lnxt[0]; lcur[1] = lnxt[1];
+        }
       }
       ++nt;
     }
