@@ -128,7 +128,7 @@ static SplitPlan plan_split(const fix_attn_problem* p, const Dims& d) {
 
 // Workspace layout (all offsets 256-byte aligned).
 struct Ws {
-  size_t status, chunks, order, safe, L, vt, vm, vml, tot, rho, hr, lvt;   // forward and backward
+  size_t status, chunks, order, safe, L, Lt, vt, vm, vml, tot, rho, hr, lvt;   // forward and backward
   size_t dow, dot, domh, doml, dsafe, hmax, ptt, delta, A, dG, dtot, dwp, dgf;   // backward only
   size_t parts, cpart, partial;                            // dk/dv work split
   size_t total;
@@ -149,6 +149,7 @@ static Ws layout(const Dims& d, bool bwd, const SplitPlan& sp) {
   w.order = take((size_t)(d.nchunks > 0 ? d.nchunks : 1) * sizeof(int));
   w.safe = take((size_t)(d.nchunks > 0 ? d.nchunks : 1) * d.Hkv * sizeof(int));
   w.L = take(nkv * 4);
+  w.Lt = take(nkv * 4);   // L channel-major [Hkv][Dv][N], for the forward's epilogue
   w.vt = take(nkv * 2);
   w.vm = take(nkv * 2);
   w.vml = take(nkv * 2);
@@ -354,8 +355,8 @@ static fix_status upload_schedule(const fix_attn_problem* p, const Dims& d, cons
 }
 
 static fix_status run_prefix(const Dims& d, const fix_attn_problem* p, const Ws& ws, char* base,
-                             const float* g, const void* v, bool want_vt, const SplitPlan* sp,
-                             int* hmax, bool reuse, cudaStream_t st) {
+                             const float* g, const void* v, bool want_vt, bool want_lt,
+                             const SplitPlan* sp, int* hmax, bool reuse, cudaStream_t st) {
   const Chunk* chunks = reinterpret_cast<const Chunk*>(base + ws.chunks);
   FIX_TRY(upload_schedule(p, d, ws, base, sp, reuse, st));
   if (d.nchunks == 0) return FIX_OK;
@@ -368,6 +369,7 @@ static fix_status run_prefix(const Dims& d, const fix_attn_problem* p, const Ws&
   }
   prefix_kernel<<<dim3(d.nchunks, d.Hkv, (d.Dv + 31) / 32), 256, 0, st>>>(
       d, chunks, g, static_cast<const __nv_bfloat16*>(v), reinterpret_cast<float*>(base + ws.L),
+      want_lt ? reinterpret_cast<float*>(base + ws.Lt) : nullptr,
       want_vt ? reinterpret_cast<uint16_t*>(base + ws.vt) : nullptr,
       reinterpret_cast<__nv_bfloat16*>(base + ws.vm),
       reinterpret_cast<__nv_bfloat16*>(base + ws.vml), reinterpret_cast<float*>(base + ws.tot),
@@ -429,7 +431,7 @@ fix_status fix_attn_fwd(const fix_attn_problem* p, const void* q, const void* k,
   if (d.N == 0) return FIX_OK;
   const bool tc = p->algo != FIX_ALGO_SIMT && tc_fwd_supported(d);
   FIX_TRY(mark(p, FIX_STAGE_FWD_PREFIX, 0, st));
-  FIX_TRY(run_prefix(d, p, ws, base, g, v, tc, nullptr, nullptr, false, st));
+  FIX_TRY(run_prefix(d, p, ws, base, g, v, tc, tc, nullptr, nullptr, false, st));
   FIX_TRY(mark(p, FIX_STAGE_FWD_PREFIX, 1, st));
   const Chunk* chunks = reinterpret_cast<const Chunk*>(base + ws.chunks);
   const float* L = reinterpret_cast<const float*>(base + ws.L);
@@ -439,7 +441,8 @@ fix_status fix_attn_fwd(const fix_attn_problem* p, const void* q, const void* k,
     FIX_TRY(tc_fwd(d, chunks, reinterpret_cast<const int*>(base + ws.order), q, k,
                    reinterpret_cast<const uint16_t*>(base + ws.vt),
                    reinterpret_cast<const __nv_bfloat16*>(base + ws.vm),
-                   reinterpret_cast<const __nv_bfloat16*>(base + ws.vml), v, L, tot,
+                   reinterpret_cast<const __nv_bfloat16*>(base + ws.vml), v, L,
+                   reinterpret_cast<const float*>(base + ws.Lt), tot,
                    reinterpret_cast<const float*>(base + ws.rho),
                    reinterpret_cast<const float*>(base + ws.hr),
                    reinterpret_cast<const float*>(base + ws.lvt),
@@ -493,7 +496,7 @@ fix_status fix_attn_bwd(const fix_attn_problem* p, const void* q, const void* k,
     return FIX_OK;
   }
   FIX_TRY(mark(p, FIX_STAGE_BWD_PREFIX, 0, st));
-  FIX_TRY(run_prefix(d, p, ws, base, g, v, tc, tc ? &sp : nullptr,
+  FIX_TRY(run_prefix(d, p, ws, base, g, v, tc, false, tc ? &sp : nullptr,
                      tc ? reinterpret_cast<int*>(base + ws.hmax) : nullptr, reuse, st));
   FIX_TRY(mark(p, FIX_STAGE_BWD_PREFIX, 1, st));
   const Chunk* chunks = reinterpret_cast<const Chunk*>(base + ws.chunks);

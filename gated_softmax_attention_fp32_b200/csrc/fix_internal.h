@@ -23,7 +23,7 @@ struct DecodeDims {
 template <int NW>
 __global__ void upload_kernel(const __grid_constant__ Blob<NW> b, uint32_t* dst, int nwords);
 __global__ void prefix_kernel(Dims d, const Chunk* chunks, const float* g, const __nv_bfloat16* v,
-                              float* L, uint16_t* vt, __nv_bfloat16* vm, __nv_bfloat16* vml,
+                              float* L, float* Lt, uint16_t* vt, __nv_bfloat16* vm, __nv_bfloat16* vml,
                               float* tot, float* rho, float* hr, float* lvt, int* safe,
                               int* badflag, int* hmax);
 __global__ void chunk_total_kernel(Dims d, const Chunk* chunks, const float* x, float* tot);
@@ -68,7 +68,7 @@ bool tc_fwd_supported(const Dims& d);
 fix_status tc_fwd(const Dims& d, const Chunk* chunks, const int* order, const void* q,
                   const void* k, const uint16_t* vt, const __nv_bfloat16* vm,
                   const __nv_bfloat16* vml, const void* v,
-                  const float* L, const float* tot, const float* rho, const float* hr,
+                  const float* L, const float* Lt, const float* tot, const float* rho, const float* hr,
                   const float* lvt, const int* safe,
                   const void* w, const void* z, void* y, bool y_f32, float* o_s, float* m_s,
                   float* rstd_s, int* status, cudaStream_t st);

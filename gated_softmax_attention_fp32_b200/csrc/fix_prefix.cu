@@ -57,11 +57,13 @@ constexpr int kPrefixRows = FIX_CHUNK / kPrefixGroups;    // rows per thread
 
 __global__ void __launch_bounds__(kPrefixThreads) prefix_kernel(
     Dims d, const Chunk* __restrict__ chunks, const float* __restrict__ g,
-    const __nv_bfloat16* __restrict__ v, float* __restrict__ L, uint16_t* __restrict__ vt,
+    const __nv_bfloat16* __restrict__ v, float* __restrict__ L, float* __restrict__ Lt,
+    uint16_t* __restrict__ vt,
     __nv_bfloat16* __restrict__ vm, __nv_bfloat16* __restrict__ vml, float* __restrict__ tot,
     float* __restrict__ rho, float* __restrict__ hr, float* __restrict__ lvt,
     int* __restrict__ safe, int* __restrict__ badflag, int* __restrict__ hmax) {
   __shared__ float part[kPrefixThreads], pmin[kPrefixThreads], pmax[kPrefixThreads];
+  __shared__ float tr[32][FIX_CHUNK + 1];   // the slab of L, channel-major (for Lt)
   const int Dv = d.Dv;
   const int cl = threadIdx.x & 31, grp = threadIdx.x >> 5;
   const int c = blockIdx.z * 32 + cl;
@@ -118,9 +120,21 @@ __global__ void __launch_bounds__(kPrefixThreads) prefix_kernel(
     if (u < nr) {
       lv[u] += off;
       L[base + (size_t)(r0 + u) * rs] = lv[u];
+      if (Lt) tr[cl][r0 + u] = lv[u];
     }
   const size_t ti = ((size_t)ci * d.Hkv + kv) * Dv + c;
   if (grp == 0 && act) tot[ti] = total;
+  if (Lt) {
+    // L channel-major: a warp writes 32 consecutive tokens of one channel
+    __syncthreads();
+    const int lane = threadIdx.x & 31;
+    for (int j = grp; j < 32; j += kPrefixGroups) {
+      const int cj = blockIdx.z * 32 + j;
+      if (cj >= Dv) break;
+      float* dst = Lt + ((size_t)kv * Dv + cj) * d.N + ch.tok0;
+      for (int r = lane; r < ch.len; r += 32) dst[r] = tr[j][r];
+    }
+  }
   if (!vt) return;  // uniform: the exact kernels need only L and tot
   float vmax = 0.f, xmax = 0.f;
 #pragma unroll

@@ -103,12 +103,15 @@ __device__ __forceinline__ uint4 pack8(const float* x, bool f16) {
   }
   return r;
 }
-// Whether 8 scale factors are normal fp16 numbers no larger than 2, so that a
-// packed fp16 multiply by them loses nothing to range.
+// Whether 8 scale factors are no larger than 2, so that a packed fp16
+// multiply by them cannot overflow.  A factor below fp16's normal range
+// (2^-14) loses relative precision or becomes 0, but every value it scales is
+// then already below 2^-14 of its undecayed size (absolute error under
+// 2^-24 of it).
 __device__ __forceinline__ bool f16_factors(const float* f) {
   bool ok = true;
 #pragma unroll
-  for (int e = 0; e < 8; ++e) ok = ok && f[e] >= 6.2e-5f && f[e] <= 2.f;
+  for (int e = 0; e < 8; ++e) ok = ok && f[e] <= 2.f;
   return ok;
 }
 
@@ -1264,11 +1267,14 @@ __global__ void __launch_bounds__(kFixThreads, 1) dkv_diag_exact_kernel(const Pa
 #pragma unroll
         for (int u = 0; u < 4; ++u) ls[u] = sL[(4 * cg + u) * BN + s_dv];
         for (int t = t_dv; t < n; ++t) {   // warp-uniform t: broadcast reads
-          const float pts = t > s_dv ? sP[t * Lay::kPs + s_dv] : 0.f;
+          // selected, not multiplied by zero: exp(L_t - L_s) overflows for t < s
+          if (t > s_dv) {
+            const float pts = sP[t * Lay::kPs + s_dv];
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int b = 4 * cg + u;
-            dvb[u] += pts * ex2((sL[b * BN + t] - ls[u]) * LOG2E) * sDo[b * BN + t];
+            for (int u = 0; u < 4; ++u) {
+              const int b = 4 * cg + u;
+              dvb[u] += pts * ex2((sL[b * BN + t] - ls[u]) * LOG2E) * sDo[b * BN + t];
+            }
           }
         }
 #pragma unroll

@@ -27,14 +27,15 @@
 //   * diagonal block: exp(G_t - G_s) = exp(L_t - rho) exp(rho - L_s), both
 //     factors in [e^-80, e^80]; Vm_s = v_s exp(rho - L_s) comes from the
 //     prefix pass as bf16 hi + lo, and P as bf16 hi + lo, so the block costs
-//     three MMAs (P_hi Vm_hi + P_lo Vm_hi + P_hi Vm_lo) and is near-exact.
-//     The s = t pair is left out of the MMAs.
-//   * epilogue: o_t = alpha_t exp(L_t - rho) A_t + P_tt v_t (alpha_t =
-//     exp(m_used - m_t) undoes the lazily updated row shift; the s = t term
-//     is exact in fp32), then the RMSNorm.
+//     three MMAs (P_hi Vm_hi + P_lo Vm_hi + P_hi Vm_lo) and is near-exact
+//     (keys s <= t, the s = t pair included).
+//   * epilogue: o_t = alpha_t exp(L_t - rho) A_t (alpha_t = exp(m_used - m_t)
+//     undoes the lazily updated row shift), then the RMSNorm.  L comes from
+//     a channel-major copy (prefix pass), so that the row factors of a warp's
+//     32 rows are one coalesced load per channel.
 // Channels outside the split's range (prefix pass: rho = 0, Vm = 0) get no
 // fold beyond 2^k_c, and the softmax warps add their exact diagonal sum
-// exp(L_t) A_t + sum_{s<t} P_ts exp(L_t - L_s) v_s (fp32) in place; the
+// exp(L_t) A_t + sum_{s<=t} P_ts exp(L_t - L_s) v_s (fp32) in place; the
 // epilogue then applies no row factor to them.
 //
 // Warp roles (384 threads):
@@ -98,7 +99,7 @@ struct Layout {
   static constexpr int kF = kVl + BN * DV * 2;           // [2][DV] f32 fold factors
   static constexpr int kBad = kF + 2 * DV * 4;           // [2][DV] int out-of-range flags
   static constexpr int kAnyBad = kBad + 2 * DV * 4;      // [2] int
-  static constexpr int kRows = kAnyBad + 16;             // [2][4][BM] f32: alpha, P_tt, m, l
+  static constexpr int kRows = kAnyBad + 16;             // [2][4][BM] f32: alpha, (unused), m, l
   static constexpr int kPlo = kRows + 2 * 4 * BM * 4;    // [BM][33] u32: diagonal P_lo, key chunks 0-1
   static constexpr int kEpiW = kPlo + BM * 33 * 4;       // [DV] f32 w
   static constexpr int kEpiRho = kEpiW + DV * 4;         // [DV] f32 rho of the epilogue's tile
@@ -120,6 +121,7 @@ struct Params {
   const __nv_bfloat16* k;
   const __nv_bfloat16* v;
   const float* L;
+  const float* Lt;            // L channel-major [Hkv][DV][N]
   const float* tot;
   const float* rho;
   const float* hr;
@@ -405,7 +407,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (x.len <= 0) continue;
       const int tb = nt & 1, use = nt >> 1;
       const uint32_t acol = lane_base + 256u + (uint32_t)(tb * DV);
-      float m_used = -INFINITY, m_true = -INFINITY, s_diag = 0.f;
+      float m_used = -INFINITY, m_true = -INFINITY;
       float l_used = 0.f;   // without the norm: sum of P relative to m_used
       for (int it = 0; it < x.nblk; ++it) {
         const bool diag = it == x.nblk - 1;
@@ -508,8 +510,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (d.no_norm) l_used += ls;
         } else {
-          // pass 1: the row maximum (diagonal block: keys s <= t; S_tt kept
-          // for the exact s = t term)
+          // pass 1: the row maximum (diagonal block: keys s <= t)
           float mx = -INFINITY;
 #pragma unroll
           for (int c4 = 0; c4 < BN / 32; ++c4) {
@@ -518,10 +519,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_wait_ld(xs);
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
-              const float sv = __uint_as_float(xs[e]);
               const int key = c4 * 32 + e;
-              mx = key <= r ? fmaxf(mx, sv) : mx;
-              s_diag = key == r ? sv : s_diag;
+              mx = key <= r ? fmaxf(mx, __uint_as_float(xs[e])) : mx;
             }
           }
           m_true = fmaxf(m_true, mx * d.scale);
@@ -574,9 +573,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float moff = m_used * LOG2E;
           if (diag && sAnyBad[tb]) {
             // exact diagonal sums of out-of-range channels, in fp32 from the
-            // fp32 logits: A_tc <- exp(L_t) A_tc + sum_{s<t} P_ts exp(L_t - L_s) v_s
+            // fp32 logits: A_tc <- exp(L_t) A_tc + sum_{s<=t} P_ts exp(L_t - L_s) v_s
             const int* bad = sBad + tb * DV;
-            const int nk = r < x.len ? r : 0;
+            const int nk = r < x.len ? r + 1 : 0;
             const size_t rowL = ((size_t)x.tok0 + (r < x.len ? r : 0)) * vrs + (size_t)x.kv * DV;
             const float* Lk = P.L + (size_t)x.tok0 * vrs + (size_t)x.kv * DV;
             const __nv_bfloat16* vk = P.v + (size_t)x.tok0 * vrs + (size_t)x.kv * DV;
@@ -622,8 +621,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
               for (int e = 0; e < 32; e += 2) {
                 const int key = c4 * 32 + e;
-                const float p0 = key < r ? ex2(__uint_as_float(xs[e]) * c1 - moff) : 0.f;
-                const float p1 = key + 1 < r ? ex2(__uint_as_float(xs[e + 1]) * c1 - moff) : 0.f;
+                const float p0 = key <= r ? ex2(__uint_as_float(xs[e]) * c1 - moff) : 0.f;
+                const float p1 = key + 1 <= r ? ex2(__uint_as_float(xs[e + 1]) * c1 - moff) : 0.f;
                 if (d.no_norm) l_used += p0 + p1;
                 ph[e >> 1] = pack_bf16(p0, p1);
                 const float h0 = __uint_as_float(ph[e >> 1] << 16);
@@ -661,11 +660,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (use >= 1 && !__all_sync(0xffffffffu, mbar_wait(&bar->rows_free[tb], (use - 1) & 1, ctl))) { ok = false; break; }
       float* rows = sRows + tb * 4 * BM;
       const float alpha = ex2((m_used - m_true) * LOG2E);
-      const float ptt = ex2((s_diag * d.scale - m_true) * LOG2E);
       rows[r] = alpha;
-      rows[BM + r] = ptt;                                          // P_tt
       rows[2 * BM + r] = m_true;
-      rows[3 * BM + r] = alpha * l_used + ptt;                     // l (no norm)
+      rows[3 * BM + r] = alpha * l_used;                           // l (no norm)
       mbar_arrive(&bar->rows_ready[tb]);
       ++nt;
     }
@@ -781,21 +778,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             f8[e] = ex2(delta[e] * LOG2E + vt_exponent(l8[e]) - kexp[e]);
           }
         }
-        // factors in fp16 when they are normal fp16 numbers (always with g <=
-        // 0): then V'' = Vt f is one packed fp16 multiply per channel pair on
-        // the FMA pipe, with no conversion; otherwise in fp32
-        bool h16 = true;
+        // Factors no larger than 2 (always with g <= 0) go to fp16: V'' = Vt f
+        // is then one packed fp16 multiply per channel pair, with no
+        // conversion.  A factor below fp16's normal range (2^-14) loses
+        // relative precision or becomes 0, but then every value it scales is
+        // already below 2^-14 of its undecayed size, an absolute error under
+        // 2^-24 |v|.  Factors that are all exactly 1 leave Vt as it is;
+        // larger ones take the fp32 path.
+        bool h16 = true, unit = true;
         __half2 fh[4];
         if (!diag) {
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            h16 = h16 && f8[2 * u] >= 6.2e-5f && f8[2 * u + 1] >= 6.2e-5f && f8[2 * u] <= 2.f &&
-                  f8[2 * u + 1] <= 2.f;
+            h16 = h16 && f8[2 * u] <= 2.f && f8[2 * u + 1] <= 2.f;
+            unit = unit && f8[2 * u] == 1.f && f8[2 * u + 1] == 1.f;
             fh[u] = __floats2half2_rn(f8[2 * u], f8[2 * u + 1]);
           }
         }
         if (!wg_and(2, kVsThreads, mbar_wait(&bar->v_full[sv], (vc >> 1) & 1, ctl))) { ok = false; break; }
-        if (!diag) {
+        if (!diag && !unit) {
           uint8_t* vb = reinterpret_cast<uint8_t*>(sV + sv * BN * DV) + half * (BN * 128);
           if (h16) {
 #pragma unroll 4
@@ -857,18 +858,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int tb = nt & 1, use = nt >> 1;
       const bool valid = r < x.len;
       const size_t tk = (size_t)x.tok0 + (valid ? r : 0);
-      const float* Lr = P.L + tk * vrs + (size_t)x.kv * DV;
-      const __nv_bfloat16* vr = P.v + tk * vrs + (size_t)x.kv * DV;
+      // L of this row, channel-major: for a channel, the warp's 32 rows are
+      // 32 consecutive floats
+      const float* Lr = P.Lt + (size_t)x.kv * DV * d.N + tk;
       const size_t orow = tk * ors + (size_t)x.h * DV;
-      // While the tile's MMAs run, pull this row's L, v (and output gate)
-      // into L2.
+      // While the tile's MMAs run, pull the tile's L (and this row's output
+      // gate) into L2.
+      if (et < DV && x.len > 0) {
+        const char* lc = reinterpret_cast<const char*>(P.Lt + ((size_t)x.kv * DV + et) * d.N + x.tok0);
+        for (int b = 0; b < x.len * 4; b += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(lc + b));
+      }
       if (valid) {
-#pragma unroll
-        for (int b = 0; b < DV * 4; b += 128)
-          asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<const char*>(Lr) + b));
-#pragma unroll
-        for (int b = 0; b < DV * 2; b += 128)
-          asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<const char*>(vr) + b));
         if (P.z) {
 #pragma unroll
           for (int b = 0; b < DV * 2; b += 128)
@@ -890,31 +890,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       const float* rows = sRows + tb * 4 * BM;
-      const float alpha = rows[r], ptt = rows[BM + r], mt = rows[2 * BM + r], lsum = rows[3 * BM + r];
+      const float alpha = rows[r], mt = rows[2 * BM + r], lsum = rows[3 * BM + r];
       const uint32_t acol = lane_base + 256u + (uint32_t)(tb * DV);
-      // o for channels [32 u, 32 u + 32): alpha exp(L - rho) A + P_tt v
-      // (no row factor for out-of-range channels)
+      // o for channels [32 u, 32 u + 32): alpha exp(L - rho) A (A holds the
+      // s = t term too; no row factor for out-of-range channels)
       auto chunk_o = [&](int u, float (&o)[32]) {
         uint32_t xa[32];
         tmem_ld32(acol + u * 32, xa);
-        float4 l4[8];
-        uint4 v4[4];
+        float le[32];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) l4[q] = reinterpret_cast<const float4*>(Lr + u * 32)[q];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) v4[q] = reinterpret_cast<const uint4*>(vr + u * 32)[q];
-        tmem_wait_ld();
+        for (int e = 0; e < 32; ++e) le[e] = Lr[(size_t)(u * 32 + e) * d.N];
+        tmem_wait_ld(xa);
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
           const int c = u * 32 + e;
-          const float4 lq = l4[e >> 2];
-          const float le = (e & 3) == 0 ? lq.x : (e & 3) == 1 ? lq.y : (e & 3) == 2 ? lq.z : lq.w;
-          const uint4 vq = v4[e >> 3];
-          const uint32_t vw = ((e >> 1) & 3) == 0 ? vq.x : ((e >> 1) & 3) == 1 ? vq.y
-                            : ((e >> 1) & 3) == 2 ? vq.z : vq.w;
-          const float ve = __uint_as_float((e & 1) ? (vw & 0xFFFF0000u) : (vw << 16));
-          const float fac = eBad[c] ? 1.f : ex2((le - eRho[c]) * LOG2E);
-          o[e] = alpha * fac * __uint_as_float(xa[e]) + ptt * ve;
+          const float fac = eBad[c] ? 1.f : ex2((le[e] - eRho[c]) * LOG2E);
+          o[e] = alpha * fac * __uint_as_float(xa[e]);
         }
       };
       // pass 1: the sum of squares (and the saved o)
@@ -1066,7 +1057,7 @@ int tc_fwd_kernel_count(const Dims&) { return 1; }
 fix_status tc_fwd(const Dims& d, const Chunk* chunks, const int* order, const void* q,
                   const void* k, const uint16_t* vt, const __nv_bfloat16* vm,
                   const __nv_bfloat16* vml, const void* v,
-                  const float* L, const float* tot, const float* rho, const float* hr,
+                  const float* L, const float* Lt, const float* tot, const float* rho, const float* hr,
                   const float* lvt, const int* safe,
                   const void* w, const void* z, void* y, bool y_f32, float* o_s, float* m_s,
                   float* rstd_s, int* status, cudaStream_t st) {
@@ -1081,6 +1072,7 @@ fix_status tc_fwd(const Dims& d, const Chunk* chunks, const int* order, const vo
   prm.k = static_cast<const __nv_bfloat16*>(k);
   prm.v = static_cast<const __nv_bfloat16*>(v);
   prm.L = L;
+  prm.Lt = Lt;
   prm.tot = tot;
   prm.rho = rho;
   prm.hr = hr;

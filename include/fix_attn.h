@@ -203,9 +203,9 @@ fix_status fix_attn_decode(const fix_attn_problem *p, const int32_t *seqlens, co
 fix_status fix_attn_device_status(const void *workspace, void *stream);
 
 /* Largest workspace fix_attn_fwd_noalloc can provide: 16 MiB.  The forward's
- * workspace is about 10 bytes per (token, kv head, value channel) plus a few
- * KB, so the array covers N * Hkv * Dv up to about 1.6 million: e.g. 3,200
- * tokens x 4 kv heads x Dv 128, or 6,400 tokens x 4 kv heads x Dv 64.
+ * workspace is about 14 bytes per (token, kv head, value channel) plus a few
+ * KB, so the array covers N * Hkv * Dv up to about 1.18 million: e.g. 2,300
+ * tokens x 4 kv heads x Dv 128, or 4,600 tokens x 4 kv heads x Dv 64.
  * fix_attn_workspace_bytes(p, 0) gives the exact figure for a problem. */
 #define FIX_NOALLOC_MAX_WORKSPACE_BYTES (16u * 1024u * 1024u)
 

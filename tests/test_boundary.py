@@ -91,10 +91,11 @@ def _expected_workspace(seqlens, Hq, Hkv, Dk, Dv, backward):
         o = _ceil(o + nbytes, 256) * 256
 
     nkv, nch = N * Hkv * Dv, nchunks * Hkv * Dv
-    # status, chunk table, order, safe flags, L, Vt, Vm hi, Vm lo, then the
-    # per-(chunk, kv head, channel) tot, rho, hr and log2 max |Vt|
-    for nbytes in (256, nc1 * 16, nc1 * 4, nc1 * Hkv * 4, nkv * 4, nkv * 2, nkv * 2, nkv * 2,
-                   nch * 4, nch * 4, nch * 4, nch * 4):
+    # status, chunk table, order, safe flags, L and its channel-major copy,
+    # Vt, Vm hi, Vm lo, then the per-(chunk, kv head, channel) tot, rho, hr
+    # and log2 max |Vt|
+    for nbytes in (256, nc1 * 16, nc1 * 4, nc1 * Hkv * 4, nkv * 4, nkv * 4, nkv * 2, nkv * 2,
+                   nkv * 2, nch * 4, nch * 4, nch * 4, nch * 4):
         take(nbytes)
     if not backward:
         return o
