@@ -55,7 +55,7 @@ constexpr int kPrefixThreads = 256;
 constexpr int kPrefixGroups = kPrefixThreads / 32;        // row groups of 32 channels
 constexpr int kPrefixRows = FIX_CHUNK / kPrefixGroups;    // rows per thread
 
-__global__ void __launch_bounds__(kPrefixThreads) prefix_kernel(
+__global__ void __launch_bounds__(kPrefixThreads, 4) prefix_kernel(
     Dims d, const Chunk* __restrict__ chunks, const float* __restrict__ g,
     const __nv_bfloat16* __restrict__ v, float* __restrict__ L, float* __restrict__ Lt,
     uint16_t* __restrict__ vt,

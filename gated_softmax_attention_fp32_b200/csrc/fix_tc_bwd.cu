@@ -115,6 +115,13 @@ __device__ __forceinline__ bool f16_factors(const float* f) {
   return ok;
 }
 
+// Rewrites in place this thread's 16-byte column chunk `col` of rows r0,
+// r0 + step, ... (< rows) of a 128-byte-swizzled operand tile, fn(value, row)
+// giving the new value: the loads of a batch of rows come before its stores
+// (the compiler cannot move a load above a store to the same array).
+template <typename Fn>
+__device__ __forceinline__ void rewrite_rows(uint8_t* tile, int rows, int r0, int step, int col, Fn fn);
+
 __device__ __forceinline__ void unpack8(uint4 u, bool f16, float* x) {
   const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
@@ -128,6 +135,35 @@ __device__ __forceinline__ void unpack8(uint4 u, bool f16, float* x) {
       x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
     }
   }
+}
+
+template <typename Fn>
+__device__ __forceinline__ void rewrite_rows(uint8_t* tile, int rows, int r0, int step, int col, Fn fn) {
+  constexpr int kB = 4;   // rows per batch
+#pragma unroll 1
+  for (int s0 = r0; s0 < rows; s0 += kB * step) {
+    uint4 x[kB];
+#pragma unroll
+    for (int i = 0; i < kB; ++i) {
+      const int r = s0 + i * step;
+      if (r < rows) x[i] = *reinterpret_cast<const uint4*>(tile + sw_off(rows, r, col));
+    }
+#pragma unroll
+    for (int i = 0; i < kB; ++i) {
+      const int r = s0 + i * step;
+      if (r < rows) *reinterpret_cast<uint4*>(tile + sw_off(rows, r, col)) = fn(x[i], r);
+    }
+  }
+}
+
+__device__ __forceinline__ uint4 hmul8(uint4 v, const __half2 (&fh)[4]) {
+  uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    __half2 h = __hmul2(*reinterpret_cast<const __half2*>(&w4[u]), fh[u]);
+    w4[u] = *reinterpret_cast<uint32_t*>(&h);
+  }
+  return make_uint4(w4[0], w4[1], w4[2], w4[3]);
 }
 
 // =========================================================================== dq
@@ -413,12 +449,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (phase == 1) {
         const bool stored_f16 = P.dsafe[(size_t)ci * d.Hq + h] != 0;
         if (stored_f16 != (cta_f16 != 0)) {
-          for (int rr = r0; rr < BN; rr += kRowsPerPass) {
-            uint4* p = reinterpret_cast<uint4*>(sO + sw_off(BN, rr, lc * 8));
+          rewrite_rows(sO, BN, r0, kRowsPerPass, lc * 8, [&](uint4 v, int) {
             float x[8];
-            unpack8(*p, stored_f16, x);
-            *p = pack8(x, cta_f16 != 0);
-          }
+            unpack8(v, stored_f16, x);
+            return pack8(x, cta_f16 != 0);
+          });
           fence_proxy_async_smem();
         }
       }
@@ -452,23 +487,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         __half2 fh[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) fh[u] = __floats2half2_rn(f8[2 * u], f8[2 * u + 1]);
-        for (int rr = r0; rr < BN; rr += kRowsPerPass) {
-          uint4* p = reinterpret_cast<uint4*>(vb + sw_off(BN, rr, lc * 8));
-          uint4 xv = *p;
-          __half2* hx = reinterpret_cast<__half2*>(&xv);
-#pragma unroll
-          for (int u = 0; u < 4; ++u) hx[u] = __hmul2(hx[u], fh[u]);
-          *p = xv;
-        }
+        rewrite_rows(vb, BN, r0, kRowsPerPass, lc * 8, [&](uint4 v, int) { return hmul8(v, fh); });
       } else {
-        for (int rr = r0; rr < BN; rr += kRowsPerPass) {
-          uint4* p = reinterpret_cast<uint4*>(vb + sw_off(BN, rr, lc * 8));
+        rewrite_rows(vb, BN, r0, kRowsPerPass, lc * 8, [&](uint4 v, int) {
           float x[8];
-          unpack8(*p, true, x);
+          unpack8(v, true, x);
 #pragma unroll
           for (int e = 0; e < 8; ++e) x[e] *= f8[e];
-          *p = pack8(x, cta_f16);
-        }
+          return pack8(x, cta_f16);
+        });
       }
       fence_proxy_async_smem();
       mbar_arrive(&bar->v_ready[st]);
@@ -876,14 +903,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           unit = unit && ve == 0.f;
         }
         if (!unit || !cta_f16) {
-          for (int rr = r0; rr < BN; rr += kRowsPerPass) {
-            uint4* p = reinterpret_cast<uint4*>(sV + sw_off(BN, rr, lc * 8));
+          rewrite_rows(sV, BN, r0, kRowsPerPass, lc * 8, [&](uint4 v, int) {
             float x[8];
-            unpack8(*p, true, x);
+            unpack8(v, true, x);
 #pragma unroll
             for (int e = 0; e < 8; ++e) x[e] *= sc[e];
-            *p = pack8(x, cta_f16 != 0);
-          }
+            return pack8(x, cta_f16 != 0);
+          });
         }
         fence_proxy_async_smem();
       }
@@ -949,23 +975,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             __half2 fh[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u) fh[u] = __floats2half2_rn(f8[2 * u], f8[2 * u + 1]);
-            for (int rr = r0; rr < BQ; rr += kRowsPerPass) {
-              uint4* p = reinterpret_cast<uint4*>(xb + sw_off(BQ, rr, lc * 8));
-              uint4 xv = *p;
-              __half2* hx = reinterpret_cast<__half2*>(&xv);
-#pragma unroll
-              for (int u = 0; u < 4; ++u) hx[u] = __hmul2(hx[u], fh[u]);
-              *p = rr < qlen ? xv : make_uint4(0u, 0u, 0u, 0u);
-            }
+            rewrite_rows(xb, BQ, r0, kRowsPerPass, lc * 8, [&](uint4 v, int rr) {
+              return rr < qlen ? hmul8(v, fh) : make_uint4(0u, 0u, 0u, 0u);
+            });
           } else {
-            for (int rr = r0; rr < BQ; rr += kRowsPerPass) {
-              uint4* p = reinterpret_cast<uint4*>(xb + sw_off(BQ, rr, lc * 8));
+            rewrite_rows(xb, BQ, r0, kRowsPerPass, lc * 8, [&](uint4 v, int rr) {
               float x[8];
-              unpack8(*p, in_f16, x);
+              unpack8(v, in_f16, x);
 #pragma unroll
               for (int e = 0; e < 8; ++e) x[e] = rr < qlen ? x[e] * f8[e] : 0.f;
-              *p = pack8(x, cta_f16 != 0);
-            }
+              return pack8(x, cta_f16 != 0);
+            });
           }
           fence_proxy_async_smem();
         }

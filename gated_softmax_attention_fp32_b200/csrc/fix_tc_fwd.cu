@@ -74,7 +74,7 @@ constexpr int kThreads = 384;
 constexpr int kVsThreads = 64;   // V-scaling threads (warps 2-3)
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // lazy row-max update, natural-log units
-constexpr int kPolyOf4 = 1;      // of every 4 softmax exponentials, how many (0 or 1) by polynomial
+constexpr int kPolyPairEvery = 4;  // one pair of softmax exponentials in this many by polynomial (0: none)
 __host__ __device__ constexpr uint32_t col_s(int b) { return b ? 128u : 0u; }
 
 struct Bars {
@@ -470,19 +470,34 @@ __global__ void __launch_bounds__(kThreads, 1)
               l_used *= rr;
               m_used = m_new;
             }
+            // packed pairs: the scaling and the running sum as f32x2, one pair
+            // of exponentials in kPolyPairEvery as a polynomial on the FMA pipe,
+            // the rest on the MUFU unit (both well inside fp16's rounding)
             const float moff = m_used * LOG2E;
+            const uint64_t c1x2 = f2_pack(c1, c1), mo2 = f2_pack(-moff, -moff);
+            uint64_t lsa = f2_pack(0.f, 0.f), lsb = lsa;
             uint32_t pk[16];
 #pragma unroll
             for (int e = 0; e < 32; e += 2) {
-              const float a0 = __uint_as_float(xs[e]) * c1 - moff;
-              const float a1 = __uint_as_float(xs[e + 1]) * c1 - moff;
-              // one exponential in four on the FMA pipe (kPolyOf4), the rest
-              // on the MUFU unit; both well inside fp16's rounding
-              const float p0 = ex2(a0);
-              const float p1 = ((e >> 1) & 1) && kPolyOf4 ? exp2_poly3(a1) : ex2(a1);
-              ls += p0 + p1;
+              const uint64_t a2 =
+                  f2_fma(f2_pack(__uint_as_float(xs[e]), __uint_as_float(xs[e + 1])), c1x2, mo2);
+              uint64_t p2;
+              if (kPolyPairEvery > 0 && (e >> 1) % kPolyPairEvery == kPolyPairEvery - 1) {
+                p2 = exp2_poly3_x2(a2);
+              } else {
+                float a0, a1;
+                f2_unpack(a2, a0, a1);
+                p2 = f2_pack(ex2(a0), ex2(a1));
+              }
+              if ((e >> 1) & 1) lsb = f2_add(lsb, p2);
+              else lsa = f2_add(lsa, p2);
+              float p0, p1;
+              f2_unpack(p2, p0, p1);
               pk[e >> 1] = pack_f16(p0, p1);
             }
+            float s0, s1;
+            f2_unpack(f2_add(lsa, lsb), s0, s1);
+            ls += s0 + s1;
             tmem_st16(sbase + c4 * 16, pk);
             return true;
           };
@@ -798,28 +813,37 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!wg_and(2, kVsThreads, mbar_wait(&bar->v_full[sv], (vc >> 1) & 1, ctl))) { ok = false; break; }
         if (!diag && !unit) {
           uint8_t* vb = reinterpret_cast<uint8_t*>(sV + sv * BN * DV) + half * (BN * 128);
-          if (h16) {
-#pragma unroll 4
-            for (int s = r0; s < BN; s += kRowsPerPass) {
-              uint4* p = reinterpret_cast<uint4*>(vb + s * 128 + ((lcc ^ (s & 7)) << 4));
-              uint4 xv = *p;
-              __half2* hx = reinterpret_cast<__half2*>(&xv);
+          // rows in batches of 8: all loads of a batch before its stores (the
+          // compiler cannot move a load above a store to the same array)
+          constexpr int kBatch = 8;
+          static_assert((BN / kRowsPerPass) % kBatch == 0, "row batches");
+#pragma unroll 1
+          for (int s0 = r0; s0 < BN; s0 += kBatch * kRowsPerPass) {
+            uint4 xv[kBatch];
 #pragma unroll
-              for (int u = 0; u < 4; ++u) hx[u] = __hmul2(hx[u], fh[u]);
-              *p = xv;
+            for (int i = 0; i < kBatch; ++i) {
+              const int s = s0 + i * kRowsPerPass;
+              xv[i] = *reinterpret_cast<const uint4*>(vb + s * 128 + ((lcc ^ (s & 7)) << 4));
             }
-          } else {
-#pragma unroll 4
-            for (int s = r0; s < BN; s += kRowsPerPass) {
-              uint4* p = reinterpret_cast<uint4*>(vb + s * 128 + ((lcc ^ (s & 7)) << 4));
-              uint4 xv = *p;
-              uint32_t w4[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+            for (int i = 0; i < kBatch; ++i) {
+              uint32_t w4[4] = {xv[i].x, xv[i].y, xv[i].z, xv[i].w};
 #pragma unroll
               for (int u = 0; u < 4; ++u) {
-                const float2 ab = __half22float2(*reinterpret_cast<const __half2*>(&w4[u]));
-                w4[u] = pack_f16(ab.x * f8[2 * u], ab.y * f8[2 * u + 1]);
+                if (h16) {
+                  __half2 h = __hmul2(*reinterpret_cast<const __half2*>(&w4[u]), fh[u]);
+                  w4[u] = *reinterpret_cast<uint32_t*>(&h);
+                } else {
+                  const float2 ab = __half22float2(*reinterpret_cast<const __half2*>(&w4[u]));
+                  w4[u] = pack_f16(ab.x * f8[2 * u], ab.y * f8[2 * u + 1]);
+                }
               }
-              *p = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+              xv[i] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+            }
+#pragma unroll
+            for (int i = 0; i < kBatch; ++i) {
+              const int s = s0 + i * kRowsPerPass;
+              *reinterpret_cast<uint4*>(vb + s * 128 + ((lcc ^ (s & 7)) << 4)) = xv[i];
             }
           }
           fence_proxy_async_smem();
@@ -892,9 +916,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float* rows = sRows + tb * 4 * BM;
       const float alpha = rows[r], mt = rows[2 * BM + r], lsum = rows[3 * BM + r];
       const uint32_t acol = lane_base + 256u + (uint32_t)(tb * DV);
-      // o for channels [32 u, 32 u + 32): alpha exp(L - rho) A (A holds the
-      // s = t term too; no row factor for out-of-range channels)
-      auto chunk_o = [&](int u, float (&o)[32]) {
+      // pass 1, channels [32 u, 32 u + 32): o = alpha exp(L - rho) A (A holds
+      // the s = t term too; no row factor for out-of-range channels), its
+      // sum of squares, and o written back over A.  The next chunk's L is
+      // pulled into L1 while this one is computed.
+      float ss = 0.f;
+      auto prefetch_l1 = [&](int u) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+          asm volatile("prefetch.global.L1 [%0];" ::"l"(Lr + (size_t)(u * 32 + e) * d.N));
+      };
+      prefetch_l1(0);
+#pragma unroll 1
+      for (int u = 0; u < kU; ++u) {
+        if (u + 1 < kU) prefetch_l1(u + 1);
         uint32_t xa[32];
         tmem_ld32(acol + u * 32, xa);
         float le[32];
@@ -905,41 +940,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int e = 0; e < 32; ++e) {
           const int c = u * 32 + e;
           const float fac = eBad[c] ? 1.f : ex2((le[e] - eRho[c]) * LOG2E);
-          o[e] = alpha * fac * __uint_as_float(xa[e]);
+          const float o = alpha * fac * __uint_as_float(xa[e]);
+          ss += o * o;
+          xa[e] = __float_as_uint(o);
         }
-      };
-      // pass 1: the sum of squares (and the saved o)
-      float ss = 0.f;
-#pragma unroll 1
-      for (int u = 0; u < kU; ++u) {
-        float o[32];
-        chunk_o(u, o);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) ss += o[e] * o[e];
-        if (P.o_s && valid && !d.no_norm) {
-          float4* dst = reinterpret_cast<float4*>(P.o_s + orow + u * 32);
-#pragma unroll
-          for (int q = 0; q < 8; ++q) dst[q] = make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
-        }
+        tmem_st32(acol + u * 32, xa);
       }
+      tmem_wait_st();
       // the RMSNorm, or without it the softmax denominator: y = o / l; the
       // saved tensors are then o / l, the log-sum-exp and ones
       const float rstd = d.no_norm ? 1.0f / lsum : 1.0f / sqrtf(ss / (float)DV + d.eps);
-      // pass 2: y (and without the norm the saved o / l)
-#pragma unroll 1
-      for (int u = 0; u < kU; ++u) {
-        float o[32];
-        chunk_o(u, o);
-        // without the norm the saved o / l
-        if (P.o_s && d.no_norm && valid) {
+      // pass 2: y and the saved o, from o in TMEM (the next chunk's load in
+      // flight)
+      auto pass2 = [&](int u, uint32_t (&xo)[32]) {
+        float* o = reinterpret_cast<float*>(xo);   // in place
+        if (P.o_s && valid) {
+          const float so = d.no_norm ? rstd : 1.f;
           float4* dst = reinterpret_cast<float4*>(P.o_s + orow + u * 32);
 #pragma unroll
           for (int q = 0; q < 8; ++q)
-            dst[q] = make_float4(o[4 * q] * rstd, o[4 * q + 1] * rstd, o[4 * q + 2] * rstd, o[4 * q + 3] * rstd);
+            dst[q] = make_float4(o[4 * q] * so, o[4 * q + 1] * so, o[4 * q + 2] * so, o[4 * q + 3] * so);
         }
-        float* yv = o;   // y = o rstd w (swish(z)), in place
 #pragma unroll
-        for (int e = 0; e < 32; ++e) yv[e] *= rstd * sW[u * 32 + e];
+        for (int e = 0; e < 32; ++e) o[e] *= rstd * sW[u * 32 + e];
         if (P.z) {
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
@@ -947,8 +970,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t w4[4] = {z4.x, z4.y, z4.z, z4.w};
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-              yv[8 * q + 2 * i] *= swish(__uint_as_float(w4[i] << 16));
-              yv[8 * q + 2 * i + 1] *= swish(__uint_as_float(w4[i] & 0xFFFF0000u));
+              o[8 * q + 2 * i] *= swish(__uint_as_float(w4[i] << 16));
+              o[8 * q + 2 * i + 1] *= swish(__uint_as_float(w4[i] & 0xFFFF0000u));
             }
           }
         }
@@ -956,14 +979,35 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (P.y_f32) {
             float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(P.y) + orow + u * 32);
 #pragma unroll
-            for (int q = 0; q < 8; ++q) dst[q] = make_float4(yv[4 * q], yv[4 * q + 1], yv[4 * q + 2], yv[4 * q + 3]);
+            for (int q = 0; q < 8; ++q) dst[q] = make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
           } else {
             uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(P.y) + orow + u * 32);
 #pragma unroll
             for (int q = 0; q < 4; ++q)
-              dst[q] = make_uint4(pack_bf16(yv[8 * q], yv[8 * q + 1]), pack_bf16(yv[8 * q + 2], yv[8 * q + 3]),
-                                  pack_bf16(yv[8 * q + 4], yv[8 * q + 5]), pack_bf16(yv[8 * q + 6], yv[8 * q + 7]));
+              dst[q] = make_uint4(pack_bf16(o[8 * q], o[8 * q + 1]), pack_bf16(o[8 * q + 2], o[8 * q + 3]),
+                                  pack_bf16(o[8 * q + 4], o[8 * q + 5]), pack_bf16(o[8 * q + 6], o[8 * q + 7]));
           }
+        }
+      };
+      {
+        uint32_t xa[32], xb[32];
+        tmem_ld32(acol, xa);
+        tmem_wait_ld(xa);
+        if (kU > 1) tmem_ld32(acol + 32, xb);
+        pass2(0, xa);
+        if (kU > 1) {
+          tmem_wait_ld(xb);
+          if (kU > 2) tmem_ld32(acol + 64, xa);
+          pass2(1, xb);
+        }
+        if (kU > 2) {
+          tmem_wait_ld(xa);
+          if (kU > 3) tmem_ld32(acol + 96, xb);
+          pass2(2, xa);
+        }
+        if (kU > 3) {
+          tmem_wait_ld(xb);
+          pass2(3, xb);
         }
       }
       if (P.o_s && valid) {
