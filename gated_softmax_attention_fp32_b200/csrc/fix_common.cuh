@@ -21,10 +21,17 @@ constexpr int kPreSplit = 4;
 // (31 KB of the 32 KB that kernel parameters may take).
 constexpr int kBlobMaxWords = 7936;
 
-// exp for the 16-bit tensor-core operands (pre-decayed values and gradients,
-// rounded to fp16 / bf16 right after): exp2f of x log2(e), whose error is far
-// below their rounding.  The exact CUDA-core kernels keep expf.
-__device__ __forceinline__ float exp_op(float x) { return exp2f(x * 1.4426950408889634f); }
+// e^x for the 16-bit tensor-core operands (pre-decayed values and gradients)
+// that the prefix pass and the backward preprocess produce: the MUFU 2^x
+// approximation of x log2(e) (relative error about 2^-22, far below their 8-
+// or 11-bit significands and the ~16 bits of a hi/lo pair; results below
+// fp32's normal range become 0, which every 16-bit store does anyway).  The
+// exact CUDA-core kernels keep expf.
+__device__ __forceinline__ float exp_op(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x * 1.4426950408889634f));
+  return y;
+}
 // Largest half-range of a chunk's prefix sums that the in-chunk split
 // exp(L_t - rho) * exp(rho - L_s) keeps inside float range (e^80 ~ 5.5e34),
 // and the largest |rho| for which the forward's column factor exp(rho) stays

@@ -294,37 +294,50 @@ def fix_attn_noalloc_device_status(stream=None) -> int:
     return int(load().fix_attn_noalloc_device_status(_stream(stream)))
 
 
+def _check(ws, where):
+    s = fix_attn_device_status(ws)
+    if s != 0:
+        raise FixStatusError(s, where)
+
+
 class _FixAttn(torch.autograd.Function):
     @staticmethod
-    def forward(ctx, q, k, v, g, w, z, cu_seqlens, cu_host, scale, eps, algo, o_norm):
+    def forward(ctx, q, k, v, g, w, z, cu_seqlens, cu_host, scale, eps, algo, o_norm, check):
         ws = training_workspace(q, k, v, cu_seqlens, cu_host, algo, g, o_norm)
         y, saved = fix_attn_fwd(q, k, v, g, w, cu_seqlens, cu_host, scale, eps, save=True,
                                 algo=algo, workspace=ws, o_gate=z, o_norm=o_norm)
+        if check:
+            _check(ws, "fix_attn forward (device status)")
         ctx.save_for_backward(q, k, v, g, w, z, *saved)
-        ctx.cfg = (cu_seqlens, cu_host, scale, eps, algo, o_norm)
+        ctx.cfg = (cu_seqlens, cu_host, scale, eps, algo, o_norm, check)
         ctx.ws = ws
         return y
 
     @staticmethod
     def backward(ctx, dy):
         q, k, v, g, w, z, o_s, m_s, r_s = ctx.saved_tensors
-        cu, cu_host, scale, eps, algo, o_norm = ctx.cfg
+        cu, cu_host, scale, eps, algo, o_norm, check = ctx.cfg
         dq, dk, dv, dg, dw, dz = fix_attn_bwd(q, k, v, g, w, dy.to(torch.bfloat16).contiguous(),
                                               (o_s, m_s, r_s), cu, cu_host, scale, eps, algo,
                                               workspace=ctx.ws, reuse_forward_workspace=True,
                                               o_gate=z, o_norm=o_norm)
+        if check:
+            _check(ctx.ws, "fix_attn backward (device status)")
         ctx.ws = None
-        return dq, dk, dv, dg, dw, dz, None, None, None, None, None, None
+        return dq, dk, dv, dg, dw, dz, None, None, None, None, None, None, None
 
 
 def fix_attn(q, k, v, g, o_norm_weight=None, cu_seqlens=None, cu_seqlens_host=None, scale=None,
-             eps=1e-6, algo="auto", o_gate=None, o_norm=True):
+             eps=1e-6, algo="auto", o_gate=None, o_norm=True, check_status=True):
     """FiX attention, differentiable, with the FiX README's arguments ("Quick
     Start"): y = RMSNorm(FiX attention(q, k, v, g)) * o_norm_weight
     [* swish(o_gate)]; with ``o_norm=False`` the output is the attention
     average o_t / l_t [* swish(o_gate)].  g [B,T,Hkv,Dv] (element-wise gate)
-    or [B,T,Hkv] (scalar gate)."""
+    or [B,T,Hkv] (scalar gate).  ``check_status`` reads the device status
+    word after the forward and after the backward (each read synchronises
+    the stream) and raises FixStatusError if a bounded device wait expired;
+    pass False to keep the calls asynchronous."""
     if o_norm and o_norm_weight is None:
         raise ValueError("o_norm=True needs o_norm_weight")
     return _FixAttn.apply(q, k, v, g, o_norm_weight, o_gate, cu_seqlens, cu_seqlens_host, scale,
-                          eps, algo, o_norm)
+                          eps, algo, o_norm, check_status)

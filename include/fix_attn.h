@@ -64,10 +64,12 @@ typedef enum {
 
 enum { FIX_DTYPE_BF16 = 0, FIX_DTYPE_F32 = 1 };
 
-/* Kernel family.  FIX_ALGO_AUTO picks the tensor-core (tcgen05) kernels.
- * FIX_ALGO_SIMT runs the exact fp32 CUDA-core kernels (every decay factor
- * exp(G_t - G_s) formed element by element); it is much slower and serves as
- * a second, independent GPU path for cross-checks. */
+/* Kernel family.  FIX_ALGO_AUTO picks the tensor-core (tcgen05) kernels
+ * where they apply: Dk and Dv in {64, 128}, at least 128 tokens in all, and
+ * for the backward at most 16 q heads per kv head; other problems run on the
+ * exact kernels.  FIX_ALGO_SIMT runs the exact fp32 CUDA-core kernels (every
+ * decay factor exp(G_t - G_s) formed element by element); it is much slower
+ * and serves as a second, independent GPU path for cross-checks. */
 enum { FIX_ALGO_AUTO = 0, FIX_ALGO_SIMT = 1, FIX_ALGO_TC = 2 };
 
 /* fix_attn_problem.flags.
@@ -122,10 +124,10 @@ enum {
   FIX_STAGE_BWD_DKV = 5,    /* dk/dv partial sums (tensor-core kernel, else  */
                             /* the exact dk, dv, dG kernel)                  */
   FIX_STAGE_BWD_DG = 6,     /* reverse cumsum dG -> dg                        */
-  FIX_STAGE_BWD_FINISH = 7, /* tensor-core path: combine of the dk/dv        */
-                            /* partials into dk, dv, dG, and the exact       */
-                            /* kernels (they return at once unless a channel */
-                            /* is outside the split's range)                 */
+  FIX_STAGE_BWD_FINISH = 7, /* tensor-core path: the exact diagonal terms of */
+                            /* channels outside the split's range (returns   */
+                            /* at once without them), then the combine of    */
+                            /* the dk/dv partials into dk, dv, dG            */
   FIX_NUM_STAGES = 8
 };
 

@@ -411,3 +411,23 @@ def test_decode_long_context_rows(cuda_lib):
             r = fix_ref.forward_rows(case["q"], case["k"], case["v"], case["g"], case["w"],
                                      (0, 0), L, h, [L - 1], None, case["eps"])
             check_fwd(y[b, h].double().cpu().numpy()[None], r["y"], f"decode L={L} h={h}")
+
+
+# ------------------------------------------------------------------ autograd
+def test_autograd_wrapper_matches_direct_calls(cuda_lib):
+    """fix_attn (the README's call, as a torch.autograd.Function) gives the
+    same y and gradients as the direct forward/backward calls, bit for bit,
+    with the device status checked after each."""
+    from gated_softmax_attention_fp32_b200 import fixattn
+    case = synth.make_case(1, 300, 4, 2, 64, 64, seed=21)
+    t = {k: case[k].cuda() for k in ("q", "k", "v", "g", "w", "dy")}
+    leaves = {k: t[k].clone().requires_grad_(True) for k in ("q", "k", "v", "g", "w")}
+    y = fixattn.fix_attn(leaves["q"], leaves["k"], leaves["v"], leaves["g"], leaves["w"])
+    y.backward(t["dy"])
+    yd, saved = fixattn.fix_attn_fwd(t["q"], t["k"], t["v"], t["g"], t["w"], save=True)
+    dq, dk, dv, dg, dw, _ = fixattn.fix_attn_bwd(t["q"], t["k"], t["v"], t["g"], t["w"], t["dy"],
+                                                 saved)
+    torch.cuda.synchronize()
+    assert torch.equal(y.detach(), yd)
+    for name, ref in (("q", dq), ("k", dk), ("v", dv), ("g", dg), ("w", dw)):
+        assert torch.equal(leaves[name].grad, ref), name
