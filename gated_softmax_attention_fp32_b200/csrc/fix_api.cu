@@ -367,7 +367,9 @@ static fix_status run_prefix(const Dims& d, const fix_attn_problem* p, const Ws&
       return FIX_ERR_CUDA;
     return FIX_OK;
   }
-  prefix_kernel<<<dim3(d.nchunks, d.Hkv, (d.Dv + 31) / 32), 256, 0, st>>>(
+  const size_t psmem = prefix_smem_bytes(d.Dv, want_lt);
+  if (!set_smem_limit(reinterpret_cast<const void*>(prefix_kernel), (int)psmem)) return FIX_ERR_CUDA;
+  prefix_kernel<<<dim3(d.nchunks, d.Hkv), 256, psmem, st>>>(
       d, chunks, g, static_cast<const __nv_bfloat16*>(v), reinterpret_cast<float*>(base + ws.L),
       want_lt ? reinterpret_cast<float*>(base + ws.Lt) : nullptr,
       want_vt ? reinterpret_cast<uint16_t*>(base + ws.vt) : nullptr,
@@ -600,11 +602,10 @@ fix_status fix_attn_bwd(const fix_attn_problem* p, const void* q, const void* k,
   if (tc) FIX_TRY(tc_bwd(p, d, ta, 2, st));
   FIX_TRY(mark(p, FIX_STAGE_BWD_FINISH, 1, st));
   FIX_TRY(mark(p, FIX_STAGE_BWD_DG, 0, st));
-  chunk_total_kernel<<<dim3(d.nchunks, d.Hkv, (d.Dv + 31) / 32), 256, 0, st>>>(d, chunks, dG, dtot);
+  chunk_total_kernel<<<dim3(d.nchunks, d.Hkv), 256, 0, st>>>(d, chunks, dG, dtot);
   FIX_TRY(launched());
   float* dgf = d.scalar_gate ? reinterpret_cast<float*>(base + ws.dgf) : dg;
-  reverse_cumsum_kernel<<<dim3(d.nchunks, d.Hkv, (d.Dv + 31) / 32), 256, 0, st>>>(d, chunks, dG,
-                                                                                 dtot, dgf);
+  reverse_cumsum_kernel<<<dim3(d.nchunks, d.Hkv), 256, 0, st>>>(d, chunks, dG, dtot, dgf);
   FIX_TRY(launched());
   if (d.scalar_gate) {
     // a scalar gate acts on every channel: its gradient is the channel sum

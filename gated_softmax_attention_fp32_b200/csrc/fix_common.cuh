@@ -16,7 +16,7 @@
 
 #define FIX_CHUNK 128
 // CTAs per chunk in the backward preprocess (FIX_CHUNK / kPreSplit rows each).
-constexpr int kPreSplit = 4;
+constexpr int kPreSplit = 2;
 // Largest schedule piece one upload launch carries in its parameter block
 // (31 KB of the 32 KB that kernel parameters may take).
 constexpr int kBlobMaxWords = 7936;
@@ -113,6 +113,37 @@ __device__ __forceinline__ float swish_grad(float z) {
   return sg * (1.0f + z * (1.0f - sg));
 }
 __device__ __forceinline__ __nv_bfloat16 f2bf(float x) { return __float2bfloat16_rn(x); }
+
+// 4 consecutive values from an 8-byte (bf16) or 16-byte (fp32) aligned
+// address into floats; zeros for a null address.
+__device__ __forceinline__ void ld4b(const __nv_bfloat16* p, float* x) {
+  if (!p) {
+    x[0] = x[1] = x[2] = x[3] = 0.f;
+    return;
+  }
+  const uint2 u = *reinterpret_cast<const uint2*>(p);
+  x[0] = __uint_as_float(u.x << 16);
+  x[1] = __uint_as_float(u.x & 0xFFFF0000u);
+  x[2] = __uint_as_float(u.y << 16);
+  x[3] = __uint_as_float(u.y & 0xFFFF0000u);
+}
+__device__ __forceinline__ void ld4f(const float* p, float* x) {
+  if (!p) {
+    x[0] = x[1] = x[2] = x[3] = 0.f;
+    return;
+  }
+  const float4 u = *reinterpret_cast<const float4*>(p);
+  x[0] = u.x;
+  x[1] = u.y;
+  x[2] = u.z;
+  x[3] = u.w;
+}
+// 4 floats to 4 consecutive bf16 (round to nearest) at an 8-byte aligned address.
+__device__ __forceinline__ void st4b(__nv_bfloat16* p, const float* x) {
+  const __nv_bfloat162 a = __floats2bfloat162_rn(x[0], x[1]), b = __floats2bfloat162_rn(x[2], x[3]);
+  *reinterpret_cast<uint2*>(p) =
+      make_uint2(*reinterpret_cast<const uint32_t*>(&a), *reinterpret_cast<const uint32_t*>(&b));
+}
 
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll

@@ -29,21 +29,24 @@ template __global__ void upload_kernel<4096>(const __grid_constant__ Blob<4096>,
 template __global__ void upload_kernel<kBlobMaxWords>(const __grid_constant__ Blob<kBlobMaxWords>,
                                                       uint32_t*, int);
 
-// grid (nchunks, Hkv, ceil(Dv / 32)), block 256: a CTA takes 32 channels of
-// one chunk and kv head, thread = (row group of 16 rows, channel); the eight
-// groups are scanned in parallel and joined through shared memory.  Few
-// registers per thread keep many warps per SM, so that many loads are in
-// flight and one CTA's loads overlap another's scan and stores.
+// grid (nchunks, Hkv), block 256: a CTA takes one chunk of one kv head, all
+// its channels; thread = (row group of 16 rows, 4 consecutive channels), so
+// every global access is a 16-byte (g, L) or 8-byte (v and the 16-bit
+// outputs) vector and a warp covers a row's channels in one coalesced
+// stretch.  The eight row groups are scanned in parallel and joined through
+// shared memory.
 //
 // Besides L and tot, the tensor-core path needs:
+//   Lt = L channel-major [Hkv][Dv][N] (forward only), written through a
+//             shared-memory transpose so that a warp stores 32 consecutive
+//             tokens of one channel;
 //   Vt_s[c] = v_s[c] * exp(tot[c] - L_s[c])     values pre-decayed to the chunk's
 //             last row, for key blocks strictly before a query chunk, stored
 //             as fp16 times 2^-e (e = vt_exponent(lvt), lvt[c] = log2 of the
 //             column's largest |Vt|), so that no stored value exceeds 2^15;
 //   safe[ci * Hkv + kv] = every g of the chunk is <= 0 and every |v| <=
 //             FIX_F16_VMAX (then e = 0 and every later scaling is <= 1); the
-//             schedule upload sets it to 1 and every CTA of the chunk ANDs
-//             its part in;
+//             schedule upload sets it to 1 and the CTA ANDs its result in;
 //   rho[c] = (min_t L_t[c] + max_t L_t[c]) / 2,  hr[c] = (max - min) / 2,
 //   Vm_s[c] = v_s[c] * exp(rho[c] - L_s[c])       (|exponent| <= hr), stored as
 //             a pair of bf16 (hi, lo = bf16(Vm - hi)) for a near-exact
@@ -52,162 +55,240 @@ template __global__ void upload_kernel<kBlobMaxWords>(const __grid_constant__ Bl
 // inside [e^-hr, e^hr].  Channels with hr > FIX_HR_MAX or |rho| > FIX_RHO_MAX
 // are out of range (see fix_common.cuh): Vm = 0, rho = 0, hr = FIX_HR_BAD.
 constexpr int kPrefixThreads = 256;
-constexpr int kPrefixGroups = kPrefixThreads / 32;        // row groups of 32 channels
+constexpr int kPrefixGroups = kPrefixThreads / 32;        // row groups
 constexpr int kPrefixRows = FIX_CHUNK / kPrefixGroups;    // rows per thread
 
-__global__ void __launch_bounds__(kPrefixThreads, 4) prefix_kernel(
+size_t prefix_smem_bytes(int Dv, bool lt) {
+  return (size_t)4 * kPrefixGroups * Dv * sizeof(float) +
+         (lt ? (size_t)Dv * (FIX_CHUNK + 1) * sizeof(float) : 0);
+}
+
+namespace {
+__device__ __forceinline__ float4 f4_add(float4 a, float4 b) {
+  return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
+}
+__device__ __forceinline__ float4 f4_min(float4 a, float4 b) {
+  return make_float4(fminf(a.x, b.x), fminf(a.y, b.y), fminf(a.z, b.z), fminf(a.w, b.w));
+}
+__device__ __forceinline__ float4 f4_max(float4 a, float4 b) {
+  return make_float4(fmaxf(a.x, b.x), fmaxf(a.y, b.y), fmaxf(a.z, b.z), fmaxf(a.w, b.w));
+}
+__device__ __forceinline__ float f4_get(const float4& a, int k) {
+  return k == 0 ? a.x : k == 1 ? a.y : k == 2 ? a.z : a.w;
+}
+__device__ __forceinline__ void bf4_unpack(uint2 u, float* x) {
+  x[0] = __uint_as_float(u.x << 16);
+  x[1] = __uint_as_float(u.x & 0xFFFF0000u);
+  x[2] = __uint_as_float(u.y << 16);
+  x[3] = __uint_as_float(u.y & 0xFFFF0000u);
+}
+}  // namespace
+
+__global__ void __launch_bounds__(kPrefixThreads) prefix_kernel(
     Dims d, const Chunk* __restrict__ chunks, const float* __restrict__ g,
     const __nv_bfloat16* __restrict__ v, float* __restrict__ L, float* __restrict__ Lt,
-    uint16_t* __restrict__ vt,
-    __nv_bfloat16* __restrict__ vm, __nv_bfloat16* __restrict__ vml, float* __restrict__ tot,
-    float* __restrict__ rho, float* __restrict__ hr, float* __restrict__ lvt,
-    int* __restrict__ safe, int* __restrict__ badflag, int* __restrict__ hmax) {
-  __shared__ float part[kPrefixThreads], pmin[kPrefixThreads], pmax[kPrefixThreads];
-  __shared__ float tr[32][FIX_CHUNK + 1];   // the slab of L, channel-major (for Lt)
-  const int Dv = d.Dv;
-  const int cl = threadIdx.x & 31, grp = threadIdx.x >> 5;
-  const int c = blockIdx.z * 32 + cl;
-  const bool act = c < Dv;
+    uint16_t* __restrict__ vt, __nv_bfloat16* __restrict__ vm, __nv_bfloat16* __restrict__ vml,
+    float* __restrict__ tot, float* __restrict__ rho, float* __restrict__ hr,
+    float* __restrict__ lvt, int* __restrict__ safe, int* __restrict__ badflag,
+    int* __restrict__ hmax) {
+  extern __shared__ float psm[];
+  const int Dv = d.Dv, nq = Dv / 4;
+  const int lane = threadIdx.x & 31, grp = threadIdx.x >> 5;
+  const bool act = lane < nq;
+  const int c0 = 4 * (act ? lane : 0);
   const int ci = blockIdx.x, kv = blockIdx.y;
   const Chunk ch = chunks[ci];
+  float* part = psm;                        // [groups][Dv] group totals
+  float* pmin = part + kPrefixGroups * Dv;  // [groups][Dv] group minima of L
+  float* pmax = pmin + kPrefixGroups * Dv;  // [groups][Dv] group maxima
+  float* pxm = pmax + kPrefixGroups * Dv;   // [groups][Dv] group max |Vt|
+  float* tr = pxm + kPrefixGroups * Dv;     // [Dv][FIX_CHUNK + 1] L, channel-major
   // the backward's per-(chunk, q head) max |do|, raised by its preprocess
-  if (hmax && blockIdx.z == 0 && threadIdx.x < d.grp)
-    hmax[(size_t)ci * d.Hq + kv * d.grp + threadIdx.x] = 0;
+  if (hmax && threadIdx.x < d.grp) hmax[(size_t)ci * d.Hq + kv * d.grp + threadIdx.x] = 0;
   const size_t rs = (size_t)d.Hkv * Dv;
-  const size_t base = (size_t)ch.tok0 * rs + (size_t)kv * Dv + (act ? c : 0);
+  const size_t base = (size_t)ch.tok0 * rs + (size_t)kv * Dv + c0;
   const int r0 = grp * kPrefixRows;
   const int nr = act ? max(0, min(kPrefixRows, ch.len - r0)) : 0;
-  float lv[kPrefixRows], vv[kPrefixRows];
-  float acc = 0.f, lmin = INFINITY, lmax = -INFINITY;
-  bool nonpos = true;
+  float4 lv[kPrefixRows];
+  uint2 vv[kPrefixRows];
   // g and v in one round trip (v only on the tensor-core path); a scalar gate
   // ([N, Hkv]) is the same for every channel of the token
-  const size_t gbase = d.scalar_gate ? (size_t)ch.tok0 * d.Hkv + kv : base;
-  const size_t grs = d.scalar_gate ? (size_t)d.Hkv : rs;
-#pragma unroll
-  for (int u = 0; u < kPrefixRows; ++u)
-    if (u < nr) lv[u] = g[gbase + (size_t)(r0 + u) * grs];
-  if (vt) {
-#pragma unroll
-    for (int u = 0; u < kPrefixRows; ++u)
-      if (u < nr) vv[u] = bf2f(v[base + (size_t)(r0 + u) * rs]);
-  }
 #pragma unroll
   for (int u = 0; u < kPrefixRows; ++u) {
     if (u < nr) {
-      nonpos = nonpos && lv[u] <= 0.f;
-      acc += lv[u];
-      lv[u] = acc;
-      lmin = fminf(lmin, acc);
-      lmax = fmaxf(lmax, acc);
+      if (d.scalar_gate) {
+        const float x = g[((size_t)ch.tok0 + r0 + u) * d.Hkv + kv];
+        lv[u] = make_float4(x, x, x, x);
+      } else {
+        lv[u] = *reinterpret_cast<const float4*>(g + base + (size_t)(r0 + u) * rs);
+      }
     }
   }
-  part[threadIdx.x] = acc;
-  pmin[threadIdx.x] = lmin;
-  pmax[threadIdx.x] = lmax;
-  __syncthreads();
-  float off = 0.f, total = 0.f, cmin = INFINITY, cmax = -INFINITY;
+  if (vt) {
 #pragma unroll
-  for (int q = 0; q < kPrefixGroups; ++q) {
-    const float pq = part[q * 32 + cl];
-    if (q < grp) off += pq;
-    cmin = fminf(cmin, total + pmin[q * 32 + cl]);
-    cmax = fmaxf(cmax, total + pmax[q * 32 + cl]);
-    total += pq;
+    for (int u = 0; u < kPrefixRows; ++u)
+      if (u < nr) vv[u] = *reinterpret_cast<const uint2*>(v + base + (size_t)(r0 + u) * rs);
+  }
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float4 lmin = make_float4(INFINITY, INFINITY, INFINITY, INFINITY);
+  float4 lmax = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+  bool nonpos = true;
+#pragma unroll
+  for (int u = 0; u < kPrefixRows; ++u) {
+    if (u < nr) {
+      nonpos = nonpos && lv[u].x <= 0.f && lv[u].y <= 0.f && lv[u].z <= 0.f && lv[u].w <= 0.f;
+      acc = f4_add(acc, lv[u]);
+      lv[u] = acc;
+      lmin = f4_min(lmin, acc);
+      lmax = f4_max(lmax, acc);
+    }
+  }
+  if (act) {
+    *reinterpret_cast<float4*>(part + grp * Dv + c0) = acc;
+    *reinterpret_cast<float4*>(pmin + grp * Dv + c0) = lmin;
+    *reinterpret_cast<float4*>(pmax + grp * Dv + c0) = lmax;
+  }
+  __syncthreads();
+  float4 off = make_float4(0.f, 0.f, 0.f, 0.f), total = off;
+  float4 cmin = make_float4(INFINITY, INFINITY, INFINITY, INFINITY);
+  float4 cmax = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+  if (act) {
+#pragma unroll
+    for (int q = 0; q < kPrefixGroups; ++q) {
+      const float4 pq = *reinterpret_cast<const float4*>(part + q * Dv + c0);
+      if (q < grp) off = f4_add(off, pq);
+      cmin = f4_min(cmin, f4_add(total, *reinterpret_cast<const float4*>(pmin + q * Dv + c0)));
+      cmax = f4_max(cmax, f4_add(total, *reinterpret_cast<const float4*>(pmax + q * Dv + c0)));
+      total = f4_add(total, pq);
+    }
   }
 #pragma unroll
   for (int u = 0; u < kPrefixRows; ++u)
     if (u < nr) {
-      lv[u] += off;
-      L[base + (size_t)(r0 + u) * rs] = lv[u];
-      if (Lt) tr[cl][r0 + u] = lv[u];
+      lv[u] = f4_add(lv[u], off);
+      *reinterpret_cast<float4*>(L + base + (size_t)(r0 + u) * rs) = lv[u];
+      if (Lt) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) tr[(c0 + k) * (FIX_CHUNK + 1) + r0 + u] = f4_get(lv[u], k);
+      }
     }
-  const size_t ti = ((size_t)ci * d.Hkv + kv) * Dv + c;
-  if (grp == 0 && act) tot[ti] = total;
+  const size_t ti = ((size_t)ci * d.Hkv + kv) * Dv + c0;
+  if (grp == 0 && act) *reinterpret_cast<float4*>(tot + ti) = total;
   if (Lt) {
-    // L channel-major: a warp writes 32 consecutive tokens of one channel
+    // L channel-major: a warp stores 32 consecutive tokens of one channel
     __syncthreads();
-    const int lane = threadIdx.x & 31;
-    for (int j = grp; j < 32; j += kPrefixGroups) {
-      const int cj = blockIdx.z * 32 + j;
-      if (cj >= Dv) break;
-      float* dst = Lt + ((size_t)kv * Dv + cj) * d.N + ch.tok0;
-      for (int r = lane; r < ch.len; r += 32) dst[r] = tr[j][r];
+    for (int c = grp; c < Dv; c += kPrefixGroups) {
+      float* dst = Lt + ((size_t)kv * Dv + c) * d.N + ch.tok0;
+      for (int r = lane; r < ch.len; r += 32) dst[r] = tr[c * (FIX_CHUNK + 1) + r];
     }
   }
   if (!vt) return;  // uniform: the exact kernels need only L and tot
-  float vmax = 0.f, xmax = 0.f;
+  float vmax = 0.f;
+  float4 xmax = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
   for (int u = 0; u < kPrefixRows; ++u)
     if (u < nr) {
-      vmax = fmaxf(vmax, fabsf(vv[u]));
-      xmax = fmaxf(xmax, fabsf(vv[u] * exp_op(total - lv[u])));
-    }
-  const int f16 = __syncthreads_and(nonpos && vmax <= FIX_F16_VMAX);   // part[] free after this
-  if (threadIdx.x == 0 && !f16) atomicAnd(safe + (size_t)ci * d.Hkv + kv, 0);
-  part[threadIdx.x] = xmax;
-  const float half = 0.5f * (cmax - cmin);
-  const float mid = 0.5f * (cmax + cmin);
-  const bool good = !act || (half <= FIX_HR_MAX && fabsf(mid) <= FIX_RHO_MAX);
-  const float ref = good ? mid : 0.f;
-  if (__syncthreads_or(!good) && threadIdx.x == 0) atomicOr(badflag, 1);
-  float cx = 0.f;
+      float x[4];
+      bf4_unpack(vv[u], x);
 #pragma unroll
-  for (int q = 0; q < kPrefixGroups; ++q) cx = fmaxf(cx, part[q * 32 + cl]);
-  const float lg = cx > 0.f ? log2f(cx) : -1e30f;
-  const float sc = exp2f(-vt_exponent(lg));
+      for (int k = 0; k < 4; ++k) vmax = fmaxf(vmax, fabsf(x[k]));
+      xmax.x = fmaxf(xmax.x, fabsf(x[0] * exp_op(total.x - lv[u].x)));
+      xmax.y = fmaxf(xmax.y, fabsf(x[1] * exp_op(total.y - lv[u].y)));
+      xmax.z = fmaxf(xmax.z, fabsf(x[2] * exp_op(total.z - lv[u].z)));
+      xmax.w = fmaxf(xmax.w, fabsf(x[3] * exp_op(total.w - lv[u].w)));
+    }
+  if (act) *reinterpret_cast<float4*>(pxm + grp * Dv + c0) = xmax;
+  const int f16 = __syncthreads_and(nonpos && vmax <= FIX_F16_VMAX);
+  if (threadIdx.x == 0 && !f16) atomicAnd(safe + (size_t)ci * d.Hkv + kv, 0);
+  float ref[4], hrng[4], lg[4], sc[4];
+  bool good[4];
+  bool any_bad = false;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    hrng[k] = 0.5f * (f4_get(cmax, k) - f4_get(cmin, k));
+    const float mid = 0.5f * (f4_get(cmax, k) + f4_get(cmin, k));
+    good[k] = !act || ch.len <= 0 || (hrng[k] <= FIX_HR_MAX && fabsf(mid) <= FIX_RHO_MAX);
+    ref[k] = good[k] ? mid : 0.f;
+    any_bad = any_bad || !good[k];
+    float cx = 0.f;
+    if (act) {
+#pragma unroll
+      for (int q = 0; q < kPrefixGroups; ++q) cx = fmaxf(cx, pxm[q * Dv + c0 + k]);
+    }
+    lg[k] = cx > 0.f ? log2f(cx) : -1e30f;
+    sc[k] = exp2f(-vt_exponent(lg[k]));
+  }
+  if (__syncthreads_or(any_bad) && threadIdx.x == 0) atomicOr(badflag, 1);
   if (grp == 0 && act) {
-    rho[ti] = ref;
-    hr[ti] = ch.len > 0 ? (good ? half : FIX_HR_BAD) : 0.f;
-    lvt[ti] = lg;
+    *reinterpret_cast<float4*>(rho + ti) = make_float4(ref[0], ref[1], ref[2], ref[3]);
+    float h4[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) h4[k] = ch.len > 0 ? (good[k] ? hrng[k] : FIX_HR_BAD) : 0.f;
+    *reinterpret_cast<float4*>(hr + ti) = make_float4(h4[0], h4[1], h4[2], h4[3]);
+    *reinterpret_cast<float4*>(lvt + ti) = make_float4(lg[0], lg[1], lg[2], lg[3]);
   }
 #pragma unroll
   for (int u = 0; u < kPrefixRows; ++u)
     if (u < nr) {
+      float x[4], xt[4], xm[4], hi[4], lo[4];
+      bf4_unpack(vv[u], x);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float lk = f4_get(lv[u], k);
+        xt[k] = x[k] * exp_op(f4_get(total, k) - lk) * sc[k];
+        xm[k] = good[k] ? x[k] * exp_op(ref[k] - lk) : 0.f;
+        hi[k] = __bfloat162float(__float2bfloat16_rn(xm[k]));
+        lo[k] = xm[k] - hi[k];   // Vm = hi + lo to ~16 bits
+      }
       const size_t a = base + (size_t)(r0 + u) * rs;
-      const float xt = vv[u] * exp_op(total - lv[u]);
-      vt[a] = __half_as_ushort(__float2half_rn(xt * sc));
-      const float xm = good ? vv[u] * exp_op(ref - lv[u]) : 0.f;
-      const __nv_bfloat16 xm_hi = f2bf(xm);
-      vm[a] = xm_hi;
-      vml[a] = f2bf(xm - bf2f(xm_hi));   // Vm = hi + lo to ~16 bits
+      const __half2 t01 = __floats2half2_rn(xt[0], xt[1]), t23 = __floats2half2_rn(xt[2], xt[3]);
+      const __nv_bfloat162 h01 = __floats2bfloat162_rn(hi[0], hi[1]), h23 = __floats2bfloat162_rn(hi[2], hi[3]);
+      const __nv_bfloat162 l01 = __floats2bfloat162_rn(lo[0], lo[1]), l23 = __floats2bfloat162_rn(lo[2], lo[3]);
+      *reinterpret_cast<uint2*>(vt + a) =
+          make_uint2(*reinterpret_cast<const uint32_t*>(&t01), *reinterpret_cast<const uint32_t*>(&t23));
+      *reinterpret_cast<uint2*>(vm + a) =
+          make_uint2(*reinterpret_cast<const uint32_t*>(&h01), *reinterpret_cast<const uint32_t*>(&h23));
+      *reinterpret_cast<uint2*>(vml + a) =
+          make_uint2(*reinterpret_cast<const uint32_t*>(&l01), *reinterpret_cast<const uint32_t*>(&l23));
     }
 }
 
 // Reverse cumsum of dG within each sequence (dg_r = sum_{t >= r} dG_t), in two
 // launches over the same chunk table: chunk totals, then local reverse scans
 // plus the totals of the later chunks of the same sequence.  Both use the
-// prefix pass's block shape: grid (nchunks, Hkv, ceil(Dv / 32)), 256 threads =
-// (row group, channel), every row of a group loaded up front, groups joined
-// through shared memory.
+// prefix pass's block shape: grid (nchunks, Hkv), 256 threads = (row group,
+// 4 channels), every row of a group loaded up front as 16-byte vectors,
+// groups joined through shared memory.
 __global__ void __launch_bounds__(kPrefixThreads) chunk_total_kernel(Dims d,
                                                                      const Chunk* __restrict__ chunks,
                                                                      const float* __restrict__ x,
                                                                      float* __restrict__ tot) {
-  __shared__ float part[kPrefixThreads];
-  const int Dv = d.Dv;
-  const int cl = threadIdx.x & 31, grp = threadIdx.x >> 5;
-  const int c = blockIdx.z * 32 + cl;
-  const bool act = c < Dv;
+  __shared__ float4 part[kPrefixGroups][32];
+  const int Dv = d.Dv, nq = Dv / 4;
+  const int lane = threadIdx.x & 31, grp = threadIdx.x >> 5;
+  const bool act = lane < nq;
+  const int c0 = 4 * (act ? lane : 0);
   const int ci = blockIdx.x, kv = blockIdx.y;
   const Chunk ch = chunks[ci];
   const size_t rs = (size_t)d.Hkv * Dv;
-  const size_t base = (size_t)ch.tok0 * rs + (size_t)kv * Dv + (act ? c : 0);
+  const size_t base = (size_t)ch.tok0 * rs + (size_t)kv * Dv + c0;
   const int r0 = grp * kPrefixRows;
   const int nr = act ? max(0, min(kPrefixRows, ch.len - r0)) : 0;
-  float xv[kPrefixRows];
+  float4 xv[kPrefixRows];
 #pragma unroll
-  for (int u = 0; u < kPrefixRows; ++u) xv[u] = u < nr ? x[base + (size_t)(r0 + u) * rs] : 0.f;
-  float acc = 0.f;
+  for (int u = 0; u < kPrefixRows; ++u)
+    if (u < nr) xv[u] = *reinterpret_cast<const float4*>(x + base + (size_t)(r0 + u) * rs);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-  for (int u = 0; u < kPrefixRows; ++u) acc += xv[u];
-  part[threadIdx.x] = acc;
+  for (int u = 0; u < kPrefixRows; ++u)
+    if (u < nr) acc = f4_add(acc, xv[u]);
+  part[grp][lane] = acc;
   __syncthreads();
   if (grp == 0 && act) {
-    float t = 0.f;
+    float4 t = part[0][lane];
 #pragma unroll
-    for (int q = 0; q < kPrefixGroups; ++q) t += part[q * 32 + cl];
-    tot[((size_t)ci * d.Hkv + kv) * Dv + c] = t;
+    for (int q = 1; q < kPrefixGroups; ++q) t = f4_add(t, part[q][lane]);
+    *reinterpret_cast<float4*>(tot + ((size_t)ci * d.Hkv + kv) * Dv + c0) = t;
   }
 }
 
@@ -227,37 +308,53 @@ __global__ void __launch_bounds__(256) channel_sum_kernel(const float* __restric
 __global__ void __launch_bounds__(kPrefixThreads) reverse_cumsum_kernel(
     Dims d, const Chunk* __restrict__ chunks, const float* __restrict__ x,
     const float* __restrict__ tot, float* __restrict__ out) {
-  __shared__ float part[kPrefixThreads];
-  const int Dv = d.Dv;
-  const int cl = threadIdx.x & 31, grp = threadIdx.x >> 5;
-  const int c = blockIdx.z * 32 + cl;
-  const bool act = c < Dv;
+  __shared__ float4 part[kPrefixGroups][32], later[kPrefixGroups][32];
+  const int Dv = d.Dv, nq = Dv / 4;
+  const int lane = threadIdx.x & 31, grp = threadIdx.x >> 5;
+  const bool act = lane < nq;
+  const int c0 = 4 * (act ? lane : 0);
   const int ci = blockIdx.x, kv = blockIdx.y;
   const Chunk ch = chunks[ci];
   const size_t rs = (size_t)d.Hkv * Dv;
-  const size_t base = (size_t)ch.tok0 * rs + (size_t)kv * Dv + (act ? c : 0);
+  const size_t base = (size_t)ch.tok0 * rs + (size_t)kv * Dv + c0;
   const int r0 = grp * kPrefixRows;
   const int nr = act ? max(0, min(kPrefixRows, ch.len - r0)) : 0;
-  float xv[kPrefixRows];
+  float4 xv[kPrefixRows];
 #pragma unroll
-  for (int u = 0; u < kPrefixRows; ++u) xv[u] = u < nr ? x[base + (size_t)(r0 + u) * rs] : 0.f;
-  // the later chunks of the sequence, in order
-  float acc = 0.f;
+  for (int u = 0; u < kPrefixRows; ++u)
+    if (u < nr) xv[u] = *reinterpret_cast<const float4*>(x + base + (size_t)(r0 + u) * rs);
+  // the totals of the sequence's later chunks: row group q takes chunks
+  // j + 1 + q, j + 1 + q + 8, ... (two accumulators, so that the loads
+  // overlap); the groups' sums are then added in group order
   const int first = ci - ch.j;
-  if (act)
-    for (int jj = ch.nch - 1; jj > ch.j; --jj) acc += tot[((size_t)(first + jj) * d.Hkv + kv) * Dv + c];
-  float own = 0.f;
+  float4 la = make_float4(0.f, 0.f, 0.f, 0.f), lb = la;
+  if (act) {
+    int jj = ch.j + 1 + grp;
+    for (; jj + kPrefixGroups < ch.nch; jj += 2 * kPrefixGroups) {
+      la = f4_add(la, *reinterpret_cast<const float4*>(tot + ((size_t)(first + jj) * d.Hkv + kv) * Dv + c0));
+      lb = f4_add(lb, *reinterpret_cast<const float4*>(
+                          tot + ((size_t)(first + jj + kPrefixGroups) * d.Hkv + kv) * Dv + c0));
+    }
+    if (jj < ch.nch)
+      la = f4_add(la, *reinterpret_cast<const float4*>(tot + ((size_t)(first + jj) * d.Hkv + kv) * Dv + c0));
+  }
+  float4 own = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-  for (int u = 0; u < kPrefixRows; ++u) own += xv[u];
-  part[threadIdx.x] = own;
+  for (int u = 0; u < kPrefixRows; ++u)
+    if (u < nr) own = f4_add(own, xv[u]);
+  part[grp][lane] = own;
+  later[grp][lane] = f4_add(la, lb);
   __syncthreads();
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+  for (int q = 0; q < kPrefixGroups; ++q) acc = f4_add(acc, later[q][lane]);
   // then the later row groups of this chunk, from the last one down
-  for (int q = kPrefixGroups - 1; q > grp; --q) acc += part[q * 32 + cl];
+  for (int q = kPrefixGroups - 1; q > grp; --q) acc = f4_add(acc, part[q][lane]);
 #pragma unroll
   for (int u = kPrefixRows - 1; u >= 0; --u)
     if (u < nr) {
-      acc += xv[u];
-      out[base + (size_t)(r0 + u) * rs] = acc;
+      acc = f4_add(acc, xv[u]);
+      *reinterpret_cast<float4*>(out + base + (size_t)(r0 + u) * rs) = acc;
     }
 }
 

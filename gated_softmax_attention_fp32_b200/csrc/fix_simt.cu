@@ -159,7 +159,7 @@ __global__ void __launch_bounds__(256) fwd_simt_kernel(
 
 // ---------------------------------------------------------------------------
 // Backward preprocess (shared by all kernel families).  Pass 1, grid
-// (nchunks * kPreSplit, Hkv), 8 warps: a CTA takes a quarter of a chunk's rows
+// (nchunks * kPreSplit, Hkv), 8 warps: a CTA takes half of a chunk's rows
 // for one kv head, a warp a row at a time over the kv group's q heads:
 //   RMSNorm backward   n = o rstd,  dn = dy w,  do = rstd (dn - n mean(dn n))
 //   A_t[c]  = sum_{h in group} do_t[c] (o_t[c] - P_tt v_t[c])
@@ -175,7 +175,7 @@ __global__ void __launch_bounds__(256) fwd_simt_kernel(
 // ---------------------------------------------------------------------------
 constexpr int kPreWarps = 8;
 
-__global__ void __launch_bounds__(kPreWarps * 32, 3) bwd_pre_kernel(
+__global__ void __launch_bounds__(kPreWarps * 32, 2) bwd_pre_kernel(
     Dims d, const Chunk* __restrict__ chunks, const __nv_bfloat16* __restrict__ q,
     const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
     const float* __restrict__ o_s, const float* __restrict__ m_s,
@@ -192,96 +192,116 @@ __global__ void __launch_bounds__(kPreWarps * 32, 3) bwd_pre_kernel(
   const Chunk ch = chunks[ci];
   for (int i = threadIdx.x; i < d.grp; i += blockDim.x) hmax[i] = 0.f;
   __syncthreads();
+  // lane = 4 consecutive channels (16-byte fp32 / 8-byte bf16 accesses)
+  const int c0 = 4 * lane;
+  const bool cv = c0 < Dv, ck = c0 < Dk;
   float wv[4], dwl[4];
+  ld4b(w && cv ? w + c0 : nullptr, wv);
 #pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const int c = lane + 32 * u;
-    wv[u] = (c < Dv && w) ? bf2f(w[c]) : 0.f;
-    dwl[u] = 0.f;
-  }
+  for (int u = 0; u < 4; ++u) dwl[u] = 0.f;
   const size_t ors = (size_t)d.Hq * Dv, vrs = (size_t)d.Hkv * Dv;
   const size_t qrs = (size_t)d.Hq * Dk, krs = (size_t)d.Hkv * Dk;
   constexpr int kRows = FIX_CHUNK / kPreSplit;
   const int rend = min(ch.len, (sub + 1) * kRows);
-  for (int r = sub * kRows + warp; r < rend; r += kPreWarps) {
-    const size_t t = (size_t)ch.tok0 + r;
-    float acc[4] = {0.f, 0.f, 0.f, 0.f}, vr[4], kr[4];
+  const int r0 = sub * kRows + warp;
+  const int nrows = rend > r0 ? (rend - r0 + kPreWarps - 1) / kPreWarps : 0;
+  const int grp = d.grp, nitems = nrows * grp;
+  // The warp's (row, q head) items in order, each item's loads issued two
+  // items ahead of its computation.
+  struct In {
+    float rs, mt, q[4], o[4], dy[4], z[4], vr[4], kr[4];
+  };
+  auto load = [&](int it, In& in) {
+    const int i = it / grp, hh = it % grp;
+    const size_t t = (size_t)ch.tok0 + r0 + i * kPreWarps;
+    const int h = kv * grp + hh;
+    const size_t a = t * ors + (size_t)h * Dv + c0;
+    in.rs = rstd_s[t * d.Hq + h];
+    in.mt = m_s[t * d.Hq + h];
+    ld4b(ck ? q + t * qrs + (size_t)h * Dk + c0 : nullptr, in.q);
+    ld4f(cv ? o_s + a : nullptr, in.o);
+    ld4b(cv ? dy + a : nullptr, in.dy);
+    ld4b(z && cv ? z + a : nullptr, in.z);
+    if (hh == 0) {
+      ld4b(cv ? v + t * vrs + (size_t)kv * Dv + c0 : nullptr, in.vr);
+      ld4b(ck ? k + t * krs + (size_t)kv * Dk + c0 : nullptr, in.kr);
+    }
+  };
+  In cur, nx1, nx2;   // items it, it + 1, it + 2
+  if (nitems > 0) load(0, cur);
+  if (nitems > 1) load(1, nx1);
+  float acc[4] = {0.f, 0.f, 0.f, 0.f}, vr[4] = {0.f, 0.f, 0.f, 0.f}, kr[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int it = 0; it < nitems; ++it) {
+    if (it + 2 < nitems) load(it + 2, nx2);
+    const int i = it / grp, hh = it % grp;
+    const size_t t = (size_t)ch.tok0 + r0 + i * kPreWarps;
+    const int h = kv * grp + hh;
+    if (hh == 0) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        vr[u] = cur.vr[u];
+        kr[u] = cur.kr[u];
+        acc[u] = 0.f;
+      }
+    }
+    float sdot = 0.f;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) sdot += cur.q[u] * kr[u];
+    const float ptt = expf(warp_sum(sdot) * d.scale - cur.mt);
+    if (ptt_out && lane == 0) ptt_out[t * d.Hq + h] = ptt;
+    // output gate: y = u swish(z) with u the normed (or, without the norm,
+    // the averaged) output; du = dy swish(z), dz = dy u swish'(z)
+    float du[4], dn[4], n[4], dot_ = 0.f;
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const int c = lane + 32 * u;
-      vr[u] = c < Dv ? bf2f(v[t * vrs + (size_t)kv * Dv + c]) : 0.f;
-      kr[u] = c < Dk ? bf2f(k[t * krs + (size_t)kv * Dk + c]) : 0.f;
+      du[u] = z ? cur.dy[u] * swish(cur.z[u]) : cur.dy[u];
+      n[u] = d.no_norm ? cur.o[u] : cur.o[u] * cur.rs;
+      dn[u] = d.no_norm ? du[u] : du[u] * wv[u];
+      dot_ += dn[u] * n[u];
+      if (!d.no_norm) dwl[u] += du[u] * n[u];
     }
-    for (int hh = 0; hh < d.grp; ++hh) {
-      const int h = kv * d.grp + hh;
-      const float rs_ = rstd_s[t * d.Hq + h];
-      const float mt = m_s[t * d.Hq + h];
-      float sdot = 0.f, ov[4], dyv[4];
+    dot_ = warp_sum(dot_) / (float)Dv;
+    // without the norm: do = du, and sum_c do o (the softmax-denominator
+    // term of dS) goes to the dq and dk/dv kernels
+    if (d.no_norm && lane == 0) delta_out[t * d.Hq + h] = dot_ * (float)Dv;
+    float dov[4], mx = 0.f;
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int c = lane + 32 * u;
-        const size_t a = t * ors + (size_t)h * Dv + c;
-        if (c < Dk) sdot += bf2f(q[t * qrs + (size_t)h * Dk + c]) * kr[u];
-        ov[u] = c < Dv ? o_s[a] : 0.f;
-        dyv[u] = c < Dv ? bf2f(dy[a]) : 0.f;
-      }
-      const float ptt = expf(warp_sum(sdot) * d.scale - mt);
-      if (ptt_out && lane == 0) ptt_out[t * d.Hq + h] = ptt;
-      // output gate: y = u swish(z) with u the normed (or, without the norm,
-      // the averaged) output; du = dy swish(z), dz = dy u swish'(z)
-      float du[4], zv[4];
+    for (int u = 0; u < 4; ++u) {
+      dov[u] = d.no_norm ? du[u] : cur.rs * (dn[u] - n[u] * dot_);
+      acc[u] += dov[u] * (cur.o[u] - ptt * vr[u]);
+      mx = fmaxf(mx, fabsf(dov[u]));
+    }
+    if (cv) {
+      const size_t a = t * ors + (size_t)h * Dv + c0;
+      *reinterpret_cast<float4*>(do_ws + a) = make_float4(dov[0], dov[1], dov[2], dov[3]);
+      if (z) {
+        float g4[4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int c = lane + 32 * u;
-        zv[u] = (z && c < Dv) ? bf2f(z[t * ors + (size_t)h * Dv + c]) : 0.f;
-        du[u] = z ? dyv[u] * swish(zv[u]) : dyv[u];
-      }
-      float dn[4], n[4], dot_ = 0.f;
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        n[u] = d.no_norm ? ov[u] : ov[u] * rs_;
-        dn[u] = d.no_norm ? du[u] : du[u] * wv[u];
-        dot_ += dn[u] * n[u];
-        if (!d.no_norm) dwl[u] += du[u] * n[u];
-      }
-      dot_ = warp_sum(dot_) / (float)Dv;
-      // without the norm: do = du, and sum_c do o (the softmax-denominator
-      // term of dS) goes to the dq and dk/dv kernels
-      if (d.no_norm && lane == 0) delta_out[t * d.Hq + h] = dot_ * (float)Dv;
-      float mx = 0.f;
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int c = lane + 32 * u;
-        if (c >= Dv) continue;
-        const float dov = d.no_norm ? du[u] : rs_ * (dn[u] - n[u] * dot_);
-        do_ws[t * ors + (size_t)h * Dv + c] = dov;
-        acc[u] += dov * (ov[u] - ptt * vr[u]);
-        mx = fmaxf(mx, fabsf(dov));
-        if (z) {
-          const float uo = d.no_norm ? ov[u] : n[u] * wv[u];
-          dz[t * ors + (size_t)h * Dv + c] = f2bf(dyv[u] * uo * swish_grad(zv[u]));
+        for (int u = 0; u < 4; ++u) {
+          const float uo = d.no_norm ? cur.o[u] : n[u] * wv[u];
+          g4[u] = cur.dy[u] * uo * swish_grad(cur.z[u]);
         }
-      }
-      if (hmax_g) {
-        mx = warp_max(mx);
-        if (lane == 0) atomicMax(reinterpret_cast<int*>(&hmax[hh]), __float_as_int(mx));
+        st4b(dz + a, g4);
       }
     }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int c = lane + 32 * u;
-      if (c < Dv) A[t * vrs + (size_t)kv * Dv + c] = acc[u];
+    if (hmax_g) {
+      mx = warp_max(mx);
+      if (lane == 0) atomicMax(reinterpret_cast<int*>(&hmax[hh]), __float_as_int(mx));
     }
+    if (hh == grp - 1 && cv)
+      *reinterpret_cast<float4*>(A + t * vrs + (size_t)kv * Dv + c0) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    cur = nx1;
+    nx1 = nx2;
   }
 #pragma unroll
-  for (int u = 0; u < 4; ++u) red[warp][lane + 32 * u] = dwl[u];
+  for (int u = 0; u < 4; ++u) red[warp][c0 + u] = cv ? dwl[u] : 0.f;
   __syncthreads();
-  const int c0 = threadIdx.x;
-  if (c0 < Dv) {
+  const int cw = threadIdx.x;
+  if (cw < Dv) {
     float sm = 0.f;
 #pragma unroll
-    for (int i = 0; i < kPreWarps; ++i) sm += red[i][c0];
-    dwpart[((size_t)blockIdx.x * d.Hkv + kv) * Dv + c0] = sm;
+    for (int i = 0; i < kPreWarps; ++i) sm += red[i][cw];
+    dwpart[((size_t)blockIdx.x * d.Hkv + kv) * Dv + cw] = sm;
   }
   if (hmax_g)
     for (int i = threadIdx.x; i < d.grp; i += blockDim.x)
@@ -313,47 +333,66 @@ __global__ void __launch_bounds__(kPreWarps * 32) bwd_pre_ops_kernel(
       dsafe[(size_t)ci * d.Hq + kv * d.grp + i] =
           (chunk_safe && __int_as_float(hmax_g[(size_t)ci * d.Hq + kv * d.grp + i]) <= FIX_F16_VMAX) ? 1 : 0;
   const size_t ors = (size_t)d.Hq * Dv, vrs = (size_t)d.Hkv * Dv;
-  float rh[4], good[4];
+  // lane = 4 consecutive channels
+  const int c0 = 4 * lane;
+  const bool cv = c0 < Dv;
+  const size_t tb = ((size_t)ci * d.Hkv + kv) * Dv + c0;
+  float rh[4], hq[4], good[4];
+  ld4f(cv ? rho + tb : nullptr, rh);
+  ld4f(cv ? hr + tb : nullptr, hq);
 #pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const int c = lane + 32 * u;
-    const size_t ti = ((size_t)ci * d.Hkv + kv) * Dv + c;
-    rh[u] = c < Dv ? rho[ti] : 0.f;
-    good[u] = (c < Dv && hr[ti] <= FIX_HR_MAX) ? 1.f : 0.f;
-  }
+  for (int u = 0; u < 4; ++u) good[u] = (cv && hq[u] <= FIX_HR_MAX) ? 1.f : 0.f;
   constexpr int kRows = FIX_CHUNK / kPreSplit;
   const int rend = min(ch.len, (sub + 1) * kRows);
-  for (int r = sub * kRows + warp; r < rend; r += kPreWarps) {
-    const size_t t = (size_t)ch.tok0 + r;
-    float lr[4];
+  const int r0 = sub * kRows + warp;
+  const int nrows = rend > r0 ? (rend - r0 + kPreWarps - 1) / kPreWarps : 0;
+  const int grp = d.grp, nitems = nrows * grp;
+  // the warp's (row, q head) items, loads issued two items ahead
+  struct In {
+    float d[4], l[4];
+  };
+  auto load = [&](int it, In& in) {
+    const int i = it / grp, hh = it % grp;
+    const size_t t = (size_t)ch.tok0 + r0 + i * kPreWarps;
+    ld4f(cv ? do_ws + t * ors + (size_t)(kv * grp + hh) * Dv + c0 : nullptr, in.d);
+    if (hh == 0) ld4f(cv ? L + t * vrs + (size_t)kv * Dv + c0 : nullptr, in.l);
+  };
+  In cur, nx1, nx2;
+  if (nitems > 0) load(0, cur);
+  if (nitems > 1) load(1, nx1);
+  float lr[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int it = 0; it < nitems; ++it) {
+    if (it + 2 < nitems) load(it + 2, nx2);
+    const int i = it / grp, hh = it % grp;
+    const size_t t = (size_t)ch.tok0 + r0 + i * kPreWarps;
+    const int h = kv * grp + hh;
+    if (hh == 0) {
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int c = lane + 32 * u;
-      lr[u] = c < Dv ? L[t * vrs + (size_t)kv * Dv + c] : 0.f;
+      for (int u = 0; u < 4; ++u) lr[u] = cur.l[u];
     }
-    for (int hh = 0; hh < d.grp; ++hh) {
-      const int h = kv * d.grp + hh;
-      const bool f16 =
-          chunk_safe && __int_as_float(hmax_g[(size_t)ci * d.Hq + h]) <= FIX_F16_VMAX;
-      float dov[4];
+    const bool f16 = chunk_safe && __int_as_float(hmax_g[(size_t)ci * d.Hq + h]) <= FIX_F16_VMAX;
+    if (cv) {
+      float xt[4], hi[4], lo[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        const int c = lane + 32 * u;
-        dov[u] = c < Dv ? do_ws[t * ors + (size_t)h * Dv + c] : 0.f;
+        xt[u] = cur.d[u] * exp_op(lr[u]);
+        const float xm = good[u] != 0.f ? cur.d[u] * exp_op(lr[u] - rh[u]) : 0.f;
+        hi[u] = bf2f(f2bf(xm));
+        lo[u] = xm - hi[u];
       }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int c = lane + 32 * u;
-        if (c >= Dv) continue;
-        const size_t a = t * ors + (size_t)h * Dv + c;
-        const float xt = dov[u] * exp_op(lr[u]);
-        dot[a] = f16 ? __half_as_ushort(__float2half_rn(xt)) : __bfloat16_as_ushort(f2bf(xt));
-        const float xm = good[u] != 0.f ? dov[u] * exp_op(lr[u] - rh[u]) : 0.f;
-        const __nv_bfloat16 hi = f2bf(xm);
-        domh[a] = hi;
-        doml[a] = f2bf(xm - bf2f(hi));
+      const size_t a = t * ors + (size_t)h * Dv + c0;
+      if (f16) {
+        const __half2 x01 = __floats2half2_rn(xt[0], xt[1]), x23 = __floats2half2_rn(xt[2], xt[3]);
+        *reinterpret_cast<uint2*>(dot + a) =
+            make_uint2(*reinterpret_cast<const uint32_t*>(&x01), *reinterpret_cast<const uint32_t*>(&x23));
+      } else {
+        st4b(reinterpret_cast<__nv_bfloat16*>(dot + a), xt);
       }
+      st4b(domh + a, hi);   // hi is already bf16-exact
+      st4b(doml + a, lo);
     }
+    cur = nx1;
+    nx1 = nx2;
   }
 }
 

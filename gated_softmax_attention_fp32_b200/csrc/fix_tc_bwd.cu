@@ -1070,19 +1070,32 @@ __global__ void __launch_bounds__(256) dkv_combine_kernel(const Params P) {
   const int halves = (ch.len + BQ - 1) / BQ;
   const int nd = (d.grp * halves + P.tiles_per_part - 1) / P.tiles_per_part;
   float fk[VK] = {}, fd[VV] = {}, fo[VV] = {};
-  for (int q = 0; q < cp.x; ++q) {
-    const float* prow = P.partial + (((size_t)(cp.y + q) * d.Hkv + kv) * BN + s) * kCols;
-    float a[VK], b[VV];
-    ldf<VK>(prow + ck, a);
-    ldf<VV>(prow + DK + cv, b);
+  // slots four at a time: a batch's loads in flight together, the sums in
+  // slot order
+  constexpr int kSB = 4;
+  for (int q0 = 0; q0 < cp.x; q0 += kSB) {
+    float a[kSB][VK], b[kSB][VV];
 #pragma unroll
-    for (int e = 0; e < VK; ++e) fk[e] += a[e];
-    if (q < nd) {
+    for (int i = 0; i < kSB; ++i) {
+      if (q0 + i < cp.x) {
+        const float* prow = P.partial + (((size_t)(cp.y + q0 + i) * d.Hkv + kv) * BN + s) * kCols;
+        ldf<VK>(prow + ck, a[i]);
+        ldf<VV>(prow + DK + cv, b[i]);
+      }
+    }
 #pragma unroll
-      for (int e = 0; e < VV; ++e) fd[e] += b[e];
-    } else {
+    for (int i = 0; i < kSB; ++i) {
+      const int q = q0 + i;
+      if (q >= cp.x) break;
 #pragma unroll
-      for (int e = 0; e < VV; ++e) fo[e] += b[e];
+      for (int e = 0; e < VK; ++e) fk[e] += a[i][e];
+      if (q < nd) {
+#pragma unroll
+        for (int e = 0; e < VV; ++e) fd[e] += b[i][e];
+      } else {
+#pragma unroll
+        for (int e = 0; e < VV; ++e) fo[e] += b[i][e];
+      }
     }
   }
   // dk = scale * sum dS^T Q

@@ -107,7 +107,7 @@ def _expected_workspace(seqlens, Hq, Hkv, Dk, Dv, backward):
                  for L in seqlens for j in range(_ceil(L, 128)))
     for nbytes in (N * Hq * Dv * 4, N * Hq * Dv * 2, N * Hq * Dv * 2, N * Hq * Dv * 2,
                    nc1 * Hq * 4, nc1 * Hq * 4, N * Hq * 4, N * Hq * 4, nkv * 4, nkv * 4, nch * 4,
-                   nc1 * 4 * Hkv * Dv * 4, max(nparts, 1) * 16, nc1 * 8,
+                   nc1 * 2 * Hkv * Dv * 4, max(nparts, 1) * 16, nc1 * 8,
                    nparts * Hkv * 128 * (Dk + Dv) * 4):
         take(nbytes)
     return o
