@@ -26,7 +26,7 @@ __global__ void prefix_kernel(Dims d, const Chunk* chunks, const float* g, const
                               float* L, float* Lt, uint16_t* vt, __nv_bfloat16* vm, __nv_bfloat16* vml,
                               float* tot, float* rho, float* hr, float* lvt, int* safe,
                               int* badflag, int* hmax);
-// Dynamic shared memory of prefix_kernel (grid (nchunks, Hkv), 256 threads);
+// Dynamic shared memory of prefix_kernel (grid (nchunks, Hkv), 512 threads);
 // lt: the channel-major copy of L is written.
 size_t prefix_smem_bytes(int Dv, bool lt);
 __global__ void chunk_total_kernel(Dims d, const Chunk* chunks, const float* x, float* tot);

@@ -29,11 +29,11 @@ template __global__ void upload_kernel<4096>(const __grid_constant__ Blob<4096>,
 template __global__ void upload_kernel<kBlobMaxWords>(const __grid_constant__ Blob<kBlobMaxWords>,
                                                       uint32_t*, int);
 
-// grid (nchunks, Hkv), block 256: a CTA takes one chunk of one kv head, all
-// its channels; thread = (row group of 16 rows, 4 consecutive channels), so
+// grid (nchunks, Hkv), block 512: a CTA takes one chunk of one kv head, all
+// its channels; thread = (row group of 8 rows, 4 consecutive channels), so
 // every global access is a 16-byte (g, L) or 8-byte (v and the 16-bit
 // outputs) vector and a warp covers a row's channels in one coalesced
-// stretch.  The eight row groups are scanned in parallel and joined through
+// stretch.  The sixteen row groups are scanned in parallel and joined through
 // shared memory.
 //
 // Besides L and tot, the tensor-core path needs:
@@ -54,12 +54,17 @@ template __global__ void upload_kernel<kBlobMaxWords>(const __grid_constant__ Bl
 // so that exp(G_t - G_s) = exp(L_t - rho) * exp(rho - L_s) with both factors
 // inside [e^-hr, e^hr].  Channels with hr > FIX_HR_MAX or |rho| > FIX_RHO_MAX
 // are out of range (see fix_common.cuh): Vm = 0, rho = 0, hr = FIX_HR_BAD.
-constexpr int kPrefixThreads = 256;
+constexpr int kPrefixThreads = 256;                       // dG scans
 constexpr int kPrefixGroups = kPrefixThreads / 32;        // row groups
 constexpr int kPrefixRows = FIX_CHUNK / kPrefixGroups;    // rows per thread
+// the prefix pass itself: twice the warps, half the rows each, so that two
+// of its dependent per-thread chains run on every scheduler
+constexpr int kPfxThreads = 512;
+constexpr int kPfxGroups = kPfxThreads / 32;
+constexpr int kPfxRows = FIX_CHUNK / kPfxGroups;
 
 size_t prefix_smem_bytes(int Dv, bool lt) {
-  return (size_t)4 * kPrefixGroups * Dv * sizeof(float) +
+  return (size_t)4 * kPfxGroups * Dv * sizeof(float) +
          (lt ? (size_t)Dv * (FIX_CHUNK + 1) * sizeof(float) : 0);
 }
 
@@ -84,7 +89,7 @@ __device__ __forceinline__ void bf4_unpack(uint2 u, float* x) {
 }
 }  // namespace
 
-__global__ void __launch_bounds__(kPrefixThreads) prefix_kernel(
+__global__ void __launch_bounds__(kPfxThreads) prefix_kernel(
     Dims d, const Chunk* __restrict__ chunks, const float* __restrict__ g,
     const __nv_bfloat16* __restrict__ v, float* __restrict__ L, float* __restrict__ Lt,
     uint16_t* __restrict__ vt, __nv_bfloat16* __restrict__ vm, __nv_bfloat16* __restrict__ vml,
@@ -99,22 +104,22 @@ __global__ void __launch_bounds__(kPrefixThreads) prefix_kernel(
   const int ci = blockIdx.x, kv = blockIdx.y;
   const Chunk ch = chunks[ci];
   float* part = psm;                        // [groups][Dv] group totals
-  float* pmin = part + kPrefixGroups * Dv;  // [groups][Dv] group minima of L
-  float* pmax = pmin + kPrefixGroups * Dv;  // [groups][Dv] group maxima
-  float* pxm = pmax + kPrefixGroups * Dv;   // [groups][Dv] group max |Vt|
-  float* tr = pxm + kPrefixGroups * Dv;     // [Dv][FIX_CHUNK + 1] L, channel-major
+  float* pmin = part + kPfxGroups * Dv;  // [groups][Dv] group minima of L
+  float* pmax = pmin + kPfxGroups * Dv;  // [groups][Dv] group maxima
+  float* pxm = pmax + kPfxGroups * Dv;   // [groups][Dv] group max |Vt|
+  float* tr = pxm + kPfxGroups * Dv;     // [Dv][FIX_CHUNK + 1] L, channel-major
   // the backward's per-(chunk, q head) max |do|, raised by its preprocess
   if (hmax && threadIdx.x < d.grp) hmax[(size_t)ci * d.Hq + kv * d.grp + threadIdx.x] = 0;
   const size_t rs = (size_t)d.Hkv * Dv;
   const size_t base = (size_t)ch.tok0 * rs + (size_t)kv * Dv + c0;
-  const int r0 = grp * kPrefixRows;
-  const int nr = act ? max(0, min(kPrefixRows, ch.len - r0)) : 0;
-  float4 lv[kPrefixRows];
-  uint2 vv[kPrefixRows];
+  const int r0 = grp * kPfxRows;
+  const int nr = act ? max(0, min(kPfxRows, ch.len - r0)) : 0;
+  float4 lv[kPfxRows];
+  uint2 vv[kPfxRows];
   // g and v in one round trip (v only on the tensor-core path); a scalar gate
   // ([N, Hkv]) is the same for every channel of the token
 #pragma unroll
-  for (int u = 0; u < kPrefixRows; ++u) {
+  for (int u = 0; u < kPfxRows; ++u) {
     if (u < nr) {
       if (d.scalar_gate) {
         const float x = g[((size_t)ch.tok0 + r0 + u) * d.Hkv + kv];
@@ -126,7 +131,7 @@ __global__ void __launch_bounds__(kPrefixThreads) prefix_kernel(
   }
   if (vt) {
 #pragma unroll
-    for (int u = 0; u < kPrefixRows; ++u)
+    for (int u = 0; u < kPfxRows; ++u)
       if (u < nr) vv[u] = *reinterpret_cast<const uint2*>(v + base + (size_t)(r0 + u) * rs);
   }
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -134,7 +139,7 @@ __global__ void __launch_bounds__(kPrefixThreads) prefix_kernel(
   float4 lmax = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
   bool nonpos = true;
 #pragma unroll
-  for (int u = 0; u < kPrefixRows; ++u) {
+  for (int u = 0; u < kPfxRows; ++u) {
     if (u < nr) {
       nonpos = nonpos && lv[u].x <= 0.f && lv[u].y <= 0.f && lv[u].z <= 0.f && lv[u].w <= 0.f;
       acc = f4_add(acc, lv[u]);
@@ -154,7 +159,7 @@ __global__ void __launch_bounds__(kPrefixThreads) prefix_kernel(
   float4 cmax = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
   if (act) {
 #pragma unroll
-    for (int q = 0; q < kPrefixGroups; ++q) {
+    for (int q = 0; q < kPfxGroups; ++q) {
       const float4 pq = *reinterpret_cast<const float4*>(part + q * Dv + c0);
       if (q < grp) off = f4_add(off, pq);
       cmin = f4_min(cmin, f4_add(total, *reinterpret_cast<const float4*>(pmin + q * Dv + c0)));
@@ -163,7 +168,7 @@ __global__ void __launch_bounds__(kPrefixThreads) prefix_kernel(
     }
   }
 #pragma unroll
-  for (int u = 0; u < kPrefixRows; ++u)
+  for (int u = 0; u < kPfxRows; ++u)
     if (u < nr) {
       lv[u] = f4_add(lv[u], off);
       *reinterpret_cast<float4*>(L + base + (size_t)(r0 + u) * rs) = lv[u];
@@ -177,7 +182,7 @@ __global__ void __launch_bounds__(kPrefixThreads) prefix_kernel(
   if (Lt) {
     // L channel-major: a warp stores 32 consecutive tokens of one channel
     __syncthreads();
-    for (int c = grp; c < Dv; c += kPrefixGroups) {
+    for (int c = grp; c < Dv; c += kPfxGroups) {
       float* dst = Lt + ((size_t)kv * Dv + c) * d.N + ch.tok0;
       for (int r = lane; r < ch.len; r += 32) dst[r] = tr[c * (FIX_CHUNK + 1) + r];
     }
@@ -186,7 +191,7 @@ __global__ void __launch_bounds__(kPrefixThreads) prefix_kernel(
   float vmax = 0.f;
   float4 xmax = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-  for (int u = 0; u < kPrefixRows; ++u)
+  for (int u = 0; u < kPfxRows; ++u)
     if (u < nr) {
       float x[4];
       bf4_unpack(vv[u], x);
@@ -213,7 +218,7 @@ __global__ void __launch_bounds__(kPrefixThreads) prefix_kernel(
     float cx = 0.f;
     if (act) {
 #pragma unroll
-      for (int q = 0; q < kPrefixGroups; ++q) cx = fmaxf(cx, pxm[q * Dv + c0 + k]);
+      for (int q = 0; q < kPfxGroups; ++q) cx = fmaxf(cx, pxm[q * Dv + c0 + k]);
     }
     lg[k] = cx > 0.f ? log2f(cx) : -1e30f;
     sc[k] = exp2f(-vt_exponent(lg[k]));
@@ -228,7 +233,7 @@ __global__ void __launch_bounds__(kPrefixThreads) prefix_kernel(
     *reinterpret_cast<float4*>(lvt + ti) = make_float4(lg[0], lg[1], lg[2], lg[3]);
   }
 #pragma unroll
-  for (int u = 0; u < kPrefixRows; ++u)
+  for (int u = 0; u < kPfxRows; ++u)
     if (u < nr) {
       float x[4], xt[4], xm[4], hi[4], lo[4];
       bf4_unpack(vv[u], x);

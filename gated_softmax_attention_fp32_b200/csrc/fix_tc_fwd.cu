@@ -38,18 +38,22 @@
 // exp(L_t) A_t + sum_{s<=t} P_ts exp(L_t - L_s) v_s (fp32) in place; the
 // epilogue then applies no row factor to them.
 //
-// Warp roles (384 threads):
+// Warp roles (320 threads):
 //   warp 0       TMA producer: Q per tile, K and V (Vt / Vm hi) through
 //                2-stage rings, Vm lo of the diagonal block
 //   warp 1       MMA issuer (one thread) and TMEM owner
-//   warps 2-3    V scaling: V'' in shared memory, the tile's fold factors
-//   warps 4-7    softmax, a thread per query row: S -> P in TMEM.  Earlier
+//   warps 2-5    softmax, a thread per query row: S -> P in TMEM.  Earlier
 //                blocks in one pass (lazy row-max reference, moved in place
 //                when a 32-key chunk exceeds it), the diagonal in two (row
-//                max first); the fold; the exact sums of out-of-range channels
-//   warps 8-11   epilogue of the previous tile, overlapping this one's MMAs:
-//                a thread per row, its L, v and output rows loaded and
-//                stored with 16-byte accesses
+//                max first); the fold; the exact sums of out-of-range
+//                channels; then half of the tile's epilogue (channels
+//                [0, DV/2)) before the next tile
+//   warps 6-9    V scaling: V'' in shared memory, the tile's fold factors;
+//                then the other half of the tile's epilogue.  One warp of
+//                each group per SM sub-partition.
+// The epilogue (a thread per row: o = alpha exp(L - rho) A written back over
+// A, the RMSNorm's sum of squares joined across the two halves, then y and
+// the saved o) runs while the next tile's first QK^T MMAs and V loads do.
 // TMEM (512 columns): S/P double buffer at 0 and 128 (P written over S as
 // 16-bit pairs; the diagonal's P_lo in the buffer's upper half), and the
 // accumulator A double-buffered by tile parity at 256 and 256 + DV.
@@ -70,8 +74,8 @@ using namespace sm100;
 
 constexpr int BM = 128;          // query rows per tile
 constexpr int BN = FIX_CHUNK;    // keys per block
-constexpr int kThreads = 384;
-constexpr int kVsThreads = 64;   // V-scaling threads (warps 2-3)
+constexpr int kThreads = 320;
+constexpr int kVsThreads = 128;  // V-scaling threads (warps 6-9)
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // lazy row-max update, natural-log units
 constexpr int kPolyPairEvery = 4;  // one pair of softmax exponentials in this many by polynomial (0: none)
@@ -86,7 +90,7 @@ struct Bars {
   uint64_t pv_done;
   uint64_t acc_full[2], acc_empty[2];
   uint64_t fold_ready[2];
-  uint64_t rows_ready[2], rows_free[2];
+  uint64_t rows_ready[2];
   uint64_t drain;
 };
 
@@ -102,9 +106,8 @@ struct Layout {
   static constexpr int kRows = kAnyBad + 16;             // [2][4][BM] f32: alpha, (unused), m, l
   static constexpr int kPlo = kRows + 2 * 4 * BM * 4;    // [BM][33] u32: diagonal P_lo, key chunks 0-1
   static constexpr int kEpiW = kPlo + BM * 33 * 4;       // [DV] f32 w
-  static constexpr int kEpiRho = kEpiW + DV * 4;         // [DV] f32 rho of the epilogue's tile
-  static constexpr int kEpiBad = kEpiRho + DV * 4;       // [DV] int
-  static constexpr int kBars = (kEpiBad + DV * 4 + 7) / 8 * 8;
+  static constexpr int kSS = kEpiW + DV * 4;             // [2][BM] f32: the epilogue halves' sums of squares
+  static constexpr int kBars = (kSS + 2 * BM * 4 + 7) / 8 * 8;
   static constexpr int kTmem = kBars + (int)sizeof(Bars);
   static constexpr int kAbort = kTmem + 4;
   static constexpr int kBytes = kAbort + 4;
@@ -166,9 +169,9 @@ __device__ __forceinline__ Tile tile_info(const Params& P, int t) {
   return x;
 }
 
-// Named barriers for the threads of one role (ids 1..3; 0 is __syncthreads):
-// id 2 the V-scaling warps, id 3 the epilogue warps.
-__device__ __forceinline__ void wg_sync(int id, int n) {
+// Named barriers (ids 1..2; 0 is __syncthreads): id 1 the epilogue's two
+// groups (softmax and V-scaling warps, 256 threads), id 2 the V-scaling warps.
+__device__ __forceinline__ void named_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 __device__ __forceinline__ int wg_and(int id, int n, int pred) {
@@ -197,7 +200,8 @@ __device__ __forceinline__ int wg_or(int id, int n, int pred) {
 }
 
 template <int DK, int DV>
-__global__ void __launch_bounds__(kThreads, 1)
+// 10 warps of at most 200 registers (64,000 of the SM's 65,536): one CTA per SM
+__global__ void __maxnreg__(200)
     fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_vt, const __grid_constant__ CUtensorMap tm_vm,
                   const __grid_constant__ CUtensorMap tm_vml, const Params P) {
@@ -238,10 +242,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bar->s_full[s], 1);
       mbar_init(&bar->p_full[s], 128);
       mbar_init(&bar->acc_full[s], 1);
-      mbar_init(&bar->acc_empty[s], 128);
+      mbar_init(&bar->acc_empty[s], 256);
       mbar_init(&bar->fold_ready[s], kVsThreads);
       mbar_init(&bar->rows_ready[s], 128);
-      mbar_init(&bar->rows_free[s], 128);
     }
     mbar_init(&bar->vlo_empty, 1);
     mbar_init(&bar->pv_done, 1);
@@ -249,13 +252,135 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_fence_init();
   }
   if (warp == 1) tmem_alloc(sTmem, kTmemCols);
-  if (tid >= 256 && tid - 256 < DV)
-    reinterpret_cast<float*>(smem + Lay::kEpiW)[tid - 256] =
-        (P.w && !d.no_norm) ? bf2f(P.w[tid - 256]) : 1.f;
+  if (tid >= 192 && tid - 192 < DV)
+    reinterpret_cast<float*>(smem + Lay::kEpiW)[tid - 192] =
+        (P.w && !d.no_norm) ? bf2f(P.w[tid - 192]) : 1.f;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *sTmem;
+
+  // ---------------------------------------------------------------- epilogue
+  // The epilogue of a tile is shared by the softmax warps (group 0, channels
+  // [0, DV/2)) and the V-scaling warps (group 1, [DV/2, DV)): a thread per
+  // tile row (its TMEM lane), row r = 32 (warp % 4) + lane in both groups.
+  // Pass 1 forms o = alpha exp(L - rho) A (A holds the s = t term too; no row
+  // factor for out-of-range channels), writes it back over A and sums its
+  // squares; the two halves' sums meet in shared memory; pass 2 writes y and
+  // the saved o.  Both groups call it for every tile they take, also after a
+  // failed wait (ok_in false): its first named barrier (id 1, both groups)
+  // votes, so that both groups leave together.
+  float* sSS = reinterpret_cast<float*>(smem + Lay::kSS);
+  const float* sW = reinterpret_cast<const float*>(smem + Lay::kEpiW);
+  const size_t ors = (size_t)d.Hq * DV;
+  constexpr int kU = DV / 32;          // 32-channel chunks
+  constexpr int kUH = kU / 2;          // chunks per group
+  auto epilogue = [&](const Tile& x, int tb, int grpid, bool ok_in, float alpha, float mt,
+                      float lsum) -> bool {
+    if (!wg_and(1, 256, ok_in)) return false;
+    tc_fence_after();
+    const int r = (warp & 3) * 32 + lane;
+    const uint32_t acol = tmem + ((uint32_t)((warp & 3) * 32) << 16) + 256u + (uint32_t)(tb * DV);
+    const bool valid = r < x.len;
+    const size_t tk = (size_t)x.tok0 + (valid ? r : 0);
+    // L of this row, channel-major: for a channel, the warp's 32 rows are 32
+    // consecutive floats
+    const float* Lr = P.Lt + (size_t)x.kv * DV * d.N + tk;
+    const size_t orow = tk * ors + (size_t)x.h * DV;
+    const size_t cb = ((size_t)x.ci * d.Hkv + x.kv) * DV;
+    const int u0 = grpid * kUH;
+    float ss = 0.f;
+    auto prefetch_l1 = [&](int u) {
+#pragma unroll
+      for (int e = 0; e < 32; ++e)
+        asm volatile("prefetch.global.L1 [%0];" ::"l"(Lr + (size_t)(u * 32 + e) * d.N));
+    };
+    prefetch_l1(u0);
+#pragma unroll 1
+    for (int u = u0; u < u0 + kUH; ++u) {
+      if (u + 1 < u0 + kUH) prefetch_l1(u + 1);
+      uint32_t xa[32];
+      tmem_ld32(acol + u * 32, xa);
+      float le[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) le[e] = Lr[(size_t)(u * 32 + e) * d.N];
+      tmem_wait_ld(xa);
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const int c = u * 32 + e;
+        // rho and hr of channel c: the same address across the warp
+        const bool bad = P.hr[cb + c] > FIX_HR_MAX;
+        const float fac = bad ? 1.f : ex2((le[e] - P.rho[cb + c]) * LOG2E);
+        const float o = alpha * fac * __uint_as_float(xa[e]);
+        ss += o * o;
+        xa[e] = __float_as_uint(o);
+      }
+      tmem_st32(acol + u * 32, xa);
+    }
+    tmem_wait_st();
+    sSS[grpid * BM + r] = ss;
+    named_sync(1, 256);
+    ss = sSS[r] + sSS[BM + r];
+    // the RMSNorm, or without it the softmax denominator: y = o / l; the
+    // saved tensors are then o / l, the log-sum-exp and ones
+    const float rstd = d.no_norm ? 1.0f / lsum : 1.0f / sqrtf(ss / (float)DV + d.eps);
+    auto pass2 = [&](int u, uint32_t (&xo)[32]) {
+      float* o = reinterpret_cast<float*>(xo);   // in place
+      if (P.o_s && valid) {
+        const float so = d.no_norm ? rstd : 1.f;
+        float4* dst = reinterpret_cast<float4*>(P.o_s + orow + u * 32);
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          dst[q] = make_float4(o[4 * q] * so, o[4 * q + 1] * so, o[4 * q + 2] * so, o[4 * q + 3] * so);
+      }
+#pragma unroll
+      for (int e = 0; e < 32; ++e) o[e] *= rstd * sW[u * 32 + e];
+      if (P.z) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint4 z4 = reinterpret_cast<const uint4*>(P.z + orow + u * 32)[q];
+          const uint32_t w4[4] = {z4.x, z4.y, z4.z, z4.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            o[8 * q + 2 * i] *= swish(__uint_as_float(w4[i] << 16));
+            o[8 * q + 2 * i + 1] *= swish(__uint_as_float(w4[i] & 0xFFFF0000u));
+          }
+        }
+      }
+      if (valid) {
+        if (P.y_f32) {
+          float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(P.y) + orow + u * 32);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) dst[q] = make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+        } else {
+          uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(P.y) + orow + u * 32);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            dst[q] = make_uint4(pack_bf16(o[8 * q], o[8 * q + 1]), pack_bf16(o[8 * q + 2], o[8 * q + 3]),
+                                pack_bf16(o[8 * q + 4], o[8 * q + 5]), pack_bf16(o[8 * q + 6], o[8 * q + 7]));
+        }
+      }
+    };
+    {
+      // pass 2 from o in TMEM, the next chunk's load in flight
+      uint32_t xa[32], xb[32];
+      tmem_ld32(acol + u0 * 32, xa);
+      tmem_wait_ld(xa);
+      if (kUH > 1) tmem_ld32(acol + (u0 + 1) * 32, xb);
+      pass2(u0, xa);
+      if (kUH > 1) {
+        tmem_wait_ld(xb);
+        pass2(u0 + 1, xb);
+      }
+    }
+    if (grpid == 0 && P.o_s && valid) {
+      P.m_s[tk * d.Hq + x.h] = d.no_norm ? mt + logf(lsum) : mt;
+      P.rstd_s[tk * d.Hq + x.h] = d.no_norm ? 1.f : rstd;
+    }
+    tc_fence_before();
+    mbar_arrive(&bar->acc_empty[tb]);
+    return true;
+  };
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -393,10 +518,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_commit(&bar->drain);
       mbar_wait(&bar->drain, 0, Ctl{P.status, nullptr, ctl.limit_ns});
     }
-  } else if (warp >= 4 && warp < 8) {
+  } else if (warp >= 2 && warp < 6) {
     // ------------------------------------------------------------ softmax
-    const int r = (warp - 4) * 32 + lane;              // query row in the tile
-    const uint32_t lane_base = tmem + ((uint32_t)((warp - 4) * 32) << 16);
+    const int r = (warp & 3) * 32 + lane;              // query row in the tile
+    const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const float c1 = d.scale * LOG2E;
     int g = 0, nt = 0;
     bool ok = true;
@@ -670,20 +795,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(&bar->p_full[b]);
         ++g;
       }
-      if (!ok) break;
-      // per-row results of the tile for its epilogue
-      if (use >= 1 && !__all_sync(0xffffffffu, mbar_wait(&bar->rows_free[tb], (use - 1) & 1, ctl))) { ok = false; break; }
+      // per-row results of the tile, for the V-scaling warps' half of its
+      // epilogue, then this group's half once the diagonal PV has completed
       float* rows = sRows + tb * 4 * BM;
       const float alpha = ex2((m_used - m_true) * LOG2E);
-      rows[r] = alpha;
-      rows[2 * BM + r] = m_true;
-      rows[3 * BM + r] = alpha * l_used;                           // l (no norm)
-      mbar_arrive(&bar->rows_ready[tb]);
+      if (ok) {
+        rows[r] = alpha;
+        rows[2 * BM + r] = m_true;
+        rows[3 * BM + r] = alpha * l_used;                         // l (no norm)
+        mbar_arrive(&bar->rows_ready[tb]);
+        ok = __all_sync(0xffffffffu, mbar_wait(&bar->acc_full[tb], use & 1, ctl));
+      }
+      ok = epilogue(x, tb, 0, ok, alpha, m_true, alpha * l_used);
       ++nt;
     }
-  } else if (warp == 2 || warp == 3) {
+  } else if (warp >= 6) {
     // ------------------------------------------------------------ V scaling
-    const int dt = tid - 64;                         // 0..63
+    const int dt = tid - 192;                        // 0..127
     constexpr int kChunks = DV / 8;                  // 16-byte chunks per row
     constexpr int kRowsPerPass = kVsThreads / kChunks;
     const int lc = dt % kChunks;                     // logical chunk: channels lc*8 .. +7
@@ -697,10 +825,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Tile x = tile_info(P, t);
       if (x.len <= 0) continue;
       const int tb = nt & 1, use = nt >> 1;
+      // (a failed wait ends the tile's work: break leaves this block, and
+      // the epilogue below is still entered, to vote)
+      do {
+      // pull the tile's L (channel-major) into L2 for its epilogue
+      if (dt < DV) {
+        const char* lp = reinterpret_cast<const char*>(P.Lt + ((size_t)x.kv * DV + dt) * d.N + x.tok0);
+        for (int b = 0; b < x.len * 4; b += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(lp + b));
+      }
       // the fold factors of two tiles ago are consumed once its diagonal PV
       // has completed (it follows the fold)
       // (every wait of this warpgroup ends in a vote on a named barrier, so
-      // that all 128 threads leave together after an abort)
+      // that all its threads leave together after an abort)
       if (!wg_and(2, kVsThreads, use < 1 || mbar_wait(&bar->acc_full[tb], (use - 1) & 1, ctl))) { ok = false; break; }
       // tile-wide power-of-two scale k_c of the earlier blocks' operands:
       // not needed (0) when every earlier chunk is fp16-safe (g <= 0)
@@ -855,169 +991,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           lcur[0] = lnxt[0]; lcur[1] = lnxt[1];
         }
       }
-      ++nt;
-    }
-  } else if (warp >= 8) {
-    // ------------------------------------------------------------ epilogue
-    // A thread per tile row (its TMEM lane): two passes over the row's
-    // channels in chunks of 32, the first for the RMSNorm's sum of squares
-    // (and the saved o), the second for y.  The row's L, v (and output gate)
-    // are contiguous: each thread loads them with 16-byte accesses.
-    const int ew = warp - 8;                         // TMEM lanes [32 ew, 32 ew + 32)
-    const uint32_t lane_base = tmem + ((uint32_t)(ew * 32) << 16);
-    const int r = ew * 32 + lane;                    // tile row
-    const float* sW = reinterpret_cast<const float*>(smem + Lay::kEpiW);
-    float* eRho = reinterpret_cast<float*>(smem + Lay::kEpiRho);
-    int* eBad = reinterpret_cast<int*>(smem + Lay::kEpiBad);
-    const int et = tid - 256;                        // 0..127
-    const size_t ors = (size_t)d.Hq * DV;
-    constexpr int kU = DV / 32;                      // 32-channel chunks
-    int nt = 0;
-    bool ok = true;
-    for (int round = 0; ok && round < rounds; ++round) {
-      const int t = tile_of(round, G, cta);
-      if (t >= P.ntiles) continue;
-      const Tile x = tile_info(P, t);
-      if (x.len <= 0) continue;
-      const int tb = nt & 1, use = nt >> 1;
-      const bool valid = r < x.len;
-      const size_t tk = (size_t)x.tok0 + (valid ? r : 0);
-      // L of this row, channel-major: for a channel, the warp's 32 rows are
-      // 32 consecutive floats
-      const float* Lr = P.Lt + (size_t)x.kv * DV * d.N + tk;
-      const size_t orow = tk * ors + (size_t)x.h * DV;
-      // While the tile's MMAs run, pull the tile's L (and this row's output
-      // gate) into L2.
-      if (et < DV && x.len > 0) {
-        const char* lc = reinterpret_cast<const char*>(P.Lt + ((size_t)x.kv * DV + et) * d.N + x.tok0);
-        for (int b = 0; b < x.len * 4; b += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(lc + b));
+      } while (false);
+      // this group's half of the tile's epilogue: the softmax warps' per-row
+      // results and the diagonal PV come first
+      float alpha = 0.f, mt = 0.f, lsum = 1.f;
+      if (ok) {
+        ok = wg_and(2, kVsThreads, mbar_wait(&bar->rows_ready[tb], use & 1, ctl) &&
+                                       mbar_wait(&bar->acc_full[tb], use & 1, ctl));
+        const float* rows = sRows + tb * 4 * BM;
+        const int rr = (warp & 3) * 32 + lane;
+        alpha = rows[rr];
+        mt = rows[2 * BM + rr];
+        lsum = rows[3 * BM + rr];
       }
-      if (valid) {
-        if (P.z) {
-#pragma unroll
-          for (int b = 0; b < DV * 2; b += 128)
-            asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<const char*>(P.z + orow) + b));
-        }
-      }
-      // channel data of this tile (the previous tile's readers are done:
-      // every epilogue thread passed the sync at the end of that tile)
-      if (et < DV) {
-        const size_t ti = ((size_t)x.ci * d.Hkv + x.kv) * DV + et;
-        eRho[et] = P.rho[ti];
-        eBad[et] = P.hr[ti] > FIX_HR_MAX ? 1 : 0;
-      }
-      wg_sync(3, 128);
-      if (!wg_and(3, 128, mbar_wait(&bar->acc_full[tb], use & 1, ctl) &&
-                              mbar_wait(&bar->rows_ready[tb], use & 1, ctl))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const float* rows = sRows + tb * 4 * BM;
-      const float alpha = rows[r], mt = rows[2 * BM + r], lsum = rows[3 * BM + r];
-      const uint32_t acol = lane_base + 256u + (uint32_t)(tb * DV);
-      // pass 1, channels [32 u, 32 u + 32): o = alpha exp(L - rho) A (A holds
-      // the s = t term too; no row factor for out-of-range channels), its
-      // sum of squares, and o written back over A.  The next chunk's L is
-      // pulled into L1 while this one is computed.
-      float ss = 0.f;
-      auto prefetch_l1 = [&](int u) {
-#pragma unroll
-        for (int e = 0; e < 32; ++e)
-          asm volatile("prefetch.global.L1 [%0];" ::"l"(Lr + (size_t)(u * 32 + e) * d.N));
-      };
-      prefetch_l1(0);
-#pragma unroll 1
-      for (int u = 0; u < kU; ++u) {
-        if (u + 1 < kU) prefetch_l1(u + 1);
-        uint32_t xa[32];
-        tmem_ld32(acol + u * 32, xa);
-        float le[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) le[e] = Lr[(size_t)(u * 32 + e) * d.N];
-        tmem_wait_ld(xa);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int c = u * 32 + e;
-          const float fac = eBad[c] ? 1.f : ex2((le[e] - eRho[c]) * LOG2E);
-          const float o = alpha * fac * __uint_as_float(xa[e]);
-          ss += o * o;
-          xa[e] = __float_as_uint(o);
-        }
-        tmem_st32(acol + u * 32, xa);
-      }
-      tmem_wait_st();
-      // the RMSNorm, or without it the softmax denominator: y = o / l; the
-      // saved tensors are then o / l, the log-sum-exp and ones
-      const float rstd = d.no_norm ? 1.0f / lsum : 1.0f / sqrtf(ss / (float)DV + d.eps);
-      // pass 2: y and the saved o, from o in TMEM (the next chunk's load in
-      // flight)
-      auto pass2 = [&](int u, uint32_t (&xo)[32]) {
-        float* o = reinterpret_cast<float*>(xo);   // in place
-        if (P.o_s && valid) {
-          const float so = d.no_norm ? rstd : 1.f;
-          float4* dst = reinterpret_cast<float4*>(P.o_s + orow + u * 32);
-#pragma unroll
-          for (int q = 0; q < 8; ++q)
-            dst[q] = make_float4(o[4 * q] * so, o[4 * q + 1] * so, o[4 * q + 2] * so, o[4 * q + 3] * so);
-        }
-#pragma unroll
-        for (int e = 0; e < 32; ++e) o[e] *= rstd * sW[u * 32 + e];
-        if (P.z) {
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const uint4 z4 = reinterpret_cast<const uint4*>(P.z + orow + u * 32)[q];
-            const uint32_t w4[4] = {z4.x, z4.y, z4.z, z4.w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              o[8 * q + 2 * i] *= swish(__uint_as_float(w4[i] << 16));
-              o[8 * q + 2 * i + 1] *= swish(__uint_as_float(w4[i] & 0xFFFF0000u));
-            }
-          }
-        }
-        if (valid) {
-          if (P.y_f32) {
-            float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(P.y) + orow + u * 32);
-#pragma unroll
-            for (int q = 0; q < 8; ++q) dst[q] = make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
-          } else {
-            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(P.y) + orow + u * 32);
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              dst[q] = make_uint4(pack_bf16(o[8 * q], o[8 * q + 1]), pack_bf16(o[8 * q + 2], o[8 * q + 3]),
-                                  pack_bf16(o[8 * q + 4], o[8 * q + 5]), pack_bf16(o[8 * q + 6], o[8 * q + 7]));
-          }
-        }
-      };
-      {
-        uint32_t xa[32], xb[32];
-        tmem_ld32(acol, xa);
-        tmem_wait_ld(xa);
-        if (kU > 1) tmem_ld32(acol + 32, xb);
-        pass2(0, xa);
-        if (kU > 1) {
-          tmem_wait_ld(xb);
-          if (kU > 2) tmem_ld32(acol + 64, xa);
-          pass2(1, xb);
-        }
-        if (kU > 2) {
-          tmem_wait_ld(xa);
-          if (kU > 3) tmem_ld32(acol + 96, xb);
-          pass2(2, xa);
-        }
-        if (kU > 3) {
-          tmem_wait_ld(xb);
-          pass2(3, xb);
-        }
-      }
-      if (P.o_s && valid) {
-        P.m_s[tk * d.Hq + x.h] = d.no_norm ? mt + logf(lsum) : mt;
-        P.rstd_s[tk * d.Hq + x.h] = d.no_norm ? 1.f : rstd;
-      }
-      tc_fence_before();
-      mbar_arrive(&bar->acc_empty[tb]);
-      mbar_arrive(&bar->rows_free[tb]);
-      wg_sync(3, 128);
+      ok = epilogue(x, tb, 1, ok, alpha, mt, lsum);
       ++nt;
     }
   }
