@@ -189,9 +189,17 @@ static fix_status check_device() {
   return major == 10 ? FIX_OK : FIX_ERR_ARCH;
 }
 
-static fix_status launched() {
-  return cudaGetLastError() == cudaSuccess ? FIX_OK : FIX_ERR_CUDA;
+#ifdef FIX_TEST_HOOKS
+int g_test_last_cuda_error = 0;   // test builds: the last launch error seen
+#endif
+fix_status launch_status() {
+  const cudaError_t e = cudaGetLastError();
+#ifdef FIX_TEST_HOOKS
+  if (e != cudaSuccess) g_test_last_cuda_error = (int)e;
+#endif
+  return e == cudaSuccess ? FIX_OK : FIX_ERR_CUDA;
 }
+static fix_status launched() { return launch_status(); }
 
 // Records the profiling event of `stage` (begin = 0 / end = 1) if requested.
 static fix_status mark(const fix_attn_problem* p, int stage, int end, cudaStream_t st) {
@@ -233,12 +241,12 @@ bool set_smem_limit(const void* func, int bytes) {
       if (bytes <= e.bytes) return true;
       if (cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
           cudaSuccess)
-        return false;
+        return launch_status() == FIX_OK;
       e.bytes = bytes;
       return true;
     }
   if (cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
-    return false;
+    return launch_status() == FIX_OK;   // records the error (it is pending)
   done.push_back(Entry{func, dev, bytes});
   return true;
 }

@@ -292,5 +292,5 @@ extern "C" fix_status fix_attn_decode(const fix_attn_problem* p, const int32_t* 
       reinterpret_cast<const float*>(base + ws.o), reinterpret_cast<const float*>(base + ws.tot),
       static_cast<const __nv_bfloat16*>(o_norm_weight), static_cast<const __nv_bfloat16*>(o_gate),
       y, p->y_dtype == FIX_DTYPE_F32);
-  return cudaGetLastError() == cudaSuccess ? FIX_OK : FIX_ERR_CUDA;
+  return launch_status();
 }

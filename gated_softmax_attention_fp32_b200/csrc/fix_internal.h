@@ -67,6 +67,9 @@ __global__ void dkv_simt_kernel(Dims d, const Chunk* chunks, const __nv_bfloat16
 // increase, so the launch path makes no further runtime calls for it (which
 // keeps the calls cheap and lets a stream capture record the launches).
 bool set_smem_limit(const void* func, int bytes);
+// FIX_OK if no launch error is pending, else FIX_ERR_CUDA (test builds
+// record the error for fix_attn_test_last_cuda_error).
+fix_status launch_status();
 bool tc_fwd_supported(const Dims& d);
 fix_status tc_fwd(const Dims& d, const Chunk* chunks, const int* order, const void* q,
                   const void* k, const uint16_t* vt, const __nv_bfloat16* vm,

@@ -206,8 +206,8 @@ __global__ void __launch_bounds__(kPreWarps * 32, 2) bwd_pre_kernel(
   const int r0 = sub * kRows + warp;
   const int nrows = rend > r0 ? (rend - r0 + kPreWarps - 1) / kPreWarps : 0;
   const int grp = d.grp, nitems = nrows * grp;
-  // The warp's (row, q head) items in order, each item's loads issued two
-  // items ahead of its computation.
+  // The warp's (row, q head) items in order, each item's loads issued while
+  // the previous item is computed.
   struct In {
     float rs, mt, q[4], o[4], dy[4], z[4], vr[4], kr[4];
   };
@@ -227,12 +227,8 @@ __global__ void __launch_bounds__(kPreWarps * 32, 2) bwd_pre_kernel(
       ld4b(ck ? k + t * krs + (size_t)kv * Dk + c0 : nullptr, in.kr);
     }
   };
-  In cur, nx1, nx2;   // items it, it + 1, it + 2
-  if (nitems > 0) load(0, cur);
-  if (nitems > 1) load(1, nx1);
   float acc[4] = {0.f, 0.f, 0.f, 0.f}, vr[4] = {0.f, 0.f, 0.f, 0.f}, kr[4] = {0.f, 0.f, 0.f, 0.f};
-  for (int it = 0; it < nitems; ++it) {
-    if (it + 2 < nitems) load(it + 2, nx2);
+  auto process = [&](int it, const In& cur) {
     const int i = it / grp, hh = it % grp;
     const size_t t = (size_t)ch.tok0 + r0 + i * kPreWarps;
     const int h = kv * grp + hh;
@@ -290,9 +286,19 @@ __global__ void __launch_bounds__(kPreWarps * 32, 2) bwd_pre_kernel(
     }
     if (hh == grp - 1 && cv)
       *reinterpret_cast<float4*>(A + t * vrs + (size_t)kv * Dv + c0) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-    cur = nx1;
-    nx1 = nx2;
+  };
+  // two item buffers used in place, the next item's loads in flight while
+  // one is computed (a copy between buffers would wait for them)
+  In b0, b1;
+  if (nitems > 0) load(0, b0);
+  for (int it = 0; it < nitems; it += 2) {
+    if (it + 1 < nitems) load(it + 1, b1);
+    process(it, b0);
+    if (it + 1 >= nitems) break;
+    if (it + 2 < nitems) load(it + 2, b0);
+    process(it + 1, b1);
   }
+
 #pragma unroll
   for (int u = 0; u < 4; ++u) red[warp][c0 + u] = cv ? dwl[u] : 0.f;
   __syncthreads();
@@ -357,12 +363,8 @@ __global__ void __launch_bounds__(kPreWarps * 32) bwd_pre_ops_kernel(
     ld4f(cv ? do_ws + t * ors + (size_t)(kv * grp + hh) * Dv + c0 : nullptr, in.d);
     if (hh == 0) ld4f(cv ? L + t * vrs + (size_t)kv * Dv + c0 : nullptr, in.l);
   };
-  In cur, nx1, nx2;
-  if (nitems > 0) load(0, cur);
-  if (nitems > 1) load(1, nx1);
   float lr[4] = {0.f, 0.f, 0.f, 0.f};
-  for (int it = 0; it < nitems; ++it) {
-    if (it + 2 < nitems) load(it + 2, nx2);
+  auto process = [&](int it, const In& cur) {
     const int i = it / grp, hh = it % grp;
     const size_t t = (size_t)ch.tok0 + r0 + i * kPreWarps;
     const int h = kv * grp + hh;
@@ -391,9 +393,23 @@ __global__ void __launch_bounds__(kPreWarps * 32) bwd_pre_ops_kernel(
       st4b(domh + a, hi);   // hi is already bf16-exact
       st4b(doml + a, lo);
     }
-    cur = nx1;
-    nx1 = nx2;
+  };
+  // three item buffers used in place (a copy between them would wait for
+  // the loads in flight)
+  In b0, b1, b2;
+  if (nitems > 0) load(0, b0);
+  if (nitems > 1) load(1, b1);
+  for (int it = 0; it < nitems; it += 3) {
+    if (it + 2 < nitems) load(it + 2, b2);
+    process(it, b0);
+    if (it + 1 >= nitems) break;
+    if (it + 3 < nitems) load(it + 3, b0);
+    process(it + 1, b1);
+    if (it + 2 >= nitems) break;
+    if (it + 4 < nitems) load(it + 4, b1);
+    process(it + 2, b2);
   }
+
 }
 
 // dw = sum of the partials in a fixed order (deterministic).  grid

@@ -1421,7 +1421,7 @@ static fix_status launch(const Params& prm, const void* vt, const void* vm, int 
     kern<<<(unsigned)(nparts * d.Hkv), kThreads, smem, st>>>(mq, mk, mvt, mvm, mdomh, mdoml, mdot,
                                                             prm);
   }
-  return cudaGetLastError() == cudaSuccess ? FIX_OK : FIX_ERR_CUDA;
+  return launch_status();
 }
 
 // The exact terms of out-of-range channels, then the combine of the dk/dv
@@ -1435,7 +1435,7 @@ static fix_status launch_combine(const Params& prm, long long nslots, cudaStream
   if (!set_smem_limit(reinterpret_cast<const void*>(fix), smem)) return FIX_ERR_CUDA;
   fix<<<dim3(d.nchunks, d.Hkv), kFixThreads, smem, st>>>(prm);
   dkv_combine_kernel<DK, DV><<<dim3(d.nchunks * (BN / 8), d.Hkv), 256, 0, st>>>(prm);
-  return cudaGetLastError() == cudaSuccess ? FIX_OK : FIX_ERR_CUDA;
+  return launch_status();
 }
 
 }  // namespace tcb

@@ -200,8 +200,10 @@ __device__ __forceinline__ int wg_or(int id, int n, int pred) {
 }
 
 template <int DK, int DV>
-// 10 warps of at most 200 registers (64,000 of the SM's 65,536): one CTA per SM
-__global__ void __maxnreg__(200)
+// 10 warps, one CTA per SM.  Each SM sub-partition holds 16,384 registers
+// and takes every fourth warp, so two of them hold three warps: at most 168
+// registers a thread.
+__global__ void __maxnreg__(168)
     fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_vt, const __grid_constant__ CUtensorMap tm_vm,
                   const __grid_constant__ CUtensorMap tm_vml, const Params P) {
@@ -1073,7 +1075,7 @@ static fix_status launch(const Params& prm, const void* q, const void* k, const 
   if (!sms) sms = num_sms();
   const int grid = prm.ntiles < sms ? prm.ntiles : sms;
   kern<<<(unsigned)grid, kThreads, smem, st>>>(mq, mk, mvt, mvm, mvml, prm);
-  return cudaGetLastError() == cudaSuccess ? FIX_OK : FIX_ERR_CUDA;
+  return launch_status();
 }
 
 }  // namespace tcf

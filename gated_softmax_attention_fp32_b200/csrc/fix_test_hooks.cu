@@ -28,6 +28,13 @@ int test_stall_forward() { return g_stall.load(); }
 
 extern "C" void fix_attn_test_stall_forward(int on) { fix::g_stall.store(on ? 1 : 0); }
 
+// The last CUDA error a launch in the library reported (cudaError_t), for
+// diagnosing FIX_ERR_CUDA in tests.
+namespace fix {
+extern int g_test_last_cuda_error;
+}
+extern "C" int fix_attn_test_last_cuda_error(void) { return fix::g_test_last_cuda_error; }
+
 namespace {
 __global__ void exp2_poly_kernel(const float* __restrict__ x, float* __restrict__ out, int n) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
