@@ -38,9 +38,8 @@
 // exp(L_t) A_t + sum_{s<=t} P_ts exp(L_t - L_s) v_s (fp32) in place; the
 // epilogue then applies no row factor to them.
 //
-// Warp roles (320 threads):
-//   warp 0       TMA producer: Q per tile, K and V (Vt / Vm hi) through
-//                2-stage rings, Vm lo of the diagonal block
+// Warp roles (352 threads):
+//   warp 0       TMA producer: Q per tile, K through a 2-stage ring
 //   warp 1       MMA issuer (one thread) and TMEM owner
 //   warps 2-5    softmax, a thread per query row: S -> P in TMEM.  Earlier
 //                blocks in one pass (lazy row-max reference, moved in place
@@ -51,6 +50,9 @@
 //   warps 6-9    V scaling: V'' in shared memory, the tile's fold factors;
 //                then the other half of the tile's epilogue.  One warp of
 //                each group per SM sub-partition.
+//   warp 10      TMA producer: V (Vt / Vm hi) through a 2-stage ring, Vm lo
+//                of the diagonal block (apart from K, whose loads then run
+//                ahead of the V ring's waits)
 // The epilogue (a thread per row: o = alpha exp(L - rho) A written back over
 // A, the RMSNorm's sum of squares joined across the two halves, then y and
 // the saved o) runs while the next tile's first QK^T MMAs and V loads do.
@@ -74,7 +76,7 @@ using namespace sm100;
 
 constexpr int BM = 128;          // query rows per tile
 constexpr int BN = FIX_CHUNK;    // keys per block
-constexpr int kThreads = 320;
+constexpr int kThreads = 352;
 constexpr int kVsThreads = 128;  // V-scaling threads (warps 6-9)
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // lazy row-max update, natural-log units
@@ -99,15 +101,19 @@ struct Layout {
   static constexpr int kQ = 0;
   static constexpr int kK = kQ + BM * DK * 2;
   static constexpr int kV = kK + 2 * BN * DK * 2;
-  static constexpr int kVl = kV + 2 * BN * DV * 2;       // Vm lo of the diagonal block
-  static constexpr int kF = kVl + BN * DV * 2;           // [2][DV] f32 fold factors
+  // Vm lo of the diagonal block; from a tile's last MMA to the next diagonal
+  // load, the epilogue's staging tiles (8 warps x 32 rows x 32 fp32)
+  static constexpr int kVl = kV + 2 * BN * DV * 2;
+  static constexpr int kVlBytes = BN * DV * 2 > 8 * 4096 ? BN * DV * 2 : 8 * 4096;
+  static constexpr int kF = kVl + kVlBytes;              // [2][DV] f32 fold factors
   static constexpr int kBad = kF + 2 * DV * 4;           // [2][DV] int out-of-range flags
   static constexpr int kAnyBad = kBad + 2 * DV * 4;      // [2] int
   static constexpr int kRows = kAnyBad + 16;             // [2][4][BM] f32: alpha, (unused), m, l
   static constexpr int kPlo = kRows + 2 * 4 * BM * 4;    // [BM][33] u32: diagonal P_lo, key chunks 0-1
   static constexpr int kEpiW = kPlo + BM * 33 * 4;       // [DV] f32 w
   static constexpr int kSS = kEpiW + DV * 4;             // [2][BM] f32: the epilogue halves' sums of squares
-  static constexpr int kBars = (kSS + 2 * BM * 4 + 7) / 8 * 8;
+  static constexpr int kEC = kSS + 2 * BM * 4;           // [2][DV] f32: rho log2e, NaN out of range
+  static constexpr int kBars = (kEC + 2 * DV * 4 + 7) / 8 * 8;
   static constexpr int kTmem = kBars + (int)sizeof(Bars);
   static constexpr int kAbort = kTmem + 4;
   static constexpr int kBytes = kAbort + 4;
@@ -199,10 +205,108 @@ __device__ __forceinline__ int wg_or(int id, int n, int pred) {
   return out;
 }
 
+// Exact diagonal sums of out-of-range channels, in fp32 from the fp32 logits
+// of the diagonal block (TMEM columns sbase..sbase+BN of this warp's rows):
+//   A_tc <- exp(L_t) A_tc + sum_{s<=t} P_ts exp(L_t - L_s) v_s.
+// The decay goes through each 8-key sub-block's first key b:
+// exp(L_t - L_s) = exp(L_t - L_b) exp(L_b - L_s).  The key factors
+// w_s = exp(L_b - L_s) v_s cost one exponential per key (a lane per key,
+// shared by the warp's rows through shuffles), the row factors one per row
+// and sub-block.  A sub-block whose keys spread more than 60 from L_b takes
+// the direct exponential per pair; within 60 no key factor leaves the fp32
+// range and a row factor that underflows only drops terms below e^-27 of
+// their own size.  Rows before a sub-block skip it (its row factor may not
+// be finite there).  Channels go in groups of 32, their sums kept in shared
+// memory (one row of 33 floats a thread), keys chunk by chunk.
+// Not inlined: it runs only for tiles holding such channels, and its
+// registers stay out of the softmax loop.
+template <int DV>
+__device__ __noinline__ void diag_exact_sums(const float* Lrow, const float* LtK, int N,
+                                             const __nv_bfloat16* vk, int vrs, const int* bad,
+                                             float* eacc, int nk, int len, int lane,
+                                             uint32_t sbase, uint32_t acol, float c1, float moff) {
+  int nbad = 0;
+  for (int c = 0; c < DV; ++c) nbad += bad[c];
+#pragma unroll 1
+  for (int g0 = 0; g0 < nbad; g0 += 32) {
+    for (int j = 0; j < 32; ++j) eacc[j] = 0.f;
+#pragma unroll 1
+    for (int c4 = 0; c4 < BN / 32; ++c4) {
+      uint32_t xs[32];
+      tmem_ld32(sbase + c4 * 32, xs);
+      tmem_wait_ld(xs);
+      float* pv = reinterpret_cast<float*>(xs);   // P_ts, in place
+#pragma unroll
+      for (int e = 0; e < 32; ++e)
+        pv[e] = c4 * 32 + e < nk ? ex2(__uint_as_float(xs[e]) * c1 - moff) : 0.f;
+      const int sk = c4 * 32 + lane;                // this lane's key
+      const bool kin = sk < len;
+      int j = 0;
+#pragma unroll 1
+      for (int c = 0; c < DV; ++c) {
+        if (!bad[c]) continue;                      // tile-uniform
+        if (j >= g0 && j < g0 + 32) {
+          const float lt = Lrow[c];
+          const float ls = kin ? LtK[(size_t)c * N + sk] : 0.f;
+          const float vs = kin ? bf2f(vk[(size_t)sk * vrs + c]) : 0.f;
+          const float lb = __shfl_sync(0xffffffffu, ls, lane & ~7);
+          float spread = kin ? fabsf(lb - ls) : 0.f;
+          spread = fmaxf(spread, __shfl_xor_sync(0xffffffffu, spread, 1));
+          spread = fmaxf(spread, __shfl_xor_sync(0xffffffffu, spread, 2));
+          spread = fmaxf(spread, __shfl_xor_sync(0xffffffffu, spread, 4));
+          const float ws = kin && spread <= 60.f ? ex2((lb - ls) * LOG2E) * vs : 0.f;
+          float acc = 0.f;
+#pragma unroll
+          for (int sb = 0; sb < 4; ++sb) {
+            const float lbs = __shfl_sync(0xffffffffu, lb, sb * 8);
+            const float sps = __shfl_sync(0xffffffffu, spread, sb * 8);
+            const bool row_in = c4 * 32 + sb * 8 < nk;
+            if (sps <= 60.f) {
+              float part = 0.f;
+#pragma unroll
+              for (int e = 0; e < 8; ++e)
+                part += pv[sb * 8 + e] * __shfl_sync(0xffffffffu, ws, sb * 8 + e);
+              if (row_in) acc += ex2((lt - lbs) * LOG2E) * part;
+            } else {
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const float lse = __shfl_sync(0xffffffffu, ls, sb * 8 + e);
+                const float vse = __shfl_sync(0xffffffffu, vs, sb * 8 + e);
+                if (c4 * 32 + sb * 8 + e < nk) acc += pv[sb * 8 + e] * ex2((lt - lse) * LOG2E) * vse;
+              }
+            }
+          }
+          eacc[j - g0] += acc;
+        }
+        ++j;
+      }
+    }
+    // into A, column chunk by column chunk
+    int jj = 0;
+#pragma unroll 1
+    for (int cc = 0; cc < DV / 32; ++cc) {
+      uint32_t xa[32];
+      tmem_ld32(acol + cc * 32, xa);
+      tmem_wait_ld(xa);
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const int c = cc * 32 + e;
+        if (bad[c]) {
+          if (jj >= g0 && jj < g0 + 32)
+            xa[e] = __float_as_uint(ex2(Lrow[c] * LOG2E) * __uint_as_float(xa[e]) + eacc[jj - g0]);
+          ++jj;
+        }
+      }
+      tmem_st32(acol + cc * 32, xa);
+    }
+    tmem_wait_st();
+  }
+}
+
+// 11 warps, one CTA per SM.  Each SM sub-partition holds 16,384 registers
+// and takes every fourth warp, so three of them hold three warps: at most
+// 168 registers a thread.
 template <int DK, int DV>
-// 10 warps, one CTA per SM.  Each SM sub-partition holds 16,384 registers
-// and takes every fourth warp, so two of them hold three warps: at most 168
-// registers a thread.
 __global__ void __maxnreg__(168)
     fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_vt, const __grid_constant__ CUtensorMap tm_vm,
@@ -225,6 +329,7 @@ __global__ void __maxnreg__(168)
   int* sBad = reinterpret_cast<int*>(smem + Lay::kBad);
   int* sAnyBad = reinterpret_cast<int*>(smem + Lay::kAnyBad);
   float* sRows = reinterpret_cast<float*>(smem + Lay::kRows);
+  float* sEC = reinterpret_cast<float*>(smem + Lay::kEC);
   Bars* bar = reinterpret_cast<Bars*>(smem + Lay::kBars);
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(smem + Lay::kTmem);
   volatile int* sAbort = reinterpret_cast<volatile int*>(smem + Lay::kAbort);
@@ -248,7 +353,7 @@ __global__ void __maxnreg__(168)
       mbar_init(&bar->fold_ready[s], kVsThreads);
       mbar_init(&bar->rows_ready[s], 128);
     }
-    mbar_init(&bar->vlo_empty, 1);
+    mbar_init(&bar->vlo_empty, 1 + 256);   // the diagonal MMAs, then the epilogue
     mbar_init(&bar->pv_done, 1);
     mbar_init(&bar->drain, 1);
     mbar_fence_init();
@@ -269,9 +374,13 @@ __global__ void __maxnreg__(168)
   // Pass 1 forms o = alpha exp(L - rho) A (A holds the s = t term too; no row
   // factor for out-of-range channels), writes it back over A and sums its
   // squares; the two halves' sums meet in shared memory; pass 2 writes y and
-  // the saved o.  Both groups call it for every tile they take, also after a
-  // failed wait (ok_in false): its first named barrier (id 1, both groups)
-  // votes, so that both groups leave together.
+  // the saved o.  Its stores go through a per-warp staging tile in shared
+  // memory (the diagonal's Vm lo buffer, free from the tile's last MMA until
+  // the epilogue releases it): written a row per thread, read back a row per
+  // 8 lanes, so that every global store covers whole 128-byte lines.  Both
+  // groups call it for every tile they take, also after a failed wait (ok_in
+  // false): its first named barrier (id 1, both groups) votes, so that both
+  // groups leave together.
   float* sSS = reinterpret_cast<float*>(smem + Lay::kSS);
   const float* sW = reinterpret_cast<const float*>(smem + Lay::kEpiW);
   const size_t ors = (size_t)d.Hq * DV;
@@ -288,32 +397,29 @@ __global__ void __maxnreg__(168)
     // L of this row, channel-major: for a channel, the warp's 32 rows are 32
     // consecutive floats
     const float* Lr = P.Lt + (size_t)x.kv * DV * d.N + tk;
-    const size_t orow = tk * ors + (size_t)x.h * DV;
-    const size_t cb = ((size_t)x.ci * d.Hkv + x.kv) * DV;
+    const float* ec = sEC + tb * DV;
     const int u0 = grpid * kUH;
     float ss = 0.f;
-    auto prefetch_l1 = [&](int u) {
+    // all of this group's L loads in flight at once (the tile's L was pulled
+    // into L2 when the tile began)
+    float le[kUH][32];
 #pragma unroll
-      for (int e = 0; e < 32; ++e)
-        asm volatile("prefetch.global.L1 [%0];" ::"l"(Lr + (size_t)(u * 32 + e) * d.N));
-    };
-    prefetch_l1(u0);
-#pragma unroll 1
-    for (int u = u0; u < u0 + kUH; ++u) {
-      if (u + 1 < u0 + kUH) prefetch_l1(u + 1);
+    for (int h = 0; h < kUH; ++h)
+#pragma unroll
+      for (int e = 0; e < 32; ++e) le[h][e] = Lr[(size_t)((u0 + h) * 32 + e) * d.N];
+#pragma unroll
+    for (int h = 0; h < kUH; ++h) {
+      const int u = u0 + h;
       uint32_t xa[32];
       tmem_ld32(acol + u * 32, xa);
-      float le[32];
-#pragma unroll
-      for (int e = 0; e < 32; ++e) le[e] = Lr[(size_t)(u * 32 + e) * d.N];
       tmem_wait_ld(xa);
 #pragma unroll
       for (int e = 0; e < 32; ++e) {
-        const int c = u * 32 + e;
-        // rho and hr of channel c: the same address across the warp
-        const bool bad = P.hr[cb + c] > FIX_HR_MAX;
-        const float fac = bad ? 1.f : ex2((le[e] - P.rho[cb + c]) * LOG2E);
-        const float o = alpha * fac * __uint_as_float(xa[e]);
+        // exp2(L log2e - rho log2e), or 1 for an out-of-range channel (NaN
+        // in its slot); the same shared-memory word across the warp
+        const float b = ec[u * 32 + e];
+        const float f = ex2(fmaf(le[h][e], LOG2E, -b));
+        const float o = alpha * (b != b ? 1.f : f) * __uint_as_float(xa[e]);
         ss += o * o;
         xa[e] = __float_as_uint(o);
       }
@@ -326,54 +432,56 @@ __global__ void __maxnreg__(168)
     // the RMSNorm, or without it the softmax denominator: y = o / l; the
     // saved tensors are then o / l, the log-sum-exp and ones
     const float rstd = d.no_norm ? 1.0f / lsum : 1.0f / sqrtf(ss / (float)DV + d.eps);
-    auto pass2 = [&](int u, uint32_t (&xo)[32]) {
-      float* o = reinterpret_cast<float*>(xo);   // in place
-      if (P.o_s && valid) {
-        const float so = d.no_norm ? rstd : 1.f;
-        float4* dst = reinterpret_cast<float4*>(P.o_s + orow + u * 32);
+    // staging tile of this warp: [32 rows][8 float4], float4 q of row i at
+    // slot q ^ (i & 7), so that both the row writes and the column reads of
+    // eight lanes hit eight different 16-byte bank groups
+    float4* stg = reinterpret_cast<float4*>(smem + Lay::kVl) + (warp - 2) * 256;
+    const int cq = lane & 7;               // float4 of the row this lane stores
+    auto pass2 = [&](int u, const uint32_t (&xo)[32]) {
 #pragma unroll
-        for (int q = 0; q < 8; ++q)
-          dst[q] = make_float4(o[4 * q] * so, o[4 * q + 1] * so, o[4 * q + 2] * so, o[4 * q + 3] * so);
-      }
-#pragma unroll
-      for (int e = 0; e < 32; ++e) o[e] *= rstd * sW[u * 32 + e];
-      if (P.z) {
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const uint4 z4 = reinterpret_cast<const uint4*>(P.z + orow + u * 32)[q];
-          const uint32_t w4[4] = {z4.x, z4.y, z4.z, z4.w};
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            o[8 * q + 2 * i] *= swish(__uint_as_float(w4[i] << 16));
-            o[8 * q + 2 * i + 1] *= swish(__uint_as_float(w4[i] & 0xFFFF0000u));
+      for (int q = 0; q < 8; ++q)
+        stg[lane * 8 + (q ^ (lane & 7))] =
+            make_float4(__uint_as_float(xo[4 * q]), __uint_as_float(xo[4 * q + 1]),
+                        __uint_as_float(xo[4 * q + 2]), __uint_as_float(xo[4 * q + 3]));
+      __syncwarp();
+      const int c0 = u * 32 + cq * 4;
+      const float w0 = sW[c0], w1 = sW[c0 + 1], w2 = sW[c0 + 2], w3 = sW[c0 + 3];
+#pragma unroll 4
+      for (int i = 0; i < 8; ++i) {
+        const int rr = i * 4 + (lane >> 3);  // row of the warp's 32
+        const float rs = __shfl_sync(0xffffffffu, rstd, rr);
+        const float4 o = stg[rr * 8 + (cq ^ (rr & 7))];
+        const int row = (warp & 3) * 32 + rr;
+        if (row < x.len) {
+          const size_t at = ((size_t)x.tok0 + row) * ors + (size_t)x.h * DV + c0;
+          if (P.o_s) {
+            const float so = d.no_norm ? rs : 1.f;
+            *reinterpret_cast<float4*>(P.o_s + at) = make_float4(o.x * so, o.y * so, o.z * so, o.w * so);
           }
+          float y0 = o.x * rs * w0, y1 = o.y * rs * w1, y2 = o.z * rs * w2, y3 = o.w * rs * w3;
+          if (P.z) {
+            const uint2 z2 = *reinterpret_cast<const uint2*>(P.z + at);
+            y0 *= swish(__uint_as_float(z2.x << 16));
+            y1 *= swish(__uint_as_float(z2.x & 0xFFFF0000u));
+            y2 *= swish(__uint_as_float(z2.y << 16));
+            y3 *= swish(__uint_as_float(z2.y & 0xFFFF0000u));
+          }
+          if (P.y_f32)
+            *reinterpret_cast<float4*>(reinterpret_cast<float*>(P.y) + at) = make_float4(y0, y1, y2, y3);
+          else
+            *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(P.y) + at) =
+                make_uint2(pack_bf16(y0, y1), pack_bf16(y2, y3));
         }
       }
-      if (valid) {
-        if (P.y_f32) {
-          float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(P.y) + orow + u * 32);
-#pragma unroll
-          for (int q = 0; q < 8; ++q) dst[q] = make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
-        } else {
-          uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(P.y) + orow + u * 32);
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            dst[q] = make_uint4(pack_bf16(o[8 * q], o[8 * q + 1]), pack_bf16(o[8 * q + 2], o[8 * q + 3]),
-                                pack_bf16(o[8 * q + 4], o[8 * q + 5]), pack_bf16(o[8 * q + 6], o[8 * q + 7]));
-        }
-      }
+      __syncwarp();   // the tile is rewritten by the next chunk
     };
-    {
-      // pass 2 from o in TMEM, the next chunk's load in flight
-      uint32_t xa[32], xb[32];
-      tmem_ld32(acol + u0 * 32, xa);
+#pragma unroll 1
+    for (int u = u0; u < u0 + kUH; ++u) {
+      // pass 2 from o in TMEM
+      uint32_t xa[32];
+      tmem_ld32(acol + u * 32, xa);
       tmem_wait_ld(xa);
-      if (kUH > 1) tmem_ld32(acol + (u0 + 1) * 32, xb);
-      pass2(u0, xa);
-      if (kUH > 1) {
-        tmem_wait_ld(xb);
-        pass2(u0 + 1, xb);
-      }
+      pass2(u, xa);
     }
     if (grpid == 0 && P.o_s && valid) {
       P.m_s[tk * d.Hq + x.h] = d.no_norm ? mt + logf(lsum) : mt;
@@ -381,13 +489,16 @@ __global__ void __maxnreg__(168)
     }
     tc_fence_before();
     mbar_arrive(&bar->acc_empty[tb]);
+    // the staging tiles go back to the next diagonal's Vm lo (a TMA write)
+    fence_proxy_async_smem();
+    mbar_arrive(&bar->vlo_empty);
     return true;
   };
 
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
+    // ------------------------------------------------------- TMA producer: Q, K
     if (lane == 0) {
-      int kc = 0, vc = 0, nq = 0, ndiag = 0;
+      int kc = 0, nq = 0;
       bool ok = !P.stall;   // a stalled producer (test builds) issues nothing
       for (int round = 0; ok && round < rounds; ++round) {
         const int t = tile_of(round, G, cta);
@@ -410,6 +521,29 @@ __global__ void __maxnreg__(168)
           for (int hh = 0; hh < DK / 64; ++hh)
             tma_load_3d(sK + st * BN * DK + hh * BN * 64, &tm_k, &bar->k_full[st], hh * 64, x.kv, ktok);
           ++kc;
+        }
+      }
+      // every issued copy must land before the CTA may exit (also after an
+      // abort): wait for the last one or two issued per ring, timeout only
+      const Ctl drain{P.status, nullptr, ctl.limit_ns};
+      for (int n = kc - 1; n >= 0 && n >= kc - 2; --n) mbar_wait(&bar->k_full[n & 1], (n >> 1) & 1, drain);
+      if (nq > 0) mbar_wait(&bar->q_full, (nq - 1) & 1, drain);
+    }
+  } else if (warp == 10) {
+    // ------------------------------------------- TMA producer: V (Vt or Vm hi), Vm lo
+    // (its own warp, so that the K ring runs ahead of the V ring's waits)
+    if (lane == 0) {
+      int vc = 0, ndiag = 0;
+      bool ok = !P.stall;
+      for (int round = 0; ok && round < rounds; ++round) {
+        const int t = tile_of(round, G, cta);
+        if (t >= P.ntiles) continue;
+        const Tile x = tile_info(P, t);
+        if (x.len <= 0) continue;
+        for (int it = 0; it < x.nblk; ++it) {
+          const bool diag = it == x.nblk - 1;
+          const int j = diag ? x.j : x.j - 1 - it;
+          const int ktok = x.seq0 + j * BN;
           const int sv = vc & 1;
           if (vc >= 2 && !mbar_wait(&bar->v_empty[sv], ((vc >> 1) & 1) ^ 1, ctl)) { ok = false; break; }
           if (diag && ndiag > 0 && !mbar_wait(&bar->vlo_empty, (ndiag - 1) & 1, ctl)) { ok = false; break; }
@@ -425,12 +559,8 @@ __global__ void __maxnreg__(168)
           ++vc;
         }
       }
-      // every issued copy must land before the CTA may exit (also after an
-      // abort): wait for the last one or two issued per ring, timeout only
       const Ctl drain{P.status, nullptr, ctl.limit_ns};
-      for (int n = kc - 1; n >= 0 && n >= kc - 2; --n) mbar_wait(&bar->k_full[n & 1], (n >> 1) & 1, drain);
       for (int n = vc - 1; n >= 0 && n >= vc - 2; --n) mbar_wait(&bar->v_full[n & 1], (n >> 1) & 1, drain);
-      if (nq > 0) mbar_wait(&bar->q_full, (nq - 1) & 1, drain);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -714,38 +844,11 @@ __global__ void __maxnreg__(168)
           }
           const float moff = m_used * LOG2E;
           if (diag && sAnyBad[tb]) {
-            // exact diagonal sums of out-of-range channels, in fp32 from the
-            // fp32 logits: A_tc <- exp(L_t) A_tc + sum_{s<=t} P_ts exp(L_t - L_s) v_s
-            const int* bad = sBad + tb * DV;
-            const int nk = r < x.len ? r + 1 : 0;
             const size_t rowL = ((size_t)x.tok0 + (r < x.len ? r : 0)) * vrs + (size_t)x.kv * DV;
-            const float* Lk = P.L + (size_t)x.tok0 * vrs + (size_t)x.kv * DV;
-            const __nv_bfloat16* vk = P.v + (size_t)x.tok0 * vrs + (size_t)x.kv * DV;
-#pragma unroll 1
-            for (int c = 0; c < DV; ++c) {
-              if (!bad[c]) continue;   // tile-uniform
-              const float lt = P.L[rowL + c];
-              float acc = 0.f;
-#pragma unroll 1
-              for (int c4 = 0; c4 < BN / 32; ++c4) {
-                uint32_t xs[32];
-                tmem_ld32(sbase + c4 * 32, xs);
-                tmem_wait_ld();
-#pragma unroll 4
-                for (int e = 0; e < 32; ++e) {
-                  const int s = c4 * 32 + e;
-                  if (s < nk) {
-                    const float p = ex2(__uint_as_float(xs[e]) * c1 - moff);
-                    acc += p * ex2((lt - Lk[(size_t)s * vrs + c]) * LOG2E) * bf2f(vk[(size_t)s * vrs + c]);
-                  }
-                }
-              }
-              uint32_t xa;
-              asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(xa) : "r"(acol + c));
-              tmem_wait_ld();
-              tmem_st1(acol + c, __float_as_uint(ex2(lt * LOG2E) * __uint_as_float(xa) + acc));
-            }
-            tmem_wait_st();
+            diag_exact_sums<DV>(P.L + rowL, P.Lt + (size_t)x.kv * DV * d.N + x.tok0, d.N,
+                                P.v + (size_t)x.tok0 * vrs + (size_t)x.kv * DV, vrs, sBad + tb * DV,
+                                reinterpret_cast<float*>(smem + Lay::kPlo) + r * 33,
+                                r < x.len ? r + 1 : 0, x.len, lane, sbase, acol, c1, moff);
           }
           // pass 2: P, written over the S columns already read
           {
@@ -811,7 +914,7 @@ __global__ void __maxnreg__(168)
       ok = epilogue(x, tb, 0, ok, alpha, m_true, alpha * l_used);
       ++nt;
     }
-  } else if (warp >= 6) {
+  } else if (warp >= 6 && warp < 10) {
     // ------------------------------------------------------------ V scaling
     const int dt = tid - 192;                        // 0..127
     constexpr int kChunks = DV / 8;                  // 16-byte chunks per row
@@ -874,8 +977,11 @@ __global__ void __maxnreg__(168)
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const bool bad = P.hr[ti + e] > FIX_HR_MAX;
-          sF[tb * DV + lc * 8 + e] = ex2(P.rho[ti + e] * LOG2E + kexp[e]);
+          const float rho = P.rho[ti + e];
+          sF[tb * DV + lc * 8 + e] = ex2(rho * LOG2E + kexp[e]);
           sBad[tb * DV + lc * 8 + e] = bad ? 1 : 0;
+          // the epilogue's row factor exp(L - rho), or none (out of range)
+          sEC[tb * DV + lc * 8 + e] = bad ? __int_as_float(0x7fc00000) : rho * LOG2E;
         }
       }
       {
