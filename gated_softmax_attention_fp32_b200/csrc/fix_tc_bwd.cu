@@ -168,6 +168,123 @@ __device__ __forceinline__ uint4 hmul8(uint4 v, const __half2 (&fh)[4]) {
 
 // =========================================================================== dq
 
+// Named barrier (ids from 1; 0 is __syncthreads).
+__device__ __forceinline__ void named_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+// Exact diagonal dP terms of out-of-range channels c, which the MMA's dP
+// lacks: dP_ts += sum_c do_t[c] exp(L_t[c] - L_s[c]) v_s[c] for keys s <= t,
+// in fp32, added in place to the dP columns in TMEM (dp_base: this warp's
+// lanes).  As in the forward, the decay goes through each 8-key sub-block's
+// first key b: the key factors w_s[c] = exp(L_b[c] - L_s[c]) v_s[c] are
+// formed once per key (a thread per key, into shared memory), the row
+// factors do_t[c] exp(L_t[c] - L_b[c]) once per row and sub-block.  A
+// sub-block whose keys spread more than 60 from L_b, or a row whose L lies
+// more than 28 above L_b, takes the direct exponential per pair; otherwise
+// no factor and no partial product leaves the fp32 range unless the pair's
+// own exp(L_t - L_s) does, and an underflowed row factor only drops terms
+// below e^-27 of their own size.
+// Pairs above the diagonal inside a sub-block get finite values that the
+// caller's causal selection discards.  Channels go in batches of
+// kDqFixBatch.  Called by the 128 dS threads (named barrier 1), thread
+// r = row t = key s.  Not inlined: it runs only for chunks holding such
+// channels.
+constexpr int kDqFixBatch = 16;
+struct DqFixSmem {
+  float w[kDqFixBatch][BN];        // key factors
+  float lb[kDqFixBatch][BN / 8];   // L at each sub-block's first key
+  float sp[kDqFixBatch][BN / 8];   // the sub-block's spread of L
+  int idx[128];                    // the bad channels, in order
+};
+template <int DV>
+__device__ __noinline__ void dq_bad_terms(uint32_t dp_base, int r, int len, bool row_ok,
+                                          const float* Lk, const __nv_bfloat16* vk, size_t vrs,
+                                          const float* Lrow, const float* dorow,
+                                          const uint32_t* badmask, DqFixSmem* fx) {
+  const int lane = r & 31;
+  int nb = 0, before = 0;
+#pragma unroll
+  for (int w = 0; w < DV / 32; ++w) {
+    const int n = __popc(badmask[w]);
+    if (w < r / 32) before += n;
+    nb += n;
+  }
+  if (r < DV && ((badmask[r / 32] >> lane) & 1u))
+    fx->idx[before + __popc(badmask[r / 32] & ((1u << lane) - 1u))] = r;
+  const bool kin = r < len;
+#pragma unroll 1
+  for (int b0 = 0; b0 < nb; b0 += kDqFixBatch) {
+    const int nbb = min(kDqFixBatch, nb - b0);
+    named_sync(1, 128);   // the list, or the previous batch's readers
+    // key side: thread r = key s
+#pragma unroll 1
+    for (int j = 0; j < nbb; ++j) {
+      const int c = fx->idx[b0 + j];
+      const float ls = kin ? Lk[(size_t)r * vrs + c] : 0.f;
+      const float vs = kin ? bf2f(vk[(size_t)r * vrs + c]) : 0.f;
+      const float lb = __shfl_sync(0xffffffffu, ls, lane & ~7);
+      float spread = kin ? fabsf(lb - ls) : 0.f;
+      spread = fmaxf(spread, __shfl_xor_sync(0xffffffffu, spread, 1));
+      spread = fmaxf(spread, __shfl_xor_sync(0xffffffffu, spread, 2));
+      spread = fmaxf(spread, __shfl_xor_sync(0xffffffffu, spread, 4));
+      fx->w[j][r] = kin && spread <= 60.f ? ex2((lb - ls) * LOG2E) * vs : 0.f;
+      if ((lane & 7) == 0) {
+        fx->lb[j][r / 8] = lb;
+        fx->sp[j][r / 8] = spread;
+      }
+    }
+    // row side: thread r = row t
+    float dt[kDqFixBatch], lt[kDqFixBatch];
+#pragma unroll
+    for (int j = 0; j < kDqFixBatch; ++j) {
+      const int c = j < nbb ? fx->idx[b0 + j] : 0;
+      dt[j] = j < nbb && row_ok ? dorow[c] : 0.f;
+      lt[j] = j < nbb ? Lrow[c] : 0.f;
+    }
+    named_sync(1, 128);
+#pragma unroll 1
+    for (int c4 = 0; c4 < BN / 32; ++c4) {
+      uint32_t xp[32];
+      tmem_ld32(dp_base + c4 * 32, xp);
+      tmem_wait_ld(xp);
+#pragma unroll
+      for (int j = 0; j < kDqFixBatch; ++j) {
+        if (j >= nbb || !row_ok) continue;
+#pragma unroll
+        for (int sb = 0; sb < 4; ++sb) {
+          const int blk = c4 * 4 + sb, b = blk * 8;
+          if (b > r) continue;   // every key of the sub-block lies above the diagonal
+          const float lbv = fx->lb[j][blk];
+          if (fx->sp[j][blk] <= 60.f && lt[j] - lbv <= 28.f) {
+            const float a = dt[j] * ex2((lt[j] - lbv) * LOG2E);
+            const float4 w0 = *reinterpret_cast<const float4*>(&fx->w[j][b]);
+            const float4 w1 = *reinterpret_cast<const float4*>(&fx->w[j][b + 4]);
+            const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              xp[sb * 8 + e] = __float_as_uint(fmaf(a, wv[e], __uint_as_float(xp[sb * 8 + e])));
+          } else {
+            const int c = fx->idx[b0 + j];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const int key = b + e;
+              if (key <= r && key < len) {
+                const float f = ex2((lt[j] - Lk[(size_t)key * vrs + c]) * LOG2E);
+                xp[sb * 8 + e] = __float_as_uint(__uint_as_float(xp[sb * 8 + e]) +
+                                                 dt[j] * f * bf2f(vk[(size_t)key * vrs + c]));
+              }
+            }
+          }
+        }
+      }
+      tmem_st32(dp_base + c4 * 32, xp);
+    }
+    tmem_wait_st();
+  }
+}
+
+
 struct DqBars {
   uint64_t q_full, o_full, o_ready;
   uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2], v_ready[2];
@@ -183,7 +300,9 @@ struct DqLayout {
   static constexpr int kBars = kV + 2 * BN * DV * 2;
   static constexpr int kTmem = kBars + (int)sizeof(DqBars);
   static constexpr int kAbort = kTmem + 4;
-  static constexpr int kAlloc = kAbort + 4 + 1024;
+  static constexpr int kFix = (kAbort + 4 + 15) / 16 * 16;   // DqFixSmem
+  static constexpr int kAlloc = kFix + (int)sizeof(DqFixSmem) + 1024;
+  static_assert(kAlloc <= 232448, "shared memory");
 };
 
 template <int DK, int DV>
@@ -355,6 +474,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int it = 0; it < nblk; ++it) {
       if (!__all_sync(0xffffffffu, mbar_wait(&bar->s_full, it & 1, ctl))) { ok = false; break; }
       tc_fence_after();
+      if (it == 0 && any_bad)
+        dq_bad_terms<DV>(lane_base + kColP, r, ch.len, row_ok,
+                         P.L + (size_t)ch.tok0 * vrs + (size_t)kv * DV,
+                         P.v + (size_t)ch.tok0 * vrs + (size_t)kv * DV, vrs,
+                         P.L + tok * vrs + (size_t)kv * DV,
+                         P.do_ws + tok * (size_t)d.Hq * DV + (size_t)h * DV, sBadMask,
+                         reinterpret_cast<DqFixSmem*>(smem + Lay::kFix));
 #pragma unroll
       for (int c4 = 0; c4 < BN / 32; ++c4) {
         uint32_t xs[32], xp[32], pk[16];
@@ -371,32 +497,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             pk[e >> 1] = pack_bf16(p0 * (__uint_as_float(xp[e]) - dl), p1 * (__uint_as_float(xp[e + 1]) - dl));
           }
         } else {
-          if (any_bad) {
-            // out-of-range channels c: dP_ts += do_t[c] exp(L_t[c] - L_s[c])
-            // v_s[c] for keys s <= t, in fp32 (L_s, v_s are the same address
-            // across the warp)
-            const float* Lc = P.L + (size_t)ch.tok0 * vrs + (size_t)kv * DV;
-            const __nv_bfloat16* vc = P.v + (size_t)ch.tok0 * vrs + (size_t)kv * DV;
-            const int kmax = min(r, ch.len - 1);
-#pragma unroll 1
-            for (int w = 0; w < DV / 32; ++w) {
-              uint32_t msk = sBadMask[w];
-              while (msk) {
-                const int c = w * 32 + __ffs(msk) - 1;
-                msk &= msk - 1;
-                const float dtc = row_ok ? P.do_ws[tok * (size_t)d.Hq * DV + (size_t)h * DV + c] : 0.f;
-                const float ltc = P.L[tok * vrs + (size_t)kv * DV + c];
-#pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                  const int key = c4 * 32 + e;
-                  if (key <= kmax) {
-                    const float f = ex2((ltc - Lc[(size_t)key * vrs + c]) * LOG2E);
-                    xp[e] = __float_as_uint(__uint_as_float(xp[e]) + dtc * f * bf2f(vc[(size_t)key * vrs + c]));
-                  }
-                }
-              }
-            }
-          }
           // masked by selection: above the diagonal dOm Vm pairs
           // exp(L_t - rho) with exp(rho - L_s) for s > t and may overflow
 #pragma unroll
@@ -1151,8 +1251,20 @@ __global__ void __launch_bounds__(256) dkv_combine_kernel(const Params P) {
 // and the combine takes them unscaled).  One CTA per (chunk, kv head); CTAs
 // of chunks without such a channel return at once.  P is recomputed from q,
 // k and the saved row maxima as in the tensor-core kernels.
+// The decay goes through the first index f of each aligned group of 8 rows
+// (or keys): exp(L_t - L_s) = u'_t exp(L_f(t) - L_f(s)) w'_s with
+// u'_t = exp(L_t - L_f(t)) and w'_s = exp(L_f(s) - L_s), one exponential per
+// index and channel, staged with do and v folded in, and one per pair of
+// groups.  Where either group's L spreads more than kFixSpread from its
+// first index, or L rises by more than kFixRise from the key group to the
+// row group, the pairs take the direct exponential.  Within those bounds no
+// factor and no partial product leaves the fp32 range unless the pair's own
+// exp(L_t - L_s) does, and an underflowed group factor only drops terms
+// below e^-27 of their own size.
 constexpr int kFixThreads = 256;
 constexpr int kFixBatch = 8;      // bad channels staged per pass
+constexpr float kFixSpread = 30.f;
+constexpr float kFixRise = 28.f;
 
 template <int DK, int DV>
 struct FixLayout {
@@ -1163,7 +1275,11 @@ struct FixLayout {
   static constexpr int kL = kP + BN * kPs * 4;                // [kFixBatch][BN] L of the batch
   static constexpr int kV = kL + kFixBatch * BN * 4;          // [kFixBatch][BN] v
   static constexpr int kDo = kV + kFixBatch * BN * 4;         // [kFixBatch][BN] do (one head)
-  static constexpr int kM = kDo + kFixBatch * BN * 4;         // [BN] row maxima (one head)
+  static constexpr int kU = kDo + kFixBatch * BN * 4;         // [kFixBatch][BN] u' do
+  static constexpr int kWp = kU + kFixBatch * BN * 4;         // [kFixBatch][BN] w'
+  static constexpr int kLg = kWp + kFixBatch * BN * 4;        // [kFixBatch][BN / 8] L at each group's first index
+  static constexpr int kSp = kLg + kFixBatch * (BN / 8) * 4;  // [kFixBatch][BN / 8] the group's spread of L
+  static constexpr int kM = kSp + kFixBatch * (BN / 8) * 4;   // [BN] row maxima (one head)
   static constexpr int kIdx = kM + BN * 4;                    // [DV] bad channel list
   static constexpr int kBytes = kIdx + DV * 4 + 16;
   static_assert(kBytes <= 232448, "shared memory");
@@ -1187,6 +1303,10 @@ __global__ void __launch_bounds__(kFixThreads, 1) dkv_diag_exact_kernel(const Pa
   float* sL = reinterpret_cast<float*>(fsm + Lay::kL);
   float* sV = reinterpret_cast<float*>(fsm + Lay::kV);
   float* sDo = reinterpret_cast<float*>(fsm + Lay::kDo);
+  float* sU = reinterpret_cast<float*>(fsm + Lay::kU);
+  float* sWp = reinterpret_cast<float*>(fsm + Lay::kWp);
+  float* sLg = reinterpret_cast<float*>(fsm + Lay::kLg);
+  float* sSp = reinterpret_cast<float*>(fsm + Lay::kSp);
   float* sM = reinterpret_cast<float*>(fsm + Lay::kM);
   int* sIdx = reinterpret_cast<int*>(fsm + Lay::kIdx);
   int* sNb = sIdx + DV;
@@ -1284,29 +1404,67 @@ __global__ void __launch_bounds__(kFixThreads, 1) dkv_diag_exact_kernel(const Pa
     for (int b0 = 0; b0 < nbad; b0 += kFixBatch) {
       const int nb = min(kFixBatch, nbad - b0);
       __syncthreads();   // P written; the previous batch's readers are done
+      static_assert(kFixBatch * BN % kFixThreads == 0, "every lane takes part in the shuffles");
       for (int i = tid; i < kFixBatch * BN; i += kFixThreads) {
         const int b = i / BN, r = i % BN;
         const bool ok = b < nb && r < n;
         const int c = ok ? sIdx[b0 + b] : 0;
         const size_t a = (tok0 + (ok ? r : 0)) * vrs + (size_t)kv * DV + c;
-        sL[i] = ok ? P.L[a] : 0.f;
+        const float l = ok ? P.L[a] : 0.f;
+        const float dd = ok ? P.do_ws[(tok0 + r) * ors + (size_t)h * DV + c] : 0.f;
+        sL[i] = l;
         sV[i] = ok ? bf2f(P.v[a]) : 0.f;
-        sDo[i] = ok ? P.do_ws[(tok0 + r) * ors + (size_t)h * DV + c] : 0.f;
+        sDo[i] = dd;
+        // the group of 8 indices (8 lanes): its first L and its spread
+        const float lf = __shfl_sync(0xffffffffu, l, lane & ~7);
+        float sp = ok ? fabsf(l - lf) : 0.f;
+        sp = fmaxf(sp, __shfl_xor_sync(0xffffffffu, sp, 1));
+        sp = fmaxf(sp, __shfl_xor_sync(0xffffffffu, sp, 2));
+        sp = fmaxf(sp, __shfl_xor_sync(0xffffffffu, sp, 4));
+        const bool fac = ok && sp <= kFixSpread;
+        sU[i] = fac ? ex2((l - lf) * LOG2E) * dd : 0.f;
+        sWp[i] = fac ? ex2((lf - l) * LOG2E) : 0.f;
+        if ((lane & 7) == 0) {
+          sLg[i / 8] = lf;
+          sSp[i / 8] = sp;
+        }
       }
       __syncthreads();
       // dv_s[c] += sum_{t > s} P_ts exp(L_t[c] - L_s[c]) do_t[c], into the slot
       if (4 * cg < nb && s_dv < n) {
-        float ls[4], dvb[4] = {0.f, 0.f, 0.f, 0.f};
+        float ls[4], wps[4], lfs[4], dvb[4] = {0.f, 0.f, 0.f, 0.f};
+        bool fs[4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) ls[u] = sL[(4 * cg + u) * BN + s_dv];
-        for (int t = t_dv; t < n; ++t) {   // warp-uniform t: broadcast reads
-          // selected, not multiplied by zero: exp(L_t - L_s) overflows for t < s
-          if (t > s_dv) {
-            const float pts = sP[t * Lay::kPs + s_dv];
+        for (int u = 0; u < 4; ++u) {
+          const int b = 4 * cg + u;
+          ls[u] = sL[b * BN + s_dv];
+          wps[u] = sWp[b * BN + s_dv];
+          lfs[u] = sLg[b * (BN / 8) + s_dv / 8];
+          fs[u] = sSp[b * (BN / 8) + s_dv / 8] <= kFixSpread;
+        }
+        for (int g = t_dv / 8; g * 8 < n; ++g) {   // warp-uniform group: broadcast reads
+          float pts[8];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const int b = 4 * cg + u;
-              dvb[u] += pts * ex2((sL[b * BN + t] - ls[u]) * LOG2E) * sDo[b * BN + t];
+          for (int e = 0; e < 8; ++e) {
+            // selected, not multiplied by zero: exp(L_t - L_s) overflows for t < s
+            const int t = 8 * g + e;
+            pts[e] = t > s_dv && t < n ? sP[t * Lay::kPs + s_dv] : 0.f;
+          }
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int b = 4 * cg + u;
+            float acc = 0.f;
+            if (fs[u] && sSp[b * (BN / 8) + g] <= kFixSpread && sLg[b * (BN / 8) + g] - lfs[u] <= kFixRise) {
+#pragma unroll
+              for (int e = 0; e < 8; ++e) acc = fmaf(pts[e], sU[b * BN + 8 * g + e], acc);
+              dvb[u] += wps[u] * ex2((sLg[b * (BN / 8) + g] - lfs[u]) * LOG2E) * acc;
+            } else {
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const int t = 8 * g + e;
+                if (t > s_dv && t < n) acc += pts[e] * ex2((sL[b * BN + t] - ls[u]) * LOG2E) * sDo[b * BN + t];
+              }
+              dvb[u] += acc;
             }
           }
         }
@@ -1315,22 +1473,39 @@ __global__ void __launch_bounds__(kFixThreads, 1) dkv_diag_exact_kernel(const Pa
           if (4 * cg + u < nb) slot[(size_t)s_dv * (DK + DV) + DK + sIdx[b0 + 4 * cg + u]] += dvb[u];
       }
       // dP^bad_ts += sum_{c in batch} do_t[c] exp(L_t[c] - L_s[c]) v_s[c]
+      // (pairs above the diagonal get finite values there, which P = 0 then
+      // removes; the direct form selects them away instead)
       if (sb <= tb) {
         for (int b = 0; b < nb; ++b) {
-          float lt[8], dt[8], ls[8], vs[8];
+          if (sSp[b * (BN / 8) + tb] <= kFixSpread && sSp[b * (BN / 8) + sb] <= kFixSpread &&
+              sLg[b * (BN / 8) + tb] - sLg[b * (BN / 8) + sb] <= kFixRise) {
+            const float gf = ex2((sLg[b * (BN / 8) + tb] - sLg[b * (BN / 8) + sb]) * LOG2E);
+            float ut[8], ws[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            lt[i] = sL[b * BN + 8 * tb + i];
-            dt[i] = sDo[b * BN + 8 * tb + i];
-            ls[i] = sL[b * BN + 8 * sb + i];
-            vs[i] = sV[b * BN + 8 * sb + i];
+            for (int i = 0; i < 8; ++i) {
+              ut[i] = sU[b * BN + 8 * tb + i] * gf;
+              ws[i] = sWp[b * BN + 8 * sb + i] * sV[b * BN + 8 * sb + i];
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+#pragma unroll
+              for (int j = 0; j < 8; ++j) dp[i][j] = fmaf(ut[i], ws[j], dp[i][j]);
+          } else {
+            float lt[8], dt[8], ls[8], vs[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              lt[i] = sL[b * BN + 8 * tb + i];
+              dt[i] = sDo[b * BN + 8 * tb + i];
+              ls[i] = sL[b * BN + 8 * sb + i];
+              vs[i] = sV[b * BN + 8 * sb + i];
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                if (8 * sb + j <= 8 * tb + i)
+                  dp[i][j] += dt[i] * ex2((lt[i] - ls[j]) * LOG2E) * vs[j];
           }
-#pragma unroll
-          for (int i = 0; i < 8; ++i)
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-              if (8 * sb + j <= 8 * tb + i)
-                dp[i][j] += dt[i] * ex2((lt[i] - ls[j]) * LOG2E) * vs[j];
         }
       }
     }
