@@ -176,25 +176,28 @@ __device__ __forceinline__ void named_sync(int id, int n) {
 // Exact diagonal dP terms of out-of-range channels c, which the MMA's dP
 // lacks: dP_ts += sum_c do_t[c] exp(L_t[c] - L_s[c]) v_s[c] for keys s <= t,
 // in fp32, added in place to the dP columns in TMEM (dp_base: this warp's
-// lanes).  As in the forward, the decay goes through each 8-key sub-block's
-// first key b: the key factors w_s[c] = exp(L_b[c] - L_s[c]) v_s[c] are
-// formed once per key (a thread per key, into shared memory), the row
-// factors do_t[c] exp(L_t[c] - L_b[c]) once per row and sub-block.  A
-// sub-block whose keys spread more than 60 from L_b, or a row whose L lies
-// more than 28 above L_b, takes the direct exponential per pair; otherwise
-// no factor and no partial product leaves the fp32 range unless the pair's
-// own exp(L_t - L_s) does, and an underflowed row factor only drops terms
-// below e^-27 of their own size.
-// Pairs above the diagonal inside a sub-block get finite values that the
-// caller's causal selection discards.  Channels go in batches of
+// lanes).  As in the forward, the decay goes through the middle rho of each
+// 8-key sub-block's range of L: the key factors w_s[c] = exp(rho - L_s[c])
+// v_s[c] are formed once per key (a thread per key, into shared memory), the
+// row factors do_t[c] exp(L_t[c] - rho) once per row and sub-block.  A
+// sub-block whose L spreads more than 88, or a row whose L lies more than 44
+// above rho, takes the direct exponential per pair; otherwise no factor and
+// no partial product leaves the fp32 range unless the pair's own
+// exp(L_t - L_s) does, and an underflowed row factor only drops terms below
+// e^-43 of their own size.
+// A sub-block whose every L_s exceeds L_t by more than 104 is skipped: each
+// of its exponentials is below 2^-150 and flushes to zero (as the direct
+// form's would).  Pairs above the diagonal inside a sub-block get finite
+// values that the caller's causal selection discards.  Channels go in batches of
 // kDqFixBatch.  Called by the 128 dS threads (named barrier 1), thread
 // r = row t = key s.  Not inlined: it runs only for chunks holding such
 // channels.
 constexpr int kDqFixBatch = 16;
 struct DqFixSmem {
   float w[kDqFixBatch][BN];        // key factors
-  float lb[kDqFixBatch][BN / 8];   // L at each sub-block's first key
+  float lb[kDqFixBatch][BN / 8];   // the middle of each sub-block's L
   float sp[kDqFixBatch][BN / 8];   // the sub-block's spread of L
+  float lm[kDqFixBatch][BN / 8];   // the sub-block's largest L
   int idx[128];                    // the bad channels, in order
 };
 template <int DV>
@@ -223,15 +226,19 @@ __device__ __noinline__ void dq_bad_terms(uint32_t dp_base, int r, int len, bool
       const int c = fx->idx[b0 + j];
       const float ls = kin ? Lk[(size_t)r * vrs + c] : 0.f;
       const float vs = kin ? bf2f(vk[(size_t)r * vrs + c]) : 0.f;
-      const float lb = __shfl_sync(0xffffffffu, ls, lane & ~7);
-      float spread = kin ? fabsf(lb - ls) : 0.f;
-      spread = fmaxf(spread, __shfl_xor_sync(0xffffffffu, spread, 1));
-      spread = fmaxf(spread, __shfl_xor_sync(0xffffffffu, spread, 2));
-      spread = fmaxf(spread, __shfl_xor_sync(0xffffffffu, spread, 4));
-      fx->w[j][r] = kin && spread <= 60.f ? ex2((lb - ls) * LOG2E) * vs : 0.f;
+      float lmax = kin ? ls : -INFINITY, lmin = kin ? ls : INFINITY;
+#pragma unroll
+      for (int o = 1; o < 8; o <<= 1) {
+        lmax = fmaxf(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
+        lmin = fminf(lmin, __shfl_xor_sync(0xffffffffu, lmin, o));
+      }
+      const bool any = lmax >= lmin;   // the sub-block holds a key
+      const float lb = any ? 0.5f * (lmax + lmin) : 0.f, spread = any ? lmax - lmin : 0.f;
+      fx->w[j][r] = kin && spread <= 88.f ? ex2((lb - ls) * LOG2E) * vs : 0.f;
       if ((lane & 7) == 0) {
         fx->lb[j][r / 8] = lb;
         fx->sp[j][r / 8] = spread;
+        fx->lm[j][r / 8] = lmax;
       }
     }
     // row side: thread r = row t
@@ -255,8 +262,9 @@ __device__ __noinline__ void dq_bad_terms(uint32_t dp_base, int r, int len, bool
         for (int sb = 0; sb < 4; ++sb) {
           const int blk = c4 * 4 + sb, b = blk * 8;
           if (b > r) continue;   // every key of the sub-block lies above the diagonal
+          if (lt[j] - fx->lm[j][blk] < -104.f) continue;   // every term flushes to zero
           const float lbv = fx->lb[j][blk];
-          if (fx->sp[j][blk] <= 60.f && lt[j] - lbv <= 28.f) {
+          if (fx->sp[j][blk] <= 88.f && lt[j] - lbv <= 44.f) {
             const float a = dt[j] * ex2((lt[j] - lbv) * LOG2E);
             const float4 w0 = *reinterpret_cast<const float4*>(&fx->w[j][b]);
             const float4 w1 = *reinterpret_cast<const float4*>(&fx->w[j][b + 4]);
@@ -1251,19 +1259,21 @@ __global__ void __launch_bounds__(256) dkv_combine_kernel(const Params P) {
 // and the combine takes them unscaled).  One CTA per (chunk, kv head); CTAs
 // of chunks without such a channel return at once.  P is recomputed from q,
 // k and the saved row maxima as in the tensor-core kernels.
-// The decay goes through the first index f of each aligned group of 8 rows
-// (or keys): exp(L_t - L_s) = u'_t exp(L_f(t) - L_f(s)) w'_s with
-// u'_t = exp(L_t - L_f(t)) and w'_s = exp(L_f(s) - L_s), one exponential per
+// The decay goes through the middle f of each aligned group of 8 rows' (or
+// keys') range of L: exp(L_t - L_s) = u'_t exp(f(t) - f(s)) w'_s with
+// u'_t = exp(L_t - f(t)) and w'_s = exp(f(s) - L_s), one exponential per
 // index and channel, staged with do and v folded in, and one per pair of
-// groups.  Where either group's L spreads more than kFixSpread from its
-// first index, or L rises by more than kFixRise from the key group to the
-// row group, the pairs take the direct exponential.  Within those bounds no
+// groups.  Where either group's L spreads more than kFixSpread, or the
+// middle rises by more than kFixRise from the key group to the row group,
+// the pairs take the direct exponential.  Within those bounds no
 // factor and no partial product leaves the fp32 range unless the pair's own
 // exp(L_t - L_s) does, and an underflowed group factor only drops terms
-// below e^-27 of their own size.
+// below e^-27 of their own size.  A pair of groups whose every L_t lies more
+// than 104 below every L_s is skipped: each of its exponentials is below
+// 2^-150 and flushes to zero (as the direct form's would).
 constexpr int kFixThreads = 256;
 constexpr int kFixBatch = 8;      // bad channels staged per pass
-constexpr float kFixSpread = 30.f;
+constexpr float kFixSpread = 60.f;
 constexpr float kFixRise = 28.f;
 
 template <int DK, int DV>
@@ -1277,9 +1287,11 @@ struct FixLayout {
   static constexpr int kDo = kV + kFixBatch * BN * 4;         // [kFixBatch][BN] do (one head)
   static constexpr int kU = kDo + kFixBatch * BN * 4;         // [kFixBatch][BN] u' do
   static constexpr int kWp = kU + kFixBatch * BN * 4;         // [kFixBatch][BN] w'
-  static constexpr int kLg = kWp + kFixBatch * BN * 4;        // [kFixBatch][BN / 8] L at each group's first index
+  static constexpr int kLg = kWp + kFixBatch * BN * 4;        // [kFixBatch][BN / 8] the middle of each group's L
   static constexpr int kSp = kLg + kFixBatch * (BN / 8) * 4;  // [kFixBatch][BN / 8] the group's spread of L
-  static constexpr int kM = kSp + kFixBatch * (BN / 8) * 4;   // [BN] row maxima (one head)
+  static constexpr int kLx = kSp + kFixBatch * (BN / 8) * 4;  // [kFixBatch][BN / 8] the group's largest L
+  static constexpr int kLn = kLx + kFixBatch * (BN / 8) * 4;  // [kFixBatch][BN / 8] its smallest L
+  static constexpr int kM = kLn + kFixBatch * (BN / 8) * 4;   // [BN] row maxima (one head)
   static constexpr int kIdx = kM + BN * 4;                    // [DV] bad channel list
   static constexpr int kBytes = kIdx + DV * 4 + 16;
   static_assert(kBytes <= 232448, "shared memory");
@@ -1307,6 +1319,8 @@ __global__ void __launch_bounds__(kFixThreads, 1) dkv_diag_exact_kernel(const Pa
   float* sWp = reinterpret_cast<float*>(fsm + Lay::kWp);
   float* sLg = reinterpret_cast<float*>(fsm + Lay::kLg);
   float* sSp = reinterpret_cast<float*>(fsm + Lay::kSp);
+  float* sLx = reinterpret_cast<float*>(fsm + Lay::kLx);
+  float* sLn = reinterpret_cast<float*>(fsm + Lay::kLn);
   float* sM = reinterpret_cast<float*>(fsm + Lay::kM);
   int* sIdx = reinterpret_cast<int*>(fsm + Lay::kIdx);
   int* sNb = sIdx + DV;
@@ -1415,18 +1429,23 @@ __global__ void __launch_bounds__(kFixThreads, 1) dkv_diag_exact_kernel(const Pa
         sL[i] = l;
         sV[i] = ok ? bf2f(P.v[a]) : 0.f;
         sDo[i] = dd;
-        // the group of 8 indices (8 lanes): its first L and its spread
-        const float lf = __shfl_sync(0xffffffffu, l, lane & ~7);
-        float sp = ok ? fabsf(l - lf) : 0.f;
-        sp = fmaxf(sp, __shfl_xor_sync(0xffffffffu, sp, 1));
-        sp = fmaxf(sp, __shfl_xor_sync(0xffffffffu, sp, 2));
-        sp = fmaxf(sp, __shfl_xor_sync(0xffffffffu, sp, 4));
+        // the group of 8 indices (8 lanes): the middle of its L and its spread
+        float lx = ok ? l : -INFINITY, ln = ok ? l : INFINITY;
+#pragma unroll
+        for (int o = 1; o < 8; o <<= 1) {
+          lx = fmaxf(lx, __shfl_xor_sync(0xffffffffu, lx, o));
+          ln = fminf(ln, __shfl_xor_sync(0xffffffffu, ln, o));
+        }
+        const bool any = lx >= ln;   // the group holds an index
+        const float lf = any ? 0.5f * (lx + ln) : 0.f, sp = any ? lx - ln : 0.f;
         const bool fac = ok && sp <= kFixSpread;
         sU[i] = fac ? ex2((l - lf) * LOG2E) * dd : 0.f;
         sWp[i] = fac ? ex2((lf - l) * LOG2E) : 0.f;
         if ((lane & 7) == 0) {
           sLg[i / 8] = lf;
           sSp[i / 8] = sp;
+          sLx[i / 8] = lx;
+          sLn[i / 8] = ln;
         }
       }
       __syncthreads();
@@ -1453,6 +1472,7 @@ __global__ void __launch_bounds__(kFixThreads, 1) dkv_diag_exact_kernel(const Pa
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             const int b = 4 * cg + u;
+            if (sLx[b * (BN / 8) + g] - ls[u] < -104.f) continue;   // every term flushes to zero
             float acc = 0.f;
             if (fs[u] && sSp[b * (BN / 8) + g] <= kFixSpread && sLg[b * (BN / 8) + g] - lfs[u] <= kFixRise) {
 #pragma unroll
@@ -1477,6 +1497,7 @@ __global__ void __launch_bounds__(kFixThreads, 1) dkv_diag_exact_kernel(const Pa
       // removes; the direct form selects them away instead)
       if (sb <= tb) {
         for (int b = 0; b < nb; ++b) {
+          if (sLx[b * (BN / 8) + tb] - sLn[b * (BN / 8) + sb] < -104.f) continue;   // every term flushes to zero
           if (sSp[b * (BN / 8) + tb] <= kFixSpread && sSp[b * (BN / 8) + sb] <= kFixSpread &&
               sLg[b * (BN / 8) + tb] - sLg[b * (BN / 8) + sb] <= kFixRise) {
             const float gf = ex2((sLg[b * (BN / 8) + tb] - sLg[b * (BN / 8) + sb]) * LOG2E);

@@ -93,6 +93,7 @@ struct Bars {
   uint64_t acc_full[2], acc_empty[2];
   uint64_t fold_ready[2];
   uint64_t rows_ready[2];
+  uint64_t xs_sync;   // the softmax warps' meeting point in the exact sums
   uint64_t drain;
 };
 
@@ -208,99 +209,146 @@ __device__ __forceinline__ int wg_or(int id, int n, int pred) {
 // Exact diagonal sums of out-of-range channels, in fp32 from the fp32 logits
 // of the diagonal block (TMEM columns sbase..sbase+BN of this warp's rows):
 //   A_tc <- exp(L_t) A_tc + sum_{s<=t} P_ts exp(L_t - L_s) v_s.
-// The decay goes through each 8-key sub-block's first key b:
-// exp(L_t - L_s) = exp(L_t - L_b) exp(L_b - L_s).  The key factors
-// w_s = exp(L_b - L_s) v_s cost one exponential per key (a lane per key,
-// shared by the warp's rows through shuffles), the row factors one per row
-// and sub-block.  A sub-block whose keys spread more than 60 from L_b takes
-// the direct exponential per pair; within 60 no key factor leaves the fp32
-// range and a row factor that underflows only drops terms below e^-27 of
-// their own size.  Rows before a sub-block skip it (its row factor may not
-// be finite there).  Channels go in groups of 32, their sums kept in shared
-// memory (one row of 33 floats a thread), keys chunk by chunk.
-// Not inlined: it runs only for tiles holding such channels, and its
-// registers stay out of the softmax loop.
-template <int DV>
-__device__ __noinline__ void diag_exact_sums(const float* Lrow, const float* LtK, int N,
-                                             const __nv_bfloat16* vk, int vrs, const int* bad,
-                                             float* eacc, int nk, int len, int lane,
-                                             uint32_t sbase, uint32_t acol, float c1, float moff) {
+// Called by the 128 softmax threads together (thread r = row t = key s),
+// which meet on an mbarrier: sync_n meetings have taken place before, the
+// count after the call is returned, or -1 after an abort (bounded waits).
+// The decay goes through the middle rho of each 8-key sub-block's range of L:
+// exp(L_t - L_s) = exp(L_t - rho) exp(rho - L_s).  Channels go in groups:
+// the key factors w_s = exp(rho - L_s) v_s (a thread per key, all loads of
+// the group in flight at once), rho, the sub-block's spread of L and its
+// largest L go to shared memory (the P_lo staging area, free until pass 2);
+// then each row takes one exponential per sub-block.  A sub-block whose L
+// spreads more than 88 (|L_s - rho| > 44), or where the row's L lies more
+// than 44 above rho, takes the direct exponential per pair; otherwise no
+// factor and no partial product leaves the fp32 range unless the pair's own
+// exp(L_t - L_s) does, and a row factor that underflows only drops terms
+// below e^-43 of their own size.  A sub-block whose every L_s exceeds L_t by more than 104
+// is skipped: each of its exponentials is below 2^-150 and flushes to zero
+// (as the direct form's would).  Not inlined: it runs only for tiles holding
+// such channels, and its registers stay out of the softmax loop.
+constexpr int kExactGroup = 16;
+template <int DK, int DV>
+__device__ __noinline__ int diag_exact_sums(const float* Lrow, const float* LtK, int N,
+                                            const __nv_bfloat16* vk, int vrs, uint8_t* smem,
+                                            int tb, int nk, int r, uint32_t sbase, uint32_t acol,
+                                            float c1, float moff, int sync_n, int* status) {
+  using Lay = Layout<DK, DV>;
+  const Ctl ctl{status, reinterpret_cast<volatile int*>(smem + Lay::kAbort)};
+  constexpr int kG = kExactGroup, kSB = BN / 8;
+  const int lane = r & 31;
+  const int* bad = reinterpret_cast<const int*>(smem + Lay::kBad) + tb * DV;
+  float* stg = reinterpret_cast<float*>(smem + Lay::kPlo);
+  uint64_t* sync_bar = &reinterpret_cast<Bars*>(smem + Lay::kBars)->xs_sync;
+  int* list = reinterpret_cast<int*>(stg);   // [DV] the bad channels, in order
+  float* sw = stg + DV;                      // [kG][BN] key factors
+  float* slb = sw + kG * BN;                 // [kG][kSB] the middle of the sub-block's L
+  float* ssp = slb + kG * kSB;               // [kG][kSB] its spread of L
+  float* slm = ssp + kG * kSB;               // [kG][kSB] its largest L
+  auto sync = [&]() -> bool {
+    mbar_arrive(sync_bar);
+    const bool ok = mbar_wait(sync_bar, sync_n & 1, ctl);
+    ++sync_n;
+    return __all_sync(0xffffffffu, ok);
+  };
+  if (r == 0) {
+    int n = 0;
+    for (int c = 0; c < DV; ++c)
+      if (bad[c]) list[n++] = c;
+  }
   int nbad = 0;
   for (int c = 0; c < DV; ++c) nbad += bad[c];
+  const bool kin = nk > 0;   // this thread's key (nk = 0 exactly for rows past the chunk)
 #pragma unroll 1
-  for (int g0 = 0; g0 < nbad; g0 += 32) {
-    for (int j = 0; j < 32; ++j) eacc[j] = 0.f;
-#pragma unroll 1
-    for (int c4 = 0; c4 < BN / 32; ++c4) {
-      uint32_t xs[32];
-      tmem_ld32(sbase + c4 * 32, xs);
-      tmem_wait_ld(xs);
-      float* pv = reinterpret_cast<float*>(xs);   // P_ts, in place
+  for (int g0 = 0; g0 < nbad; g0 += kG) {
+    const int ng = min(kG, nbad - g0);
+    if (!sync()) return -1;   // the list written; the previous group's readers done
+    // key side: thread r = key s
+    {
+      float ls[kG], vs[kG];
 #pragma unroll
-      for (int e = 0; e < 32; ++e)
-        pv[e] = c4 * 32 + e < nk ? ex2(__uint_as_float(xs[e]) * c1 - moff) : 0.f;
-      const int sk = c4 * 32 + lane;                // this lane's key
-      const bool kin = sk < len;
-      int j = 0;
-#pragma unroll 1
-      for (int c = 0; c < DV; ++c) {
-        if (!bad[c]) continue;                      // tile-uniform
-        if (j >= g0 && j < g0 + 32) {
-          const float lt = Lrow[c];
-          const float ls = kin ? LtK[(size_t)c * N + sk] : 0.f;
-          const float vs = kin ? bf2f(vk[(size_t)sk * vrs + c]) : 0.f;
-          const float lb = __shfl_sync(0xffffffffu, ls, lane & ~7);
-          float spread = kin ? fabsf(lb - ls) : 0.f;
-          spread = fmaxf(spread, __shfl_xor_sync(0xffffffffu, spread, 1));
-          spread = fmaxf(spread, __shfl_xor_sync(0xffffffffu, spread, 2));
-          spread = fmaxf(spread, __shfl_xor_sync(0xffffffffu, spread, 4));
-          const float ws = kin && spread <= 60.f ? ex2((lb - ls) * LOG2E) * vs : 0.f;
-          float acc = 0.f;
+      for (int j = 0; j < kG; ++j) {
+        const int c = j < ng ? list[g0 + j] : 0;
+        ls[j] = j < ng && kin ? LtK[(size_t)c * N + r] : 0.f;
+        vs[j] = j < ng && kin ? bf2f(vk[(size_t)r * vrs + c]) : 0.f;
+      }
 #pragma unroll
-          for (int sb = 0; sb < 4; ++sb) {
-            const float lbs = __shfl_sync(0xffffffffu, lb, sb * 8);
-            const float sps = __shfl_sync(0xffffffffu, spread, sb * 8);
-            const bool row_in = c4 * 32 + sb * 8 < nk;
-            if (sps <= 60.f) {
-              float part = 0.f;
+      for (int j = 0; j < kG; ++j) {
+        if (j < ng) {   // uniform
+          float lm = kin ? ls[j] : -INFINITY, ln = kin ? ls[j] : INFINITY;
 #pragma unroll
-              for (int e = 0; e < 8; ++e)
-                part += pv[sb * 8 + e] * __shfl_sync(0xffffffffu, ws, sb * 8 + e);
-              if (row_in) acc += ex2((lt - lbs) * LOG2E) * part;
-            } else {
-#pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                const float lse = __shfl_sync(0xffffffffu, ls, sb * 8 + e);
-                const float vse = __shfl_sync(0xffffffffu, vs, sb * 8 + e);
-                if (c4 * 32 + sb * 8 + e < nk) acc += pv[sb * 8 + e] * ex2((lt - lse) * LOG2E) * vse;
-              }
-            }
+          for (int o = 1; o < 8; o <<= 1) {
+            lm = fmaxf(lm, __shfl_xor_sync(0xffffffffu, lm, o));
+            ln = fminf(ln, __shfl_xor_sync(0xffffffffu, ln, o));
           }
-          eacc[j - g0] += acc;
+          const bool any = lm >= ln;   // the sub-block holds a key
+          const float rho = any ? 0.5f * (lm + ln) : 0.f, sp = any ? lm - ln : 0.f;
+          sw[j * BN + r] = kin && sp <= 88.f ? ex2((rho - ls[j]) * LOG2E) * vs[j] : 0.f;
+          if ((lane & 7) == 0) {
+            slb[j * kSB + r / 8] = rho;
+            ssp[j * kSB + r / 8] = sp;
+            slm[j * kSB + r / 8] = lm;
+          }
         }
-        ++j;
       }
     }
-    // into A, column chunk by column chunk
-    int jj = 0;
-#pragma unroll 1
-    for (int cc = 0; cc < DV / 32; ++cc) {
-      uint32_t xa[32];
-      tmem_ld32(acol + cc * 32, xa);
-      tmem_wait_ld(xa);
+    // row side: thread r = row t
+    float lt[kG], acc[kG];
 #pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        const int c = cc * 32 + e;
-        if (bad[c]) {
-          if (jj >= g0 && jj < g0 + 32)
-            xa[e] = __float_as_uint(ex2(Lrow[c] * LOG2E) * __uint_as_float(xa[e]) + eacc[jj - g0]);
-          ++jj;
+    for (int j = 0; j < kG; ++j) {
+      lt[j] = j < ng ? Lrow[list[g0 + j]] : 0.f;
+      acc[j] = 0.f;
+    }
+    if (!sync()) return -1;
+    // a sub-block of 8 keys at a time: its P_ts from the logits in TMEM
+#pragma unroll 1
+    for (int blk = 0; blk < kSB; ++blk) {
+      const int b = blk * 8;
+      if (!__any_sync(0xffffffffu, b < nk)) break;     // the warp's rows all lie above
+      uint32_t x8[8];
+      tmem_ld8_wait(sbase + b, x8);
+      if (b >= nk) continue;                            // every key above the diagonal
+      float pv[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) pv[e] = b + e < nk ? ex2(__uint_as_float(x8[e]) * c1 - moff) : 0.f;
+#pragma unroll
+      for (int j = 0; j < kG; ++j) {
+        if (j >= ng) continue;
+        if (lt[j] - slm[j * kSB + blk] < -104.f) continue;   // every term flushes to zero
+        const float lbv = slb[j * kSB + blk];
+        if (ssp[j * kSB + blk] <= 88.f && lt[j] - lbv <= 44.f) {
+          const float4 w0 = *reinterpret_cast<const float4*>(sw + j * BN + b);
+          const float4 w1 = *reinterpret_cast<const float4*>(sw + j * BN + b + 4);
+          const float part = pv[0] * w0.x + pv[1] * w0.y + pv[2] * w0.z + pv[3] * w0.w +
+                             pv[4] * w1.x + pv[5] * w1.y + pv[6] * w1.z + pv[7] * w1.w;
+          acc[j] += ex2((lt[j] - lbv) * LOG2E) * part;
+        } else {
+          const int c = list[g0 + j];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int key = b + e;
+            if (key < nk)
+              acc[j] += pv[e] * ex2((lt[j] - LtK[(size_t)c * N + key]) * LOG2E) *
+                        bf2f(vk[(size_t)key * vrs + c]);
+          }
         }
       }
-      tmem_st32(acol + cc * 32, xa);
+    }
+    // into A, a column per channel
+#pragma unroll
+    for (int j = 0; j < kG; ++j) {
+      if (j < ng) {
+        const uint32_t col = acol + (uint32_t)list[g0 + j];
+        const float a = __uint_as_float(tmem_ld1(col));
+        tmem_wait_ld();
+        tmem_st1(col, __float_as_uint(ex2(lt[j] * LOG2E) * a + acc[j]));
+      }
     }
     tmem_wait_st();
   }
+  // the staging area goes back to the P_lo staging of pass 2 once every
+  // thread is done with the last group
+  if (!sync()) return -1;
+  return sync_n;
 }
 
 // 11 warps, one CTA per SM.  Each SM sub-partition holds 16,384 registers
@@ -356,6 +404,7 @@ __global__ void __maxnreg__(168)
     mbar_init(&bar->vlo_empty, 1 + 256);   // the diagonal MMAs, then the epilogue
     mbar_init(&bar->pv_done, 1);
     mbar_init(&bar->drain, 1);
+    mbar_init(&bar->xs_sync, 128);
     mbar_fence_init();
   }
   if (warp == 1) tmem_alloc(sTmem, kTmemCols);
@@ -402,14 +451,12 @@ __global__ void __maxnreg__(168)
     float ss = 0.f;
     // all of this group's L loads in flight at once (the tile's L was pulled
     // into L2 when the tile began)
-    float le[kUH][32];
-#pragma unroll
-    for (int h = 0; h < kUH; ++h)
-#pragma unroll
-      for (int e = 0; e < 32; ++e) le[h][e] = Lr[(size_t)((u0 + h) * 32 + e) * d.N];
-#pragma unroll
+#pragma unroll 1
     for (int h = 0; h < kUH; ++h) {
       const int u = u0 + h;
+      float le[1][32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) le[0][e] = Lr[(size_t)(u * 32 + e) * d.N];
       uint32_t xa[32];
       tmem_ld32(acol + u * 32, xa);
       tmem_wait_ld(xa);
@@ -418,7 +465,7 @@ __global__ void __maxnreg__(168)
         // exp2(L log2e - rho log2e), or 1 for an out-of-range channel (NaN
         // in its slot); the same shared-memory word across the warp
         const float b = ec[u * 32 + e];
-        const float f = ex2(fmaf(le[h][e], LOG2E, -b));
+        const float f = ex2(fmaf(le[0][e], LOG2E, -b));
         const float o = alpha * (b != b ? 1.f : f) * __uint_as_float(xa[e]);
         ss += o * o;
         xa[e] = __float_as_uint(o);
@@ -656,6 +703,7 @@ __global__ void __maxnreg__(168)
     const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const float c1 = d.scale * LOG2E;
     int g = 0, nt = 0;
+    int xs_n = 0;   // meetings on xs_sync so far
     bool ok = true;
     for (int round = 0; ok && round < rounds; ++round) {
       const int t = tile_of(round, G, cta);
@@ -676,20 +724,57 @@ __global__ void __maxnreg__(168)
         if (!diag) {
           // One pass: P = exp(S scale - m_used) chunk by chunk (fp16, over the
           // S columns already read), with the next chunk's TMEM load in
-          // flight.  A chunk whose maximum exceeds m_used by more than the
-          // lazy threshold moves the reference (warp-wide): the P already
-          // written in this block, the running sum and A (the earlier blocks,
-          // once their last PV has completed) are scaled by exp(m_used - m_new).
+          // flight.  The exponentials of a chunk start at once with the
+          // current reference, beside its maximum; a chunk whose maximum
+          // exceeds m_used by more than the lazy threshold (rare) moves the
+          // reference (warp-wide) and is redone: the P already written in
+          // this block, the running sum and A (the earlier blocks, once their
+          // last PV has completed) are scaled by exp(m_used - m_new).  The
+          // tile's first chunk sets the reference from its own maximum.
           float ls = 0.f;
           auto chunk = [&](const uint32_t (&xs)[32], int c4) -> bool {
-            float ma = __uint_as_float(xs[0]), mb = __uint_as_float(xs[1]);
+            // packed pairs: the scaling and the running sum as f32x2, one pair
+            // of exponentials in kPolyPairEvery as a polynomial on the FMA pipe,
+            // the rest on the MUFU unit (both well inside fp16's rounding)
+            uint32_t pk[16];
+            auto expo = [&]() -> float {
+              const float moff = m_used * LOG2E;
+              const uint64_t c1x2 = f2_pack(c1, c1), mo2 = f2_pack(-moff, -moff);
+              uint64_t lsa = f2_pack(0.f, 0.f), lsb = lsa;
 #pragma unroll
-            for (int e = 2; e < 32; e += 2) {
-              ma = fmaxf(ma, __uint_as_float(xs[e]));
-              mb = fmaxf(mb, __uint_as_float(xs[e + 1]));
-            }
-            const float cm = fmaxf(ma, mb) * d.scale;
+              for (int e = 0; e < 32; e += 2) {
+                const uint64_t a2 =
+                    f2_fma(f2_pack(__uint_as_float(xs[e]), __uint_as_float(xs[e + 1])), c1x2, mo2);
+                uint64_t p2;
+                if (kPolyPairEvery > 0 && (e >> 1) % kPolyPairEvery == kPolyPairEvery - 1) {
+                  p2 = exp2_poly3_x2(a2);
+                } else {
+                  float a0, a1;
+                  f2_unpack(a2, a0, a1);
+                  p2 = f2_pack(ex2(a0), ex2(a1));
+                }
+                if ((e >> 1) & 1) lsb = f2_add(lsb, p2);
+                else lsa = f2_add(lsa, p2);
+                float p0, p1;
+                f2_unpack(p2, p0, p1);
+                pk[e >> 1] = pack_f16(p0, p1);
+              }
+              float s0, s1;
+              f2_unpack(f2_add(lsa, lsb), s0, s1);
+              return s0 + s1;
+            };
+            // the chunk maximum, four independent chains
+            float m4[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) m4[k] = __uint_as_float(xs[k]);
+#pragma unroll
+            for (int e = 4; e < 32; e += 4)
+#pragma unroll
+              for (int k = 0; k < 4; ++k) m4[k] = fmaxf(m4[k], __uint_as_float(xs[e + k]));
+            const float cm = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * d.scale;
             m_true = fmaxf(m_true, cm);
+            if (it == 0 && c4 == 0) m_used = m_true;   // the tile's first chunk
+            float lsc = expo();
             if (__any_sync(0xffffffffu, cm > m_used + kRescaleThreshold)) {
               const float m_new = fmaxf(m_used, m_true);
               const float rr = m_used == -INFINITY ? 0.f : ex2((m_used - m_new) * LOG2E);
@@ -697,16 +782,16 @@ __global__ void __maxnreg__(168)
                 tmem_wait_st();
                 const __half2 r2 = __float2half2_rn(rr);
                 for (int cp = 0; cp < c4; ++cp) {
-                  uint32_t pk[16];
-                  tmem_ld16(sbase + cp * 16, pk);
+                  uint32_t pq[16];
+                  tmem_ld16(sbase + cp * 16, pq);
                   tmem_wait_ld();
 #pragma unroll
                   for (int e = 0; e < 16; ++e) {
-                    __half2 h = *reinterpret_cast<__half2*>(&pk[e]);
+                    __half2 h = *reinterpret_cast<__half2*>(&pq[e]);
                     h = __hmul2(h, r2);
-                    pk[e] = *reinterpret_cast<uint32_t*>(&h);
+                    pq[e] = *reinterpret_cast<uint32_t*>(&h);
                   }
-                  tmem_st16(sbase + cp * 16, pk);
+                  tmem_st16(sbase + cp * 16, pq);
                 }
               }
               if (it > 0) {
@@ -726,35 +811,9 @@ __global__ void __maxnreg__(168)
               ls *= rr;
               l_used *= rr;
               m_used = m_new;
+              lsc = expo();   // this chunk again, with the new reference
             }
-            // packed pairs: the scaling and the running sum as f32x2, one pair
-            // of exponentials in kPolyPairEvery as a polynomial on the FMA pipe,
-            // the rest on the MUFU unit (both well inside fp16's rounding)
-            const float moff = m_used * LOG2E;
-            const uint64_t c1x2 = f2_pack(c1, c1), mo2 = f2_pack(-moff, -moff);
-            uint64_t lsa = f2_pack(0.f, 0.f), lsb = lsa;
-            uint32_t pk[16];
-#pragma unroll
-            for (int e = 0; e < 32; e += 2) {
-              const uint64_t a2 =
-                  f2_fma(f2_pack(__uint_as_float(xs[e]), __uint_as_float(xs[e + 1])), c1x2, mo2);
-              uint64_t p2;
-              if (kPolyPairEvery > 0 && (e >> 1) % kPolyPairEvery == kPolyPairEvery - 1) {
-                p2 = exp2_poly3_x2(a2);
-              } else {
-                float a0, a1;
-                f2_unpack(a2, a0, a1);
-                p2 = f2_pack(ex2(a0), ex2(a1));
-              }
-              if ((e >> 1) & 1) lsb = f2_add(lsb, p2);
-              else lsa = f2_add(lsa, p2);
-              float p0, p1;
-              f2_unpack(p2, p0, p1);
-              pk[e >> 1] = pack_f16(p0, p1);
-            }
-            float s0, s1;
-            f2_unpack(f2_add(lsa, lsb), s0, s1);
-            ls += s0 + s1;
+            ls += lsc;
             tmem_st16(sbase + c4 * 16, pk);
             return true;
           };
@@ -845,10 +904,14 @@ __global__ void __maxnreg__(168)
           const float moff = m_used * LOG2E;
           if (diag && sAnyBad[tb]) {
             const size_t rowL = ((size_t)x.tok0 + (r < x.len ? r : 0)) * vrs + (size_t)x.kv * DV;
-            diag_exact_sums<DV>(P.L + rowL, P.Lt + (size_t)x.kv * DV * d.N + x.tok0, d.N,
-                                P.v + (size_t)x.tok0 * vrs + (size_t)x.kv * DV, vrs, sBad + tb * DV,
-                                reinterpret_cast<float*>(smem + Lay::kPlo) + r * 33,
-                                r < x.len ? r + 1 : 0, x.len, lane, sbase, acol, c1, moff);
+            xs_n = diag_exact_sums<DK, DV>(P.L + rowL, P.Lt + (size_t)x.kv * DV * d.N + x.tok0, d.N,
+                                           P.v + (size_t)x.tok0 * vrs + (size_t)x.kv * DV, (int)vrs,
+                                           smem, tb, r < x.len ? r + 1 : 0, r, sbase, acol, c1, moff,
+                                           xs_n, P.status);
+            if (xs_n < 0) {
+              ok = false;
+              break;
+            }
           }
           // pass 2: P, written over the S columns already read
           {
