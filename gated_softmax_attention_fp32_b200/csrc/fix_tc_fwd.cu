@@ -774,8 +774,12 @@ __global__ void __maxnreg__(168)
             const float cm = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * d.scale;
             m_true = fmaxf(m_true, cm);
             if (it == 0 && c4 == 0) m_used = m_true;   // the tile's first chunk
-            float lsc = expo();
-            if (__any_sync(0xffffffffu, cm > m_used + kRescaleThreshold)) {
+            // (one copy of the exponentials: a chunk that moves the reference
+            // takes the loop twice, the second time within the threshold)
+            float lsc;
+            while (true) {
+              lsc = expo();
+              if (!__any_sync(0xffffffffu, cm > m_used + kRescaleThreshold)) break;
               const float m_new = fmaxf(m_used, m_true);
               const float rr = m_used == -INFINITY ? 0.f : ex2((m_used - m_new) * LOG2E);
               if (c4 > 0) {
@@ -810,30 +814,29 @@ __global__ void __maxnreg__(168)
               }
               ls *= rr;
               l_used *= rr;
-              m_used = m_new;
-              lsc = expo();   // this chunk again, with the new reference
+              m_used = m_new;   // this chunk again, with the new reference
             }
             ls += lsc;
             tmem_st16(sbase + c4 * 16, pk);
             return true;
           };
+          // two chunks per pass (one code copy each), the next chunk's load
+          // in flight while one is computed
           uint32_t xa[32], xb[32];
           tmem_ld32(sbase, xa);
           tmem_wait_ld(xa);
-          tmem_ld32(sbase + 32, xb);
-          bool good = chunk(xa, 0);
-          tmem_wait_ld(xb);
-          if (good) {
-            tmem_ld32(sbase + 64, xa);
-            good = chunk(xb, 1);
-            tmem_wait_ld(xa);
-          }
-          if (good) {
-            tmem_ld32(sbase + 96, xb);
-            good = chunk(xa, 2);
+          bool good = true;
+#pragma unroll 1
+          for (int c4 = 0; c4 < BN / 32; c4 += 2) {
+            tmem_ld32(sbase + (c4 + 1) * 32, xb);
+            good = chunk(xa, c4);
             tmem_wait_ld(xb);
+            if (!good) break;
+            if (c4 + 2 < BN / 32) tmem_ld32(sbase + (c4 + 2) * 32, xa);
+            good = chunk(xb, c4 + 1);
+            if (c4 + 2 < BN / 32) tmem_wait_ld(xa);
+            if (!good) break;
           }
-          if (good) good = chunk(xb, 3);
           if (!good) {
             tmem_wait_ld();   // no TMEM load may stay in flight
             ok = false;
