@@ -528,7 +528,9 @@ fix_status fix_attn_bwd(const fix_attn_problem* p, const void* q, const void* k,
   FIX_TRY(mark(p, FIX_STAGE_BWD_PRE, 0, st));
   int* hmax = reinterpret_cast<int*>(base + ws.hmax);
   float* delta = reinterpret_cast<float*>(base + ws.delta);
-  bwd_pre_kernel<<<dim3(d.nchunks * kPreSplit, d.Hkv), 256, d.grp * sizeof(float), st>>>(
+  const size_t pre_smem = bwd_pre_smem_bytes(d.grp);
+  if (!set_smem_limit(reinterpret_cast<const void*>(bwd_pre_kernel), (int)pre_smem)) return FIX_ERR_CUDA;
+  bwd_pre_kernel<<<dim3(d.nchunks * kPreSplit, d.Hkv), 256, pre_smem, st>>>(
       d, chunks, qb, kb, vb, o_s, m_s, rstd_s, static_cast<const __nv_bfloat16*>(dy),
       static_cast<const __nv_bfloat16*>(w), static_cast<const __nv_bfloat16*>(z),
       static_cast<__nv_bfloat16*>(dz), dow, A, delta, dwp, tc ? hmax : nullptr,

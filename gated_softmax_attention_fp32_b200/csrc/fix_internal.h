@@ -46,6 +46,7 @@ __global__ void bwd_pre_kernel(Dims d, const Chunk* chunks, const __nv_bfloat16*
                                const __nv_bfloat16* w, const __nv_bfloat16* z,
                                __nv_bfloat16* dz, float* do_ws, float* A, float* delta,
                                float* dwpart, int* hmax_g, float* ptt);
+size_t bwd_pre_smem_bytes(int grp);   // dynamic shared memory of bwd_pre_kernel
 __global__ void bwd_pre_ops_kernel(Dims d, const Chunk* chunks, const float* L, const float* rho,
                                    const float* hr, const int* safe, const float* do_ws,
                                    const int* hmax_g, uint16_t* dot, __nv_bfloat16* domh,

@@ -171,11 +171,24 @@ __global__ void __launch_bounds__(256) fwd_simt_kernel(
 //   hmax[ci * Hq + h]  max |do| over the chunk (float bits, atomicMax; zeroed
 //                      by the prefix pass), only for the tensor-core kernels;
 //   ptt[t * Hq + h]    P_tt, for the tensor-core dk/dv combine (optional).
-// Dynamic shared memory: grp floats.
+// A warp's (row, q head) items arrive through a ring of kPreStages stages in
+// shared memory (cp.async, each lane copying its own 4 channels), so that
+// kPreStages - 1 items are in flight beside the one computed without
+// holding registers.  Dynamic shared memory: bwd_pre_smem_bytes(grp).
 // ---------------------------------------------------------------------------
 constexpr int kPreWarps = 8;
+constexpr int kPreStages = 4;
+// one stage of a warp: q (32 x 8 B), o (32 x 16), dy, z, v, k (32 x 8 each),
+// rstd and m (32 x 4 each: every lane copies the row's scalar)
+constexpr int kPreStageBytes = 2048;
+constexpr int kPsQ = 0, kPsO = 256, kPsDy = 768, kPsZ = 1024, kPsV = 1280, kPsK = 1536,
+              kPsRs = 1792, kPsM = 1920;
 
-__global__ void __launch_bounds__(kPreWarps * 32, 2) bwd_pre_kernel(
+size_t bwd_pre_smem_bytes(int grp) {
+  return (size_t)(grp + 3) / 4 * 16 + (size_t)kPreWarps * kPreStages * kPreStageBytes;
+}
+
+__global__ void __launch_bounds__(kPreWarps * 32, 3) bwd_pre_kernel(
     Dims d, const Chunk* __restrict__ chunks, const __nv_bfloat16* __restrict__ q,
     const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
     const float* __restrict__ o_s, const float* __restrict__ m_s,
@@ -185,7 +198,10 @@ __global__ void __launch_bounds__(kPreWarps * 32, 2) bwd_pre_kernel(
     float* __restrict__ delta_out, float* __restrict__ dwpart, int* __restrict__ hmax_g,
     float* __restrict__ ptt_out) {
   __shared__ float red[kPreWarps][128];
-  extern __shared__ float hmax[];   // [grp] max |do| per head
+  extern __shared__ __align__(16) float pre_smem[];
+  float* hmax = pre_smem;   // [grp] max |do| per head
+  uint8_t* ring = reinterpret_cast<uint8_t*>(pre_smem + (d.grp + 3) / 4 * 4) +
+                  (size_t)(threadIdx.x >> 5) * kPreStages * kPreStageBytes;
   const int Dv = d.Dv, Dk = d.Dk, kv = blockIdx.y;
   const int ci = blockIdx.x / kPreSplit, sub = blockIdx.x % kPreSplit;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -206,25 +222,51 @@ __global__ void __launch_bounds__(kPreWarps * 32, 2) bwd_pre_kernel(
   const int r0 = sub * kRows + warp;
   const int nrows = rend > r0 ? (rend - r0 + kPreWarps - 1) / kPreWarps : 0;
   const int grp = d.grp, nitems = nrows * grp;
-  // The warp's (row, q head) items in order, each item's loads issued while
-  // the previous item is computed.
+  // The warp's (row, q head) items in order, through the stage ring.
   struct In {
     float rs, mt, q[4], o[4], dy[4], z[4], vr[4], kr[4];
   };
-  auto load = [&](int it, In& in) {
+  auto issue = [&](int it) {
+    uint8_t* sb = ring + (it % kPreStages) * kPreStageBytes;
     const int i = it / grp, hh = it % grp;
     const size_t t = (size_t)ch.tok0 + r0 + i * kPreWarps;
     const int h = kv * grp + hh;
     const size_t a = t * ors + (size_t)h * Dv + c0;
-    in.rs = rstd_s[t * d.Hq + h];
-    in.mt = m_s[t * d.Hq + h];
-    ld4b(ck ? q + t * qrs + (size_t)h * Dk + c0 : nullptr, in.q);
-    ld4f(cv ? o_s + a : nullptr, in.o);
-    ld4b(cv ? dy + a : nullptr, in.dy);
-    ld4b(z && cv ? z + a : nullptr, in.z);
+    cp_async<4>(sb + kPsRs + lane * 4, rstd_s + t * d.Hq + h, true);
+    cp_async<4>(sb + kPsM + lane * 4, m_s + t * d.Hq + h, true);
+    cp_async<8>(sb + kPsQ + lane * 8, ck ? q + t * qrs + (size_t)h * Dk + c0 : q, ck);
+    cp_async<16>(sb + kPsO + lane * 16, cv ? o_s + a : o_s, cv);
+    cp_async<8>(sb + kPsDy + lane * 8, cv ? dy + a : dy, cv);
+    if (z) cp_async<8>(sb + kPsZ + lane * 8, cv ? z + a : z, cv);
     if (hh == 0) {
-      ld4b(cv ? v + t * vrs + (size_t)kv * Dv + c0 : nullptr, in.vr);
-      ld4b(ck ? k + t * krs + (size_t)kv * Dk + c0 : nullptr, in.kr);
+      cp_async<8>(sb + kPsV + lane * 8, cv ? v + t * vrs + (size_t)kv * Dv + c0 : v, cv);
+      cp_async<8>(sb + kPsK + lane * 8, ck ? k + t * krs + (size_t)kv * Dk + c0 : k, ck);
+    }
+  };
+  auto unpack_bf4 = [](const uint8_t* p, float* x) {
+    const uint2 u = *reinterpret_cast<const uint2*>(p);
+    x[0] = __uint_as_float(u.x << 16);
+    x[1] = __uint_as_float(u.x & 0xFFFF0000u);
+    x[2] = __uint_as_float(u.y << 16);
+    x[3] = __uint_as_float(u.y & 0xFFFF0000u);
+  };
+  auto fetch = [&](int it, In& in) {
+    const uint8_t* sb = ring + (it % kPreStages) * kPreStageBytes;
+    const int hh = it % grp;
+    in.rs = *reinterpret_cast<const float*>(sb + kPsRs + lane * 4);
+    in.mt = *reinterpret_cast<const float*>(sb + kPsM + lane * 4);
+    unpack_bf4(sb + kPsQ + lane * 8, in.q);
+    const float4 o4 = *reinterpret_cast<const float4*>(sb + kPsO + lane * 16);
+    in.o[0] = o4.x;
+    in.o[1] = o4.y;
+    in.o[2] = o4.z;
+    in.o[3] = o4.w;
+    unpack_bf4(sb + kPsDy + lane * 8, in.dy);
+    if (z) unpack_bf4(sb + kPsZ + lane * 8, in.z);
+    else in.z[0] = in.z[1] = in.z[2] = in.z[3] = 0.f;
+    if (hh == 0) {
+      unpack_bf4(sb + kPsV + lane * 8, in.vr);
+      unpack_bf4(sb + kPsK + lane * 8, in.kr);
     }
   };
   float acc[4] = {0.f, 0.f, 0.f, 0.f}, vr[4] = {0.f, 0.f, 0.f, 0.f}, kr[4] = {0.f, 0.f, 0.f, 0.f};
@@ -287,16 +329,19 @@ __global__ void __launch_bounds__(kPreWarps * 32, 2) bwd_pre_kernel(
     if (hh == grp - 1 && cv)
       *reinterpret_cast<float4*>(A + t * vrs + (size_t)kv * Dv + c0) = make_float4(acc[0], acc[1], acc[2], acc[3]);
   };
-  // two item buffers used in place, the next item's loads in flight while
-  // one is computed (a copy between buffers would wait for them)
-  In b0, b1;
-  if (nitems > 0) load(0, b0);
-  for (int it = 0; it < nitems; it += 2) {
-    if (it + 1 < nitems) load(it + 1, b1);
-    process(it, b0);
-    if (it + 1 >= nitems) break;
-    if (it + 2 < nitems) load(it + 2, b0);
-    process(it + 1, b1);
+  // each lane reads back only what it copied itself: its own wait is enough
+#pragma unroll
+  for (int p = 0; p < kPreStages - 1; ++p) {
+    if (p < nitems) issue(p);
+    cp_async_commit();
+  }
+  for (int it = 0; it < nitems; ++it) {
+    if (it + kPreStages - 1 < nitems) issue(it + kPreStages - 1);   // over item it - 1's stage
+    cp_async_commit();
+    cp_async_wait<kPreStages - 1>();
+    In cur;
+    fetch(it, cur);
+    process(it, cur);
   }
 
 #pragma unroll
