@@ -226,7 +226,7 @@ __device__ __forceinline__ int wg_or(int id, int n, int pred) {
 // is skipped: each of its exponentials is below 2^-150 and flushes to zero
 // (as the direct form's would).  Not inlined: it runs only for tiles holding
 // such channels, and its registers stay out of the softmax loop.
-constexpr int kExactGroup = 16;
+constexpr int kExactGroup = 8;
 template <int DK, int DV>
 __device__ __noinline__ int diag_exact_sums(const float* Lrow, const float* LtK, int N,
                                             const __nv_bfloat16* vk, int vrs, uint8_t* smem,
@@ -244,6 +244,9 @@ __device__ __noinline__ int diag_exact_sums(const float* Lrow, const float* LtK,
   float* slb = sw + kG * BN;                 // [kG][kSB] the middle of the sub-block's L
   float* ssp = slb + kG * kSB;               // [kG][kSB] its spread of L
   float* slm = ssp + kG * kSB;               // [kG][kSB] its largest L
+  float* slt = slm + kG * kSB;               // [kG][BM] L_t of each thread's row
+  float* sacc = slt + kG * BM;               // [kG][BM] each thread's sums
+  static_assert(DV + kG * BN + 3 * kG * kSB + 2 * kG * BM <= BM * 33, "staging area");
   auto sync = [&]() -> bool {
     mbar_arrive(sync_bar);
     const bool ok = mbar_wait(sync_bar, sync_n & 1, ctl);
@@ -291,12 +294,18 @@ __device__ __noinline__ int diag_exact_sums(const float* Lrow, const float* LtK,
         }
       }
     }
-    // row side: thread r = row t
-    float lt[kG], acc[kG];
+    // row side: thread r = row t; its L_t and sums live in shared memory
+    // ([j][row], conflict-free), so that the loops below stay rolled (one
+    // short code copy)
+    {
+      float lt[kG];
 #pragma unroll
-    for (int j = 0; j < kG; ++j) {
-      lt[j] = j < ng ? Lrow[list[g0 + j]] : 0.f;
-      acc[j] = 0.f;
+      for (int j = 0; j < kG; ++j) lt[j] = j < ng ? Lrow[list[g0 + j]] : 0.f;
+#pragma unroll
+      for (int j = 0; j < kG; ++j) {
+        slt[j * BM + r] = lt[j];
+        sacc[j * BM + r] = 0.f;
+      }
     }
     if (!sync()) return -1;
     // a sub-block of 8 keys at a time: its P_ts from the logits in TMEM
@@ -310,38 +319,38 @@ __device__ __noinline__ int diag_exact_sums(const float* Lrow, const float* LtK,
       float pv[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) pv[e] = b + e < nk ? ex2(__uint_as_float(x8[e]) * c1 - moff) : 0.f;
-#pragma unroll
-      for (int j = 0; j < kG; ++j) {
-        if (j >= ng) continue;
-        if (lt[j] - slm[j * kSB + blk] < -104.f) continue;   // every term flushes to zero
+#pragma unroll 1
+      for (int j = 0; j < ng; ++j) {
+        const float lt = slt[j * BM + r];
+        if (lt - slm[j * kSB + blk] < -104.f) continue;   // every term flushes to zero
         const float lbv = slb[j * kSB + blk];
-        if (ssp[j * kSB + blk] <= 88.f && lt[j] - lbv <= 44.f) {
+        float add;
+        if (ssp[j * kSB + blk] <= 88.f && lt - lbv <= 44.f) {
           const float4 w0 = *reinterpret_cast<const float4*>(sw + j * BN + b);
           const float4 w1 = *reinterpret_cast<const float4*>(sw + j * BN + b + 4);
           const float part = pv[0] * w0.x + pv[1] * w0.y + pv[2] * w0.z + pv[3] * w0.w +
                              pv[4] * w1.x + pv[5] * w1.y + pv[6] * w1.z + pv[7] * w1.w;
-          acc[j] += ex2((lt[j] - lbv) * LOG2E) * part;
+          add = ex2((lt - lbv) * LOG2E) * part;
         } else {
           const int c = list[g0 + j];
-#pragma unroll
+          add = 0.f;
+#pragma unroll 1
           for (int e = 0; e < 8; ++e) {
             const int key = b + e;
             if (key < nk)
-              acc[j] += pv[e] * ex2((lt[j] - LtK[(size_t)c * N + key]) * LOG2E) *
-                        bf2f(vk[(size_t)key * vrs + c]);
+              add += pv[e] * ex2((lt - LtK[(size_t)c * N + key]) * LOG2E) * bf2f(vk[(size_t)key * vrs + c]);
           }
         }
+        sacc[j * BM + r] += add;
       }
     }
     // into A, a column per channel
-#pragma unroll
-    for (int j = 0; j < kG; ++j) {
-      if (j < ng) {
-        const uint32_t col = acol + (uint32_t)list[g0 + j];
-        const float a = __uint_as_float(tmem_ld1(col));
-        tmem_wait_ld();
-        tmem_st1(col, __float_as_uint(ex2(lt[j] * LOG2E) * a + acc[j]));
-      }
+#pragma unroll 1
+    for (int j = 0; j < ng; ++j) {
+      const uint32_t col = acol + (uint32_t)list[g0 + j];
+      const float a = __uint_as_float(tmem_ld1(col));
+      tmem_wait_ld();
+      tmem_st1(col, __float_as_uint(ex2(slt[j * BM + r] * LOG2E) * a + sacc[j * BM + r]));
     }
     tmem_wait_st();
   }
