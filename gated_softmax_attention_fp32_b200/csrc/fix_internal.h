@@ -26,8 +26,10 @@ __global__ void prefix_kernel(Dims d, const Chunk* chunks, const float* g, const
                               float* L, float* Lt, uint16_t* vt, __nv_bfloat16* vm, __nv_bfloat16* vml,
                               float* tot, float* rho, float* hr, float* lvt, int* safe,
                               int* badflag, int* hmax);
-// Dynamic shared memory of prefix_kernel (grid (nchunks, Hkv), 512 threads);
-// lt: the channel-major copy of L is written.
+// Launch shape of prefix_kernel: grid (nchunks, Hkv, prefix_slices(Dv)), 256
+// threads, prefix_smem_bytes(Dv, lt) of dynamic shared memory (lt: the
+// channel-major copy of L is written).
+int prefix_slices(int Dv);
 size_t prefix_smem_bytes(int Dv, bool lt);
 __global__ void chunk_total_kernel(Dims d, const Chunk* chunks, const float* x, float* tot);
 __global__ void channel_sum_kernel(const float* x, long long rows, int D, float* out);

@@ -29,12 +29,13 @@ template __global__ void upload_kernel<4096>(const __grid_constant__ Blob<4096>,
 template __global__ void upload_kernel<kBlobMaxWords>(const __grid_constant__ Blob<kBlobMaxWords>,
                                                       uint32_t*, int);
 
-// grid (nchunks, Hkv), block 512: a CTA takes one chunk of one kv head, all
-// its channels; thread = (row group of 8 rows, 4 consecutive channels), so
-// every global access is a 16-byte (g, L) or 8-byte (v and the 16-bit
-// outputs) vector and a warp covers a row's channels in one coalesced
-// stretch.  The sixteen row groups are scanned in parallel and joined through
-// shared memory.
+// grid (nchunks, Hkv, channel slices of 64), block 256: a CTA takes one
+// chunk of one kv head and up to 64 of its channels; a half-warp covers a
+// row of the slice (a lane per 4 consecutive channels: 16-byte g and L, and
+// 8-byte v and 16-bit output accesses), so a warp covers two rows and every
+// row group (a half-warp) 8 rows.  The sixteen row groups are scanned in
+// parallel and joined through shared memory.  Slicing the channels gives
+// two CTAs per (chunk, kv head) at Dv = 128 and several CTAs per SM.
 //
 // Besides L and tot, the tensor-core path needs:
 //   Lt = L channel-major [Hkv][Dv][N] (forward only), written through a
@@ -57,15 +58,19 @@ template __global__ void upload_kernel<kBlobMaxWords>(const __grid_constant__ Bl
 constexpr int kPrefixThreads = 256;                       // dG scans
 constexpr int kPrefixGroups = kPrefixThreads / 32;        // row groups
 constexpr int kPrefixRows = FIX_CHUNK / kPrefixGroups;    // rows per thread
-// the prefix pass itself: twice the warps, half the rows each, so that two
-// of its dependent per-thread chains run on every scheduler
-constexpr int kPfxThreads = 512;
-constexpr int kPfxGroups = kPfxThreads / 32;
+// the prefix pass itself: channel slices of 64, a half-warp per row
+constexpr int kPfxThreads = 256;
+constexpr int kPfxLanes = 16;                             // lanes per row
+constexpr int kPfxSlice = 4 * kPfxLanes;                  // channels per CTA
+constexpr int kPfxGroups = kPfxThreads / kPfxLanes;       // row groups
 constexpr int kPfxRows = FIX_CHUNK / kPfxGroups;
 
+int prefix_slices(int Dv) { return Dv > kPfxSlice ? Dv / kPfxSlice : 1; }
+
 size_t prefix_smem_bytes(int Dv, bool lt) {
-  return (size_t)4 * kPfxGroups * Dv * sizeof(float) +
-         (lt ? (size_t)Dv * (FIX_CHUNK + 1) * sizeof(float) : 0);
+  const int sl = Dv < kPfxSlice ? Dv : kPfxSlice;
+  return (size_t)4 * kPfxGroups * sl * sizeof(float) +
+         (lt ? (size_t)sl * (FIX_CHUNK + 1) * sizeof(float) : 0);
 }
 
 namespace {
@@ -89,7 +94,7 @@ __device__ __forceinline__ void bf4_unpack(uint2 u, float* x) {
 }
 }  // namespace
 
-__global__ void __launch_bounds__(kPfxThreads) prefix_kernel(
+__global__ void __launch_bounds__(kPfxThreads, 2) prefix_kernel(
     Dims d, const Chunk* __restrict__ chunks, const float* __restrict__ g,
     const __nv_bfloat16* __restrict__ v, float* __restrict__ L, float* __restrict__ Lt,
     uint16_t* __restrict__ vt, __nv_bfloat16* __restrict__ vm, __nv_bfloat16* __restrict__ vml,
@@ -97,19 +102,26 @@ __global__ void __launch_bounds__(kPfxThreads) prefix_kernel(
     float* __restrict__ lvt, int* __restrict__ safe, int* __restrict__ badflag,
     int* __restrict__ hmax) {
   extern __shared__ float psm[];
-  const int Dv = d.Dv, nq = Dv / 4;
-  const int lane = threadIdx.x & 31, grp = threadIdx.x >> 5;
-  const bool act = lane < nq;
-  const int c0 = 4 * (act ? lane : 0);
+  const int Dv = d.Dv;
+  const int sl = Dv < kPfxSlice ? Dv : kPfxSlice;   // channels of this CTA
+  const int cb = blockIdx.z * sl;                    // its first channel
+  const int nq = sl / 4;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int qd = lane % kPfxLanes;                   // channel quad in the slice
+  const int grp = warp * (32 / kPfxLanes) + lane / kPfxLanes;   // row group
+  const bool act = qd < nq;
+  const int cl = 4 * (act ? qd : 0);                 // channel in the slice
+  const int c0 = cb + cl;
   const int ci = blockIdx.x, kv = blockIdx.y;
   const Chunk ch = chunks[ci];
-  float* part = psm;                        // [groups][Dv] group totals
-  float* pmin = part + kPfxGroups * Dv;  // [groups][Dv] group minima of L
-  float* pmax = pmin + kPfxGroups * Dv;  // [groups][Dv] group maxima
-  float* pxm = pmax + kPfxGroups * Dv;   // [groups][Dv] group max |Vt|
-  float* tr = pxm + kPfxGroups * Dv;     // [Dv][FIX_CHUNK + 1] L, channel-major
+  float* part = psm;                     // [groups][sl] group totals
+  float* pmin = part + kPfxGroups * sl;  // [groups][sl] group minima of L
+  float* pmax = pmin + kPfxGroups * sl;  // [groups][sl] group maxima
+  float* pxm = pmax + kPfxGroups * sl;   // [groups][sl] group max |Vt|
+  float* tr = pxm + kPfxGroups * sl;     // [sl][FIX_CHUNK + 1] L, channel-major
   // the backward's per-(chunk, q head) max |do|, raised by its preprocess
-  if (hmax && threadIdx.x < d.grp) hmax[(size_t)ci * d.Hq + kv * d.grp + threadIdx.x] = 0;
+  if (hmax && blockIdx.z == 0 && threadIdx.x < d.grp)
+    hmax[(size_t)ci * d.Hq + kv * d.grp + threadIdx.x] = 0;
   const size_t rs = (size_t)d.Hkv * Dv;
   const size_t base = (size_t)ch.tok0 * rs + (size_t)kv * Dv + c0;
   const int r0 = grp * kPfxRows;
@@ -149,9 +161,9 @@ __global__ void __launch_bounds__(kPfxThreads) prefix_kernel(
     }
   }
   if (act) {
-    *reinterpret_cast<float4*>(part + grp * Dv + c0) = acc;
-    *reinterpret_cast<float4*>(pmin + grp * Dv + c0) = lmin;
-    *reinterpret_cast<float4*>(pmax + grp * Dv + c0) = lmax;
+    *reinterpret_cast<float4*>(part + grp * sl + cl) = acc;
+    *reinterpret_cast<float4*>(pmin + grp * sl + cl) = lmin;
+    *reinterpret_cast<float4*>(pmax + grp * sl + cl) = lmax;
   }
   __syncthreads();
   float4 off = make_float4(0.f, 0.f, 0.f, 0.f), total = off;
@@ -160,10 +172,10 @@ __global__ void __launch_bounds__(kPfxThreads) prefix_kernel(
   if (act) {
 #pragma unroll
     for (int q = 0; q < kPfxGroups; ++q) {
-      const float4 pq = *reinterpret_cast<const float4*>(part + q * Dv + c0);
+      const float4 pq = *reinterpret_cast<const float4*>(part + q * sl + cl);
       if (q < grp) off = f4_add(off, pq);
-      cmin = f4_min(cmin, f4_add(total, *reinterpret_cast<const float4*>(pmin + q * Dv + c0)));
-      cmax = f4_max(cmax, f4_add(total, *reinterpret_cast<const float4*>(pmax + q * Dv + c0)));
+      cmin = f4_min(cmin, f4_add(total, *reinterpret_cast<const float4*>(pmin + q * sl + cl)));
+      cmax = f4_max(cmax, f4_add(total, *reinterpret_cast<const float4*>(pmax + q * sl + cl)));
       total = f4_add(total, pq);
     }
   }
@@ -174,7 +186,7 @@ __global__ void __launch_bounds__(kPfxThreads) prefix_kernel(
       *reinterpret_cast<float4*>(L + base + (size_t)(r0 + u) * rs) = lv[u];
       if (Lt) {
 #pragma unroll
-        for (int k = 0; k < 4; ++k) tr[(c0 + k) * (FIX_CHUNK + 1) + r0 + u] = f4_get(lv[u], k);
+        for (int k = 0; k < 4; ++k) tr[(cl + k) * (FIX_CHUNK + 1) + r0 + u] = f4_get(lv[u], k);
       }
     }
   const size_t ti = ((size_t)ci * d.Hkv + kv) * Dv + c0;
@@ -182,8 +194,8 @@ __global__ void __launch_bounds__(kPfxThreads) prefix_kernel(
   if (Lt) {
     // L channel-major: a warp stores 32 consecutive tokens of one channel
     __syncthreads();
-    for (int c = grp; c < Dv; c += kPfxGroups) {
-      float* dst = Lt + ((size_t)kv * Dv + c) * d.N + ch.tok0;
+    for (int c = warp; c < sl; c += kPfxThreads / 32) {
+      float* dst = Lt + ((size_t)kv * Dv + cb + c) * d.N + ch.tok0;
       for (int r = lane; r < ch.len; r += 32) dst[r] = tr[c * (FIX_CHUNK + 1) + r];
     }
   }
@@ -202,7 +214,7 @@ __global__ void __launch_bounds__(kPfxThreads) prefix_kernel(
       xmax.z = fmaxf(xmax.z, fabsf(x[2] * exp_op(total.z - lv[u].z)));
       xmax.w = fmaxf(xmax.w, fabsf(x[3] * exp_op(total.w - lv[u].w)));
     }
-  if (act) *reinterpret_cast<float4*>(pxm + grp * Dv + c0) = xmax;
+  if (act) *reinterpret_cast<float4*>(pxm + grp * sl + cl) = xmax;
   const int f16 = __syncthreads_and(nonpos && vmax <= FIX_F16_VMAX);
   if (threadIdx.x == 0 && !f16) atomicAnd(safe + (size_t)ci * d.Hkv + kv, 0);
   float ref[4], hrng[4], lg[4], sc[4];
@@ -218,7 +230,7 @@ __global__ void __launch_bounds__(kPfxThreads) prefix_kernel(
     float cx = 0.f;
     if (act) {
 #pragma unroll
-      for (int q = 0; q < kPfxGroups; ++q) cx = fmaxf(cx, pxm[q * Dv + c0 + k]);
+      for (int q = 0; q < kPfxGroups; ++q) cx = fmaxf(cx, pxm[q * sl + cl + k]);
     }
     lg[k] = cx > 0.f ? log2f(cx) : -1e30f;
     sc[k] = exp2f(-vt_exponent(lg[k]));
