@@ -377,7 +377,7 @@ static fix_status run_prefix(const Dims& d, const fix_attn_problem* p, const Ws&
   }
   const size_t psmem = prefix_smem_bytes(d.Dv, want_lt);
   if (!set_smem_limit(reinterpret_cast<const void*>(prefix_kernel), (int)psmem)) return FIX_ERR_CUDA;
-  prefix_kernel<<<dim3(d.nchunks, d.Hkv), 512, psmem, st>>>(
+  prefix_kernel<<<dim3(d.nchunks, d.Hkv, prefix_slices(d.Dv)), 256, psmem, st>>>(
       d, chunks, g, static_cast<const __nv_bfloat16*>(v), reinterpret_cast<float*>(base + ws.L),
       want_lt ? reinterpret_cast<float*>(base + ws.Lt) : nullptr,
       want_vt ? reinterpret_cast<uint16_t*>(base + ws.vt) : nullptr,
