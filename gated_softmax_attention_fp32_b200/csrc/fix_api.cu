@@ -106,8 +106,11 @@ static SplitPlan plan_split(const fix_attn_problem* p, const Dims& d) {
     for (int j = 0; j < nc; ++j) total += mult * d.grp * tiles64_host(L, j);
   });
   total *= d.Hkv;
+  // about one part per SM: each dk/dv CTA's set-up (barriers, TMEM, its key
+  // chunk's K and V) and epilogue are paid once per part, and fewer parts
+  // mean fewer partial slots for the combine to read
   constexpr int kSMs = 148;
-  long long P = (total + 2 * kSMs - 1) / (2 * kSMs);
+  long long P = (total + kSMs - 1) / kSMs;
   if (P < 4) P = 4;
   if (P > (1 << 30)) P = 1 << 30;
   sp.P = (int)P;

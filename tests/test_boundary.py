@@ -78,7 +78,7 @@ def _expected_workspace(seqlens, Hq, Hkv, Dk, Dv, backward):
     """The workspace layout written out from its documented parts: 256-byte
     aligned buffers, and for the backward the dk/dv split (per key chunk, its
     diagonal tiles and its later tiles, each cut into runs of at most P tiles,
-    P sized for about two runs per SM of a 148-SM B200), one partial slot of
+    P sized for about one run per SM of a 148-SM B200), one partial slot of
     128 rows x (Dk + Dv) floats per run and kv head."""
     grp = Hq // Hkv
     N = sum(seqlens)
@@ -102,7 +102,7 @@ def _expected_workspace(seqlens, Hq, Hkv, Dk, Dv, backward):
     t64 = lambda L, j: (L - 128 * j + 63) // 64          # query tiles from chunk j on
     half = lambda L, j: (min(128, L - 128 * j) + 63) // 64
     total = Hkv * sum(grp * t64(L, j) for L in seqlens for j in range(_ceil(L, 128)))
-    P = max(4, _ceil(total, 2 * 148))
+    P = max(4, _ceil(total, 148))
     nparts = sum(_ceil(grp * half(L, j), P) + _ceil(grp * (t64(L, j) - half(L, j)), P)
                  for L in seqlens for j in range(_ceil(L, 128)))
     for nbytes in (N * Hq * Dv * 4, N * Hq * Dv * 2, N * Hq * Dv * 2, N * Hq * Dv * 2,
