@@ -540,7 +540,7 @@ fix_status fix_attn_bwd(const fix_attn_problem* p, const void* q, const void* k,
       tc ? reinterpret_cast<float*>(base + ws.ptt) : nullptr);
   FIX_TRY(launched());
   if (tc) {
-    bwd_pre_ops_kernel<<<dim3(d.nchunks * kPreSplit, d.Hkv), 256, 0, st>>>(
+    bwd_pre_ops_kernel<<<dim3(d.nchunks * kPreOpsSplit, d.Hkv), 256, 0, st>>>(
         d, chunks, L, reinterpret_cast<const float*>(base + ws.rho),
         reinterpret_cast<const float*>(base + ws.hr), reinterpret_cast<const int*>(base + ws.safe),
         dow, hmax, dot, domh, doml, dsafe);
@@ -615,10 +615,10 @@ fix_status fix_attn_bwd(const fix_attn_problem* p, const void* q, const void* k,
   if (tc) FIX_TRY(tc_bwd(p, d, ta, 2, st));
   FIX_TRY(mark(p, FIX_STAGE_BWD_FINISH, 1, st));
   FIX_TRY(mark(p, FIX_STAGE_BWD_DG, 0, st));
-  chunk_total_kernel<<<dim3(d.nchunks, d.Hkv), 256, 0, st>>>(d, chunks, dG, dtot);
+  chunk_total_kernel<<<dim3(d.nchunks, d.Hkv, prefix_slices(d.Dv)), 256, 0, st>>>(d, chunks, dG, dtot);
   FIX_TRY(launched());
   float* dgf = d.scalar_gate ? reinterpret_cast<float*>(base + ws.dgf) : dg;
-  reverse_cumsum_kernel<<<dim3(d.nchunks, d.Hkv), 256, 0, st>>>(d, chunks, dG, dtot, dgf);
+  reverse_cumsum_kernel<<<dim3(d.nchunks, d.Hkv, prefix_slices(d.Dv)), 256, 0, st>>>(d, chunks, dG, dtot, dgf);
   FIX_TRY(launched());
   if (d.scalar_gate) {
     // a scalar gate acts on every channel: its gradient is the channel sum

@@ -17,6 +17,9 @@
 #define FIX_CHUNK 128
 // CTAs per chunk in the backward preprocess (FIX_CHUNK / kPreSplit rows each).
 constexpr int kPreSplit = 2;
+// CTAs per chunk in the preprocess's second pass (its items are smaller, so
+// more CTAs keep enough loads in flight)
+constexpr int kPreOpsSplit = 8;
 // Largest schedule piece one upload launch carries in its parameter block
 // (31 KB of the 32 KB that kernel parameters may take).
 constexpr int kBlobMaxWords = 7936;

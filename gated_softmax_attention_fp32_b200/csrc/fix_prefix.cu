@@ -55,8 +55,10 @@ template __global__ void upload_kernel<kBlobMaxWords>(const __grid_constant__ Bl
 // so that exp(G_t - G_s) = exp(L_t - rho) * exp(rho - L_s) with both factors
 // inside [e^-hr, e^hr].  Channels with hr > FIX_HR_MAX or |rho| > FIX_RHO_MAX
 // are out of range (see fix_common.cuh): Vm = 0, rho = 0, hr = FIX_HR_BAD.
-constexpr int kPrefixThreads = 256;                       // dG scans
-constexpr int kPrefixGroups = kPrefixThreads / 32;        // row groups
+// the dG scans: the same slicing as the prefix pass (64-channel slices, a
+// half-warp per row, 16 row groups of 8 rows)
+constexpr int kPrefixThreads = 256;
+constexpr int kPrefixGroups = kPrefixThreads / 16;        // row groups
 constexpr int kPrefixRows = FIX_CHUNK / kPrefixGroups;    // rows per thread
 // the prefix pass itself: channel slices of 64, a half-warp per row
 constexpr int kPfxThreads = 256;
@@ -280,11 +282,14 @@ __global__ void __launch_bounds__(kPrefixThreads) chunk_total_kernel(Dims d,
                                                                      const Chunk* __restrict__ chunks,
                                                                      const float* __restrict__ x,
                                                                      float* __restrict__ tot) {
-  __shared__ float4 part[kPrefixGroups][32];
-  const int Dv = d.Dv, nq = Dv / 4;
-  const int lane = threadIdx.x & 31, grp = threadIdx.x >> 5;
-  const bool act = lane < nq;
-  const int c0 = 4 * (act ? lane : 0);
+  __shared__ float4 part[kPrefixGroups][16];
+  const int Dv = d.Dv;
+  const int sl = Dv < kPfxSlice ? Dv : kPfxSlice;
+  const int nq = sl / 4;
+  const int lane = threadIdx.x & 31, qd = lane & 15;
+  const int grp = (threadIdx.x >> 5) * 2 + (lane >> 4);
+  const bool act = qd < nq;
+  const int c0 = blockIdx.z * sl + 4 * (act ? qd : 0);
   const int ci = blockIdx.x, kv = blockIdx.y;
   const Chunk ch = chunks[ci];
   const size_t rs = (size_t)d.Hkv * Dv;
@@ -299,12 +304,12 @@ __global__ void __launch_bounds__(kPrefixThreads) chunk_total_kernel(Dims d,
 #pragma unroll
   for (int u = 0; u < kPrefixRows; ++u)
     if (u < nr) acc = f4_add(acc, xv[u]);
-  part[grp][lane] = acc;
+  part[grp][qd] = acc;
   __syncthreads();
   if (grp == 0 && act) {
-    float4 t = part[0][lane];
+    float4 t = part[0][qd];
 #pragma unroll
-    for (int q = 1; q < kPrefixGroups; ++q) t = f4_add(t, part[q][lane]);
+    for (int q = 1; q < kPrefixGroups; ++q) t = f4_add(t, part[q][qd]);
     *reinterpret_cast<float4*>(tot + ((size_t)ci * d.Hkv + kv) * Dv + c0) = t;
   }
 }
@@ -325,11 +330,14 @@ __global__ void __launch_bounds__(256) channel_sum_kernel(const float* __restric
 __global__ void __launch_bounds__(kPrefixThreads) reverse_cumsum_kernel(
     Dims d, const Chunk* __restrict__ chunks, const float* __restrict__ x,
     const float* __restrict__ tot, float* __restrict__ out) {
-  __shared__ float4 part[kPrefixGroups][32], later[kPrefixGroups][32];
-  const int Dv = d.Dv, nq = Dv / 4;
-  const int lane = threadIdx.x & 31, grp = threadIdx.x >> 5;
-  const bool act = lane < nq;
-  const int c0 = 4 * (act ? lane : 0);
+  __shared__ float4 part[kPrefixGroups][16], later[kPrefixGroups][16];
+  const int Dv = d.Dv;
+  const int sl = Dv < kPfxSlice ? Dv : kPfxSlice;
+  const int nq = sl / 4;
+  const int lane = threadIdx.x & 31, qd = lane & 15;
+  const int grp = (threadIdx.x >> 5) * 2 + (lane >> 4);
+  const bool act = qd < nq;
+  const int c0 = blockIdx.z * sl + 4 * (act ? qd : 0);
   const int ci = blockIdx.x, kv = blockIdx.y;
   const Chunk ch = chunks[ci];
   const size_t rs = (size_t)d.Hkv * Dv;
@@ -341,7 +349,7 @@ __global__ void __launch_bounds__(kPrefixThreads) reverse_cumsum_kernel(
   for (int u = 0; u < kPrefixRows; ++u)
     if (u < nr) xv[u] = *reinterpret_cast<const float4*>(x + base + (size_t)(r0 + u) * rs);
   // the totals of the sequence's later chunks: row group q takes chunks
-  // j + 1 + q, j + 1 + q + 8, ... (two accumulators, so that the loads
+  // j + 1 + q, j + 1 + q + 16, ... (two accumulators, so that the loads
   // overlap); the groups' sums are then added in group order
   const int first = ci - ch.j;
   float4 la = make_float4(0.f, 0.f, 0.f, 0.f), lb = la;
@@ -359,14 +367,14 @@ __global__ void __launch_bounds__(kPrefixThreads) reverse_cumsum_kernel(
 #pragma unroll
   for (int u = 0; u < kPrefixRows; ++u)
     if (u < nr) own = f4_add(own, xv[u]);
-  part[grp][lane] = own;
-  later[grp][lane] = f4_add(la, lb);
+  part[grp][qd] = own;
+  later[grp][qd] = f4_add(la, lb);
   __syncthreads();
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-  for (int q = 0; q < kPrefixGroups; ++q) acc = f4_add(acc, later[q][lane]);
+  for (int q = 0; q < kPrefixGroups; ++q) acc = f4_add(acc, later[q][qd]);
   // then the later row groups of this chunk, from the last one down
-  for (int q = kPrefixGroups - 1; q > grp; --q) acc = f4_add(acc, part[q][lane]);
+  for (int q = kPrefixGroups - 1; q > grp; --q) acc = f4_add(acc, part[q][qd]);
 #pragma unroll
   for (int u = kPrefixRows - 1; u >= 0; --u)
     if (u < nr) {

@@ -360,9 +360,9 @@ __global__ void __launch_bounds__(kPreWarps * 32, 3) bwd_pre_kernel(
 }
 
 // ---------------------------------------------------------------------------
-// Backward preprocess, pass 2 (tensor-core kernels only), same grid: the
-// row-scaled upstream gradients in the two references of the forward split,
-// as 16-bit MMA operands:
+// Backward preprocess, pass 2 (tensor-core kernels only), grid
+// (nchunks * kPreOpsSplit, Hkv): the row-scaled upstream gradients in the two
+// references of the forward split, as 16-bit MMA operands:
 //   dOt_t = do_t exp(L_t)          (key blocks before the query chunk): fp16
 //                                  when dsafe, else bf16
 //   dOm_t = do_t exp(L_t - rho)    (the diagonal block; 0 for channels outside
@@ -375,7 +375,7 @@ __global__ void __launch_bounds__(kPreWarps * 32) bwd_pre_ops_kernel(
     const float* __restrict__ do_ws, const int* __restrict__ hmax_g, uint16_t* __restrict__ dot,
     __nv_bfloat16* __restrict__ domh, __nv_bfloat16* __restrict__ doml, int* __restrict__ dsafe) {
   const int Dv = d.Dv, kv = blockIdx.y;
-  const int ci = blockIdx.x / kPreSplit, sub = blockIdx.x % kPreSplit;
+  const int ci = blockIdx.x / kPreOpsSplit, sub = blockIdx.x % kPreOpsSplit;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const Chunk ch = chunks[ci];
   const bool chunk_safe = safe[(size_t)ci * d.Hkv + kv] != 0;
@@ -393,7 +393,7 @@ __global__ void __launch_bounds__(kPreWarps * 32) bwd_pre_ops_kernel(
   ld4f(cv ? hr + tb : nullptr, hq);
 #pragma unroll
   for (int u = 0; u < 4; ++u) good[u] = (cv && hq[u] <= FIX_HR_MAX) ? 1.f : 0.f;
-  constexpr int kRows = FIX_CHUNK / kPreSplit;
+  constexpr int kRows = FIX_CHUNK / kPreOpsSplit;
   const int rend = min(ch.len, (sub + 1) * kRows);
   const int r0 = sub * kRows + warp;
   const int nrows = rend > r0 ? (rend - r0 + kPreWarps - 1) / kPreWarps : 0;
