@@ -80,7 +80,12 @@ constexpr int kThreads = 352;
 constexpr int kVsThreads = 128;  // V-scaling threads (warps 6-9)
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // lazy row-max update, natural-log units
-constexpr int kPolyPairEvery = 4;  // one pair of softmax exponentials in this many by polynomial (0: none)
+// One pair of softmax exponentials in this many by the FMA-pipe polynomial
+// (0: none).  Off: with one softmax warp per scheduler the softmax is bound
+// by issue and latency, not by the MUFU unit, and the polynomial's extra
+// instructions cost more than the MUFU time they save (measured: 2.8K
+// against 3.1-3.3K cycles per block with one pair in four).
+constexpr int kPolyPairEvery = 0;
 __host__ __device__ constexpr uint32_t col_s(int b) { return b ? 128u : 0u; }
 
 struct Bars {
@@ -742,9 +747,9 @@ __global__ void __maxnreg__(168)
           // tile's first chunk sets the reference from its own maximum.
           float ls = 0.f;
           auto chunk = [&](const uint32_t (&xs)[32], int c4) -> bool {
-            // packed pairs: the scaling and the running sum as f32x2, one pair
-            // of exponentials in kPolyPairEvery as a polynomial on the FMA pipe,
-            // the rest on the MUFU unit (both well inside fp16's rounding)
+            // packed pairs: the scaling and the running sum as f32x2; the
+            // exponentials on the MUFU unit, or one pair in kPolyPairEvery as a
+            // polynomial on the FMA pipe (both well inside fp16's rounding)
             uint32_t pk[16];
             auto expo = [&]() -> float {
               const float moff = m_used * LOG2E;
