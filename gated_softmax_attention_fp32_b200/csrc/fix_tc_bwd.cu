@@ -378,7 +378,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int cta_f16 = __syncthreads_and(my_safe);
   tc_fence_after();
   const uint32_t tmem = *sTmem;
-  constexpr uint32_t kColS = 0, kColP = 128, kColQ = 256;
+  // TMEM: S (then dS over its first half) double-buffered at 0 and 384, so
+  // that the next block's QK^T runs while the dS warps work on this one;
+  // dP at 128, the dQ accumulator at 256
+  constexpr uint32_t kColP = 128, kColQ = 256;
+  auto col_sb = [](int it) -> uint32_t { return (it & 1) ? 384u : 0u; };
+  static_assert(256 + DK <= 384, "TMEM columns");
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -430,34 +435,52 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idesc_dp = idesc_bf16(128, BN, false, false, cta_f16 != 0);
       constexpr uint32_t idesc_dq = idesc_bf16(128, DK, false, true);
       const uint32_t q_addr = smem_u32(sQ), o_addr = smem_u32(sO);
-      bool ok = mbar_wait(&bar->q_full, 0, ctl) && mbar_wait(&bar->o_ready, 0, ctl);
-      for (int it = 0; ok && it < nblk; ++it) {
-        const int st = it & 1;
-        const uint32_t ph = (it >> 1) & 1;
-        if (!mbar_wait(&bar->k_full[st], ph, ctl) || !mbar_wait(&bar->v_ready[st], ph, ctl)) break;
-        if (it == 1 && !mbar_wait(&bar->o_ready, 1, ctl)) break;
-        tc_fence_after();
-        const uint32_t k_addr = smem_u32(sK + st * BN * DK), v_addr = smem_u32(sV + st * BN * DV);
+      // S of block it + 1 (QK^T, into the other S buffer) is issued right
+      // after dP of block it, so that it runs while the dS warps work
+      auto issue_s = [&](int it) {
+        const uint32_t k_addr = smem_u32(sK + (it & 1) * BN * DK);
 #pragma unroll
         for (int kk = 0; kk < DK / 16; ++kk) {
           const uint32_t off = (kk >> 2) * (BN * 128) + (kk & 3) * 32;
-          mma_ss(tmem + kColS, desc_add(desc_sw128(q_addr, 16, 1024), off), desc_add(desc_sw128(k_addr, 16, 1024), off),
-                 idesc_s, kk > 0);
+          mma_ss(tmem + col_sb(it), desc_add(desc_sw128(q_addr, 16, 1024), off),
+                 desc_add(desc_sw128(k_addr, 16, 1024), off), idesc_s, kk > 0);
         }
+      };
+      bool ok = mbar_wait(&bar->q_full, 0, ctl) && mbar_wait(&bar->o_ready, 0, ctl);
+      if (ok && nblk > 0) {
+        ok = mbar_wait(&bar->k_full[0], 0, ctl);
+        if (ok) {
+          tc_fence_after();
+          issue_s(0);
+        }
+      }
+      for (int it = 0; ok && it < nblk; ++it) {
+        const int st = it & 1;
+        const uint32_t ph = (it >> 1) & 1;
+        if (!mbar_wait(&bar->v_ready[st], ph, ctl)) break;
+        if (it == 1 && !mbar_wait(&bar->o_ready, 1, ctl)) break;
+        tc_fence_after();
+        const uint32_t k_addr = smem_u32(sK + st * BN * DK), v_addr = smem_u32(sV + st * BN * DV);
 #pragma unroll
         for (int kk = 0; kk < DV / 16; ++kk) {
           const uint32_t off = (kk >> 2) * (BN * 128) + (kk & 3) * 32;
           mma_ss(tmem + kColP, desc_add(desc_sw128(o_addr, 16, 1024), off), desc_add(desc_sw128(v_addr, 16, 1024), off),
                  it == 0 ? idesc_dp0 : idesc_dp, kk > 0);
         }
-        tc_commit(&bar->s_full);
+        tc_commit(&bar->s_full);   // S (issued before) and dP of block it
         if (it == 0) tc_commit(&bar->dp0_done);
+        if (it + 1 < nblk) {
+          // its K stage was released by block it - 1's dQ MMAs, issued before
+          if (!mbar_wait(&bar->k_full[(it + 1) & 1], ((it + 1) >> 1) & 1, ctl)) break;
+          tc_fence_after();
+          issue_s(it + 1);
+        }
         if (!mbar_wait(&bar->ds_ready, it & 1, ctl)) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
           const uint64_t b = desc_add(desc_sw128(k_addr, BN * 128, 1024), kk * 2048);
-          mma_ts(tmem + kColQ, tmem + kColS + kk * 8, b, idesc_dq, (it > 0 || kk > 0));
+          mma_ts(tmem + kColQ, tmem + col_sb(it) + kk * 8, b, idesc_dq, (it > 0 || kk > 0));
         }
         tc_commit(&bar->k_empty[st]);
         tc_commit(&bar->v_empty[st]);
@@ -492,7 +515,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int c4 = 0; c4 < BN / 32; ++c4) {
         uint32_t xs[32], xp[32], pk[16];
-        tmem_ld32(lane_base + kColS + c4 * 32, xs);
+        tmem_ld32(lane_base + col_sb(it) + c4 * 32, xs);
         tmem_ld32(lane_base + kColP + c4 * 32, xp);
         tmem_wait_ld();
         // rows past the chunk's end only feed dQ rows that are never stored;
@@ -515,7 +538,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             pk[e >> 1] = pack_bf16(d0, d1);
           }
         }
-        tmem_st16(lane_base + kColS + c4 * 16, pk);
+        tmem_st16(lane_base + col_sb(it) + c4 * 16, pk);
       }
       tmem_wait_st();
       tc_fence_before();
