@@ -661,7 +661,7 @@ struct KvLayout {
   static constexpr int kQ = kV + BN * DV * 2;               // stage region
   static constexpr int kStageOff = BQ * (DK + DV) * 2;      // bytes per later-block stage
   static constexpr int kStageDiag = BQ * (DK + 2 * DV) * 2; // bytes per diagonal stage
-  static constexpr int kM = kQ + kQStages * kStageOff;      // stages x [64] f32 row max
+  static constexpr int kM = kQ + kQStages * kStageOff;      // stages x [64] f32 row max x log2(e)
   static_assert(2 * kStageDiag <= kQStages * kStageOff, "diagonal stages must fit the region");
   static constexpr int kDl = kM + kQStages * BQ * 4;        // stages x [64] f32 sum do o
   static constexpr int kBars = kDl + kQStages * BQ * 4;
@@ -906,7 +906,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      const float* mrow = sM + st * BQ;
+      const float* mrow = sM + st * BQ;       // row maxima times log2(e)
       const float* dlrow = sDl + st * BQ;     // zeros with the norm
       const bool full = !dmode && qlen == BQ;
       const int lo = dmode ? s - t.half * BQ : 0;   // first valid query column
@@ -923,8 +923,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           // full later tile: no masking
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
-            const float p0 = ex2(__uint_as_float(xs[e]) * c1 - mrow[32 * h + e] * LOG2E);
-            const float p1 = ex2(__uint_as_float(xs[e + 1]) * c1 - mrow[32 * h + e + 1] * LOG2E);
+            const float p0 = ex2(fmaf(__uint_as_float(xs[e]), c1, -mrow[32 * h + e]));
+            const float p1 = ex2(fmaf(__uint_as_float(xs[e + 1]), c1, -mrow[32 * h + e + 1]));
             ph[e >> 1] = cta_f16 ? pack_f16(p0, p1) : pack_bf16(p0, p1);
             pd[e >> 1] = pack_bf16(p0 * (__uint_as_float(xp[e]) - dlrow[32 * h + e]),
                                    p1 * (__uint_as_float(xp[e + 1]) - dlrow[32 * h + e + 1]));
@@ -939,7 +939,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int u = 0; u < 2; ++u) {
               const int qi = 32 * h + e + u;
               const bool valid = qi >= lo && qi < qlen;
-              p[u] = valid ? ex2(__uint_as_float(xs[e + u]) * c1 - mrow[qi] * LOG2E) : 0.f;
+              p[u] = valid ? ex2(fmaf(__uint_as_float(xs[e + u]), c1, -mrow[qi])) : 0.f;
               pv[u] = (dmode && qi == lo) ? 0.f : p[u];
             }
             if (dmode) {
@@ -1121,7 +1121,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           fence_proxy_async_smem();
         }
         if (dt < BQ) {
-          sM[st * BQ + dt] = cur.m;
+          sM[st * BQ + dt] = cur.m * LOG2E;   // in log2 units, as the exponentials take it
           sDl[st * BQ + dt] = cur.dl;
         }
         mbar_arrive(&bar->x_ready[st]);
