@@ -185,7 +185,8 @@ constexpr int kPsQ = 0, kPsO = 256, kPsDy = 768, kPsZ = 1024, kPsV = 1280, kPsK 
               kPsRs = 1792, kPsM = 1920;
 
 size_t bwd_pre_smem_bytes(int grp) {
-  return (size_t)(grp + 3) / 4 * 16 + (size_t)kPreWarps * kPreStages * kPreStageBytes;
+  return (size_t)(grp + 3) / 4 * 16 + (size_t)kPreWarps * grp * 32 * sizeof(float) +
+         (size_t)kPreWarps * kPreStages * kPreStageBytes;
 }
 
 __global__ void __launch_bounds__(kPreWarps * 32, 3) bwd_pre_kernel(
@@ -200,7 +201,10 @@ __global__ void __launch_bounds__(kPreWarps * 32, 3) bwd_pre_kernel(
   __shared__ float red[kPreWarps][128];
   extern __shared__ __align__(16) float pre_smem[];
   float* hmax = pre_smem;   // [grp] max |do| per head
-  uint8_t* ring = reinterpret_cast<uint8_t*>(pre_smem + (d.grp + 3) / 4 * 4) +
+  // [warps][grp][32] each lane's running max |do| per head, joined once at
+  // the end instead of a warp reduction per item
+  float* lmax = pre_smem + (d.grp + 3) / 4 * 4 + (size_t)(threadIdx.x >> 5) * d.grp * 32;
+  uint8_t* ring = reinterpret_cast<uint8_t*>(pre_smem + (d.grp + 3) / 4 * 4 + kPreWarps * d.grp * 32) +
                   (size_t)(threadIdx.x >> 5) * kPreStages * kPreStageBytes;
   const int Dv = d.Dv, Dk = d.Dk, kv = blockIdx.y;
   const int ci = blockIdx.x / kPreSplit, sub = blockIdx.x % kPreSplit;
@@ -322,13 +326,12 @@ __global__ void __launch_bounds__(kPreWarps * 32, 3) bwd_pre_kernel(
         st4b(dz + a, g4);
       }
     }
-    if (hmax_g) {
-      mx = warp_max(mx);
-      if (lane == 0) atomicMax(reinterpret_cast<int*>(&hmax[hh]), __float_as_int(mx));
-    }
+    if (hmax_g) lmax[hh * 32 + lane] = fmaxf(lmax[hh * 32 + lane], mx);
     if (hh == grp - 1 && cv)
       *reinterpret_cast<float4*>(A + t * vrs + (size_t)kv * Dv + c0) = make_float4(acc[0], acc[1], acc[2], acc[3]);
   };
+  if (hmax_g)
+    for (int hh = 0; hh < grp; ++hh) lmax[hh * 32 + lane] = 0.f;   // lane-private slots
   // each lane reads back only what it copied itself: its own wait is enough
 #pragma unroll
   for (int p = 0; p < kPreStages - 1; ++p) {
@@ -344,6 +347,11 @@ __global__ void __launch_bounds__(kPreWarps * 32, 3) bwd_pre_kernel(
     process(it, cur);
   }
 
+  if (hmax_g)
+    for (int hh = 0; hh < grp; ++hh) {
+      const float mx = warp_max(lmax[hh * 32 + lane]);
+      if (lane == 0) atomicMax(reinterpret_cast<int*>(&hmax[hh]), __float_as_int(mx));
+    }
 #pragma unroll
   for (int u = 0; u < 4; ++u) red[warp][c0 + u] = cv ? dwl[u] : 0.f;
   __syncthreads();
